@@ -1,0 +1,165 @@
+"""Seeded synthetic inputs for the routed-MoE FFN layer (Hy3 shapes).
+
+Workloads (all synthetic; the pages publish no dataset or trained weight for
+this layer):
+
+=========  =====  ====  ===  ==  ====  ===============================================
+name         T      d    E   k    F    structure
+=========  =====  ====  ===  ==  ====  ===============================================
+tiny          64   256   16   4   128  x ~ N(0,1), W ~ N(0, 0.02^2)
+decode        64  4096  192   8  1536  as tiny: logit std 0.02*sqrt(4096) = 1.28
+prefill     4096  4096  192   8  1536  as decode, ~170.7 rows per expert
+skewed     16384  4096  192   8  1536  + per-expert logit bias 0.5*ln(Zipf(1.1) rank weight)
+fp8         8192  4096  192   8  1536  expert weights e4m3 + fp32 scale per output row
+=========  =====  ====  ===  ==  ====  ===============================================
+
+The Hy3 sizes (d=4096, 192 routed experts, top-8, expert d_ff=1536, router
+scaling 2.826) are those of "Tencent Hy3-295B 架构深度拆解" (pillumina.github.io),
+§2.1 hyper-parameter table and §2.3 parameter breakdown.
+
+Draw order, from one torch.Generator seeded with ``seed``: x, W_gate,
+W_gate_up (expert by expert), W_down (expert by expert). Each tensor is drawn
+as fp32 N(0,1), multiplied by its standard deviation and rounded to bf16
+(round-to-nearest-even, torch's cast). The bf16 bit patterns are what both the
+oracle and the CUDA path consume.
+
+Layouts (row-major, contiguous):
+  x          [T, d]        bf16
+  w_gate     [E, d]        bf16
+  w_gate_up  [E, 2F, d]    bf16   rows [0, F) are the gate rows, [F, 2F) the up rows
+  w_down     [E, d, F]     bf16
+  gate_bias  [E]           fp32 or None (added to the router logits)
+FP8 workloads add ``q_gate_up`` [E, 2F, d] / ``q_down`` [E, d, F] as uint8
+e4m3 codes and ``s_gate_up`` [E, 2F] / ``s_down`` [E, d] fp32 scales, with the
+weight meaning q * s.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerShape:
+    T: int
+    d: int
+    E: int
+    k: int
+    F: int
+    scale: float = 2.826
+    x_std: float = 1.0
+    w_std: float = 0.02
+    zipf_bias: bool = False
+    fp8: bool = False
+
+    @property
+    def R(self) -> int:
+        """Routed rows: one per (token, slot)."""
+        return self.T * self.k
+
+
+CONFIGS = {
+    "tiny": LayerShape(T=64, d=256, E=16, k=4, F=128),
+    "decode": LayerShape(T=64, d=4096, E=192, k=8, F=1536),
+    "prefill": LayerShape(T=4096, d=4096, E=192, k=8, F=1536),
+    "skewed": LayerShape(T=16384, d=4096, E=192, k=8, F=1536, zipf_bias=True),
+    "fp8": LayerShape(T=8192, d=4096, E=192, k=8, F=1536, fp8=True),
+}
+
+
+def shape_of(name_or_shape) -> LayerShape:
+    if isinstance(name_or_shape, LayerShape):
+        return name_or_shape
+    return CONFIGS[name_or_shape]
+
+
+def zipf_logit_bias(E: int, s: float = 1.1) -> torch.Tensor:
+    """Per-expert logit bias 0.5*ln(p_r), p_r = r^-s / sum_r' r'^-s, rank r = e+1.
+
+    Expert e takes rank e+1 (identity mapping), so expert 0 is the hottest.
+    """
+    r = torch.arange(1, E + 1, dtype=torch.float64)
+    w = r.pow(-s)
+    p = w / w.sum()
+    return (0.5 * torch.log(p)).to(torch.float32)
+
+
+def _normal(gen: torch.Generator, shape, std: float, device) -> torch.Tensor:
+    t = torch.randn(shape, generator=gen, dtype=torch.float32, device=device)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(torch.bfloat16)
+
+
+def encode_e4m3_rows(w: torch.Tensor):
+    """Per-output-row FP8 (e4m3) encoding of a bf16 weight block [..., rows, cols].
+
+    s_row = max_c |w[row, c]| / 448 (1.0 for an all-zero row);
+    q = e4m3(w / s_row) with round-to-nearest-even (torch's cast). Returns the
+    uint8 codes and the fp32 scales.
+    """
+    wf = w.float()
+    s = wf.abs().amax(dim=-1) / 448.0
+    s = torch.where(s == 0, torch.ones_like(s), s)
+    q = (wf / s.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return q, s.to(torch.float32)
+
+
+def tensor_shapes(cfg) -> dict:
+    """Shapes of the layer's tensors (the layouts listed in the module docstring)."""
+    cfg = shape_of(cfg)
+    T, d, E, F = cfg.T, cfg.d, cfg.E, cfg.F
+    return {"x": (T, d), "w_gate": (E, d), "w_gate_up": (E, 2 * F, d), "w_down": (E, d, F),
+            "gate_bias": (E,), "s_gate_up": (E, 2 * F), "s_down": (E, d)}
+
+
+def make_layer(cfg, seed: int = 0, device="cpu", T: Optional[int] = None,
+               with_experts: bool = True) -> dict:
+    """Draw one layer's inputs. ``T`` overrides the token count of ``cfg``.
+
+    ``with_experts=False`` stops after x and W_gate (the first two draws), for
+    router-only work; those two tensors are identical to the full draw's.
+    """
+    cfg = shape_of(cfg)
+    if T is not None:
+        cfg = dataclasses.replace(cfg, T=T)
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    shp = tensor_shapes(cfg)
+    E = cfg.E
+
+    x = _normal(gen, shp["x"], cfg.x_std, dev)
+    w_gate = _normal(gen, shp["w_gate"], cfg.w_std, dev)
+    if not with_experts:
+        return {"cfg": cfg, "seed": seed, "x": x, "w_gate": w_gate,
+                "gate_bias": zipf_logit_bias(E).to(dev) if cfg.zipf_bias else None}
+    w_gate_up = torch.empty(shp["w_gate_up"], dtype=torch.bfloat16, device=dev)
+    for e in range(E):
+        w_gate_up[e] = _normal(gen, shp["w_gate_up"][1:], cfg.w_std, dev)
+    w_down = torch.empty(shp["w_down"], dtype=torch.bfloat16, device=dev)
+    for e in range(E):
+        w_down[e] = _normal(gen, shp["w_down"][1:], cfg.w_std, dev)
+
+    out = {
+        "cfg": cfg,
+        "seed": seed,
+        "x": x,
+        "w_gate": w_gate,
+        "w_gate_up": w_gate_up,
+        "w_down": w_down,
+        "gate_bias": zipf_logit_bias(E).to(dev) if cfg.zipf_bias else None,
+    }
+    if cfg.fp8:
+        q_gu = torch.empty(shp["w_gate_up"], dtype=torch.uint8, device=dev)
+        s_gu = torch.empty(shp["s_gate_up"], dtype=torch.float32, device=dev)
+        q_d = torch.empty(shp["w_down"], dtype=torch.uint8, device=dev)
+        s_d = torch.empty(shp["s_down"], dtype=torch.float32, device=dev)
+        for e in range(E):
+            q_gu[e], s_gu[e] = encode_e4m3_rows(w_gate_up[e])
+            q_d[e], s_d[e] = encode_e4m3_rows(w_down[e])
+        out.update(q_gate_up=q_gu, s_gate_up=s_gu, q_down=q_d, s_down=s_d)
+    return out

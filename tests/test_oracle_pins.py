@@ -1,0 +1,308 @@
+"""Pins of the fp64 oracle against facts the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a value the
+pages print, a closed form, a special case that reduces to a textbook routine
+(numpy/torch), or brute force on tiny inputs. Together they are chosen so that
+a dropped term, a wrong sign, a wrong index or a transposed operand anywhere
+in the oracle fails at least one of them.
+"""
+
+import dataclasses
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synthetic import LayerShape, make_layer, tensor_shapes
+from sparse_moe_transformer_gemm_b200 import work
+
+
+def _f64(t):
+    """Exact widening of a bf16/fp32 torch tensor with torch (independent of the oracle)."""
+    return t.detach().cpu().to(torch.float64).numpy()
+
+
+def _layer(shape, seed=0, **kw):
+    return make_layer(shape, seed=seed, **kw)
+
+
+def _np_logits(L):
+    return _f64(L["x"]) @ _f64(L["w_gate"]).T + (
+        0.0 if L.get("gate_bias") is None else _f64(L["gate_bias"])[None, :])
+
+
+def _np_expert(x64, wgu64, wd64, e, F):
+    """Textbook SwiGLU MLP (no bias): down( SiLU(x Wg^T) * (x Wu^T) )."""
+    g = x64 @ wgu64[e, :F, :].T
+    u = x64 @ wgu64[e, F:, :].T
+    h = g / (1.0 + np.exp(-g)) * u
+    return h @ wd64[e].T
+
+
+# ------------------------------------------------------------------ formats
+
+def test_bf16_rounding_matches_torch_cast_on_random_fp32_bit_patterns():
+    rng = np.random.default_rng(1)
+    raw = rng.integers(0, 2**32, size=200_000, dtype=np.uint64).astype(np.uint32)
+    # exact ties: low half 0x8000, with both parities of the kept half
+    ties = (rng.integers(0, 2**16, size=20_000, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000
+    v = np.concatenate([raw, ties]).view(np.float32)
+    v = v[np.isfinite(v)]
+    want = oracle.bf16_bits(torch.from_numpy(v).to(torch.bfloat16))
+    got = oracle.bf16_from_double(v.astype(np.float64))
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("value,expected", [
+    (8.2, 8.1875),          # spacing 2^-4 at [8,16): 131.2 quanta -> 131
+    (8.23, 8.25),           # 131.68 quanta -> 132
+    (1.0 + 2.0**-8, 1.0),   # exact tie -> even mantissa (0)
+    (1.0 + 3 * 2.0**-8, 1.0 + 2.0**-6),  # exact tie between mantissas 1 and 2 -> 2
+    (2.0**-133, 2.0**-133),  # smallest subnormal
+    (2.0**-134, 0.0),       # tie between 0 and the smallest subnormal -> 0
+    (3 * 2.0**-134, 2.0**-132),  # tie between 1 and 2 subnormal quanta -> 2
+    (-0.0, -0.0),
+    ((2.0 - 2.0**-8) * 2.0**127, math.inf),  # tie at the top -> rounds up to infinity
+    ((2.0 - 2.0**-7) * 2.0**127, (2.0 - 2.0**-7) * 2.0**127),  # largest finite bf16
+])
+def test_bf16_rounding_hand_cases(value, expected):
+    got = oracle.double_from_bf16(oracle.bf16_from_double(np.array([value])))[0]
+    assert got == expected and math.copysign(1, got) == math.copysign(1, expected)
+
+
+def test_e4m3_decode_matches_torch_for_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.double_from_e4m3(codes)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0**-9 and got[0x08] == 2.0**-6
+
+
+# ------------------------------------------------------------------ combine
+
+def test_fp32_combine_keeps_small_expert_outputs(golden):
+    """The pages' example: a large branch output (8.2) next to small ones (0.03).
+
+    With the outputs already in bf16 (8.1875 and 0.030029296875) a bf16
+    running sum drops every small term; a wide sum keeps them.
+    """
+    ex = golden["fp32_combine_example"]
+    big = oracle.double_from_bf16(oracle.bf16_from_double(np.array([ex["large_output"]])))[0]
+    small = oracle.double_from_bf16(oracle.bf16_from_double(np.array([ex["small_output"]])))[0]
+    assert (big, small) == (8.1875, 0.030029296875)
+    y = np.array([[[big]] + [[small]] * 7], dtype=np.float64)  # [1, 8, 1]
+    out = oracle.double_from_bf16(oracle.combine(y, np.ones((1, 8))))[0, 0]
+    exact = big + 7 * small
+    assert out == 8.375 and abs(out - exact) <= 2.0**-5
+    # what a bf16 running sum would give, by hand: every partial sum rounds back
+    running = big
+    for _ in range(7):
+        running = oracle.double_from_bf16(oracle.bf16_from_double(np.array([running + small])))[0]
+    assert running == 8.1875 != out
+
+
+# ------------------------------------------------------------------ routing
+
+def test_selected_weights_sum_to_scale(golden):
+    scale = golden["sum_of_selected_weights"]["value"]
+    L = _layer("decode", with_experts=False, T=48)
+    r = oracle.route(oracle.bf16_bits(L["x"]), oracle.bf16_bits(L["w_gate"]), 8, scale)
+    assert np.allclose(r["w"].sum(axis=1), scale, rtol=1e-12, atol=0)
+    assert np.all(np.diff(r["w"], axis=1) <= 0)  # descending score order
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 5, 8])
+def test_topk_is_the_best_subset_by_brute_force(k):
+    shape = LayerShape(T=60, d=64, E=8, k=k, F=16, w_std=0.2)
+    L = _layer(shape, seed=k)
+    r = oracle.route(oracle.bf16_bits(L["x"]), oracle.bf16_bits(L["w_gate"]), k, 2.826)
+    s = 1.0 / (1.0 + np.exp(-_np_logits(L)))
+    checked = 0
+    for t in range(shape.T):
+        sums = sorted(((sum(s[t, list(c)]), c) for c in itertools.combinations(range(8), k)),
+                      reverse=True)
+        if len(sums) > 1 and sums[0][0] - sums[1][0] < 1e-12:
+            continue
+        assert set(r["idx"][t]) == set(sums[0][1])
+        checked += 1
+        # gap is the k-th minus the (k+1)-th largest score
+        srt = np.sort(s[t])[::-1]
+        want_gap = srt[k - 1] - srt[k] if k < 8 else math.inf
+        assert r["gap"][t] == pytest.approx(want_gap, rel=1e-9, abs=1e-15)
+    assert checked > 50
+
+
+def test_k1_matches_softmax_argmax_and_takes_the_full_scale(golden):
+    """k = 1: sigmoid top-1 = softmax top-1, and the single weight is the scale."""
+    L = _layer("tiny", seed=3)
+    r = oracle.route(oracle.bf16_bits(L["x"]), oracle.bf16_bits(L["w_gate"]), 1, 2.826)
+    z = _np_logits(L)
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    assert np.array_equal(r["idx"][:, 0], p.argmax(axis=1))
+    assert np.allclose(r["w"][:, 0], golden["router_scaling_factor"]["value"], rtol=1e-15, atol=0)
+
+
+def test_equal_scores_take_lowest_indices_and_split_the_scale(golden):
+    L = _layer("decode", with_experts=False, T=4)
+    x0 = np.zeros((4, 4096), dtype=np.uint16)   # all logits 0 -> every score 0.5
+    r = oracle.route(x0, oracle.bf16_bits(L["w_gate"]), 8, 2.826)
+    assert np.array_equal(r["idx"], np.tile(np.arange(8, dtype=np.int32), (4, 1)))
+    assert np.allclose(r["w"], 2.826 / 8, rtol=1e-15, atol=0)
+    assert round(float(r["w"][0, 0]), 3) == golden["equal_split_weight"]["printed"]
+    assert np.all(r["gap"] == 0.0)
+
+
+def test_scaled_weight_example(golden):
+    """A normalised weight of 0.12 becomes 0.12 * 2.826 = 0.33912 (page prints 0.338)."""
+    ex = golden["scaled_example"]
+    s1, s2 = 0.12, 0.88
+    bias = np.array([math.log(s1 / (1 - s1)), math.log(s2 / (1 - s2))], dtype=np.float32)
+    r = oracle.route(np.zeros((1, 8), np.uint16), np.zeros((2, 8), np.uint16), 2, 2.826,
+                     gate_bias=bias)
+    w_small = r["w"][0, list(r["idx"][0]).index(0)]
+    assert w_small == pytest.approx(ex["before"] * 2.826, abs=1e-6)
+    assert abs(w_small - ex["printed_after"]) < 2e-3
+
+
+def test_gate_bias_is_added_to_the_logits_before_the_sigmoid():
+    rng = np.random.default_rng(7)
+    E, k = 12, 4
+    b = rng.normal(size=E).astype(np.float32)
+    r = oracle.route(np.zeros((1, 16), np.uint16), np.zeros((E, 16), np.uint16), k, 2.826,
+                     gate_bias=b)
+    sig = [1.0 / (1.0 + math.exp(-float(v))) for v in b]
+    want = sorted(range(E), key=lambda e: (-sig[e], e))[:k]
+    assert list(r["idx"][0]) == want
+    tot = sum(sig[e] for e in want)
+    assert np.allclose(r["w"][0], [2.826 * sig[e] / tot for e in want], rtol=1e-14)
+
+
+# ------------------------------------------------------------------ experts / layer
+
+def test_k1_layer_is_the_textbook_swiglu_mlp_of_the_argmax_expert():
+    shape = LayerShape(T=24, d=96, E=6, k=1, F=80)
+    L = _layer(shape, seed=11)
+    O = oracle.OracleLayer(L)
+    r = oracle.forward_tokens(O)
+    x64, wgu, wd = _f64(L["x"]), _f64(L["w_gate_up"]), _f64(L["w_down"])
+    e_star = _np_logits(L).argmax(axis=1)
+    for t in range(shape.T):
+        want = 2.826 * _np_expert(x64[t:t + 1], wgu, wd, e_star[t], shape.F)[0]
+        assert r["idx"][t, 0] == e_star[t]
+        assert np.allclose(r["out_f64"][t], want, rtol=1e-9, atol=1e-12)
+    assert np.array_equal(r["out_bf16"], oracle.bf16_from_double(r["out_f64"]))
+
+
+def test_k_equals_E_is_the_dense_weighted_sum_over_all_experts():
+    shape = LayerShape(T=16, d=64, E=5, k=5, F=48)
+    L = _layer(shape, seed=5)
+    r = oracle.forward_tokens(oracle.OracleLayer(L))
+    x64, wgu, wd = _f64(L["x"]), _f64(L["w_gate_up"]), _f64(L["w_down"])
+    s = 1.0 / (1.0 + np.exp(-_np_logits(L)))
+    w = 2.826 * s / s.sum(axis=1, keepdims=True)
+    want = sum(w[:, e:e + 1] * _np_expert(x64, wgu, wd, e, shape.F) for e in range(shape.E))
+    assert np.allclose(r["out_f64"], want, rtol=1e-9, atol=1e-12)
+    assert np.all(np.isinf(r["gap"]))
+
+
+def test_zero_up_weights_give_zero_output():
+    shape = LayerShape(T=10, d=64, E=4, k=2, F=32)
+    L = _layer(shape, seed=2)
+    L["w_gate_up"][:, shape.F:, :] = 0
+    r = oracle.forward_tokens(oracle.OracleLayer(L))
+    assert np.all(r["out_f64"] == 0.0)
+
+
+def test_token_order_invariance_is_bitwise():
+    L = _layer("tiny", seed=4)
+    perm = torch.randperm(64, generator=torch.Generator().manual_seed(0))
+    L2 = dict(L, x=L["x"][perm].contiguous())
+    a = oracle.forward_tokens(oracle.OracleLayer(L))
+    b = oracle.forward_tokens(oracle.OracleLayer(L2))
+    assert np.array_equal(a["out_bf16"][perm.numpy()], b["out_bf16"])
+
+
+def test_expert_relabelling_invariance_is_bitwise():
+    L = _layer("tiny", seed=6)
+    perm = torch.randperm(16, generator=torch.Generator().manual_seed(1))  # new e -> old perm[e]
+    L2 = dict(L, w_gate=L["w_gate"][perm].contiguous(), w_gate_up=L["w_gate_up"][perm].contiguous(),
+              w_down=L["w_down"][perm].contiguous())
+    a = oracle.forward_tokens(oracle.OracleLayer(L))
+    b = oracle.forward_tokens(oracle.OracleLayer(L2))
+    assert np.array_equal(a["out_bf16"], b["out_bf16"])
+    assert np.array_equal(perm.numpy()[b["idx"]], a["idx"])
+
+
+def test_output_is_linear_in_the_scale():
+    L = _layer("tiny", seed=8)
+    one = oracle.forward_tokens(oracle.OracleLayer(L, scale=1.0))["out_f64"]
+    big = oracle.forward_tokens(oracle.OracleLayer(L, scale=2.826))["out_f64"]
+    assert np.allclose(big / 2.826, one, rtol=1e-12, atol=1e-18)
+
+
+def test_fp8_expert_matches_textbook_mlp_on_decoded_weights():
+    shape = LayerShape(T=6, d=64, E=3, k=1, F=32, fp8=True)
+    L = _layer(shape, seed=9)
+    dec = lambda q, s: (torch.from_numpy(q.cpu().numpy()).view(torch.float8_e4m3fn)  # noqa: E731
+                        .to(torch.float64) * s.to(torch.float64)[..., None]).numpy()
+    wgu = dec(L["q_gate_up"], L["s_gate_up"])
+    wd = dec(L["q_down"], L["s_down"])
+    x64 = _f64(L["x"])
+    experts = np.array([0, 1, 2, 0, 1, 2], np.int32)
+    y = oracle.expert_rows(oracle.bf16_bits(L["x"]), experts, L["q_gate_up"].numpy(),
+                           L["q_down"].numpy(), L["s_gate_up"].numpy(), L["s_down"].numpy())
+    for t in range(6):
+        want = _np_expert(x64[t:t + 1], wgu, wd, experts[t], shape.F)[0]
+        assert np.allclose(y[t], want, rtol=1e-9, atol=1e-13)
+
+
+def test_fp8_layer_stays_within_quantisation_error_of_the_bf16_layer():
+    shape = LayerShape(T=32, d=256, E=8, k=2, F=128, fp8=True)
+    L = _layer(shape, seed=10)
+    q = oracle.forward_tokens(oracle.OracleLayer(L))["out_f64"]
+    ref = oracle.forward_tokens(oracle.OracleLayer(dict(L, cfg=dataclasses.replace(shape, fp8=False))))["out_f64"]
+    rel = np.linalg.norm(q - ref) / np.linalg.norm(ref)
+    assert 1e-4 < rel < 0.08   # e4m3: 3 mantissa bits, relative step <= 2^-3
+
+
+# ------------------------------------------------------------------ sizes and work
+
+def test_per_expert_parameter_count_matches_the_page(golden):
+    g = golden["expert_shapes"]
+    shp = tensor_shapes("decode")
+    gu = math.prod(shp["w_gate_up"][1:])
+    dn = math.prod(shp["w_down"][1:])
+    assert (shp["w_gate_up"][0], shp["x"][1], shp["w_down"][2]) == (g["n_routed_experts"], g["d"],
+                                                                    g["d_ff_expert"])
+    assert gu + dn == 18_874_368
+    assert round(gu / 1e6, 2) * 1e6 == g["gate_up_params"]
+    assert round(dn / 1e6, 2) * 1e6 == g["down_params"]
+    assert round((gu + dn) / 1e6, 2) * 1e6 == g["params_per_expert"]
+
+
+def test_per_expert_flops_match_the_page(golden):
+    f = work.expert_flops_per_token(4096, 1536)
+    assert f == 37_748_736
+    assert float(f"{f:.2e}") == golden["flops_per_token_per_expert"]["printed"]
+
+
+# ------------------------------------------------------------------ permute definition
+
+@pytest.mark.parametrize("T,k,E", [(100, 4, 16), (1, 8, 192), (257, 8, 192), (33, 1, 3)])
+def test_permute_definition_matches_stable_argsort(T, k, E):
+    rng = np.random.default_rng(T * 31 + k)
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    r = oracle.permute(idx, E)
+    flat = idx.ravel()
+    order = np.argsort(flat, kind="stable")        # row -> slot
+    want_row_of = np.empty_like(order)
+    want_row_of[order] = np.arange(flat.size)
+    assert np.array_equal(r["row_of"], want_row_of)
+    assert np.array_equal(r["counts"], np.bincount(flat, minlength=E))
+    assert np.array_equal(r["offsets"], np.concatenate([[0], np.cumsum(np.bincount(flat, minlength=E))]))
