@@ -1,0 +1,386 @@
+"""Benchmark of the routed-MoE FFN layer (Hy3 shapes) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|prefill|skewed|fp8]
+                    [--impl ours|reference] [--path auto|stream|gemm]
+
+One step = one pass of the whole layer (route, group, gate_up, down, combine)
+over one batch of T synthetic tokens, inputs resident in HBM. Rank 0 prints one
+JSON line. With N > 1 (torchrun) every rank runs an independent replica on its
+own batch (tokens are independent: no collective on the data path) and the
+value is the tokens of all ranks over the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (each
+step a bounded sample of the same workload), rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synthetic import CONFIGS, make_layer  # noqa: E402
+from sparse_moe_transformer_gemm_b200 import work  # noqa: E402
+
+WORKLOADS = {
+    "decode": "Hy3 MoE layer decode: T=64 tokens, d=4096, E=192, top-8, d_ff=1536 SwiGLU, "
+              "scale 2.826, fp32 combine; x bf16 N(0,1), W_gate/experts bf16 N(0,0.02)",
+    "prefill": "Hy3 MoE layer prefill: T=4096 tokens, same shapes/dtypes/init as decode",
+    "skewed": "Hy3 MoE layer, skewed routing: T=16384, logit bias 0.5*ln(Zipf(1.1) rank weight)",
+    "fp8": "Hy3 MoE layer FP8 weights: T=8192, experts e4m3 + fp32 per-output-row scales",
+    "tiny": "Tiny MoE layer: T=64, d=256, E=16, top-4, d_ff=128",
+}
+
+# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
+# kernel, from the capture summarised in profiles/ (None until captured for the
+# kernel as it now stands).
+NCU_TRAFFIC = {}
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, world, rank):
+    """The fp64 CPU oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+
+    shape = CONFIGS[args.config]
+    layer = make_layer(shape, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
+    O = oracle.OracleLayer(layer)
+    del layer
+    # size each step's token sample so that one step is ~args.ref_step_seconds of CPU work
+    t0 = time.perf_counter()
+    oracle.forward_tokens(O, np.array([0], np.int32))
+    one = max(time.perf_counter() - t0, 1e-6)
+    per_step = int(max(1, min(shape.T, round(args.ref_step_seconds * oracle.num_threads() / one))))
+    rng = np.random.default_rng(0)
+    samples = [rng.choice(shape.T, size=per_step, replace=False).astype(np.int32)
+               for _ in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        oracle.forward_tokens(O, samples[i])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.forward_tokens(O, samples[args.warmup + i])
+    dt = time.perf_counter() - t0
+    tok_s = per_step * args.steps / dt
+    line = {
+        "impl": "reference", "metric": "MoE-layer tokens/s", "value": tok_s, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, seed 0)",
+        "config": {"workload": WORKLOADS[args.config], "T": shape.T},
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{per_step} random tokens of the {shape.T}-token batch per step"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(layer, shape, seconds: float):
+    """The oracle timed on the host cores on a bounded sample of the workload."""
+    import numpy as np
+    import oracle
+
+    O = oracle.OracleLayer(layer)
+    t0 = time.perf_counter()
+    oracle.forward_tokens(O, np.array([0], np.int32))
+    one = max(time.perf_counter() - t0, 1e-6)
+    n = int(max(1, min(shape.T, round(seconds * oracle.num_threads() / one))))
+    toks = np.arange(n, dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.forward_tokens(O, toks)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {n} of the {shape.T} tokens of the same batch ({dt:.1f} s)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "stream", "gemm"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    if args.steps is None:
+        args.steps = 10 if args.impl == "reference" else {"decode": 2000, "tiny": 2000}.get(
+            args.config, 200)
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    from sparse_moe_transformer_gemm_b200 import moe
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    shape = CONFIGS[args.config]
+    layer = make_layer(shape, seed=rank, device=dev)
+    cfg = moe.config_of(shape, None if args.path == "auto" else args.path)
+    T, d, E, k, F = shape.T, shape.d, shape.E, shape.k, shape.F
+    R = T * k
+    ws = moe.workspace(cfg, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    wgu, sgu, wd, sd = moe.layer_args(layer)
+    x, wg, gb = layer["x"], layer["w_gate"], layer["gate_bias"]
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty(R, dtype=torch.int32, device=dev)
+    xp = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
+    h = torch.empty((R, F), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+
+    stages = ["route", "permute", "gate_up", "down", "combine"]
+    n_launch = {"route": 1, "permute": 3, "gate_up": 1, "down": 1, "combine": 1}
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_route(cfg, x, wg, gb, idx, w, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.moe_permute(cfg, idx, x, counts, offsets, row_of, xp, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        moe.moe_expert_gate_up(cfg, xp, offsets, wgu, sgu, h, ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        moe.moe_expert_down(cfg, h, offsets, wd, sd, y, ws, stream)
+        if ev is not None:
+            ev[4].record(stream)
+        moe.moe_combine(cfg, y, row_of, w, out, ws, stream)
+        if ev is not None:
+            ev[5].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    assert moe.moe_read_status(ws, stream) == moe.MOE_OK
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t_begin.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    status = moe.moe_read_status(ws, stream)
+    ms = t_begin.elapsed_time(t_end) / args.steps
+    stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps
+                for j, s in enumerate(stages)}
+    if pg:
+        tm = torch.tensor([ms], device=dev)
+        pg.all_reduce(tm, op=pg.ReduceOp.MAX)
+        ms = float(tm.item())
+
+    # touched experts of this batch (for the algorithmic bytes)
+    touched = int((counts > 0).sum().item())
+    rows = int(offsets[-1].item())
+    peaks, peak_src = load_peaks()
+    fp8 = shape.fp8
+    lw = work.layer_work(T, d, E, k, F, touched, fp8)
+    gw = work.gate_up_work(rows, touched, d, F, fp8)
+    dw = work.down_work(rows, touched, d, F, fp8)
+    dominant = max(("gate_up", "down"), key=lambda s: stage_ms[s])
+    dom_work = gw if dominant == "gate_up" else dw
+    dom_s = stage_ms[dominant] / 1e3
+    kernel_name = f"{dominant}_{'gemm' if args.path == 'gemm' else 'stream'}"
+    use_stream = args.path == "stream" or (args.path == "auto" and T * k <= 8 * E)
+    kernel_name = f"{dominant}_{'stream' if use_stream else 'gemm'}"
+    if use_stream:
+        achieved = dom_work["bytes"] / dom_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = dom_work["flops"] / dom_s / 1e12
+        pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                "frac": achieved / pk}
+    roof["traffic"] = NCU_TRAFFIC.get((args.config, kernel_name))
+    roof["kernel"] = kernel_name
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+    roof["algorithmic_bytes_per_launch"] = dom_work["bytes"]
+    roof["algorithmic_flops_per_launch"] = dom_work["flops"]
+
+    # end to end through moe_forward: pinned host x in, pinned host out back, every step
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_steps = max(3, args.steps // 2)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            x_dev.copy_(x_host, non_blocking=True)
+            moe.moe_forward(cfg, x_dev, wg, gb, wgu, sgu, wd, sd, out, ws, stream)
+            out_host.copy_(out, non_blocking=True)
+    stream.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            x_dev.copy_(x_host, non_blocking=True)
+            moe.moe_forward(cfg, x_dev, wg, gb, wgu, sgu, wd, sd, out, ws, stream)
+            out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if pg:
+        tm = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(tm, op=pg.ReduceOp.MAX)
+        e2e_ms = float(tm.item())
+    status2 = moe.moe_read_status(ws, stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(layer, shape, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": "MoE-layer tokens/s", "value": world * T / (ms / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 weights, bf16 activations, fp32 accumulate" if fp8 else
+                     "bf16 (fp32 accumulate, fp32 combine)",
+            "data": "synthetic (seeded; random-init weights of the Hy3 MoE layer shapes)",
+            "config": {"workload": WORKLOADS[args.config], "T": T, "d": d, "E": E, "k": k,
+                       "d_ff": F, "path": args.path, "parallelism": f"replicas x{world}",
+                       "l2": "no flush: each step streams the touched experts' weights "
+                             f"({touched} experts, {touched * work.expert_bytes(d, F, fp8) / 1e9:.2f} GB) "
+                             "through the 126 MB L2"},
+            "roofline": roof,
+            "layer_roofline": {
+                "hbm_frac": lw["bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "tensor_frac": lw["flops"] / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                "algorithmic_bytes": lw["bytes"], "algorithmic_flops": lw["flops"],
+                "touched_experts": touched},
+            "stage_ms": stage_ms,
+            "clocks": clocks.summary(),
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
+                    "ms_per_step": e2e_ms, "api": "moe_forward"},
+            "gpu_launches": sum(n_launch.values()) * args.steps,
+            "status": [moe.moe_status_string(status), moe.moe_status_string(status2)],
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,160 @@
+/*
+ * moe.h -- C ABI of the routed-MoE FFN layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (Hy3 routed experts; "Tencent Hy3-295B 架构深度拆解",
+ * pillumina.github.io, §2.3 parameter breakdown and §4.1 routing flow;
+ * "DeepSeek V4-Flash 架构 QA", cctoctofx.netlify.app, Q4.5 and Q8.4; Hy3
+ * commentary, wmrh.cn/news/24252, §2.3 fp32 combine):
+ *
+ *   logits = x W_gate^T (+ gate_bias)          fp32 accumulate
+ *   s      = sigmoid(logits)
+ *   top-k  = k largest s per token, equal scores -> lower expert index
+ *   w_j    = scale * s_j / sum_{i in top-k} s_i
+ *   y_j    = W_down[e_j] ( SiLU(W_gate_rows[e_j] x) * (W_up_rows[e_j] x) )
+ *   out    = bf16( sum_j w_j * float(y_j) )     fp32 sum, one final cast
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers, row-major and contiguous, 16-byte
+ *   aligned. bf16 tensors are passed as void* (IEEE bfloat16 bit patterns).
+ * - Layouts: x [T, d]; w_gate [E, d]; w_gate_up [E, 2*d_ff, d] with rows
+ *   [0, d_ff) the gate projection and [d_ff, 2*d_ff) the up projection;
+ *   w_down [E, d, d_ff]; topk_idx [T, k] int32; topk_w [T, k] fp32 (both in
+ *   descending score order); out [T, d].
+ * - FP8 weights (MOE_FLAG_FP8_WEIGHTS): w_gate_up / w_down hold e4m3 codes
+ *   (one byte each) in the same layouts, and s_gate_up [E, 2*d_ff] /
+ *   s_down [E, d] hold fp32 per-output-row scales; the weight value is
+ *   code * scale. Without the flag both scale pointers must be NULL.
+ * - Grouping ("permuted rows"): token-slot s = t*k + j goes to row
+ *   row_of[s] = offsets[e] + (number of earlier slots s' < s with the same
+ *   expert e = topk_idx[s]); offsets[e] = sum_{e' < e} counts[e'],
+ *   offsets[E] = T*k. Rows of one expert are contiguous and keep slot order.
+ * - Supported shapes: T >= 1; d and d_ff multiples of 128; 1 <= E <= 256;
+ *   1 <= k <= min(E, 32); T*k*max(d, d_ff) < 2^31. Anything else returns
+ *   MOE_ERR_UNSUPPORTED_SHAPE before any launch.
+ * - ws is a caller-owned device workspace of at least moe_workspace_size(cfg)
+ *   bytes, 256-byte aligned, initialised once with moe_workspace_init. The
+ *   library allocates no memory and keeps no state between calls other than
+ *   per-device kernel attributes and a driver entry point looked up once.
+ * - stream is a cudaStream_t (NULL = legacy default stream). Every call is
+ *   asynchronous on it; no call synchronises, except moe_read_status.
+ * - Return value: MOE_OK (0) or a negative MOE_ERR_* code. Argument errors are
+ *   reported before any work is queued. MOE_ERR_CUDA means a launch failed
+ *   (cudaGetLastError). Faults inside kernels are not converted; kernels
+ *   whose waits are bounded record MOE_ERR_TIMEOUT in the workspace status
+ *   word instead of hanging (read it with moe_read_status).
+ * - Values: NaN/Inf inputs give unspecified outputs. Results are
+ *   deterministic: the same inputs give bitwise-identical outputs.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)       /* NULL pointer, misalignment, bad flag mix */
+#define MOE_ERR_UNSUPPORTED_SHAPE (-2) /* shape outside the supported set above */
+#define MOE_ERR_WORKSPACE (-3)         /* ws_bytes < moe_workspace_size(cfg) */
+#define MOE_ERR_CUDA (-4)              /* a CUDA launch or runtime call failed */
+#define MOE_ERR_TIMEOUT (-5)           /* a bounded device wait gave up */
+
+#define MOE_FLAG_FP8_WEIGHTS 0x1u /* expert weights are e4m3 codes + fp32 row scales */
+#define MOE_FLAG_STREAM_PATH 0x2u /* experts on the weight-streaming (decode) kernels */
+#define MOE_FLAG_GEMM_PATH 0x4u   /* experts on the tensor-core grouped GEMMs */
+/* With neither path flag the library picks by the mean rows per expert T*k/E. */
+
+typedef struct moe_config {
+    int32_t T;      /* tokens */
+    int32_t d;      /* hidden size (4096 for Hy3) */
+    int32_t E;      /* routed experts (192) */
+    int32_t k;      /* experts per token (8) */
+    int32_t d_ff;   /* expert intermediate size (1536) */
+    float scale;    /* router_scaling_factor (2.826) */
+    uint32_t flags; /* MOE_FLAG_* */
+} moe_config;
+
+/* Bytes of workspace every entry point below needs for cfg (0 if cfg is
+ * invalid). Covers the routing scratch, the grouping, the permuted activations
+ * [T*k, d], the intermediate h [T*k, d_ff] and the expert outputs [T*k, d]. */
+MOE_API size_t moe_workspace_size(const moe_config* cfg);
+
+/* Zero the workspace's control words (status word and routing counters) for
+ * cfg. Call once after allocating ws, before any other call that uses it. */
+MOE_API int moe_workspace_init(const moe_config* cfg, void* ws, size_t ws_bytes, void* stream);
+
+/* Router: logits = x w_gate^T (+ gate_bias, nullable [E] fp32, added before the
+ * sigmoid), sigmoid, top-k (ties -> lower index), renormalise over the k
+ * selected scores and multiply by cfg->scale. Writes topk_idx [T, k] int32 and
+ * topk_w [T, k] fp32 in descending score order.
+ * Pages: "Tencent Hy3-295B 架构深度拆解" §4.1 (router lines and steps 1-5);
+ * Hy3 commentary §3.3 for a logit bias added before the sigmoid. */
+MOE_API int moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+              int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream);
+
+/* Group token-slots by expert (the grouping defined above): writes counts [E],
+ * offsets [E+1], row_of [T*k] (int32) and x_perm [T*k, d] bf16 with
+ * x_perm[row_of[t*k+j]] = x[t]. Pages: the per-expert loop with index_add_ of
+ * "DeepSeek V4-Flash 架构 QA" Q8.4, re-expressed as a grouping for batched
+ * expert GEMMs ("Tencent Hy3-Flash QA" Q6.4, grouped MM). */
+MOE_API int moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x, int32_t* counts,
+                int32_t* offsets, int32_t* row_of, void* x_perm, void* ws, size_t ws_bytes,
+                void* stream);
+
+/* gate_up step of the SwiGLU experts on grouped rows: for each expert e and
+ * each of its rows r in [offsets[e], offsets[e+1]):
+ *   h[r, f] = bf16( SiLU(g) * u ),  g = <x_perm[r], w_gate_up[e, f]>,
+ *   u = <x_perm[r], w_gate_up[e, d_ff + f]>, fp32 accumulate and epilogue.
+ * h is [T*k, d_ff] bf16. Pages: "DeepSeek V4-Flash 架构 QA" Q4.5 (SwiGLU);
+ * "Tencent Hy3-295B 架构深度拆解" §2.3 (fused gate_up_proj 2*1536 x 4096). */
+MOE_API int moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                       const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* down step: y[r, i] = bf16( <h[r], w_down[e, i]> ), fp32 accumulate; y is
+ * [T*k, d] bf16. Pages: "Tencent Hy3-295B 架构深度拆解" §2.3 (down_proj
+ * 4096 x 1536). */
+MOE_API int moe_expert_down(const moe_config* cfg, const void* h, const int32_t* offsets,
+                    const void* w_down, const float* s_down, void* y, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/* Both expert steps (h lives in ws): y [T*k, d] bf16 from x_perm. */
+MOE_API int moe_experts(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                const void* w_gate_up, const float* s_gate_up, const void* w_down,
+                const float* s_down, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* fp32 combine and unpermute: out[t, :] = bf16_rne( sum_{j<k} topk_w[t, j] *
+ * float(y[row_of[t*k + j], :]) ), summed in fp32 in j order, one final cast.
+ * Pages: Hy3 commentary §2.3 (enable_moe_fp32_combine = true: convert the
+ * branch outputs to fp32 before adding, cast back once). */
+MOE_API int moe_combine(const moe_config* cfg, const void* y, const int32_t* row_of, const float* topk_w,
+                void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer: route, group, experts, combine. out [T, d] bf16. The
+ * intermediates live in ws. Resets the workspace status word first. */
+MOE_API int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+                const void* w_gate_up, const float* s_gate_up, const void* w_down,
+                const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise stream, then read and clear the workspace status word: MOE_OK,
+ * or MOE_ERR_TIMEOUT if a bounded device wait gave up since the last read. */
+MOE_API int moe_read_status(void* ws, void* stream);
+
+/* Static text for a status code. */
+MOE_API const char* moe_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,59 @@
+// combine.cu -- fp32 weighted combine and unpermute.
+//
+// enable_moe_fp32_combine (Hy3 commentary, wmrh.cn/news/24252, §2.3): the
+// expert branch outputs are converted to fp32, summed with their routing
+// weights in fp32 and cast back to bf16 once, so that small contributions
+// next to a large one are not rounded away. The weighted sum over the k
+// selected experts replaces the pages' per-expert loop with index_add_
+// ("DeepSeek V4-Flash 架构 QA", Q8.4) by a gather: token t reads its k expert
+// rows y[row_of[t*k + j]] (no atomics, fixed j order, deterministic).
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+__global__ void __launch_bounds__(256)
+combine_kernel(const __nv_bfloat16* __restrict__ y, const int* __restrict__ row_of,
+               const float* __restrict__ w, int k, int d, __nv_bfloat16* __restrict__ out) {
+    __shared__ int rows[32];
+    __shared__ float wts[32];
+    const long t = blockIdx.x;
+    if (threadIdx.x < k) {
+        rows[threadIdx.x] = row_of[t * k + threadIdx.x];
+        wts[threadIdx.x] = w[t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < d / 8; v += blockDim.x) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const int r = rows[j];
+            if (r < 0) continue;
+            const uint4 u = *reinterpret_cast<const uint4*>(y + (long)r * d + v * 8);
+            float f[8];
+            bf16x8_to_float(u, f);
+            const float wj = wts[j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(out + t * d + v * 8) = o;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const moe_config& c, const void* y, const int32_t* row_of,
+                           const float* topk_w, void* out, cudaStream_t s) {
+    combine_kernel<<<c.T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(y), row_of, topk_w, c.k,
+                                       c.d, static_cast<__nv_bfloat16*>(out));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,68 @@
+// common.cuh -- small device helpers shared by the library's kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace moe {
+
+// bf16 pair (packed in a 32-bit word, low half first) -> two floats. Exact.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
+// Eight bf16 in a 16-byte vector -> eight floats.
+__device__ __forceinline__ void bf16x8_to_float(const uint4& v, float f[8]) {
+    float2 a = bf16x2_to_float2(v.x), b = bf16x2_to_float2(v.y);
+    float2 c = bf16x2_to_float2(v.z), d = bf16x2_to_float2(v.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+// Two e4m3 codes (low byte first) -> two floats, exactly (via the hardware
+// e4m3x2 -> f16x2 conversion; every e4m3 value is an f16 value).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t v) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)v, __NV_E4M3);
+    return __half22float2(*reinterpret_cast<__half2*>(&h));
+}
+
+// Sixteen e4m3 codes in a 16-byte vector -> sixteen floats.
+__device__ __forceinline__ void e4m3x16_to_float(const uint4& v, float f[16]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 lo = e4m3x2_to_float2((uint16_t)(w[i] & 0xFFFF));
+        float2 hi = e4m3x2_to_float2((uint16_t)(w[i] >> 16));
+        f[4 * i + 0] = lo.x; f[4 * i + 1] = lo.y; f[4 * i + 2] = hi.x; f[4 * i + 3] = hi.y;
+    }
+}
+
+// Round a float to bf16 (nearest-even) and return the 16-bit pattern.
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+    __nv_bfloat16 b = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&b);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    return (uint32_t)float_to_bf16_bits(lo) | ((uint32_t)float_to_bf16_bits(hi) << 16);
+}
+
+// Read-only, L1-bypassing 16-byte load for data streamed exactly once.
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float sigmoidf_acc(float z) { return 1.0f / (1.0f + expf(-z)); }
+
+}  // namespace moe

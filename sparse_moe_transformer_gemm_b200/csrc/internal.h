@@ -1,0 +1,90 @@
+// internal.h -- workspace layout and kernel launchers shared by the library's
+// translation units. Not part of the public ABI (that is include/moe.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kRouterTokens = 8;        // tokens per router CTA
+constexpr int kRouterExperts = 32;      // experts per router CTA (8 warps x 4)
+constexpr int kPermuteChunk = 2048;     // token-slots per ranking chunk
+constexpr int kStreamMaxTokens = 8;     // rows per pass of the streaming expert kernels
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Byte offsets of every workspace region. The control words (status word and
+// router counters) come first so that one memset clears them.
+struct WsLayout {
+    size_t status;    // int32 status word (+ padding)
+    size_t counters;  // int32 [ceil(T / kRouterTokens)] router arrival counters
+    size_t control_end;
+    size_t logits;    // fp32 [T, E]
+    size_t hist;      // int32 [n_chunks, E]
+    size_t rank;      // int32 [T*k]
+    size_t idx;       // int32 [T*k]
+    size_t w;         // fp32  [T*k]
+    size_t counts;    // int32 [E]
+    size_t offsets;   // int32 [E+1]
+    size_t row_of;    // int32 [T*k]
+    size_t xperm;     // bf16 [T*k, d]
+    size_t h;         // bf16 [T*k, d_ff]
+    size_t y;         // bf16 [T*k, d]
+    size_t sched;     // int32 GEMM tile scheduling scratch
+    size_t total;
+};
+
+inline int n_router_groups(const moe_config& c) {
+    return (c.T + kRouterTokens - 1) / kRouterTokens;
+}
+inline int n_permute_chunks(const moe_config& c) {
+    long R = (long)c.T * c.k;
+    return (int)((R + kPermuteChunk - 1) / kPermuteChunk);
+}
+
+inline WsLayout ws_layout(const moe_config& c) {
+    WsLayout L{};
+    size_t R = (size_t)c.T * c.k;
+    size_t o = 0;
+    L.status = o;   o += 256;
+    L.counters = o; o = align256(o + sizeof(int32_t) * n_router_groups(c));
+    L.control_end = o;
+    L.logits = o;   o = align256(o + sizeof(float) * (size_t)c.T * c.E);
+    L.hist = o;     o = align256(o + sizeof(int32_t) * (size_t)n_permute_chunks(c) * c.E);
+    L.rank = o;     o = align256(o + sizeof(int32_t) * R);
+    L.idx = o;      o = align256(o + sizeof(int32_t) * R);
+    L.w = o;        o = align256(o + sizeof(float) * R);
+    L.counts = o;   o = align256(o + sizeof(int32_t) * c.E);
+    L.offsets = o;  o = align256(o + sizeof(int32_t) * (c.E + 1));
+    L.row_of = o;   o = align256(o + sizeof(int32_t) * R);
+    L.xperm = o;    o = align256(o + 2 * R * c.d);
+    L.h = o;        o = align256(o + 2 * R * c.d_ff);
+    L.y = o;        o = align256(o + 2 * R * c.d);
+    L.sched = o;    o = align256(o + sizeof(int32_t) * 4 * (c.E + 1));
+    L.total = o;
+    return L;
+}
+
+// ---- launchers (each returns cudaError_t of the launch) ----
+cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
+                          const float* gate_bias, int32_t* idx, float* w, float* logits,
+                          int32_t* counters, cudaStream_t s);
+
+cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
+                           int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,
+                           int32_t* rank, cudaStream_t s);
+
+cudaError_t launch_gate_up_stream(const moe_config& c, const void* x_perm, const int32_t* offsets,
+                                  const void* w_gate_up, const float* s_gate_up, void* h,
+                                  cudaStream_t s);
+cudaError_t launch_down_stream(const moe_config& c, const void* h, const int32_t* offsets,
+                               const void* w_down, const float* s_down, void* y, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_config& c, const void* y, const int32_t* row_of,
+                           const float* topk_w, void* out, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,227 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument checks, the
+// workspace carve-up and the kernel launches. Host code only.
+#include <math.h>
+
+#include "internal.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr uint32_t kKnownFlags = MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH | MOE_FLAG_GEMM_PATH;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const moe_config* c) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if ((c->flags & ~kKnownFlags) != 0) return MOE_ERR_INVALID_ARG;
+    if ((c->flags & MOE_FLAG_STREAM_PATH) && (c->flags & MOE_FLAG_GEMM_PATH))
+        return MOE_ERR_INVALID_ARG;
+    if (!isfinite(c->scale)) return MOE_ERR_INVALID_ARG;
+    if (c->T < 1 || c->E < 1 || c->E > 256 || c->k < 1 || c->k > c->E || c->k > 32)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->d < 128 || c->d % 128 != 0 || c->d > 8192) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (c->d_ff < 128 || c->d_ff % 128 != 0 || c->d_ff > 8192) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const long long R = (long long)c->T * c->k;
+    const long long wide = c->d > c->d_ff ? c->d : c->d_ff;
+    if (R * wide >= (1LL << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+// Expert weights: bf16 without the FP8 flag (no scales), e4m3 + scales with it.
+int check_expert_weights(const moe_config* c, const void* w, const float* s) {
+    if (!w || !aligned16(w)) return MOE_ERR_INVALID_ARG;
+    if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
+        if (!s) return MOE_ERR_INVALID_ARG;
+    } else if (s) {
+        return MOE_ERR_INVALID_ARG;
+    }
+    return MOE_OK;
+}
+
+int check_ws(const moe_config* c, const void* ws, size_t ws_bytes) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(*c).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                   \
+    do {                                \
+        int rc_ = (expr);               \
+        if (rc_ != MOE_OK) return rc_;  \
+    } while (0)
+
+// Rows per expert below which the weight-streaming kernels are used.
+bool use_stream_path(const moe_config* c) {
+    if (c->flags & MOE_FLAG_STREAM_PATH) return true;
+    return true;  // the tensor-core grouped GEMM path is selected here once present
+}
+
+int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offsets,
+                    const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
+                    cudaStream_t s) {
+    (void)ws;
+    if (c->flags & MOE_FLAG_GEMM_PATH) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (use_stream_path(c))
+        return cuda_status(launch_gate_up_stream(*c, x_perm, offsets, w_gate_up, s_gate_up, h, s));
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+}
+
+int experts_down(const moe_config* c, const void* h, const int32_t* offsets, const void* w_down,
+                 const float* s_down, void* y, void* ws, cudaStream_t s) {
+    (void)ws;
+    if (c->flags & MOE_FLAG_GEMM_PATH) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (use_stream_path(c))
+        return cuda_status(launch_down_stream(*c, h, offsets, w_down, s_down, y, s));
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config* cfg) {
+    if (check_cfg(cfg) != MOE_OK) return 0;
+    return ws_layout(*cfg).total;
+}
+
+int moe_workspace_init(const moe_config* cfg, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    return cuda_status(cudaMemsetAsync(ws, 0, ws_layout(*cfg).control_end,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+              int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!x || !w_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    const WsLayout L = ws_layout(*cfg);
+    return cuda_status(launch_router(*cfg, x, w_gate, gate_bias, topk_idx, topk_w,
+                                     at<float>(ws, L.logits), at<int32_t>(ws, L.counters),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x, int32_t* counts,
+                int32_t* offsets, int32_t* row_of, void* x_perm, void* ws, size_t ws_bytes,
+                void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!topk_idx || !x || !counts || !offsets || !row_of || !x_perm) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    const WsLayout L = ws_layout(*cfg);
+    return cuda_status(launch_permute(*cfg, topk_idx, x, counts, offsets, row_of, x_perm,
+                                      at<int32_t>(ws, L.hist), at<int32_t>(ws, L.rank),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                       const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
+                       size_t ws_bytes, void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!x_perm || !offsets || !h || !aligned16(x_perm) || !aligned16(h))
+        return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_expert_weights(cfg, w_gate_up, s_gate_up));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    return experts_gate_up(cfg, x_perm, offsets, w_gate_up, s_gate_up, h, ws,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_down(const moe_config* cfg, const void* h, const int32_t* offsets,
+                    const void* w_down, const float* s_down, void* y, void* ws, size_t ws_bytes,
+                    void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!h || !offsets || !y || !aligned16(h) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_expert_weights(cfg, w_down, s_down));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    return experts_down(cfg, h, offsets, w_down, s_down, y, ws, static_cast<cudaStream_t>(stream));
+}
+
+int moe_experts(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                const void* w_gate_up, const float* s_gate_up, const void* w_down,
+                const float* s_down, void* y, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!x_perm || !offsets || !y || !aligned16(x_perm) || !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_expert_weights(cfg, w_gate_up, s_gate_up));
+    MOE_TRY(check_expert_weights(cfg, w_down, s_down));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    const WsLayout L = ws_layout(*cfg);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void* h = at<void>(ws, L.h);
+    MOE_TRY(experts_gate_up(cfg, x_perm, offsets, w_gate_up, s_gate_up, h, ws, s));
+    return experts_down(cfg, h, offsets, w_down, s_down, y, ws, s);
+}
+
+int moe_combine(const moe_config* cfg, const void* y, const int32_t* row_of, const float* topk_w,
+                void* out, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!y || !row_of || !topk_w || !out || !aligned16(y) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    return cuda_status(launch_combine(*cfg, y, row_of, topk_w, out,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+                const void* w_gate_up, const float* s_gate_up, const void* w_down,
+                const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!x || !w_gate || !out || !aligned16(x) || !aligned16(w_gate) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_expert_weights(cfg, w_gate_up, s_gate_up));
+    MOE_TRY(check_expert_weights(cfg, w_down, s_down));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    const WsLayout L = ws_layout(*cfg);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* idx = at<int32_t>(ws, L.idx);
+    float* w = at<float>(ws, L.w);
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* row_of = at<int32_t>(ws, L.row_of);
+    void* xperm = at<void>(ws, L.xperm);
+    void* h = at<void>(ws, L.h);
+    void* y = at<void>(ws, L.y);
+    MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.control_end, s)));
+    MOE_TRY(cuda_status(launch_router(*cfg, x, w_gate, gate_bias, idx, w, at<float>(ws, L.logits),
+                                      at<int32_t>(ws, L.counters), s)));
+    MOE_TRY(cuda_status(launch_permute(*cfg, idx, x, at<int32_t>(ws, L.counts), offsets, row_of,
+                                       xperm, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.rank),
+                                       s)));
+    MOE_TRY(experts_gate_up(cfg, xperm, offsets, w_gate_up, s_gate_up, h, ws, s));
+    MOE_TRY(experts_down(cfg, h, offsets, w_down, s_down, y, ws, s));
+    return cuda_status(launch_combine(*cfg, y, row_of, w, out, s));
+}
+
+int moe_read_status(void* ws, void* stream) {
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t host = 0;
+    if (cudaMemcpyAsync(&host, ws, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof host, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    return host == 0 ? MOE_OK : (host < 0 ? host : MOE_ERR_TIMEOUT);
+}
+
+const char* moe_status_string(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument (null pointer, misalignment or flags)";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case MOE_ERR_WORKSPACE: return "workspace smaller than moe_workspace_size(cfg)";
+        case MOE_ERR_CUDA: return "CUDA launch or runtime error";
+        case MOE_ERR_TIMEOUT: return "a bounded device wait gave up";
+        default: return "unknown status code";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,133 @@
+// permute.cu -- group token-slots by expert (a stable counting sort) and gather
+// the activation rows into expert-contiguous order for the expert GEMMs.
+//
+// The pages run the experts as a loop over the selected experts with an
+// index_add_ accumulation ("DeepSeek V4-Flash 架构 QA", Q8.4) and name batched
+// / grouped matrix multiplication as the production form ("Tencent Hy3-Flash
+// QA", Q6.4). Grouping the rows of each expert contiguously is what makes the
+// grouped form possible.
+//
+// Definition (integer, bit-exact): slot s = t*k + j with expert e = idx[s] goes
+// to row offsets[e] + #{s' < s : idx[s'] == e}; offsets is the exclusive prefix
+// sum of the per-expert counts.
+//
+// Three launches:
+//   rank    one warp per chunk of kPermuteChunk slots: rank of each slot among
+//           the earlier slots of its chunk with the same expert
+//           (__match_any_sync per 32-slot group + running per-expert counters
+//           in shared memory), and the chunk's per-expert histogram;
+//   scan    one CTA: per expert, exclusive prefix over chunks (the chunk base),
+//           the totals (counts) and the exclusive prefix over experts (offsets);
+//   scatter one warp per slot: row = offsets[e] + chunk base + rank; copies the
+//           token's d-element row into x_perm with 16-byte vectors.
+// Slots whose expert id is outside [0, E) are dropped: row_of = -1.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int CH = kPermuteChunk;
+
+__global__ void __launch_bounds__(32)
+permute_rank_kernel(const int* __restrict__ idx, long R, int E, int* __restrict__ hist,
+                    int* __restrict__ rank) {
+    __shared__ int cnt[256];
+    const int lane = threadIdx.x;
+    for (int e = lane; e < E; e += 32) cnt[e] = 0;
+    __syncwarp();
+    const long base = (long)blockIdx.x * CH;
+    for (int g = 0; g < CH; g += 32) {
+        const long s = base + g + lane;
+        int e = (s < R) ? idx[s] : -1;
+        if (e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int before = (e >= 0) ? cnt[e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) cnt[e] = before + __popc(peers);
+        __syncwarp();
+        if (s < R) rank[s] = before + __popc(peers & ((1u << lane) - 1u));
+    }
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) hist[(long)blockIdx.x * E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(256)
+permute_scan_kernel(int* __restrict__ hist, int C, int E, int* __restrict__ counts,
+                    int* __restrict__ offsets) {
+    __shared__ int tile[32][256];
+    __shared__ int tot[256];
+    const int e = threadIdx.x;
+    int running = 0;
+    for (int c0 = 0; c0 < C; c0 += 32) {
+        const int nc = min(32, C - c0);
+        __syncthreads();
+        for (int v = threadIdx.x; v < nc * E; v += blockDim.x)
+            tile[v / E][v % E] = hist[(long)c0 * E + v];
+        __syncthreads();
+        if (e < E)
+            for (int c = 0; c < nc; ++c) {
+                const int v = tile[c][e];
+                tile[c][e] = running;
+                running += v;
+            }
+        __syncthreads();
+        for (int v = threadIdx.x; v < nc * E; v += blockDim.x)
+            hist[(long)c0 * E + v] = tile[v / E][v % E];
+    }
+    tot[e] = (e < E) ? running : 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int i = 0; i < E; ++i) {
+            const int v = tot[i];
+            tot[i] = acc;
+            acc += v;
+        }
+        offsets[E] = acc;
+    }
+    __syncthreads();
+    if (e < E) {
+        counts[e] = running;
+        offsets[e] = tot[e];
+    }
+}
+
+__global__ void __launch_bounds__(256)
+permute_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ hist,
+                       const int* __restrict__ rank, const int* __restrict__ offsets,
+                       const __nv_bfloat16* __restrict__ x, long R, int k, int E, int d,
+                       int* __restrict__ row_of, __nv_bfloat16* __restrict__ xperm) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long s = (long)blockIdx.x * 8 + warp;
+    if (s >= R) return;
+    const int e = idx[s];
+    if (e < 0 || e >= E) {
+        if (lane == 0) row_of[s] = -1;
+        return;
+    }
+    const long c = s / CH;
+    const int row = offsets[e] + hist[c * E + e] + rank[s];
+    if (lane == 0) row_of[s] = row;
+    const long t = s / k;
+    const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xperm + (long)row * d);
+    for (int v = lane; v < d / 8; v += 32) dst[v] = src[v];
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
+                           int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,
+                           int32_t* rank, cudaStream_t s) {
+    const long R = (long)c.T * c.k;
+    const int C = n_permute_chunks(c);
+    permute_rank_kernel<<<C, 32, 0, s>>>(idx, R, c.E, hist, rank);
+    permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, c.E, counts, offsets);
+    permute_scatter_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
+        idx, hist, rank, offsets, static_cast<const __nv_bfloat16*>(x), R, c.k, c.E, c.d, row_of,
+        static_cast<__nv_bfloat16*>(x_perm));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

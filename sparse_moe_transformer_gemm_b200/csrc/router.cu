@@ -1,0 +1,177 @@
+// router.cu -- fused router: logits GEMM (fp32 accumulate), sigmoid, top-k
+// with lowest-index tie-break, renormalisation over the selected scores and
+// the router scaling factor.
+//
+// Method: "Tencent Hy3-295B 架构深度拆解" (pillumina.github.io) §4.1 -- the
+// router computes fp32 logits F.linear(x.float(), W.float()), scores them with
+// an element-wise sigmoid, selects the top-8, renormalises the selected
+// sigmoid scores to sum to 1 and multiplies by router_scaling_factor 2.826.
+// The optional per-expert bias is added to the logits before the sigmoid
+// (Hy3 commentary, wmrh.cn/news/24252, §3.3).
+//
+// Structure: CTA (expert block b, token group g) computes the logits of
+// kRouterTokens tokens x kRouterExperts experts on CUDA cores and writes them
+// to the fp32 scratch logits[T, E]. The last CTA of a token group to finish
+// (an arrival counter, no waiting) reads the group's complete logit rows and
+// runs the selection: one warp per token, k rounds of a warp-wide argmax.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int RT = kRouterTokens;    // tokens per CTA
+constexpr int RE = kRouterExperts;   // experts per CTA
+constexpr int RWARPS = 8;
+constexpr int EPW = RE / RWARPS;     // experts per warp
+constexpr int KC = 1024;             // x columns staged per chunk
+static_assert(RT == RWARPS, "selection uses one warp per token");
+
+__global__ void __launch_bounds__(RWARPS * 32)
+router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wg,
+              const float* __restrict__ bias, int T, int d, int E, int k, float scale,
+              float* __restrict__ logits, int* __restrict__ counters, int* __restrict__ idx_out,
+              float* __restrict__ w_out) {
+    __shared__ __align__(16) float xs[RT][KC];
+    __shared__ int s_last;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e_base = blockIdx.x * RE + warp * EPW;
+    const int t0 = blockIdx.y * RT;
+
+    float acc[EPW][RT];
+#pragma unroll
+    for (int a = 0; a < EPW; ++a)
+#pragma unroll
+        for (int b = 0; b < RT; ++b) acc[a][b] = 0.f;
+
+    for (int kc = 0; kc < d; kc += KC) {
+        const int kw = min(KC, d - kc);  // multiple of 128
+        const int v8 = kw / 8;
+        __syncthreads();
+        for (int v = threadIdx.x; v < RT * v8; v += blockDim.x) {
+            const int tt = v / v8, c8 = (v - tt * v8) * 8;
+            float f[8];
+            if (t0 + tt < T) {
+                uint4 u = *reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt) * d + kc + c8);
+                bf16x8_to_float(u, f);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = 0.f;
+            }
+            *reinterpret_cast<float4*>(&xs[tt][c8]) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4*>(&xs[tt][c8 + 4]) = make_float4(f[4], f[5], f[6], f[7]);
+        }
+        __syncthreads();
+        for (int c = lane * 8; c < kw; c += 256) {
+            float wv[EPW][8];
+#pragma unroll
+            for (int a = 0; a < EPW; ++a) {
+                const int e = e_base + a;
+                if (e < E) {
+                    uint4 u = *reinterpret_cast<const uint4*>(wg + (size_t)e * d + kc + c);
+                    bf16x8_to_float(u, wv[a]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) wv[a][i] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < RT; ++b) {
+                const float4 p = *reinterpret_cast<const float4*>(&xs[b][c]);
+                const float4 q = *reinterpret_cast<const float4*>(&xs[b][c + 4]);
+#pragma unroll
+                for (int a = 0; a < EPW; ++a) {
+                    float s = acc[a][b];
+                    s = fmaf(wv[a][0], p.x, s); s = fmaf(wv[a][1], p.y, s);
+                    s = fmaf(wv[a][2], p.z, s); s = fmaf(wv[a][3], p.w, s);
+                    s = fmaf(wv[a][4], q.x, s); s = fmaf(wv[a][5], q.y, s);
+                    s = fmaf(wv[a][6], q.z, s); s = fmaf(wv[a][7], q.w, s);
+                    acc[a][b] = s;
+                }
+            }
+        }
+    }
+
+#pragma unroll
+    for (int a = 0; a < EPW; ++a)
+#pragma unroll
+        for (int b = 0; b < RT; ++b) acc[a][b] = warp_sum(acc[a][b]);
+    if (lane == 0) {
+#pragma unroll
+        for (int a = 0; a < EPW; ++a)
+#pragma unroll
+            for (int b = 0; b < RT; ++b) {
+                const int e = e_base + a, t = t0 + b;
+                if (e < E && t < T) logits[(size_t)t * E + e] = acc[a][b];
+            }
+    }
+
+    // Arrival: the last expert-block CTA of this token group does the selection.
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int ticket = atomicAdd(&counters[blockIdx.y], 1);
+        s_last = (ticket == (int)gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    const int t = t0 + warp;
+    if (t < T) {
+        float sc[8];  // E <= 256: expert lane + 32*q
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int e = lane + 32 * q;
+            if (e < E) {
+                float z = __ldcg(logits + (size_t)t * E + e);
+                if (bias) z += bias[e];
+                sc[q] = sigmoidf_acc(z);
+            } else {
+                sc[q] = -1.f;
+            }
+        }
+        int my_e = 0;
+        float my_s = 0.f;
+        for (int r = 0; r < k; ++r) {
+            float bv = -2.f;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (sc[q] > bv) { bv = sc[q]; be = lane + 32 * q; }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+            }
+            if (lane == r) { my_e = be; my_s = bv; }
+            if ((be & 31) == lane) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if ((be >> 5) == q) sc[q] = -1.f;
+            }
+        }
+        float sum = 0.f;
+        for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, my_s, j);
+        if (lane < k) {
+            idx_out[(size_t)t * k + lane] = my_e;
+            w_out[(size_t)t * k + lane] = scale * my_s / sum;
+        }
+    }
+    if (threadIdx.x == 0) counters[blockIdx.y] = 0;
+}
+
+}  // namespace
+
+cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
+                          const float* gate_bias, int32_t* idx, float* w, float* logits,
+                          int32_t* counters, cudaStream_t s) {
+    dim3 grid((c.E + RE - 1) / RE, n_router_groups(c));
+    router_kernel<<<grid, RWARPS * 32, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_gate), gate_bias,
+        c.T, c.d, c.E, c.k, c.scale, logits, counters, idx, w);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

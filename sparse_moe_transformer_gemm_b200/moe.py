@@ -1,0 +1,195 @@
+"""ctypes binding of libmoe_b200.so (the C ABI of include/moe.h).
+
+Argument marshalling only: every function here turns torch tensors into device
+pointers, calls the C entry point of the same name on the current (or given)
+CUDA stream and raises ``MoeError`` on a non-zero status. All arithmetic runs
+in the library's CUDA kernels; there is no fallback. Loading fails loudly if
+the library has not been built (``python -m sparse_moe_transformer_gemm_b200.build``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED_SHAPE = -2
+MOE_ERR_WORKSPACE = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_TIMEOUT = -5
+
+MOE_FLAG_FP8_WEIGHTS = 0x1
+MOE_FLAG_STREAM_PATH = 0x2
+MOE_FLAG_GEMM_PATH = 0x4
+
+EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
+            "moe_expert_gate_up", "moe_expert_down", "moe_experts", "moe_combine", "moe_forward",
+            "moe_read_status", "moe_status_string")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("flags", ctypes.c_uint32)]
+
+    def __repr__(self):
+        return (f"MoeConfig(T={self.T}, d={self.d}, E={self.E}, k={self.k}, d_ff={self.d_ff}, "
+                f"scale={self.scale}, flags={self.flags:#x})")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {code} ({moe_status_string(code)})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe_b200.so once, declaring the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m sparse_moe_transformer_gemm_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    C = ctypes.POINTER(MoeConfig)
+    sig = {
+        "moe_workspace_size": (S, [C]),
+        "moe_workspace_init": (I, [C, P, S, P]),
+        "moe_route": (I, [C, P, P, P, P, P, P, S, P]),
+        "moe_permute": (I, [C, P, P, P, P, P, P, P, S, P]),
+        "moe_expert_gate_up": (I, [C, P, P, P, P, P, P, S, P]),
+        "moe_expert_down": (I, [C, P, P, P, P, P, P, S, P]),
+        "moe_experts": (I, [C, P, P, P, P, P, P, P, P, S, P]),
+        "moe_combine": (I, [C, P, P, P, P, P, S, P]),
+        "moe_forward": (I, [C, P, P, P, P, P, P, P, P, P, S, P]),
+        "moe_read_status": (I, [P, P]),
+        "moe_status_string": (ctypes.c_char_p, [I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def config(T: int, d: int, E: int, k: int, d_ff: int, scale: float = 2.826, fp8: bool = False,
+           path: Optional[str] = None) -> MoeConfig:
+    """Build a moe_config. path: None (automatic), "stream" or "gemm"."""
+    flags = MOE_FLAG_FP8_WEIGHTS if fp8 else 0
+    if path == "stream":
+        flags |= MOE_FLAG_STREAM_PATH
+    elif path == "gemm":
+        flags |= MOE_FLAG_GEMM_PATH
+    elif path is not None:
+        raise ValueError(f"unknown path {path!r}")
+    return MoeConfig(T, d, E, k, d_ff, scale, flags)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != MOE_OK:
+        raise MoeError(fn, rc)
+
+
+def moe_status_string(code: int) -> str:
+    return lib().moe_status_string(int(code)).decode()
+
+
+def moe_workspace_size(cfg: MoeConfig) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_workspace_init(cfg: MoeConfig, ws: torch.Tensor, stream=None) -> None:
+    _check("moe_workspace_init",
+           lib().moe_workspace_init(ctypes.byref(cfg), _p(ws), ws.numel(), _s(stream)))
+
+
+def workspace(cfg: MoeConfig, device="cuda", stream=None) -> torch.Tensor:
+    """Allocate (through torch) and initialise a workspace for cfg."""
+    n = moe_workspace_size(cfg)
+    if n == 0:
+        raise MoeError("moe_workspace_size", MOE_ERR_UNSUPPORTED_SHAPE)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    moe_workspace_init(cfg, ws, stream)
+    return ws
+
+
+def moe_route(cfg, x, w_gate, gate_bias, topk_idx, topk_w, ws, stream=None) -> None:
+    _check("moe_route", lib().moe_route(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
+                                        _p(topk_idx), _p(topk_w), _p(ws), ws.numel(), _s(stream)))
+
+
+def moe_permute(cfg, topk_idx, x, counts, offsets, row_of, x_perm, ws, stream=None) -> None:
+    _check("moe_permute", lib().moe_permute(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(counts),
+                                            _p(offsets), _p(row_of), _p(x_perm), _p(ws),
+                                            ws.numel(), _s(stream)))
+
+
+def moe_expert_gate_up(cfg, x_perm, offsets, w_gate_up, s_gate_up, h, ws, stream=None) -> None:
+    _check("moe_expert_gate_up",
+           lib().moe_expert_gate_up(ctypes.byref(cfg), _p(x_perm), _p(offsets), _p(w_gate_up),
+                                    _p(s_gate_up), _p(h), _p(ws), ws.numel(), _s(stream)))
+
+
+def moe_expert_down(cfg, h, offsets, w_down, s_down, y, ws, stream=None) -> None:
+    _check("moe_expert_down",
+           lib().moe_expert_down(ctypes.byref(cfg), _p(h), _p(offsets), _p(w_down), _p(s_down),
+                                 _p(y), _p(ws), ws.numel(), _s(stream)))
+
+
+def moe_experts(cfg, x_perm, offsets, w_gate_up, s_gate_up, w_down, s_down, y, ws,
+                stream=None) -> None:
+    _check("moe_experts",
+           lib().moe_experts(ctypes.byref(cfg), _p(x_perm), _p(offsets), _p(w_gate_up),
+                             _p(s_gate_up), _p(w_down), _p(s_down), _p(y), _p(ws), ws.numel(),
+                             _s(stream)))
+
+
+def moe_combine(cfg, y, row_of, topk_w, out, ws, stream=None) -> None:
+    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _p(y), _p(row_of), _p(topk_w),
+                                            _p(out), _p(ws), ws.numel(), _s(stream)))
+
+
+def moe_forward(cfg, x, w_gate, gate_bias, w_gate_up, s_gate_up, w_down, s_down, out, ws,
+                stream=None) -> None:
+    _check("moe_forward",
+           lib().moe_forward(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias), _p(w_gate_up),
+                             _p(s_gate_up), _p(w_down), _p(s_down), _p(out), _p(ws), ws.numel(),
+                             _s(stream)))
+
+
+def moe_read_status(ws, stream=None) -> int:
+    return int(lib().moe_read_status(_p(ws), _s(stream)))
+
+
+def layer_args(layer: dict):
+    """(w_gate_up, s_gate_up, w_down, s_down) of a synthetic layer dict, FP8 or bf16."""
+    if layer["cfg"].fp8:
+        return layer["q_gate_up"], layer["s_gate_up"], layer["q_down"], layer["s_down"]
+    return layer["w_gate_up"], None, layer["w_down"], None
+
+
+def config_of(shape, path: Optional[str] = None) -> MoeConfig:
+    """moe_config for a synthetic LayerShape."""
+    return config(shape.T, shape.d, shape.E, shape.k, shape.F, shape.scale, shape.fp8, path)

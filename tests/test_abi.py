@@ -1,0 +1,136 @@
+"""The C ABI library: builds, loads without a GPU, exports what include/moe.h
+declares, and rejects bad arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_moe_transformer_gemm_b200 import build as moe_build
+from sparse_moe_transformer_gemm_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_surface():
+    assert declared_functions() == sorted(moe.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_only_the_abi_is_exported():
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert syms == set(moe.EXPORTED)
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert moe.moe_status_string(code) and moe.moe_status_string(code) != "unknown status code"
+    assert moe.moe_status_string(-99) == "unknown status code"
+
+
+HY3 = dict(T=64, d=4096, E=192, k=8, d_ff=1536)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(T=0), dict(d=100), dict(d=4096 + 64), dict(d_ff=1000), dict(E=0), dict(E=257),
+    dict(k=0), dict(k=9, E=8), dict(k=33, E=64), dict(d=8320), dict(T=1 << 20, d_ff=4096),
+])
+def test_workspace_size_rejects_unsupported_shapes(lib, bad):
+    cfg = moe.config(**{**HY3, **bad})
+    assert moe.moe_workspace_size(cfg) == 0
+
+
+def test_workspace_size_covers_the_intermediates(lib):
+    cfg = moe.config(**HY3)
+    n = moe.moe_workspace_size(cfg)
+    R = 64 * 8
+    assert n >= R * 4096 * 2 * 2 + R * 1536 * 2   # x_perm + y + h
+    big = moe.config(**{**HY3, "T": 4096})
+    assert moe.moe_workspace_size(big) > 60 * n
+
+
+FAKE = 0x10000  # an aligned address that is never dereferenced: every call below fails first
+
+
+def _call(fn, *args):
+    return getattr(moe.lib(), fn)(*args)
+
+
+def test_null_pointers_and_bad_flags_are_invalid_args(lib):
+    cfg = moe.config(**HY3)
+    ws_n = moe.moe_workspace_size(cfg)
+    P = ctypes.c_void_p
+    # moe_route with a NULL x
+    rc = _call("moe_route", ctypes.byref(cfg), None, P(FAKE), None, P(FAKE), P(FAKE), P(FAKE),
+               ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    # misaligned x
+    rc = _call("moe_route", ctypes.byref(cfg), P(FAKE + 2), P(FAKE), None, P(FAKE), P(FAKE),
+               P(FAKE), ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    # both path flags
+    both = moe.config(**HY3)
+    both.flags = moe.MOE_FLAG_STREAM_PATH | moe.MOE_FLAG_GEMM_PATH
+    assert moe.moe_workspace_size(both) == 0
+    # unknown flag bit
+    unk = moe.config(**HY3)
+    unk.flags = 0x100
+    assert moe.moe_workspace_size(unk) == 0
+    # bf16 weights given scales, FP8 weights without scales
+    rc = _call("moe_expert_gate_up", ctypes.byref(cfg), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+               P(FAKE), P(FAKE), ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    fp8 = moe.config(**HY3, fp8=True)
+    rc = _call("moe_expert_gate_up", ctypes.byref(fp8), P(FAKE), P(FAKE), P(FAKE), None,
+               P(FAKE), P(FAKE), ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    # misaligned workspace
+    rc = _call("moe_combine", ctypes.byref(cfg), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+               P(FAKE + 16), ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+
+
+def test_small_workspace_is_reported(lib):
+    cfg = moe.config(**HY3)
+    ws_n = moe.moe_workspace_size(cfg)
+    P = ctypes.c_void_p
+    rc = _call("moe_forward", ctypes.byref(cfg), P(FAKE), P(FAKE), None, P(FAKE), None, P(FAKE),
+               None, P(FAKE), P(FAKE), ws_n - 256, None)
+    assert rc == moe.MOE_ERR_WORKSPACE
+
+
+def test_unsupported_shape_is_reported_by_every_entry_point(lib):
+    cfg = moe.config(**{**HY3, "d": 100})
+    P = ctypes.c_void_p
+    f = P(FAKE)
+    cases = {
+        "moe_route": (f, f, None, f, f, f, 1 << 30, None),
+        "moe_permute": (f, f, f, f, f, f, f, 1 << 30, None),
+        "moe_expert_gate_up": (f, f, f, None, f, f, 1 << 30, None),
+        "moe_expert_down": (f, f, f, None, f, f, 1 << 30, None),
+        "moe_experts": (f, f, f, None, f, None, f, f, 1 << 30, None),
+        "moe_combine": (f, f, f, f, f, 1 << 30, None),
+        "moe_forward": (f, f, None, f, None, f, None, f, f, 1 << 30, None),
+    }
+    for fn, args in cases.items():
+        assert _call(fn, ctypes.byref(cfg), *args) == moe.MOE_ERR_UNSUPPORTED_SHAPE, fn

@@ -1,0 +1,176 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small shapes are compared on every token; the full Hy3 shapes route every
+token through both sides and compare the layer output on a seeded sample of
+tokens, in the launch configuration the benchmark uses (moe_forward with the
+automatic path choice). Tolerances are in tests/parity.py.
+"""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from sparse_moe_transformer_gemm_b200 import build as moe_build
+from sparse_moe_transformer_gemm_b200 import moe
+from synthetic import CONFIGS, LayerShape, make_layer
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": CONFIGS["tiny"],
+    # several 128-row weight tiles, ~75 rows per expert, ragged token tiles
+    "ragged": LayerShape(T=300, d=512, E=32, k=8, F=384),
+    "single_token": LayerShape(T=1, d=256, E=16, k=4, F=128),
+    "k_equals_E": LayerShape(T=20, d=256, E=8, k=8, F=128),
+    "top1": LayerShape(T=50, d=256, E=16, k=1, F=128),
+    "tiny_fp8": dataclasses.replace(CONFIGS["tiny"], fp8=True),
+    "ragged_skewed": LayerShape(T=300, d=512, E=32, k=8, F=384, zipf_bias=True),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    moe_build.build()
+    oracle.build()
+    assert torch.cuda.is_available()
+    torch.cuda.init()
+
+
+def _free(*objs):
+    for o in objs:
+        del o
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+@pytest.mark.parametrize("path", [None, "stream"])
+def test_small_shapes_every_token(name, path):
+    layer = make_layer(SMALL[name], seed=1, device="cuda")
+    route = parity.gpu_route(layer, path)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias)
+    parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer, path)
+    res = parity.check_forward(layer, out, None, route)
+    print(name, path, res)
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "skewed", "fp8"])
+def test_hy3_shapes(name):
+    shape = CONFIGS[name]
+    layer = make_layer(shape, seed=0, device="cuda")
+    route = parity.gpu_route(layer)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias)
+    near = parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer)
+    toks = parity.sample_tokens(shape.T, n=48 if shape.T > 64 else 64)
+    toks = np.unique(np.concatenate([toks, near[:8].astype(np.int32)]))
+    res = parity.check_forward(layer, out, toks, route)
+    print(name, "near-tie tokens:", len(near), near[:16].tolist(), res)
+    _free(layer, out)
+
+
+def test_all_tokens_to_the_same_experts():
+    """A logit bias of +40 on experts 0..3 sends every token to them (64 rows each);
+    the other twelve experts are empty."""
+    shape = CONFIGS["tiny"]
+    layer = make_layer(shape, seed=2, device="cuda")
+    b = torch.zeros(shape.E, dtype=torch.float32, device="cuda")
+    b[:4] = 40.0
+    layer["gate_bias"] = b
+    route = parity.gpu_route(layer)
+    assert np.all(np.sort(route[0], axis=1) == np.arange(4))
+    for path in (None, "stream"):
+        out = parity.gpu_forward(layer, path)
+        parity.check_forward(layer, out, None, route)
+
+
+def test_permute_is_bit_exact():
+    shape = LayerShape(T=3000, d=256, E=64, k=8, F=128)
+    layer = make_layer(shape, seed=3, device="cuda", with_experts=False)
+    cfg = moe.config_of(shape)
+    ws = moe.workspace(cfg)
+    T, k, E, d = shape.T, shape.k, shape.E, shape.d
+    idx, _ = parity.gpu_route(layer)
+    idx_d = torch.from_numpy(idx).cuda()
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    xp = torch.empty((T * k, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(cfg, idx_d, layer["x"], counts, offsets, row_of, xp, ws)
+    torch.cuda.synchronize()
+    ref = oracle.permute(idx, E)
+    assert np.array_equal(counts.cpu().numpy(), ref["counts"])
+    assert np.array_equal(offsets.cpu().numpy(), ref["offsets"])
+    assert np.array_equal(row_of.cpu().numpy(), ref["row_of"])
+    xb = oracle.bf16_bits(layer["x"])
+    xpb = oracle.bf16_bits(xp)
+    rows = ref["row_of"].reshape(T, k)
+    for j in range(k):
+        assert np.array_equal(xpb[rows[:, j]], xb)
+
+
+def test_fp32_combine_keeps_small_terms():
+    """Hy3 commentary §2.3 example: one branch output 8.2 and seven of 0.03 (all
+    already bf16). An fp32 sum gives 8.375 after the cast; a bf16 running sum
+    would stay at 8.1875."""
+    cfg = moe.config(T=1, d=128, E=8, k=8, d_ff=128)
+    ws = moe.workspace(cfg)
+    y = torch.full((8, 128), 0.030029296875, dtype=torch.bfloat16, device="cuda")
+    y[0] = 8.1875
+    row_of = torch.arange(8, dtype=torch.int32, device="cuda")
+    w = torch.ones(8, dtype=torch.float32, device="cuda")
+    out = torch.empty((1, 128), dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(cfg, y, row_of, w, out, ws)
+    torch.cuda.synchronize()
+    assert torch.all(out.float() == 8.375)
+
+
+def test_stage_calls_match_moe_forward_bitwise():
+    shape = SMALL["ragged"]
+    layer = make_layer(shape, seed=4, device="cuda")
+    cfg = moe.config_of(shape)
+    ws = moe.workspace(cfg)
+    T, k, E, d, F = shape.T, shape.k, shape.E, shape.d, shape.F
+    R = T * k
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(R, dtype=torch.int32, device="cuda")
+    xp = torch.empty((R, d), dtype=torch.bfloat16, device="cuda")
+    h = torch.empty((R, F), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((R, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    wgu, sgu, wd, sd = moe.layer_args(layer)
+    moe.moe_route(cfg, layer["x"], layer["w_gate"], None, idx, w, ws)
+    moe.moe_permute(cfg, idx, layer["x"], counts, offsets, row_of, xp, ws)
+    moe.moe_expert_gate_up(cfg, xp, offsets, wgu, sgu, h, ws)
+    moe.moe_expert_down(cfg, h, offsets, wd, sd, y, ws)
+    moe.moe_combine(cfg, y, row_of, w, out, ws)
+    full = parity.gpu_forward(layer)
+    assert torch.equal(out, full)
+    # the expert pieces against the oracle, row by row
+    xpb = oracle.bf16_bits(xp)
+    rows = np.arange(R)
+    experts = np.searchsorted(offsets.cpu().numpy(), rows, side="right") - 1
+    O = oracle.OracleLayer(layer)
+    y_ref, h_ref = oracle.expert_rows(xpb, experts.astype(np.int32), O.wgu, O.wd, want_h=True)
+    h_gpu = oracle.double_from_bf16(oracle.bf16_bits(h))
+    rel_h = np.linalg.norm(h_gpu - h_ref) / np.linalg.norm(h_ref)
+    assert rel_h < 4e-3, rel_h
+    y_gpu = oracle.double_from_bf16(oracle.bf16_bits(y))
+    rel_y = np.linalg.norm(y_gpu - y_ref) / np.linalg.norm(y_ref)
+    assert rel_y < 8e-3, rel_y
+
+
+def test_repeated_calls_are_bitwise_deterministic():
+    layer = make_layer(SMALL["ragged_skewed"], seed=5, device="cuda")
+    a = parity.gpu_forward(layer).clone()
+    b = parity.gpu_forward(layer)
+    assert torch.equal(a, b)
