@@ -188,6 +188,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (a smaller case of the same workload, e.g. for ncu)")
+    ap.add_argument("--tokens", type=int, default=None, help="override T")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     if args.steps is None:
@@ -214,6 +217,10 @@ def main():
         pg = dist
 
     shape = CONFIGS[args.config]
+    if args.experts or args.tokens:
+        import dataclasses
+
+        shape = dataclasses.replace(shape, E=args.experts or shape.E, T=args.tokens or shape.T)
     layer = make_layer(shape, seed=rank, device=dev)
     cfg = moe.config_of(shape, None if args.path == "auto" else args.path)
     T, d, E, k, F = shape.T, shape.d, shape.E, shape.k, shape.F
@@ -295,8 +302,7 @@ def main():
     dominant = max(("gate_up", "down"), key=lambda s: stage_ms[s])
     dom_work = gw if dominant == "gate_up" else dw
     dom_s = stage_ms[dominant] / 1e3
-    kernel_name = f"{dominant}_{'gemm' if args.path == 'gemm' else 'stream'}"
-    use_stream = args.path == "stream" or (args.path == "auto" and T * k <= 8 * E)
+    use_stream = args.path == "stream" or (args.path == "auto" and fp8)
     kernel_name = f"{dominant}_{'stream' if use_stream else 'gemm'}"
     if use_stream:
         achieved = dom_work["bytes"] / dom_s / 1e9
@@ -356,7 +362,8 @@ def main():
             "dtype": "e4m3 weights, bf16 activations, fp32 accumulate" if fp8 else
                      "bf16 (fp32 accumulate, fp32 combine)",
             "data": "synthetic (seeded; random-init weights of the Hy3 MoE layer shapes)",
-            "config": {"workload": WORKLOADS[args.config], "T": T, "d": d, "E": E, "k": k,
+            "config": {"workload": WORKLOADS[args.config] if shape == CONFIGS[args.config] else
+                       f"smaller case of {args.config}: T={T}, E={E}", "T": T, "d": d, "E": E, "k": k,
                        "d_ff": F, "path": args.path, "parallelism": f"replicas x{world}",
                        "l2": "no flush: each step streams the touched experts' weights "
                              f"({touched} experts, {touched * work.expert_bytes(d, F, fp8) / 1e9:.2f} GB) "

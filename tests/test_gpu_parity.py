@@ -47,8 +47,10 @@ def _free(*objs):
 
 
 @pytest.mark.parametrize("name", sorted(SMALL))
-@pytest.mark.parametrize("path", [None, "stream"])
+@pytest.mark.parametrize("path", [None, "stream", "gemm"])
 def test_small_shapes_every_token(name, path):
+    if path == "gemm" and SMALL[name].fp8:
+        pytest.skip("FP8 weights run on the streaming kernels")
     layer = make_layer(SMALL[name], seed=1, device="cuda")
     route = parity.gpu_route(layer, path)
     O = oracle.OracleLayer(layer)
@@ -57,6 +59,15 @@ def test_small_shapes_every_token(name, path):
     out = parity.gpu_forward(layer, path)
     res = parity.check_forward(layer, out, None, route)
     print(name, path, res)
+
+
+def test_gemm_path_on_decode_shape_matches_stream_path():
+    layer = make_layer(CONFIGS["decode"], seed=0, device="cuda")
+    a = parity.gpu_forward(layer, "stream").clone()
+    b = parity.gpu_forward(layer, "gemm")
+    rel, mx = parity.compare_out(oracle.bf16_bits(a), oracle.bf16_bits(b))
+    assert rel < 4e-3 and mx < 3e-2, (rel, mx)
+    _free(layer, a, b)
 
 
 @pytest.mark.parametrize("name", ["decode", "prefill", "skewed", "fp8"])
@@ -75,17 +86,18 @@ def test_hy3_shapes(name):
     _free(layer, out)
 
 
-def test_all_tokens_to_the_same_experts():
-    """A logit bias of +40 on experts 0..3 sends every token to them (64 rows each);
-    the other twelve experts are empty."""
-    shape = CONFIGS["tiny"]
+@pytest.mark.parametrize("T", [64, 700])
+def test_all_tokens_to_the_same_experts(T):
+    """A logit bias of +40 on experts 0..3 sends every token to them (T rows each,
+    split into several token tiles when T > 256); the other twelve are empty."""
+    shape = dataclasses.replace(CONFIGS["tiny"], T=T)
     layer = make_layer(shape, seed=2, device="cuda")
     b = torch.zeros(shape.E, dtype=torch.float32, device="cuda")
     b[:4] = 40.0
     layer["gate_bias"] = b
     route = parity.gpu_route(layer)
     assert np.all(np.sort(route[0], axis=1) == np.arange(4))
-    for path in (None, "stream"):
+    for path in (None, "stream", "gemm"):
         out = parity.gpu_forward(layer, path)
         parity.check_forward(layer, out, None, route)
 
