@@ -146,6 +146,25 @@ MOE_API int moe_forward(const moe_config* cfg, const void* x, const void* w_gate
                 const void* w_gate_up, const float* s_gate_up, const void* w_down,
                 const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of the fixed device array behind moe_route_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/* moe_route for callers that cannot allocate device memory (no workspace
+ * argument). The pages have no counterpart: this is a deployment convenience.
+ * Same routing as moe_route, bitwise. Its scratch -- fp32 logits [T, E] and
+ * one counter per 8 tokens -- lives in a device array of
+ * MOE_NOALLOC_SCRATCH_BYTES compiled into the library, held on every GPU that
+ * loads it until the process exits. Returns MOE_ERR_UNSUPPORTED_SHAPE when
+ * 4*T*E plus the counters (4*ceil(T/8) bytes, rounded up to 256) exceed that
+ * size (T <= 2728 at E = 192), besides the shape checks of moe_route. The
+ * first call on a device (that device current) looks up the array's address;
+ * make it before any stream capture. All calls share the array: calls that
+ * overlap on the GPU race and must be serialised by the caller. It calls no
+ * allocator. */
+MOE_API int moe_route_noalloc(const moe_config* cfg, const void* x, const void* w_gate,
+                              const float* gate_bias, int32_t* topk_idx, float* topk_w,
+                              void* stream);
+
 /* Synchronise stream, then read and clear the workspace status word: MOE_OK,
  * or MOE_ERR_TIMEOUT if a bounded device wait gave up since the last read. */
 MOE_API int moe_read_status(void* ws, void* stream);

@@ -30,7 +30,9 @@ MOE_FLAG_GEMM_PATH = 0x4
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
             "moe_expert_gate_up", "moe_expert_down", "moe_experts", "moe_combine", "moe_forward",
-            "moe_read_status", "moe_status_string")
+            "moe_read_status", "moe_status_string", "moe_route_noalloc")
+
+MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 
 class MoeConfig(ctypes.Structure):
@@ -75,6 +77,7 @@ def lib() -> ctypes.CDLL:
         "moe_forward": (I, [C, P, P, P, P, P, P, P, P, P, S, P]),
         "moe_read_status": (I, [P, P]),
         "moe_status_string": (ctypes.c_char_p, [I]),
+        "moe_route_noalloc": (I, [C, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -177,6 +180,14 @@ def moe_forward(cfg, x, w_gate, gate_bias, w_gate_up, s_gate_up, w_down, s_down,
            lib().moe_forward(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias), _p(w_gate_up),
                              _p(s_gate_up), _p(w_down), _p(s_down), _p(out), _p(ws), ws.numel(),
                              _s(stream)))
+
+
+def moe_route_noalloc(cfg, x, w_gate, gate_bias, topk_idx, topk_w, stream=None) -> None:
+    """moe_route without a workspace, for callers that cannot allocate device
+    memory; the scratch is a fixed 2 MiB device array inside the library."""
+    _check("moe_route_noalloc",
+           lib().moe_route_noalloc(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
+                                   _p(topk_idx), _p(topk_w), _s(stream)))
 
 
 def moe_read_status(ws, stream=None) -> int:
