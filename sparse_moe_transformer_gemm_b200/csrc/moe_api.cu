@@ -68,6 +68,18 @@ bool use_stream_path(const moe_config* c) {
     return (c->flags & MOE_FLAG_FP8_WEIGHTS) != 0;
 }
 
+// Router: tensor-core kernel where it applies (k <= 8, E a multiple of 4),
+// CUDA-core kernel otherwise.
+cudaError_t route(const moe_config* c, const void* x, const void* w_gate, const float* gate_bias,
+                  int32_t* idx, float* w, void* ws, cudaStream_t s) {
+    const WsLayout L = ws_layout(*c);
+    if (router_tc_supported(*c))
+        return launch_router_tc(*c, x, w_gate, gate_bias, idx, w, at<float>(ws, L.logits),
+                                at<int32_t>(ws, L.counters), at<int>(ws, L.status), s);
+    return launch_router(*c, x, w_gate, gate_bias, idx, w, at<float>(ws, L.logits),
+                         at<int32_t>(ws, L.counters), s);
+}
+
 int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offsets,
                     const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
                     cudaStream_t s) {
@@ -109,10 +121,8 @@ int moe_route(const moe_config* cfg, const void* x, const void* w_gate, const fl
     if (!x || !w_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_ws(cfg, ws, ws_bytes));
-    const WsLayout L = ws_layout(*cfg);
-    return cuda_status(launch_router(*cfg, x, w_gate, gate_bias, topk_idx, topk_w,
-                                     at<float>(ws, L.logits), at<int32_t>(ws, L.counters),
-                                     static_cast<cudaStream_t>(stream)));
+    return cuda_status(route(cfg, x, w_gate, gate_bias, topk_idx, topk_w, ws,
+                             static_cast<cudaStream_t>(stream)));
 }
 
 int moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x, int32_t* counts,
@@ -195,8 +205,7 @@ int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const 
     void* h = at<void>(ws, L.h);
     void* y = at<void>(ws, L.y);
     MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.control_end, s)));
-    MOE_TRY(cuda_status(launch_router(*cfg, x, w_gate, gate_bias, idx, w, at<float>(ws, L.logits),
-                                      at<int32_t>(ws, L.counters), s)));
+    MOE_TRY(cuda_status(route(cfg, x, w_gate, gate_bias, idx, w, ws, s)));
     MOE_TRY(cuda_status(launch_permute(*cfg, idx, x, at<int32_t>(ws, L.counts), offsets, row_of,
                                        xperm, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.rank),
                                        s)));

@@ -29,6 +29,9 @@ SMALL = {
     "top1": LayerShape(T=50, d=256, E=16, k=1, F=128),
     "tiny_fp8": dataclasses.replace(CONFIGS["tiny"], fp8=True),
     "ragged_skewed": LayerShape(T=300, d=512, E=32, k=8, F=384, zipf_bias=True),
+    # the CUDA-core router (k > 8, or E not a multiple of 4)
+    "k12": LayerShape(T=100, d=256, E=32, k=12, F=128),
+    "e18": LayerShape(T=90, d=256, E=18, k=4, F=128),
 }
 
 
