@@ -46,17 +46,6 @@ inline int n_permute_chunks(const moe_config& c) {
     return (int)((R + kPermuteChunk - 1) / kPermuteChunk);
 }
 
-int router_splits(int T, int d);  // K splits per 128-token tile of the tensor-core router
-
-// fp32 scratch of the router: logits [T, E] (CUDA-core kernel) or the split-K
-// partial logits [S, T rounded up to 128, E] (tensor-core kernel).
-inline size_t router_scratch_floats(const moe_config& c) {
-    const size_t a = (size_t)c.T * c.E;
-    const size_t t_pad = (size_t)((c.T + 127) / 128) * 128;
-    const size_t b = (size_t)router_splits(c.T, c.d) * t_pad * c.E;
-    return a > b ? a : b;
-}
-
 inline WsLayout ws_layout(const moe_config& c) {
     WsLayout L{};
     size_t R = (size_t)c.T * c.k;
@@ -64,7 +53,7 @@ inline WsLayout ws_layout(const moe_config& c) {
     L.status = o;   o += 256;
     L.counters = o; o = align256(o + sizeof(int32_t) * n_router_groups(c));
     L.control_end = o;
-    L.logits = o;   o = align256(o + sizeof(float) * router_scratch_floats(c));
+    L.logits = o;   o = align256(o + sizeof(float) * (size_t)c.T * c.E);
     L.hist = o;     o = align256(o + sizeof(int32_t) * (size_t)n_permute_chunks(c) * c.E);
     L.rank = o;     o = align256(o + sizeof(int32_t) * R);
     L.idx = o;      o = align256(o + sizeof(int32_t) * R);
@@ -87,8 +76,8 @@ cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate
 
 bool router_tc_supported(const moe_config& c);
 cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_gate,
-                             const float* gate_bias, int32_t* idx, float* w, float* part,
-                             int32_t* counters, int* status, cudaStream_t s);
+                             const float* gate_bias, int32_t* idx, float* w, int* status,
+                             cudaStream_t s);
 
 cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
                            int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,

@@ -68,14 +68,12 @@ bool use_stream_path(const moe_config* c) {
     return (c->flags & MOE_FLAG_FP8_WEIGHTS) != 0;
 }
 
-// Router: tensor-core kernel where it applies (k <= 8, E a multiple of 4),
-// CUDA-core kernel otherwise.
+// Router: tensor-core kernel where it applies (k <= 8), CUDA-core kernel otherwise.
 cudaError_t route(const moe_config* c, const void* x, const void* w_gate, const float* gate_bias,
                   int32_t* idx, float* w, void* ws, cudaStream_t s) {
     const WsLayout L = ws_layout(*c);
     if (router_tc_supported(*c))
-        return launch_router_tc(*c, x, w_gate, gate_bias, idx, w, at<float>(ws, L.logits),
-                                at<int32_t>(ws, L.counters), at<int>(ws, L.status), s);
+        return launch_router_tc(*c, x, w_gate, gate_bias, idx, w, at<int>(ws, L.status), s);
     return launch_router(*c, x, w_gate, gate_bias, idx, w, at<float>(ws, L.logits),
                          at<int32_t>(ws, L.counters), s);
 }

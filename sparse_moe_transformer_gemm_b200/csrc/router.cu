@@ -13,7 +13,9 @@
 // kRouterTokens tokens x kRouterExperts experts on CUDA cores and writes them
 // to the fp32 scratch logits[T, E]. The last CTA of a token group to finish
 // (an arrival counter, no waiting) reads the group's complete logit rows and
-// runs the selection: one warp per token, k rounds of a warp-wide argmax.
+// runs the selection: one warp per token, k rounds of a warp-wide argmax over
+// the (biased) logits -- the sigmoid is increasing, so this selects the k
+// largest scores -- and the sigmoid of the k selected.
 #include "common.cuh"
 #include "internal.h"
 
@@ -119,6 +121,8 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 
     const int t = t0 + warp;
     if (t < T) {
+        // The sigmoid is increasing: select on the (biased) logits, evaluate the
+        // sigmoid for the selected ones only.
         float sc[8];  // E <= 256: expert lane + 32*q
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -126,15 +130,15 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
             if (e < E) {
                 float z = __ldcg(logits + (size_t)t * E + e);
                 if (bias) z += bias[e];
-                sc[q] = sigmoidf_acc(z);
+                sc[q] = z;
             } else {
-                sc[q] = -1.f;
+                sc[q] = -INFINITY;
             }
         }
         int my_e = 0;
         float my_s = 0.f;
         for (int r = 0; r < k; ++r) {
-            float bv = -2.f;
+            float bv = -INFINITY;
             int be = 0x7fffffff;
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -145,11 +149,11 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
                 const int oe = __shfl_xor_sync(0xffffffffu, be, o);
                 if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
             }
-            if (lane == r) { my_e = be; my_s = bv; }
+            if (lane == r) { my_e = be; my_s = sigmoidf_acc(bv); }
             if ((be & 31) == lane) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    if ((be >> 5) == q) sc[q] = -1.f;
+                    if ((be >> 5) == q) sc[q] = -INFINITY;
             }
         }
         float sum = 0.f;

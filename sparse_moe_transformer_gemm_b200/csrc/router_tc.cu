@@ -7,17 +7,20 @@
 //
 // Tile: 128 tokens (MMA M, tokens in TMEM lanes) x all E experts (MMA N = E
 // rounded up to 16, <= 256) over a K slice of the hidden size, bf16 x bf16 ->
-// fp32. So that small batches still spread over the GPU, the K dimension is
-// split over S CTAs per token tile (S chosen so that tiles * S ~ SM count).
-// Every CTA writes its fp32 partial logits [128, E] to the workspace; the last
-// CTA of a token tile to arrive (arrival counter, no waiting) adds the S
-// partials in split order -- the result does not depend on arrival order --
-// and selects per token in-thread: one epilogue thread per token scans the E
-// sigmoid scores keeping a sorted top-k list (strictly greater enters, so an
-// equal score never displaces a lower expert index).
+// fp32. So that small batches still spread over the GPU, the hidden dimension
+// is split over S in {1, 2, 4, 8} CTAs per token tile, launched as one thread-
+// block cluster. Each CTA moves its partial logits from TMEM to its own shared
+// memory; after a cluster barrier, CTA j sums rows [j*128/S, (j+1)*128/S) over
+// the S CTAs through distributed shared memory, in split order (the result
+// does not depend on timing), and selects for those rows: one thread per
+// token scans its E logits keeping a sorted top-k list. The sigmoid is
+// increasing, so the k largest (biased) logits are the k largest scores;
+// strictly greater enters, so an equal value never displaces a lower expert
+// index. The sigmoid is evaluated for the k selected only.
 //
 // CTA: 192 threads -- warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
-// warps 2-5 epilogue / selection. Waits are bounded (MOE_ERR_TIMEOUT).
+// warps 2-5 epilogue / reduction / selection. Waits are bounded
+// (MOE_ERR_TIMEOUT in the status word).
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -26,7 +29,7 @@
 
 namespace moe {
 
-int router_splits(int T, int d);  // defined below, also used for the workspace size
+int router_splits(int T, int d);  // defined below
 
 namespace {
 
@@ -46,15 +49,16 @@ struct Ctrl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    int last;
 };
 
 constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Ctrl);
-static_assert(BM * (256 + 1) * 4 <= STAGES * STAGE_BYTES, "selection rows fit in the stage ring");
+static_assert(BM * (256 + 1) * 4 <= STAGES * STAGE_BYTES, "logit rows fit in the stage ring");
 
 // Top-k of one token from its E logits (a shared-memory row), then the
-// renormalised, scaled weights. Strictly greater enters the sorted list, so
-// an equal score never displaces a lower expert index.
+// renormalised, scaled weights. The sigmoid is strictly increasing, so the k
+// largest scores are the k largest (biased) logits; equal logits -- equal
+// scores -- keep the lower expert index because only a strictly greater value
+// enters the sorted list. The sigmoid is evaluated for the k selected only.
 template <int K>
 __device__ __forceinline__ void select_topk(const float* row, const float* __restrict__ bias, int E,
                                             float scale, int* __restrict__ idx_out,
@@ -62,11 +66,11 @@ __device__ __forceinline__ void select_topk(const float* row, const float* __res
     float v[K];
     int id[K];
 #pragma unroll
-    for (int j = 0; j < K; ++j) { v[j] = -1.f; id[j] = 0; }
+    for (int j = 0; j < K; ++j) { v[j] = -INFINITY; id[j] = 0; }
     for (int e = 0; e < E; ++e) {
-        const float sc = sigmoidf_acc(bias ? row[e] + __ldg(bias + e) : row[e]);
-        if (sc > v[K - 1]) {
-            v[K - 1] = sc;
+        const float z = bias ? row[e] + __ldg(bias + e) : row[e];
+        if (z > v[K - 1]) {
+            v[K - 1] = z;
             id[K - 1] = e;
 #pragma unroll
             for (int j = K - 1; j > 0; --j) {
@@ -79,7 +83,10 @@ __device__ __forceinline__ void select_topk(const float* row, const float* __res
     }
     float sum = 0.f;
 #pragma unroll
-    for (int j = 0; j < K; ++j) sum += v[j];
+    for (int j = 0; j < K; ++j) {
+        v[j] = sigmoidf_acc(v[j]);
+        sum += v[j];
+    }
 #pragma unroll
     for (int j = 0; j < K; ++j) {
         idx_out[j] = id[j];
@@ -87,22 +94,25 @@ __device__ __forceinline__ void select_topk(const float* row, const float* __res
     }
 }
 
-// grid: (token tiles, splits). tmX: x [T, d] box 64 x 128; tmW: W_gate [E, d] box 64 x n_pad.
-// part: fp32 [S][T_pad][E]; counters: one per token tile (zero on entry, reset on exit).
+// grid: (token tiles, S) with clusters of (1, S). tmX: x [T, d] box 64 x 128;
+// tmW: W_gate [E, d] box 64 x n_pad.
+template <int S>
 __global__ void __launch_bounds__(THREADS, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ bias, int T, int d, int E, int k, int n_pad,
-                 float scale, float* __restrict__ part, int* __restrict__ counters,
-                 int* __restrict__ idx_out, float* __restrict__ w_out, int* __restrict__ status) {
+                 float scale, int* __restrict__ idx_out, float* __restrict__ w_out,
+                 int* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     Ctrl& c = *reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x, split = blockIdx.y, S = gridDim.y;
+    const int tile = blockIdx.x;
+    const int split = (S > 1) ? (int)tc::cluster_ctarank() : 0;
     const int KB = d / BK;
     const int kb0 = split * KB / S, kb1 = (split + 1) * KB / S;  // S <= KB: never empty
-    const int T_pad = gridDim.x * BM;
+    const int es = E + 1;  // row stride of the logit rows in shared memory (odd: no bank conflicts)
+    float* red = reinterpret_cast<float*>(smem);  // [128][E+1], reuses the stage ring
 
     if (warp == 0 && lane == 0) {
         c.abort = 0;
@@ -110,9 +120,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         tc::prefetch_tensormap(&tmW);
     } else if (warp == 1) {
         if (lane == 0) {
-            for (int s = 0; s < STAGES; ++s) {
-                tc::mbar_init(&c.full[s], 1);
-                tc::mbar_init(&c.empty[s], 1);
+            for (int st = 0; st < STAGES; ++st) {
+                tc::mbar_init(&c.full[st], 1);
+                tc::mbar_init(&c.empty[st], 1);
             }
             tc::mbar_init(&c.acc_full, 1);
             tc::mbar_init(&c.drain, 1);
@@ -141,17 +151,17 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     atomicExch(status, MOE_ERR_TIMEOUT);
                     break;
                 }
-                uint8_t* s = smem + stage * STAGE_BYTES;
+                uint8_t* st = smem + stage * STAGE_BYTES;
                 tc::mbar_arrive_expect_tx(&c.full[stage], A_BYTES + b_bytes);
-                tc::tma_load_2d(s, &tmX, &c.full[stage], kb * BK, tile * BM);
-                tc::tma_load_2d(s + A_BYTES, &tmW, &c.full[stage], kb * BK, 0);
+                tc::tma_load_2d(st, &tmX, &c.full[stage], kb * BK, tile * BM);
+                tc::tma_load_2d(st + A_BYTES, &tmW, &c.full[stage], kb * BK, 0);
                 issued[stage] = true;
                 issued_parity[stage] = phase;
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             const int zero = 0;
-            for (int s = 0; s < STAGES; ++s)
-                if (issued[s] && !tc::mbar_wait(&c.full[s], issued_parity[s], &zero))
+            for (int st = 0; st < STAGES; ++st)
+                if (issued[st] && !tc::mbar_wait(&c.full[st], issued_parity[st], &zero))
                     atomicExch(status, MOE_ERR_TIMEOUT);
         }
     } else if (warp == 1) {
@@ -184,70 +194,62 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             if (!tc::mbar_wait(&c.drain, 0, &zero)) atomicExch(status, MOE_ERR_TIMEOUT);
         }
     } else {
-        // epilogue: TMEM -> this split's partial logits
+        // epilogue: this CTA's partial logits, TMEM -> shared memory row `row`
         const int quad = warp & 3;
-        const int row = quad * 32 + lane;               // token within the tile
-        const long t = (long)tile * BM + row;
-        float* my = part + ((long)split * T_pad + t) * E;
-        bool ok = tc::mbar_wait(&c.acc_full, 0, abort_flag);
-        if (!ok) {
+        const int row = quad * 32 + lane;
+        if (!tc::mbar_wait(&c.acc_full, 0, abort_flag)) {
             *reinterpret_cast<volatile int*>(&c.abort) = 1;
             atomicExch(status, MOE_ERR_TIMEOUT);
         } else {
             tc::fence_after_sync();
             const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16);
+            float* my = red + row * es;
             for (int c0 = 0; c0 < n_pad; c0 += 32) {
                 uint32_t r[32];
                 tc::tmem_ld32(tb + c0, r);
                 tc::tmem_ld_wait();
-                if (c0 + 32 <= E) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4*>(my + c0 + j) =
-                            make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
-                                        __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c0 + j < E) my[c0 + j] = __uint_as_float(r[j]);
-                }
+                for (int j = 0; j < 32; ++j)
+                    if (c0 + j < E) my[c0 + j] = __uint_as_float(r[j]);
             }
         }
         tc::fence_before_sync();
-        // arrival among the 128 epilogue threads (named barrier 1)
-        __threadfence();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (warp == 2 && lane == 0) {
-            const int ticket = atomicAdd(&counters[tile], 1);
-            c.last = (ticket == S - 1);
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (c.last) {
-            __threadfence();
-            // Sum the S partials of this tile in split order into shared memory
-            // (the stage ring is idle now), rows padded to E+1 floats so that
-            // the per-token reads below hit distinct banks.
-            float* red = reinterpret_cast<float*>(smem);
-            const int es = E + 1;
+    }
+
+    constexpr int ROWS = BM / S;  // rows this CTA reduces and selects
+    if constexpr (S > 1) {
+        tc::cluster_sync();  // every CTA's partial rows are in its shared memory
+        if (warp >= 2) {
             const int etid = threadIdx.x - 64;
-            const long stride = (long)T_pad * E;
-            const float* tile_part = part + (long)tile * BM * E;
-            const int n4 = BM * E / 4;
+            const uint32_t red_addr = tc::smem_u32(red);
+            uint32_t base[S];
+#pragma unroll
+            for (int sp = 0; sp < S; ++sp) base[sp] = tc::map_to_cta(red_addr, sp);
+            const int n = ROWS * E;
 #pragma unroll 4
-            for (int v = etid; v < n4; v += 128) {
-                float4 a = __ldcg(reinterpret_cast<const float4*>(tile_part) + v);
-                for (int sp = 1; sp < S; ++sp) {
-                    const float4 q =
-                        __ldcg(reinterpret_cast<const float4*>(tile_part + sp * stride) + v);
-                    a.x += q.x; a.y += q.y; a.z += q.z; a.w += q.w;
-                }
-                const int r = (v * 4) / E, e = (v * 4) - r * E;
-                float* dst = red + r * es + e;
-                dst[0] = a.x; dst[1] = a.y; dst[2] = a.z; dst[3] = a.w;
+            for (int i = etid; i < n; i += 128) {
+                const int r = split * ROWS + i / E, e = i - (i / E) * E;
+                const uint32_t off = (uint32_t)(r * es + e) * 4u;
+                float v[S];
+#pragma unroll
+                for (int sp = 0; sp < S; ++sp) v[sp] = tc::ld_cluster_f32(base[sp] + off);
+                float z = v[0];
+#pragma unroll
+                for (int sp = 1; sp < S; ++sp) z += v[sp];
+                red[r * es + e] = z;  // rows of this CTA's slice: read by no other CTA
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+        }
+        tc::cluster_sync();  // all remote reads done before any CTA moves on or exits
+    } else {
+        __syncthreads();
+    }
+    if (warp >= 2) {
+        const int etid = threadIdx.x - 64;
+        if (etid < ROWS) {
+            const int r = split * ROWS + etid;
+            const long t = (long)tile * BM + r;
             if (t < T) {
-                const float* rw = red + row * es;
+                const float* rw = red + r * es;
                 int* io = idx_out + t * k;
                 float* wo = w_out + t * k;
                 switch (k) {
@@ -261,7 +263,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     default: select_topk<8>(rw, bias, E, scale, io, wo); break;
                 }
             }
-            if (warp == 2 && lane == 0) counters[tile] = 0;
         }
     }
 
@@ -302,35 +303,62 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 }  // namespace
 
-// Splits of the hidden dimension per token tile: enough CTAs for the 148 SMs
-// of a B200 (a fixed count, so the workspace size does not depend on the device).
+// Splits of the hidden dimension per token tile: a power of two <= 8 (the
+// cluster size) such that tiles * S stays near the 148 SMs of a B200.
 int router_splits(int T, int d) {
     const int tiles = (T + BM - 1) / BM;
-    int s = 148 / tiles;
-    if (s < 1) s = 1;
-    if (s > 8) s = 8;
-    const int kb = d / BK;
-    if (s > kb) s = kb;
+    int s = 1;
+    while (s < 8 && tiles * s * 2 <= 148 && s * 2 <= d / BK) s *= 2;
     return s;
 }
 
-bool router_tc_supported(const moe_config& c) { return c.k <= 8 && c.E % 4 == 0; }
+bool router_tc_supported(const moe_config& c) { return c.k <= 8; }
+
+namespace {
+
+template <int S>
+cudaError_t launch_s(dim3 grid, const CUtensorMap& mx, const CUtensorMap& mw, const moe_config& c,
+                     int n_pad, const float* gate_bias, int32_t* idx, float* w, int* status,
+                     cudaStream_t s) {
+    cudaError_t err = cudaFuncSetAttribute(router_tc_kernel<S>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = S;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, router_tc_kernel<S>, mx, mw, gate_bias, c.T, c.d, c.E, c.k,
+                              n_pad, c.scale, idx, w, status);
+}
+
+}  // namespace
 
 cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_gate,
-                             const float* gate_bias, int32_t* idx, float* w, float* part,
-                             int32_t* counters, int* status, cudaStream_t s) {
+                             const float* gate_bias, int32_t* idx, float* w, int* status,
+                             cudaStream_t s) {
     const int tiles = (c.T + BM - 1) / BM;
     const int S = router_splits(c.T, c.d);
     const int n_pad = (c.E + 15) & ~15;
     CUtensorMap mx, mw;
     if (!make_map(&mx, x, c.T, c.d, BM) || !make_map(&mw, w_gate, c.E, c.d, n_pad))
         return cudaErrorInvalidValue;
-    cudaError_t err =
-        cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    const dim3 grid(tiles, S);
+    cudaError_t err;
+    switch (S) {
+        case 1: err = launch_s<1>(grid, mx, mw, c, n_pad, gate_bias, idx, w, status, s); break;
+        case 2: err = launch_s<2>(grid, mx, mw, c, n_pad, gate_bias, idx, w, status, s); break;
+        case 4: err = launch_s<4>(grid, mx, mw, c, n_pad, gate_bias, idx, w, status, s); break;
+        default: err = launch_s<8>(grid, mx, mw, c, n_pad, gate_bias, idx, w, status, s); break;
+    }
     if (err != cudaSuccess) return err;
-    router_tc_kernel<<<dim3(tiles, S), THREADS, SMEM, s>>>(mx, mw, gate_bias, c.T, c.d, c.E, c.k,
-                                                           n_pad, c.scale, part, counters, idx, w,
-                                                           status);
     return cudaGetLastError();
 }
 
