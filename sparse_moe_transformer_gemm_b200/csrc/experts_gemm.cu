@@ -18,10 +18,13 @@
 // epilogue thread that owns feature f holds both g and u for every token and
 // applies SiLU(g)*u in fp32 before the single bf16 rounding of h.
 //
-// Kernel: persistent, one CTA per SM, 192 threads.
-//   warp 0     TMA producer: per K block of 64, the weight tile(s) (128 rows x
-//              128 B, 128-byte swizzle) and the token boxes into a ring of
-//              shared-memory stages (full/empty mbarriers);
+// Kernel: persistent, one CTA per SM, 224 threads.
+//   warp 0     weight producer: per K block of 64, the weight tile(s) (128 rows
+//              x 128 B, 128-byte swizzle) into a ring of shared-memory stages
+//              (full/empty mbarriers), evict-first in L2;
+//   warp 6     token producer: the tile's 32-row token boxes into a second,
+//              shallower ring, evict-last in L2 (they are re-read by the CTAs
+//              that share the expert);
 //   warp 1     TMEM owner (alloc/dealloc of 512 columns) and MMA issuer:
 //              tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M=128, K=16;
 //              tcgen05.commit frees a stage / publishes an accumulator;
@@ -48,21 +51,28 @@ constexpr int NBOX = 32;    // token rows per TMA box
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int BOX_BYTES = NBOX * BK * 2;
 constexpr int B_BYTES = NMAX * BK * 2;
-constexpr int THREADS = 192;
+constexpr int THREADS = 224;
 constexpr int MAX_E = 256;
 
+// Two rings: the weight tiles (streamed from HBM once) get the deeper one, the
+// token boxes (re-read from L2 by the CTAs sharing an expert) a shallower one,
+// each filled by its own producer warp.
 template <bool GATE_UP>
 struct Shape {
     static constexpr int A_TILES = GATE_UP ? 2 : 1;
-    static constexpr int STAGE_BYTES = A_TILES * A_BYTES + B_BYTES;
-    static constexpr int STAGES = GATE_UP ? 3 : 4;
+    static constexpr int A_STAGE = A_TILES * A_BYTES;  // 32 KB / 16 KB
+    static constexpr int A_STAGES = GATE_UP ? 3 : 6;
+    static constexpr int B_STAGES = 3;
+    static constexpr int RING_BYTES = A_STAGES * A_STAGE + B_STAGES * B_BYTES;
     static constexpr int ACC_STAGES = GATE_UP ? 1 : 2;
     static constexpr int ACC_COLS = GATE_UP ? 512 : 256;  // TMEM columns per accumulator stage
 };
 
 struct Ctrl {
-    uint64_t full[4];
-    uint64_t empty[4];
+    uint64_t a_full[6];
+    uint64_t a_empty[6];
+    uint64_t b_full[3];
+    uint64_t b_empty[3];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -75,7 +85,7 @@ struct Ctrl {
 
 template <bool GATE_UP>
 constexpr int smem_bytes() {
-    return Shape<GATE_UP>::STAGES * Shape<GATE_UP>::STAGE_BYTES + 1024 + (int)sizeof(Ctrl);
+    return Shape<GATE_UP>::RING_BYTES + 1024 + (int)sizeof(Ctrl);
 }
 
 struct TileInfo {
@@ -108,6 +118,17 @@ __device__ __forceinline__ void raise_timeout(Ctrl& c, int* status) {
     atomicExch(status, MOE_ERR_TIMEOUT);
 }
 
+// Wait (bounded, abort ignored) until the last load issued into each stage of a
+// ring has landed, so that no copy is in flight when the CTA exits.
+template <int N>
+__device__ __forceinline__ void drain_ring(uint64_t* full, const bool (&issued)[N],
+                                           const uint32_t (&parity)[N], int* status) {
+    const int zero = 0;
+    for (int s = 0; s < N; ++s)
+        if (issued[s] && !tc::mbar_wait(&full[s], parity[s], &zero))
+            atomicExch(status, MOE_ERR_TIMEOUT);
+}
+
 // tmA: weights as a 2-D [rows = E*A_rows_per_expert, K] bf16 map, box 64 x 128.
 // tmB: token rows as a 2-D [R, K] bf16 map, box 64 x 32.
 // A_rows_per_expert = 2F (gate_up) or d (down); m_tiles = F/128 or d/128;
@@ -122,7 +143,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + S::STAGES * S::STAGE_BYTES);
+    uint8_t* a_ring = smem;
+    uint8_t* b_ring = smem + S::A_STAGES * S::A_STAGE;
+    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + S::RING_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = K / BK;
 
@@ -154,16 +177,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             c.tile_start[E] = carry;
             c.total = carry;
             c.abort = 0;
-        }
-        if (lane == 0) {
             tc::prefetch_tensormap(&tmA);
             tc::prefetch_tensormap(&tmB);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            for (int s = 0; s < S::STAGES; ++s) {
-                tc::mbar_init(&c.full[s], 1);
-                tc::mbar_init(&c.empty[s], 1);
+            for (int s = 0; s < S::A_STAGES; ++s) {
+                tc::mbar_init(&c.a_full[s], 1);
+                tc::mbar_init(&c.a_empty[s], 1);
+            }
+            for (int s = 0; s < S::B_STAGES; ++s) {
+                tc::mbar_init(&c.b_full[s], 1);
+                tc::mbar_init(&c.b_empty[s], 1);
             }
             for (int a = 0; a < S::ACC_STAGES; ++a) {
                 tc::mbar_init(&c.acc_full[a], 1);
@@ -185,56 +210,76 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- TMA producer
-            const uint64_t pol_w = tc::policy_evict_first();
-            const uint64_t pol_x = tc::policy_evict_last();
+            // ---------------- weight-tile producer (HBM stream, evict-first in L2)
+            const uint64_t pol = tc::policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued_parity[4] = {0, 0, 0, 0};
-            bool issued[4] = {false, false, false, false};
+            uint32_t parity[S::A_STAGES] = {};
+            bool issued[S::A_STAGES] = {};
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const TileInfo ti = decode_tile(c, E, m_tiles, t);
-                const int nb = ti.n / NBOX;
-                const uint32_t bytes = S::A_TILES * A_BYTES + nb * BOX_BYTES;
                 const int a_row = ti.e * a_rows_per_expert + ti.m * BM;
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!tc::mbar_wait(&c.empty[stage], phase ^ 1u, abort_flag)) {
+                    if (!tc::mbar_wait(&c.a_empty[stage], phase ^ 1u, abort_flag)) {
                         raise_timeout(c, status);
                         ok = false;
                         break;
                     }
-                    uint8_t* s = smem + stage * S::STAGE_BYTES;
-                    tc::mbar_arrive_expect_tx(&c.full[stage], bytes);
-                    tc::tma_load_2d_hint(s, &tmA, &c.full[stage], kb * BK, a_row, pol_w);
+                    uint8_t* s = a_ring + stage * S::A_STAGE;
+                    tc::mbar_arrive_expect_tx(&c.a_full[stage], S::A_STAGE);
+                    tc::tma_load_2d_hint(s, &tmA, &c.a_full[stage], kb * BK, a_row, pol);
                     if (GATE_UP)
-                        tc::tma_load_2d_hint(s + A_BYTES, &tmA, &c.full[stage], kb * BK,
-                                             a_row + a_rows_per_expert / 2, pol_w);
-                    uint8_t* sb = s + S::A_TILES * A_BYTES;
-                    for (int b = 0; b < nb; ++b)
-                        tc::tma_load_2d_hint(sb + b * BOX_BYTES, &tmB, &c.full[stage], kb * BK,
-                                             ti.row0 + b * NBOX, pol_x);
+                        tc::tma_load_2d_hint(s + A_BYTES, &tmA, &c.a_full[stage], kb * BK,
+                                             a_row + a_rows_per_expert / 2, pol);
                     issued[stage] = true;
-                    issued_parity[stage] = phase;
-                    if (++stage == S::STAGES) {
+                    parity[stage] = phase;
+                    if (++stage == S::A_STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
-            // drain: every load this thread issued has landed before the CTA exits
-            for (int s = 0; s < S::STAGES; ++s)
-                if (issued[s]) {
-                    const int zero = 0;
-                    if (!tc::mbar_wait(&c.full[s], issued_parity[s], &zero))
-                        atomicExch(status, MOE_ERR_TIMEOUT);
+            drain_ring(c.a_full, issued, parity, status);
+        }
+    } else if (warp == 6) {
+        if (lane == 0) {
+            // ---------------- token-box producer (L2-resident rows, evict-last)
+            const uint64_t pol = tc::policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t parity[S::B_STAGES] = {};
+            bool issued[S::B_STAGES] = {};
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const int nb = ti.n / NBOX;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&c.b_empty[stage], phase ^ 1u, abort_flag)) {
+                        raise_timeout(c, status);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* s = b_ring + stage * B_BYTES;
+                    tc::mbar_arrive_expect_tx(&c.b_full[stage], nb * BOX_BYTES);
+                    for (int b = 0; b < nb; ++b)
+                        tc::tma_load_2d_hint(s + b * BOX_BYTES, &tmB, &c.b_full[stage], kb * BK,
+                                             ti.row0 + b * NBOX, pol);
+                    issued[stage] = true;
+                    parity[stage] = phase;
+                    if (++stage == S::B_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
+            }
+            drain_ring(c.b_full, issued, parity, status);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer
-            int stage = 0;
-            uint32_t phase = 0;
+            int as = 0, bs = 0;
+            uint32_t aph = 0, bph = 0;
             bool ok = true;
             int it = 0;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
@@ -249,14 +294,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
                 const uint32_t idesc = tc::idesc_bf16_f32(BM, ti.n);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!tc::mbar_wait(&c.full[stage], phase, abort_flag)) {
+                    if (!tc::mbar_wait(&c.a_full[as], aph, abort_flag) ||
+                        !tc::mbar_wait(&c.b_full[bs], bph, abort_flag)) {
                         raise_timeout(c, status);
                         ok = false;
                         break;
                     }
                     tc::fence_after_sync();
-                    const uint32_t a_addr = tc::smem_u32(smem + stage * S::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + S::A_TILES * A_BYTES;
+                    const uint32_t a_addr = tc::smem_u32(a_ring + as * S::A_STAGE);
+                    const uint32_t b_addr = tc::smem_u32(b_ring + bs * B_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / UK; ++k) {
                         const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
@@ -267,10 +313,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             tc::mma_bf16(d_tmem + 256, tc::desc_sw128(a_addr + A_BYTES + k * UK * 2),
                                          bdesc, idesc, accum);
                     }
-                    tc::mma_commit(&c.empty[stage]);
-                    if (++stage == S::STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
+                    tc::mma_commit(&c.a_empty[as]);
+                    tc::mma_commit(&c.b_empty[bs]);
+                    if (++as == S::A_STAGES) {
+                        as = 0;
+                        aph ^= 1u;
+                    }
+                    if (++bs == S::B_STAGES) {
+                        bs = 0;
+                        bph ^= 1u;
                     }
                 }
                 if (ok) tc::mma_commit(&c.acc_full[acc]);

@@ -1,0 +1,432 @@
+// experts_gemm2.cu -- the SwiGLU experts' grouped GEMMs on pairs of SMs
+// (tcgen05 cta_group::2), for shapes whose weight rows split into 256-row tiles.
+//
+// Same mathematics as experts_gemm.cu ("DeepSeek V4-Flash 架构 QA" Q4.5 SwiGLU;
+// "Tencent Hy3-295B 架构深度拆解" §2.3 fused gate_up_proj [2F, d] and down_proj
+// [d, F]; "Tencent Hy3-Flash QA" Q6.4 grouped matmul):
+//   gate_up: h[r, f] = bf16( SiLU(<x_r, W[e, f]>) * <x_r, W[e, F + f]> )
+//   down:    y[r, i] = bf16( <h_r, Wd[e, i]> )
+//
+// A cluster of two CTAs (two SMs) computes one 256-weight-row x N-token tile
+// with M=256 MMAs: each CTA stages its own 128 weight rows and half of the N
+// token rows, and the even CTA's single MMA thread drives the tensor cores of
+// both. Compared with one CTA per 128 rows this halves the token rows each SM
+// pulls from L2 per K step and frees shared memory for a deeper weight ring
+// (more weight bytes in flight per SM, the bound of this HBM-bound stream).
+//
+// Per CTA (224 threads): warp 0 TMA producer (its weight rows + its token
+// half; completion counted on the even CTA's "full" barrier, which expects the
+// bytes of both CTAs), warp 1 TMEM owner (+ MMA issuer in the even CTA), warps
+// 2-5 epilogue of the CTA's own 128 rows, warp 6 idle. Stage release and
+// accumulator hand-off are tcgen05.commit arrivals multicast to both CTAs; the
+// epilogues hand the accumulator back with one arrival per CTA on the even
+// CTA's barrier. No TMA load uses multicast. All waits are bounded.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;       // weight rows per CTA (MMA M = 256 per pair)
+constexpr int BK = 64;
+constexpr int UK = 16;
+constexpr int NMAX = 256;     // token rows per pair tile
+constexpr int NBOX = 16;      // token rows per TMA box
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int BOX_BYTES = NBOX * BK * 2;
+constexpr int BH_BYTES = (NMAX / 2) * BK * 2;  // this CTA's half of the token rows
+constexpr int THREADS = 224;
+constexpr int MAX_E = 256;
+
+template <bool GATE_UP>
+struct Shape {
+    static constexpr int A_TILES = GATE_UP ? 2 : 1;
+    static constexpr int STAGE_BYTES = A_TILES * A_BYTES + BH_BYTES;  // 48 KB / 32 KB
+    static constexpr int STAGES = GATE_UP ? 4 : 6;
+    static constexpr int ACC_STAGES = GATE_UP ? 1 : 2;
+    static constexpr int ACC_COLS = GATE_UP ? 512 : 256;
+};
+
+struct Ctrl {
+    uint64_t full[6];       // even CTA: TMA bytes of both CTAs landed
+    uint64_t empty[6];      // both CTAs: the pair MMAs finished reading the stage
+    uint64_t acc_full[2];   // both CTAs: accumulator ready
+    uint64_t acc_empty[2];  // even CTA: both epilogues done with the accumulator
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int total;
+    int off[MAX_E + 1];
+    int tile_start[MAX_E + 1];
+};
+
+template <bool GATE_UP>
+constexpr int smem_bytes() {
+    return Shape<GATE_UP>::STAGES * Shape<GATE_UP>::STAGE_BYTES + 1024 + (int)sizeof(Ctrl);
+}
+
+struct TileInfo {
+    int e, m, row0, len, n;  // n: MMA N of the pair, a multiple of 2*NBOX
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const Ctrl& c, int E, int m_tiles, int t) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (c.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int local = t - c.tile_start[e];
+    const int n_e = c.off[e + 1] - c.off[e];
+    const int nt = (n_e + NMAX - 1) / NMAX;
+    const int j = local / m_tiles;
+    const int base = n_e / nt, rem = n_e - base * nt;
+    TileInfo ti;
+    ti.e = e;
+    ti.m = local - j * m_tiles;
+    ti.row0 = c.off[e] + j * base + min(j, rem);
+    ti.len = base + (j < rem ? 1 : 0);
+    ti.n = (ti.len + 2 * NBOX - 1) & ~(2 * NBOX - 1);
+    return ti;
+}
+
+__device__ __forceinline__ void raise_timeout(Ctrl& c, int* status) {
+    *reinterpret_cast<volatile int*>(&c.abort) = 1;
+    atomicExch(status, MOE_ERR_TIMEOUT);
+}
+
+// tmA: weights [E * a_rows_per_expert, K] bf16, box 64 x 128.
+// tmB: token rows [R, K] bf16, box 64 x 16.
+// m_tiles: 256-row weight tiles per expert (F/256 for gate_up, d/256 for down).
+template <bool GATE_UP>
+__global__ void __launch_bounds__(THREADS, 1)
+grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB, const int* __restrict__ offsets,
+                         int E, int K, int a_rows_per_expert, int m_tiles,
+                         __nv_bfloat16* __restrict__ out, int out_ld, int* __restrict__ status) {
+    using S = Shape<GATE_UP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + S::STAGES * S::STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)(tc::cluster_ctarank() & 1u);
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int KB = K / BK;
+
+    // ---- prologue: tile table (warp 0), barriers and TMEM (warp 1), in both CTAs
+    if (warp == 0) {
+        int carry = 0;
+        for (int b = 0; b <= E; b += 32) {
+            const int e = b + lane;
+            int o = 0, cnt = 0;
+            if (e <= E) {
+                o = offsets[e];
+                c.off[e] = o;
+            }
+            __syncwarp();
+            if (e < E) {
+                const int n_e = offsets[e + 1] - o;
+                cnt = ((n_e + NMAX - 1) / NMAX) * m_tiles;
+            }
+            int incl = cnt;
+#pragma unroll
+            for (int s = 1; s < 32; s <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, s);
+                if (lane >= s) incl += v;
+            }
+            if (e < E) c.tile_start[e] = carry + incl - cnt;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            c.tile_start[E] = carry;
+            c.total = carry;
+            c.abort = 0;
+            tc::prefetch_tensormap(&tmA);
+            tc::prefetch_tensormap(&tmB);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < S::STAGES; ++s) {
+                tc::mbar_init(&c.full[s], 1);
+                tc::mbar_init(&c.empty[s], 1);
+            }
+            for (int a = 0; a < S::ACC_STAGES; ++a) {
+                tc::mbar_init(&c.acc_full[a], 1);
+                tc::mbar_init(&c.acc_empty[a], 2);
+            }
+            tc::mbar_init(&c.drain, 1);
+            tc::fence_mbar_init();
+        }
+        __syncwarp();
+        tc::tmem_alloc_pair(&c.tmem_base, 512);
+        tc::tmem_relinquish_pair();
+    }
+    tc::fence_before_sync();
+    tc::cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+    tc::fence_after_sync();
+    const uint32_t tmem_base = c.tmem_base;
+    const int total = c.total;
+    const volatile int* abort_flag = &c.abort;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- producer: this CTA's weight rows and token half
+            const uint64_t pol_w = tc::policy_evict_first();
+            const uint64_t pol_x = tc::policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t parity[S::STAGES] = {};
+            bool issued[S::STAGES] = {};
+            bool ok = true;
+            for (int t = pair; t < total && ok; t += n_pairs) {
+                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const int nb = ti.n / (2 * NBOX);  // boxes per CTA
+                const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
+                const int b_row = ti.row0 + rank * (ti.n / 2);
+                const uint32_t pair_bytes = 2u * (S::A_TILES * A_BYTES + nb * BOX_BYTES);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&c.empty[stage], phase ^ 1u, abort_flag)) {
+                        raise_timeout(c, status);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.full[stage]), 0);
+                    if (leader) tc::mbar_arrive_expect_tx(&c.full[stage], pair_bytes);
+                    uint8_t* s = smem + stage * S::STAGE_BYTES;
+                    tc::tma_load_2d_pair(s, &tmA, full_leader, kb * BK, a_row, pol_w);
+                    if (GATE_UP)
+                        tc::tma_load_2d_pair(s + A_BYTES, &tmA, full_leader, kb * BK,
+                                             a_row + a_rows_per_expert / 2, pol_w);
+                    uint8_t* sb = s + S::A_TILES * A_BYTES;
+                    for (int b = 0; b < nb; ++b)
+                        tc::tma_load_2d_pair(sb + b * BOX_BYTES, &tmB, full_leader, kb * BK,
+                                             b_row + b * NBOX, pol_x);
+                    issued[stage] = true;
+                    parity[stage] = phase;
+                    if (++stage == S::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // drain: this CTA's copies have landed (the even CTA's full barrier saw
+            // every byte of both CTAs when its last phase completed)
+            if (leader) {
+                const int zero = 0;
+                for (int s = 0; s < S::STAGES; ++s)
+                    if (issued[s] && !tc::mbar_wait(&c.full[s], parity[s], &zero))
+                        atomicExch(status, MOE_ERR_TIMEOUT);
+            } else {
+                // the odd CTA's stages are released only after the pair MMAs read
+                // them, which is after they landed: wait for the last release
+                const int zero = 0;
+                for (int s = 0; s < S::STAGES; ++s)
+                    if (issued[s] && !tc::mbar_wait(&c.empty[s], parity[s], &zero))
+                        atomicExch(status, MOE_ERR_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------- MMA issuer (even CTA), M = 256 across the pair
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int it = 0;
+            for (int t = pair; t < total && ok; t += n_pairs, ++it) {
+                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const int acc = it % S::ACC_STAGES;
+                const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
+                if (!tc::mbar_wait(&c.acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
+                    raise_timeout(c, status);
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
+                const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, ti.n);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&c.full[stage], phase, abort_flag)) {
+                        raise_timeout(c, status);
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint32_t a_addr = tc::smem_u32(smem + stage * S::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + S::A_TILES * A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UK; ++k) {
+                        const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
+                        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                        tc::mma_bf16_pair(d_tmem, tc::desc_sw128(a_addr + k * UK * 2), bdesc,
+                                          idesc, accum);
+                        if (GATE_UP)
+                            tc::mma_bf16_pair(d_tmem + 256,
+                                              tc::desc_sw128(a_addr + A_BYTES + k * UK * 2), bdesc,
+                                              idesc, accum);
+                    }
+                    tc::mma_commit_pair(&c.empty[stage], 0x3);
+                    if (++stage == S::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) tc::mma_commit_pair(&c.acc_full[acc], 0x3);
+            }
+            tc::mma_commit_pair(&c.drain, 0x1);
+            const int zero = 0;
+            if (!tc::mbar_wait(&c.drain, 0, &zero)) atomicExch(status, MOE_ERR_TIMEOUT);
+        }
+    } else if (warp >= 2 && warp <= 5) {
+        // ---------------- epilogue: this CTA's 128 weight rows (TMEM lanes)
+        const int quad = warp & 3;
+        const int row_in_tile = quad * 32 + lane;
+        uint16_t* o16 = reinterpret_cast<uint16_t*>(out);
+        const bool arriver = (warp == 2 && lane == 0);
+        int it = 0;
+        for (int t = pair; t < total; t += n_pairs, ++it) {
+            const TileInfo ti = decode_tile(c, E, m_tiles, t);
+            const int acc = it % S::ACC_STAGES;
+            const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
+            if (!tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag)) {
+                raise_timeout(c, status);
+                break;
+            }
+            tc::fence_after_sync();
+            const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
+            const int col = ti.m * 2 * BM + rank * BM + row_in_tile;
+            for (int c0 = 0; c0 < ti.n; c0 += 32) {
+                uint32_t g[32];
+                tc::tmem_ld32(tbase + c0, g);
+                if constexpr (GATE_UP) {
+                    uint32_t u[32];
+                    tc::tmem_ld32(tbase + 256 + c0, u);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c0 + j;
+                        if (n < ti.len) {
+                            const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
+                            const float hv = gv / (1.f + expf(-gv)) * uv;
+                            o16[(size_t)(ti.row0 + n) * out_ld + col] = float_to_bf16_bits(hv);
+                        }
+                    }
+                } else {
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c0 + j;
+                        if (n < ti.len)
+                            o16[(size_t)(ti.row0 + n) * out_ld + col] =
+                                float_to_bf16_bits(__uint_as_float(g[j]));
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+            if (arriver)
+                tc::mbar_arrive_cluster(tc::map_to_cta(tc::smem_u32(&c.acc_empty[acc]), 0));
+        }
+    }
+
+    // Neither CTA leaves while the other may still signal its barriers or read
+    // its shared memory.
+    tc::fence_before_sync();
+    tc::cluster_sync();
+    if (warp == 1) {
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc_pair(tmem_base, 512);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_pairs() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return (n > 1 ? n : 148) / 2;
+}
+
+template <bool GATE_UP>
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const int32_t* offsets, int E,
+                   int K, int a_rows_per_expert, int m_tiles, void* out, int out_ld, int* status,
+                   cudaStream_t s) {
+    const int smem = smem_bytes<GATE_UP>();
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATE_UP>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * sm_pairs(), 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATE_UP>, a, b, offsets, E, K,
+                             a_rows_per_expert, m_tiles, static_cast<__nv_bfloat16*>(out), out_ld,
+                             status);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool pair_gemm_supported(const moe_config& c) { return c.d % 256 == 0 && c.d_ff % 256 == 0; }
+
+cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
+                                     const int32_t* offsets, const void* w_gate_up, void* h,
+                                     int* status, cudaStream_t s) {
+    CUtensorMap a, b;
+    const uint64_t R = (uint64_t)c.T * c.k;
+    if (!make_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM) ||
+        !make_map(&b, x_perm, R, c.d, NBOX))
+        return cudaErrorInvalidValue;
+    return launch<true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h, c.d_ff, status,
+                        s);
+}
+
+cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int32_t* offsets,
+                                  const void* w_down, void* y, int* status, cudaStream_t s) {
+    CUtensorMap a, b;
+    const uint64_t R = (uint64_t)c.T * c.k;
+    if (!make_map(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM) ||
+        !make_map(&b, h, R, c.d_ff, NBOX))
+        return cudaErrorInvalidValue;
+    return launch<false>(a, b, offsets, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d, status, s);
+}
+
+}  // namespace moe

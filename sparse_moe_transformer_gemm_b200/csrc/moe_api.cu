@@ -84,8 +84,10 @@ int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offs
     if (use_stream_path(c))
         return cuda_status(launch_gate_up_stream(*c, x_perm, offsets, w_gate_up, s_gate_up, h, s));
     if (c->flags & MOE_FLAG_FP8_WEIGHTS) return MOE_ERR_UNSUPPORTED_SHAPE;
-    return cuda_status(launch_gate_up_gemm(*c, x_perm, offsets, w_gate_up, h,
-                                           at<int>(ws, ws_layout(*c).status), s));
+    int* status = at<int>(ws, ws_layout(*c).status);
+    if (pair_gemm_supported(*c))
+        return cuda_status(launch_gate_up_gemm_pair(*c, x_perm, offsets, w_gate_up, h, status, s));
+    return cuda_status(launch_gate_up_gemm(*c, x_perm, offsets, w_gate_up, h, status, s));
 }
 
 int experts_down(const moe_config* c, const void* h, const int32_t* offsets, const void* w_down,
@@ -93,8 +95,10 @@ int experts_down(const moe_config* c, const void* h, const int32_t* offsets, con
     if (use_stream_path(c))
         return cuda_status(launch_down_stream(*c, h, offsets, w_down, s_down, y, s));
     if (c->flags & MOE_FLAG_FP8_WEIGHTS) return MOE_ERR_UNSUPPORTED_SHAPE;
-    return cuda_status(launch_down_gemm(*c, h, offsets, w_down, y,
-                                        at<int>(ws, ws_layout(*c).status), s));
+    int* status = at<int>(ws, ws_layout(*c).status);
+    if (pair_gemm_supported(*c))
+        return cuda_status(launch_down_gemm_pair(*c, h, offsets, w_down, y, status, s));
+    return cuda_status(launch_down_gemm(*c, h, offsets, w_down, y, status, s));
 }
 
 }  // namespace

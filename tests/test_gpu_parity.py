@@ -29,6 +29,9 @@ SMALL = {
     "top1": LayerShape(T=50, d=256, E=16, k=1, F=128),
     "tiny_fp8": dataclasses.replace(CONFIGS["tiny"], fp8=True),
     "ragged_skewed": LayerShape(T=300, d=512, E=32, k=8, F=384, zipf_bias=True),
+    # d and d_ff multiples of 256: the pair-of-SMs GEMMs (several tiles, ragged tokens)
+    "pair_small": LayerShape(T=200, d=512, E=16, k=4, F=512),
+    "pair_ragged": LayerShape(T=333, d=768, E=24, k=6, F=256, zipf_bias=True),
     # the CUDA-core router (k > 8, or E not a multiple of 4)
     "k12": LayerShape(T=100, d=256, E=32, k=12, F=128),
     "e18": LayerShape(T=90, d=256, E=18, k=4, F=128),
@@ -89,11 +92,12 @@ def test_hy3_shapes(name):
     _free(layer, out)
 
 
-@pytest.mark.parametrize("T", [64, 700])
-def test_all_tokens_to_the_same_experts(T):
+@pytest.mark.parametrize("T,F", [(64, 128), (700, 128), (700, 256)])
+def test_all_tokens_to_the_same_experts(T, F):
     """A logit bias of +40 on experts 0..3 sends every token to them (T rows each,
-    split into several token tiles when T > 256); the other twelve are empty."""
-    shape = dataclasses.replace(CONFIGS["tiny"], T=T)
+    split into several token tiles when T > 256); the other twelve are empty.
+    F = 256 runs the pair-of-SMs GEMMs, F = 128 the single-SM ones."""
+    shape = dataclasses.replace(CONFIGS["tiny"], T=T, F=F)
     layer = make_layer(shape, seed=2, device="cuda")
     b = torch.zeros(shape.E, dtype=torch.float32, device="cuda")
     b[:4] = 40.0
