@@ -316,7 +316,7 @@ def main():
     dominant = max(("gate_up", "down"), key=lambda s: stage_ms[s])
     dom_work = gw if dominant == "gate_up" else dw
     dom_s = stage_ms[dominant] / 1e3
-    use_stream = args.path == "stream" or (args.path == "auto" and fp8)
+    use_stream = args.path == "stream"
     kernel_name = f"{dominant}_{'stream' if use_stream else 'gemm'}"
     # The metric's roofline: HBM for the decode workload (weights streamed once),
     # dense bf16 tensor peak for the larger batches. The tensor peak is the

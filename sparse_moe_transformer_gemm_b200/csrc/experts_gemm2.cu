@@ -72,7 +72,8 @@ struct TileInfo {
     int e, m, row0, len, n;  // n: MMA N of the pair, a multiple of 2*NBOX
 };
 
-__device__ __forceinline__ TileInfo decode_tile(const Ctrl& c, int E, int m_tiles, int t) {
+template <typename CtrlT>
+__device__ __forceinline__ TileInfo decode_tile(const CtrlT& c, int E, int m_tiles, int t) {
     int lo = 0, hi = E - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -93,7 +94,8 @@ __device__ __forceinline__ TileInfo decode_tile(const Ctrl& c, int E, int m_tile
     return ti;
 }
 
-__device__ __forceinline__ void raise_timeout(Ctrl& c, int* status) {
+template <typename CtrlT>
+__device__ __forceinline__ void raise_timeout(CtrlT& c, int* status) {
     *reinterpret_cast<volatile int*>(&c.abort) = 1;
     atomicExch(status, MOE_ERR_TIMEOUT);
 }
@@ -291,14 +293,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             const TileInfo ti = decode_tile(c, E, m_tiles, t);
             const int acc = it % S::ACC_STAGES;
             const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
-            if (!tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag)) {
-                raise_timeout(c, status);
-                break;
-            }
+            const bool ok = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
             tc::fence_after_sync();
             const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
             const int col = ti.m * 2 * BM + rank * BM + row_in_tile;
-            for (int c0 = 0; c0 < ti.n; c0 += 32) {
+            for (int c0 = 0; ok && c0 < ti.n; c0 += 32) {
                 uint32_t g[32];
                 tc::tmem_ld32(tbase + c0, g);
                 if constexpr (GATE_UP) {
@@ -326,7 +325,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
             }
             tc::fence_before_sync();
-            asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+            if (tc::bar_any(1, 128, !ok)) {  // the four epilogue warps leave together
+                raise_timeout(c, status);
+                break;
+            }
             if (arriver)
                 tc::mbar_arrive_cluster(tc::map_to_cta(tc::smem_u32(&c.acc_empty[acc]), 0));
         }
@@ -334,6 +336,374 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 
     // Neither CTA leaves while the other may still signal its barriers or read
     // its shared memory.
+    tc::fence_before_sync();
+    tc::cluster_sync();
+    if (warp == 1) {
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc_pair(tmem_base, 512);
+    }
+}
+
+// ======================================================================
+// FP8 (e4m3) weights. The MMA stays kind::f16 (bf16 x bf16, fp32 accumulate)
+// on weights widened on chip: a producer warp TMA-loads raw e4m3 weight tiles
+// (128 rows x 64 bytes per K block, unswizzled) into a "raw" ring; four
+// converter warps widen them exactly to bf16 straight into the 128-byte-
+// swizzled operand layout of the MMA, issue the stage's token-half TMA, and
+// arrive on the even CTA's operand barrier. The per-output-row fp32 scale
+// multiplies the finished dot product in the epilogue (before SiLU for
+// gate_up, before the bf16 store for down): sum_c x_c q_c s_row = s_row
+// sum_c x_c q_c. Every e4m3 value is representable in bf16, so the widening
+// loses nothing.
+
+constexpr int THREADS_FP8 = 320;        // + warps 6-9: converters
+constexpr int RAW_BYTES = BM * BK;      // one 128 x 64 e4m3 tile
+
+template <bool GATE_UP>
+struct Fp8Shape {
+    static constexpr int A_TILES = GATE_UP ? 2 : 1;
+    static constexpr int RAW_STAGE = A_TILES * RAW_BYTES;                  // 16 KB / 8 KB
+    static constexpr int OP_STAGE = A_TILES * A_BYTES + BH_BYTES;          // 48 KB / 32 KB
+    static constexpr int RAW_STAGES = GATE_UP ? 4 : 6;
+    static constexpr int OP_STAGES = GATE_UP ? 3 : 5;
+    static constexpr int RING_BYTES = OP_STAGES * OP_STAGE + RAW_STAGES * RAW_STAGE;  // 208 KB
+    static constexpr int ACC_STAGES = GATE_UP ? 1 : 2;
+    static constexpr int ACC_COLS = GATE_UP ? 512 : 256;
+};
+
+struct Fp8Ctrl {
+    uint64_t raw_full[6];   // each CTA: its raw weight tile landed
+    uint64_t raw_empty[6];  // each CTA: its converters are done with the raw stage
+    uint64_t op_full[5];    // even CTA: both CTAs converted + token bytes of both landed
+    uint64_t op_empty[5];   // both CTAs: the pair MMAs finished reading the operand stage
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int total;
+    int off[MAX_E + 1];
+    int tile_start[MAX_E + 1];
+};
+
+template <bool GATE_UP>
+constexpr int fp8_smem_bytes() {
+    return Fp8Shape<GATE_UP>::RING_BYTES + 1024 + (int)sizeof(Fp8Ctrl);
+}
+static_assert(fp8_smem_bytes<true>() <= 232448 && fp8_smem_bytes<false>() <= 232448,
+              "fits in 227 KB");
+
+// Two e4m3 codes -> bf16x2, exactly: the hardware e4m3x2 -> f16x2 conversion,
+// then f16 -> bf16 by rebiasing the exponent (15 -> 127: +112 << 7 after the
+// 3-bit mantissa shift). e4m3-valued f16 numbers are normal or zero and carry
+// no mantissa bits below bit 7, so the shift drops nothing; zeros keep their sign.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t q) {
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)q, __NV_E4M3);
+    const uint32_t h = (uint32_t)hr.x | ((uint32_t)hr.y << 16);
+    const uint32_t mag = h & 0x7FFF7FFFu;
+    const uint32_t nz = __vcmpne2(mag, 0u);
+    return (((mag >> 3) + 0x38003800u) & nz) | (h & 0x80008000u);
+}
+
+// Convert one raw e4m3 tile (128 rows x 64 bytes, row-major) into a bf16
+// operand tile (128 rows x 128 bytes, 128-byte swizzle). 128 threads; thread
+// `ct` handles 16-byte source chunks q = ct + 128 i (row q/4, elements 16(q%4)..).
+__device__ __forceinline__ void widen_tile(const uint8_t* raw, uint8_t* op, int ct) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int q = ct + 128 * i;
+        const int row = q >> 2, c = q & 3;
+        const uint4 v = *reinterpret_cast<const uint4*>(raw + q * 16);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t b[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            b[2 * j] = e4m3x2_to_bf16x2((uint16_t)(w[j] & 0xFFFFu));
+            b[2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(w[j] >> 16));
+        }
+        uint8_t* rbase = op + row * 128;
+        const int sw = row & 7;
+        *reinterpret_cast<uint4*>(rbase + (((2 * c) ^ sw) << 4)) = make_uint4(b[0], b[1], b[2], b[3]);
+        *reinterpret_cast<uint4*>(rbase + (((2 * c + 1) ^ sw) << 4)) =
+            make_uint4(b[4], b[5], b[6], b[7]);
+    }
+}
+
+// tmA: e4m3 weights [E * a_rows_per_expert, K] bytes, box 64 x 128 (no swizzle).
+// tmB: token rows [R, K] bf16, box 64 x 16. scales: [E * a_rows_per_expert] fp32.
+template <bool GATE_UP>
+__global__ void __launch_bounds__(THREADS_FP8, 1)
+grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB,
+                             const int* __restrict__ offsets, const float* __restrict__ scales,
+                             int E, int K, int a_rows_per_expert, int m_tiles,
+                             __nv_bfloat16* __restrict__ out, int out_ld,
+                             int* __restrict__ status) {
+    using S = Fp8Shape<GATE_UP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* op_ring = smem;
+    uint8_t* raw_ring = smem + S::OP_STAGES * S::OP_STAGE;
+    Fp8Ctrl& c = *reinterpret_cast<Fp8Ctrl*>(smem + S::RING_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)(tc::cluster_ctarank() & 1u);
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int KB = K / BK;
+
+    if (warp == 0) {
+        int carry = 0;
+        for (int b = 0; b <= E; b += 32) {
+            const int e = b + lane;
+            int o = 0, cnt = 0;
+            if (e <= E) {
+                o = offsets[e];
+                c.off[e] = o;
+            }
+            __syncwarp();
+            if (e < E) {
+                const int n_e = offsets[e + 1] - o;
+                cnt = ((n_e + NMAX - 1) / NMAX) * m_tiles;
+            }
+            int incl = cnt;
+#pragma unroll
+            for (int s = 1; s < 32; s <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, s);
+                if (lane >= s) incl += v;
+            }
+            if (e < E) c.tile_start[e] = carry + incl - cnt;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            c.tile_start[E] = carry;
+            c.total = carry;
+            c.abort = 0;
+            tc::prefetch_tensormap(&tmA);
+            tc::prefetch_tensormap(&tmB);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int s = 0; s < S::RAW_STAGES; ++s) {
+                tc::mbar_init(&c.raw_full[s], 1);
+                tc::mbar_init(&c.raw_empty[s], 1);
+            }
+            for (int s = 0; s < S::OP_STAGES; ++s) {
+                tc::mbar_init(&c.op_full[s], 2);  // one converter arrival per CTA (+ token bytes)
+                tc::mbar_init(&c.op_empty[s], 1);
+            }
+            for (int a = 0; a < S::ACC_STAGES; ++a) {
+                tc::mbar_init(&c.acc_full[a], 1);
+                tc::mbar_init(&c.acc_empty[a], 2);
+            }
+            tc::mbar_init(&c.drain, 1);
+            tc::fence_mbar_init();
+        }
+        __syncwarp();
+        tc::tmem_alloc_pair(&c.tmem_base, 512);
+        tc::tmem_relinquish_pair();
+    }
+    tc::fence_before_sync();
+    tc::cluster_sync();
+    tc::fence_after_sync();
+    const uint32_t tmem_base = c.tmem_base;
+    const int total = c.total;
+    const volatile int* abort_flag = &c.abort;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- raw e4m3 weight producer (this CTA's rows, own barrier)
+            const uint64_t pol = tc::policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t parity[S::RAW_STAGES] = {};
+            bool issued[S::RAW_STAGES] = {};
+            bool ok = true;
+            for (int t = pair; t < total && ok; t += n_pairs) {
+                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&c.raw_empty[stage], phase ^ 1u, abort_flag)) {
+                        raise_timeout(c, status);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = raw_ring + stage * S::RAW_STAGE;
+                    tc::mbar_arrive_expect_tx(&c.raw_full[stage], S::RAW_STAGE);
+                    tc::tma_load_2d_hint(st, &tmA, &c.raw_full[stage], kb * BK, a_row, pol);
+                    if (GATE_UP)
+                        tc::tma_load_2d_hint(st + RAW_BYTES, &tmA, &c.raw_full[stage], kb * BK,
+                                             a_row + a_rows_per_expert / 2, pol);
+                    issued[stage] = true;
+                    parity[stage] = phase;
+                    if (++stage == S::RAW_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            const int zero = 0;
+            for (int s = 0; s < S::RAW_STAGES; ++s)
+                if (issued[s] && !tc::mbar_wait(&c.raw_full[s], parity[s], &zero))
+                    atomicExch(status, MOE_ERR_TIMEOUT);
+        }
+    } else if (warp >= 6) {
+        // ---------------- converters: raw e4m3 -> bf16 operand; token-half TMA
+        const int ct = threadIdx.x - 192;  // 0..127
+        const uint64_t pol_x = tc::policy_evict_last();
+        int rs = 0, os = 0;
+        uint32_t rph = 0, oph = 0;
+        for (int t = pair; t < total; t += n_pairs) {
+            const TileInfo ti = decode_tile(c, E, m_tiles, t);
+            const int nb = ti.n / (2 * NBOX);
+            const int b_row = ti.row0 + rank * (ti.n / 2);
+            const uint32_t b_pair_bytes = 2u * (uint32_t)(nb * BOX_BYTES);
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb) {
+                const bool got = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag) &&
+                                 tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
+                uint8_t* op = op_ring + os * S::OP_STAGE;
+                const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0);
+                if (got) {
+                    if (ct == 0)
+                        for (int b = 0; b < nb; ++b)
+                            tc::tma_load_2d_pair(op + S::A_TILES * A_BYTES + b * BOX_BYTES, &tmB,
+                                                 full_leader, kb * BK, b_row + b * NBOX, pol_x);
+                    const uint8_t* raw = raw_ring + rs * S::RAW_STAGE;
+                    widen_tile(raw, op, ct);
+                    if (GATE_UP) widen_tile(raw + RAW_BYTES, op + A_BYTES, ct);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
+                if (tc::bar_any(2, 128, !got)) {  // the four converter warps leave together
+                    raise_timeout(c, status);
+                    ok = false;
+                    break;
+                }
+                if (ct == 0) {
+                    tc::mbar_arrive(&c.raw_empty[rs]);
+                    if (leader)
+                        tc::mbar_arrive_expect_tx(&c.op_full[os], b_pair_bytes);
+                    else
+                        tc::mbar_arrive_cluster(full_leader);
+                }
+                if (++rs == S::RAW_STAGES) {
+                    rs = 0;
+                    rph ^= 1u;
+                }
+                if (++os == S::OP_STAGES) {
+                    os = 0;
+                    oph ^= 1u;
+                }
+            }
+            if (!ok) break;
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------- MMA issuer (even CTA)
+            int os = 0;
+            uint32_t oph = 0;
+            bool ok = true;
+            int it = 0;
+            for (int t = pair; t < total && ok; t += n_pairs, ++it) {
+                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const int acc = it % S::ACC_STAGES;
+                const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
+                if (!tc::mbar_wait(&c.acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
+                    raise_timeout(c, status);
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
+                const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, ti.n);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&c.op_full[os], oph, abort_flag)) {
+                        raise_timeout(c, status);
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint32_t a_addr = tc::smem_u32(op_ring + os * S::OP_STAGE);
+                    const uint32_t b_addr = a_addr + S::A_TILES * A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / UK; ++k) {
+                        const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
+                        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                        tc::mma_bf16_pair(d_tmem, tc::desc_sw128(a_addr + k * UK * 2), bdesc,
+                                          idesc, accum);
+                        if (GATE_UP)
+                            tc::mma_bf16_pair(d_tmem + 256,
+                                              tc::desc_sw128(a_addr + A_BYTES + k * UK * 2), bdesc,
+                                              idesc, accum);
+                    }
+                    tc::mma_commit_pair(&c.op_empty[os], 0x3);
+                    if (++os == S::OP_STAGES) {
+                        os = 0;
+                        oph ^= 1u;
+                    }
+                }
+                if (ok) tc::mma_commit_pair(&c.acc_full[acc], 0x3);
+            }
+            tc::mma_commit_pair(&c.drain, 0x1);
+            const int zero = 0;
+            if (!tc::mbar_wait(&c.drain, 0, &zero)) atomicExch(status, MOE_ERR_TIMEOUT);
+        }
+    } else if (warp >= 2 && warp <= 5) {
+        // ---------------- epilogue (scales applied to the finished dot products)
+        const int quad = warp & 3;
+        const int row_in_tile = quad * 32 + lane;
+        uint16_t* o16 = reinterpret_cast<uint16_t*>(out);
+        const bool arriver = (warp == 2 && lane == 0);
+        int it = 0;
+        for (int t = pair; t < total; t += n_pairs, ++it) {
+            const TileInfo ti = decode_tile(c, E, m_tiles, t);
+            const int acc = it % S::ACC_STAGES;
+            const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
+            const bool ok = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
+            tc::fence_after_sync();
+            const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
+            const int col = ti.m * 2 * BM + rank * BM + row_in_tile;
+            const long srow = (long)ti.e * a_rows_per_expert + col;
+            const float sa = __ldg(scales + srow);
+            const float sb = GATE_UP ? __ldg(scales + srow + a_rows_per_expert / 2) : 0.f;
+            for (int c0 = 0; ok && c0 < ti.n; c0 += 32) {
+                uint32_t g[32];
+                tc::tmem_ld32(tbase + c0, g);
+                if constexpr (GATE_UP) {
+                    uint32_t u[32];
+                    tc::tmem_ld32(tbase + 256 + c0, u);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c0 + j;
+                        if (n < ti.len) {
+                            const float gv = __uint_as_float(g[j]) * sa;
+                            const float uv = __uint_as_float(u[j]) * sb;
+                            const float hv = gv / (1.f + expf(-gv)) * uv;
+                            o16[(size_t)(ti.row0 + n) * out_ld + col] = float_to_bf16_bits(hv);
+                        }
+                    }
+                } else {
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = c0 + j;
+                        if (n < ti.len)
+                            o16[(size_t)(ti.row0 + n) * out_ld + col] =
+                                float_to_bf16_bits(__uint_as_float(g[j]) * sa);
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            if (tc::bar_any(1, 128, !ok)) {
+                raise_timeout(c, status);
+                break;
+            }
+            if (arriver)
+                tc::mbar_arrive_cluster(tc::map_to_cta(tc::smem_u32(&c.acc_empty[acc]), 0));
+        }
+    }
+
     tc::fence_before_sync();
     tc::cluster_sync();
     if (warp == 1) {
@@ -365,6 +735,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major [rows, cols] e4m3 codes (bytes), box of box_rows x 64 bytes, no swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -403,9 +788,61 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const int32_t* of
     return cudaGetLastError();
 }
 
+template <bool GATE_UP>
+cudaError_t launch_fp8(const CUtensorMap& a, const CUtensorMap& b, const int32_t* offsets,
+                       const float* scales, int E, int K, int a_rows_per_expert, int m_tiles,
+                       void* out, int out_ld, int* status, cudaStream_t s) {
+    const int smem = fp8_smem_bytes<GATE_UP>();
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_fp8_kernel<GATE_UP>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * sm_pairs(), 1, 1);
+    cfg.blockDim = dim3(THREADS_FP8, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_fp8_kernel<GATE_UP>, a, b, offsets, scales, E,
+                             K, a_rows_per_expert, m_tiles, static_cast<__nv_bfloat16*>(out),
+                             out_ld, status);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool pair_gemm_supported(const moe_config& c) { return c.d % 256 == 0 && c.d_ff % 256 == 0; }
+
+cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm,
+                                         const int32_t* offsets, const void* w_gate_up,
+                                         const float* s_gate_up, void* h, int* status,
+                                         cudaStream_t s) {
+    CUtensorMap a, b;
+    const uint64_t R = (uint64_t)c.T * c.k;
+    if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM) ||
+        !make_map(&b, x_perm, R, c.d, NBOX))
+        return cudaErrorInvalidValue;
+    return launch_fp8<true>(a, b, offsets, s_gate_up, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h,
+                            c.d_ff, status, s);
+}
+
+cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const int32_t* offsets,
+                                      const void* w_down, const float* s_down, void* y,
+                                      int* status, cudaStream_t s) {
+    CUtensorMap a, b;
+    const uint64_t R = (uint64_t)c.T * c.k;
+    if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM) ||
+        !make_map(&b, h, R, c.d_ff, NBOX))
+        return cudaErrorInvalidValue;
+    return launch_fp8<false>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d,
+                             status, s);
+}
 
 cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
                                      const int32_t* offsets, const void* w_gate_up, void* h,

@@ -101,6 +101,14 @@ cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
 cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int32_t* offsets,
                                   const void* w_down, void* y, int* status, cudaStream_t s);
 
+cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm,
+                                         const int32_t* offsets, const void* w_gate_up,
+                                         const float* s_gate_up, void* h, int* status,
+                                         cudaStream_t s);
+cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const int32_t* offsets,
+                                      const void* w_down, const float* s_down, void* y,
+                                      int* status, cudaStream_t s);
+
 cudaError_t launch_combine(const moe_config& c, const void* y, const int32_t* row_of,
                            const float* topk_w, void* out, cudaStream_t s);
 

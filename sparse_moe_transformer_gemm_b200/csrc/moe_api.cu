@@ -60,12 +60,13 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA
 
 // Automatic choice: the TMA-fed tensor-core tiles stream the weights faster than
 // the register-staged streaming kernels at every batch size measured on B200
-// (decode T=64: 1.12 ms vs 1.45 ms per layer), so they are the default for bf16
-// weights; FP8 weights use the streaming kernels.
+// (decode T=64: 1.07 ms vs 1.45 ms per layer), so they are the default. FP8
+// weights have a tensor-core path on SM pairs only (d, d_ff multiples of 256);
+// other FP8 shapes use the streaming kernels.
 bool use_stream_path(const moe_config* c) {
     if (c->flags & MOE_FLAG_STREAM_PATH) return true;
     if (c->flags & MOE_FLAG_GEMM_PATH) return false;
-    return (c->flags & MOE_FLAG_FP8_WEIGHTS) != 0;
+    return (c->flags & MOE_FLAG_FP8_WEIGHTS) != 0 && !pair_gemm_supported(*c);
 }
 
 // Router: tensor-core kernel where it applies (k <= 8), CUDA-core kernel otherwise.
@@ -83,8 +84,12 @@ int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offs
                     cudaStream_t s) {
     if (use_stream_path(c))
         return cuda_status(launch_gate_up_stream(*c, x_perm, offsets, w_gate_up, s_gate_up, h, s));
-    if (c->flags & MOE_FLAG_FP8_WEIGHTS) return MOE_ERR_UNSUPPORTED_SHAPE;
     int* status = at<int>(ws, ws_layout(*c).status);
+    if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
+        if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
+        return cuda_status(launch_gate_up_gemm_pair_fp8(*c, x_perm, offsets, w_gate_up, s_gate_up,
+                                                        h, status, s));
+    }
     if (pair_gemm_supported(*c))
         return cuda_status(launch_gate_up_gemm_pair(*c, x_perm, offsets, w_gate_up, h, status, s));
     return cuda_status(launch_gate_up_gemm(*c, x_perm, offsets, w_gate_up, h, status, s));
@@ -94,8 +99,12 @@ int experts_down(const moe_config* c, const void* h, const int32_t* offsets, con
                  const float* s_down, void* y, void* ws, cudaStream_t s) {
     if (use_stream_path(c))
         return cuda_status(launch_down_stream(*c, h, offsets, w_down, s_down, y, s));
-    if (c->flags & MOE_FLAG_FP8_WEIGHTS) return MOE_ERR_UNSUPPORTED_SHAPE;
     int* status = at<int>(ws, ws_layout(*c).status);
+    if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
+        if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
+        return cuda_status(
+            launch_down_gemm_pair_fp8(*c, h, offsets, w_down, s_down, y, status, s));
+    }
     if (pair_gemm_supported(*c))
         return cuda_status(launch_down_gemm_pair(*c, h, offsets, w_down, y, status, s));
     return cuda_status(launch_down_gemm(*c, h, offsets, w_down, y, status, s));
