@@ -347,36 +347,63 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 
 // ======================================================================
 // FP8 (e4m3) weights. The MMA stays kind::f16 (bf16 x bf16, fp32 accumulate)
-// on weights widened on chip: a producer warp TMA-loads raw e4m3 weight tiles
-// (128 rows x 64 bytes per K block, unswizzled) into a "raw" ring; four
-// converter warps widen them exactly to bf16 straight into the 128-byte-
-// swizzled operand layout of the MMA, issue the stage's token-half TMA, and
-// arrive on the even CTA's operand barrier. The per-output-row fp32 scale
-// multiplies the finished dot product in the epilogue (before SiLU for
-// gate_up, before the bf16 store for down): sum_c x_c q_c s_row = s_row
-// sum_c x_c q_c. Every e4m3 value is representable in bf16, so the widening
-// loses nothing.
+// on weights widened on chip. Per K block, warp 0 TMA-loads this CTA's raw
+// e4m3 weight tile(s) (128 rows x 64 bytes, unswizzled) into a "raw" ring on
+// the CTA's own barrier; warp 15 loads its half of the token rows (bf16,
+// 128-byte swizzle) into a token ring completing on the even CTA's barrier.
+// Converter warps, in groups that take K blocks round-robin (so the conversion
+// latencies of consecutive blocks overlap; 2 x 4 warps for gate_up, 3 x 3 for
+// down), widen the weights exactly to bf16 straight into the
+// 128-byte-swizzled operand layout of an "op" stage, release the raw stage and
+// arrive on the even CTA's operand barrier; the pair MMA reads A from the op
+// stage and B from the token stage and releases both. The raw stages live only
+// from load to conversion, so their ring keeps the weight stream deep. The
+// per-output-row fp32 scale multiplies the finished dot product in the
+// epilogue (before SiLU for gate_up, before the bf16 store for down):
+// sum_c x_c q_c s_row = s_row sum_c x_c q_c. Every e4m3 value is a bf16
+// value, so the widening loses nothing.
 
-constexpr int THREADS_FP8 = 320;        // + warps 6-9: converters
+constexpr int THREADS_FP8 = 512;        // warps 6-14 converters, warp 15 token producer
 constexpr int RAW_BYTES = BM * BK;      // one 128 x 64 e4m3 tile
 
 template <bool GATE_UP>
 struct Fp8Shape {
     static constexpr int A_TILES = GATE_UP ? 2 : 1;
-    static constexpr int RAW_STAGE = A_TILES * RAW_BYTES;                  // 16 KB / 8 KB
-    static constexpr int OP_STAGE = A_TILES * A_BYTES + BH_BYTES;          // 48 KB / 32 KB
-    static constexpr int RAW_STAGES = GATE_UP ? 4 : 6;
-    static constexpr int OP_STAGES = GATE_UP ? 3 : 5;
-    static constexpr int RING_BYTES = OP_STAGES * OP_STAGE + RAW_STAGES * RAW_STAGE;  // 208 KB
+    static constexpr int RAW_STAGE = A_TILES * RAW_BYTES;          // 16 KB / 8 KB
+    static constexpr int OP_STAGE = A_TILES * A_BYTES;             // 32 KB / 16 KB
+    static constexpr int RAW_STAGES = GATE_UP ? 4 : 6;  // multiples of GROUPS
+    static constexpr int B_STAGES = GATE_UP ? 3 : 4;
+    static constexpr int OP_STAGES = GATE_UP ? 3 : 6;   // >= GROUPS (see the converters)
+    // converter warps: GROUPS groups of GROUP_WARPS take K blocks round-robin
+    static constexpr int GROUPS = GATE_UP ? 2 : 3;
+    static constexpr int GROUP_WARPS = GATE_UP ? 4 : 3;
+    static constexpr int CONV_THREADS = GROUP_WARPS * 32;
+    static constexpr int RING_BYTES =
+        RAW_STAGES * RAW_STAGE + B_STAGES * BH_BYTES + OP_STAGES * OP_STAGE;  // 208 KB
     static constexpr int ACC_STAGES = GATE_UP ? 1 : 2;
     static constexpr int ACC_COLS = GATE_UP ? 512 : 256;
 };
 
+constexpr int CONV_WARPS = 9;                          // warps 6..14 (some idle for gate_up)
+constexpr int TOKEN_WARP = 6 + CONV_WARPS;
+template <bool G>
+constexpr bool groups_ok() {
+    using S = Fp8Shape<G>;
+    return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES >= S::GROUPS &&
+           S::GROUPS * S::GROUP_WARPS <= CONV_WARPS;
+}
+// Each group owns whole raw stages, and a group's previous operand wait proves
+// that the stage's last reader finished (parity waits cannot see a stale phase).
+static_assert(groups_ok<true>() && groups_ok<false>(), "converter grouping");
+static_assert(THREADS_FP8 == 32 * (TOKEN_WARP + 1), "warp roles cover the block");
+
 struct Fp8Ctrl {
-    uint64_t raw_full[6];   // each CTA: its raw weight tile landed
-    uint64_t raw_empty[6];  // each CTA: its converters are done with the raw stage
-    uint64_t op_full[5];    // even CTA: both CTAs converted + token bytes of both landed
-    uint64_t op_empty[5];   // both CTAs: the pair MMAs finished reading the operand stage
+    uint64_t raw_full[6];   // each CTA: its raw weight tile(s) landed
+    uint64_t raw_empty[6];  // each CTA: every converter warp is done with the raw stage
+    uint64_t b_full[4];     // even CTA: token bytes of both CTAs landed
+    uint64_t b_empty[4];    // both CTAs: the pair MMAs finished reading the token stage
+    uint64_t op_full[6];    // even CTA: every converter warp of both CTAs filled the op stage
+    uint64_t op_empty[6];   // both CTAs: the pair MMAs finished reading the op stage
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -394,39 +421,50 @@ constexpr int fp8_smem_bytes() {
 static_assert(fp8_smem_bytes<true>() <= 232448 && fp8_smem_bytes<false>() <= 232448,
               "fits in 227 KB");
 
-// Two e4m3 codes -> bf16x2, exactly: the hardware e4m3x2 -> f16x2 conversion,
-// then f16 -> bf16 by rebiasing the exponent (15 -> 127: +112 << 7 after the
-// 3-bit mantissa shift). e4m3-valued f16 numbers are normal or zero and carry
-// no mantissa bits below bit 7, so the shift drops nothing; zeros keep their sign.
+// Two e4m3 codes -> bf16x2, exactly: hardware e4m3x2 -> f16x2, each f16 ->
+// f32 (exact), then the high halves of the two f32 (a value with at most 4
+// significant bits has zero low halves, so keeping the high half is exact;
+// signed zeros carry over).
 __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t q) {
-    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)q, __NV_E4M3);
-    const uint32_t h = (uint32_t)hr.x | ((uint32_t)hr.y << 16);
-    const uint32_t mag = h & 0x7FFF7FFFu;
-    const uint32_t nz = __vcmpne2(mag, 0u);
-    return (((mag >> 3) + 0x38003800u) & nz) | (h & 0x80008000u);
+    uint32_t out;
+    asm("{\n\t.reg .b32 h2, f0, f1;\n\t.reg .b16 h0, h1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h2, %1;\n\t"
+        "mov.b32 {h0, h1}, h2;\n\t"
+        "cvt.f32.f16 f0, h0;\n\t"
+        "cvt.f32.f16 f1, h1;\n\t"
+        "prmt.b32 %0, f0, f1, 0x7632;\n\t}"
+        : "=r"(out)
+        : "h"(q));
+    return out;
 }
 
 // Convert one raw e4m3 tile (128 rows x 64 bytes, row-major) into a bf16
-// operand tile (128 rows x 128 bytes, 128-byte swizzle). 128 threads; thread
-// `ct` handles 16-byte source chunks q = ct + 128 i (row q/4, elements 16(q%4)..).
-__device__ __forceinline__ void widen_tile(const uint8_t* raw, uint8_t* op, int ct) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int q = ct + 128 * i;
+// operand tile (128 rows x 128 bytes, 128-byte swizzle) with CONV_THREADS threads;
+// thread `ct` handles 16-byte source chunks q = ct + CONV_THREADS i (row q/4,
+// elements 16(q%4)..16(q%4)+15).
+template <int CONV_THREADS>
+__device__ __forceinline__ void widen_tile(uint32_t raw, uint32_t op, int ct) {
+    for (int q = ct; q < 512; q += CONV_THREADS) {
         const int row = q >> 2, c = q & 3;
-        const uint4 v = *reinterpret_cast<const uint4*>(raw + q * 16);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t w[4];
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "r"(raw + q * 16));
         uint32_t b[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             b[2 * j] = e4m3x2_to_bf16x2((uint16_t)(w[j] & 0xFFFFu));
             b[2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(w[j] >> 16));
         }
-        uint8_t* rbase = op + row * 128;
+        const uint32_t rbase = op + row * 128;
         const int sw = row & 7;
-        *reinterpret_cast<uint4*>(rbase + (((2 * c) ^ sw) << 4)) = make_uint4(b[0], b[1], b[2], b[3]);
-        *reinterpret_cast<uint4*>(rbase + (((2 * c + 1) ^ sw) << 4)) =
-            make_uint4(b[4], b[5], b[6], b[7]);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rbase + (((2 * c) ^ sw) << 4)),
+                     "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3])
+                     : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         rbase + (((2 * c + 1) ^ sw) << 4)),
+                     "r"(b[4]), "r"(b[5]), "r"(b[6]), "r"(b[7])
+                     : "memory");
     }
 }
 
@@ -444,8 +482,9 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* op_ring = smem;
-    uint8_t* raw_ring = smem + S::OP_STAGES * S::OP_STAGE;
+    uint8_t* op_ring = smem;  // 1024-aligned operand stages first
+    uint8_t* b_ring = op_ring + S::OP_STAGES * S::OP_STAGE;
+    uint8_t* raw_ring = b_ring + S::B_STAGES * BH_BYTES;
     Fp8Ctrl& c = *reinterpret_cast<Fp8Ctrl*>(smem + S::RING_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)(tc::cluster_ctarank() & 1u);
@@ -487,10 +526,14 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         if (lane == 0) {
             for (int s = 0; s < S::RAW_STAGES; ++s) {
                 tc::mbar_init(&c.raw_full[s], 1);
-                tc::mbar_init(&c.raw_empty[s], 1);
+                tc::mbar_init(&c.raw_empty[s], S::GROUP_WARPS);
+            }
+            for (int s = 0; s < S::B_STAGES; ++s) {
+                tc::mbar_init(&c.b_full[s], 1);
+                tc::mbar_init(&c.b_empty[s], 1);
             }
             for (int s = 0; s < S::OP_STAGES; ++s) {
-                tc::mbar_init(&c.op_full[s], 2);  // one converter arrival per CTA (+ token bytes)
+                tc::mbar_init(&c.op_full[s], 2 * S::GROUP_WARPS);
                 tc::mbar_init(&c.op_empty[s], 1);
             }
             for (int a = 0; a < S::ACC_STAGES; ++a) {
@@ -514,7 +557,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- raw e4m3 weight producer (this CTA's rows, own barrier)
-            const uint64_t pol = tc::policy_evict_first();
+            const uint64_t pol_w = tc::policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t parity[S::RAW_STAGES] = {};
@@ -531,10 +574,10 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     uint8_t* st = raw_ring + stage * S::RAW_STAGE;
                     tc::mbar_arrive_expect_tx(&c.raw_full[stage], S::RAW_STAGE);
-                    tc::tma_load_2d_hint(st, &tmA, &c.raw_full[stage], kb * BK, a_row, pol);
+                    tc::tma_load_2d_hint(st, &tmA, &c.raw_full[stage], kb * BK, a_row, pol_w);
                     if (GATE_UP)
                         tc::tma_load_2d_hint(st + RAW_BYTES, &tmA, &c.raw_full[stage], kb * BK,
-                                             a_row + a_rows_per_expert / 2, pol);
+                                             a_row + a_rows_per_expert / 2, pol_w);
                     issued[stage] = true;
                     parity[stage] = phase;
                     if (++stage == S::RAW_STAGES) {
@@ -548,61 +591,83 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (issued[s] && !tc::mbar_wait(&c.raw_full[s], parity[s], &zero))
                     atomicExch(status, MOE_ERR_TIMEOUT);
         }
-    } else if (warp >= 6) {
-        // ---------------- converters: raw e4m3 -> bf16 operand; token-half TMA
-        const int ct = threadIdx.x - 192;  // 0..127
-        const uint64_t pol_x = tc::policy_evict_last();
-        int rs = 0, os = 0;
-        uint32_t rph = 0, oph = 0;
-        for (int t = pair; t < total; t += n_pairs) {
-            const TileInfo ti = decode_tile(c, E, m_tiles, t);
-            const int nb = ti.n / (2 * NBOX);
-            const int b_row = ti.row0 + rank * (ti.n / 2);
-            const uint32_t b_pair_bytes = 2u * (uint32_t)(nb * BOX_BYTES);
+    } else if (warp == TOKEN_WARP) {
+        if (lane == 0) {
+            // ---------------- token-half producer; completes on the even CTA's b_full
+            const uint64_t pol_x = tc::policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t parity[S::B_STAGES] = {};
+            bool issued[S::B_STAGES] = {};
             bool ok = true;
-            for (int kb = 0; kb < KB; ++kb) {
-                const bool got = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag) &&
-                                 tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
-                uint8_t* op = op_ring + os * S::OP_STAGE;
-                const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0);
-                if (got) {
-                    if (ct == 0)
-                        for (int b = 0; b < nb; ++b)
-                            tc::tma_load_2d_pair(op + S::A_TILES * A_BYTES + b * BOX_BYTES, &tmB,
-                                                 full_leader, kb * BK, b_row + b * NBOX, pol_x);
-                    const uint8_t* raw = raw_ring + rs * S::RAW_STAGE;
-                    widen_tile(raw, op, ct);
-                    if (GATE_UP) widen_tile(raw + RAW_BYTES, op + A_BYTES, ct);
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                }
-                if (tc::bar_any(2, 128, !got)) {  // the four converter warps leave together
-                    raise_timeout(c, status);
-                    ok = false;
-                    break;
-                }
-                if (ct == 0) {
-                    tc::mbar_arrive(&c.raw_empty[rs]);
-                    if (leader)
-                        tc::mbar_arrive_expect_tx(&c.op_full[os], b_pair_bytes);
-                    else
-                        tc::mbar_arrive_cluster(full_leader);
-                }
-                if (++rs == S::RAW_STAGES) {
-                    rs = 0;
-                    rph ^= 1u;
-                }
-                if (++os == S::OP_STAGES) {
-                    os = 0;
-                    oph ^= 1u;
+            for (int t = pair; t < total && ok; t += n_pairs) {
+                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const int nb = ti.n / (2 * NBOX);
+                const int b_row = ti.row0 + rank * (ti.n / 2);
+                const uint32_t pair_bytes = 2u * (uint32_t)(nb * BOX_BYTES);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&c.b_empty[stage], phase ^ 1u, abort_flag)) {
+                        raise_timeout(c, status);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.b_full[stage]), 0);
+                    if (leader) tc::mbar_arrive_expect_tx(&c.b_full[stage], pair_bytes);
+                    uint8_t* st = b_ring + stage * BH_BYTES;
+                    for (int b = 0; b < nb; ++b)
+                        tc::tma_load_2d_pair(st + b * BOX_BYTES, &tmB, full_leader, kb * BK,
+                                             b_row + b * NBOX, pol_x);
+                    issued[stage] = true;
+                    parity[stage] = phase;
+                    if (++stage == S::B_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
-            if (!ok) break;
+            const int zero = 0;
+            for (int s = 0; s < S::B_STAGES; ++s)
+                if (issued[s] && !tc::mbar_wait(leader ? &c.b_full[s] : &c.b_empty[s], parity[s], &zero))
+                    atomicExch(status, MOE_ERR_TIMEOUT);
+        }
+    } else if (warp >= 6 && warp < 6 + CONV_WARPS) {
+        // ---------------- converters: raw e4m3 -> bf16 operand (A) in the op stage.
+        // Each warp arrives on the even CTA's op_full on its own (after its
+        // writes are fenced to the async proxy); a warp whose bounded wait
+        // gave up stops, and the MMA's bounded wait on op_full then gives up.
+        const int group = (warp - 6) / S::GROUP_WARPS;
+        const int ct = threadIdx.x - 192 - group * S::CONV_THREADS;  // 0..CONV_THREADS-1
+        const uint32_t raw0 = tc::smem_u32(raw_ring), op0 = tc::smem_u32(op_ring);
+        // this CTA's K blocks in order: j = tile_iteration * KB + kb; a group
+        // converts j = group, group + GROUPS, ... (warps past the groups idle)
+        int n_my_tiles = 0;
+        for (int t = pair; t < total; t += n_pairs) ++n_my_tiles;
+        const long n_blocks = (long)n_my_tiles * KB;
+        for (long jb = (group < S::GROUPS ? group : n_blocks); jb < n_blocks; jb += S::GROUPS) {
+            const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
+            const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
+            const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
+            if (!tc::mbar_wait(&c.raw_full[rs], rph, abort_flag) ||
+                !tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag)) {
+                raise_timeout(c, status);
+                break;
+            }
+            const uint32_t raw = raw0 + rs * S::RAW_STAGE;
+            const uint32_t op = op0 + os * S::OP_STAGE;
+            widen_tile<S::CONV_THREADS>(raw, op, ct);
+            if (GATE_UP) widen_tile<S::CONV_THREADS>(raw + RAW_BYTES, op + A_BYTES, ct);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(&c.raw_empty[rs]);
+                tc::mbar_arrive_cluster(tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
+            }
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
-            // ---------------- MMA issuer (even CTA)
-            int os = 0;
-            uint32_t oph = 0;
+            // ---------------- MMA issuer (even CTA): A from the op stage, B from the raw stage
+            int bs = 0, os = 0;
+            uint32_t oph = 0, bph = 0;
             bool ok = true;
             int it = 0;
             for (int t = pair; t < total && ok; t += n_pairs, ++it) {
@@ -617,14 +682,15 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
                 const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, ti.n);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!tc::mbar_wait(&c.op_full[os], oph, abort_flag)) {
+                    if (!tc::mbar_wait(&c.op_full[os], oph, abort_flag) ||
+                        !tc::mbar_wait(&c.b_full[bs], bph, abort_flag)) {
                         raise_timeout(c, status);
                         ok = false;
                         break;
                     }
                     tc::fence_after_sync();
                     const uint32_t a_addr = tc::smem_u32(op_ring + os * S::OP_STAGE);
-                    const uint32_t b_addr = a_addr + S::A_TILES * A_BYTES;
+                    const uint32_t b_addr = tc::smem_u32(b_ring + bs * BH_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / UK; ++k) {
                         const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
@@ -637,9 +703,14 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                                               idesc, accum);
                     }
                     tc::mma_commit_pair(&c.op_empty[os], 0x3);
+                    tc::mma_commit_pair(&c.b_empty[bs], 0x3);
                     if (++os == S::OP_STAGES) {
                         os = 0;
                         oph ^= 1u;
+                    }
+                    if (++bs == S::B_STAGES) {
+                        bs = 0;
+                        bph ^= 1u;
                     }
                 }
                 if (ok) tc::mma_commit_pair(&c.acc_full[acc], 0x3);
