@@ -15,7 +15,9 @@ from typing import Optional
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+# MOE_B200_LIB selects another build of the same library (e.g. for A/B timing).
+LIB_PATH = os.environ.get("MOE_B200_LIB") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1
