@@ -125,6 +125,20 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def slowest_rank_ms(ms: float, dist=None, device=None) -> float:
+    """Max over ranks of a per-rank device time (identity without a process group)."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput of independent replicas: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms / 1e3)
+
+
 def dist_setup():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -300,10 +314,7 @@ def main():
     ms = t_begin.elapsed_time(t_end) / args.steps
     stage_ms = {s: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps
                 for j, s in enumerate(stages)}
-    if pg:
-        tm = torch.tensor([ms], device=dev)
-        pg.all_reduce(tm, op=pg.ReduceOp.MAX)
-        ms = float(tm.item())
+    ms = slowest_rank_ms(ms, pg, dev)
 
     # touched experts of this batch (for the algorithmic bytes)
     touched = int((counts > 0).sum().item())
@@ -364,10 +375,7 @@ def main():
         e1.record(stream)
     stream.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if pg:
-        tm = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(tm, op=pg.ReduceOp.MAX)
-        e2e_ms = float(tm.item())
+    e2e_ms = slowest_rank_ms(e2e_ms, pg, dev)
     status2 = moe.moe_read_status(ws, stream)
 
     cpu = None
@@ -376,7 +384,7 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": "MoE-layer tokens/s", "value": world * T / (ms / 1e3), "unit": "tokens/s",
+            "metric": "MoE-layer tokens/s", "value": replica_value(T, world, ms), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 weights, bf16 activations, fp32 accumulate" if fp8 else
@@ -396,7 +404,7 @@ def main():
                 "touched_experts": touched},
             "stage_ms": stage_ms,
             "clocks": clocks.summary(),
-            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": replica_value(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
                     "ms_per_step": e2e_ms, "api": "moe_forward"},
             "gpu_launches": sum(n_launch.values()) * args.steps,
