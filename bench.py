@@ -262,13 +262,20 @@ def main():
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     row_of = torch.empty(R, dtype=torch.int32, device=dev)
-    xp = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
+    gather = R <= moe.MOE_GATHER_MAX_SLOTS  # moe_forward's grouping rule
+    tok = torch.empty(R, dtype=torch.int32, device=dev)
+    xp = None if gather else torch.empty((R, d), dtype=torch.bfloat16, device=dev)
     h = torch.empty((R, F), dtype=torch.bfloat16, device=dev)
     y = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
     out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
 
     stages = ["route", "permute", "gate_up", "down", "combine"]
-    n_launch = {"route": 1, "permute": 3, "gate_up": 1, "down": 1, "combine": 1}
+    # small batches: one grouping launch, and gate_up gathers its token rows inside
+    # the GEMM on the bf16 SM-pair path (a row-gather kernel first on the others);
+    # large batches: rank/scan/scatter with the permuted copy, then gate_up
+    fused_gather = (not shape.fp8 and args.path != "stream" and d % 256 == 0 and F % 256 == 0)
+    n_launch = {"route": 1, "permute": 1 if gather else 3,
+                "gate_up": 2 if gather and not fused_gather else 1, "down": 1, "combine": 1}
 
     def step(ev=None):
         if ev is not None:
@@ -276,10 +283,16 @@ def main():
         moe.moe_route(cfg, x, wg, gb, idx, w, ws, stream)
         if ev is not None:
             ev[1].record(stream)
-        moe.moe_permute(cfg, idx, x, counts, offsets, row_of, xp, ws, stream)
+        if gather:
+            moe.moe_permute_index(cfg, idx, counts, offsets, row_of, tok, ws, stream)
+        else:
+            moe.moe_permute(cfg, idx, x, counts, offsets, row_of, xp, ws, stream)
         if ev is not None:
             ev[2].record(stream)
-        moe.moe_expert_gate_up(cfg, xp, offsets, wgu, sgu, h, ws, stream)
+        if gather:
+            moe.moe_expert_gate_up_gather(cfg, x, tok, offsets, wgu, sgu, h, ws, stream)
+        else:
+            moe.moe_expert_gate_up(cfg, xp, offsets, wgu, sgu, h, ws, stream)
         if ev is not None:
             ev[3].record(stream)
         moe.moe_expert_down(cfg, h, offsets, wd, sd, y, ws, stream)

@@ -111,6 +111,15 @@ MOE_API int moe_permute(const moe_config* cfg, const int32_t* topk_idx, const vo
                 int32_t* offsets, int32_t* row_of, void* x_perm, void* ws, size_t ws_bytes,
                 void* stream);
 
+/* The grouping of moe_permute without the activation copy: writes counts,
+ * offsets and row_of exactly as moe_permute does, and token_of_row [T*k]
+ * int32 with token_of_row[row_of[t*k+j]] = t for every kept slot (rows at or
+ * beyond offsets[E] are not written). For moe_expert_gate_up_gather, which
+ * reads the token rows of x by these indices. Same pages as moe_permute. */
+MOE_API int moe_permute_index(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
+                      int32_t* offsets, int32_t* row_of, int32_t* token_of_row, void* ws,
+                      size_t ws_bytes, void* stream);
+
 /* gate_up step of the SwiGLU experts on grouped rows: for each expert e and
  * each of its rows r in [offsets[e], offsets[e+1]):
  *   h[r, f] = bf16( SiLU(g) * u ),  g = <x_perm[r], w_gate_up[e, f]>,
@@ -120,6 +129,17 @@ MOE_API int moe_permute(const moe_config* cfg, const int32_t* topk_idx, const vo
 MOE_API int moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
                        const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
                        size_t ws_bytes, void* stream);
+
+/* moe_expert_gate_up with the grouped rows read from x by index: the row r
+ * of expert e is x[token_of_row[r]] (x [T, d] bf16, token_of_row as written
+ * by moe_permute_index, every entry in [0, T) for rows below offsets[E]).
+ * Result identical to moe_permute + moe_expert_gate_up. The bf16 tensor-core
+ * SM-pair kernel gathers the rows with TMA as it loads them; the other paths
+ * first copy them into the workspace. */
+MOE_API int moe_expert_gate_up_gather(const moe_config* cfg, const void* x,
+                              const int32_t* token_of_row, const int32_t* offsets,
+                              const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
+                              size_t ws_bytes, void* stream);
 
 /* down step: y[r, i] = bf16( <h[r], w_down[e, i]> ), fp32 accumulate; y is
  * [T*k, d] bf16. Pages: "Tencent Hy3-295B 架构深度拆解" §2.3 (down_proj
@@ -140,8 +160,16 @@ MOE_API int moe_experts(const moe_config* cfg, const void* x_perm, const int32_t
 MOE_API int moe_combine(const moe_config* cfg, const void* y, const int32_t* row_of, const float* topk_w,
                 void* out, void* ws, size_t ws_bytes, void* stream);
 
-/* The whole layer: route, group, experts, combine. out [T, d] bf16. The
- * intermediates live in ws. Resets the workspace status word first. */
+/* Batches of at most this many token-slots (T*k) are grouped by index
+ * (moe_permute_index) and their gate_up GEMM gathers the token rows itself
+ * (moe_expert_gate_up_gather); larger batches write the permuted copy
+ * (moe_permute + moe_expert_gate_up): once tiles hold many tokens, the
+ * one-row TMA gathers cost more than the copy. */
+#define MOE_GATHER_MAX_SLOTS 4096
+
+/* The whole layer: route, group, gate_up, down, combine (the grouping and
+ * gate_up as MOE_GATHER_MAX_SLOTS says). out [T, d] bf16. The intermediates
+ * live in ws. Resets the workspace status word first. */
 MOE_API int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
                 const void* w_gate_up, const float* s_gate_up, const void* w_down,
                 const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream);

@@ -13,7 +13,12 @@
 namespace moe {
 namespace {
 
-__global__ void __launch_bounds__(256)
+// CTA (token t, column block b): 128 threads, one 8-column vector each. The k
+// expert rows are loaded 8 at a time before their FMAs (independent loads in
+// flight), the FMAs run in j order.
+constexpr int CT = 128;
+
+__global__ void __launch_bounds__(CT)
 combine_kernel(const __nv_bfloat16* __restrict__ y, const int* __restrict__ row_of,
                const float* __restrict__ w, int k, int d, __nv_bfloat16* __restrict__ out) {
     __shared__ int rows[32];
@@ -24,34 +29,45 @@ combine_kernel(const __nv_bfloat16* __restrict__ y, const int* __restrict__ row_
         wts[threadIdx.x] = w[t * k + threadIdx.x];
     }
     __syncthreads();
-    for (int v = threadIdx.x; v < d / 8; v += blockDim.x) {
-        float acc[8];
+    const int v = blockIdx.y * CT + threadIdx.x;
+    if (v >= d / 8) return;
+    float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-        for (int j = 0; j < k; ++j) {
-            const int r = rows[j];
-            if (r < 0) continue;
-            const uint4 u = *reinterpret_cast<const uint4*>(y + (long)r * d + v * 8);
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int j0 = 0; j0 < k; j0 += 8) {
+        uint4 u[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+            const int j = j0 + jj;
+            const int r = (j < k) ? rows[j] : -1;
+            u[jj] = (r >= 0) ? __ldcs(reinterpret_cast<const uint4*>(y + (long)r * d) + v)
+                             : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+            const int j = j0 + jj;
+            if (j >= k || rows[j] < 0) continue;
             float f[8];
-            bf16x8_to_float(u, f);
+            bf16x8_to_float(u[jj], f);
             const float wj = wts[j];
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
         }
-        uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        *reinterpret_cast<uint4*>(out + t * d + v * 8) = o;
     }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(out + t * d + v * 8) = o;
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const moe_config& c, const void* y, const int32_t* row_of,
                            const float* topk_w, void* out, cudaStream_t s) {
-    combine_kernel<<<c.T, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(y), row_of, topk_w, c.k,
+    const dim3 grid(c.T, (c.d / 8 + CT - 1) / CT);
+    combine_kernel<<<grid, CT, 0, s>>>(static_cast<const __nv_bfloat16*>(y), row_of, topk_w, c.k,
                                        c.d, static_cast<__nv_bfloat16*>(out));
     return cudaGetLastError();
 }

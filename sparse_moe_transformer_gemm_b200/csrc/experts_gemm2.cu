@@ -40,6 +40,29 @@ constexpr int BOX_BYTES = NBOX * BK * 2;
 constexpr int BH_BYTES = (NMAX / 2) * BK * 2;  // this CTA's half of the token rows
 constexpr int THREADS = 224;
 constexpr int MAX_E = 256;
+constexpr int EPI_N = 32;                          // tokens per epilogue chunk
+constexpr int EPI_BYTES = 2 * EPI_N * BM * 2;      // double-buffered [EPI_N][BM] bf16 tile
+
+// Token-row tensor maps with boxes of 16, 32, 64 and 128 rows: a CTA's half of
+// a tile (a multiple of 16 rows, at most 128) loads as at most four boxes
+// (its binary decomposition) instead of up to eight 16-row boxes. The gather
+// variant uses m[0] only, with a one-row box.
+struct TokenMaps {
+    CUtensorMap m[4];
+};
+
+__device__ __forceinline__ void load_token_rows(uint8_t* dst, const TokenMaps& tm,
+                                                uint32_t bar_leader, int kx, int row, int rows,
+                                                uint64_t pol) {
+    // one copy site in a rolled loop: an unrolled form with four predicated copies
+    // measured slower on B200 even where only the 16-row box was used
+    for (int off = 0; off < rows;) {
+        const int rem = rows - off;
+        const int lg = rem >= 8 * NBOX ? 3 : rem >= 4 * NBOX ? 2 : rem >= 2 * NBOX ? 1 : 0;
+        tc::tma_load_2d_pair(dst + off * (BK * 2), &tm.m[lg], bar_leader, kx, row + off, pol);
+        off += NBOX << lg;
+    }
+}
 
 template <bool GATE_UP>
 struct Shape {
@@ -65,7 +88,8 @@ struct Ctrl {
 
 template <bool GATE_UP>
 constexpr int smem_bytes() {
-    return Shape<GATE_UP>::STAGES * Shape<GATE_UP>::STAGE_BYTES + 1024 + (int)sizeof(Ctrl);
+    return Shape<GATE_UP>::STAGES * Shape<GATE_UP>::STAGE_BYTES + EPI_BYTES + 1024 +
+           (int)sizeof(Ctrl);
 }
 
 struct TileInfo {
@@ -101,19 +125,24 @@ __device__ __forceinline__ void raise_timeout(CtrlT& c, int* status) {
 }
 
 // tmA: weights [E * a_rows_per_expert, K] bf16, box 64 x 128.
-// tmB: token rows [R, K] bf16, box 64 x 16.
+// tmB: token rows [R, K] bf16, boxes of 64 columns x 16/32/64/128 rows.
 // m_tiles: 256-row weight tiles per expert (F/256 for gate_up, d/256 for down).
-template <bool GATE_UP>
+// GATHER: tmB maps the unpermuted token rows x [T, K] with a one-row box and
+// the token rows of each tile are gathered by index (token_of_row) with
+// tile::gather4 instead of being read from a permuted copy.
+template <bool GATE_UP, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ CUtensorMap tmB, const int* __restrict__ offsets,
-                         int E, int K, int a_rows_per_expert, int m_tiles,
-                         __nv_bfloat16* __restrict__ out, int out_ld, int* __restrict__ status) {
+                         const __grid_constant__ TokenMaps tmB, const int* __restrict__ offsets,
+                         const int* __restrict__ token_of_row, int E, int K,
+                         int a_rows_per_expert, int m_tiles, __nv_bfloat16* __restrict__ out,
+                         int out_ld, int* __restrict__ status) {
     using S = Shape<GATE_UP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + S::STAGES * S::STAGE_BYTES);
+    uint16_t* epi = reinterpret_cast<uint16_t*>(smem + S::STAGES * S::STAGE_BYTES);
+    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + S::STAGES * S::STAGE_BYTES + EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)(tc::cluster_ctarank() & 1u);
     const bool leader = rank == 0;
@@ -149,7 +178,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             c.total = carry;
             c.abort = 0;
             tc::prefetch_tensormap(&tmA);
-            tc::prefetch_tensormap(&tmB);
+            for (int m = 0; m < (GATHER ? 1 : 4); ++m) tc::prefetch_tensormap(&tmB.m[m]);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -176,61 +205,73 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     const volatile int* abort_flag = &c.abort;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- producer: this CTA's weight rows and token half
-            const uint64_t pol_w = tc::policy_evict_first();
-            const uint64_t pol_x = tc::policy_evict_last();
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t parity[S::STAGES] = {};
-            bool issued[S::STAGES] = {};
-            bool ok = true;
-            for (int t = pair; t < total && ok; t += n_pairs) {
-                const TileInfo ti = decode_tile(c, E, m_tiles, t);
-                const int nb = ti.n / (2 * NBOX);  // boxes per CTA
-                const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
-                const int b_row = ti.row0 + rank * (ti.n / 2);
-                const uint32_t pair_bytes = 2u * (S::A_TILES * A_BYTES + nb * BOX_BYTES);
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!tc::mbar_wait(&c.empty[stage], phase ^ 1u, abort_flag)) {
-                        raise_timeout(c, status);
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.full[stage]), 0);
+        // ---------------- producer: this CTA's weight rows and token half. Lane 0
+        // waits for each stage and issues the weight loads and (copy path) the
+        // token boxes; with GATHER every lane l with 4l < half also gathers rows
+        // 4l..4l+3 of x with one tile::gather4.
+        const uint64_t pol_w = tc::policy_evict_first();
+        const uint64_t pol_x = tc::policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t parity[S::STAGES] = {};
+        bool issued[S::STAGES] = {};
+        bool ok = true;
+        if (!GATHER && lane != 0) ok = false;  // the copy path issues from lane 0 alone
+        for (int t = pair; t < total && ok; t += n_pairs) {
+            const TileInfo ti = decode_tile(c, E, m_tiles, t);
+            const int half = ti.n / 2;
+            const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
+            const int b_row = ti.row0 + rank * half;
+            const uint32_t pair_bytes = 2u * (S::A_TILES * A_BYTES + half * BK * 2);
+            int tok[4] = {0, 0, 0, 0};
+            if (GATHER) {
+                // rows past the tile's end repeat its first row (in range, ignored)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = b_row + 4 * lane + i;
+                    tok[i] = token_of_row[r < ti.row0 + ti.len ? r : ti.row0];
+                }
+            }
+            for (int kb = 0; kb < KB; ++kb) {
+                if (lane == 0 && !tc::mbar_wait(&c.empty[stage], phase ^ 1u, abort_flag)) {
+                    raise_timeout(c, status);
+                    ok = false;
+                }
+                if (GATHER) ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.full[stage]), 0);
+                uint8_t* s = smem + stage * S::STAGE_BYTES;
+                uint8_t* sb = s + S::A_TILES * A_BYTES;
+                if (lane == 0) {
                     if (leader) tc::mbar_arrive_expect_tx(&c.full[stage], pair_bytes);
-                    uint8_t* s = smem + stage * S::STAGE_BYTES;
                     tc::tma_load_2d_pair(s, &tmA, full_leader, kb * BK, a_row, pol_w);
                     if (GATE_UP)
                         tc::tma_load_2d_pair(s + A_BYTES, &tmA, full_leader, kb * BK,
                                              a_row + a_rows_per_expert / 2, pol_w);
-                    uint8_t* sb = s + S::A_TILES * A_BYTES;
-                    for (int b = 0; b < nb; ++b)
-                        tc::tma_load_2d_pair(sb + b * BOX_BYTES, &tmB, full_leader, kb * BK,
-                                             b_row + b * NBOX, pol_x);
+                    if (!GATHER)
+                        load_token_rows(sb, tmB, full_leader, kb * BK, b_row, half, pol_x);
                     issued[stage] = true;
                     parity[stage] = phase;
-                    if (++stage == S::STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                }
+                if (GATHER) {
+                    __syncwarp();
+                    if (4 * lane < half)
+                        tc::tma_gather4_pair(sb + lane * (4 * BK * 2), &tmB.m[0], full_leader,
+                                             kb * BK, tok[0], tok[1], tok[2], tok[3], pol_x);
+                }
+                if (++stage == S::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
+        }
+        if (lane == 0) {
             // drain: this CTA's copies have landed (the even CTA's full barrier saw
             // every byte of both CTAs when its last phase completed)
-            if (leader) {
-                const int zero = 0;
-                for (int s = 0; s < S::STAGES; ++s)
-                    if (issued[s] && !tc::mbar_wait(&c.full[s], parity[s], &zero))
-                        atomicExch(status, MOE_ERR_TIMEOUT);
-            } else {
-                // the odd CTA's stages are released only after the pair MMAs read
-                // them, which is after they landed: wait for the last release
-                const int zero = 0;
-                for (int s = 0; s < S::STAGES; ++s)
-                    if (issued[s] && !tc::mbar_wait(&c.empty[s], parity[s], &zero))
-                        atomicExch(status, MOE_ERR_TIMEOUT);
-            }
+            const int zero = 0;
+            for (int s = 0; s < S::STAGES; ++s)
+                if (issued[s] && !tc::mbar_wait(leader ? &c.full[s] : &c.empty[s], parity[s], &zero))
+                    atomicExch(status, MOE_ERR_TIMEOUT);
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
@@ -283,9 +324,13 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             if (!tc::mbar_wait(&c.drain, 0, &zero)) atomicExch(status, MOE_ERR_TIMEOUT);
         }
     } else if (warp >= 2 && warp <= 5) {
-        // ---------------- epilogue: this CTA's 128 weight rows (TMEM lanes)
+        // ---------------- epilogue: this CTA's 128 weight rows (TMEM lanes). Per
+        // chunk of 32 tokens each warp writes its 32 rows x 32 tokens as bf16 into
+        // a shared [32 tokens][128 rows] tile (two buffers, alternating); after a
+        // named barrier the four warps store the tile as 256-byte row segments of
+        // the output with 16-byte vectors.
         const int quad = warp & 3;
-        const int row_in_tile = quad * 32 + lane;
+        const int et = threadIdx.x - 64;  // 0..127
         uint16_t* o16 = reinterpret_cast<uint16_t*>(out);
         const bool arriver = (warp == 2 && lane == 0);
         int it = 0;
@@ -293,11 +338,16 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             const TileInfo ti = decode_tile(c, E, m_tiles, t);
             const int acc = it % S::ACC_STAGES;
             const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
-            const bool ok = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
+            const bool waited = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
+            if (tc::bar_any(1, 128, !waited)) {  // the four warps leave together
+                raise_timeout(c, status);
+                break;
+            }
             tc::fence_after_sync();
             const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
-            const int col = ti.m * 2 * BM + rank * BM + row_in_tile;
-            for (int c0 = 0; ok && c0 < ti.n; c0 += 32) {
+            const int col0 = ti.m * 2 * BM + rank * BM;
+            for (int c0 = 0, buf = 0; c0 < ti.n; c0 += EPI_N, buf ^= 1) {
+                uint16_t* tile = epi + buf * (EPI_N * BM);
                 uint32_t g[32];
                 tc::tmem_ld32(tbase + c0, g);
                 if constexpr (GATE_UP) {
@@ -306,29 +356,29 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int n = c0 + j;
-                        if (n < ti.len) {
-                            const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
-                            const float hv = gv / (1.f + expf(-gv)) * uv;
-                            o16[(size_t)(ti.row0 + n) * out_ld + col] = float_to_bf16_bits(hv);
-                        }
+                        const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
+                        tile[j * BM + quad * 32 + lane] = float_to_bf16_bits(gv / (1.f + expf(-gv)) * uv);
                     }
                 } else {
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = c0 + j;
-                        if (n < ti.len)
-                            o16[(size_t)(ti.row0 + n) * out_ld + col] =
-                                float_to_bf16_bits(__uint_as_float(g[j]));
-                    }
+                    for (int j = 0; j < 32; ++j)
+                        tile[j * BM + quad * 32 + lane] = float_to_bf16_bits(__uint_as_float(g[j]));
+                }
+                tc::bar_sync(1, 128);
+#pragma unroll
+                for (int q = 0; q < EPI_N * BM / 8 / 128; ++q) {
+                    const int id = et + 128 * q;
+                    const int n = id / (BM / 8), ch = id % (BM / 8);
+                    if (c0 + n < ti.len)
+                        *reinterpret_cast<uint4*>(o16 + (size_t)(ti.row0 + c0 + n) * out_ld + col0 +
+                                                  ch * 8) =
+                            *reinterpret_cast<const uint4*>(tile + n * BM + ch * 8);
                 }
             }
+            // every warp's TMEM reads are complete before the accumulator is handed back
             tc::fence_before_sync();
-            if (tc::bar_any(1, 128, !ok)) {  // the four epilogue warps leave together
-                raise_timeout(c, status);
-                break;
-            }
+            tc::bar_sync(1, 128);
             if (arriver)
                 tc::mbar_arrive_cluster(tc::map_to_cta(tc::smem_u32(&c.acc_empty[acc]), 0));
         }
@@ -473,7 +523,7 @@ __device__ __forceinline__ void widen_tile(uint32_t raw, uint32_t op, int ct) {
 template <bool GATE_UP>
 __global__ void __launch_bounds__(THREADS_FP8, 1)
 grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
-                             const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ TokenMaps tmB,
                              const int* __restrict__ offsets, const float* __restrict__ scales,
                              int E, int K, int a_rows_per_expert, int m_tiles,
                              __nv_bfloat16* __restrict__ out, int out_ld,
@@ -520,7 +570,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             c.total = carry;
             c.abort = 0;
             tc::prefetch_tensormap(&tmA);
-            tc::prefetch_tensormap(&tmB);
+            for (int m = 0; m < 4; ++m) tc::prefetch_tensormap(&tmB.m[m]);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -614,9 +664,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.b_full[stage]), 0);
                     if (leader) tc::mbar_arrive_expect_tx(&c.b_full[stage], pair_bytes);
                     uint8_t* st = b_ring + stage * BH_BYTES;
-                    for (int b = 0; b < nb; ++b)
-                        tc::tma_load_2d_pair(st + b * BOX_BYTES, &tmB, full_leader, kb * BK,
-                                             b_row + b * NBOX, pol_x);
+                    load_token_rows(st, tmB, full_leader, kb * BK, b_row, ti.n / 2, pol_x);
                     issued[stage] = true;
                     parity[stage] = phase;
                     if (++stage == S::B_STAGES) {
@@ -825,6 +873,12 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_token_maps(TokenMaps* tm, const void* base, uint64_t rows, uint64_t cols) {
+    for (int lg = 0; lg < 4; ++lg)
+        if (!make_map(&tm->m[lg], base, rows, cols, NBOX << lg)) return false;
+    return true;
+}
+
 int sm_pairs() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
@@ -832,12 +886,12 @@ int sm_pairs() {
     return (n > 1 ? n : 148) / 2;
 }
 
-template <bool GATE_UP>
-cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const int32_t* offsets, int E,
+template <bool GATE_UP, bool GATHER = false>
+cudaError_t launch(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets, int E,
                    int K, int a_rows_per_expert, int m_tiles, void* out, int out_ld, int* status,
-                   cudaStream_t s) {
+                   cudaStream_t s, const int32_t* token_of_row = nullptr) {
     const int smem = smem_bytes<GATE_UP>();
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATE_UP>,
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATE_UP, GATHER>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -852,15 +906,15 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const int32_t* of
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATE_UP>, a, b, offsets, E, K,
-                             a_rows_per_expert, m_tiles, static_cast<__nv_bfloat16*>(out), out_ld,
-                             status);
+    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATE_UP, GATHER>, a, b, offsets,
+                             token_of_row, E, K, a_rows_per_expert, m_tiles,
+                             static_cast<__nv_bfloat16*>(out), out_ld, status);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
 template <bool GATE_UP>
-cudaError_t launch_fp8(const CUtensorMap& a, const CUtensorMap& b, const int32_t* offsets,
+cudaError_t launch_fp8(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets,
                        const float* scales, int E, int K, int a_rows_per_expert, int m_tiles,
                        void* out, int out_ld, int* status, cudaStream_t s) {
     const int smem = fp8_smem_bytes<GATE_UP>();
@@ -894,10 +948,11 @@ cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm
                                          const int32_t* offsets, const void* w_gate_up,
                                          const float* s_gate_up, void* h, int* status,
                                          cudaStream_t s) {
-    CUtensorMap a, b;
+    CUtensorMap a;
+    TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
     if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM) ||
-        !make_map(&b, x_perm, R, c.d, NBOX))
+        !make_token_maps(&b, x_perm, R, c.d))
         return cudaErrorInvalidValue;
     return launch_fp8<true>(a, b, offsets, s_gate_up, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h,
                             c.d_ff, status, s);
@@ -906,10 +961,11 @@ cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm
 cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const int32_t* offsets,
                                       const void* w_down, const float* s_down, void* y,
                                       int* status, cudaStream_t s) {
-    CUtensorMap a, b;
+    CUtensorMap a;
+    TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
     if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM) ||
-        !make_map(&b, h, R, c.d_ff, NBOX))
+        !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
     return launch_fp8<false>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d,
                              status, s);
@@ -918,21 +974,36 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
 cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
                                      const int32_t* offsets, const void* w_gate_up, void* h,
                                      int* status, cudaStream_t s) {
-    CUtensorMap a, b;
+    CUtensorMap a;
+    TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
     if (!make_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM) ||
-        !make_map(&b, x_perm, R, c.d, NBOX))
+        !make_token_maps(&b, x_perm, R, c.d))
         return cudaErrorInvalidValue;
     return launch<true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h, c.d_ff, status,
                         s);
 }
 
+cudaError_t launch_gate_up_gemm_pair_gather(const moe_config& c, const void* x,
+                                            const int32_t* token_of_row, const int32_t* offsets,
+                                            const void* w_gate_up, void* h, int* status,
+                                            cudaStream_t s) {
+    CUtensorMap a;
+    TokenMaps b = {};
+    if (!make_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM) ||
+        !make_map(&b.m[0], x, (uint64_t)c.T, c.d, 1))
+        return cudaErrorInvalidValue;
+    return launch<true, true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h, c.d_ff,
+                              status, s, token_of_row);
+}
+
 cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int32_t* offsets,
                                   const void* w_down, void* y, int* status, cudaStream_t s) {
-    CUtensorMap a, b;
+    CUtensorMap a;
+    TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
     if (!make_map(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM) ||
-        !make_map(&b, h, R, c.d_ff, NBOX))
+        !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
     return launch<false>(a, b, offsets, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d, status, s);
 }

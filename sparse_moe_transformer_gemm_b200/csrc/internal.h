@@ -23,7 +23,7 @@ struct WsLayout {
     size_t status;    // int32 status word (+ padding)
     size_t counters;  // int32 [ceil(T / kRouterTokens)] router arrival counters
     size_t control_end;
-    size_t logits;    // fp32 [T, E]
+    size_t logits;    // fp32 [router_ksplit, T, E] partial router logits
     size_t hist;      // int32 [n_chunks, E]
     size_t rank;      // int32 [T*k]
     size_t idx;       // int32 [T*k]
@@ -31,6 +31,7 @@ struct WsLayout {
     size_t counts;    // int32 [E]
     size_t offsets;   // int32 [E+1]
     size_t row_of;    // int32 [T*k]
+    size_t tok;       // int32 [T*k] token of each grouped row
     size_t xperm;     // bf16 [T*k, d]
     size_t h;         // bf16 [T*k, d_ff]
     size_t y;         // bf16 [T*k, d]
@@ -40,6 +41,20 @@ struct WsLayout {
 
 inline int n_router_groups(const moe_config& c) {
     return (c.T + kRouterTokens - 1) / kRouterTokens;
+}
+constexpr int kRouterCtasPerSm = 2;     // CUDA-core router CTAs resident per SM
+constexpr int kRouterMaxSplit = 16;     // K slices of the CUDA-core router at most
+
+// K slices of the CUDA-core router: the largest power of two (at most
+// kRouterMaxSplit, keeping d / slices a multiple of 128) whose grid still runs
+// in one wave on 148 SMs.
+inline int router_ksplit(const moe_config& c) {
+    const int base = ((c.E + kRouterExperts - 1) / kRouterExperts) * n_router_groups(c);
+    int ks = 1;
+    while (2 * ks <= kRouterMaxSplit && base * 2 * ks <= kRouterCtasPerSm * 148 &&
+           (c.d / 128) % (2 * ks) == 0)
+        ks *= 2;
+    return ks;
 }
 inline int n_permute_chunks(const moe_config& c) {
     long R = (long)c.T * c.k;
@@ -53,7 +68,7 @@ inline WsLayout ws_layout(const moe_config& c) {
     L.status = o;   o += 256;
     L.counters = o; o = align256(o + sizeof(int32_t) * n_router_groups(c));
     L.control_end = o;
-    L.logits = o;   o = align256(o + sizeof(float) * (size_t)c.T * c.E);
+    L.logits = o;   o = align256(o + sizeof(float) * router_ksplit(c) * (size_t)c.T * c.E);
     L.hist = o;     o = align256(o + sizeof(int32_t) * (size_t)n_permute_chunks(c) * c.E);
     L.rank = o;     o = align256(o + sizeof(int32_t) * R);
     L.idx = o;      o = align256(o + sizeof(int32_t) * R);
@@ -61,6 +76,7 @@ inline WsLayout ws_layout(const moe_config& c) {
     L.counts = o;   o = align256(o + sizeof(int32_t) * c.E);
     L.offsets = o;  o = align256(o + sizeof(int32_t) * (c.E + 1));
     L.row_of = o;   o = align256(o + sizeof(int32_t) * R);
+    L.tok = o;      o = align256(o + sizeof(int32_t) * R);
     L.xperm = o;    o = align256(o + 2 * R * c.d);
     L.h = o;        o = align256(o + 2 * R * c.d_ff);
     L.y = o;        o = align256(o + 2 * R * c.d);
@@ -72,7 +88,7 @@ inline WsLayout ws_layout(const moe_config& c) {
 // ---- launchers (each returns cudaError_t of the launch) ----
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
                           const float* gate_bias, int32_t* idx, float* w, float* logits,
-                          int32_t* counters, cudaStream_t s);
+                          int32_t* counters, int ksplit, cudaStream_t s);
 
 bool router_tc_supported(const moe_config& c);
 cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_gate,
@@ -82,6 +98,12 @@ cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_g
 cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
                            int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,
                            int32_t* rank, cudaStream_t s);
+
+cudaError_t launch_permute_index(const moe_config& c, const int32_t* idx, int32_t* counts,
+                                 int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
+                                 int32_t* hist, int32_t* rank, cudaStream_t s);
+cudaError_t launch_gather_rows(const moe_config& c, const void* x, const int32_t* token_of_row,
+                               const int32_t* offsets, void* x_perm, cudaStream_t s);
 
 cudaError_t launch_gate_up_stream(const moe_config& c, const void* x_perm, const int32_t* offsets,
                                   const void* w_gate_up, const float* s_gate_up, void* h,
@@ -100,6 +122,10 @@ cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
                                      int* status, cudaStream_t s);
 cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int32_t* offsets,
                                   const void* w_down, void* y, int* status, cudaStream_t s);
+cudaError_t launch_gate_up_gemm_pair_gather(const moe_config& c, const void* x,
+                                            const int32_t* token_of_row, const int32_t* offsets,
+                                            const void* w_gate_up, void* h, int* status,
+                                            cudaStream_t s);
 
 cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm,
                                          const int32_t* offsets, const void* w_gate_up,

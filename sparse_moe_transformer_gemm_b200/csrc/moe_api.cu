@@ -69,14 +69,19 @@ bool use_stream_path(const moe_config* c) {
     return (c->flags & MOE_FLAG_FP8_WEIGHTS) != 0 && !pair_gemm_supported(*c);
 }
 
-// Router: tensor-core kernel where it applies (k <= 8), CUDA-core kernel otherwise.
+// Router: the tensor-core kernel where it applies (k <= 8) and the batch fills
+// more than one 128-token tile; small batches (decode) use the K-split CUDA-core
+// kernel, whose grid covers the SMs where the tensor-core one runs a handful
+// of CTAs.
+constexpr int kRouterTcMinTokens = 129;
+
 cudaError_t route(const moe_config* c, const void* x, const void* w_gate, const float* gate_bias,
                   int32_t* idx, float* w, void* ws, cudaStream_t s) {
     const WsLayout L = ws_layout(*c);
-    if (router_tc_supported(*c))
+    if (router_tc_supported(*c) && c->T >= kRouterTcMinTokens)
         return launch_router_tc(*c, x, w_gate, gate_bias, idx, w, at<int>(ws, L.status), s);
     return launch_router(*c, x, w_gate, gate_bias, idx, w, at<float>(ws, L.logits),
-                         at<int32_t>(ws, L.counters), s);
+                         at<int32_t>(ws, L.counters), router_ksplit(*c), s);
 }
 
 int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offsets,
@@ -93,6 +98,21 @@ int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offs
     if (pair_gemm_supported(*c))
         return cuda_status(launch_gate_up_gemm_pair(*c, x_perm, offsets, w_gate_up, h, status, s));
     return cuda_status(launch_gate_up_gemm(*c, x_perm, offsets, w_gate_up, h, status, s));
+}
+
+// gate_up on token rows gathered by index: the bf16 SM-pair GEMM gathers the
+// rows of x itself (TMA tile::gather4); every other path first gathers them
+// into the workspace's x_perm region with a copy kernel.
+int experts_gate_up_gather(const moe_config* c, const void* x, const int32_t* token_of_row,
+                           const int32_t* offsets, const void* w_gate_up, const float* s_gate_up,
+                           void* h, void* ws, cudaStream_t s) {
+    const WsLayout L = ws_layout(*c);
+    if (!use_stream_path(c) && !(c->flags & MOE_FLAG_FP8_WEIGHTS) && pair_gemm_supported(*c))
+        return cuda_status(launch_gate_up_gemm_pair_gather(*c, x, token_of_row, offsets, w_gate_up,
+                                                           h, at<int>(ws, L.status), s));
+    void* xperm = at<void>(ws, L.xperm);
+    MOE_TRY(cuda_status(launch_gather_rows(*c, x, token_of_row, offsets, xperm, s)));
+    return experts_gate_up(c, xperm, offsets, w_gate_up, s_gate_up, h, ws, s);
 }
 
 int experts_down(const moe_config* c, const void* h, const int32_t* offsets, const void* w_down,
@@ -147,6 +167,31 @@ int moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x, i
     return cuda_status(launch_permute(*cfg, topk_idx, x, counts, offsets, row_of, x_perm,
                                       at<int32_t>(ws, L.hist), at<int32_t>(ws, L.rank),
                                       static_cast<cudaStream_t>(stream)));
+}
+
+int moe_permute_index(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
+                      int32_t* offsets, int32_t* row_of, int32_t* token_of_row, void* ws,
+                      size_t ws_bytes, void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!topk_idx || !counts || !offsets || !row_of || !token_of_row) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    const WsLayout L = ws_layout(*cfg);
+    return cuda_status(launch_permute_index(*cfg, topk_idx, counts, offsets, row_of, token_of_row,
+                                            at<int32_t>(ws, L.hist), at<int32_t>(ws, L.rank),
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_gate_up_gather(const moe_config* cfg, const void* x, const int32_t* token_of_row,
+                              const int32_t* offsets, const void* w_gate_up,
+                              const float* s_gate_up, void* h, void* ws, size_t ws_bytes,
+                              void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (!x || !token_of_row || !offsets || !h || !aligned16(x) || !aligned16(h))
+        return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_expert_weights(cfg, w_gate_up, s_gate_up));
+    MOE_TRY(check_ws(cfg, ws, ws_bytes));
+    return experts_gate_up_gather(cfg, x, token_of_row, offsets, w_gate_up, s_gate_up, h, ws,
+                                  static_cast<cudaStream_t>(stream));
 }
 
 int moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
@@ -212,15 +257,24 @@ int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const 
     float* w = at<float>(ws, L.w);
     int32_t* offsets = at<int32_t>(ws, L.offsets);
     int32_t* row_of = at<int32_t>(ws, L.row_of);
-    void* xperm = at<void>(ws, L.xperm);
+    int32_t* counts = at<int32_t>(ws, L.counts);
+    int32_t* hist = at<int32_t>(ws, L.hist);
+    int32_t* rank = at<int32_t>(ws, L.rank);
     void* h = at<void>(ws, L.h);
     void* y = at<void>(ws, L.y);
     MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.control_end, s)));
     MOE_TRY(cuda_status(route(cfg, x, w_gate, gate_bias, idx, w, ws, s)));
-    MOE_TRY(cuda_status(launch_permute(*cfg, idx, x, at<int32_t>(ws, L.counts), offsets, row_of,
-                                       xperm, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.rank),
-                                       s)));
-    MOE_TRY(experts_gate_up(cfg, xperm, offsets, w_gate_up, s_gate_up, h, ws, s));
+    if ((long long)cfg->T * cfg->k <= MOE_GATHER_MAX_SLOTS) {
+        int32_t* tok = at<int32_t>(ws, L.tok);
+        MOE_TRY(cuda_status(
+            launch_permute_index(*cfg, idx, counts, offsets, row_of, tok, hist, rank, s)));
+        MOE_TRY(experts_gate_up_gather(cfg, x, tok, offsets, w_gate_up, s_gate_up, h, ws, s));
+    } else {
+        void* xperm = at<void>(ws, L.xperm);
+        MOE_TRY(cuda_status(
+            launch_permute(*cfg, idx, x, counts, offsets, row_of, xperm, hist, rank, s)));
+        MOE_TRY(experts_gate_up(cfg, xperm, offsets, w_gate_up, s_gate_up, h, ws, s));
+    }
     MOE_TRY(experts_down(cfg, h, offsets, w_down, s_down, y, ws, s));
     return cuda_status(launch_combine(*cfg, y, row_of, w, out, s));
 }

@@ -11,7 +11,7 @@
 // to row offsets[e] + #{s' < s : idx[s'] == e}; offsets is the exclusive prefix
 // sum of the per-expert counts.
 //
-// Three launches:
+// Three launches (moe_permute):
 //   rank    one warp per chunk of kPermuteChunk slots: rank of each slot among
 //           the earlier slots of its chunk with the same expert
 //           (__match_any_sync per 32-slot group + running per-expert counters
@@ -21,6 +21,12 @@
 //   scatter one warp per slot: row = offsets[e] + chunk base + rank; copies the
 //           token's d-element row into x_perm with 16-byte vectors.
 // Slots whose expert id is outside [0, E) are dropped: row_of = -1.
+//
+// moe_permute_index runs the same rank and scan and replaces the scatter by an
+// index-only one (thread per slot) that also writes token_of_row, the token of
+// each grouped row; the gate_up GEMM then gathers the token rows from x
+// itself and no permuted copy of the activations is written. Small batches
+// (at most 4096 slots) run all of it in one CTA.
 #include "common.cuh"
 #include "internal.h"
 
@@ -115,7 +121,155 @@ permute_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ hist
     for (int v = lane; v < d / 8; v += 32) dst[v] = src[v];
 }
 
+// Index-only scatter, one thread per slot: row_of and its inverse
+// token_of_row[row] = t, for expert GEMMs that gather the token rows
+// themselves.
+__global__ void __launch_bounds__(256)
+permute_index_kernel(const int* __restrict__ idx, const int* __restrict__ hist,
+                     const int* __restrict__ rank, const int* __restrict__ offsets, long R, int k,
+                     int E, int* __restrict__ row_of, int* __restrict__ token_of_row) {
+    const long s = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= R) return;
+    const int e = idx[s];
+    if (e < 0 || e >= E) {
+        row_of[s] = -1;
+        return;
+    }
+    const int row = offsets[e] + hist[(s / CH) * E + e] + rank[s];
+    row_of[s] = row;
+    token_of_row[row] = (int)(s / k);
+}
+
+// The whole index-only grouping in one CTA for small batches (R <= SW * 128
+// slots, decode): warp w owns the slots [w*per, (w+1)*per). Pass 1 counts each
+// warp's slots per expert; a scan over warps (per expert) and over experts
+// gives each warp's first row per expert; pass 2 ranks the slots again in the
+// same order and writes row_of and token_of_row. Same result as the
+// rank/scan/scatter launches.
+constexpr int SW = 32;  // warps of the small-batch kernel
+constexpr long kSmallSlots = SW * 128;
+
+__global__ void __launch_bounds__(SW * 32)
+permute_small_kernel(const int* __restrict__ idx, long R, int k, int E, int* __restrict__ counts,
+                     int* __restrict__ offsets, int* __restrict__ row_of,
+                     int* __restrict__ token_of_row) {
+    __shared__ int cnt[SW][256];
+    __shared__ int base[256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per = (int)(((R + SW - 1) / SW + 31) & ~31L);
+    for (int i = threadIdx.x; i < SW * 256; i += blockDim.x) cnt[i >> 8][i & 255] = 0;
+    __syncthreads();
+    const long s0 = (long)warp * per;
+    for (int g = 0; g < per; g += 32) {
+        const long s = s0 + g + lane;
+        int e = (s < R) ? idx[s] : -1;
+        if (e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // per expert: exclusive prefix over warps; totals into base[]
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int w = 0; w < SW; ++w) {
+            const int v = cnt[w][e];
+            cnt[w][e] = run;
+            run += v;
+        }
+        base[e] = run;
+        counts[e] = run;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // exclusive prefix over experts: lane handles experts [8*lane, 8*lane+8)
+        int v[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            v[i] = (e < E) ? base[e] : 0;
+            sum += v[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            if (e < E) {
+                base[e] = run;
+                offsets[e] = run;
+            }
+            run += v[i];
+        }
+        if (lane == 31) offsets[E] = incl;
+    }
+    __syncthreads();
+    for (int g = 0; g < per; g += 32) {
+        const long s = s0 + g + lane;
+        int e = (s < R) ? idx[s] : -1;
+        if (e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int before = (e >= 0) ? cnt[warp][e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] = before + __popc(peers);
+        __syncwarp();
+        if (s < R) {
+            if (e < 0) {
+                row_of[s] = -1;
+            } else {
+                const int row = base[e] + before + __popc(peers & ((1u << lane) - 1u));
+                row_of[s] = row;
+                token_of_row[row] = (int)(s / k);
+            }
+        }
+    }
+}
+
+// x_perm[row] = x[token_of_row[row]] for rows [0, offsets[E]): one warp per row.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ token_of_row,
+                   const int* __restrict__ offsets, long R, int E, int d,
+                   __nv_bfloat16* __restrict__ xperm) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long row = (long)blockIdx.x * 8 + warp;
+    if (row >= R || row >= offsets[E]) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (long)token_of_row[row] * d);
+    uint4* dst = reinterpret_cast<uint4*>(xperm + row * d);
+    for (int v = lane; v < d / 8; v += 32) dst[v] = src[v];
+}
+
 }  // namespace
+
+cudaError_t launch_permute_index(const moe_config& c, const int32_t* idx, int32_t* counts,
+                                 int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
+                                 int32_t* hist, int32_t* rank, cudaStream_t s) {
+    const long R = (long)c.T * c.k;
+    if (R <= kSmallSlots) {
+        permute_small_kernel<<<1, SW * 32, 0, s>>>(idx, R, c.k, c.E, counts, offsets, row_of,
+                                                   token_of_row);
+        return cudaGetLastError();
+    }
+    const int C = n_permute_chunks(c);
+    permute_rank_kernel<<<C, 32, 0, s>>>(idx, R, c.E, hist, rank);
+    permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, c.E, counts, offsets);
+    permute_index_kernel<<<(unsigned)((R + 255) / 256), 256, 0, s>>>(idx, hist, rank, offsets, R,
+                                                                     c.k, c.E, row_of, token_of_row);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const moe_config& c, const void* x, const int32_t* token_of_row,
+                               const int32_t* offsets, void* x_perm, cudaStream_t s) {
+    const long R = (long)c.T * c.k;
+    gather_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), token_of_row, offsets, R, c.E, c.d,
+        static_cast<__nv_bfloat16*>(x_perm));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
                            int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,

@@ -9,13 +9,15 @@
 // The optional per-expert bias is added to the logits before the sigmoid
 // (Hy3 commentary, wmrh.cn/news/24252, §3.3).
 //
-// Structure: CTA (expert block b, token group g) computes the logits of
-// kRouterTokens tokens x kRouterExperts experts on CUDA cores and writes them
-// to the fp32 scratch logits[T, E]. The last CTA of a token group to finish
-// (an arrival counter, no waiting) reads the group's complete logit rows and
-// runs the selection: one warp per token, k rounds of a warp-wide argmax over
-// the (biased) logits -- the sigmoid is increasing, so this selects the k
-// largest scores -- and the sigmoid of the k selected.
+// Structure: CTA (expert block b, token group g, K slice z) computes the
+// partial logits of kRouterTokens tokens x kRouterExperts experts over the
+// z-th of gridDim.z equal slices of d on CUDA cores and writes them to the fp32
+// scratch logits[z][T, E]. Small batches split K so that the grid covers the
+// SMs (decode: 64 tokens -> 48 CTAs unsplit, 384 with 8 slices). The last CTA
+// of a token group to finish (an arrival counter, no waiting) sums the slices
+// in z order and runs the selection: one warp per token, k rounds of a
+// warp-wide argmax over the (biased) logits -- the sigmoid is increasing, so
+// this selects the k largest scores -- and the sigmoid of the k selected.
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,7 +31,15 @@ constexpr int EPW = RE / RWARPS;     // experts per warp
 constexpr int KC = 1024;             // x columns staged per chunk
 static_assert(RT == RWARPS, "selection uses one warp per token");
 
-__global__ void __launch_bounds__(RWARPS * 32)
+__device__ __forceinline__ void load_w(uint4 (&u)[EPW], const __nv_bfloat16* __restrict__ wg,
+                                       int e_base, int E, int d, int col) {
+#pragma unroll
+    for (int a = 0; a < EPW; ++a)
+        u[a] = (e_base + a < E) ? *reinterpret_cast<const uint4*>(wg + (size_t)(e_base + a) * d + col)
+                                : make_uint4(0, 0, 0, 0);
+}
+
+__global__ void __launch_bounds__(RWARPS * 32, kRouterCtasPerSm)
 router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wg,
               const float* __restrict__ bias, int T, int d, int E, int k, float scale,
               float* __restrict__ logits, int* __restrict__ counters, int* __restrict__ idx_out,
@@ -39,6 +49,9 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e_base = blockIdx.x * RE + warp * EPW;
     const int t0 = blockIdx.y * RT;
+    const int ks = gridDim.z;
+    const int dk = d / ks;  // a multiple of 128
+    const int k0 = blockIdx.z * dk;
 
     float acc[EPW][RT];
 #pragma unroll
@@ -46,8 +59,8 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 #pragma unroll
         for (int b = 0; b < RT; ++b) acc[a][b] = 0.f;
 
-    for (int kc = 0; kc < d; kc += KC) {
-        const int kw = min(KC, d - kc);  // multiple of 128
+    for (int kc = k0; kc < k0 + dk; kc += KC) {
+        const int kw = min(KC, k0 + dk - kc);  // multiple of 128
         const int v8 = kw / 8;
         __syncthreads();
         for (int v = threadIdx.x; v < RT * v8; v += blockDim.x) {
@@ -64,19 +77,16 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
             *reinterpret_cast<float4*>(&xs[tt][c8 + 4]) = make_float4(f[4], f[5], f[6], f[7]);
         }
         __syncthreads();
+        // the weight vectors of the next column step are in flight while the
+        // current ones are used
+        uint4 cur[EPW];
+        load_w(cur, wg, e_base, E, d, kc + lane * 8);
         for (int c = lane * 8; c < kw; c += 256) {
+            uint4 nxt[EPW];
+            if (c + 256 < kw) load_w(nxt, wg, e_base, E, d, kc + c + 256);
             float wv[EPW][8];
 #pragma unroll
-            for (int a = 0; a < EPW; ++a) {
-                const int e = e_base + a;
-                if (e < E) {
-                    uint4 u = *reinterpret_cast<const uint4*>(wg + (size_t)e * d + kc + c);
-                    bf16x8_to_float(u, wv[a]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) wv[a][i] = 0.f;
-                }
-            }
+            for (int a = 0; a < EPW; ++a) bf16x8_to_float(cur[a], wv[a]);
 #pragma unroll
             for (int b = 0; b < RT; ++b) {
                 const float4 p = *reinterpret_cast<const float4*>(&xs[b][c]);
@@ -91,6 +101,8 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
                     acc[a][b] = s;
                 }
             }
+#pragma unroll
+            for (int a = 0; a < EPW; ++a) cur[a] = nxt[a];
         }
     }
 
@@ -104,7 +116,7 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 #pragma unroll
             for (int b = 0; b < RT; ++b) {
                 const int e = e_base + a, t = t0 + b;
-                if (e < E && t < T) logits[(size_t)t * E + e] = acc[a][b];
+                if (e < E && t < T) logits[((size_t)blockIdx.z * T + t) * E + e] = acc[a][b];
             }
     }
 
@@ -113,7 +125,7 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
     __syncthreads();
     if (threadIdx.x == 0) {
         const int ticket = atomicAdd(&counters[blockIdx.y], 1);
-        s_last = (ticket == (int)gridDim.x - 1);
+        s_last = (ticket == (int)(gridDim.x * gridDim.z) - 1);
     }
     __syncthreads();
     if (!s_last) return;
@@ -125,12 +137,23 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
         // sigmoid for the selected ones only.
         float sc[8];  // E <= 256: expert lane + 32*q
 #pragma unroll
+        for (int q = 0; q < 8; ++q) sc[q] = 0.f;
+        // slices summed in order 0, 1, ...; all loads of a slice are independent
+#pragma unroll
+        for (int p = 0; p < kRouterMaxSplit; ++p) {
+            if (p < ks) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int e = lane + 32 * q;
+                    if (e < E) sc[q] += __ldcg(logits + ((size_t)p * T + t) * E + e);
+                }
+            }
+        }
+#pragma unroll
         for (int q = 0; q < 8; ++q) {
             const int e = lane + 32 * q;
             if (e < E) {
-                float z = __ldcg(logits + (size_t)t * E + e);
-                if (bias) z += bias[e];
-                sc[q] = z;
+                if (bias) sc[q] += bias[e];
             } else {
                 sc[q] = -INFINITY;
             }
@@ -170,8 +193,8 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
                           const float* gate_bias, int32_t* idx, float* w, float* logits,
-                          int32_t* counters, cudaStream_t s) {
-    dim3 grid((c.E + RE - 1) / RE, n_router_groups(c));
+                          int32_t* counters, int ksplit, cudaStream_t s) {
+    dim3 grid((c.E + RE - 1) / RE, n_router_groups(c), ksplit);
     router_kernel<<<grid, RWARPS * 32, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_gate), gate_bias,
         c.T, c.d, c.E, c.k, c.scale, logits, counters, idx, w);

@@ -121,6 +121,11 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 // returns the OR of `pred` over them. Loops that wait on mbarriers use it so
 // that a thread whose bounded wait gave up still arrives and the group leaves
 // the loop together (a plain named barrier would wait for it forever).
+// Named barrier over `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ bool bar_any(int id, int count, bool pred) {
     uint32_t r;
     asm volatile(
@@ -286,6 +291,21 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
         ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1),
         "l"(policy)
+        : "memory");
+}
+
+// Four rows (indices r0..r3 of a 2-D map with a one-row box) of 64 columns
+// each, gathered into 4 consecutive 128-byte rows of this CTA's shared memory;
+// completion counted on an mbarrier of the even CTA of the pair.
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster_addr, int c0, int r0, int r1,
+                                                 int r2, int r3, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+        ".mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(r0), "r"(r1),
+        "r"(r2), "r"(r3), "l"(policy)
         : "memory");
 }
 

@@ -31,10 +31,14 @@ MOE_FLAG_STREAM_PATH = 0x2
 MOE_FLAG_GEMM_PATH = 0x4
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
-            "moe_expert_gate_up", "moe_expert_down", "moe_experts", "moe_combine", "moe_forward",
-            "moe_read_status", "moe_status_string", "moe_route_noalloc")
+            "moe_permute_index", "moe_expert_gate_up", "moe_expert_gate_up_gather",
+            "moe_expert_down", "moe_experts", "moe_combine", "moe_forward", "moe_read_status",
+            "moe_status_string", "moe_route_noalloc")
 
 MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
+# batches of at most this many token-slots (T*k) gather their token rows inside
+# the gate_up GEMM; larger ones write the permuted copy (moe_forward's rule)
+MOE_GATHER_MAX_SLOTS = 4096
 
 
 class MoeConfig(ctypes.Structure):
@@ -72,7 +76,9 @@ def lib() -> ctypes.CDLL:
         "moe_workspace_init": (I, [C, P, S, P]),
         "moe_route": (I, [C, P, P, P, P, P, P, S, P]),
         "moe_permute": (I, [C, P, P, P, P, P, P, P, S, P]),
+        "moe_permute_index": (I, [C, P, P, P, P, P, P, S, P]),
         "moe_expert_gate_up": (I, [C, P, P, P, P, P, P, S, P]),
+        "moe_expert_gate_up_gather": (I, [C, P, P, P, P, P, P, P, S, P]),
         "moe_expert_down": (I, [C, P, P, P, P, P, P, S, P]),
         "moe_experts": (I, [C, P, P, P, P, P, P, P, P, S, P]),
         "moe_combine": (I, [C, P, P, P, P, P, S, P]),
@@ -149,6 +155,21 @@ def moe_permute(cfg, topk_idx, x, counts, offsets, row_of, x_perm, ws, stream=No
     _check("moe_permute", lib().moe_permute(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(counts),
                                             _p(offsets), _p(row_of), _p(x_perm), _p(ws),
                                             ws.numel(), _s(stream)))
+
+
+def moe_permute_index(cfg, topk_idx, counts, offsets, row_of, token_of_row, ws,
+                      stream=None) -> None:
+    _check("moe_permute_index",
+           lib().moe_permute_index(ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(offsets),
+                                   _p(row_of), _p(token_of_row), _p(ws), ws.numel(), _s(stream)))
+
+
+def moe_expert_gate_up_gather(cfg, x, token_of_row, offsets, w_gate_up, s_gate_up, h, ws,
+                              stream=None) -> None:
+    _check("moe_expert_gate_up_gather",
+           lib().moe_expert_gate_up_gather(ctypes.byref(cfg), _p(x), _p(token_of_row),
+                                           _p(offsets), _p(w_gate_up), _p(s_gate_up), _p(h),
+                                           _p(ws), ws.numel(), _s(stream)))
 
 
 def moe_expert_gate_up(cfg, x_perm, offsets, w_gate_up, s_gate_up, h, ws, stream=None) -> None:

@@ -28,6 +28,14 @@ def test_header_declares_the_binding_surface():
     assert declared_functions() == sorted(moe.EXPORTED)
 
 
+def test_header_constants_match_the_binding():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    m = re.search(r"#define MOE_GATHER_MAX_SLOTS (\d+)", text)
+    assert m and int(m.group(1)) == moe.MOE_GATHER_MAX_SLOTS
+    m = re.search(r"#define MOE_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == moe.MOE_NOALLOC_SCRATCH_BYTES
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
@@ -126,6 +134,8 @@ def test_unsupported_shape_is_reported_by_every_entry_point(lib):
     cases = {
         "moe_route": (f, f, None, f, f, f, 1 << 30, None),
         "moe_permute": (f, f, f, f, f, f, f, 1 << 30, None),
+        "moe_permute_index": (f, f, f, f, f, f, 1 << 30, None),
+        "moe_expert_gate_up_gather": (f, f, f, f, None, f, f, 1 << 30, None),
         "moe_expert_gate_up": (f, f, f, None, f, f, 1 << 30, None),
         "moe_expert_down": (f, f, f, None, f, f, 1 << 30, None),
         "moe_experts": (f, f, f, None, f, None, f, f, 1 << 30, None),

@@ -34,6 +34,8 @@ SMALL = {
     # d and d_ff multiples of 256: the pair-of-SMs GEMMs (several tiles, ragged tokens)
     "pair_small": LayerShape(T=200, d=512, E=16, k=4, F=512),
     "pair_ragged": LayerShape(T=333, d=768, E=24, k=6, F=256, zipf_bias=True),
+    # fewer grouped rows (6) than the smallest token box (16 rows)
+    "pair_tiny": LayerShape(T=3, d=512, E=8, k=2, F=256),
     # the CUDA-core router (k > 8, or E not a multiple of 4)
     "k12": LayerShape(T=100, d=256, E=32, k=12, F=128),
     "e18": LayerShape(T=90, d=256, E=18, k=4, F=128),
@@ -95,6 +97,19 @@ def test_hy3_shapes(name):
     _free(layer, out)
 
 
+@pytest.mark.parametrize("T", [1, 7, 64, 128, 129, 300])
+def test_hy3_router_on_both_kernels(T):
+    """The Hy3 router shape (d=4096, E=192, k=8, zipf bias) at batch sizes on
+    both sides of the switch between the K-split CUDA-core router (T <= 128)
+    and the tensor-core one (T >= 129)."""
+    shape = dataclasses.replace(CONFIGS["decode"], T=T, zipf_bias=True)
+    layer = make_layer(shape, seed=T, device="cuda", with_experts=False)
+    route = parity.gpu_route(layer)
+    ref = oracle.route(oracle.bf16_bits(layer["x"]), oracle.bf16_bits(layer["w_gate"]), shape.k,
+                       shape.scale, layer["gate_bias"].cpu().numpy())
+    parity.check_route(*route, ref)
+
+
 @pytest.mark.parametrize("T,F", [(64, 128), (700, 128), (700, 256)])
 def test_all_tokens_to_the_same_experts(T, F):
     """A logit bias of +40 on experts 0..3 sends every token to them (T rows each,
@@ -135,6 +150,65 @@ def test_permute_is_bit_exact():
     rows = ref["row_of"].reshape(T, k)
     for j in range(k):
         assert np.array_equal(xpb[rows[:, j]], xb)
+
+
+@pytest.mark.parametrize("T,E", [(3000, 64), (512, 64), (500, 256), (1, 16)])
+def test_permute_index_is_bit_exact(T, E):
+    """moe_permute_index: the same grouping as moe_permute, plus token_of_row,
+    the inverse of row_of (token of each grouped row). At most 4096 slots run
+    the one-CTA kernel, more the rank/scan/scatter launches."""
+    shape = LayerShape(T=T, d=256, E=E, k=8, F=128)
+    layer = make_layer(shape, seed=3, device="cuda", with_experts=False)
+    cfg = moe.config_of(shape)
+    ws = moe.workspace(cfg)
+    T, k, E = shape.T, shape.k, shape.E
+    idx, _ = parity.gpu_route(layer)
+    idx_d = torch.from_numpy(idx).cuda()
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    tok = torch.full((T * k,), -1, dtype=torch.int32, device="cuda")
+    moe.moe_permute_index(cfg, idx_d, counts, offsets, row_of, tok, ws)
+    torch.cuda.synchronize()
+    ref = oracle.permute(idx, E)
+    assert np.array_equal(counts.cpu().numpy(), ref["counts"])
+    assert np.array_equal(offsets.cpu().numpy(), ref["offsets"])
+    assert np.array_equal(row_of.cpu().numpy(), ref["row_of"])
+    want = np.empty(T * k, dtype=np.int32)
+    want[ref["row_of"]] = np.arange(T * k) // k
+    assert np.array_equal(tok.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("name,path", [
+    ("pair_small", None), ("pair_ragged", None), ("pair_ragged", "gemm"), ("ragged", None),
+    ("tiny", "stream"), ("pair_fp8", None), ("single_token", None)])
+def test_gate_up_gather_equals_permuted_copy_bitwise(name, path):
+    """moe_expert_gate_up_gather (rows of x read by index inside the GEMM on the
+    bf16 SM-pair path, a row-gather kernel elsewhere) gives the same bits as
+    moe_permute + moe_expert_gate_up."""
+    shape = SMALL[name]
+    layer = make_layer(shape, seed=11, device="cuda")
+    cfg = moe.config_of(shape, path)
+    ws = moe.workspace(cfg)
+    T, k, E, d, F = shape.T, shape.k, shape.E, shape.d, shape.F
+    R = T * k
+    idx, _ = parity.gpu_route(layer)
+    idx_d = torch.from_numpy(idx).cuda()
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(R, dtype=torch.int32, device="cuda")
+    tok = torch.empty(R, dtype=torch.int32, device="cuda")
+    xp = torch.empty((R, d), dtype=torch.bfloat16, device="cuda")
+    h_copy = torch.empty((R, F), dtype=torch.bfloat16, device="cuda")
+    h_gather = torch.empty((R, F), dtype=torch.bfloat16, device="cuda")
+    wgu, sgu, _, _ = moe.layer_args(layer)
+    moe.moe_permute(cfg, idx_d, layer["x"], counts, offsets, row_of, xp, ws)
+    moe.moe_expert_gate_up(cfg, xp, offsets, wgu, sgu, h_copy, ws)
+    moe.moe_permute_index(cfg, idx_d, counts, offsets, row_of, tok, ws)
+    moe.moe_expert_gate_up_gather(cfg, layer["x"], tok, offsets, wgu, sgu, h_gather, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_status(ws) == moe.MOE_OK
+    assert torch.equal(h_copy, h_gather)
 
 
 def test_fp32_combine_keeps_small_terms():
