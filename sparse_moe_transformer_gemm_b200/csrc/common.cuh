@@ -65,4 +65,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __device__ __forceinline__ float sigmoidf_acc(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// SwiGLU's SiLU(g) * u with the fast exponential and division intrinsics: their
+// relative error (~1e-6) sits far below the bf16 rounding of the result
+// (2^-9), and for g below about -87 the quotient is 0, SiLU's limit.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
 }  // namespace moe

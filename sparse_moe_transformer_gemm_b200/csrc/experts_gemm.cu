@@ -360,7 +360,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         const int n = c0 + j;
                         if (n < ti.len) {
                             const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
-                            const float hv = gv / (1.f + expf(-gv)) * uv;
+                            const float hv = silu_mul(gv, uv);
                             o16[(size_t)(ti.row0 + n) * out_ld + col] = float_to_bf16_bits(hv);
                         }
                     }

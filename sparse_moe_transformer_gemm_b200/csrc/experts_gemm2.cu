@@ -14,10 +14,11 @@
 // pulls from L2 per K step and frees shared memory for a deeper weight ring
 // (more weight bytes in flight per SM, the bound of this HBM-bound stream).
 //
-// Per CTA (224 threads): warp 0 TMA producer (its weight rows + its token
+// Per CTA (320 threads): warp 0 TMA producer (its weight rows + its token
 // half; completion counted on the even CTA's "full" barrier, which expects the
 // bytes of both CTAs), warp 1 TMEM owner (+ MMA issuer in the even CTA), warps
-// 2-5 epilogue of the CTA's own 128 rows, warp 6 idle. Stage release and
+// 2-9 epilogue of the CTA's own 128 rows in two groups of four warps (one per
+// TMEM lane quarter) that take alternate 32-token chunks. Stage release and
 // accumulator hand-off are tcgen05.commit arrivals multicast to both CTAs; the
 // epilogues hand the accumulator back with one arrival per CTA on the even
 // CTA's barrier. No TMA load uses multicast. All waits are bounded.
@@ -38,10 +39,11 @@ constexpr int NBOX = 16;      // token rows per TMA box
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int BOX_BYTES = NBOX * BK * 2;
 constexpr int BH_BYTES = (NMAX / 2) * BK * 2;  // this CTA's half of the token rows
-constexpr int THREADS = 224;
+constexpr int EPI_GROUPS = 2;                      // epilogue warp groups (4 warps each)
+constexpr int THREADS = 64 + 128 * EPI_GROUPS;     // producer, MMA, epilogue warps
 constexpr int MAX_E = 256;
 constexpr int EPI_N = 32;                          // tokens per epilogue chunk
-constexpr int EPI_BYTES = 2 * EPI_N * BM * 2;      // double-buffered [EPI_N][BM] bf16 tile
+constexpr int EPI_BYTES = 2 * EPI_N * BM * 2;      // two [EPI_N][BM] bf16 staging tiles
 
 // Token-row tensor maps with boxes of 16, 32, 64 and 128 rows: a CTA's half of
 // a tile (a multiple of 16 rows, at most 128) loads as at most four boxes
@@ -323,14 +325,18 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             const int zero = 0;
             if (!tc::mbar_wait(&c.drain, 0, &zero)) atomicExch(status, MOE_ERR_TIMEOUT);
         }
-    } else if (warp >= 2 && warp <= 5) {
-        // ---------------- epilogue: this CTA's 128 weight rows (TMEM lanes). Per
-        // chunk of 32 tokens each warp writes its 32 rows x 32 tokens as bf16 into
-        // a shared [32 tokens][128 rows] tile (two buffers, alternating); after a
-        // named barrier the four warps store the tile as 256-byte row segments of
-        // the output with 16-byte vectors.
+    } else if (warp >= 2 && warp < 2 + 4 * EPI_GROUPS) {
+        // ---------------- epilogue: this CTA's 128 weight rows (TMEM lanes). Group
+        // g takes the 32-token chunks g, g + EPI_GROUPS, ...: each of its warps
+        // writes its 32 rows x 32 tokens as bf16 into the group's shared [32
+        // tokens][128 rows] tile, and after a named barrier the group stores the
+        // tile as 256-byte row segments of the output with 16-byte vectors.
+        // Named barriers: 1 + g within a group, 1 + EPI_GROUPS across all groups.
         const int quad = warp & 3;
-        const int et = threadIdx.x - 64;  // 0..127
+        const int grp = (warp - 2) >> 2;
+        const int et = threadIdx.x - 64 - 128 * grp;  // 0..127 within the group
+        const int bar_grp = 1 + grp, bar_all = 1 + EPI_GROUPS;
+        uint16_t* tile = epi + grp * (EPI_N * BM);
         uint16_t* o16 = reinterpret_cast<uint16_t*>(out);
         const bool arriver = (warp == 2 && lane == 0);
         int it = 0;
@@ -339,15 +345,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             const int acc = it % S::ACC_STAGES;
             const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
             const bool waited = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
-            if (tc::bar_any(1, 128, !waited)) {  // the four warps leave together
+            if (tc::bar_any(bar_all, 128 * EPI_GROUPS, !waited)) {  // all warps leave together
                 raise_timeout(c, status);
                 break;
             }
             tc::fence_after_sync();
             const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
             const int col0 = ti.m * 2 * BM + rank * BM;
-            for (int c0 = 0, buf = 0; c0 < ti.n; c0 += EPI_N, buf ^= 1) {
-                uint16_t* tile = epi + buf * (EPI_N * BM);
+            for (int c0 = grp * EPI_N; c0 < ti.n; c0 += EPI_GROUPS * EPI_N) {
                 uint32_t g[32];
                 tc::tmem_ld32(tbase + c0, g);
                 if constexpr (GATE_UP) {
@@ -357,7 +362,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
-                        tile[j * BM + quad * 32 + lane] = float_to_bf16_bits(gv / (1.f + expf(-gv)) * uv);
+                        tile[j * BM + quad * 32 + lane] = float_to_bf16_bits(silu_mul(gv, uv));
                     }
                 } else {
                     tc::tmem_ld_wait();
@@ -365,7 +370,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                     for (int j = 0; j < 32; ++j)
                         tile[j * BM + quad * 32 + lane] = float_to_bf16_bits(__uint_as_float(g[j]));
                 }
-                tc::bar_sync(1, 128);
+                tc::bar_sync(bar_grp, 128);  // the group's tile is written
 #pragma unroll
                 for (int q = 0; q < EPI_N * BM / 8 / 128; ++q) {
                     const int id = et + 128 * q;
@@ -375,10 +380,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                                   ch * 8) =
                             *reinterpret_cast<const uint4*>(tile + n * BM + ch * 8);
                 }
+                tc::bar_sync(bar_grp, 128);  // the group's tile is read
             }
             // every warp's TMEM reads are complete before the accumulator is handed back
             tc::fence_before_sync();
-            tc::bar_sync(1, 128);
+            tc::bar_sync(bar_all, 128 * EPI_GROUPS);
             if (arriver)
                 tc::mbar_arrive_cluster(tc::map_to_cta(tc::smem_u32(&c.acc_empty[acc]), 0));
         }
@@ -798,7 +804,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                         if (n < ti.len) {
                             const float gv = __uint_as_float(g[j]) * sa;
                             const float uv = __uint_as_float(u[j]) * sb;
-                            const float hv = gv / (1.f + expf(-gv)) * uv;
+                            const float hv = silu_mul(gv, uv);
                             o16[(size_t)(ti.row0 + n) * out_ld + col] = float_to_bf16_bits(hv);
                         }
                     }

@@ -97,7 +97,7 @@ __device__ void gate_up_rows(const uint8_t* __restrict__ wexp, const float* __re
         for (int t = 0; t < NT; ++t) {
             const float gt = warp_sum(g[t]) * sg, ut = warp_sum(u[t]) * su;
             if (lane == t) {
-                const float hv = gt / (1.f + expf(-gt)) * ut;
+                const float hv = silu_mul(gt, ut);
                 reinterpret_cast<uint16_t*>(h)[(row0 + t) * F + f] = float_to_bf16_bits(hv);
             }
         }
