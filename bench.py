@@ -46,10 +46,10 @@ WORKLOADS = {
 # the touched experts at decode, with the routed rows at prefill). An entry is
 # removed when its kernel changes.
 NCU_TRAFFIC = {
-    # profiles/grouped_gemm_pair_decode_E96_T32.md: 2.2454 GB for 89 touched experts
-    ("decode", "gate_up_gemm"): {"per": "touched_expert", "bytes": 2.2454e9 / 89},
-    # profiles/grouped_gemm_pair_prefill_E96_T2048.md: 2.6578 GB for 16384 routed rows
-    ("prefill", "gate_up_gemm"): {"per": "row", "bytes": 2.6578e9 / 16384},
+    # profiles/grouped_gemm_pair_decode_E96_T32.md: 2.2442 GB for 89 touched experts
+    ("decode", "gate_up_gemm"): {"per": "touched_expert", "bytes": 2.2442e9 / 89},
+    # profiles/grouped_gemm_pair_prefill_E96_T2048.md: 2.6391 GB for 16384 routed rows
+    ("prefill", "gate_up_gemm"): {"per": "row", "bytes": 2.6391e9 / 16384},
 }
 
 
@@ -363,33 +363,64 @@ def main():
     roof["algorithmic_bytes_per_launch"] = dom_work["bytes"]
     roof["algorithmic_flops_per_launch"] = dom_work["flops"]
 
-    # end to end through moe_forward: pinned host x in, pinned host out back, every step
+    # End to end through moe_forward: every step copies its input from pinned host
+    # memory and its output back to pinned host memory. The copies run on two
+    # more streams (one per direction, so both copy engines work at once),
+    # double-buffered, so that step i+1's input and step i-1's output cross PCIe
+    # while step i computes (a serving loop's pipelining); the timed region spans
+    # all copies and launches of the e2e_steps steps.
     x_host = x.cpu().pin_memory()
-    out_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
+    out_host = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    out_dev = [torch.empty((T, d), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    h2d_stream = torch.cuda.Stream(device=dev)
+    d2h_stream = torch.cuda.Stream(device=dev)
     e2e_steps = max(3, args.steps // 2)
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            x_dev.copy_(x_host, non_blocking=True)
-            moe.moe_forward(cfg, x_dev, wg, gb, wgu, sgu, wd, sd, out, ws, stream)
-            out_host.copy_(out, non_blocking=True)
+
+    def e2e_run(n):
+        fwd = [None, None]
+        d2h = [None, None]
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(h2d_stream):
+                if fwd[b] is not None:
+                    h2d_stream.wait_event(fwd[b])  # step i-2 has consumed x_dev[b]
+                x_dev[b].copy_(x_host, non_blocking=True)
+                h2d = torch.cuda.Event()
+                h2d.record(h2d_stream)
+            stream.wait_event(h2d)
+            if d2h[b] is not None:
+                stream.wait_event(d2h[b])  # step i-2's output has been read back
+            moe.moe_forward(cfg, x_dev[b], wg, gb, wgu, sgu, wd, sd, out_dev[b], ws, stream)
+            fwd[b] = torch.cuda.Event()
+            fwd[b].record(stream)
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(fwd[b])
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                d2h[b] = torch.cuda.Event()
+                d2h[b].record(d2h_stream)
+        for st in (h2d_stream, d2h_stream):
+            done = torch.cuda.Event()
+            done.record(st)
+            stream.wait_event(done)
+
+    e2e_run(args.warmup)
     stream.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            x_dev.copy_(x_host, non_blocking=True)
-            moe.moe_forward(cfg, x_dev, wg, gb, wgu, sgu, wd, sd, out, ws, stream)
-            out_host.copy_(out, non_blocking=True)
-        e1.record(stream)
+    e0.record(stream)
+    h2d_stream.wait_event(e0)
+    d2h_stream.wait_event(e0)
+    e2e_run(e2e_steps)
+    e1.record(stream)
     stream.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     e2e_ms = slowest_rank_ms(e2e_ms, pg, dev)
     status2 = moe.moe_read_status(ws, stream)
+    e2e_same = bool(torch.equal(out_host[(e2e_steps - 1) % 2], out.cpu()))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -419,7 +450,9 @@ def main():
             "clocks": clocks.summary(),
             "e2e": {"value": replica_value(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
-                    "ms_per_step": e2e_ms, "api": "moe_forward"},
+                    "ms_per_step": e2e_ms, "api": "moe_forward",
+                    "copies": "one stream per direction, double-buffered, overlapping the compute",
+                    "output_equals_staged": e2e_same},
             "gpu_launches": sum(n_launch.values()) * args.steps,
             "status": [moe.moe_status_string(status), moe.moe_status_string(status2)],
             "cpu_baseline": cpu,

@@ -65,6 +65,45 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __device__ __forceinline__ float sigmoidf_acc(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// Warp-collective top-k of one token's router scores. sc[q] holds the biased
+// logit of expert lane + 32 q (-INFINITY where that expert does not exist, so
+// E <= 256). k <= 32 rounds of a warp-wide argmax, ties to the lower expert
+// index; the sigmoid is increasing, so these are the k largest scores. Lane
+// j < k writes the j-th selection: idx_row[j] and
+// w_row[j] = scale * sigmoid_j / sum of the k sigmoids (summed in j order).
+__device__ __forceinline__ void warp_select_topk(float (&sc)[8], int k, float scale,
+                                                 int* __restrict__ idx_row,
+                                                 float* __restrict__ w_row) {
+    const int lane = threadIdx.x & 31;
+    int my_e = 0;
+    float my_s = 0.f;
+    for (int r = 0; r < k; ++r) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (sc[q] > bv) { bv = sc[q]; be = lane + 32 * q; }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+        }
+        if (lane == r) { my_e = be; my_s = sigmoidf_acc(bv); }
+        if ((be & 31) == lane) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if ((be >> 5) == q) sc[q] = -INFINITY;
+        }
+    }
+    float sum = 0.f;
+    for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, my_s, j);
+    if (lane < k) {
+        idx_row[lane] = my_e;
+        w_row[lane] = scale * my_s / sum;
+    }
+}
+
 // SwiGLU's SiLU(g) * u with the fast exponential and division intrinsics: their
 // relative error (~1e-6) sits far below the bf16 rounding of the result
 // (2^-9), and for g below about -87 the quotient is 0, SiLU's limit.

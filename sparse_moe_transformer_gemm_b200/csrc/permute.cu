@@ -12,10 +12,11 @@
 // sum of the per-expert counts.
 //
 // Three launches (moe_permute):
-//   rank    one warp per chunk of kPermuteChunk slots: rank of each slot among
-//           the earlier slots of its chunk with the same expert
-//           (__match_any_sync per 32-slot group + running per-expert counters
-//           in shared memory), and the chunk's per-expert histogram;
+//   rank    one CTA per chunk of kPermuteChunk slots, a warp per quarter of it:
+//           rank of each slot among the earlier slots of its chunk with the
+//           same expert (__match_any_sync per 32-slot group, running
+//           per-expert counters in shared memory, the earlier warps' counts
+//           added in a second pass), and the chunk's per-expert histogram;
 //   scan    one CTA: per expert, exclusive prefix over chunks (the chunk base),
 //           the totals (counts) and the exclusive prefix over experts (offsets);
 //   scatter one warp per slot: row = offsets[e] + chunk base + rank; copies the
@@ -35,27 +36,66 @@ namespace {
 
 constexpr int CH = kPermuteChunk;
 
-__global__ void __launch_bounds__(32)
+// One warp copies a row of n16 16-byte vectors, eight loads in flight per lane.
+__device__ __forceinline__ void copy_row(uint4* __restrict__ dst, const uint4* __restrict__ src,
+                                         int n16, int lane) {
+    for (int v0 = lane; v0 < n16; v0 += 32 * 8) {
+        uint4 u[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (v0 + 32 * i < n16) u[i] = src[v0 + 32 * i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (v0 + 32 * i < n16) dst[v0 + 32 * i] = u[i];
+    }
+}
+
+// Ranking: CTA per chunk of CH slots, RW warps on consecutive sub-chunks of
+// CH / RW slots. Each warp ranks its slots among its own earlier ones; the
+// per-expert counts of the warps are then prefix-summed so that a second pass
+// adds each warp's base.
+constexpr int RW = 4;
+constexpr int SUB = CH / RW;
+
+__global__ void __launch_bounds__(RW * 32)
 permute_rank_kernel(const int* __restrict__ idx, long R, int E, int* __restrict__ hist,
                     int* __restrict__ rank) {
-    __shared__ int cnt[256];
-    const int lane = threadIdx.x;
-    for (int e = lane; e < E; e += 32) cnt[e] = 0;
-    __syncwarp();
-    const long base = (long)blockIdx.x * CH;
-    for (int g = 0; g < CH; g += 32) {
+    __shared__ int cnt[RW][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < RW * 256; i += blockDim.x) cnt[i >> 8][i & 255] = 0;
+    __syncthreads();
+    const long base = (long)blockIdx.x * CH + (long)warp * SUB;
+    for (int g = 0; g < SUB; g += 32) {
         const long s = base + g + lane;
         int e = (s < R) ? idx[s] : -1;
         if (e >= E) e = -1;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int before = (e >= 0) ? cnt[e] : 0;
+        const int before = (e >= 0) ? cnt[warp][e] : 0;
         __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1) cnt[e] = before + __popc(peers);
+        if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] = before + __popc(peers);
         __syncwarp();
         if (s < R) rank[s] = before + __popc(peers & ((1u << lane) - 1u));
     }
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) hist[(long)blockIdx.x * E + e] = cnt[e];
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < RW; ++w) {
+            const int v = cnt[w][e];
+            cnt[w][e] = run;
+            run += v;
+        }
+        hist[(long)blockIdx.x * E + e] = run;
+    }
+    __syncthreads();
+    if (warp == 0) return;  // warp 0's base is 0 for every expert
+    for (int g = 0; g < SUB; g += 32) {
+        const long s = base + g + lane;
+        if (s < R) {
+            const int e = idx[s];
+            if (e >= 0 && e < E) rank[s] += cnt[warp][e];
+        }
+    }
 }
 
 __global__ void __launch_bounds__(256)
@@ -83,14 +123,28 @@ permute_scan_kernel(int* __restrict__ hist, int C, int E, int* __restrict__ coun
     }
     tot[e] = (e < E) ? running : 0;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int i = 0; i < E; ++i) {
-            const int v = tot[i];
-            tot[i] = acc;
-            acc += v;
+    if (threadIdx.x < 32) {
+        // exclusive prefix over the experts: lane handles experts [8*lane, 8*lane+8)
+        const int lane = threadIdx.x;
+        int v[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v[i] = tot[lane * 8 + i];
+            sum += v[i];
         }
-        offsets[E] = acc;
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            tot[lane * 8 + i] = run;
+            run += v[i];
+        }
+        if (lane == 31) offsets[E] = incl;
     }
     __syncthreads();
     if (e < E) {
@@ -118,7 +172,7 @@ permute_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ hist
     const long t = s / k;
     const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
     uint4* dst = reinterpret_cast<uint4*>(xperm + (long)row * d);
-    for (int v = lane; v < d / 8; v += 32) dst[v] = src[v];
+    copy_row(dst, src, d / 8, lane);
 }
 
 // Index-only scatter, one thread per slot: row_of and its inverse
@@ -240,7 +294,7 @@ gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ 
     if (row >= R || row >= offsets[E]) return;
     const uint4* src = reinterpret_cast<const uint4*>(x + (long)token_of_row[row] * d);
     uint4* dst = reinterpret_cast<uint4*>(xperm + row * d);
-    for (int v = lane; v < d / 8; v += 32) dst[v] = src[v];
+    copy_row(dst, src, d / 8, lane);
 }
 
 }  // namespace
@@ -255,7 +309,7 @@ cudaError_t launch_permute_index(const moe_config& c, const int32_t* idx, int32_
         return cudaGetLastError();
     }
     const int C = n_permute_chunks(c);
-    permute_rank_kernel<<<C, 32, 0, s>>>(idx, R, c.E, hist, rank);
+    permute_rank_kernel<<<C, RW * 32, 0, s>>>(idx, R, c.E, hist, rank);
     permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, c.E, counts, offsets);
     permute_index_kernel<<<(unsigned)((R + 255) / 256), 256, 0, s>>>(idx, hist, rank, offsets, R,
                                                                      c.k, c.E, row_of, token_of_row);
@@ -276,7 +330,7 @@ cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* 
                            int32_t* rank, cudaStream_t s) {
     const long R = (long)c.T * c.k;
     const int C = n_permute_chunks(c);
-    permute_rank_kernel<<<C, 32, 0, s>>>(idx, R, c.E, hist, rank);
+    permute_rank_kernel<<<C, RW * 32, 0, s>>>(idx, R, c.E, hist, rank);
     permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, c.E, counts, offsets);
     permute_scatter_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
         idx, hist, rank, offsets, static_cast<const __nv_bfloat16*>(x), R, c.k, c.E, c.d, row_of,

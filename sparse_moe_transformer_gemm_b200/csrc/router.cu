@@ -158,33 +158,7 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
                 sc[q] = -INFINITY;
             }
         }
-        int my_e = 0;
-        float my_s = 0.f;
-        for (int r = 0; r < k; ++r) {
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (sc[q] > bv) { bv = sc[q]; be = lane + 32 * q; }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-            }
-            if (lane == r) { my_e = be; my_s = sigmoidf_acc(bv); }
-            if ((be & 31) == lane) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    if ((be >> 5) == q) sc[q] = -INFINITY;
-            }
-        }
-        float sum = 0.f;
-        for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, my_s, j);
-        if (lane < k) {
-            idx_out[(size_t)t * k + lane] = my_e;
-            w_out[(size_t)t * k + lane] = scale * my_s / sum;
-        }
+        warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k);
     }
     if (threadIdx.x == 0) counters[blockIdx.y] = 0;
 }

@@ -11,12 +11,12 @@
 // is split over S in {1, 2, 4, 8} CTAs per token tile, launched as one thread-
 // block cluster. Each CTA moves its partial logits from TMEM to its own shared
 // memory; after a cluster barrier, CTA j sums rows [j*128/S, (j+1)*128/S) over
-// the S CTAs through distributed shared memory, in split order (the result
-// does not depend on timing), and selects for those rows: one thread per
-// token scans its E logits keeping a sorted top-k list. The sigmoid is
-// increasing, so the k largest (biased) logits are the k largest scores;
-// strictly greater enters, so an equal value never displaces a lower expert
-// index. The sigmoid is evaluated for the k selected only.
+// the S CTAs through distributed shared memory (16-byte loads, several in
+// flight per thread), in split order (the result does not depend on timing),
+// and selects for those rows (a thread per row where a CTA has 64 or more, a
+// warp per row otherwise), ties to the lower expert index. The sigmoid is
+// increasing, so the k largest (biased) logits are the k largest scores; it
+// is evaluated for the k selected only.
 //
 // CTA: 192 threads -- warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 2-5 epilogue / reduction / selection. Waits are bounded
@@ -52,17 +52,22 @@ struct Ctrl {
 };
 
 constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Ctrl);
-static_assert(BM * (256 + 1) * 4 <= STAGES * STAGE_BYTES, "logit rows fit in the stage ring");
+// Row stride (floats) of the logit rows in shared memory: a multiple of 4 (16-byte
+// rows) that is 4 mod 32, so a warp's 16-byte row stores take the minimum of
+// four wavefronts.
+__host__ __device__ constexpr int logit_stride(int E) { return ((E + 31) / 32) * 32 + 4; }
+static_assert(BM * logit_stride(256) * 4 <= STAGES * STAGE_BYTES, "logit rows fit in the ring");
 
-// Top-k of one token from its E logits (a shared-memory row), then the
-// renormalised, scaled weights. The sigmoid is strictly increasing, so the k
-// largest scores are the k largest (biased) logits; equal logits -- equal
-// scores -- keep the lower expert index because only a strictly greater value
-// enters the sorted list. The sigmoid is evaluated for the k selected only.
+// Top-k of one token by one thread, from its E logits (a shared-memory row):
+// a sorted list of the k largest (biased) logits where only a strictly greater
+// value enters, so equal values keep the lower expert index; then the sigmoid
+// of the k selected, renormalised (summed in list order) and scaled. Used
+// where a CTA selects for many rows (S <= 2), one thread per row.
 template <int K>
-__device__ __forceinline__ void select_topk(const float* row, const float* __restrict__ bias, int E,
-                                            float scale, int* __restrict__ idx_out,
-                                            float* __restrict__ w_out) {
+__device__ __forceinline__ void thread_select_topk(const float* row,
+                                                   const float* __restrict__ bias, int E,
+                                                   float scale, int* __restrict__ idx_out,
+                                                   float* __restrict__ w_out) {
     float v[K];
     int id[K];
 #pragma unroll
@@ -111,8 +116,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     const int split = (S > 1) ? (int)tc::cluster_ctarank() : 0;
     const int KB = d / BK;
     const int kb0 = split * KB / S, kb1 = (split + 1) * KB / S;  // S <= KB: never empty
-    const int es = E + 1;  // row stride of the logit rows in shared memory (odd: no bank conflicts)
-    float* red = reinterpret_cast<float*>(smem);  // [128][E+1], reuses the stage ring
+    const int es = logit_stride(E);
+    float* red = reinterpret_cast<float*>(smem);  // [128][es], reuses the stage ring
 
     if (warp == 0 && lane == 0) {
         c.abort = 0;
@@ -204,13 +209,15 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             tc::fence_after_sync();
             const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16);
             float* my = red + row * es;
-            for (int c0 = 0; c0 < n_pad; c0 += 32) {
+            for (int c0 = 0; c0 < n_pad; c0 += 32) {  // n_pad <= es - 4: inside the row
                 uint32_t r[32];
                 tc::tmem_ld32(tb + c0, r);
                 tc::tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (c0 + j < E) my[c0 + j] = __uint_as_float(r[j]);
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4*>(my + c0 + j) =
+                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                    __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
             }
         }
         tc::fence_before_sync();
@@ -220,49 +227,81 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     if constexpr (S > 1) {
         tc::cluster_sync();  // every CTA's partial rows are in its shared memory
         if (warp >= 2) {
+            // 16-byte vectors of this CTA's rows; U vectors (U*S loads) in flight
+            constexpr int U = S >= 8 ? 2 : 16 / S;
             const int etid = threadIdx.x - 64;
             const uint32_t red_addr = tc::smem_u32(red);
             uint32_t base[S];
 #pragma unroll
             for (int sp = 0; sp < S; ++sp) base[sp] = tc::map_to_cta(red_addr, sp);
-            const int n = ROWS * E;
-#pragma unroll 4
-            for (int i = etid; i < n; i += 128) {
-                const int r = split * ROWS + i / E, e = i - (i / E) * E;
-                const uint32_t off = (uint32_t)(r * es + e) * 4u;
-                float v[S];
+            const int v_row = (E + 3) / 4;
+            const int n = ROWS * v_row;
+            for (int i0 = etid; i0 < n; i0 += 128 * U) {
+                float4 v[U][S];
 #pragma unroll
-                for (int sp = 0; sp < S; ++sp) v[sp] = tc::ld_cluster_f32(base[sp] + off);
-                float z = v[0];
+                for (int u = 0; u < U; ++u) {
+                    const int i = i0 + 128 * u;
+                    if (i < n) {
+                        const int r = split * ROWS + i / v_row, e4 = i - (i / v_row) * v_row;
+                        const uint32_t off = (uint32_t)(r * es + 4 * e4) * 4u;
 #pragma unroll
-                for (int sp = 1; sp < S; ++sp) z += v[sp];
-                red[r * es + e] = z;  // rows of this CTA's slice: read by no other CTA
+                        for (int sp = 0; sp < S; ++sp) v[u][sp] = tc::ld_cluster_f32x4(base[sp] + off);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int i = i0 + 128 * u;
+                    if (i < n) {
+                        const int r = split * ROWS + i / v_row, e4 = i - (i / v_row) * v_row;
+                        float4 z = v[u][0];
+#pragma unroll
+                        for (int sp = 1; sp < S; ++sp) {
+                            z.x += v[u][sp].x; z.y += v[u][sp].y;
+                            z.z += v[u][sp].z; z.w += v[u][sp].w;
+                        }
+                        // rows of this CTA's slice: read by no other CTA
+                        *reinterpret_cast<float4*>(red + r * es + 4 * e4) = z;
+                    }
+                }
             }
         }
         tc::cluster_sync();  // all remote reads done before any CTA moves on or exits
     } else {
         __syncthreads();
     }
-    if (warp >= 2) {
-        const int etid = threadIdx.x - 64;
-        if (etid < ROWS) {
-            const int r = split * ROWS + etid;
-            const long t = (long)tile * BM + r;
-            if (t < T) {
-                const float* rw = red + r * es;
-                int* io = idx_out + t * k;
-                float* wo = w_out + t * k;
-                switch (k) {
-                    case 1: select_topk<1>(rw, bias, E, scale, io, wo); break;
-                    case 2: select_topk<2>(rw, bias, E, scale, io, wo); break;
-                    case 3: select_topk<3>(rw, bias, E, scale, io, wo); break;
-                    case 4: select_topk<4>(rw, bias, E, scale, io, wo); break;
-                    case 5: select_topk<5>(rw, bias, E, scale, io, wo); break;
-                    case 6: select_topk<6>(rw, bias, E, scale, io, wo); break;
-                    case 7: select_topk<7>(rw, bias, E, scale, io, wo); break;
-                    default: select_topk<8>(rw, bias, E, scale, io, wo); break;
-                }
+    if (warp >= 2 && ROWS >= 64) {
+        // one thread per token row of this CTA's slice
+        const int rr = threadIdx.x - 64;
+        const long t = (long)tile * BM + split * ROWS + rr;
+        if (rr < ROWS && t < T) {
+            const float* rw = red + (split * ROWS + rr) * es;
+            int* io = idx_out + t * k;
+            float* wo = w_out + t * k;
+            switch (k) {
+                case 1: thread_select_topk<1>(rw, bias, E, scale, io, wo); break;
+                case 2: thread_select_topk<2>(rw, bias, E, scale, io, wo); break;
+                case 3: thread_select_topk<3>(rw, bias, E, scale, io, wo); break;
+                case 4: thread_select_topk<4>(rw, bias, E, scale, io, wo); break;
+                case 5: thread_select_topk<5>(rw, bias, E, scale, io, wo); break;
+                case 6: thread_select_topk<6>(rw, bias, E, scale, io, wo); break;
+                case 7: thread_select_topk<7>(rw, bias, E, scale, io, wo); break;
+                default: thread_select_topk<8>(rw, bias, E, scale, io, wo); break;
             }
+        }
+    } else if (warp >= 2) {
+        // one warp per token row of this CTA's slice
+        for (int rr = warp - 2; rr < ROWS; rr += 4) {
+            const int r = split * ROWS + rr;
+            const long t = (long)tile * BM + r;
+            if (t >= T) break;
+            const float* rw = red + r * es;
+            float sc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = lane + 32 * q;
+                sc[q] = (e < E) ? rw[e] + (bias ? __ldg(bias + e) : 0.f) : -INFINITY;
+            }
+            warp_select_topk(sc, k, scale, idx_out + t * k, w_out + t * k);
         }
     }
 
