@@ -67,33 +67,43 @@ __device__ __forceinline__ float sigmoidf_acc(float z) { return 1.0f / (1.0f + e
 
 // Warp-collective top-k of one token's router scores. sc[q] holds the biased
 // logit of expert lane + 32 q (-INFINITY where that expert does not exist, so
-// E <= 256). k <= 32 rounds of a warp-wide argmax, ties to the lower expert
-// index; the sigmoid is increasing, so these are the k largest scores. Lane
+// E <= 256). k <= 32 rounds; each takes the warp maximum with one redux.sync
+// on an order-preserving unsigned key of the value and, among the lanes that
+// hold it, the lowest expert index with a second one (ties to the lower
+// index). The sigmoid is increasing, so these are the k largest scores. Lane
 // j < k writes the j-th selection: idx_row[j] and
 // w_row[j] = scale * sigmoid_j / sum of the k sigmoids (summed in j order).
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t b = __float_as_uint(f + 0.0f);  // -0 -> +0
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+}
+
 __device__ __forceinline__ void warp_select_topk(float (&sc)[8], int k, float scale,
                                                  int* __restrict__ idx_row,
                                                  float* __restrict__ w_row) {
     const int lane = threadIdx.x & 31;
+    uint32_t key[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) key[q] = order_key(sc[q]);  // removed entries get key 0
     int my_e = 0;
     float my_s = 0.f;
     for (int r = 0; r < k; ++r) {
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
+        uint32_t bk = key[0];
+        int bq = 0;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (sc[q] > bv) { bv = sc[q]; be = lane + 32 * q; }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-        }
-        if (lane == r) { my_e = be; my_s = sigmoidf_acc(bv); }
-        if ((be & 31) == lane) {
+        for (int q = 1; q < 8; ++q)
+            if (key[q] > bk) { bk = key[q]; bq = q; }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t be = __reduce_min_sync(0xffffffffu,
+                                              bk == m ? (uint32_t)(lane + 32 * bq) : 0xffffffffu);
+        if (lane == r) { my_e = (int)be; my_s = sigmoidf_acc(key_value(m)); }
+        if ((int)(be & 31u) == lane) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                if ((be >> 5) == q) sc[q] = -INFINITY;
+                if ((int)(be >> 5) == q) key[q] = 0u;
         }
     }
     float sum = 0.f;

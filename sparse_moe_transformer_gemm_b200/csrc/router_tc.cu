@@ -13,10 +13,9 @@
 // memory; after a cluster barrier, CTA j sums rows [j*128/S, (j+1)*128/S) over
 // the S CTAs through distributed shared memory (16-byte loads, several in
 // flight per thread), in split order (the result does not depend on timing),
-// and selects for those rows (a thread per row where a CTA has 64 or more, a
-// warp per row otherwise), ties to the lower expert index. The sigmoid is
-// increasing, so the k largest (biased) logits are the k largest scores; it
-// is evaluated for the k selected only.
+// and selects for those rows, one thread per row, ties to the lower expert
+// index. The sigmoid is increasing, so the k largest (biased) logits are the k
+// largest scores; it is evaluated for the k selected only.
 //
 // CTA: 192 threads -- warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 2-5 epilogue / reduction / selection. Waits are bounded
@@ -49,6 +48,8 @@ struct Ctrl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    // the logit bias (0 where none, and past E: the selection reads 8 at a time)
+    alignas(16) float bias[256 + 8];
 };
 
 constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Ctrl);
@@ -56,32 +57,48 @@ constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Ctrl);
 // rows) that is 4 mod 32, so a warp's 16-byte row stores take the minimum of
 // four wavefronts.
 __host__ __device__ constexpr int logit_stride(int E) { return ((E + 31) / 32) * 32 + 4; }
-static_assert(BM * logit_stride(256) * 4 <= STAGES * STAGE_BYTES, "logit rows fit in the ring");
+// (the selection reads up to 7 floats past a row's E logits; the ring has room)
+static_assert(BM * logit_stride(256) * 4 + 32 <= STAGES * STAGE_BYTES, "logit rows fit in the ring");
 
-// Top-k of one token by one thread, from its E logits (a shared-memory row):
-// a sorted list of the k largest (biased) logits where only a strictly greater
-// value enters, so equal values keep the lower expert index; then the sigmoid
-// of the k selected, renormalised (summed in list order) and scaled. Used
-// where a CTA selects for many rows (S <= 2), one thread per row.
+// Top-k of one token by one thread, from its E logits (a shared-memory row,
+// 16-byte aligned, read as float4: with a row stride of 4 mod 32 floats the
+// 16-byte reads of a warp's rows take the minimum number of wavefronts): a
+// sorted list of the k largest (biased) logits where only a strictly greater
+// value enters, so equal values keep the lower expert index (experts are
+// visited in increasing order); then the sigmoid of the k selected,
+// renormalised (summed in list order) and scaled. A warp per token (k rounds
+// of a warp-wide argmax, one token at a time per warp) measured ~3 us per
+// token here, far slower than this scan; the bias is staged in shared memory
+// (per-element global loads of it made the scan ~3x slower).
 template <int K>
-__device__ __forceinline__ void thread_select_topk(const float* row,
-                                                   const float* __restrict__ bias, int E,
+__device__ __forceinline__ void thread_select_topk(const float* row, const float* sbias, int E,
                                                    float scale, int* __restrict__ idx_out,
                                                    float* __restrict__ w_out) {
     float v[K];
     int id[K];
 #pragma unroll
     for (int j = 0; j < K; ++j) { v[j] = -INFINITY; id[j] = 0; }
-    for (int e = 0; e < E; ++e) {
-        const float z = bias ? row[e] + __ldg(bias + e) : row[e];
-        if (z > v[K - 1]) {
-            v[K - 1] = z;
-            id[K - 1] = e;
+    for (int e0 = 0; e0 < E; e0 += 8) {
+        // 8 logits and their biases in flight, then visited in increasing order
+        const float4 a0 = *reinterpret_cast<const float4*>(row + e0);
+        const float4 a1 = *reinterpret_cast<const float4*>(row + e0 + 4);
+        const float4 b0 = *reinterpret_cast<const float4*>(sbias + e0);
+        const float4 b1 = *reinterpret_cast<const float4*>(sbias + e0 + 4);
+        const float z8[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
+                             a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
 #pragma unroll
-            for (int j = K - 1; j > 0; --j) {
-                if (v[j] > v[j - 1]) {
-                    const float tv = v[j]; v[j] = v[j - 1]; v[j - 1] = tv;
-                    const int ti = id[j]; id[j] = id[j - 1]; id[j - 1] = ti;
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u;
+            const float z = z8[u];
+            if (e < E && z > v[K - 1]) {
+                v[K - 1] = z;
+                id[K - 1] = e;
+#pragma unroll
+                for (int j = K - 1; j > 0; --j) {
+                    if (v[j] > v[j - 1]) {
+                        const float tv = v[j]; v[j] = v[j - 1]; v[j - 1] = tv;
+                        const int ti = id[j]; id[j] = id[j - 1]; id[j - 1] = ti;
+                    }
                 }
             }
         }
@@ -119,6 +136,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     const int es = logit_stride(E);
     float* red = reinterpret_cast<float*>(smem);  // [128][es], reuses the stage ring
 
+    if (warp >= 2) {
+        for (int e = threadIdx.x - 64; e < 256 + 8; e += 128)
+            c.bias[e] = (bias && e < E) ? bias[e] : 0.f;
+    }
     if (warp == 0 && lane == 0) {
         c.abort = 0;
         tc::prefetch_tensormap(&tmX);
@@ -269,7 +290,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     } else {
         __syncthreads();
     }
-    if (warp >= 2 && ROWS >= 64) {
+    if (warp >= 2) {
         // one thread per token row of this CTA's slice
         const int rr = threadIdx.x - 64;
         const long t = (long)tile * BM + split * ROWS + rr;
@@ -278,30 +299,15 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             int* io = idx_out + t * k;
             float* wo = w_out + t * k;
             switch (k) {
-                case 1: thread_select_topk<1>(rw, bias, E, scale, io, wo); break;
-                case 2: thread_select_topk<2>(rw, bias, E, scale, io, wo); break;
-                case 3: thread_select_topk<3>(rw, bias, E, scale, io, wo); break;
-                case 4: thread_select_topk<4>(rw, bias, E, scale, io, wo); break;
-                case 5: thread_select_topk<5>(rw, bias, E, scale, io, wo); break;
-                case 6: thread_select_topk<6>(rw, bias, E, scale, io, wo); break;
-                case 7: thread_select_topk<7>(rw, bias, E, scale, io, wo); break;
-                default: thread_select_topk<8>(rw, bias, E, scale, io, wo); break;
+                case 1: thread_select_topk<1>(rw, c.bias, E, scale, io, wo); break;
+                case 2: thread_select_topk<2>(rw, c.bias, E, scale, io, wo); break;
+                case 3: thread_select_topk<3>(rw, c.bias, E, scale, io, wo); break;
+                case 4: thread_select_topk<4>(rw, c.bias, E, scale, io, wo); break;
+                case 5: thread_select_topk<5>(rw, c.bias, E, scale, io, wo); break;
+                case 6: thread_select_topk<6>(rw, c.bias, E, scale, io, wo); break;
+                case 7: thread_select_topk<7>(rw, c.bias, E, scale, io, wo); break;
+                default: thread_select_topk<8>(rw, c.bias, E, scale, io, wo); break;
             }
-        }
-    } else if (warp >= 2) {
-        // one warp per token row of this CTA's slice
-        for (int rr = warp - 2; rr < ROWS; rr += 4) {
-            const int r = split * ROWS + rr;
-            const long t = (long)tile * BM + r;
-            if (t >= T) break;
-            const float* rw = red + r * es;
-            float sc[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int e = lane + 32 * q;
-                sc[q] = (e < E) ? rw[e] + (bias ? __ldg(bias + e) : 0.f) : -INFINITY;
-            }
-            warp_select_topk(sc, k, scale, idx_out + t * k, w_out + t * k);
         }
     }
 
