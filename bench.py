@@ -46,10 +46,10 @@ WORKLOADS = {
 # the touched experts at decode, with the routed rows at prefill). An entry is
 # removed when its kernel changes.
 NCU_TRAFFIC = {
-    # profiles/grouped_gemm_pair_decode_E96_T32.md: 2.2442 GB for 89 touched experts
-    ("decode", "gate_up_gemm"): {"per": "touched_expert", "bytes": 2.2442e9 / 89},
-    # profiles/grouped_gemm_pair_prefill_E96_T2048.md: 2.6391 GB for 16384 routed rows
-    ("prefill", "gate_up_gemm"): {"per": "row", "bytes": 2.6391e9 / 16384},
+    # profiles/grouped_gemm_pair_decode_E96_T32.md: 2.2437 GB for 89 touched experts
+    ("decode", "gate_up_gemm"): {"per": "touched_expert", "bytes": 2.2437e9 / 89},
+    # profiles/grouped_gemm_pair_prefill_E96_T2048.md: 2.5880 GB for 16384 routed rows
+    ("prefill", "gate_up_gemm"): {"per": "row", "bytes": 2.5880e9 / 16384},
 }
 
 
@@ -250,12 +250,18 @@ def main():
 
         shape = dataclasses.replace(shape, E=args.experts or shape.E, T=args.tokens or shape.T)
     layer = make_layer(shape, seed=rank, device=dev)
-    cfg = moe.config_of(shape, None if args.path == "auto" else args.path)
     T, d, E, k, F = shape.T, shape.d, shape.E, shape.k, shape.F
+    # bf16 weights on the tensor-core pair kernels are packed once, at load time
+    # (moe_pack_weights), outside every timed region
+    packed = not shape.fp8 and args.path != "stream" and d % 256 == 0 and F % 256 == 0
+    cfg = moe.config_of(shape, None if args.path == "auto" else args.path, packed=packed)
     R = T * k
     ws = moe.workspace(cfg, device=dev)
     stream = torch.cuda.Stream(device=dev)
     wgu, sgu, wd, sd = moe.layer_args(layer)
+    if packed:
+        wgu, wd = moe.pack_layer_weights(cfg, wgu, wd)
+        torch.cuda.synchronize(dev)
     x, wg, gb = layer["x"], layer["w_gate"], layer["gate_bias"]
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
@@ -437,6 +443,9 @@ def main():
             "config": {"workload": WORKLOADS[args.config] if shape == CONFIGS[args.config] else
                        f"smaller case of {args.config}: T={T}, E={E}", "T": T, "d": d, "E": E, "k": k,
                        "d_ff": F, "path": args.path, "parallelism": f"replicas x{world}",
+                       "weights": ("e4m3 + fp32 row scales" if fp8 else
+                                   "bf16, packed in 128x64 blocks once at load (moe_pack_weights)"
+                                   if packed else "bf16, row-major"),
                        "l2": "no flush: each step streams the touched experts' weights "
                              f"({touched} experts, {touched * work.expert_bytes(d, F, fp8) / 1e9:.2f} GB) "
                              "through the 126 MB L2"},

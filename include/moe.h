@@ -25,6 +25,16 @@
  *   (one byte each) in the same layouts, and s_gate_up [E, 2*d_ff] /
  *   s_down [E, d] hold fp32 per-output-row scales; the weight value is
  *   code * scale. Without the flag both scale pointers must be NULL.
+ * - Packed bf16 weights (MOE_FLAG_PACKED_WEIGHTS): w_gate_up and w_down hold
+ *   the same values rearranged by moe_pack_weights into 16 KB blocks of 128
+ *   rows x 64 columns (block (e, rb, kb) = rows [128 rb, 128 rb + 128) and
+ *   columns [64 kb, 64 kb + 64) of expert e, row-major inside the block;
+ *   blocks ordered by e, then rb, then kb), so that every weight tile the
+ *   tensor-core kernels load is one contiguous span of memory (measured on
+ *   B200: gate_up 4-6% faster). Needs bf16 weights, d and d_ff multiples of
+ *   256 and the tensor-core path: with MOE_FLAG_FP8_WEIGHTS or
+ *   MOE_FLAG_STREAM_PATH it is MOE_ERR_INVALID_ARG, with other shapes
+ *   MOE_ERR_UNSUPPORTED_SHAPE.
  * - Grouping ("permuted rows"): token-slot s = t*k + j goes to row
  *   row_of[s] = offsets[e] + (number of earlier slots s' < s with the same
  *   expert e = topk_idx[s]); offsets[e] = sum_{e' < e} counts[e'],
@@ -72,6 +82,11 @@ extern "C" {
 #define MOE_FLAG_FP8_WEIGHTS 0x1u /* expert weights are e4m3 codes + fp32 row scales */
 #define MOE_FLAG_STREAM_PATH 0x2u /* experts on the weight-streaming (decode) kernels */
 #define MOE_FLAG_GEMM_PATH 0x4u   /* experts on the tensor-core grouped GEMMs */
+#define MOE_FLAG_PACKED_WEIGHTS 0x8u /* bf16 expert weights in moe_pack_weights' layout */
+
+/* Which expert weight moe_pack_weights rearranges. */
+#define MOE_WEIGHTS_GATE_UP 0 /* w_gate_up [E, 2*d_ff, d] */
+#define MOE_WEIGHTS_DOWN 1    /* w_down [E, d, d_ff] */
 /* With neither path flag the library picks by the mean rows per expert T*k/E. */
 
 typedef struct moe_config {
@@ -173,6 +188,18 @@ MOE_API int moe_combine(const moe_config* cfg, const void* y, const int32_t* row
 MOE_API int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
                 const void* w_gate_up, const float* s_gate_up, const void* w_down,
                 const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Rearrange one bf16 expert weight (which = MOE_WEIGHTS_GATE_UP or
+ * MOE_WEIGHTS_DOWN, row-major as above) into the packed layout described
+ * under MOE_FLAG_PACKED_WEIGHTS: w_packed has the same size and must not
+ * overlap w. A pure permutation of the values (bit-exact), done once when
+ * the weights are loaded; the layer's mathematics is unchanged. cfg->flags
+ * may carry MOE_FLAG_PACKED_WEIGHTS or not; d and d_ff must be multiples of
+ * 256 (else MOE_ERR_UNSUPPORTED_SHAPE) and the FP8 flag must be clear. This
+ * storage form is not in the pages; it serves the tensor-core kernels'
+ * tile loads. */
+MOE_API int moe_pack_weights(const moe_config* cfg, int which, const void* w, void* w_packed,
+                     void* stream);
 
 /* Bytes of the fixed device array behind moe_route_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES (2u << 20)

@@ -126,7 +126,8 @@ __device__ __forceinline__ void raise_timeout(CtrlT& c, int* status) {
     atomicExch(status, MOE_ERR_TIMEOUT);
 }
 
-// tmA: weights [E * a_rows_per_expert, K] bf16, box 64 x 128.
+// tmA: weights [E * a_rows_per_expert, K] bf16, box 64 x 128; with packed_a the
+// same bytes in 128 x 64 blocks, viewed as [E * a_rows_per_expert * K / 64, 64].
 // tmB: token rows [R, K] bf16, boxes of 64 columns x 16/32/64/128 rows.
 // m_tiles: 256-row weight tiles per expert (F/256 for gate_up, d/256 for down).
 // GATHER: tmB maps the unpermuted token rows x [T, K] with a one-row box and
@@ -137,8 +138,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ TokenMaps tmB, const int* __restrict__ offsets,
                          const int* __restrict__ token_of_row, int E, int K,
-                         int a_rows_per_expert, int m_tiles, __nv_bfloat16* __restrict__ out,
-                         int out_ld, int* __restrict__ status) {
+                         int a_rows_per_expert, int m_tiles, int packed_a,
+                         __nv_bfloat16* __restrict__ out, int out_ld, int* __restrict__ status) {
     using S = Shape<GATE_UP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -246,10 +247,20 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                 uint8_t* sb = s + S::A_TILES * A_BYTES;
                 if (lane == 0) {
                     if (leader) tc::mbar_arrive_expect_tx(&c.full[stage], pair_bytes);
-                    tc::tma_load_2d_pair(s, &tmA, full_leader, kb * BK, a_row, pol_w);
-                    if (GATE_UP)
-                        tc::tma_load_2d_pair(s + A_BYTES, &tmA, full_leader, kb * BK,
-                                             a_row + a_rows_per_expert / 2, pol_w);
+                    if (packed_a) {
+                        // 128 x 64 blocks stored contiguously: block (row / 128, kb)
+                        tc::tma_load_2d_pair(s, &tmA, full_leader, 0, ((a_row / BM) * KB + kb) * BM,
+                                             pol_w);
+                        if (GATE_UP)
+                            tc::tma_load_2d_pair(
+                                s + A_BYTES, &tmA, full_leader, 0,
+                                (((a_row + a_rows_per_expert / 2) / BM) * KB + kb) * BM, pol_w);
+                    } else {
+                        tc::tma_load_2d_pair(s, &tmA, full_leader, kb * BK, a_row, pol_w);
+                        if (GATE_UP)
+                            tc::tma_load_2d_pair(s + A_BYTES, &tmA, full_leader, kb * BK,
+                                                 a_row + a_rows_per_expert / 2, pol_w);
+                    }
                     if (!GATHER)
                         load_token_rows(sb, tmB, full_leader, kb * BK, b_row, half, pol_x);
                     issued[stage] = true;
@@ -879,6 +890,14 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Expert weights [rows_total, cols] bf16, box 64 x 128; packed: the same bytes as
+// [rows_total * cols / 64, 64] (128 x 64 blocks).
+bool make_weight_map(CUtensorMap* m, const void* w, uint64_t rows_total, uint64_t cols,
+                     bool packed) {
+    return packed ? make_map(m, w, rows_total * (cols / BK), BK, BM)
+                  : make_map(m, w, rows_total, cols, BM);
+}
+
 bool make_token_maps(TokenMaps* tm, const void* base, uint64_t rows, uint64_t cols) {
     for (int lg = 0; lg < 4; ++lg)
         if (!make_map(&tm->m[lg], base, rows, cols, NBOX << lg)) return false;
@@ -894,8 +913,9 @@ int sm_pairs() {
 
 template <bool GATE_UP, bool GATHER = false>
 cudaError_t launch(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets, int E,
-                   int K, int a_rows_per_expert, int m_tiles, void* out, int out_ld, int* status,
-                   cudaStream_t s, const int32_t* token_of_row = nullptr) {
+                   int K, int a_rows_per_expert, int m_tiles, bool packed_a, void* out,
+                   int out_ld, int* status, cudaStream_t s,
+                   const int32_t* token_of_row = nullptr) {
     const int smem = smem_bytes<GATE_UP>();
     cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATE_UP, GATHER>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -913,7 +933,7 @@ cudaError_t launch(const CUtensorMap& a, const TokenMaps& b, const int32_t* offs
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATE_UP, GATHER>, a, b, offsets,
-                             token_of_row, E, K, a_rows_per_expert, m_tiles,
+                             token_of_row, E, K, a_rows_per_expert, m_tiles, (int)packed_a,
                              static_cast<__nv_bfloat16*>(out), out_ld, status);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
@@ -978,40 +998,71 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
 }
 
 cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
-                                     const int32_t* offsets, const void* w_gate_up, void* h,
-                                     int* status, cudaStream_t s) {
+                                     const int32_t* offsets, const void* w_gate_up, bool packed,
+                                     void* h, int* status, cudaStream_t s) {
     CUtensorMap a;
     TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
-    if (!make_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM) ||
+    if (!make_weight_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, packed) ||
         !make_token_maps(&b, x_perm, R, c.d))
         return cudaErrorInvalidValue;
-    return launch<true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h, c.d_ff, status,
-                        s);
+    return launch<true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), packed, h, c.d_ff,
+                        status, s);
 }
 
 cudaError_t launch_gate_up_gemm_pair_gather(const moe_config& c, const void* x,
                                             const int32_t* token_of_row, const int32_t* offsets,
-                                            const void* w_gate_up, void* h, int* status,
-                                            cudaStream_t s) {
+                                            const void* w_gate_up, bool packed, void* h,
+                                            int* status, cudaStream_t s) {
     CUtensorMap a;
     TokenMaps b = {};
-    if (!make_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM) ||
+    if (!make_weight_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, packed) ||
         !make_map(&b.m[0], x, (uint64_t)c.T, c.d, 1))
         return cudaErrorInvalidValue;
-    return launch<true, true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h, c.d_ff,
-                              status, s, token_of_row);
+    return launch<true, true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), packed, h,
+                              c.d_ff, status, s, token_of_row);
 }
 
 cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int32_t* offsets,
-                                  const void* w_down, void* y, int* status, cudaStream_t s) {
+                                  const void* w_down, bool packed, void* y, int* status,
+                                  cudaStream_t s) {
     CUtensorMap a;
     TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
-    if (!make_map(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM) ||
+    if (!make_weight_map(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, packed) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
-    return launch<false>(a, b, offsets, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d, status, s);
+    return launch<false>(a, b, offsets, c.E, c.d_ff, c.d, c.d / (2 * BM), packed, y, c.d, status,
+                         s);
+}
+
+namespace {
+
+// Packed block layout: 16-byte chunk i of the output is chunk i % 8 of row
+// (i / 8) % 128 of block i / 1024; block b holds rows [128 (b / KB), +128) and
+// columns [64 (b % KB), +64) of the [E * rows, cols] source (KB = cols / 64).
+__global__ void __launch_bounds__(256)
+pack_weights_kernel(const uint4* __restrict__ w, uint4* __restrict__ wp, long n16, int cols) {
+    const int kbs = cols / BK;
+    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
+         i += (long)gridDim.x * blockDim.x) {
+        const long b = i >> 10;
+        const int r = (int)((i >> 3) & 127), ch = (int)(i & 7);
+        const long row = (b / kbs) * BM + r;
+        const long col = (b % kbs) * BK + ch * 8;
+        wp[i] = w[(row * cols + col) / 8];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_weights(int E, int rows, int cols, const void* w, void* w_packed,
+                                cudaStream_t s) {
+    const long n16 = (long)E * rows * cols / 8;
+    const long blocks = (n16 + 255) / 256;
+    pack_weights_kernel<<<(unsigned)(blocks < 148L * 64 ? blocks : 148L * 64), 256, 0, s>>>(
+        static_cast<const uint4*>(w), static_cast<uint4*>(w_packed), n16, cols);
+    return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -118,14 +118,18 @@ cudaError_t launch_down_gemm(const moe_config& c, const void* h, const int32_t* 
 
 bool pair_gemm_supported(const moe_config& c);
 cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
-                                     const int32_t* offsets, const void* w_gate_up, void* h,
-                                     int* status, cudaStream_t s);
+                                     const int32_t* offsets, const void* w_gate_up, bool packed,
+                                     void* h, int* status, cudaStream_t s);
 cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int32_t* offsets,
-                                  const void* w_down, void* y, int* status, cudaStream_t s);
+                                  const void* w_down, bool packed, void* y, int* status,
+                                  cudaStream_t s);
 cudaError_t launch_gate_up_gemm_pair_gather(const moe_config& c, const void* x,
                                             const int32_t* token_of_row, const int32_t* offsets,
-                                            const void* w_gate_up, void* h, int* status,
-                                            cudaStream_t s);
+                                            const void* w_gate_up, bool packed, void* h,
+                                            int* status, cudaStream_t s);
+// Rearranges E x [rows, cols] bf16 into 128 x 64 blocks (see MOE_FLAG_PACKED_WEIGHTS).
+cudaError_t launch_pack_weights(int E, int rows, int cols, const void* w, void* w_packed,
+                                cudaStream_t s);
 
 cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm,
                                          const int32_t* offsets, const void* w_gate_up,

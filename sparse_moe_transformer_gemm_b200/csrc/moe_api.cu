@@ -8,7 +8,8 @@ using namespace moe;
 
 namespace {
 
-constexpr uint32_t kKnownFlags = MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH | MOE_FLAG_GEMM_PATH;
+constexpr uint32_t kKnownFlags = MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH | MOE_FLAG_GEMM_PATH |
+                                 MOE_FLAG_PACKED_WEIGHTS;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -16,6 +17,9 @@ int check_cfg(const moe_config* c) {
     if (!c) return MOE_ERR_INVALID_ARG;
     if ((c->flags & ~kKnownFlags) != 0) return MOE_ERR_INVALID_ARG;
     if ((c->flags & MOE_FLAG_STREAM_PATH) && (c->flags & MOE_FLAG_GEMM_PATH))
+        return MOE_ERR_INVALID_ARG;
+    if ((c->flags & MOE_FLAG_PACKED_WEIGHTS) &&
+        (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH)))
         return MOE_ERR_INVALID_ARG;
     if (!isfinite(c->scale)) return MOE_ERR_INVALID_ARG;
     if (c->T < 1 || c->E < 1 || c->E > 256 || c->k < 1 || c->k > c->E || c->k > 32)
@@ -25,8 +29,12 @@ int check_cfg(const moe_config* c) {
     const long long R = (long long)c->T * c->k;
     const long long wide = c->d > c->d_ff ? c->d : c->d_ff;
     if (R * wide >= (1LL << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if ((c->flags & MOE_FLAG_PACKED_WEIGHTS) && !pair_gemm_supported(*c))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
     return MOE_OK;
 }
+
+bool packed(const moe_config* c) { return (c->flags & MOE_FLAG_PACKED_WEIGHTS) != 0; }
 
 // Expert weights: bf16 without the FP8 flag (no scales), e4m3 + scales with it.
 int check_expert_weights(const moe_config* c, const void* w, const float* s) {
@@ -96,7 +104,7 @@ int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offs
                                                         h, status, s));
     }
     if (pair_gemm_supported(*c))
-        return cuda_status(launch_gate_up_gemm_pair(*c, x_perm, offsets, w_gate_up, h, status, s));
+        return cuda_status(launch_gate_up_gemm_pair(*c, x_perm, offsets, w_gate_up, packed(c), h, status, s));
     return cuda_status(launch_gate_up_gemm(*c, x_perm, offsets, w_gate_up, h, status, s));
 }
 
@@ -109,7 +117,7 @@ int experts_gate_up_gather(const moe_config* c, const void* x, const int32_t* to
     const WsLayout L = ws_layout(*c);
     if (!use_stream_path(c) && !(c->flags & MOE_FLAG_FP8_WEIGHTS) && pair_gemm_supported(*c))
         return cuda_status(launch_gate_up_gemm_pair_gather(*c, x, token_of_row, offsets, w_gate_up,
-                                                           h, at<int>(ws, L.status), s));
+                                                           packed(c), h, at<int>(ws, L.status), s));
     void* xperm = at<void>(ws, L.xperm);
     MOE_TRY(cuda_status(launch_gather_rows(*c, x, token_of_row, offsets, xperm, s)));
     return experts_gate_up(c, xperm, offsets, w_gate_up, s_gate_up, h, ws, s);
@@ -126,7 +134,7 @@ int experts_down(const moe_config* c, const void* h, const int32_t* offsets, con
             launch_down_gemm_pair_fp8(*c, h, offsets, w_down, s_down, y, status, s));
     }
     if (pair_gemm_supported(*c))
-        return cuda_status(launch_down_gemm_pair(*c, h, offsets, w_down, y, status, s));
+        return cuda_status(launch_down_gemm_pair(*c, h, offsets, w_down, packed(c), y, status, s));
     return cuda_status(launch_down_gemm(*c, h, offsets, w_down, y, status, s));
 }
 
@@ -277,6 +285,23 @@ int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const 
     }
     MOE_TRY(experts_down(cfg, h, offsets, w_down, s_down, y, ws, s));
     return cuda_status(launch_combine(*cfg, y, row_of, w, out, s));
+}
+
+int moe_pack_weights(const moe_config* cfg, int which, const void* w, void* w_packed,
+                     void* stream) {
+    MOE_TRY(check_cfg(cfg));
+    if (cfg->flags & MOE_FLAG_FP8_WEIGHTS) return MOE_ERR_INVALID_ARG;
+    if (which != MOE_WEIGHTS_GATE_UP && which != MOE_WEIGHTS_DOWN) return MOE_ERR_INVALID_ARG;
+    if (!w || !w_packed || !aligned16(w) || !aligned16(w_packed)) return MOE_ERR_INVALID_ARG;
+    if (!pair_gemm_supported(*cfg)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const int rows = which == MOE_WEIGHTS_GATE_UP ? 2 * cfg->d_ff : cfg->d;
+    const int cols = which == MOE_WEIGHTS_GATE_UP ? cfg->d : cfg->d_ff;
+    const size_t bytes = (size_t)cfg->E * rows * cols * 2;
+    const char* a = static_cast<const char*>(w);
+    const char* b = static_cast<const char*>(w_packed);
+    if (a < b + bytes && b < a + bytes) return MOE_ERR_INVALID_ARG;  // overlap
+    return cuda_status(launch_pack_weights(cfg->E, rows, cols, w, w_packed,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int moe_read_status(void* ws, void* stream) {

@@ -29,11 +29,14 @@ MOE_ERR_TIMEOUT = -5
 MOE_FLAG_FP8_WEIGHTS = 0x1
 MOE_FLAG_STREAM_PATH = 0x2
 MOE_FLAG_GEMM_PATH = 0x4
+MOE_FLAG_PACKED_WEIGHTS = 0x8
+MOE_WEIGHTS_GATE_UP = 0
+MOE_WEIGHTS_DOWN = 1
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
             "moe_permute_index", "moe_expert_gate_up", "moe_expert_gate_up_gather",
             "moe_expert_down", "moe_experts", "moe_combine", "moe_forward", "moe_read_status",
-            "moe_status_string", "moe_route_noalloc")
+            "moe_status_string", "moe_route_noalloc", "moe_pack_weights")
 
 MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 # batches of at most this many token-slots (T*k) gather their token rows inside
@@ -86,6 +89,7 @@ def lib() -> ctypes.CDLL:
         "moe_read_status": (I, [P, P]),
         "moe_status_string": (ctypes.c_char_p, [I]),
         "moe_route_noalloc": (I, [C, P, P, P, P, P, P]),
+        "moe_pack_weights": (I, [C, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -96,9 +100,12 @@ def lib() -> ctypes.CDLL:
 
 
 def config(T: int, d: int, E: int, k: int, d_ff: int, scale: float = 2.826, fp8: bool = False,
-           path: Optional[str] = None) -> MoeConfig:
-    """Build a moe_config. path: None (automatic), "stream" or "gemm"."""
+           path: Optional[str] = None, packed: bool = False) -> MoeConfig:
+    """Build a moe_config. path: None (automatic), "stream" or "gemm"; packed: the
+    bf16 expert weights are in moe_pack_weights' layout."""
     flags = MOE_FLAG_FP8_WEIGHTS if fp8 else 0
+    if packed:
+        flags |= MOE_FLAG_PACKED_WEIGHTS
     if path == "stream":
         flags |= MOE_FLAG_STREAM_PATH
     elif path == "gemm":
@@ -213,6 +220,12 @@ def moe_route_noalloc(cfg, x, w_gate, gate_bias, topk_idx, topk_w, stream=None) 
                                    _p(topk_idx), _p(topk_w), _s(stream)))
 
 
+def moe_pack_weights(cfg, which, w, w_packed, stream=None) -> None:
+    """Rearrange one bf16 expert weight into the packed 128 x 64 block layout."""
+    _check("moe_pack_weights", lib().moe_pack_weights(ctypes.byref(cfg), int(which), _p(w),
+                                                      _p(w_packed), _s(stream)))
+
+
 def moe_read_status(ws, stream=None) -> int:
     return int(lib().moe_read_status(_p(ws), _s(stream)))
 
@@ -224,6 +237,17 @@ def layer_args(layer: dict):
     return layer["w_gate_up"], None, layer["w_down"], None
 
 
-def config_of(shape, path: Optional[str] = None) -> MoeConfig:
+def config_of(shape, path: Optional[str] = None, packed: bool = False) -> MoeConfig:
     """moe_config for a synthetic LayerShape."""
-    return config(shape.T, shape.d, shape.E, shape.k, shape.F, shape.scale, shape.fp8, path)
+    return config(shape.T, shape.d, shape.E, shape.k, shape.F, shape.scale, shape.fp8, path,
+                  packed)
+
+
+def pack_layer_weights(cfg: MoeConfig, w_gate_up: torch.Tensor, w_down: torch.Tensor,
+                       stream=None):
+    """(packed w_gate_up, packed w_down): new tensors in moe_pack_weights' layout."""
+    gu = torch.empty_like(w_gate_up)
+    dn = torch.empty_like(w_down)
+    moe_pack_weights(cfg, MOE_WEIGHTS_GATE_UP, w_gate_up, gu, stream)
+    moe_pack_weights(cfg, MOE_WEIGHTS_DOWN, w_down, dn, stream)
+    return gu, dn

@@ -34,6 +34,38 @@ def test_header_constants_match_the_binding():
     assert m and int(m.group(1)) == moe.MOE_GATHER_MAX_SLOTS
     m = re.search(r"#define MOE_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
     assert m and int(m.group(1)) << int(m.group(2)) == moe.MOE_NOALLOC_SCRATCH_BYTES
+    for name in ("MOE_FLAG_FP8_WEIGHTS", "MOE_FLAG_STREAM_PATH", "MOE_FLAG_GEMM_PATH",
+                 "MOE_FLAG_PACKED_WEIGHTS"):
+        m = re.search(r"#define %s (0x[0-9a-f]+)u" % name, text)
+        assert m and int(m.group(1), 16) == getattr(moe, name), name
+    for name in ("MOE_WEIGHTS_GATE_UP", "MOE_WEIGHTS_DOWN"):
+        m = re.search(r"#define %s (\d+)" % name, text)
+        assert m and int(m.group(1)) == getattr(moe, name), name
+
+
+def test_packed_weights_flag_rules(lib):
+    assert moe.moe_workspace_size(moe.config(**HY3, packed=True)) > 0
+    assert moe.moe_workspace_size(moe.config(**HY3, packed=True, fp8=True)) == 0
+    assert moe.moe_workspace_size(moe.config(**HY3, packed=True, path="stream")) == 0
+    assert moe.moe_workspace_size(moe.config(**HY3, packed=True, path="gemm")) > 0
+    # the tensor-core pair kernels need d and d_ff multiples of 256
+    assert moe.moe_workspace_size(moe.config(**{**HY3, "d": 384}, packed=True)) == 0
+    assert moe.moe_workspace_size(moe.config(**{**HY3, "d": 384})) > 0
+
+
+def test_pack_weights_rejects_bad_arguments(lib):
+    P = ctypes.c_void_p
+    cfg = moe.config(**HY3)
+    n = 192 * 2 * 1536 * 4096 * 2
+    call = lambda c, which, a, b: _call("moe_pack_weights", ctypes.byref(c), which, a, b, None)  # noqa: E731
+    assert call(cfg, 2, P(FAKE), P(FAKE + n)) == moe.MOE_ERR_INVALID_ARG
+    assert call(cfg, moe.MOE_WEIGHTS_GATE_UP, None, P(FAKE + n)) == moe.MOE_ERR_INVALID_ARG
+    assert call(cfg, moe.MOE_WEIGHTS_GATE_UP, P(FAKE), P(FAKE + 8)) == moe.MOE_ERR_INVALID_ARG
+    assert call(cfg, moe.MOE_WEIGHTS_GATE_UP, P(FAKE), P(FAKE + n - 16)) == moe.MOE_ERR_INVALID_ARG
+    assert call(moe.config(**HY3, fp8=True), moe.MOE_WEIGHTS_DOWN, P(FAKE), P(FAKE + n)) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert call(moe.config(**{**HY3, "d_ff": 384}), moe.MOE_WEIGHTS_DOWN, P(FAKE),
+                P(FAKE + n)) == moe.MOE_ERR_UNSUPPORTED_SHAPE
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -141,6 +173,7 @@ def test_unsupported_shape_is_reported_by_every_entry_point(lib):
         "moe_experts": (f, f, f, None, f, None, f, f, 1 << 30, None),
         "moe_combine": (f, f, f, f, f, 1 << 30, None),
         "moe_forward": (f, f, None, f, None, f, None, f, f, 1 << 30, None),
+        "moe_pack_weights": (moe.MOE_WEIGHTS_GATE_UP, f, P(FAKE + (1 << 34)), None),
     }
     for fn, args in cases.items():
         assert _call(fn, ctypes.byref(cfg), *args) == moe.MOE_ERR_UNSUPPORTED_SHAPE, fn

@@ -211,6 +211,43 @@ def test_gate_up_gather_equals_permuted_copy_bitwise(name, path):
     assert torch.equal(h_copy, h_gather)
 
 
+def test_pack_weights_is_a_block_permutation():
+    """moe_pack_weights: 128-row x 64-column blocks, ordered by expert, row block,
+    column block, row-major inside -- checked against torch's view/permute."""
+    E, F, d = 3, 256, 512
+    cfg = moe.config(T=1, d=d, E=E, k=1, d_ff=F)
+    g = torch.Generator(device="cpu").manual_seed(9)
+    for which, rows, cols in ((moe.MOE_WEIGHTS_GATE_UP, 2 * F, d), (moe.MOE_WEIGHTS_DOWN, d, F)):
+        w = torch.randn((E, rows, cols), generator=g).to(torch.bfloat16).cuda()
+        wp = torch.empty_like(w)
+        moe.moe_pack_weights(cfg, which, w, wp)
+        torch.cuda.synchronize()
+        want = w.view(E, rows // 128, 128, cols // 64, 64).permute(0, 1, 3, 2, 4).contiguous()
+        assert torch.equal(wp.view(-1), want.view(-1))
+
+
+@pytest.mark.parametrize("shape", [
+    SMALL["pair_small"], SMALL["pair_ragged"],
+    LayerShape(T=700, d=512, E=16, k=8, F=256),   # 5600 slots: the permuted-copy path
+    CONFIGS["decode"],
+], ids=["pair_small", "pair_ragged", "copy_path", "hy3_decode"])
+def test_packed_weights_give_identical_outputs(shape):
+    """MOE_FLAG_PACKED_WEIGHTS changes only where the weight tiles are read from:
+    moe_forward's output is bitwise the same as with the row-major weights."""
+    layer = make_layer(shape, seed=13, device="cuda")
+    want = parity.gpu_forward(layer).clone()
+    cfg = moe.config_of(shape, packed=True)
+    gu, dn = moe.pack_layer_weights(cfg, layer["w_gate_up"], layer["w_down"])
+    ws = moe.workspace(cfg)
+    out = torch.empty_like(want)
+    moe.moe_forward(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"), gu, None, dn, None,
+                    out, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_status(ws) == moe.MOE_OK
+    assert torch.equal(out, want)
+    _free(layer, gu, dn)
+
+
 def test_fp32_combine_keeps_small_terms():
     """Hy3 commentary §2.3 example: one branch output 8.2 and seven of 0.03 (all
     already bf16). An fp32 sum gives 8.375 after the cast; a bf16 running sum
