@@ -9,6 +9,14 @@ JSON line. With N > 1 (torchrun) every rank runs an independent replica on its
 own batch (tokens are independent: no collective on the data path) and the
 value is the tokens of all ranks over the slowest rank's time.
 
+The step is timed through the public entry points one stage at a time
+(moe_route, moe_permute_index or moe_permute, moe_expert_gate_up_gather or
+moe_expert_gate_up, moe_expert_down, moe_combine -- the same sequence
+moe_forward runs), with CUDA events on the launching stream; ``e2e`` times
+moe_forward with the input copied in from and the output copied back to pinned
+host memory every step. bf16 expert weights for the tensor-core kernels are
+packed once at load (moe_pack_weights), outside every timed region.
+
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (each
 step a bounded sample of the same workload), rank 0 only.
 """

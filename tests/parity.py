@@ -1,7 +1,7 @@
 """Shared helpers of the GPU parity tests: run the CUDA path through the C ABI
 and compare it with the fp64 oracle.
 
-Tolerances (fixed by the layer's specification for this build):
+Tolerances (fixed by the layer's parity specification):
   * routing: selected expert sets equal, bit-exact, for every token whose gap
     between the k-th and (k+1)-th oracle score is >= 1e-5; tokens below that
     gap are reported and their selection only has to be a valid top-k within
