@@ -23,6 +23,16 @@
  *        y_i = sum_f h_f Wd[e, i, f]
  *   6. out_i   = bf16_rne( sum_j w_j * y_{j,i} )
  *
+ * The complete Hy3 MoE block adds two optional pieces (same pages: §4.1 step 2
+ * and the Flash QA's Q4.3 / Q4.7):
+ *   - e_score_correction_bias b_e, added to the sigmoid scores for the choice
+ *     only: step 3 ranks c_e = s_e + b_e, while step 4 still renormalises the
+ *     unbiased s_j of the chosen experts;
+ *   - one shared expert (a SwiGLU with its own weights, applied to every
+ *     token with weight 1): step 6 becomes
+ *       out_i = bf16_rne( sum_j w_j * y_{j,i} + y_shared_i ),
+ *     the shared term added last, inside the same fp64 sum.
+ *
  * Every sum is a plain left-to-right fp64 loop; inputs are bf16 bit patterns
  * (or e4m3 codes with fp32 scales) widened exactly to double. The only
  * rounding to a narrow type is the single final bf16 cast of step 6.
@@ -127,28 +137,30 @@ static double weight_at(const void* w, const float* scales, long e, long rows, l
 /* ---------------------------------------------------------------- routing */
 
 typedef struct {
-    double s;
+    double key; /* what the choice ranks: s, plus the score bias when given */
+    double s;   /* sigmoid score */
     int e;
 } scored_expert;
 
-/* Descending score; equal scores: lower expert index first. */
+/* Descending key; equal keys: lower expert index first. */
 static int by_score_then_index(const void* pa, const void* pb)
 {
     const scored_expert* a = (const scored_expert*)pa;
     const scored_expert* b = (const scored_expert*)pb;
-    if (a->s > b->s)
+    if (a->key > b->key)
         return -1;
-    if (a->s < b->s)
+    if (a->key < b->key)
         return 1;
     return (a->e < b->e) ? -1 : (a->e > b->e);
 }
 
-/* Route one token: steps 1-4 above. Writes k indices (descending score), their
+/* Route one token: steps 1-4 above. Writes k indices (descending key), their
  * k weights, optionally all E logits and scores, and the gap between the k-th
- * and (k+1)-th largest score (+inf when k == E). */
+ * and (k+1)-th largest key (+inf when k == E). score_bias may be NULL. */
 static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
-                        const uint16_t* wg, const float* gate_bias, int32_t* idx, double* w,
-                        double* logits_out, double* scores_out, double* gap)
+                        const uint16_t* wg, const float* gate_bias, const float* score_bias,
+                        int32_t* idx, double* w, double* logits_out, double* scores_out,
+                        double* gap)
 {
     scored_expert* order = (scored_expert*)malloc(sizeof(scored_expert) * (size_t)E);
     double sel_sum = 0.0;
@@ -160,6 +172,7 @@ static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
         if (gate_bias)
             logit += (double)gate_bias[e];
         order[e].s = sigmoid(logit);
+        order[e].key = score_bias ? order[e].s + (double)score_bias[e] : order[e].s;
         order[e].e = e;
         if (logits_out)
             logits_out[e] = logit;
@@ -173,7 +186,7 @@ static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
         idx[j] = order[j].e;
         w[j] = scale * order[j].s / sel_sum;
     }
-    *gap = (k < E) ? order[k - 1].s - order[k].s : INFINITY;
+    *gap = (k < E) ? order[k - 1].key - order[k].key : INFINITY;
     free(order);
 }
 
@@ -210,14 +223,16 @@ static void expert_token(int d, int F, long e, const uint16_t* xrow, const void*
 /* Step 6 for one token: out_i = bf16_rne( sum_j w_j * y_{j,i} ), the sum in
  * fp64 over j = 0..k-1 in order. y is [k, d]. acc (may be NULL) receives the
  * sum before the cast. */
-static void combine_token(int k, int d, const double* y, const double* w, double* acc,
-                          uint16_t* out)
+static void combine_token(int k, int d, const double* y, const double* w, const double* y_shared,
+                          double* acc, uint16_t* out)
 {
     int i, j;
     for (i = 0; i < d; ++i) {
         double a = 0.0;
         for (j = 0; j < k; ++j)
             a += w[j] * y[(long)j * d + i];
+        if (y_shared)
+            a += y_shared[i];
         if (acc)
             acc[i] = a;
         out[i] = double_to_bf16(a);
@@ -231,7 +246,7 @@ void oracle_combine(int n, int k, int d, const double* y, const double* w, uint1
 {
     long r;
     for (r = 0; r < n; ++r)
-        combine_token(k, d, y + r * (long)k * d, w + r * (long)k, NULL, out + r * (long)d);
+        combine_token(k, d, y + r * (long)k * d, w + r * (long)k, NULL, NULL, out + r * (long)d);
 }
 
 
@@ -275,20 +290,29 @@ void oracle_double_from_e4m3(const uint8_t* q, double* out, long n)
         out[i] = e4m3_to_double(q[i]);
 }
 
-/* Steps 1-4 for tokens [0, T). logits/scores may be NULL ([T, E] otherwise). */
-int oracle_route(int T, int d, int E, int k, double scale, const uint16_t* x,
-                 const uint16_t* wg, const float* gate_bias, int32_t* idx, double* w,
-                 double* logits, double* scores, double* gap)
+/* Steps 1-4 for tokens [0, T), with the optional score bias [E] (NULL: none).
+ * logits/scores may be NULL ([T, E] otherwise). */
+int oracle_route2(int T, int d, int E, int k, double scale, const uint16_t* x,
+                  const uint16_t* wg, const float* gate_bias, const float* score_bias,
+                  int32_t* idx, double* w, double* logits, double* scores, double* gap)
 {
     long t;
     if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E)
         return -1;
 #pragma omp parallel for schedule(dynamic, 4)
     for (t = 0; t < T; ++t)
-        route_token(d, E, k, scale, x + t * (long)d, wg, gate_bias, idx + t * (long)k,
-                    w + t * (long)k, logits ? logits + t * (long)E : NULL,
+        route_token(d, E, k, scale, x + t * (long)d, wg, gate_bias, score_bias,
+                    idx + t * (long)k, w + t * (long)k, logits ? logits + t * (long)E : NULL,
                     scores ? scores + t * (long)E : NULL, gap + t);
     return 0;
+}
+
+/* Steps 1-4 without a score bias. */
+int oracle_route(int T, int d, int E, int k, double scale, const uint16_t* x,
+                 const uint16_t* wg, const float* gate_bias, int32_t* idx, double* w,
+                 double* logits, double* scores, double* gap)
+{
+    return oracle_route2(T, d, E, k, scale, x, wg, gate_bias, NULL, idx, w, logits, scores, gap);
 }
 
 /* Step 5 for n (row, expert) pairs: rows of xrows [n, d], experts[n]. h [n, F]
@@ -305,17 +329,23 @@ int oracle_expert_rows(int n, int d, int F, const uint16_t* xrows, const int32_t
     return 0;
 }
 
-/* Steps 1-6 for the n tokens listed in tokens[] (indices into x [T, d]).
+/* Steps 1-6 for the n tokens listed in tokens[] (indices into x [T, d]), with
+ * the optional score bias [E] and shared expert (sh_wgu [2F, d], sh_wd [d, F]
+ * in the routed experts' format, with row scales sh_s_gu [2F] / sh_s_d [d] for
+ * e4m3 codes; sh_wgu NULL: no shared expert).
  * Outputs per listed token: out_f64 [n, d] (the fp64 sum before the cast),
  * out_bf16 [n, d], idx [n, k], w [n, k], gap [n]. */
-int oracle_forward_tokens(int T, int d, int E, int k, int F, double scale, const uint16_t* x,
-                          const uint16_t* wg, const float* gate_bias, const void* wgu,
-                          const float* s_gu, const void* wd, const float* s_d,
-                          const int32_t* tokens, int n, double* out_f64, uint16_t* out_bf16,
-                          int32_t* idx, double* w, double* gap)
+int oracle_forward_tokens2(int T, int d, int E, int k, int F, double scale, const uint16_t* x,
+                           const uint16_t* wg, const float* gate_bias, const float* score_bias,
+                           const void* wgu, const float* s_gu, const void* wd, const float* s_d,
+                           const void* sh_wgu, const float* sh_s_gu, const void* sh_wd,
+                           const float* sh_s_d, const int32_t* tokens, int n, double* out_f64,
+                           uint16_t* out_bf16, int32_t* idx, double* w, double* gap)
 {
     long r;
     if (d <= 0 || E <= 0 || k <= 0 || k > E || F <= 0)
+        return -1;
+    if ((sh_wgu == NULL) != (sh_wd == NULL))
         return -1;
     for (r = 0; r < n; ++r)
         if (tokens[r] < 0 || tokens[r] >= T)
@@ -324,16 +354,33 @@ int oracle_forward_tokens(int T, int d, int E, int k, int F, double scale, const
     for (r = 0; r < n; ++r) {
         const uint16_t* xrow = x + (long)tokens[r] * d;
         double* y = (double*)malloc(sizeof(double) * (size_t)k * d);
+        double* ysh = sh_wgu ? (double*)malloc(sizeof(double) * (size_t)d) : NULL;
         int j;
-        route_token(d, E, k, scale, xrow, wg, gate_bias, idx + r * (long)k, w + r * (long)k,
-                    NULL, NULL, gap + r);
+        route_token(d, E, k, scale, xrow, wg, gate_bias, score_bias, idx + r * (long)k,
+                    w + r * (long)k, NULL, NULL, gap + r);
         for (j = 0; j < k; ++j)
             expert_token(d, F, idx[r * (long)k + j], xrow, wgu, s_gu, wd, s_d, NULL,
                          y + (long)j * d);
-        combine_token(k, d, y, w + r * (long)k, out_f64 + r * (long)d, out_bf16 + r * (long)d);
+        if (ysh)
+            expert_token(d, F, 0, xrow, sh_wgu, sh_s_gu, sh_wd, sh_s_d, NULL, ysh);
+        combine_token(k, d, y, w + r * (long)k, ysh, out_f64 + r * (long)d,
+                      out_bf16 + r * (long)d);
+        free(ysh);
         free(y);
     }
     return 0;
+}
+
+/* Steps 1-6 without a score bias or shared expert. */
+int oracle_forward_tokens(int T, int d, int E, int k, int F, double scale, const uint16_t* x,
+                          const uint16_t* wg, const float* gate_bias, const void* wgu,
+                          const float* s_gu, const void* wd, const float* s_d,
+                          const int32_t* tokens, int n, double* out_f64, uint16_t* out_bf16,
+                          int32_t* idx, double* w, double* gap)
+{
+    return oracle_forward_tokens2(T, d, E, k, F, scale, x, wg, gate_bias, NULL, wgu, s_gu, wd,
+                                  s_d, NULL, NULL, NULL, NULL, tokens, n, out_f64, out_bf16, idx,
+                                  w, gap);
 }
 
 /* The grouping that the library's permute step defines (integer work):

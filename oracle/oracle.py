@@ -47,11 +47,16 @@ def _load():
         lib.oracle_double_from_e4m3.argtypes = [P, P, L]
         lib.oracle_route.argtypes = [I, I, I, I, D, P, P, P, P, P, P, P, P]
         lib.oracle_route.restype = I
+        lib.oracle_route2.argtypes = [I, I, I, I, D, P, P, P, P, P, P, P, P, P]
+        lib.oracle_route2.restype = I
         lib.oracle_expert_rows.argtypes = [I, I, I, P, P, P, P, P, P, P, P]
         lib.oracle_expert_rows.restype = I
         lib.oracle_forward_tokens.argtypes = [I, I, I, I, I, D, P, P, P, P, P, P, P, P, I, P, P,
                                               P, P, P]
         lib.oracle_forward_tokens.restype = I
+        lib.oracle_forward_tokens2.argtypes = [I, I, I, I, I, D, P, P, P, P, P, P, P, P, P, P, P,
+                                               P, P, I, P, P, P, P, P]
+        lib.oracle_forward_tokens2.restype = I
         lib.oracle_combine.argtypes = [I, I, I, P, P, P]
         lib.oracle_permute.argtypes = [I, I, I, P, P, P, P]
         lib.oracle_permute.restype = I
@@ -102,11 +107,14 @@ def double_from_e4m3(q: np.ndarray) -> np.ndarray:
     return out
 
 
-def route(x, wg, k: int, scale: float, gate_bias=None, want_scores: bool = False):
+def route(x, wg, k: int, scale: float, gate_bias=None, want_scores: bool = False,
+          score_bias=None):
     """Steps 1-4 for all tokens. x [T,d] / wg [E,d] uint16 bf16 bits.
 
-    Returns dict(idx int32 [T,k], w f64 [T,k], gap f64 [T], and with
-    want_scores also logits/scores f64 [T,E]).
+    gate_bias [E] is added to the logits (before the sigmoid); score_bias [E]
+    (e_score_correction_bias) to the scores for the choice only. Returns
+    dict(idx int32 [T,k], w f64 [T,k], gap f64 [T] -- between the k-th and
+    (k+1)-th ranked value -- and with want_scores also logits/scores f64 [T,E]).
     """
     x = np.ascontiguousarray(x, dtype=np.uint16)
     wg = np.ascontiguousarray(wg, dtype=np.uint16)
@@ -118,8 +126,9 @@ def route(x, wg, k: int, scale: float, gate_bias=None, want_scores: bool = False
     gap = np.empty((T,), dtype=np.float64)
     logits = np.empty((T, E), dtype=np.float64) if want_scores else None
     scores = np.empty((T, E), dtype=np.float64) if want_scores else None
-    rc = _load().oracle_route(T, d, E, k, float(scale), _ptr(x), _ptr(wg), _ptr(gb), _ptr(idx),
-                              _ptr(w), _ptr(logits), _ptr(scores), _ptr(gap))
+    sb = None if score_bias is None else np.ascontiguousarray(score_bias, dtype=np.float32)
+    rc = _load().oracle_route2(T, d, E, k, float(scale), _ptr(x), _ptr(wg), _ptr(gb), _ptr(sb),
+                               _ptr(idx), _ptr(w), _ptr(logits), _ptr(scores), _ptr(gap))
     if rc != 0:
         raise ValueError("oracle_route: bad arguments")
     out = {"idx": idx, "w": w, "gap": gap}
@@ -162,10 +171,12 @@ def forward_tokens(layer: "OracleLayer", tokens=None):
     idx = np.empty((n, L.k), dtype=np.int32)
     w = np.empty((n, L.k), dtype=np.float64)
     gap = np.empty((n,), dtype=np.float64)
-    rc = _load().oracle_forward_tokens(L.T, L.d, L.E, L.k, L.F, float(L.scale), _ptr(L.x),
-                                       _ptr(L.wg), _ptr(L.gate_bias), _ptr(L.wgu), _ptr(L.s_gu),
-                                       _ptr(L.wd), _ptr(L.s_d), _ptr(tokens), n, _ptr(out_f64),
-                                       _ptr(out_bf16), _ptr(idx), _ptr(w), _ptr(gap))
+    rc = _load().oracle_forward_tokens2(L.T, L.d, L.E, L.k, L.F, float(L.scale), _ptr(L.x),
+                                        _ptr(L.wg), _ptr(L.gate_bias), _ptr(L.score_bias),
+                                        _ptr(L.wgu), _ptr(L.s_gu), _ptr(L.wd), _ptr(L.s_d),
+                                        _ptr(L.sh_wgu), _ptr(L.sh_s_gu), _ptr(L.sh_wd),
+                                        _ptr(L.sh_s_d), _ptr(tokens), n, _ptr(out_f64),
+                                        _ptr(out_bf16), _ptr(idx), _ptr(w), _ptr(gap))
     if rc != 0:
         raise ValueError("oracle_forward_tokens: bad arguments")
     return {"out_f64": out_f64, "out_bf16": out_bf16, "idx": idx, "w": w, "gap": gap,
@@ -212,6 +223,9 @@ class OracleLayer:
         gb = layer.get("gate_bias")
         self.gate_bias = None if gb is None else np.ascontiguousarray(gb.detach().cpu().numpy(),
                                                                       dtype=np.float32)
+        sb = layer.get("score_bias")
+        self.score_bias = None if sb is None else np.ascontiguousarray(
+            sb.detach().cpu().numpy(), dtype=np.float32)
         if cfg.fp8:
             self.wgu = np.ascontiguousarray(layer["q_gate_up"].cpu().numpy())
             self.wd = np.ascontiguousarray(layer["q_down"].cpu().numpy())
@@ -222,3 +236,15 @@ class OracleLayer:
             self.wd = bf16_bits(layer["w_down"])
             self.s_gu = None
             self.s_d = None
+        # the shared expert (optional), in the routed experts' format
+        self.sh_wgu = self.sh_wd = self.sh_s_gu = self.sh_s_d = None
+        if cfg.fp8 and layer.get("q_shared_gate_up") is not None:
+            self.sh_wgu = np.ascontiguousarray(layer["q_shared_gate_up"].cpu().numpy())
+            self.sh_wd = np.ascontiguousarray(layer["q_shared_down"].cpu().numpy())
+            self.sh_s_gu = np.ascontiguousarray(layer["s_shared_gate_up"].cpu().numpy(),
+                                                dtype=np.float32)
+            self.sh_s_d = np.ascontiguousarray(layer["s_shared_down"].cpu().numpy(),
+                                               dtype=np.float32)
+        elif not cfg.fp8 and layer.get("w_shared_gate_up") is not None:
+            self.sh_wgu = bf16_bits(layer["w_shared_gate_up"])
+            self.sh_wd = bf16_bits(layer["w_shared_down"])

@@ -18,9 +18,11 @@ scaling 2.826) are those of "Tencent Hy3-295B 架构深度拆解" (pillumina.git
 §2.1 hyper-parameter table and §2.3 parameter breakdown.
 
 Draw order, from one torch.Generator seeded with ``seed``: x, W_gate,
-W_gate_up (expert by expert), W_down (expert by expert). Each tensor is drawn
-as fp32 N(0,1), multiplied by its standard deviation and rounded to bf16
-(round-to-nearest-even, torch's cast). The bf16 bit patterns are what both the
+W_gate_up (expert by expert), W_down (expert by expert), then -- only for
+shapes that ask for them -- the shared expert's W_gate_up and W_down and the
+e_score_correction_bias. Each weight is drawn as fp32 N(0,1), multiplied by
+its standard deviation and rounded to bf16 (round-to-nearest-even, torch's
+cast); the score bias stays fp32. The bf16 bit patterns are what both the
 oracle and the CUDA path consume.
 
 Layouts (row-major, contiguous):
@@ -29,6 +31,10 @@ Layouts (row-major, contiguous):
   w_gate_up  [E, 2F, d]    bf16   rows [0, F) are the gate rows, [F, 2F) the up rows
   w_down     [E, d, F]     bf16
   gate_bias  [E]           fp32 or None (added to the router logits)
+  score_bias [E]           fp32 or None (e_score_correction_bias: added to the
+                           sigmoid scores for the choice of experts only)
+  w_shared_gate_up [2F, d], w_shared_down [d, F]   bf16, when the shape has a
+                           shared expert (q_/s_shared_* for FP8 shapes)
 FP8 workloads add ``q_gate_up`` [E, 2F, d] / ``q_down`` [E, d, F] as uint8
 e4m3 codes and ``s_gate_up`` [E, 2F] / ``s_down`` [E, d] fp32 scales, with the
 weight meaning q * s.
@@ -54,6 +60,8 @@ class LayerShape:
     w_std: float = 0.02
     zipf_bias: bool = False
     fp8: bool = False
+    shared: bool = False          # one shared expert (SwiGLU, d_ff = F), weight 1
+    score_bias_std: float = 0.0   # e_score_correction_bias ~ N(0, std^2) when > 0
 
     @property
     def R(self) -> int:
@@ -152,7 +160,14 @@ def make_layer(cfg, seed: int = 0, device="cpu", T: Optional[int] = None,
         "w_gate_up": w_gate_up,
         "w_down": w_down,
         "gate_bias": zipf_logit_bias(E).to(dev) if cfg.zipf_bias else None,
+        "score_bias": None,
     }
+    if cfg.shared:
+        out["w_shared_gate_up"] = _normal(gen, shp["w_gate_up"][1:], cfg.w_std, dev)
+        out["w_shared_down"] = _normal(gen, shp["w_down"][1:], cfg.w_std, dev)
+    if cfg.score_bias_std > 0:
+        out["score_bias"] = torch.randn((E,), generator=gen, dtype=torch.float32,
+                                        device=dev) * cfg.score_bias_std
     if cfg.fp8:
         q_gu = torch.empty(shp["w_gate_up"], dtype=torch.uint8, device=dev)
         s_gu = torch.empty(shp["s_gate_up"], dtype=torch.float32, device=dev)
@@ -162,4 +177,9 @@ def make_layer(cfg, seed: int = 0, device="cpu", T: Optional[int] = None,
             q_gu[e], s_gu[e] = encode_e4m3_rows(w_gate_up[e])
             q_d[e], s_d[e] = encode_e4m3_rows(w_down[e])
         out.update(q_gate_up=q_gu, s_gate_up=s_gu, q_down=q_d, s_down=s_d)
+        if cfg.shared:
+            qs_gu, ss_gu = encode_e4m3_rows(out["w_shared_gate_up"])
+            qs_d, ss_d = encode_e4m3_rows(out["w_shared_down"])
+            out.update(q_shared_gate_up=qs_gu, s_shared_gate_up=ss_gu, q_shared_down=qs_d,
+                       s_shared_down=ss_d)
     return out

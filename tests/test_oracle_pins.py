@@ -306,3 +306,125 @@ def test_permute_definition_matches_stable_argsort(T, k, E):
     assert np.array_equal(r["row_of"], want_row_of)
     assert np.array_equal(r["counts"], np.bincount(flat, minlength=E))
     assert np.array_equal(r["offsets"], np.concatenate([[0], np.cumsum(np.bincount(flat, minlength=E))]))
+
+
+# ------------------------------------------------------------------ the complete Hy3 block:
+# e_score_correction_bias (choice only) and the shared expert (weight 1)
+
+def _bits(t):
+    return oracle.bf16_bits(t)
+
+
+def _unit_router(logits):
+    """x = e_0 and W_gate rows with the given first entries: the logits are exact."""
+    E = len(logits)
+    x = torch.zeros((1, 16), dtype=torch.bfloat16)
+    x[0, 0] = 1.0
+    wg = torch.zeros((E, 16), dtype=torch.bfloat16)
+    wg[:, 0] = torch.tensor(logits, dtype=torch.float32).to(torch.bfloat16)
+    assert [float(v) for v in wg[:, 0]] == list(map(float, logits))
+    return _bits(x), _bits(wg)
+
+
+def test_zero_score_bias_changes_nothing():
+    L = _layer(LayerShape(T=40, d=64, E=12, k=4, F=32), seed=21)
+    x, wg = _bits(L["x"]), _bits(L["w_gate"])
+    a = oracle.route(x, wg, 4, 2.826)
+    b = oracle.route(x, wg, 4, 2.826, score_bias=np.zeros(12, np.float32))
+    for key in ("idx", "w", "gap"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+def test_score_bias_chooses_but_does_not_weight(golden):
+    """A large bias on four experts forces them into the top-4; their weights
+    are the renormalised UNBIASED sigmoid scores (numpy, independent)."""
+    assert "choice only" in golden["score_correction_bias"]["claim"]
+    L = _layer(LayerShape(T=30, d=64, E=12, k=4, F=32), seed=22)
+    forced = [2, 5, 7, 11]
+    sb = np.zeros(12, np.float32)
+    sb[forced] = 10.0
+    r = oracle.route(_bits(L["x"]), _bits(L["w_gate"]), 4, 2.826, score_bias=sb)
+    s = 1.0 / (1.0 + np.exp(-_np_logits(L)))
+    for t in range(30):
+        order = sorted(forced, key=lambda e: (-s[t, e], e))
+        assert list(r["idx"][t]) == order
+        assert np.allclose(r["w"][t], 2.826 * s[t, order] / s[t, order].sum(), rtol=1e-12)
+
+
+def test_constant_score_bias_keeps_the_routing():
+    L = _layer(LayerShape(T=50, d=64, E=16, k=4, F=32), seed=24)
+    x, wg = _bits(L["x"]), _bits(L["w_gate"])
+    a = oracle.route(x, wg, 4, 2.826)
+    b = oracle.route(x, wg, 4, 2.826, score_bias=np.full(16, 0.37, np.float32))
+    assert np.array_equal(a["idx"], b["idx"])
+    assert np.array_equal(a["w"], b["w"])
+
+
+def test_score_bias_acts_after_the_sigmoid():
+    """Logits 5 and 6 (a saturated sigmoid): +0.01 on expert 0's SCORE beats
+    sigma(6) - sigma(5) = 0.0042, while +0.01 on its LOGIT does not."""
+    x, wg = _unit_router([5.0, 6.0])
+    r = oracle.route(x, wg, 1, 2.826, score_bias=np.array([0.01, 0.0], np.float32))
+    assert r["idx"][0, 0] == 0 and r["w"][0, 0] == 2.826
+    r = oracle.route(x, wg, 1, 2.826, gate_bias=np.array([0.01, 0.0], np.float32))
+    assert r["idx"][0, 0] == 1
+
+
+def test_gap_is_measured_on_the_ranked_value():
+    """Logits 0, 1, 2 and a score bias of 0.5 on expert 0: the ranked values
+    are 1.0, sigma(1), sigma(2); k=1 picks expert 0 with gap 1 - sigma(2)."""
+    x, wg = _unit_router([0.0, 1.0, 2.0])
+    r = oracle.route(x, wg, 1, 2.826, score_bias=np.array([0.5, 0.0, 0.0], np.float32))
+    assert r["idx"][0, 0] == 0
+    assert math.isclose(r["gap"][0], 1.0 - 1.0 / (1.0 + math.exp(-2.0)), rel_tol=1e-14)
+
+
+def _np_shared(L):
+    x64 = _f64(L["x"])
+    F = L["cfg"].F
+    gu, dn = _f64(L["w_shared_gate_up"]), _f64(L["w_shared_down"])
+    return _np_expert(x64, gu[None], dn[None], 0, F)
+
+
+def test_shared_expert_is_added_with_weight_one():
+    L = _layer(LayerShape(T=12, d=64, E=6, k=2, F=32, shared=True), seed=23)
+    O = oracle.OracleLayer(L)
+    r = oracle.forward_tokens(O)
+    O.sh_wgu = O.sh_wd = None
+    r0 = oracle.forward_tokens(O)
+    assert np.array_equal(r["idx"], r0["idx"])
+    assert np.allclose(r["out_f64"] - r0["out_f64"], _np_shared(L), rtol=1e-9, atol=1e-12)
+
+
+def test_shared_expert_alone_is_the_textbook_mlp():
+    shape = LayerShape(T=10, d=64, E=4, k=2, F=32, shared=True)
+    L = _layer(shape, seed=25)
+    L["w_gate_up"][:, shape.F:, :] = 0          # every routed expert outputs 0
+    r = oracle.forward_tokens(oracle.OracleLayer(L))
+    assert np.allclose(r["out_f64"], _np_shared(L), rtol=1e-9, atol=1e-12)
+    assert np.array_equal(r["out_bf16"], oracle.bf16_from_double(r["out_f64"]))
+
+
+def test_fp8_shared_expert_uses_codes_times_row_scales():
+    shape = LayerShape(T=8, d=64, E=4, k=2, F=32, shared=True, fp8=True)
+    L = _layer(shape, seed=26)
+    L["q_gate_up"][:, shape.F:, :] = 0          # routed outputs 0
+    r = oracle.forward_tokens(oracle.OracleLayer(L))
+    dec = lambda q, s: (q.view(torch.float8_e4m3fn).to(torch.float64) *  # noqa: E731
+                        s.to(torch.float64)[:, None]).numpy()
+    gu = dec(L["q_shared_gate_up"], L["s_shared_gate_up"])
+    dn = dec(L["q_shared_down"], L["s_shared_down"])
+    want = _np_expert(_f64(L["x"]), gu[None], dn[None], 0, shape.F)
+    assert np.allclose(r["out_f64"], want, rtol=1e-9, atol=1e-12)
+
+
+def test_moe_layer_parameter_count_with_the_shared_expert_matches_the_page(golden):
+    shp = tensor_shapes("decode")
+    per_expert = math.prod(shp["w_gate_up"][1:]) + math.prod(shp["w_down"][1:])
+    L = _layer(LayerShape(T=1, d=256, E=2, k=1, F=128, shared=True), seed=0)
+    assert L["w_shared_gate_up"].shape[1:] == L["w_gate_up"].shape[2:]  # same SwiGLU shape
+    layer = math.prod(shp["w_gate"]) + (shp["w_gate_up"][0] + 1) * per_expert
+    assert round(layer / 1e9, 2) * 1e9 == golden["moe_layer_params"]["printed"]
+    assert round(per_expert / 1e6, 2) * 1e6 == golden["moe_layer_params"]["shared_expert_params_printed"]
+    frac = per_expert / ((shp["w_gate_up"][0] + 1) * per_expert)
+    assert round(100 * frac, 2) == golden["shared_expert_fraction"]["printed_percent"]
