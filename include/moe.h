@@ -35,6 +35,15 @@
  *   256 and the tensor-core path: with MOE_FLAG_FP8_WEIGHTS or
  *   MOE_FLAG_STREAM_PATH it is MOE_ERR_INVALID_ARG, with other shapes
  *   MOE_ERR_UNSUPPORTED_SHAPE.
+ * - Shared expert (MOE_FLAG_SHARED_EXPERT; "Tencent Hy3-Flash QA" Q4.7, the
+ *   complete Hy3 block): w_gate_up / w_down (and s_gate_up / s_down) hold
+ *   E + 1 experts, and expert E is a shared expert that every token uses with
+ *   weight 1 on top of its k routed experts:
+ *     out = bf16( sum_j w_j * float(y_j) + float(y_shared) )   (shared last).
+ *   The routing arrays stay [T, k]; the grouping, the expert GEMMs and the
+ *   combine work on k + 1 slots per token (slot k of every token is expert E)
+ *   and E + 1 experts: row_of has T*(k+1) entries, counts E+1, offsets E+2,
+ *   x_perm / h / y T*(k+1) rows. Needs E <= 255.
  * - Grouping ("permuted rows"): token-slot s = t*k + j goes to row
  *   row_of[s] = offsets[e] + (number of earlier slots s' < s with the same
  *   expert e = topk_idx[s]); offsets[e] = sum_{e' < e} counts[e'],
@@ -83,6 +92,7 @@ extern "C" {
 #define MOE_FLAG_STREAM_PATH 0x2u /* experts on the weight-streaming (decode) kernels */
 #define MOE_FLAG_GEMM_PATH 0x4u   /* experts on the tensor-core grouped GEMMs */
 #define MOE_FLAG_PACKED_WEIGHTS 0x8u /* bf16 expert weights in moe_pack_weights' layout */
+#define MOE_FLAG_SHARED_EXPERT 0x10u /* expert E of the weights is a shared expert (below) */
 
 /* Which expert weight moe_pack_weights rearranges. */
 #define MOE_WEIGHTS_GATE_UP 0 /* w_gate_up [E, 2*d_ff, d] */
@@ -116,6 +126,15 @@ MOE_API int moe_workspace_init(const moe_config* cfg, void* ws, size_t ws_bytes,
  * Hy3 commentary §3.3 for a logit bias added before the sigmoid. */
 MOE_API int moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
               int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_route with the complete Hy3 block's e_score_correction_bias: score_bias
+ * (nullable [E] fp32) is added to the sigmoid scores for the choice of the k
+ * experts only; topk_w still renormalises the unbiased sigmoid scores of the
+ * chosen experts ("Tencent Hy3-295B 架构深度拆解" §4.1 steps 2-4; "Tencent
+ * Hy3-Flash QA" Q4.3). NULL gives moe_route exactly. */
+MOE_API int moe_route2(const moe_config* cfg, const void* x, const void* w_gate,
+               const float* gate_bias, const float* score_bias, int32_t* topk_idx, float* topk_w,
+               void* ws, size_t ws_bytes, void* stream);
 
 /* Group token-slots by expert (the grouping defined above): writes counts [E],
  * offsets [E+1], row_of [T*k] (int32) and x_perm [T*k, d] bf16 with
@@ -200,6 +219,14 @@ MOE_API int moe_forward(const moe_config* cfg, const void* x, const void* w_gate
  * tile loads. */
 MOE_API int moe_pack_weights(const moe_config* cfg, int which, const void* w, void* w_packed,
                      void* stream);
+
+/* moe_forward with the optional score_bias of moe_route2 (NULL gives
+ * moe_forward exactly). Together with MOE_FLAG_SHARED_EXPERT this is the
+ * complete Hy3 MoE block. */
+MOE_API int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate,
+                 const float* gate_bias, const float* score_bias, const void* w_gate_up,
+                 const float* s_gate_up, const void* w_down, const float* s_down, void* out,
+                 void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of the fixed device array behind moe_route_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES (2u << 20)

@@ -6,7 +6,9 @@
 // next to a large one are not rounded away. The weighted sum over the k
 // selected experts replaces the pages' per-expert loop with index_add_
 // ("DeepSeek V4-Flash 架构 QA", Q8.4) by a gather: token t reads its k expert
-// rows y[row_of[t*k + j]] (no atomics, fixed j order, deterministic).
+// rows y[row_of[t*k + j]] (no atomics, fixed j order, deterministic). With a
+// shared expert ("Tencent Hy3-Flash QA" Q4.7) each token has one more slot,
+// the last, weighted 1.
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,13 +22,15 @@ constexpr int CT = 128;
 
 __global__ void __launch_bounds__(CT)
 combine_kernel(const __nv_bfloat16* __restrict__ y, const int* __restrict__ row_of,
-               const float* __restrict__ w, int k, int d, __nv_bfloat16* __restrict__ out) {
-    __shared__ int rows[32];
-    __shared__ float wts[32];
+               const float* __restrict__ w, int k_routed, int k, int d,
+               __nv_bfloat16* __restrict__ out) {
+    // k slots per token; slots at and past k_routed (the shared expert) weigh 1
+    __shared__ int rows[33];
+    __shared__ float wts[33];
     const long t = blockIdx.x;
     if (threadIdx.x < k) {
         rows[threadIdx.x] = row_of[t * k + threadIdx.x];
-        wts[threadIdx.x] = w[t * k + threadIdx.x];
+        wts[threadIdx.x] = threadIdx.x < k_routed ? w[t * k_routed + threadIdx.x] : 1.0f;
     }
     __syncthreads();
     const int v = blockIdx.y * CT + threadIdx.x;
@@ -68,7 +72,8 @@ cudaError_t launch_combine(const moe_config& c, const void* y, const int32_t* ro
                            const float* topk_w, void* out, cudaStream_t s) {
     const dim3 grid(c.T, (c.d / 8 + CT - 1) / CT);
     combine_kernel<<<grid, CT, 0, s>>>(static_cast<const __nv_bfloat16*>(y), row_of, topk_w, c.k,
-                                       c.d, static_cast<__nv_bfloat16*>(out));
+                                       c.k + shared_slots(c), c.d,
+                                       static_cast<__nv_bfloat16*>(out));
     return cudaGetLastError();
 }
 

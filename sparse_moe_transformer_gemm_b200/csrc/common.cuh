@@ -81,9 +81,14 @@ __device__ __forceinline__ float key_value(uint32_t key) {
     return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
 }
 
+//
+// With prob (the lane's 8 sigmoid scores; sc then holds the choice values
+// score + e_score_correction_bias), the weights renormalise prob of the chosen
+// experts instead of the sigmoid of the ranked values.
 __device__ __forceinline__ void warp_select_topk(float (&sc)[8], int k, float scale,
                                                  int* __restrict__ idx_row,
-                                                 float* __restrict__ w_row) {
+                                                 float* __restrict__ w_row,
+                                                 const float* prob = nullptr) {
     const int lane = threadIdx.x & 31;
     uint32_t key[8];
 #pragma unroll
@@ -99,7 +104,14 @@ __device__ __forceinline__ void warp_select_topk(float (&sc)[8], int k, float sc
         const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
         const uint32_t be = __reduce_min_sync(0xffffffffu,
                                               bk == m ? (uint32_t)(lane + 32 * bq) : 0xffffffffu);
-        if (lane == r) { my_e = (int)be; my_s = sigmoidf_acc(key_value(m)); }
+        float pv = 0.f;
+        if (prob) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if ((int)(be >> 5) == q) pv = prob[q];
+            pv = __shfl_sync(0xffffffffu, pv, (int)(be & 31u));
+        }
+        if (lane == r) { my_e = (int)be; my_s = prob ? pv : sigmoidf_acc(key_value(m)); }
         if ((int)(be & 31u) == lane) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)

@@ -61,39 +61,53 @@ inline int n_permute_chunks(const moe_config& c) {
     return (int)((R + kPermuteChunk - 1) / kPermuteChunk);
 }
 
+// The shared expert (MOE_FLAG_SHARED_EXPERT) is expert E of the weight arrays
+// and slot k of every token: the grouping, the expert GEMMs and the combine
+// run on the "grouped" configuration with E + 1 experts and k + 1 slots.
+inline int shared_slots(const moe_config& c) {
+    return (c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0;
+}
+inline moe_config grouped_config(const moe_config& c) {
+    moe_config g = c;
+    g.E += shared_slots(c);
+    g.k += shared_slots(c);
+    return g;
+}
+
 inline WsLayout ws_layout(const moe_config& c) {
     WsLayout L{};
-    size_t R = (size_t)c.T * c.k;
+    const moe_config g = grouped_config(c);
+    size_t R = (size_t)g.T * g.k;
     size_t o = 0;
     L.status = o;   o += 256;
     L.counters = o; o = align256(o + sizeof(int32_t) * n_router_groups(c));
     L.control_end = o;
     L.logits = o;   o = align256(o + sizeof(float) * router_ksplit(c) * (size_t)c.T * c.E);
-    L.hist = o;     o = align256(o + sizeof(int32_t) * (size_t)n_permute_chunks(c) * c.E);
+    L.hist = o;     o = align256(o + sizeof(int32_t) * (size_t)n_permute_chunks(g) * g.E);
     L.rank = o;     o = align256(o + sizeof(int32_t) * R);
     L.idx = o;      o = align256(o + sizeof(int32_t) * R);
     L.w = o;        o = align256(o + sizeof(float) * R);
-    L.counts = o;   o = align256(o + sizeof(int32_t) * c.E);
-    L.offsets = o;  o = align256(o + sizeof(int32_t) * (c.E + 1));
+    L.counts = o;   o = align256(o + sizeof(int32_t) * g.E);
+    L.offsets = o;  o = align256(o + sizeof(int32_t) * (g.E + 1));
     L.row_of = o;   o = align256(o + sizeof(int32_t) * R);
     L.tok = o;      o = align256(o + sizeof(int32_t) * R);
     L.xperm = o;    o = align256(o + 2 * R * c.d);
     L.h = o;        o = align256(o + 2 * R * c.d_ff);
     L.y = o;        o = align256(o + 2 * R * c.d);
-    L.sched = o;    o = align256(o + sizeof(int32_t) * 4 * (c.E + 1));
+    L.sched = o;    o = align256(o + sizeof(int32_t) * 4 * (g.E + 1));
     L.total = o;
     return L;
 }
 
 // ---- launchers (each returns cudaError_t of the launch) ----
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
-                          const float* gate_bias, int32_t* idx, float* w, float* logits,
-                          int32_t* counters, int ksplit, cudaStream_t s);
+                          const float* gate_bias, const float* score_bias, int32_t* idx, float* w,
+                          float* logits, int32_t* counters, int ksplit, cudaStream_t s);
 
 bool router_tc_supported(const moe_config& c);
 cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_gate,
-                             const float* gate_bias, int32_t* idx, float* w, int* status,
-                             cudaStream_t s);
+                             const float* gate_bias, const float* score_bias, int32_t* idx,
+                             float* w, int* status, cudaStream_t s);
 
 cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
                            int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,

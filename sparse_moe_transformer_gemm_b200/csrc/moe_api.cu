@@ -9,7 +9,7 @@ using namespace moe;
 namespace {
 
 constexpr uint32_t kKnownFlags = MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH | MOE_FLAG_GEMM_PATH |
-                                 MOE_FLAG_PACKED_WEIGHTS;
+                                 MOE_FLAG_PACKED_WEIGHTS | MOE_FLAG_SHARED_EXPERT;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -22,11 +22,12 @@ int check_cfg(const moe_config* c) {
         (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH)))
         return MOE_ERR_INVALID_ARG;
     if (!isfinite(c->scale)) return MOE_ERR_INVALID_ARG;
-    if (c->T < 1 || c->E < 1 || c->E > 256 || c->k < 1 || c->k > c->E || c->k > 32)
+    if (c->T < 1 || c->E < 1 || c->E > 256 - shared_slots(*c) || c->k < 1 || c->k > c->E ||
+        c->k > 32)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->d < 128 || c->d % 128 != 0 || c->d > 8192) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (c->d_ff < 128 || c->d_ff % 128 != 0 || c->d_ff > 8192) return MOE_ERR_UNSUPPORTED_SHAPE;
-    const long long R = (long long)c->T * c->k;
+    const long long R = (long long)c->T * (c->k + shared_slots(*c));
     const long long wide = c->d > c->d_ff ? c->d : c->d_ff;
     if (R * wide >= (1LL << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if ((c->flags & MOE_FLAG_PACKED_WEIGHTS) && !pair_gemm_supported(*c))
@@ -84,28 +85,31 @@ bool use_stream_path(const moe_config* c) {
 constexpr int kRouterTcMinTokens = 129;
 
 cudaError_t route(const moe_config* c, const void* x, const void* w_gate, const float* gate_bias,
-                  int32_t* idx, float* w, void* ws, cudaStream_t s) {
+                  const float* score_bias, int32_t* idx, float* w, void* ws, cudaStream_t s) {
     const WsLayout L = ws_layout(*c);
     if (router_tc_supported(*c) && c->T >= kRouterTcMinTokens)
-        return launch_router_tc(*c, x, w_gate, gate_bias, idx, w, at<int>(ws, L.status), s);
-    return launch_router(*c, x, w_gate, gate_bias, idx, w, at<float>(ws, L.logits),
+        return launch_router_tc(*c, x, w_gate, gate_bias, score_bias, idx, w,
+                                at<int>(ws, L.status), s);
+    return launch_router(*c, x, w_gate, gate_bias, score_bias, idx, w, at<float>(ws, L.logits),
                          at<int32_t>(ws, L.counters), router_ksplit(*c), s);
 }
 
 int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offsets,
                     const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
                     cudaStream_t s) {
+    const moe_config g = grouped_config(*c);  // the shared expert is expert E
     if (use_stream_path(c))
-        return cuda_status(launch_gate_up_stream(*c, x_perm, offsets, w_gate_up, s_gate_up, h, s));
+        return cuda_status(launch_gate_up_stream(g, x_perm, offsets, w_gate_up, s_gate_up, h, s));
     int* status = at<int>(ws, ws_layout(*c).status);
     if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
         if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
-        return cuda_status(launch_gate_up_gemm_pair_fp8(*c, x_perm, offsets, w_gate_up, s_gate_up,
+        return cuda_status(launch_gate_up_gemm_pair_fp8(g, x_perm, offsets, w_gate_up, s_gate_up,
                                                         h, status, s));
     }
     if (pair_gemm_supported(*c))
-        return cuda_status(launch_gate_up_gemm_pair(*c, x_perm, offsets, w_gate_up, packed(c), h, status, s));
-    return cuda_status(launch_gate_up_gemm(*c, x_perm, offsets, w_gate_up, h, status, s));
+        return cuda_status(
+            launch_gate_up_gemm_pair(g, x_perm, offsets, w_gate_up, packed(c), h, status, s));
+    return cuda_status(launch_gate_up_gemm(g, x_perm, offsets, w_gate_up, h, status, s));
 }
 
 // gate_up on token rows gathered by index: the bf16 SM-pair GEMM gathers the
@@ -116,8 +120,9 @@ int experts_gate_up_gather(const moe_config* c, const void* x, const int32_t* to
                            void* h, void* ws, cudaStream_t s) {
     const WsLayout L = ws_layout(*c);
     if (!use_stream_path(c) && !(c->flags & MOE_FLAG_FP8_WEIGHTS) && pair_gemm_supported(*c))
-        return cuda_status(launch_gate_up_gemm_pair_gather(*c, x, token_of_row, offsets, w_gate_up,
-                                                           packed(c), h, at<int>(ws, L.status), s));
+        return cuda_status(launch_gate_up_gemm_pair_gather(grouped_config(*c), x, token_of_row,
+                                                           offsets, w_gate_up, packed(c), h,
+                                                           at<int>(ws, L.status), s));
     void* xperm = at<void>(ws, L.xperm);
     MOE_TRY(cuda_status(launch_gather_rows(*c, x, token_of_row, offsets, xperm, s)));
     return experts_gate_up(c, xperm, offsets, w_gate_up, s_gate_up, h, ws, s);
@@ -125,17 +130,23 @@ int experts_gate_up_gather(const moe_config* c, const void* x, const int32_t* to
 
 int experts_down(const moe_config* c, const void* h, const int32_t* offsets, const void* w_down,
                  const float* s_down, void* y, void* ws, cudaStream_t s) {
+    const moe_config g = grouped_config(*c);
     if (use_stream_path(c))
-        return cuda_status(launch_down_stream(*c, h, offsets, w_down, s_down, y, s));
+        return cuda_status(launch_down_stream(g, h, offsets, w_down, s_down, y, s));
     int* status = at<int>(ws, ws_layout(*c).status);
     if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
         if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
         return cuda_status(
-            launch_down_gemm_pair_fp8(*c, h, offsets, w_down, s_down, y, status, s));
+            launch_down_gemm_pair_fp8(g, h, offsets, w_down, s_down, y, status, s));
     }
     if (pair_gemm_supported(*c))
-        return cuda_status(launch_down_gemm_pair(*c, h, offsets, w_down, packed(c), y, status, s));
-    return cuda_status(launch_down_gemm(*c, h, offsets, w_down, y, status, s));
+        return cuda_status(launch_down_gemm_pair(g, h, offsets, w_down, packed(c), y, status, s));
+    return cuda_status(launch_down_gemm(g, h, offsets, w_down, y, status, s));
+}
+
+// Batches of at most MOE_GATHER_MAX_SLOTS grouped token-slots gather in the GEMM.
+bool gather_batch(const moe_config* c) {
+    return (long long)c->T * (c->k + shared_slots(*c)) <= MOE_GATHER_MAX_SLOTS;
 }
 
 }  // namespace
@@ -154,14 +165,20 @@ int moe_workspace_init(const moe_config* cfg, void* ws, size_t ws_bytes, void* s
                                        static_cast<cudaStream_t>(stream)));
 }
 
-int moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
-              int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+int moe_route2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+               const float* score_bias, int32_t* topk_idx, float* topk_w, void* ws,
+               size_t ws_bytes, void* stream) {
     MOE_TRY(check_cfg(cfg));
     if (!x || !w_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_ws(cfg, ws, ws_bytes));
-    return cuda_status(route(cfg, x, w_gate, gate_bias, topk_idx, topk_w, ws,
+    return cuda_status(route(cfg, x, w_gate, gate_bias, score_bias, topk_idx, topk_w, ws,
                              static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+              int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+    return moe_route2(cfg, x, w_gate, gate_bias, nullptr, topk_idx, topk_w, ws, ws_bytes, stream);
 }
 
 int moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x, int32_t* counts,
@@ -250,9 +267,10 @@ int moe_combine(const moe_config* cfg, const void* y, const int32_t* row_of, con
                                       static_cast<cudaStream_t>(stream)));
 }
 
-int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
-                const void* w_gate_up, const float* s_gate_up, const void* w_down,
-                const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream) {
+int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+                 const float* score_bias, const void* w_gate_up, const float* s_gate_up,
+                 const void* w_down, const float* s_down, void* out, void* ws, size_t ws_bytes,
+                 void* stream) {
     MOE_TRY(check_cfg(cfg));
     if (!x || !w_gate || !out || !aligned16(x) || !aligned16(w_gate) || !aligned16(out))
         return MOE_ERR_INVALID_ARG;
@@ -271,8 +289,8 @@ int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const 
     void* h = at<void>(ws, L.h);
     void* y = at<void>(ws, L.y);
     MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.control_end, s)));
-    MOE_TRY(cuda_status(route(cfg, x, w_gate, gate_bias, idx, w, ws, s)));
-    if ((long long)cfg->T * cfg->k <= MOE_GATHER_MAX_SLOTS) {
+    MOE_TRY(cuda_status(route(cfg, x, w_gate, gate_bias, score_bias, idx, w, ws, s)));
+    if (gather_batch(cfg)) {
         int32_t* tok = at<int32_t>(ws, L.tok);
         MOE_TRY(cuda_status(
             launch_permute_index(*cfg, idx, counts, offsets, row_of, tok, hist, rank, s)));
@@ -287,6 +305,13 @@ int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const 
     return cuda_status(launch_combine(*cfg, y, row_of, w, out, s));
 }
 
+int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+                const void* w_gate_up, const float* s_gate_up, const void* w_down,
+                const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream) {
+    return moe_forward2(cfg, x, w_gate, gate_bias, nullptr, w_gate_up, s_gate_up, w_down, s_down,
+                        out, ws, ws_bytes, stream);
+}
+
 int moe_pack_weights(const moe_config* cfg, int which, const void* w, void* w_packed,
                      void* stream) {
     MOE_TRY(check_cfg(cfg));
@@ -296,11 +321,12 @@ int moe_pack_weights(const moe_config* cfg, int which, const void* w, void* w_pa
     if (!pair_gemm_supported(*cfg)) return MOE_ERR_UNSUPPORTED_SHAPE;
     const int rows = which == MOE_WEIGHTS_GATE_UP ? 2 * cfg->d_ff : cfg->d;
     const int cols = which == MOE_WEIGHTS_GATE_UP ? cfg->d : cfg->d_ff;
-    const size_t bytes = (size_t)cfg->E * rows * cols * 2;
+    const int experts = cfg->E + shared_slots(*cfg);  // the shared expert is packed too
+    const size_t bytes = (size_t)experts * rows * cols * 2;
     const char* a = static_cast<const char*>(w);
     const char* b = static_cast<const char*>(w_packed);
     if (a < b + bytes && b < a + bytes) return MOE_ERR_INVALID_ARG;  // overlap
-    return cuda_status(launch_pack_weights(cfg->E, rows, cols, w, w_packed,
+    return cuda_status(launch_pack_weights(experts, rows, cols, w, w_packed,
                                            static_cast<cudaStream_t>(stream)));
 }
 

@@ -36,6 +36,25 @@ namespace {
 
 constexpr int CH = kPermuteChunk;
 
+// The expert of token-slot s. Without a shared expert the slots are the
+// routing array itself (kk == k); with one, every token has kk = k + 1 slots
+// and its last slot is the shared expert e_shared.
+struct Slots {
+    const int* idx;  // [T, k]
+    int k, kk, e_shared;
+};
+
+__device__ __forceinline__ int slot_expert(const Slots& m, long s) {
+    if (m.kk == m.k) return m.idx[s];
+    const long t = s / m.kk;
+    const int j = (int)(s - t * m.kk);
+    return j < m.k ? m.idx[t * m.k + j] : m.e_shared;
+}
+
+inline Slots slots_of(const moe_config& c, const int32_t* idx) {
+    return Slots{idx, c.k, c.k + shared_slots(c), c.E};
+}
+
 // One warp copies a row of n16 16-byte vectors, eight loads in flight per lane.
 __device__ __forceinline__ void copy_row(uint4* __restrict__ dst, const uint4* __restrict__ src,
                                          int n16, int lane) {
@@ -58,8 +77,7 @@ constexpr int RW = 4;
 constexpr int SUB = CH / RW;
 
 __global__ void __launch_bounds__(RW * 32)
-permute_rank_kernel(const int* __restrict__ idx, long R, int E, int* __restrict__ hist,
-                    int* __restrict__ rank) {
+permute_rank_kernel(Slots sl, long R, int E, int* __restrict__ hist, int* __restrict__ rank) {
     __shared__ int cnt[RW][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < RW * 256; i += blockDim.x) cnt[i >> 8][i & 255] = 0;
@@ -67,7 +85,7 @@ permute_rank_kernel(const int* __restrict__ idx, long R, int E, int* __restrict_
     const long base = (long)blockIdx.x * CH + (long)warp * SUB;
     for (int g = 0; g < SUB; g += 32) {
         const long s = base + g + lane;
-        int e = (s < R) ? idx[s] : -1;
+        int e = (s < R) ? slot_expert(sl, s) : -1;
         if (e >= E) e = -1;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int before = (e >= 0) ? cnt[warp][e] : 0;
@@ -92,7 +110,7 @@ permute_rank_kernel(const int* __restrict__ idx, long R, int E, int* __restrict_
     for (int g = 0; g < SUB; g += 32) {
         const long s = base + g + lane;
         if (s < R) {
-            const int e = idx[s];
+            const int e = slot_expert(sl, s);
             if (e >= 0 && e < E) rank[s] += cnt[warp][e];
         }
     }
@@ -154,14 +172,14 @@ permute_scan_kernel(int* __restrict__ hist, int C, int E, int* __restrict__ coun
 }
 
 __global__ void __launch_bounds__(256)
-permute_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ hist,
-                       const int* __restrict__ rank, const int* __restrict__ offsets,
-                       const __nv_bfloat16* __restrict__ x, long R, int k, int E, int d,
-                       int* __restrict__ row_of, __nv_bfloat16* __restrict__ xperm) {
+permute_scatter_kernel(Slots sl, const int* __restrict__ hist, const int* __restrict__ rank,
+                       const int* __restrict__ offsets, const __nv_bfloat16* __restrict__ x,
+                       long R, int E, int d, int* __restrict__ row_of,
+                       __nv_bfloat16* __restrict__ xperm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long s = (long)blockIdx.x * 8 + warp;
     if (s >= R) return;
-    const int e = idx[s];
+    const int e = slot_expert(sl, s);
     if (e < 0 || e >= E) {
         if (lane == 0) row_of[s] = -1;
         return;
@@ -169,7 +187,7 @@ permute_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ hist
     const long c = s / CH;
     const int row = offsets[e] + hist[c * E + e] + rank[s];
     if (lane == 0) row_of[s] = row;
-    const long t = s / k;
+    const long t = s / sl.kk;
     const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
     uint4* dst = reinterpret_cast<uint4*>(xperm + (long)row * d);
     copy_row(dst, src, d / 8, lane);
@@ -179,19 +197,19 @@ permute_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ hist
 // token_of_row[row] = t, for expert GEMMs that gather the token rows
 // themselves.
 __global__ void __launch_bounds__(256)
-permute_index_kernel(const int* __restrict__ idx, const int* __restrict__ hist,
-                     const int* __restrict__ rank, const int* __restrict__ offsets, long R, int k,
-                     int E, int* __restrict__ row_of, int* __restrict__ token_of_row) {
+permute_index_kernel(Slots sl, const int* __restrict__ hist, const int* __restrict__ rank,
+                     const int* __restrict__ offsets, long R, int E, int* __restrict__ row_of,
+                     int* __restrict__ token_of_row) {
     const long s = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= R) return;
-    const int e = idx[s];
+    const int e = slot_expert(sl, s);
     if (e < 0 || e >= E) {
         row_of[s] = -1;
         return;
     }
     const int row = offsets[e] + hist[(s / CH) * E + e] + rank[s];
     row_of[s] = row;
-    token_of_row[row] = (int)(s / k);
+    token_of_row[row] = (int)(s / sl.kk);
 }
 
 // The whole index-only grouping in one CTA for small batches (R <= SW * 128
@@ -204,7 +222,7 @@ constexpr int SW = 32;  // warps of the small-batch kernel
 constexpr long kSmallSlots = SW * 128;
 
 __global__ void __launch_bounds__(SW * 32)
-permute_small_kernel(const int* __restrict__ idx, long R, int k, int E, int* __restrict__ counts,
+permute_small_kernel(Slots sl, long R, int E, int* __restrict__ counts,
                      int* __restrict__ offsets, int* __restrict__ row_of,
                      int* __restrict__ token_of_row) {
     __shared__ int cnt[SW][256];
@@ -216,7 +234,7 @@ permute_small_kernel(const int* __restrict__ idx, long R, int k, int E, int* __r
     const long s0 = (long)warp * per;
     for (int g = 0; g < per; g += 32) {
         const long s = s0 + g + lane;
-        int e = (s < R) ? idx[s] : -1;
+        int e = (s < R) ? slot_expert(sl, s) : -1;
         if (e >= E) e = -1;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] += __popc(peers);
@@ -265,7 +283,7 @@ permute_small_kernel(const int* __restrict__ idx, long R, int k, int E, int* __r
     __syncthreads();
     for (int g = 0; g < per; g += 32) {
         const long s = s0 + g + lane;
-        int e = (s < R) ? idx[s] : -1;
+        int e = (s < R) ? slot_expert(sl, s) : -1;
         if (e >= E) e = -1;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int before = (e >= 0) ? cnt[warp][e] : 0;
@@ -278,7 +296,7 @@ permute_small_kernel(const int* __restrict__ idx, long R, int k, int E, int* __r
             } else {
                 const int row = base[e] + before + __popc(peers & ((1u << lane) - 1u));
                 row_of[s] = row;
-                token_of_row[row] = (int)(s / k);
+                token_of_row[row] = (int)(s / sl.kk);
             }
         }
     }
@@ -302,25 +320,28 @@ gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ 
 cudaError_t launch_permute_index(const moe_config& c, const int32_t* idx, int32_t* counts,
                                  int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
                                  int32_t* hist, int32_t* rank, cudaStream_t s) {
-    const long R = (long)c.T * c.k;
+    const moe_config g = grouped_config(c);
+    const Slots sl = slots_of(c, idx);
+    const long R = (long)g.T * g.k;
     if (R <= kSmallSlots) {
-        permute_small_kernel<<<1, SW * 32, 0, s>>>(idx, R, c.k, c.E, counts, offsets, row_of,
+        permute_small_kernel<<<1, SW * 32, 0, s>>>(sl, R, g.E, counts, offsets, row_of,
                                                    token_of_row);
         return cudaGetLastError();
     }
-    const int C = n_permute_chunks(c);
-    permute_rank_kernel<<<C, RW * 32, 0, s>>>(idx, R, c.E, hist, rank);
-    permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, c.E, counts, offsets);
-    permute_index_kernel<<<(unsigned)((R + 255) / 256), 256, 0, s>>>(idx, hist, rank, offsets, R,
-                                                                     c.k, c.E, row_of, token_of_row);
+    const int C = n_permute_chunks(g);
+    permute_rank_kernel<<<C, RW * 32, 0, s>>>(sl, R, g.E, hist, rank);
+    permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, g.E, counts, offsets);
+    permute_index_kernel<<<(unsigned)((R + 255) / 256), 256, 0, s>>>(sl, hist, rank, offsets, R,
+                                                                     g.E, row_of, token_of_row);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const moe_config& c, const void* x, const int32_t* token_of_row,
                                const int32_t* offsets, void* x_perm, cudaStream_t s) {
-    const long R = (long)c.T * c.k;
+    const moe_config g = grouped_config(c);
+    const long R = (long)g.T * g.k;
     gather_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), token_of_row, offsets, R, c.E, c.d,
+        static_cast<const __nv_bfloat16*>(x), token_of_row, offsets, R, g.E, c.d,
         static_cast<__nv_bfloat16*>(x_perm));
     return cudaGetLastError();
 }
@@ -328,12 +349,14 @@ cudaError_t launch_gather_rows(const moe_config& c, const void* x, const int32_t
 cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
                            int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,
                            int32_t* rank, cudaStream_t s) {
-    const long R = (long)c.T * c.k;
-    const int C = n_permute_chunks(c);
-    permute_rank_kernel<<<C, RW * 32, 0, s>>>(idx, R, c.E, hist, rank);
-    permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, c.E, counts, offsets);
+    const moe_config g = grouped_config(c);
+    const Slots sl = slots_of(c, idx);
+    const long R = (long)g.T * g.k;
+    const int C = n_permute_chunks(g);
+    permute_rank_kernel<<<C, RW * 32, 0, s>>>(sl, R, g.E, hist, rank);
+    permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, g.E, counts, offsets);
     permute_scatter_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
-        idx, hist, rank, offsets, static_cast<const __nv_bfloat16*>(x), R, c.k, c.E, c.d, row_of,
+        sl, hist, rank, offsets, static_cast<const __nv_bfloat16*>(x), R, g.E, c.d, row_of,
         static_cast<__nv_bfloat16*>(x_perm));
     return cudaGetLastError();
 }

@@ -17,7 +17,9 @@
 // of a token group to finish (an arrival counter, no waiting) sums the slices
 // in z order and runs the selection: one warp per token, k rounds of a
 // warp-wide argmax over the (biased) logits -- the sigmoid is increasing, so
-// this selects the k largest scores -- and the sigmoid of the k selected.
+// this selects the k largest scores -- and the sigmoid of the k selected. With
+// an e_score_correction_bias ("Tencent Hy3-295B 架构深度拆解" §4.1 step 2) the
+// choice ranks sigmoid + bias and the weights renormalise the sigmoid scores.
 #include "common.cuh"
 #include "internal.h"
 
@@ -41,7 +43,8 @@ __device__ __forceinline__ void load_w(uint4 (&u)[EPW], const __nv_bfloat16* __r
 
 __global__ void __launch_bounds__(RWARPS * 32, kRouterCtasPerSm)
 router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wg,
-              const float* __restrict__ bias, int T, int d, int E, int k, float scale,
+              const float* __restrict__ bias, const float* __restrict__ sbias, int T, int d,
+              int E, int k, float scale,
               float* __restrict__ logits, int* __restrict__ counters, int* __restrict__ idx_out,
               float* __restrict__ w_out) {
     __shared__ __align__(16) float xs[RT][KC];
@@ -158,7 +161,20 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
                 sc[q] = -INFINITY;
             }
         }
-        warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k);
+        if (sbias) {
+            // e_score_correction_bias: the choice ranks sigmoid + bias, the
+            // weights renormalise the sigmoid scores of the chosen experts
+            float prob[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = lane + 32 * q;
+                prob[q] = (e < E) ? sigmoidf_acc(sc[q]) : 0.f;
+                sc[q] = (e < E) ? prob[q] + sbias[e] : -INFINITY;
+            }
+            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k, prob);
+        } else {
+            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k);
+        }
     }
     if (threadIdx.x == 0) counters[blockIdx.y] = 0;
 }
@@ -166,12 +182,12 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 }  // namespace
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
-                          const float* gate_bias, int32_t* idx, float* w, float* logits,
-                          int32_t* counters, int ksplit, cudaStream_t s) {
+                          const float* gate_bias, const float* score_bias, int32_t* idx, float* w,
+                          float* logits, int32_t* counters, int ksplit, cudaStream_t s) {
     dim3 grid((c.E + RE - 1) / RE, n_router_groups(c), ksplit);
     router_kernel<<<grid, RWARPS * 32, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_gate), gate_bias,
-        c.T, c.d, c.E, c.k, c.scale, logits, counters, idx, w);
+        score_bias, c.T, c.d, c.E, c.k, c.scale, logits, counters, idx, w);
     return cudaGetLastError();
 }
 

@@ -50,6 +50,7 @@ struct Ctrl {
     int abort;
     // the logit bias (0 where none, and past E: the selection reads 8 at a time)
     alignas(16) float bias[256 + 8];
+    alignas(16) float sbias[256 + 8];  // the e_score_correction_bias, when given
 };
 
 constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + (int)sizeof(Ctrl);
@@ -70,14 +71,17 @@ static_assert(BM * logit_stride(256) * 4 + 32 <= STAGES * STAGE_BYTES, "logit ro
 // of a warp-wide argmax, one token at a time per warp) measured ~3 us per
 // token here, far slower than this scan; the bias is staged in shared memory
 // (per-element global loads of it made the scan ~3x slower).
-template <int K>
-__device__ __forceinline__ void thread_select_topk(const float* row, const float* sbias, int E,
-                                                   float scale, int* __restrict__ idx_out,
+template <int K, bool SB>
+__device__ __forceinline__ void thread_select_topk(const float* row, const float* sbias,
+                                                   const float* cbias, int E, float scale,
+                                                   int* __restrict__ idx_out,
                                                    float* __restrict__ w_out) {
-    float v[K];
+    // SB: rank sigmoid(logit) + cbias (the e_score_correction_bias) and keep
+    // the sigmoid scores p of the list for the weights
+    float v[K], p[K];
     int id[K];
 #pragma unroll
-    for (int j = 0; j < K; ++j) { v[j] = -INFINITY; id[j] = 0; }
+    for (int j = 0; j < K; ++j) { v[j] = -INFINITY; p[j] = 0.f; id[j] = 0; }
     for (int e0 = 0; e0 < E; e0 += 8) {
         // 8 logits and their biases in flight, then visited in increasing order
         const float4 a0 = *reinterpret_cast<const float4*>(row + e0);
@@ -89,14 +93,20 @@ __device__ __forceinline__ void thread_select_topk(const float* row, const float
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int e = e0 + u;
-            const float z = z8[u];
+            float z = z8[u], pz = 0.f;
+            if (SB && e < E) {
+                pz = sigmoidf_acc(z);
+                z = pz + cbias[e];
+            }
             if (e < E && z > v[K - 1]) {
                 v[K - 1] = z;
+                p[K - 1] = pz;
                 id[K - 1] = e;
 #pragma unroll
                 for (int j = K - 1; j > 0; --j) {
                     if (v[j] > v[j - 1]) {
                         const float tv = v[j]; v[j] = v[j - 1]; v[j - 1] = tv;
+                        const float tp = p[j]; p[j] = p[j - 1]; p[j - 1] = tp;
                         const int ti = id[j]; id[j] = id[j - 1]; id[j - 1] = ti;
                     }
                 }
@@ -106,7 +116,7 @@ __device__ __forceinline__ void thread_select_topk(const float* row, const float
     float sum = 0.f;
 #pragma unroll
     for (int j = 0; j < K; ++j) {
-        v[j] = sigmoidf_acc(v[j]);
+        v[j] = SB ? p[j] : sigmoidf_acc(v[j]);
         sum += v[j];
     }
 #pragma unroll
@@ -121,7 +131,8 @@ __device__ __forceinline__ void thread_select_topk(const float* row, const float
 template <int S>
 __global__ void __launch_bounds__(THREADS, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                 const float* __restrict__ bias, int T, int d, int E, int k, int n_pad,
+                 const float* __restrict__ bias, const float* __restrict__ sbias, int T,
+                 int d, int E, int k, int n_pad,
                  float scale, int* __restrict__ idx_out, float* __restrict__ w_out,
                  int* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
@@ -137,8 +148,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     float* red = reinterpret_cast<float*>(smem);  // [128][es], reuses the stage ring
 
     if (warp >= 2) {
-        for (int e = threadIdx.x - 64; e < 256 + 8; e += 128)
+        for (int e = threadIdx.x - 64; e < 256 + 8; e += 128) {
             c.bias[e] = (bias && e < E) ? bias[e] : 0.f;
+            c.sbias[e] = (sbias && e < E) ? sbias[e] : 0.f;
+        }
     }
     if (warp == 0 && lane == 0) {
         c.abort = 0;
@@ -298,15 +311,28 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const float* rw = red + (split * ROWS + rr) * es;
             int* io = idx_out + t * k;
             float* wo = w_out + t * k;
-            switch (k) {
-                case 1: thread_select_topk<1>(rw, c.bias, E, scale, io, wo); break;
-                case 2: thread_select_topk<2>(rw, c.bias, E, scale, io, wo); break;
-                case 3: thread_select_topk<3>(rw, c.bias, E, scale, io, wo); break;
-                case 4: thread_select_topk<4>(rw, c.bias, E, scale, io, wo); break;
-                case 5: thread_select_topk<5>(rw, c.bias, E, scale, io, wo); break;
-                case 6: thread_select_topk<6>(rw, c.bias, E, scale, io, wo); break;
-                case 7: thread_select_topk<7>(rw, c.bias, E, scale, io, wo); break;
-                default: thread_select_topk<8>(rw, c.bias, E, scale, io, wo); break;
+            if (sbias) {
+                switch (k) {
+                    case 1: thread_select_topk<1, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 2: thread_select_topk<2, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 3: thread_select_topk<3, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 4: thread_select_topk<4, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 5: thread_select_topk<5, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 6: thread_select_topk<6, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 7: thread_select_topk<7, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    default: thread_select_topk<8, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                }
+            } else {
+                switch (k) {
+                    case 1: thread_select_topk<1, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 2: thread_select_topk<2, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 3: thread_select_topk<3, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 4: thread_select_topk<4, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 5: thread_select_topk<5, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 6: thread_select_topk<6, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    case 7: thread_select_topk<7, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                    default: thread_select_topk<8, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
+                }
             }
         }
     }
@@ -363,8 +389,8 @@ namespace {
 
 template <int S>
 cudaError_t launch_s(dim3 grid, const CUtensorMap& mx, const CUtensorMap& mw, const moe_config& c,
-                     int n_pad, const float* gate_bias, int32_t* idx, float* w, int* status,
-                     cudaStream_t s) {
+                     int n_pad, const float* gate_bias, const float* score_bias, int32_t* idx,
+                     float* w, int* status, cudaStream_t s) {
     cudaError_t err = cudaFuncSetAttribute(router_tc_kernel<S>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (err != cudaSuccess) return err;
@@ -380,15 +406,15 @@ cudaError_t launch_s(dim3 grid, const CUtensorMap& mx, const CUtensorMap& mw, co
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, router_tc_kernel<S>, mx, mw, gate_bias, c.T, c.d, c.E, c.k,
-                              n_pad, c.scale, idx, w, status);
+    return cudaLaunchKernelEx(&cfg, router_tc_kernel<S>, mx, mw, gate_bias, score_bias, c.T, c.d,
+                              c.E, c.k, n_pad, c.scale, idx, w, status);
 }
 
 }  // namespace
 
 cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_gate,
-                             const float* gate_bias, int32_t* idx, float* w, int* status,
-                             cudaStream_t s) {
+                             const float* gate_bias, const float* score_bias, int32_t* idx,
+                             float* w, int* status, cudaStream_t s) {
     const int tiles = (c.T + BM - 1) / BM;
     const int S = router_splits(c.T, c.d);
     const int n_pad = (c.E + 15) & ~15;
@@ -398,10 +424,10 @@ cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_g
     const dim3 grid(tiles, S);
     cudaError_t err;
     switch (S) {
-        case 1: err = launch_s<1>(grid, mx, mw, c, n_pad, gate_bias, idx, w, status, s); break;
-        case 2: err = launch_s<2>(grid, mx, mw, c, n_pad, gate_bias, idx, w, status, s); break;
-        case 4: err = launch_s<4>(grid, mx, mw, c, n_pad, gate_bias, idx, w, status, s); break;
-        default: err = launch_s<8>(grid, mx, mw, c, n_pad, gate_bias, idx, w, status, s); break;
+        case 1: err = launch_s<1>(grid, mx, mw, c, n_pad, gate_bias, score_bias, idx, w, status, s); break;
+        case 2: err = launch_s<2>(grid, mx, mw, c, n_pad, gate_bias, score_bias, idx, w, status, s); break;
+        case 4: err = launch_s<4>(grid, mx, mw, c, n_pad, gate_bias, score_bias, idx, w, status, s); break;
+        default: err = launch_s<8>(grid, mx, mw, c, n_pad, gate_bias, score_bias, idx, w, status, s); break;
     }
     if (err != cudaSuccess) return err;
     return cudaGetLastError();

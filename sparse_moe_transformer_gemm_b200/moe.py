@@ -30,13 +30,15 @@ MOE_FLAG_FP8_WEIGHTS = 0x1
 MOE_FLAG_STREAM_PATH = 0x2
 MOE_FLAG_GEMM_PATH = 0x4
 MOE_FLAG_PACKED_WEIGHTS = 0x8
+MOE_FLAG_SHARED_EXPERT = 0x10
 MOE_WEIGHTS_GATE_UP = 0
 MOE_WEIGHTS_DOWN = 1
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
             "moe_permute_index", "moe_expert_gate_up", "moe_expert_gate_up_gather",
             "moe_expert_down", "moe_experts", "moe_combine", "moe_forward", "moe_read_status",
-            "moe_status_string", "moe_route_noalloc", "moe_pack_weights")
+            "moe_status_string", "moe_route_noalloc", "moe_pack_weights", "moe_route2",
+            "moe_forward2")
 
 MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 # batches of at most this many token-slots (T*k) gather their token rows inside
@@ -90,6 +92,8 @@ def lib() -> ctypes.CDLL:
         "moe_status_string": (ctypes.c_char_p, [I]),
         "moe_route_noalloc": (I, [C, P, P, P, P, P, P]),
         "moe_pack_weights": (I, [C, I, P, P, P]),
+        "moe_route2": (I, [C, P, P, P, P, P, P, P, S, P]),
+        "moe_forward2": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -100,12 +104,15 @@ def lib() -> ctypes.CDLL:
 
 
 def config(T: int, d: int, E: int, k: int, d_ff: int, scale: float = 2.826, fp8: bool = False,
-           path: Optional[str] = None, packed: bool = False) -> MoeConfig:
+           path: Optional[str] = None, packed: bool = False, shared: bool = False) -> MoeConfig:
     """Build a moe_config. path: None (automatic), "stream" or "gemm"; packed: the
-    bf16 expert weights are in moe_pack_weights' layout."""
+    bf16 expert weights are in moe_pack_weights' layout; shared: expert E of the
+    weight arrays is a shared expert."""
     flags = MOE_FLAG_FP8_WEIGHTS if fp8 else 0
     if packed:
         flags |= MOE_FLAG_PACKED_WEIGHTS
+    if shared:
+        flags |= MOE_FLAG_SHARED_EXPERT
     if path == "stream":
         flags |= MOE_FLAG_STREAM_PATH
     elif path == "gemm":
@@ -212,6 +219,20 @@ def moe_forward(cfg, x, w_gate, gate_bias, w_gate_up, s_gate_up, w_down, s_down,
                              _s(stream)))
 
 
+def moe_route2(cfg, x, w_gate, gate_bias, score_bias, topk_idx, topk_w, ws, stream=None) -> None:
+    _check("moe_route2", lib().moe_route2(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
+                                          _p(score_bias), _p(topk_idx), _p(topk_w), _p(ws),
+                                          ws.numel(), _s(stream)))
+
+
+def moe_forward2(cfg, x, w_gate, gate_bias, score_bias, w_gate_up, s_gate_up, w_down, s_down,
+                 out, ws, stream=None) -> None:
+    _check("moe_forward2",
+           lib().moe_forward2(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
+                              _p(score_bias), _p(w_gate_up), _p(s_gate_up), _p(w_down),
+                              _p(s_down), _p(out), _p(ws), ws.numel(), _s(stream)))
+
+
 def moe_route_noalloc(cfg, x, w_gate, gate_bias, topk_idx, topk_w, stream=None) -> None:
     """moe_route without a workspace, for callers that cannot allocate device
     memory; the scratch is a fixed 2 MiB device array inside the library."""
@@ -231,16 +252,24 @@ def moe_read_status(ws, stream=None) -> int:
 
 
 def layer_args(layer: dict):
-    """(w_gate_up, s_gate_up, w_down, s_down) of a synthetic layer dict, FP8 or bf16."""
-    if layer["cfg"].fp8:
-        return layer["q_gate_up"], layer["s_gate_up"], layer["q_down"], layer["s_down"]
-    return layer["w_gate_up"], None, layer["w_down"], None
+    """(w_gate_up, s_gate_up, w_down, s_down) of a synthetic layer dict, FP8 or bf16;
+    with a shared expert, its weights follow the routed ones as expert E."""
+    cfg = layer["cfg"]
+    if cfg.fp8:
+        args = [layer["q_gate_up"], layer["s_gate_up"], layer["q_down"], layer["s_down"]]
+        sh = ("q_shared_gate_up", "s_shared_gate_up", "q_shared_down", "s_shared_down")
+    else:
+        args = [layer["w_gate_up"], None, layer["w_down"], None]
+        sh = ("w_shared_gate_up", None, "w_shared_down", None)
+    if getattr(cfg, "shared", False):
+        args = [a if n is None else torch.cat([a, layer[n][None]]) for a, n in zip(args, sh)]
+    return tuple(args)
 
 
 def config_of(shape, path: Optional[str] = None, packed: bool = False) -> MoeConfig:
     """moe_config for a synthetic LayerShape."""
     return config(shape.T, shape.d, shape.E, shape.k, shape.F, shape.scale, shape.fp8, path,
-                  packed)
+                  packed, getattr(shape, "shared", False))
 
 
 def pack_layer_weights(cfg: MoeConfig, w_gate_up: torch.Tensor, w_down: torch.Tensor,

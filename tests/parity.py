@@ -30,7 +30,8 @@ def gpu_route(layer, path=None):
     ws = moe.workspace(cfg)
     idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
     w = torch.empty((T, k), dtype=torch.float32, device="cuda")
-    moe.moe_route(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"), idx, w, ws)
+    moe.moe_route2(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"),
+                   layer.get("score_bias"), idx, w, ws)
     torch.cuda.synchronize()
     assert moe.moe_read_status(ws) == moe.MOE_OK
     return idx.cpu().numpy(), w.cpu().numpy()
@@ -43,8 +44,8 @@ def gpu_forward(layer, path=None, ws=None, out=None):
         ws = moe.workspace(cfg)
     if out is None:
         out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
-    moe.moe_forward(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"),
-                    *moe.layer_args(layer), out, ws)
+    moe.moe_forward2(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"),
+                     layer.get("score_bias"), *moe.layer_args(layer), out, ws)
     torch.cuda.synchronize()
     assert moe.moe_read_status(ws) == moe.MOE_OK
     return out
@@ -82,13 +83,20 @@ def check_near_tie_selection(gpu_idx, scores, t, k):
 
 def oracle_out_with_selection(O, t, experts):
     """Oracle output of token t when it is routed to ``experts`` (weights from the
-    oracle's fp64 scores, renormalised over that set)."""
+    oracle's fp64 sigmoid scores, renormalised over that set; the shared expert,
+    if any, added last with weight 1)."""
     scores = oracle.route(O.x[t:t + 1], O.wg, O.k, O.scale, O.gate_bias, want_scores=True)["scores"]
     experts = np.asarray(experts, np.int32)
     xrows = np.repeat(O.x[t:t + 1], len(experts), axis=0)
     y = oracle.expert_rows(xrows, experts, O.wgu, O.wd, O.s_gu, O.s_d)
     s = scores[0, experts]
     w = O.scale * s / s.sum()
+    if O.sh_wgu is not None:
+        y_sh = oracle.expert_rows(O.x[t:t + 1], np.zeros(1, np.int32), O.sh_wgu[None],
+                                  O.sh_wd[None], None if O.sh_s_gu is None else O.sh_s_gu[None],
+                                  None if O.sh_s_d is None else O.sh_s_d[None])
+        y = np.concatenate([y, y_sh])
+        w = np.concatenate([w, [1.0]])
     return oracle.combine(y[None], w[None])[0]
 
 

@@ -35,7 +35,7 @@ def test_header_constants_match_the_binding():
     m = re.search(r"#define MOE_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
     assert m and int(m.group(1)) << int(m.group(2)) == moe.MOE_NOALLOC_SCRATCH_BYTES
     for name in ("MOE_FLAG_FP8_WEIGHTS", "MOE_FLAG_STREAM_PATH", "MOE_FLAG_GEMM_PATH",
-                 "MOE_FLAG_PACKED_WEIGHTS"):
+                 "MOE_FLAG_PACKED_WEIGHTS", "MOE_FLAG_SHARED_EXPERT"):
         m = re.search(r"#define %s (0x[0-9a-f]+)u" % name, text)
         assert m and int(m.group(1), 16) == getattr(moe, name), name
     for name in ("MOE_WEIGHTS_GATE_UP", "MOE_WEIGHTS_DOWN"):
@@ -51,6 +51,15 @@ def test_packed_weights_flag_rules(lib):
     # the tensor-core pair kernels need d and d_ff multiples of 256
     assert moe.moe_workspace_size(moe.config(**{**HY3, "d": 384}, packed=True)) == 0
     assert moe.moe_workspace_size(moe.config(**{**HY3, "d": 384})) > 0
+
+
+def test_shared_expert_flag_rules(lib):
+    plain = moe.moe_workspace_size(moe.config(**HY3))
+    shared = moe.moe_workspace_size(moe.config(**HY3, shared=True))
+    assert shared > plain  # one more slot per token in the grouped buffers
+    assert moe.moe_workspace_size(moe.config(**{**HY3, "E": 255}, shared=True)) > 0
+    assert moe.moe_workspace_size(moe.config(**{**HY3, "E": 256}, shared=True)) == 0
+    assert moe.moe_workspace_size(moe.config(**{**HY3, "E": 256})) > 0
 
 
 def test_pack_weights_rejects_bad_arguments(lib):
@@ -174,6 +183,8 @@ def test_unsupported_shape_is_reported_by_every_entry_point(lib):
         "moe_combine": (f, f, f, f, f, 1 << 30, None),
         "moe_forward": (f, f, None, f, None, f, None, f, f, 1 << 30, None),
         "moe_pack_weights": (moe.MOE_WEIGHTS_GATE_UP, f, P(FAKE + (1 << 34)), None),
+        "moe_route2": (f, f, None, None, f, f, f, 1 << 30, None),
+        "moe_forward2": (f, f, None, None, f, None, f, None, f, f, 1 << 30, None),
     }
     for fn, args in cases.items():
         assert _call(fn, ctypes.byref(cfg), *args) == moe.MOE_ERR_UNSUPPORTED_SHAPE, fn

@@ -248,6 +248,84 @@ def test_packed_weights_give_identical_outputs(shape):
     _free(layer, gu, dn)
 
 
+# The complete Hy3 MoE block: e_score_correction_bias (choice only) and one
+# shared expert (expert E of the weights, weight 1, added last in the combine).
+BLOCK = {
+    # pair GEMMs, tensor-core router
+    "block_pair": LayerShape(T=200, d=512, E=16, k=4, F=512, shared=True, score_bias_std=0.05),
+    # single-SM GEMMs (d_ff % 256 != 0), tensor-core router
+    "block_ragged": LayerShape(T=300, d=512, E=32, k=8, F=384, shared=True,
+                               score_bias_std=0.05),
+    # CUDA-core router (k > 8)
+    "block_k12": LayerShape(T=100, d=256, E=32, k=12, F=128, shared=True, score_bias_std=0.05),
+    # FP8 weights for the routed and the shared expert
+    "block_fp8": LayerShape(T=333, d=768, E=24, k=6, F=512, fp8=True, shared=True,
+                            score_bias_std=0.05),
+    # T*(k+1) = 6300 slots: the permuted-copy grouping
+    "block_copy": LayerShape(T=700, d=512, E=16, k=8, F=256, shared=True, score_bias_std=0.05),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BLOCK))
+@pytest.mark.parametrize("path", [None, "stream", "gemm"])
+def test_complete_block_every_token(name, path):
+    sh = BLOCK[name]
+    if path == "gemm" and sh.fp8 and (sh.d % 256 or sh.F % 256):
+        pytest.skip("FP8 weights on the tensor cores need d and d_ff multiples of 256")
+    layer = make_layer(sh, seed=31, device="cuda")
+    route = parity.gpu_route(layer, path)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias, score_bias=O.score_bias)
+    parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer, path)
+    res = parity.check_forward(layer, out, None, route)
+    print(name, path, res)
+
+
+def test_complete_hy3_block_decode():
+    """Hy3 shapes with the shared expert and a score bias: every token's routing
+    and output (decode, so the in-GEMM row gather on 193 experts)."""
+    shape = dataclasses.replace(CONFIGS["decode"], shared=True, score_bias_std=0.05)
+    layer = make_layer(shape, seed=3, device="cuda")
+    route = parity.gpu_route(layer)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias, score_bias=O.score_bias)
+    near = parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer)
+    res = parity.check_forward(layer, out, None, route)
+    print("hy3 block decode, near ties:", len(near), res)
+    _free(layer, out)
+
+
+def test_route2_without_score_bias_is_moe_route_bitwise():
+    layer = make_layer(SMALL["pair_small"], seed=6, device="cuda", with_experts=False)
+    a = parity.gpu_route(layer)
+    cfg = moe.config_of(layer["cfg"])
+    ws = moe.workspace(cfg)
+    T, k = layer["cfg"].T, layer["cfg"].k
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_route(cfg, layer["x"], layer["w_gate"], None, idx, w, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(a[0], idx.cpu().numpy()) and np.array_equal(a[1], w.cpu().numpy())
+
+
+def test_complete_block_with_packed_weights_is_bitwise_the_same():
+    shape = BLOCK["block_pair"]
+    layer = make_layer(shape, seed=8, device="cuda")
+    want = parity.gpu_forward(layer).clone()
+    cfg = moe.config_of(shape, packed=True)
+    wgu, _, wd, _ = moe.layer_args(layer)
+    gu, dn = moe.pack_layer_weights(cfg, wgu, wd)
+    ws = moe.workspace(cfg)
+    out = torch.empty_like(want)
+    moe.moe_forward2(cfg, layer["x"], layer["w_gate"], None, layer["score_bias"], gu, None, dn,
+                     None, out, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_status(ws) == moe.MOE_OK
+    assert torch.equal(out, want)
+
+
 def test_fp32_combine_keeps_small_terms():
     """Hy3 commentary §2.3 example: one branch output 8.2 and seven of 0.03 (all
     already bf16). An fp32 sum gives 8.375 after the cast; a bf16 running sum
