@@ -32,6 +32,9 @@
  *     token with weight 1): step 6 becomes
  *       out_i = bf16_rne( sum_j w_j * y_{j,i} + y_shared_i ),
  *     the shared term added last, inside the same fp64 sum.
+ * and route_norm (Flash QA Q4.9): the router scores an RMS-normalised copy of
+ * the token, xn_c = x_c / sqrt(mean_c' x_c'^2 + eps) * g_c (g: the norm's
+ * weight); step 1 uses xn in place of x, the experts still take x.
  *
  * Every sum is a plain left-to-right fp64 loop; inputs are bf16 bit patterns
  * (or e4m3 codes with fp32 scales) widened exactly to double. The only
@@ -159,16 +162,28 @@ static int by_score_then_index(const void* pa, const void* pb)
  * and (k+1)-th largest key (+inf when k == E). score_bias may be NULL. */
 static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
                         const uint16_t* wg, const float* gate_bias, const float* score_bias,
-                        int32_t* idx, double* w, double* logits_out, double* scores_out,
-                        double* gap)
+                        const float* norm_w, double norm_eps, int32_t* idx, double* w,
+                        double* logits_out, double* scores_out, double* gap)
 {
     scored_expert* order = (scored_expert*)malloc(sizeof(scored_expert) * (size_t)E);
+    double* xr = (double*)malloc(sizeof(double) * (size_t)d);
     double sel_sum = 0.0;
     int e, c, j;
+    for (c = 0; c < d; ++c)
+        xr[c] = bf16_to_double(xrow[c]);
+    if (norm_w) {
+        /* route_norm: RMSNorm of the token for the router only */
+        double ms = 0.0, inv;
+        for (c = 0; c < d; ++c)
+            ms += xr[c] * xr[c];
+        inv = 1.0 / sqrt(ms / d + norm_eps);
+        for (c = 0; c < d; ++c)
+            xr[c] = xr[c] * inv * (double)norm_w[c];
+    }
     for (e = 0; e < E; ++e) {
         double logit = 0.0;
         for (c = 0; c < d; ++c)
-            logit += bf16_to_double(xrow[c]) * bf16_to_double(wg[(long)e * d + c]);
+            logit += xr[c] * bf16_to_double(wg[(long)e * d + c]);
         if (gate_bias)
             logit += (double)gate_bias[e];
         order[e].s = sigmoid(logit);
@@ -187,6 +202,7 @@ static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
         w[j] = scale * order[j].s / sel_sum;
     }
     *gap = (k < E) ? order[k - 1].key - order[k].key : INFINITY;
+    free(xr);
     free(order);
 }
 
@@ -290,18 +306,20 @@ void oracle_double_from_e4m3(const uint8_t* q, double* out, long n)
         out[i] = e4m3_to_double(q[i]);
 }
 
-/* Steps 1-4 for tokens [0, T), with the optional score bias [E] (NULL: none).
+/* Steps 1-4 for tokens [0, T), with the optional score bias [E] (NULL: none)
+ * and route_norm weight [d] (NULL: no route_norm; norm_eps its epsilon).
  * logits/scores may be NULL ([T, E] otherwise). */
 int oracle_route2(int T, int d, int E, int k, double scale, const uint16_t* x,
                   const uint16_t* wg, const float* gate_bias, const float* score_bias,
-                  int32_t* idx, double* w, double* logits, double* scores, double* gap)
+                  const float* norm_w, double norm_eps, int32_t* idx, double* w, double* logits,
+                  double* scores, double* gap)
 {
     long t;
-    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E)
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || (norm_w && !(norm_eps > 0.0)))
         return -1;
 #pragma omp parallel for schedule(dynamic, 4)
     for (t = 0; t < T; ++t)
-        route_token(d, E, k, scale, x + t * (long)d, wg, gate_bias, score_bias,
+        route_token(d, E, k, scale, x + t * (long)d, wg, gate_bias, score_bias, norm_w, norm_eps,
                     idx + t * (long)k, w + t * (long)k, logits ? logits + t * (long)E : NULL,
                     scores ? scores + t * (long)E : NULL, gap + t);
     return 0;
@@ -312,7 +330,8 @@ int oracle_route(int T, int d, int E, int k, double scale, const uint16_t* x,
                  const uint16_t* wg, const float* gate_bias, int32_t* idx, double* w,
                  double* logits, double* scores, double* gap)
 {
-    return oracle_route2(T, d, E, k, scale, x, wg, gate_bias, NULL, idx, w, logits, scores, gap);
+    return oracle_route2(T, d, E, k, scale, x, wg, gate_bias, NULL, NULL, 0.0, idx, w, logits,
+                         scores, gap);
 }
 
 /* Step 5 for n (row, expert) pairs: rows of xrows [n, d], experts[n]. h [n, F]
@@ -337,6 +356,7 @@ int oracle_expert_rows(int n, int d, int F, const uint16_t* xrows, const int32_t
  * out_bf16 [n, d], idx [n, k], w [n, k], gap [n]. */
 int oracle_forward_tokens2(int T, int d, int E, int k, int F, double scale, const uint16_t* x,
                            const uint16_t* wg, const float* gate_bias, const float* score_bias,
+                           const float* norm_w, double norm_eps,
                            const void* wgu, const float* s_gu, const void* wd, const float* s_d,
                            const void* sh_wgu, const float* sh_s_gu, const void* sh_wd,
                            const float* sh_s_d, const int32_t* tokens, int n, double* out_f64,
@@ -345,7 +365,7 @@ int oracle_forward_tokens2(int T, int d, int E, int k, int F, double scale, cons
     long r;
     if (d <= 0 || E <= 0 || k <= 0 || k > E || F <= 0)
         return -1;
-    if ((sh_wgu == NULL) != (sh_wd == NULL))
+    if ((sh_wgu == NULL) != (sh_wd == NULL) || (norm_w && !(norm_eps > 0.0)))
         return -1;
     for (r = 0; r < n; ++r)
         if (tokens[r] < 0 || tokens[r] >= T)
@@ -356,8 +376,8 @@ int oracle_forward_tokens2(int T, int d, int E, int k, int F, double scale, cons
         double* y = (double*)malloc(sizeof(double) * (size_t)k * d);
         double* ysh = sh_wgu ? (double*)malloc(sizeof(double) * (size_t)d) : NULL;
         int j;
-        route_token(d, E, k, scale, xrow, wg, gate_bias, score_bias, idx + r * (long)k,
-                    w + r * (long)k, NULL, NULL, gap + r);
+        route_token(d, E, k, scale, xrow, wg, gate_bias, score_bias, norm_w, norm_eps,
+                    idx + r * (long)k, w + r * (long)k, NULL, NULL, gap + r);
         for (j = 0; j < k; ++j)
             expert_token(d, F, idx[r * (long)k + j], xrow, wgu, s_gu, wd, s_d, NULL,
                          y + (long)j * d);
@@ -378,9 +398,9 @@ int oracle_forward_tokens(int T, int d, int E, int k, int F, double scale, const
                           const int32_t* tokens, int n, double* out_f64, uint16_t* out_bf16,
                           int32_t* idx, double* w, double* gap)
 {
-    return oracle_forward_tokens2(T, d, E, k, F, scale, x, wg, gate_bias, NULL, wgu, s_gu, wd,
-                                  s_d, NULL, NULL, NULL, NULL, tokens, n, out_f64, out_bf16, idx,
-                                  w, gap);
+    return oracle_forward_tokens2(T, d, E, k, F, scale, x, wg, gate_bias, NULL, NULL, 0.0, wgu,
+                                  s_gu, wd, s_d, NULL, NULL, NULL, NULL, tokens, n, out_f64,
+                                  out_bf16, idx, w, gap);
 }
 
 /* The grouping that the library's permute step defines (integer work):

@@ -47,15 +47,15 @@ def _load():
         lib.oracle_double_from_e4m3.argtypes = [P, P, L]
         lib.oracle_route.argtypes = [I, I, I, I, D, P, P, P, P, P, P, P, P]
         lib.oracle_route.restype = I
-        lib.oracle_route2.argtypes = [I, I, I, I, D, P, P, P, P, P, P, P, P, P]
+        lib.oracle_route2.argtypes = [I, I, I, I, D, P, P, P, P, P, D, P, P, P, P, P]
         lib.oracle_route2.restype = I
         lib.oracle_expert_rows.argtypes = [I, I, I, P, P, P, P, P, P, P, P]
         lib.oracle_expert_rows.restype = I
         lib.oracle_forward_tokens.argtypes = [I, I, I, I, I, D, P, P, P, P, P, P, P, P, I, P, P,
                                               P, P, P]
         lib.oracle_forward_tokens.restype = I
-        lib.oracle_forward_tokens2.argtypes = [I, I, I, I, I, D, P, P, P, P, P, P, P, P, P, P, P,
-                                               P, P, I, P, P, P, P, P]
+        lib.oracle_forward_tokens2.argtypes = [I, I, I, I, I, D, P, P, P, P, P, D, P, P, P, P, P,
+                                               P, P, P, P, I, P, P, P, P, P]
         lib.oracle_forward_tokens2.restype = I
         lib.oracle_combine.argtypes = [I, I, I, P, P, P]
         lib.oracle_permute.argtypes = [I, I, I, P, P, P, P]
@@ -108,11 +108,13 @@ def double_from_e4m3(q: np.ndarray) -> np.ndarray:
 
 
 def route(x, wg, k: int, scale: float, gate_bias=None, want_scores: bool = False,
-          score_bias=None):
+          score_bias=None, norm_w=None, norm_eps: float = 1e-6):
     """Steps 1-4 for all tokens. x [T,d] / wg [E,d] uint16 bf16 bits.
 
     gate_bias [E] is added to the logits (before the sigmoid); score_bias [E]
-    (e_score_correction_bias) to the scores for the choice only. Returns
+    (e_score_correction_bias) to the scores for the choice only; norm_w [d]
+    turns on route_norm (the router scores the token's RMSNorm with that weight
+    and norm_eps). Returns
     dict(idx int32 [T,k], w f64 [T,k], gap f64 [T] -- between the k-th and
     (k+1)-th ranked value -- and with want_scores also logits/scores f64 [T,E]).
     """
@@ -127,8 +129,10 @@ def route(x, wg, k: int, scale: float, gate_bias=None, want_scores: bool = False
     logits = np.empty((T, E), dtype=np.float64) if want_scores else None
     scores = np.empty((T, E), dtype=np.float64) if want_scores else None
     sb = None if score_bias is None else np.ascontiguousarray(score_bias, dtype=np.float32)
+    nw = None if norm_w is None else np.ascontiguousarray(norm_w, dtype=np.float32)
     rc = _load().oracle_route2(T, d, E, k, float(scale), _ptr(x), _ptr(wg), _ptr(gb), _ptr(sb),
-                               _ptr(idx), _ptr(w), _ptr(logits), _ptr(scores), _ptr(gap))
+                               _ptr(nw), float(norm_eps), _ptr(idx), _ptr(w), _ptr(logits),
+                               _ptr(scores), _ptr(gap))
     if rc != 0:
         raise ValueError("oracle_route: bad arguments")
     out = {"idx": idx, "w": w, "gap": gap}
@@ -173,7 +177,7 @@ def forward_tokens(layer: "OracleLayer", tokens=None):
     gap = np.empty((n,), dtype=np.float64)
     rc = _load().oracle_forward_tokens2(L.T, L.d, L.E, L.k, L.F, float(L.scale), _ptr(L.x),
                                         _ptr(L.wg), _ptr(L.gate_bias), _ptr(L.score_bias),
-                                        _ptr(L.wgu), _ptr(L.s_gu), _ptr(L.wd), _ptr(L.s_d),
+                                        _ptr(L.norm_w), float(L.norm_eps), _ptr(L.wgu), _ptr(L.s_gu), _ptr(L.wd), _ptr(L.s_d),
                                         _ptr(L.sh_wgu), _ptr(L.sh_s_gu), _ptr(L.sh_wd),
                                         _ptr(L.sh_s_d), _ptr(tokens), n, _ptr(out_f64),
                                         _ptr(out_bf16), _ptr(idx), _ptr(w), _ptr(gap))
@@ -223,6 +227,10 @@ class OracleLayer:
         gb = layer.get("gate_bias")
         self.gate_bias = None if gb is None else np.ascontiguousarray(gb.detach().cpu().numpy(),
                                                                       dtype=np.float32)
+        nw = layer.get("route_norm_weight")
+        self.norm_w = None if nw is None else np.ascontiguousarray(nw.detach().cpu().numpy(),
+                                                                   dtype=np.float32)
+        self.norm_eps = float(getattr(cfg, "route_norm_eps", 1e-6))
         sb = layer.get("score_bias")
         self.score_bias = None if sb is None else np.ascontiguousarray(
             sb.detach().cpu().numpy(), dtype=np.float32)

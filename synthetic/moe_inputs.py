@@ -19,8 +19,8 @@ scaling 2.826) are those of "Tencent Hy3-295B 架构深度拆解" (pillumina.git
 
 Draw order, from one torch.Generator seeded with ``seed``: x, W_gate,
 W_gate_up (expert by expert), W_down (expert by expert), then -- only for
-shapes that ask for them -- the shared expert's W_gate_up and W_down and the
-e_score_correction_bias. Each weight is drawn as fp32 N(0,1), multiplied by
+shapes that ask for them -- the shared expert's W_gate_up and W_down, the
+e_score_correction_bias and the route_norm weight. Each weight is drawn as fp32 N(0,1), multiplied by
 its standard deviation and rounded to bf16 (round-to-nearest-even, torch's
 cast); the score bias stays fp32. The bf16 bit patterns are what both the
 oracle and the CUDA path consume.
@@ -35,6 +35,7 @@ Layouts (row-major, contiguous):
                            sigmoid scores for the choice of experts only)
   w_shared_gate_up [2F, d], w_shared_down [d, F]   bf16, when the shape has a
                            shared expert (q_/s_shared_* for FP8 shapes)
+  route_norm_weight [d]    fp32 or None (the RMSNorm weight of the router input)
 FP8 workloads add ``q_gate_up`` [E, 2F, d] / ``q_down`` [E, d, F] as uint8
 e4m3 codes and ``s_gate_up`` [E, 2F] / ``s_down`` [E, d] fp32 scales, with the
 weight meaning q * s.
@@ -62,6 +63,8 @@ class LayerShape:
     fp8: bool = False
     shared: bool = False          # one shared expert (SwiGLU, d_ff = F), weight 1
     score_bias_std: float = 0.0   # e_score_correction_bias ~ N(0, std^2) when > 0
+    route_norm: bool = False      # RMSNorm of the router's input, weight 1 + N(0, 0.1^2)
+    route_norm_eps: float = 1e-6
 
     @property
     def R(self) -> int:
@@ -168,6 +171,10 @@ def make_layer(cfg, seed: int = 0, device="cpu", T: Optional[int] = None,
     if cfg.score_bias_std > 0:
         out["score_bias"] = torch.randn((E,), generator=gen, dtype=torch.float32,
                                         device=dev) * cfg.score_bias_std
+    out["route_norm_weight"] = None
+    if cfg.route_norm:
+        out["route_norm_weight"] = 1.0 + 0.1 * torch.randn((cfg.d,), generator=gen,
+                                                           dtype=torch.float32, device=dev)
     if cfg.fp8:
         q_gu = torch.empty(shp["w_gate_up"], dtype=torch.uint8, device=dev)
         s_gu = torch.empty(shp["s_gate_up"], dtype=torch.float32, device=dev)

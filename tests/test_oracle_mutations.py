@@ -34,6 +34,11 @@ MUTATIONS = {
     "score_bias_in_the_weights": ("sel_sum += order[j].s;", "sel_sum += order[j].key;"),
     "shared_expert_dropped": ("a += y_shared[i];", "a += 0.0 * y_shared[i];"),
     "shared_expert_scaled": ("a += y_shared[i];", "a += 2.826 * y_shared[i];"),
+    "route_norm_not_normalising": ("xr[c] = xr[c] * inv * (double)norm_w[c];",
+                                   "xr[c] = xr[c] * (double)norm_w[c];"),
+    "route_norm_weight_dropped": ("xr[c] = xr[c] * inv * (double)norm_w[c];", "xr[c] = xr[c] * inv;"),
+    "route_norm_eps_outside_root": ("inv = 1.0 / sqrt(ms / d + norm_eps);",
+                                    "inv = 1.0 / (sqrt(ms / d) + norm_eps);"),
 }
 
 

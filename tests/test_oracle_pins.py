@@ -428,3 +428,72 @@ def test_moe_layer_parameter_count_with_the_shared_expert_matches_the_page(golde
     assert round(per_expert / 1e6, 2) * 1e6 == golden["moe_layer_params"]["shared_expert_params_printed"]
     frac = per_expert / ((shp["w_gate_up"][0] + 1) * per_expert)
     assert round(100 * frac, 2) == golden["shared_expert_fraction"]["printed_percent"]
+
+
+# ------------------------------------------------------------------ route_norm:
+# the router scores RMSNorm(x) (weight g, eps inside the root); the experts take x
+
+def _np_rmsnorm(x64, g, eps):
+    return x64 / np.sqrt((x64 * x64).mean(axis=1, keepdims=True) + eps) * g[None, :]
+
+
+def test_route_norm_scores_the_rmsnorm_of_the_token():
+    shape = LayerShape(T=20, d=64, E=10, k=3, F=32, route_norm=True)
+    L = _layer(shape, seed=41)
+    g = L["route_norm_weight"].numpy().astype(np.float64)
+    r = oracle.route(_bits(L["x"]), _bits(L["w_gate"]), 3, 2.826, want_scores=True,
+                     norm_w=L["route_norm_weight"].numpy(), norm_eps=1e-6)
+    want = _np_rmsnorm(_f64(L["x"]), g, 1e-6) @ _f64(L["w_gate"]).T
+    assert np.allclose(r["logits"], want, rtol=1e-12, atol=1e-14)
+    s = 1.0 / (1.0 + np.exp(-want))
+    for t in range(20):
+        assert list(r["idx"][t]) == sorted(range(10), key=lambda e: (-s[t, e], e))[:3]
+
+
+def test_route_norm_makes_the_routing_independent_of_the_token_scale():
+    shape = LayerShape(T=30, d=64, E=12, k=4, F=32, route_norm=True)
+    L = _layer(shape, seed=42)
+    nw = L["route_norm_weight"].numpy()
+    x1, x4 = _bits(L["x"]), _bits(L["x"] * 4)       # x4 = 4 x exactly (bf16)
+    a = oracle.route(x1, _bits(L["w_gate"]), 4, 2.826, norm_w=nw)
+    b = oracle.route(x4, _bits(L["w_gate"]), 4, 2.826, norm_w=nw)
+    assert np.array_equal(a["idx"], b["idx"])
+    assert np.allclose(a["w"], b["w"], rtol=1e-5)
+    c = oracle.route(x1, _bits(L["w_gate"]), 4, 2.826)
+    d = oracle.route(x4, _bits(L["w_gate"]), 4, 2.826)
+    assert not np.allclose(c["w"], d["w"], rtol=1e-3)   # without route_norm it is not
+
+
+def test_route_norm_epsilon_sits_inside_the_root():
+    """Tokens of size ~2^-12 (mean square ~6e-8, below eps = 1e-6): only
+    x / sqrt(mean(x^2) + eps) reproduces the oracle's logits."""
+    shape = LayerShape(T=8, d=64, E=6, k=2, F=32, route_norm=True)
+    L = _layer(shape, seed=43)
+    xs = (L["x"].float() * 2.0 ** -12).to(torch.bfloat16)
+    g = L["route_norm_weight"].numpy().astype(np.float64)
+    r = oracle.route(_bits(xs), _bits(L["w_gate"]), 2, 2.826, want_scores=True,
+                     norm_w=L["route_norm_weight"].numpy(), norm_eps=1e-6)
+    want = _np_rmsnorm(_f64(xs), g, 1e-6) @ _f64(L["w_gate"]).T
+    assert np.allclose(r["logits"], want, rtol=1e-12, atol=1e-16)
+
+
+def test_zero_route_norm_weight_gives_equal_scores():
+    L = _layer(LayerShape(T=5, d=64, E=8, k=3, F=32, route_norm=True), seed=44)
+    r = oracle.route(_bits(L["x"]), _bits(L["w_gate"]), 3, 2.826,
+                     norm_w=np.zeros(64, np.float32))
+    assert np.all(r["idx"] == np.arange(3)[None, :])
+    assert np.allclose(r["w"], 2.826 / 3, rtol=1e-15)
+
+
+def test_route_norm_leaves_the_experts_on_the_token():
+    """k = E: out = sum_e w_e(RMSNorm(x)) * expert_e(x) -- the weights come from
+    the normalised token, the expert outputs from the token itself."""
+    shape = LayerShape(T=6, d=64, E=4, k=4, F=32, route_norm=True)
+    L = _layer(shape, seed=45)
+    r = oracle.forward_tokens(oracle.OracleLayer(L))
+    x64, wgu, wd = _f64(L["x"]), _f64(L["w_gate_up"]), _f64(L["w_down"])
+    g = L["route_norm_weight"].numpy().astype(np.float64)
+    s = 1.0 / (1.0 + np.exp(-(_np_rmsnorm(x64, g, 1e-6) @ _f64(L["w_gate"]).T)))
+    w = 2.826 * s / s.sum(axis=1, keepdims=True)
+    want = sum(w[:, e:e + 1] * _np_expert(x64, wgu, wd, e, shape.F) for e in range(4))
+    assert np.allclose(r["out_f64"], want, rtol=1e-9, atol=1e-12)
