@@ -227,6 +227,9 @@ def main():
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (a smaller case of the same workload, e.g. for ncu)")
     ap.add_argument("--tokens", type=int, default=None, help="override T")
+    ap.add_argument("--block", action="store_true",
+                    help="the complete Hy3 block: + a shared expert and an "
+                         "e_score_correction_bias (N(0, 0.05^2))")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     if args.steps is None:
@@ -252,29 +255,35 @@ def main():
                                 device_id=dev)
         pg = dist
 
+    import dataclasses
+
     shape = CONFIGS[args.config]
     if args.experts or args.tokens:
-        import dataclasses
-
         shape = dataclasses.replace(shape, E=args.experts or shape.E, T=args.tokens or shape.T)
+    if args.block:
+        shape = dataclasses.replace(shape, shared=True, score_bias_std=0.05)
     layer = make_layer(shape, seed=rank, device=dev)
     T, d, E, k, F = shape.T, shape.d, shape.E, shape.k, shape.F
     # bf16 weights on the tensor-core pair kernels are packed once, at load time
     # (moe_pack_weights), outside every timed region
     packed = not shape.fp8 and args.path != "stream" and d % 256 == 0 and F % 256 == 0
     cfg = moe.config_of(shape, None if args.path == "auto" else args.path, packed=packed)
-    R = T * k
+    # grouped slots per token (the shared expert, when present, is slot k of
+    # every token and expert E)
+    ks = k + (1 if shape.shared else 0)
+    Eg = E + (1 if shape.shared else 0)
+    R = T * ks
     ws = moe.workspace(cfg, device=dev)
     stream = torch.cuda.Stream(device=dev)
     wgu, sgu, wd, sd = moe.layer_args(layer)
     if packed:
         wgu, wd = moe.pack_layer_weights(cfg, wgu, wd)
         torch.cuda.synchronize(dev)
-    x, wg, gb = layer["x"], layer["w_gate"], layer["gate_bias"]
+    x, wg, gb, sb = layer["x"], layer["w_gate"], layer["gate_bias"], layer["score_bias"]
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
-    counts = torch.empty(E, dtype=torch.int32, device=dev)
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    counts = torch.empty(Eg, dtype=torch.int32, device=dev)
+    offsets = torch.empty(Eg + 1, dtype=torch.int32, device=dev)
     row_of = torch.empty(R, dtype=torch.int32, device=dev)
     gather = R <= moe.MOE_GATHER_MAX_SLOTS  # moe_forward's grouping rule
     tok = torch.empty(R, dtype=torch.int32, device=dev)
@@ -294,7 +303,7 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        moe.moe_route(cfg, x, wg, gb, idx, w, ws, stream)
+        moe.moe_route2(cfg, x, wg, gb, sb, idx, w, ws, stream)
         if ev is not None:
             ev[1].record(stream)
         if gather:
@@ -348,7 +357,8 @@ def main():
     rows = int(offsets[-1].item())
     peaks, peak_src = load_peaks()
     fp8 = shape.fp8
-    lw = work.layer_work(T, d, E, k, F, touched, fp8)
+    # the shared expert counts as one more touched expert with T more rows
+    lw = work.layer_work(T, d, E, ks, F, touched, fp8)
     gw = work.gate_up_work(rows, touched, d, F, fp8)
     dw = work.down_work(rows, touched, d, F, fp8)
     dominant = max(("gate_up", "down"), key=lambda s: stage_ms[s])
@@ -405,7 +415,7 @@ def main():
             stream.wait_event(h2d)
             if d2h[b] is not None:
                 stream.wait_event(d2h[b])  # step i-2's output has been read back
-            moe.moe_forward(cfg, x_dev[b], wg, gb, wgu, sgu, wd, sd, out_dev[b], ws, stream)
+            moe.moe_forward2(cfg, x_dev[b], wg, gb, sb, wgu, sgu, wd, sd, out_dev[b], ws, stream)
             fwd[b] = torch.cuda.Event()
             fwd[b].record(stream)
             with torch.cuda.stream(d2h_stream):
@@ -448,8 +458,12 @@ def main():
             "dtype": "e4m3 weights, bf16 activations, fp32 accumulate" if fp8 else
                      "bf16 (fp32 accumulate, fp32 combine)",
             "data": "synthetic (seeded; random-init weights of the Hy3 MoE layer shapes)",
-            "config": {"workload": WORKLOADS[args.config] if shape == CONFIGS[args.config] else
-                       f"smaller case of {args.config}: T={T}, E={E}", "T": T, "d": d, "E": E, "k": k,
+            "config": {"workload": (WORKLOADS[args.config] if shape == CONFIGS[args.config] else
+                                    f"{args.config} with the complete Hy3 block (+ a shared expert "
+                                    "and an e_score_correction_bias)" if args.block and
+                                    (T, E) == (CONFIGS[args.config].T, CONFIGS[args.config].E) else
+                                    f"smaller case of {args.config}: T={T}, E={E}"),
+                       "T": T, "d": d, "E": E, "k": k,
                        "d_ff": F, "path": args.path, "parallelism": f"replicas x{world}",
                        "weights": ("e4m3 + fp32 row scales" if fp8 else
                                    "bf16, packed in 128x64 blocks once at load (moe_pack_weights)"
@@ -467,7 +481,7 @@ def main():
             "clocks": clocks.summary(),
             "e2e": {"value": replica_value(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
-                    "ms_per_step": e2e_ms, "api": "moe_forward",
+                    "ms_per_step": e2e_ms, "api": "moe_forward2",
                     "copies": "one stream per direction, double-buffered, overlapping the compute",
                     "output_equals_staged": e2e_same},
             "gpu_launches": sum(n_launch.values()) * args.steps,
