@@ -12,8 +12,11 @@ from .oracle import (  # noqa: F401
     build,
     combine,
     double_from_bf16,
+    double_from_e2m1,
     double_from_e4m3,
+    double_from_e8m0,
     expert_rows,
+    expert_rows_fp4,
     forward_tokens,
     num_threads,
     permute,

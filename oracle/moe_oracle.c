@@ -36,6 +36,14 @@
  * the token, xn_c = x_c / sqrt(mean_c' x_c'^2 + eps) * g_c (g: the norm's
  * weight); step 1 uses xn in place of x, the experts still take x.
  *
+ * The second routing and precision variant of the pages ("Tencent Hy3-295B
+ * 架构深度拆解" §2.2 and §2.7, the V4-Flash column): the score of step 2 may
+ * be sqrt(softplus(logit)) instead of the sigmoid (same steps 3-4, with its own
+ * scale, 1.5 on the page), and the routed experts may be FP4: E2M1 codes (1
+ * sign, 2 exponent bits with bias 1, 1 mantissa bit; two per byte, the even
+ * element in the low nibble) with one E8M0 scale 2^(b-127) per 32 consecutive
+ * elements of a row; the weight value is code * scale.
+ *
  * Every sum is a plain left-to-right fp64 loop; inputs are bf16 bit patterns
  * (or e4m3 codes with fp32 scales) widened exactly to double. The only
  * rounding to a narrow type is the single final bf16 cast of step 6.
@@ -79,6 +87,23 @@ static double e4m3_to_double(uint8_t q)
     else
         v = ldexp(1.0 + (double)mant / 8.0, ex - 7);
     return sign ? -v : v;
+}
+
+/* e2m1 (OCP MX FP4): 1 sign, 2 exponent bits (bias 1), 1 mantissa bit, no
+ * infinities or NaN. exp 0 is subnormal: mant/2 * 2^0. */
+static double e2m1_to_double(uint8_t nib)
+{
+    int sign = (nib >> 3) & 1;
+    int ex = (nib >> 1) & 0x3;
+    int mant = nib & 0x1;
+    double v = (ex == 0) ? 0.5 * mant : ldexp(1.0 + 0.5 * mant, ex - 1);
+    return sign ? -v : v;
+}
+
+/* e8m0 (OCP MX scale): 2^(b - 127); 0xFF is NaN. */
+static double e8m0_to_double(uint8_t b)
+{
+    return (b == 0xFF) ? NAN : ldexp(1.0, (int)b - 127);
 }
 
 /* Round half to even of a non-negative double to an integer-valued double. */
@@ -126,6 +151,15 @@ static uint16_t double_to_bf16(double v)
 
 static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+/* softplus(z) = ln(1 + e^z), evaluated without overflow. */
+static double softplus(double z) { return (z > 0.0) ? z + log1p(exp(-z)) : log1p(exp(z)); }
+
+/* Step 2's score: 0 = sigmoid (Hy3), 1 = sqrt(softplus) (the V4-Flash router). */
+static double score_of(double z, int score_fn)
+{
+    return score_fn == 1 ? sqrt(softplus(z)) : sigmoid(z);
+}
+
 /* Weight element (expert e, row r, column c) of a [E, rows, cols] block that is
  * either bf16 (scales == NULL) or e4m3 codes with per-row fp32 scales. */
 static double weight_at(const void* w, const float* scales, long e, long rows, long cols,
@@ -135,6 +169,18 @@ static double weight_at(const void* w, const float* scales, long e, long rows, l
     if (scales == NULL)
         return bf16_to_double(((const uint16_t*)w)[off]);
     return e4m3_to_double(((const uint8_t*)w)[off]) * (double)scales[e * rows + r];
+}
+
+/* Weight element (expert e, row r, column c) of a [E, rows, cols] block of FP4
+ * codes (two per byte, the even element in the low nibble) with E8M0 scales
+ * [E, rows, cols/32], one per 32 consecutive elements of a row. */
+static double weight_at_fp4(const uint8_t* w, const uint8_t* scales, long e, long rows, long cols,
+                            long r, long c)
+{
+    long off = (e * rows + r) * cols + c;
+    uint8_t byte = w[off >> 1];
+    uint8_t nib = (off & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+    return e2m1_to_double(nib) * e8m0_to_double(scales[(e * rows + r) * (cols / 32) + c / 32]);
 }
 
 /* ---------------------------------------------------------------- routing */
@@ -162,8 +208,8 @@ static int by_score_then_index(const void* pa, const void* pb)
  * and (k+1)-th largest key (+inf when k == E). score_bias may be NULL. */
 static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
                         const uint16_t* wg, const float* gate_bias, const float* score_bias,
-                        const float* norm_w, double norm_eps, int32_t* idx, double* w,
-                        double* logits_out, double* scores_out, double* gap)
+                        const float* norm_w, double norm_eps, int score_fn, int32_t* idx,
+                        double* w, double* logits_out, double* scores_out, double* gap)
 {
     scored_expert* order = (scored_expert*)malloc(sizeof(scored_expert) * (size_t)E);
     double* xr = (double*)malloc(sizeof(double) * (size_t)d);
@@ -186,7 +232,7 @@ static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
             logit += xr[c] * bf16_to_double(wg[(long)e * d + c]);
         if (gate_bias)
             logit += (double)gate_bias[e];
-        order[e].s = sigmoid(logit);
+        order[e].s = score_of(logit, score_fn);
         order[e].key = score_bias ? order[e].s + (double)score_bias[e] : order[e].s;
         order[e].e = e;
         if (logits_out)
@@ -228,6 +274,32 @@ static void expert_token(int d, int F, long e, const uint16_t* xrow, const void*
         double acc = 0.0;
         for (f = 0; f < F; ++f)
             acc += hh[f] * weight_at(wd, s_d, e, d, F, i, f);
+        y[i] = acc;
+    }
+    if (!h)
+        free(hh);
+}
+
+/* Step 5 with FP4 expert weights (same mathematics). */
+static void expert_token_fp4(int d, int F, long e, const uint16_t* xrow, const uint8_t* wgu,
+                             const uint8_t* s_gu, const uint8_t* wd, const uint8_t* s_d,
+                             double* h, double* y)
+{
+    double* hh = h ? h : (double*)malloc(sizeof(double) * (size_t)F);
+    int f, c, i;
+    for (f = 0; f < F; ++f) {
+        double g = 0.0, u = 0.0;
+        for (c = 0; c < d; ++c) {
+            double xc = bf16_to_double(xrow[c]);
+            g += xc * weight_at_fp4(wgu, s_gu, e, 2L * F, d, f, c);
+            u += xc * weight_at_fp4(wgu, s_gu, e, 2L * F, d, (long)F + f, c);
+        }
+        hh[f] = g * sigmoid(g) * u;
+    }
+    for (i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (f = 0; f < F; ++f)
+            acc += hh[f] * weight_at_fp4(wd, s_d, e, d, F, i, f);
         y[i] = acc;
     }
     if (!h)
@@ -311,17 +383,19 @@ void oracle_double_from_e4m3(const uint8_t* q, double* out, long n)
  * logits/scores may be NULL ([T, E] otherwise). */
 int oracle_route2(int T, int d, int E, int k, double scale, const uint16_t* x,
                   const uint16_t* wg, const float* gate_bias, const float* score_bias,
-                  const float* norm_w, double norm_eps, int32_t* idx, double* w, double* logits,
-                  double* scores, double* gap)
+                  const float* norm_w, double norm_eps, int score_fn, int32_t* idx, double* w,
+                  double* logits, double* scores, double* gap)
 {
     long t;
-    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || (norm_w && !(norm_eps > 0.0)))
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || (norm_w && !(norm_eps > 0.0)) ||
+        score_fn < 0 || score_fn > 1)
         return -1;
 #pragma omp parallel for schedule(dynamic, 4)
     for (t = 0; t < T; ++t)
         route_token(d, E, k, scale, x + t * (long)d, wg, gate_bias, score_bias, norm_w, norm_eps,
-                    idx + t * (long)k, w + t * (long)k, logits ? logits + t * (long)E : NULL,
-                    scores ? scores + t * (long)E : NULL, gap + t);
+                    score_fn, idx + t * (long)k, w + t * (long)k,
+                    logits ? logits + t * (long)E : NULL, scores ? scores + t * (long)E : NULL,
+                    gap + t);
     return 0;
 }
 
@@ -330,7 +404,7 @@ int oracle_route(int T, int d, int E, int k, double scale, const uint16_t* x,
                  const uint16_t* wg, const float* gate_bias, int32_t* idx, double* w,
                  double* logits, double* scores, double* gap)
 {
-    return oracle_route2(T, d, E, k, scale, x, wg, gate_bias, NULL, NULL, 0.0, idx, w, logits,
+    return oracle_route2(T, d, E, k, scale, x, wg, gate_bias, NULL, NULL, 0.0, 0, idx, w, logits,
                          scores, gap);
 }
 
@@ -376,7 +450,7 @@ int oracle_forward_tokens2(int T, int d, int E, int k, int F, double scale, cons
         double* y = (double*)malloc(sizeof(double) * (size_t)k * d);
         double* ysh = sh_wgu ? (double*)malloc(sizeof(double) * (size_t)d) : NULL;
         int j;
-        route_token(d, E, k, scale, xrow, wg, gate_bias, score_bias, norm_w, norm_eps,
+        route_token(d, E, k, scale, xrow, wg, gate_bias, score_bias, norm_w, norm_eps, 0,
                     idx + r * (long)k, w + r * (long)k, NULL, NULL, gap + r);
         for (j = 0; j < k; ++j)
             expert_token(d, F, idx[r * (long)k + j], xrow, wgu, s_gu, wd, s_d, NULL,
@@ -401,6 +475,68 @@ int oracle_forward_tokens(int T, int d, int E, int k, int F, double scale, const
     return oracle_forward_tokens2(T, d, E, k, F, scale, x, wg, gate_bias, NULL, NULL, 0.0, wgu,
                                   s_gu, wd, s_d, NULL, NULL, NULL, NULL, tokens, n, out_f64,
                                   out_bf16, idx, w, gap);
+}
+
+void oracle_double_from_e2m1(const uint8_t* nibbles, double* out, long n)
+{
+    long i;
+    for (i = 0; i < n; ++i)
+        out[i] = e2m1_to_double(nibbles[i] & 0xF);
+}
+
+void oracle_double_from_e8m0(const uint8_t* b, double* out, long n)
+{
+    long i;
+    for (i = 0; i < n; ++i)
+        out[i] = e8m0_to_double(b[i]);
+}
+
+/* Step 5 with FP4 experts for n (row, expert) pairs (see oracle_expert_rows). */
+int oracle_expert_rows_fp4(int n, int d, int F, const uint16_t* xrows, const int32_t* experts,
+                           const uint8_t* wgu, const uint8_t* s_gu, const uint8_t* wd,
+                           const uint8_t* s_d, double* h, double* y)
+{
+    long r;
+    if (d % 32 || F % 32)
+        return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < n; ++r)
+        expert_token_fp4(d, F, experts[r], xrows + r * (long)d, wgu, s_gu, wd, s_d,
+                         h ? h + r * (long)F : NULL, y + r * (long)d);
+    return 0;
+}
+
+/* Steps 1-6 of the second variant for the listed tokens: score_fn as in
+ * oracle_route2, FP4 routed experts, optional score bias; no shared expert. */
+int oracle_forward_tokens_fp4(int T, int d, int E, int k, int F, double scale, const uint16_t* x,
+                              const uint16_t* wg, const float* gate_bias, const float* score_bias,
+                              int score_fn, const uint8_t* wgu, const uint8_t* s_gu,
+                              const uint8_t* wd, const uint8_t* s_d, const int32_t* tokens, int n,
+                              double* out_f64, uint16_t* out_bf16, int32_t* idx, double* w,
+                              double* gap)
+{
+    long r;
+    if (d <= 0 || E <= 0 || k <= 0 || k > E || F <= 0 || d % 32 || F % 32 || score_fn < 0 ||
+        score_fn > 1)
+        return -1;
+    for (r = 0; r < n; ++r)
+        if (tokens[r] < 0 || tokens[r] >= T)
+            return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < n; ++r) {
+        const uint16_t* xrow = x + (long)tokens[r] * d;
+        double* y = (double*)malloc(sizeof(double) * (size_t)k * d);
+        int j;
+        route_token(d, E, k, scale, xrow, wg, gate_bias, score_bias, NULL, 0.0, score_fn,
+                    idx + r * (long)k, w + r * (long)k, NULL, NULL, gap + r);
+        for (j = 0; j < k; ++j)
+            expert_token_fp4(d, F, idx[r * (long)k + j], xrow, wgu, s_gu, wd, s_d, NULL,
+                             y + (long)j * d);
+        combine_token(k, d, y, w + r * (long)k, NULL, out_f64 + r * (long)d,
+                      out_bf16 + r * (long)d);
+        free(y);
+    }
+    return 0;
 }
 
 /* The grouping that the library's permute step defines (integer work):

@@ -47,7 +47,7 @@ def _load():
         lib.oracle_double_from_e4m3.argtypes = [P, P, L]
         lib.oracle_route.argtypes = [I, I, I, I, D, P, P, P, P, P, P, P, P]
         lib.oracle_route.restype = I
-        lib.oracle_route2.argtypes = [I, I, I, I, D, P, P, P, P, P, D, P, P, P, P, P]
+        lib.oracle_route2.argtypes = [I, I, I, I, D, P, P, P, P, P, D, I, P, P, P, P, P]
         lib.oracle_route2.restype = I
         lib.oracle_expert_rows.argtypes = [I, I, I, P, P, P, P, P, P, P, P]
         lib.oracle_expert_rows.restype = I
@@ -58,6 +58,13 @@ def _load():
                                                P, P, P, P, I, P, P, P, P, P]
         lib.oracle_forward_tokens2.restype = I
         lib.oracle_combine.argtypes = [I, I, I, P, P, P]
+        lib.oracle_double_from_e2m1.argtypes = [P, P, L]
+        lib.oracle_double_from_e8m0.argtypes = [P, P, L]
+        lib.oracle_expert_rows_fp4.argtypes = [I, I, I, P, P, P, P, P, P, P, P]
+        lib.oracle_expert_rows_fp4.restype = I
+        lib.oracle_forward_tokens_fp4.argtypes = [I, I, I, I, I, D, P, P, P, P, I, P, P, P, P, P,
+                                                  I, P, P, P, P, P]
+        lib.oracle_forward_tokens_fp4.restype = I
         lib.oracle_permute.argtypes = [I, I, I, P, P, P, P]
         lib.oracle_permute.restype = I
         _lib = lib
@@ -107,14 +114,18 @@ def double_from_e4m3(q: np.ndarray) -> np.ndarray:
     return out
 
 
+SCORE_FNS = {"sigmoid": 0, "sqrtsoftplus": 1}
+
+
 def route(x, wg, k: int, scale: float, gate_bias=None, want_scores: bool = False,
-          score_bias=None, norm_w=None, norm_eps: float = 1e-6):
+          score_bias=None, norm_w=None, norm_eps: float = 1e-6, score_fn: str = "sigmoid"):
     """Steps 1-4 for all tokens. x [T,d] / wg [E,d] uint16 bf16 bits.
 
     gate_bias [E] is added to the logits (before the sigmoid); score_bias [E]
     (e_score_correction_bias) to the scores for the choice only; norm_w [d]
     turns on route_norm (the router scores the token's RMSNorm with that weight
-    and norm_eps). Returns
+    and norm_eps); score_fn "sqrtsoftplus" scores sqrt(softplus(logit)) instead of
+    the sigmoid. Returns
     dict(idx int32 [T,k], w f64 [T,k], gap f64 [T] -- between the k-th and
     (k+1)-th ranked value -- and with want_scores also logits/scores f64 [T,E]).
     """
@@ -131,8 +142,8 @@ def route(x, wg, k: int, scale: float, gate_bias=None, want_scores: bool = False
     sb = None if score_bias is None else np.ascontiguousarray(score_bias, dtype=np.float32)
     nw = None if norm_w is None else np.ascontiguousarray(norm_w, dtype=np.float32)
     rc = _load().oracle_route2(T, d, E, k, float(scale), _ptr(x), _ptr(wg), _ptr(gb), _ptr(sb),
-                               _ptr(nw), float(norm_eps), _ptr(idx), _ptr(w), _ptr(logits),
-                               _ptr(scores), _ptr(gap))
+                               _ptr(nw), float(norm_eps), SCORE_FNS[score_fn], _ptr(idx), _ptr(w),
+                               _ptr(logits), _ptr(scores), _ptr(gap))
     if rc != 0:
         raise ValueError("oracle_route: bad arguments")
     out = {"idx": idx, "w": w, "gap": gap}
@@ -163,6 +174,36 @@ def expert_rows(xrows, experts, wgu, wd, s_gu=None, s_d=None, want_h: bool = Fal
     return (y, h) if want_h else y
 
 
+def double_from_e2m1(nibbles: np.ndarray) -> np.ndarray:
+    nb = np.ascontiguousarray(nibbles, dtype=np.uint8)
+    out = np.empty(nb.shape, dtype=np.float64)
+    _load().oracle_double_from_e2m1(_ptr(nb), _ptr(out), nb.size)
+    return out
+
+
+def double_from_e8m0(b: np.ndarray) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    out = np.empty(b.shape, dtype=np.float64)
+    _load().oracle_double_from_e8m0(_ptr(b), _ptr(out), b.size)
+    return out
+
+
+def expert_rows_fp4(xrows, experts, wgu4, sgu8, wd4, sd8, want_h: bool = False):
+    """Step 5 with FP4 experts: packed E2M1 codes wgu4 [E,2F,d/2] / wd4 [E,d,F/2]
+    and E8M0 block-32 scales sgu8 [E,2F,d/32] / sd8 [E,d,F/32]."""
+    xrows = np.ascontiguousarray(xrows, dtype=np.uint16)
+    experts = np.ascontiguousarray(experts, dtype=np.int32)
+    n, d = xrows.shape
+    F = wd4.shape[2] * 2
+    arrs = [np.ascontiguousarray(a, dtype=np.uint8) for a in (wgu4, sgu8, wd4, sd8)]
+    h = np.empty((n, F), dtype=np.float64) if want_h else None
+    y = np.empty((n, d), dtype=np.float64)
+    if _load().oracle_expert_rows_fp4(n, d, F, _ptr(xrows), _ptr(experts), *map(_ptr, arrs),
+                                      _ptr(h), _ptr(y)) != 0:
+        raise ValueError("oracle_expert_rows_fp4: bad arguments")
+    return (y, h) if want_h else y
+
+
 def forward_tokens(layer: "OracleLayer", tokens=None):
     """Steps 1-6 for the listed tokens (all tokens when None)."""
     L = layer
@@ -175,6 +216,16 @@ def forward_tokens(layer: "OracleLayer", tokens=None):
     idx = np.empty((n, L.k), dtype=np.int32)
     w = np.empty((n, L.k), dtype=np.float64)
     gap = np.empty((n,), dtype=np.float64)
+    if L.fp4:
+        rc = _load().oracle_forward_tokens_fp4(
+            L.T, L.d, L.E, L.k, L.F, float(L.scale), _ptr(L.x), _ptr(L.wg), _ptr(L.gate_bias),
+            _ptr(L.score_bias), SCORE_FNS[L.score_fn], _ptr(L.wgu4), _ptr(L.sgu8), _ptr(L.wd4),
+            _ptr(L.sd8), _ptr(tokens), n, _ptr(out_f64), _ptr(out_bf16), _ptr(idx), _ptr(w),
+            _ptr(gap))
+        if rc != 0:
+            raise ValueError("oracle_forward_tokens_fp4: bad arguments")
+        return {"out_f64": out_f64, "out_bf16": out_bf16, "idx": idx, "w": w, "gap": gap,
+                "tokens": tokens}
     rc = _load().oracle_forward_tokens2(L.T, L.d, L.E, L.k, L.F, float(L.scale), _ptr(L.x),
                                         _ptr(L.wg), _ptr(L.gate_bias), _ptr(L.score_bias),
                                         _ptr(L.norm_w), float(L.norm_eps), _ptr(L.wgu), _ptr(L.s_gu), _ptr(L.wd), _ptr(L.s_d),
@@ -231,6 +282,13 @@ class OracleLayer:
         self.norm_w = None if nw is None else np.ascontiguousarray(nw.detach().cpu().numpy(),
                                                                    dtype=np.float32)
         self.norm_eps = float(getattr(cfg, "route_norm_eps", 1e-6))
+        self.score_fn = getattr(cfg, "score_fn", "sigmoid")
+        self.fp4 = bool(getattr(cfg, "fp4", False))
+        if self.fp4:
+            self.wgu4 = np.ascontiguousarray(layer["q4_gate_up"].cpu().numpy())
+            self.sgu8 = np.ascontiguousarray(layer["s4_gate_up"].cpu().numpy())
+            self.wd4 = np.ascontiguousarray(layer["q4_down"].cpu().numpy())
+            self.sd8 = np.ascontiguousarray(layer["s4_down"].cpu().numpy())
         sb = layer.get("score_bias")
         self.score_bias = None if sb is None else np.ascontiguousarray(
             sb.detach().cpu().numpy(), dtype=np.float32)

@@ -65,6 +65,8 @@ class LayerShape:
     score_bias_std: float = 0.0   # e_score_correction_bias ~ N(0, std^2) when > 0
     route_norm: bool = False      # RMSNorm of the router's input, weight 1 + N(0, 0.1^2)
     route_norm_eps: float = 1e-6
+    fp4: bool = False             # routed experts as E2M1 codes + E8M0 block-32 scales
+    score_fn: str = "sigmoid"     # or "sqrtsoftplus" (the second routing variant)
 
     @property
     def R(self) -> int:
@@ -119,6 +121,41 @@ def encode_e4m3_rows(w: torch.Tensor):
     return q, s.to(torch.float32)
 
 
+E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)  # magnitudes of codes 0..7
+
+
+def encode_e2m1_blocks(w: torch.Tensor):
+    """FP4 (OCP MX E2M1) encoding of a bf16 weight block [..., rows, cols], one
+    E8M0 scale per 32 consecutive elements of a row (cols % 32 == 0).
+
+    Scale 2^e with e = ceil(log2(amax / 6)) (so every |w| / scale <= 6; e = -127
+    for an all-zero block), stored as the byte e + 127; codes round |w| / scale
+    to the nearest E2M1 magnitude, ties to the even code, with the sign in bit
+    3; two codes per byte, the even element in the low nibble. Returns
+    (packed uint8 [..., rows, cols/2], scales uint8 [..., rows, cols/32]).
+    """
+    wf = w.float()
+    *lead, rows, cols = wf.shape
+    blk = wf.reshape(*lead, rows, cols // 32, 32)
+    amax = blk.abs().amax(dim=-1)
+    e = torch.where(amax > 0, torch.ceil(torch.log2(amax / 6.0)), torch.full_like(amax, -127.0))
+    e = e.clamp(-127, 127)
+    scale = torch.pow(2.0, e)
+    v = (blk / scale.unsqueeze(-1)).clamp(-6.0, 6.0)
+    grid = torch.tensor(E2M1_GRID, dtype=torch.float32, device=w.device)
+    a = v.abs().contiguous()
+    hi = torch.searchsorted(grid, a).clamp(max=7)     # first grid value >= a
+    lo = (hi - 1).clamp(min=0)
+    d_lo, d_hi = a - grid[lo], grid[hi] - a
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = torch.where(take_hi, hi, lo)
+    code = torch.where(a == grid[hi], hi, code)      # exact grid values
+    nib = (code + ((v < 0) & (code > 0)).to(code.dtype) * 8).to(torch.uint8)
+    nib = nib.reshape(*lead, rows, cols)
+    packed = (nib[..., 0::2] | (nib[..., 1::2] << 4)).to(torch.uint8)
+    return packed, (e + 127).to(torch.uint8)
+
+
 def tensor_shapes(cfg) -> dict:
     """Shapes of the layer's tensors (the layouts listed in the module docstring)."""
     cfg = shape_of(cfg)
@@ -171,6 +208,10 @@ def make_layer(cfg, seed: int = 0, device="cpu", T: Optional[int] = None,
     if cfg.score_bias_std > 0:
         out["score_bias"] = torch.randn((E,), generator=gen, dtype=torch.float32,
                                         device=dev) * cfg.score_bias_std
+    if cfg.fp4:
+        q4_gu, s4_gu = encode_e2m1_blocks(w_gate_up)
+        q4_d, s4_d = encode_e2m1_blocks(w_down)
+        out.update(q4_gate_up=q4_gu, s4_gate_up=s4_gu, q4_down=q4_d, s4_down=s4_d)
     out["route_norm_weight"] = None
     if cfg.route_norm:
         out["route_norm_weight"] = 1.0 + 0.1 * torch.randn((cfg.d,), generator=gen,

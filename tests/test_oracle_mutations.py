@@ -39,6 +39,13 @@ MUTATIONS = {
     "route_norm_weight_dropped": ("xr[c] = xr[c] * inv * (double)norm_w[c];", "xr[c] = xr[c] * inv;"),
     "route_norm_eps_outside_root": ("inv = 1.0 / sqrt(ms / d + norm_eps);",
                                     "inv = 1.0 / (sqrt(ms / d) + norm_eps);"),
+    "sqrt_softplus_without_root": ("return score_fn == 1 ? sqrt(softplus(z)) : sigmoid(z);",
+                                   "return score_fn == 1 ? softplus(z) : sigmoid(z);"),
+    "e2m1_exponent_bias": ("ldexp(1.0 + 0.5 * mant, ex - 1)", "ldexp(1.0 + 0.5 * mant, ex - 2)"),
+    "e8m0_bias": ("ldexp(1.0, (int)b - 127)", "ldexp(1.0, (int)b - 128)"),
+    "fp4_nibble_order": ("(off & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF)",
+                         "(off & 1) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4)"),
+    "fp4_block_size": ("(cols / 32) + c / 32]", "(cols / 32) + c / 64]"),
 }
 
 

@@ -497,3 +497,93 @@ def test_route_norm_leaves_the_experts_on_the_token():
     w = 2.826 * s / s.sum(axis=1, keepdims=True)
     want = sum(w[:, e:e + 1] * _np_expert(x64, wgu, wd, e, shape.F) for e in range(4))
     assert np.allclose(r["out_f64"], want, rtol=1e-9, atol=1e-12)
+
+
+# ------------------------------------------------------------------ the second routing and
+# precision variant: sqrt(softplus) scores, FP4 (E2M1 + E8M0 block-32) routed experts
+
+# OCP Microscaling (MX) formats v1.0: E2M1 magnitudes of codes 0..7 (bit 3 = sign)
+SPEC_E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _np_decode_fp4(packed, scales):
+    """Independent numpy decode: [..., rows, cols/2] nibbles + [..., rows, cols/32]
+    E8M0 bytes -> float64 [..., rows, cols]."""
+    lo, hi = packed & 0xF, packed >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(*packed.shape[:-1], packed.shape[-1] * 2)
+    mag = np.asarray(SPEC_E2M1)[codes & 7] * np.where(codes & 8, -1.0, 1.0)
+    sc = np.ldexp(1.0, scales.astype(np.int64) - 127)
+    return mag * np.repeat(sc, 32, axis=-1)
+
+
+def test_e2m1_decode_matches_the_spec_table():
+    got = oracle.double_from_e2m1(np.arange(16, dtype=np.uint8))
+    want = SPEC_E2M1 + [-v for v in SPEC_E2M1]
+    assert [float(v) for v in got] == want
+
+
+def test_e8m0_decode_is_a_power_of_two():
+    got = oracle.double_from_e8m0(np.array([127, 128, 120, 0, 254, 255], np.uint8))
+    assert list(got[:5]) == [1.0, 2.0, 2.0 ** -7, 2.0 ** -127, 2.0 ** 127]
+    assert math.isnan(got[5])
+
+
+def test_fp4_encoding_rounds_to_the_grid_within_half_a_step():
+    from synthetic.moe_inputs import encode_e2m1_blocks
+
+    w = (torch.randn((3, 64, 96), generator=torch.Generator().manual_seed(3)) * 0.02).to(
+        torch.bfloat16)
+    q, s = encode_e2m1_blocks(w)
+    dec = _np_decode_fp4(q.numpy(), s.numpy())
+    ref = _f64(w)
+    scale = np.repeat(np.ldexp(1.0, s.numpy().astype(np.int64) - 127), 32, axis=-1)
+    # the grid step at magnitude m (in scale units): 0.5 below 2, 1 below 4, 2 above
+    m = np.abs(ref) / scale
+    step = np.where(m < 2, 0.5, np.where(m < 4, 1.0, 2.0))
+    assert np.all(np.abs(dec - ref) <= 0.5 * step * scale + 1e-12)
+    assert np.all(np.abs(ref).reshape(3, 64, 3, 32).max(-1) <= 6 * scale[..., ::32] + 1e-12)
+
+
+def test_fp4_expert_is_the_textbook_mlp_on_decoded_weights():
+    shape = LayerShape(T=6, d=64, E=3, k=1, F=64, fp4=True)
+    L = _layer(shape, seed=61)
+    O = oracle.OracleLayer(L)
+    gu = _np_decode_fp4(O.wgu4, O.sgu8)
+    dn = _np_decode_fp4(O.wd4, O.sd8)
+    experts = np.array([0, 1, 2, 2, 1, 0], np.int32)
+    y = oracle.expert_rows_fp4(O.x, experts, O.wgu4, O.sgu8, O.wd4, O.sd8)
+    x64 = _f64(L["x"])
+    for r, e in enumerate(experts):
+        want = _np_expert(x64[r:r + 1], gu, dn, e, shape.F)[0]
+        assert np.allclose(y[r], want, rtol=1e-9, atol=1e-12)
+
+
+def test_sqrt_softplus_scores_and_weights():
+    shape = LayerShape(T=25, d=64, E=16, k=6, F=32, scale=1.5, score_fn="sqrtsoftplus")
+    L = _layer(shape, seed=62)
+    r = oracle.route(_bits(L["x"]), _bits(L["w_gate"]), 6, 1.5, want_scores=True,
+                     score_fn="sqrtsoftplus")
+    z = _np_logits(L)
+    s = np.sqrt(np.log1p(np.exp(z)))
+    assert np.allclose(r["scores"], s, rtol=1e-12)
+    for t in range(25):
+        want = sorted(range(16), key=lambda e: (-s[t, e], e))[:6]
+        assert list(r["idx"][t]) == want
+        assert list(r["idx"][t]) == sorted(range(16), key=lambda e: (-z[t, e], e))[:6]
+        assert np.allclose(r["w"][t], 1.5 * s[t, want] / s[t, want].sum(), rtol=1e-12)
+    x, wg = _unit_router([0.0, -1.0])
+    r1 = oracle.route(x, wg, 1, 1.5, want_scores=True, score_fn="sqrtsoftplus")
+    assert math.isclose(r1["scores"][0, 0], math.sqrt(math.log(2.0)), rel_tol=1e-15)
+    assert r1["idx"][0, 0] == 0 and r1["w"][0, 0] == 1.5
+
+
+def test_fp4_layer_routes_like_its_router_and_sums_its_experts():
+    shape = LayerShape(T=8, d=64, E=6, k=2, F=64, scale=1.5, fp4=True, score_fn="sqrtsoftplus")
+    L = _layer(shape, seed=63)
+    O = oracle.OracleLayer(L)
+    r = oracle.forward_tokens(O)
+    rr = oracle.route(O.x, O.wg, 2, 1.5, score_fn="sqrtsoftplus")
+    assert np.array_equal(r["idx"], rr["idx"]) and np.array_equal(r["w"], rr["w"])
+    y = oracle.expert_rows_fp4(np.repeat(O.x, 2, axis=0), r["idx"].reshape(-1), O.wgu4, O.sgu8,
+                               O.wd4, O.sd8).reshape(8, 2, 64)
+    assert np.allclose(r["out_f64"], (r["w"][:, :, None] * y).sum(axis=1), rtol=1e-12, atol=1e-15)
