@@ -151,6 +151,9 @@ static uint16_t double_to_bf16(double v)
 
 static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+/* SwiGLU's SiLU(g) * u, SiLU(z) = z * sigmoid(z). */
+static double silu_times(double g, double u) { return g * sigmoid(g) * u; }
+
 /* softplus(z) = ln(1 + e^z), evaluated without overflow. */
 static double softplus(double z) { return (z > 0.0) ? z + log1p(exp(-z)) : log1p(exp(z)); }
 
@@ -268,7 +271,7 @@ static void expert_token(int d, int F, long e, const uint16_t* xrow, const void*
             g += xc * weight_at(wgu, s_gu, e, 2L * F, d, f, c);
             u += xc * weight_at(wgu, s_gu, e, 2L * F, d, (long)F + f, c);
         }
-        hh[f] = g * sigmoid(g) * u;
+        hh[f] = silu_times(g, u);
     }
     for (i = 0; i < d; ++i) {
         double acc = 0.0;
@@ -294,7 +297,7 @@ static void expert_token_fp4(int d, int F, long e, const uint16_t* xrow, const u
             g += xc * weight_at_fp4(wgu, s_gu, e, 2L * F, d, f, c);
             u += xc * weight_at_fp4(wgu, s_gu, e, 2L * F, d, (long)F + f, c);
         }
-        hh[f] = g * sigmoid(g) * u;
+        hh[f] = silu_times(g, u);
     }
     for (i = 0; i < d; ++i) {
         double acc = 0.0;

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
 
 MUTATIONS = {
-    "silu_on_up_operand": ("hh[f] = g * sigmoid(g) * u;", "hh[f] = u * sigmoid(u) * g;"),
+    "silu_on_up_operand": ("return g * sigmoid(g) * u;", "return u * sigmoid(u) * g;"),
     "sigmoid_sign": ("return 1.0 / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(z));"),
     "no_renormalisation": ("w[j] = scale * order[j].s / sel_sum;", "w[j] = scale * order[j].s;"),
     "tie_break_to_higher_index": ("return (a->e < b->e) ? -1 : (a->e > b->e);",
