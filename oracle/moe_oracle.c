@@ -426,14 +426,16 @@ int oracle_expert_rows(int n, int d, int F, const uint16_t* xrows, const int32_t
 }
 
 /* Steps 1-6 for the n tokens listed in tokens[] (indices into x [T, d]), with
- * the optional score bias [E] and shared expert (sh_wgu [2F, d], sh_wd [d, F]
+ * the optional score bias [E], the optional RMSNorm of the router input
+ * (norm_w [d], norm_eps), the score function (0 sigmoid, 1 sqrt-softplus) and
+ * the optional shared expert (sh_wgu [2F, d], sh_wd [d, F]
  * in the routed experts' format, with row scales sh_s_gu [2F] / sh_s_d [d] for
  * e4m3 codes; sh_wgu NULL: no shared expert).
  * Outputs per listed token: out_f64 [n, d] (the fp64 sum before the cast),
  * out_bf16 [n, d], idx [n, k], w [n, k], gap [n]. */
 int oracle_forward_tokens2(int T, int d, int E, int k, int F, double scale, const uint16_t* x,
                            const uint16_t* wg, const float* gate_bias, const float* score_bias,
-                           const float* norm_w, double norm_eps,
+                           const float* norm_w, double norm_eps, int score_fn,
                            const void* wgu, const float* s_gu, const void* wd, const float* s_d,
                            const void* sh_wgu, const float* sh_s_gu, const void* sh_wd,
                            const float* sh_s_d, const int32_t* tokens, int n, double* out_f64,
@@ -442,7 +444,8 @@ int oracle_forward_tokens2(int T, int d, int E, int k, int F, double scale, cons
     long r;
     if (d <= 0 || E <= 0 || k <= 0 || k > E || F <= 0)
         return -1;
-    if ((sh_wgu == NULL) != (sh_wd == NULL) || (norm_w && !(norm_eps > 0.0)))
+    if ((sh_wgu == NULL) != (sh_wd == NULL) || (norm_w && !(norm_eps > 0.0)) || score_fn < 0 ||
+        score_fn > 1)
         return -1;
     for (r = 0; r < n; ++r)
         if (tokens[r] < 0 || tokens[r] >= T)
@@ -453,7 +456,7 @@ int oracle_forward_tokens2(int T, int d, int E, int k, int F, double scale, cons
         double* y = (double*)malloc(sizeof(double) * (size_t)k * d);
         double* ysh = sh_wgu ? (double*)malloc(sizeof(double) * (size_t)d) : NULL;
         int j;
-        route_token(d, E, k, scale, xrow, wg, gate_bias, score_bias, norm_w, norm_eps, 0,
+        route_token(d, E, k, scale, xrow, wg, gate_bias, score_bias, norm_w, norm_eps, score_fn,
                     idx + r * (long)k, w + r * (long)k, NULL, NULL, gap + r);
         for (j = 0; j < k; ++j)
             expert_token(d, F, idx[r * (long)k + j], xrow, wgu, s_gu, wd, s_d, NULL,
@@ -475,7 +478,7 @@ int oracle_forward_tokens(int T, int d, int E, int k, int F, double scale, const
                           const int32_t* tokens, int n, double* out_f64, uint16_t* out_bf16,
                           int32_t* idx, double* w, double* gap)
 {
-    return oracle_forward_tokens2(T, d, E, k, F, scale, x, wg, gate_bias, NULL, NULL, 0.0, wgu,
+    return oracle_forward_tokens2(T, d, E, k, F, scale, x, wg, gate_bias, NULL, NULL, 0.0, 0, wgu,
                                   s_gu, wd, s_d, NULL, NULL, NULL, NULL, tokens, n, out_f64,
                                   out_bf16, idx, w, gap);
 }

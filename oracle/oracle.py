@@ -54,8 +54,8 @@ def _load():
         lib.oracle_forward_tokens.argtypes = [I, I, I, I, I, D, P, P, P, P, P, P, P, P, I, P, P,
                                               P, P, P]
         lib.oracle_forward_tokens.restype = I
-        lib.oracle_forward_tokens2.argtypes = [I, I, I, I, I, D, P, P, P, P, P, D, P, P, P, P, P,
-                                               P, P, P, P, I, P, P, P, P, P]
+        lib.oracle_forward_tokens2.argtypes = [I, I, I, I, I, D, P, P, P, P, P, D, I, P, P, P, P,
+                                               P, P, P, P, P, I, P, P, P, P, P]
         lib.oracle_forward_tokens2.restype = I
         lib.oracle_combine.argtypes = [I, I, I, P, P, P]
         lib.oracle_double_from_e2m1.argtypes = [P, P, L]
@@ -228,7 +228,9 @@ def forward_tokens(layer: "OracleLayer", tokens=None):
                 "tokens": tokens}
     rc = _load().oracle_forward_tokens2(L.T, L.d, L.E, L.k, L.F, float(L.scale), _ptr(L.x),
                                         _ptr(L.wg), _ptr(L.gate_bias), _ptr(L.score_bias),
-                                        _ptr(L.norm_w), float(L.norm_eps), _ptr(L.wgu), _ptr(L.s_gu), _ptr(L.wd), _ptr(L.s_d),
+                                        _ptr(L.norm_w), float(L.norm_eps),
+                                        SCORE_FNS[L.score_fn], _ptr(L.wgu), _ptr(L.s_gu),
+                                        _ptr(L.wd), _ptr(L.s_d),
                                         _ptr(L.sh_wgu), _ptr(L.sh_s_gu), _ptr(L.sh_wd),
                                         _ptr(L.sh_s_d), _ptr(tokens), n, _ptr(out_f64),
                                         _ptr(out_bf16), _ptr(idx), _ptr(w), _ptr(gap))

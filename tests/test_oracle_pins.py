@@ -587,3 +587,14 @@ def test_fp4_layer_routes_like_its_router_and_sums_its_experts():
     y = oracle.expert_rows_fp4(np.repeat(O.x, 2, axis=0), r["idx"].reshape(-1), O.wgu4, O.sgu8,
                                O.wd4, O.sd8).reshape(8, 2, 64)
     assert np.allclose(r["out_f64"], (r["w"][:, :, None] * y).sum(axis=1), rtol=1e-12, atol=1e-15)
+
+
+def test_sqrt_softplus_layer_with_k_equal_E_is_the_dense_weighted_sum():
+    shape = LayerShape(T=10, d=64, E=4, k=4, F=32, scale=1.5, score_fn="sqrtsoftplus")
+    L = _layer(shape, seed=64)
+    r = oracle.forward_tokens(oracle.OracleLayer(L))
+    x64, wgu, wd = _f64(L["x"]), _f64(L["w_gate_up"]), _f64(L["w_down"])
+    s = np.sqrt(np.log1p(np.exp(_np_logits(L))))
+    w = 1.5 * s / s.sum(axis=1, keepdims=True)
+    want = sum(w[:, e:e + 1] * _np_expert(x64, wgu, wd, e, shape.F) for e in range(4))
+    assert np.allclose(r["out_f64"], want, rtol=1e-9, atol=1e-12)
