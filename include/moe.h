@@ -136,6 +136,25 @@ MOE_API int moe_route2(const moe_config* cfg, const void* x, const void* w_gate,
                const float* gate_bias, const float* score_bias, int32_t* topk_idx, float* topk_w,
                void* ws, size_t ws_bytes, void* stream);
 
+/* Optional router inputs of the complete Hy3 block, for moe_route3 /
+ * moe_forward3 (every pointer nullable: NULL turns the piece off).
+ *   score_bias   [E] fp32 e_score_correction_bias, as in moe_route2;
+ *   norm_weight  [d] fp32 route_norm weight ("Tencent Hy3-Flash QA" Q4.9):
+ *                the router scores xn = x / sqrt(mean(x^2) + norm_eps) * g
+ *                (the experts still take x); norm_eps > 0 (1e-6 is the
+ *                RMSNorm epsilon the pages give). */
+typedef struct moe_route_options {
+    const float* score_bias;
+    const float* norm_weight;
+    float norm_eps;
+} moe_route_options;
+
+/* moe_route with the options above (opt NULL: moe_route). With a norm weight
+ * the routing runs on the CUDA-core router at every batch size. */
+MOE_API int moe_route3(const moe_config* cfg, const void* x, const void* w_gate,
+               const float* gate_bias, const moe_route_options* opt, int32_t* topk_idx,
+               float* topk_w, void* ws, size_t ws_bytes, void* stream);
+
 /* Group token-slots by expert (the grouping defined above): writes counts [E],
  * offsets [E+1], row_of [T*k] (int32) and x_perm [T*k, d] bf16 with
  * x_perm[row_of[t*k+j]] = x[t]. Pages: the per-expert loop with index_add_ of
@@ -225,6 +244,12 @@ MOE_API int moe_pack_weights(const moe_config* cfg, int which, const void* w, vo
  * complete Hy3 MoE block. */
 MOE_API int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate,
                  const float* gate_bias, const float* score_bias, const void* w_gate_up,
+                 const float* s_gate_up, const void* w_down, const float* s_down, void* out,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* moe_forward with the router options of moe_route3 (opt NULL: moe_forward). */
+MOE_API int moe_forward3(const moe_config* cfg, const void* x, const void* w_gate,
+                 const float* gate_bias, const moe_route_options* opt, const void* w_gate_up,
                  const float* s_gate_up, const void* w_down, const float* s_down, void* out,
                  void* ws, size_t ws_bytes, void* stream);
 

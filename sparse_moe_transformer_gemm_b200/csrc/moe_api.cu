@@ -84,14 +84,25 @@ bool use_stream_path(const moe_config* c) {
 // of CTAs.
 constexpr int kRouterTcMinTokens = 129;
 
+// route_norm needs the per-token sum of squares next to the logits: the
+// CUDA-core router computes both exactly in fp32 (the tensor-core router's bf16
+// operands cannot carry x * g unrounded), so it serves every batch size then.
 cudaError_t route(const moe_config* c, const void* x, const void* w_gate, const float* gate_bias,
-                  const float* score_bias, int32_t* idx, float* w, void* ws, cudaStream_t s) {
+                  const float* score_bias, const float* norm_w, float norm_eps, int32_t* idx,
+                  float* w, void* ws, cudaStream_t s) {
     const WsLayout L = ws_layout(*c);
-    if (router_tc_supported(*c) && c->T >= kRouterTcMinTokens)
+    if (!norm_w && router_tc_supported(*c) && c->T >= kRouterTcMinTokens)
         return launch_router_tc(*c, x, w_gate, gate_bias, score_bias, idx, w,
                                 at<int>(ws, L.status), s);
-    return launch_router(*c, x, w_gate, gate_bias, score_bias, idx, w, at<float>(ws, L.logits),
+    return launch_router(*c, x, w_gate, gate_bias, score_bias, norm_w, norm_eps, idx, w,
+                         at<float>(ws, L.logits), at<float>(ws, L.sumsq),
                          at<int32_t>(ws, L.counters), router_ksplit(*c), s);
+}
+
+int check_route_options(const moe_route_options* opt) {
+    if (opt && opt->norm_weight && !(opt->norm_eps > 0.f && isfinite(opt->norm_eps)))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
 }
 
 int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offsets,
@@ -165,15 +176,24 @@ int moe_workspace_init(const moe_config* cfg, void* ws, size_t ws_bytes, void* s
                                        static_cast<cudaStream_t>(stream)));
 }
 
-int moe_route2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
-               const float* score_bias, int32_t* topk_idx, float* topk_w, void* ws,
+int moe_route3(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+               const moe_route_options* opt, int32_t* topk_idx, float* topk_w, void* ws,
                size_t ws_bytes, void* stream) {
     MOE_TRY(check_cfg(cfg));
     if (!x || !w_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_route_options(opt));
     MOE_TRY(check_ws(cfg, ws, ws_bytes));
-    return cuda_status(route(cfg, x, w_gate, gate_bias, score_bias, topk_idx, topk_w, ws,
-                             static_cast<cudaStream_t>(stream)));
+    return cuda_status(route(cfg, x, w_gate, gate_bias, opt ? opt->score_bias : nullptr,
+                             opt ? opt->norm_weight : nullptr, opt ? opt->norm_eps : 0.f,
+                             topk_idx, topk_w, ws, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+               const float* score_bias, int32_t* topk_idx, float* topk_w, void* ws,
+               size_t ws_bytes, void* stream) {
+    const moe_route_options opt = {score_bias, nullptr, 0.f};
+    return moe_route3(cfg, x, w_gate, gate_bias, &opt, topk_idx, topk_w, ws, ws_bytes, stream);
 }
 
 int moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
@@ -267,11 +287,12 @@ int moe_combine(const moe_config* cfg, const void* y, const int32_t* row_of, con
                                       static_cast<cudaStream_t>(stream)));
 }
 
-int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
-                 const float* score_bias, const void* w_gate_up, const float* s_gate_up,
+int moe_forward3(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+                 const moe_route_options* opt, const void* w_gate_up, const float* s_gate_up,
                  const void* w_down, const float* s_down, void* out, void* ws, size_t ws_bytes,
                  void* stream) {
     MOE_TRY(check_cfg(cfg));
+    MOE_TRY(check_route_options(opt));
     if (!x || !w_gate || !out || !aligned16(x) || !aligned16(w_gate) || !aligned16(out))
         return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_expert_weights(cfg, w_gate_up, s_gate_up));
@@ -289,7 +310,9 @@ int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const
     void* h = at<void>(ws, L.h);
     void* y = at<void>(ws, L.y);
     MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.control_end, s)));
-    MOE_TRY(cuda_status(route(cfg, x, w_gate, gate_bias, score_bias, idx, w, ws, s)));
+    MOE_TRY(cuda_status(route(cfg, x, w_gate, gate_bias, opt ? opt->score_bias : nullptr,
+                              opt ? opt->norm_weight : nullptr, opt ? opt->norm_eps : 0.f, idx,
+                              w, ws, s)));
     if (gather_batch(cfg)) {
         int32_t* tok = at<int32_t>(ws, L.tok);
         MOE_TRY(cuda_status(
@@ -305,10 +328,19 @@ int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const
     return cuda_status(launch_combine(*cfg, y, row_of, w, out, s));
 }
 
+int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+                 const float* score_bias, const void* w_gate_up, const float* s_gate_up,
+                 const void* w_down, const float* s_down, void* out, void* ws, size_t ws_bytes,
+                 void* stream) {
+    const moe_route_options opt = {score_bias, nullptr, 0.f};
+    return moe_forward3(cfg, x, w_gate, gate_bias, &opt, w_gate_up, s_gate_up, w_down, s_down,
+                        out, ws, ws_bytes, stream);
+}
+
 int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
                 const void* w_gate_up, const float* s_gate_up, const void* w_down,
                 const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream) {
-    return moe_forward2(cfg, x, w_gate, gate_bias, nullptr, w_gate_up, s_gate_up, w_down, s_down,
+    return moe_forward3(cfg, x, w_gate, gate_bias, nullptr, w_gate_up, s_gate_up, w_down, s_down,
                         out, ws, ws_bytes, stream);
 }
 

@@ -38,7 +38,7 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permut
             "moe_permute_index", "moe_expert_gate_up", "moe_expert_gate_up_gather",
             "moe_expert_down", "moe_experts", "moe_combine", "moe_forward", "moe_read_status",
             "moe_status_string", "moe_route_noalloc", "moe_pack_weights", "moe_route2",
-            "moe_forward2")
+            "moe_forward2", "moe_route3", "moe_forward3")
 
 MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 # batches of at most this many token-slots (T*k) gather their token rows inside
@@ -54,6 +54,18 @@ class MoeConfig(ctypes.Structure):
     def __repr__(self):
         return (f"MoeConfig(T={self.T}, d={self.d}, E={self.E}, k={self.k}, d_ff={self.d_ff}, "
                 f"scale={self.scale}, flags={self.flags:#x})")
+
+
+class MoeRouteOptions(ctypes.Structure):
+    """moe_route_options: score_bias [E], norm_weight [d] (device pointers), norm_eps."""
+    _fields_ = [("score_bias", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p),
+                ("norm_eps", ctypes.c_float)]
+
+
+def route_options(score_bias=None, norm_weight=None, norm_eps: float = 1e-6):
+    return MoeRouteOptions(None if score_bias is None else score_bias.data_ptr(),
+                           None if norm_weight is None else norm_weight.data_ptr(),
+                           float(norm_eps))
 
 
 class MoeError(RuntimeError):
@@ -94,6 +106,8 @@ def lib() -> ctypes.CDLL:
         "moe_pack_weights": (I, [C, I, P, P, P]),
         "moe_route2": (I, [C, P, P, P, P, P, P, P, S, P]),
         "moe_forward2": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "moe_route3": (I, [C, P, P, P, P, P, P, P, S, P]),
+        "moe_forward3": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -231,6 +245,22 @@ def moe_forward2(cfg, x, w_gate, gate_bias, score_bias, w_gate_up, s_gate_up, w_
            lib().moe_forward2(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
                               _p(score_bias), _p(w_gate_up), _p(s_gate_up), _p(w_down),
                               _p(s_down), _p(out), _p(ws), ws.numel(), _s(stream)))
+
+
+def moe_route3(cfg, x, w_gate, gate_bias, opt, topk_idx, topk_w, ws, stream=None) -> None:
+    _check("moe_route3", lib().moe_route3(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
+                                          None if opt is None else ctypes.byref(opt),
+                                          _p(topk_idx), _p(topk_w), _p(ws), ws.numel(),
+                                          _s(stream)))
+
+
+def moe_forward3(cfg, x, w_gate, gate_bias, opt, w_gate_up, s_gate_up, w_down, s_down, out, ws,
+                 stream=None) -> None:
+    _check("moe_forward3",
+           lib().moe_forward3(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
+                              None if opt is None else ctypes.byref(opt), _p(w_gate_up),
+                              _p(s_gate_up), _p(w_down), _p(s_down), _p(out), _p(ws), ws.numel(),
+                              _s(stream)))
 
 
 def moe_route_noalloc(cfg, x, w_gate, gate_bias, topk_idx, topk_w, stream=None) -> None:

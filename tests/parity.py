@@ -30,8 +30,9 @@ def gpu_route(layer, path=None):
     ws = moe.workspace(cfg)
     idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
     w = torch.empty((T, k), dtype=torch.float32, device="cuda")
-    moe.moe_route2(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"),
-                   layer.get("score_bias"), idx, w, ws)
+    opt = moe.route_options(layer.get("score_bias"), layer.get("route_norm_weight"),
+                            getattr(layer["cfg"], "route_norm_eps", 1e-6))
+    moe.moe_route3(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"), opt, idx, w, ws)
     torch.cuda.synchronize()
     assert moe.moe_read_status(ws) == moe.MOE_OK
     return idx.cpu().numpy(), w.cpu().numpy()
@@ -44,8 +45,10 @@ def gpu_forward(layer, path=None, ws=None, out=None):
         ws = moe.workspace(cfg)
     if out is None:
         out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
-    moe.moe_forward2(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"),
-                     layer.get("score_bias"), *moe.layer_args(layer), out, ws)
+    opt = moe.route_options(layer.get("score_bias"), layer.get("route_norm_weight"),
+                            getattr(layer["cfg"], "route_norm_eps", 1e-6))
+    moe.moe_forward3(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"), opt,
+                     *moe.layer_args(layer), out, ws)
     torch.cuda.synchronize()
     assert moe.moe_read_status(ws) == moe.MOE_OK
     return out
@@ -85,7 +88,8 @@ def oracle_out_with_selection(O, t, experts):
     """Oracle output of token t when it is routed to ``experts`` (weights from the
     oracle's fp64 sigmoid scores, renormalised over that set; the shared expert,
     if any, added last with weight 1)."""
-    scores = oracle.route(O.x[t:t + 1], O.wg, O.k, O.scale, O.gate_bias, want_scores=True)["scores"]
+    scores = oracle.route(O.x[t:t + 1], O.wg, O.k, O.scale, O.gate_bias, want_scores=True,
+                          norm_w=O.norm_w, norm_eps=O.norm_eps)["scores"]
     experts = np.asarray(experts, np.int32)
     xrows = np.repeat(O.x[t:t + 1], len(experts), axis=0)
     y = oracle.expert_rows(xrows, experts, O.wgu, O.wd, O.s_gu, O.s_d)

@@ -62,6 +62,20 @@ def test_shared_expert_flag_rules(lib):
     assert moe.moe_workspace_size(moe.config(**{**HY3, "E": 256})) > 0
 
 
+def test_route_options_are_checked_before_any_launch(lib):
+    cfg = moe.config(**HY3)
+    ws_n = moe.moe_workspace_size(cfg)
+    P = ctypes.c_void_p
+    bad = moe.MoeRouteOptions(None, FAKE, 0.0)      # a norm weight needs eps > 0
+    rc = _call("moe_route3", ctypes.byref(cfg), P(FAKE), P(FAKE), None, ctypes.byref(bad),
+               P(FAKE), P(FAKE), P(FAKE), ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    bad = moe.MoeRouteOptions(None, FAKE, float("nan"))
+    rc = _call("moe_forward3", ctypes.byref(cfg), P(FAKE), P(FAKE), None, ctypes.byref(bad),
+               P(FAKE), None, P(FAKE), None, P(FAKE), P(FAKE), ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+
+
 def test_pack_weights_rejects_bad_arguments(lib):
     P = ctypes.c_void_p
     cfg = moe.config(**HY3)
@@ -185,6 +199,8 @@ def test_unsupported_shape_is_reported_by_every_entry_point(lib):
         "moe_pack_weights": (moe.MOE_WEIGHTS_GATE_UP, f, P(FAKE + (1 << 34)), None),
         "moe_route2": (f, f, None, None, f, f, f, 1 << 30, None),
         "moe_forward2": (f, f, None, None, f, None, f, None, f, f, 1 << 30, None),
+        "moe_route3": (f, f, None, None, f, f, f, 1 << 30, None),
+        "moe_forward3": (f, f, None, None, f, None, f, None, f, f, 1 << 30, None),
     }
     for fn, args in cases.items():
         assert _call(fn, ctypes.byref(cfg), *args) == moe.MOE_ERR_UNSUPPORTED_SHAPE, fn

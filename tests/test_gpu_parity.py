@@ -326,6 +326,30 @@ def test_complete_block_with_packed_weights_is_bitwise_the_same():
     assert torch.equal(out, want)
 
 
+# route_norm (RMSNorm of the router's input; the experts take x)
+NORM = {
+    "norm_decode": dataclasses.replace(CONFIGS["decode"], route_norm=True),
+    "norm_tc_sized": LayerShape(T=300, d=512, E=32, k=8, F=256, route_norm=True),
+    "norm_block": LayerShape(T=200, d=512, E=16, k=4, F=512, shared=True, score_bias_std=0.05,
+                             route_norm=True),
+}
+
+
+@pytest.mark.parametrize("name", sorted(NORM))
+def test_route_norm_every_token(name):
+    sh = NORM[name]
+    layer = make_layer(sh, seed=51, device="cuda")
+    route = parity.gpu_route(layer)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias, score_bias=O.score_bias,
+                       norm_w=O.norm_w, norm_eps=O.norm_eps)
+    parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer)
+    res = parity.check_forward(layer, out, None, route)
+    print(name, res)
+    _free(layer, out)
+
+
 def test_fp32_combine_keeps_small_terms():
     """Hy3 commentary §2.3 example: one branch output 8.2 and seven of 0.03 (all
     already bf16). An fp32 sum gives 8.375 after the cast; a bf16 running sum
