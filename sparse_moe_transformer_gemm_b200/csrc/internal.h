@@ -104,13 +104,13 @@ inline WsLayout ws_layout(const moe_config& c) {
 // ---- launchers (each returns cudaError_t of the launch) ----
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
                           const float* gate_bias, const float* score_bias, const float* norm_w,
-                          float norm_eps, int32_t* idx, float* w, float* logits, float* sumsq,
-                          int32_t* counters, int ksplit, cudaStream_t s);
+                          float norm_eps, int score_fn, int32_t* idx, float* w, float* logits,
+                          float* sumsq, int32_t* counters, int ksplit, cudaStream_t s);
 
 bool router_tc_supported(const moe_config& c);
 cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_gate,
-                             const float* gate_bias, const float* score_bias, int32_t* idx,
-                             float* w, int* status, cudaStream_t s);
+                             const float* gate_bias, const float* score_bias, int score_fn,
+                             int32_t* idx, float* w, int* status, cudaStream_t s);
 
 cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
                            int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,
@@ -123,10 +123,10 @@ cudaError_t launch_gather_rows(const moe_config& c, const void* x, const int32_t
                                const int32_t* offsets, void* x_perm, cudaStream_t s);
 
 cudaError_t launch_gate_up_stream(const moe_config& c, const void* x_perm, const int32_t* offsets,
-                                  const void* w_gate_up, const float* s_gate_up, void* h,
+                                  const void* w_gate_up, const void* s_gate_up, void* h,
                                   cudaStream_t s);
 cudaError_t launch_down_stream(const moe_config& c, const void* h, const int32_t* offsets,
-                               const void* w_down, const float* s_down, void* y, cudaStream_t s);
+                               const void* w_down, const void* s_down, void* y, cudaStream_t s);
 
 cudaError_t launch_gate_up_gemm(const moe_config& c, const void* x_perm, const int32_t* offsets,
                                 const void* w_gate_up, void* h, int* status, cudaStream_t s);

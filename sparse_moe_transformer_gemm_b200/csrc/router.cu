@@ -20,6 +20,8 @@
 // this selects the k largest scores -- and the sigmoid of the k selected. With
 // an e_score_correction_bias ("Tencent Hy3-295B 架构深度拆解" §4.1 step 2) the
 // choice ranks sigmoid + bias and the weights renormalise the sigmoid scores.
+// With score_fn 1 every "sigmoid" above reads sqrt(softplus(logit)) (the
+// V4-Flash router of the same page, §2.2), also increasing in the logit.
 #include "common.cuh"
 #include "internal.h"
 
@@ -44,8 +46,8 @@ __device__ __forceinline__ void load_w(uint4 (&u)[EPW], const __nv_bfloat16* __r
 __global__ void __launch_bounds__(RWARPS * 32, kRouterCtasPerSm)
 router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wg,
               const float* __restrict__ bias, const float* __restrict__ sbias,
-              const float* __restrict__ norm_w, float norm_eps, int T, int d, int E, int k,
-              float scale, float* __restrict__ logits, float* __restrict__ sumsq,
+              const float* __restrict__ norm_w, float norm_eps, int score_fn, int T, int d,
+              int E, int k, float scale, float* __restrict__ logits, float* __restrict__ sumsq,
               int* __restrict__ counters, int* __restrict__ idx_out, float* __restrict__ w_out) {
     __shared__ __align__(16) float xs[RT][KC];
     __shared__ int s_last;
@@ -193,12 +195,14 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const int e = lane + 32 * q;
-                prob[q] = (e < E) ? sigmoidf_acc(sc[q]) : 0.f;
+                prob[q] = (e < E) ? score_value(sc[q], score_fn) : 0.f;
                 sc[q] = (e < E) ? prob[q] + sbias[e] : -INFINITY;
             }
-            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k, prob);
+            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k, prob,
+                             score_fn);
         } else {
-            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k);
+            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k,
+                             nullptr, score_fn);
         }
     }
     if (threadIdx.x == 0) counters[blockIdx.y] = 0;
@@ -208,12 +212,12 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
                           const float* gate_bias, const float* score_bias, const float* norm_w,
-                          float norm_eps, int32_t* idx, float* w, float* logits, float* sumsq,
-                          int32_t* counters, int ksplit, cudaStream_t s) {
+                          float norm_eps, int score_fn, int32_t* idx, float* w, float* logits,
+                          float* sumsq, int32_t* counters, int ksplit, cudaStream_t s) {
     dim3 grid((c.E + RE - 1) / RE, n_router_groups(c), ksplit);
     router_kernel<<<grid, RWARPS * 32, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_gate), gate_bias,
-        score_bias, norm_w, norm_eps, c.T, c.d, c.E, c.k, c.scale, logits, sumsq, counters, idx,
+        score_bias, norm_w, norm_eps, score_fn, c.T, c.d, c.E, c.k, c.scale, logits, sumsq, counters, idx,
         w);
     return cudaGetLastError();
 }

@@ -31,8 +31,12 @@ MOE_FLAG_STREAM_PATH = 0x2
 MOE_FLAG_GEMM_PATH = 0x4
 MOE_FLAG_PACKED_WEIGHTS = 0x8
 MOE_FLAG_SHARED_EXPERT = 0x10
+MOE_FLAG_FP4_WEIGHTS = 0x20
 MOE_WEIGHTS_GATE_UP = 0
 MOE_WEIGHTS_DOWN = 1
+MOE_SCORE_SIGMOID = 0
+MOE_SCORE_SQRT_SOFTPLUS = 1
+SCORE_FNS = {"sigmoid": MOE_SCORE_SIGMOID, "sqrtsoftplus": MOE_SCORE_SQRT_SOFTPLUS}
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
             "moe_permute_index", "moe_expert_gate_up", "moe_expert_gate_up_gather",
@@ -57,15 +61,19 @@ class MoeConfig(ctypes.Structure):
 
 
 class MoeRouteOptions(ctypes.Structure):
-    """moe_route_options: score_bias [E], norm_weight [d] (device pointers), norm_eps."""
+    """moe_route_options: score_bias [E], norm_weight [d] (device pointers), norm_eps,
+    score_fn (MOE_SCORE_*)."""
     _fields_ = [("score_bias", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p),
-                ("norm_eps", ctypes.c_float)]
+                ("norm_eps", ctypes.c_float), ("score_fn", ctypes.c_int32)]
 
 
-def route_options(score_bias=None, norm_weight=None, norm_eps: float = 1e-6):
+def route_options(score_bias=None, norm_weight=None, norm_eps: float = 1e-6,
+                  score_fn: str = "sigmoid"):
+    """Router options; score_fn is "sigmoid" or "sqrtsoftplus" (or a MOE_SCORE_* value)."""
+    fn = SCORE_FNS[score_fn] if isinstance(score_fn, str) else int(score_fn)
     return MoeRouteOptions(None if score_bias is None else score_bias.data_ptr(),
                            None if norm_weight is None else norm_weight.data_ptr(),
-                           float(norm_eps))
+                           float(norm_eps), fn)
 
 
 class MoeError(RuntimeError):
@@ -118,11 +126,15 @@ def lib() -> ctypes.CDLL:
 
 
 def config(T: int, d: int, E: int, k: int, d_ff: int, scale: float = 2.826, fp8: bool = False,
-           path: Optional[str] = None, packed: bool = False, shared: bool = False) -> MoeConfig:
+           path: Optional[str] = None, packed: bool = False, shared: bool = False,
+           fp4: bool = False) -> MoeConfig:
     """Build a moe_config. path: None (automatic), "stream" or "gemm"; packed: the
     bf16 expert weights are in moe_pack_weights' layout; shared: expert E of the
-    weight arrays is a shared expert."""
+    weight arrays is a shared expert; fp4: E2M1 expert weights with E8M0 block
+    scales."""
     flags = MOE_FLAG_FP8_WEIGHTS if fp8 else 0
+    if fp4:
+        flags |= MOE_FLAG_FP4_WEIGHTS
     if packed:
         flags |= MOE_FLAG_PACKED_WEIGHTS
     if shared:
@@ -282,9 +294,11 @@ def moe_read_status(ws, stream=None) -> int:
 
 
 def layer_args(layer: dict):
-    """(w_gate_up, s_gate_up, w_down, s_down) of a synthetic layer dict, FP8 or bf16;
-    with a shared expert, its weights follow the routed ones as expert E."""
+    """(w_gate_up, s_gate_up, w_down, s_down) of a synthetic layer dict, FP4, FP8 or
+    bf16; with a shared expert, its weights follow the routed ones as expert E."""
     cfg = layer["cfg"]
+    if getattr(cfg, "fp4", False):
+        return (layer["q4_gate_up"], layer["s4_gate_up"], layer["q4_down"], layer["s4_down"])
     if cfg.fp8:
         args = [layer["q_gate_up"], layer["s_gate_up"], layer["q_down"], layer["s_down"]]
         sh = ("q_shared_gate_up", "s_shared_gate_up", "q_shared_down", "s_shared_down")
@@ -299,7 +313,7 @@ def layer_args(layer: dict):
 def config_of(shape, path: Optional[str] = None, packed: bool = False) -> MoeConfig:
     """moe_config for a synthetic LayerShape."""
     return config(shape.T, shape.d, shape.E, shape.k, shape.F, shape.scale, shape.fp8, path,
-                  packed, getattr(shape, "shared", False))
+                  packed, getattr(shape, "shared", False), getattr(shape, "fp4", False))
 
 
 def pack_layer_weights(cfg: MoeConfig, w_gate_up: torch.Tensor, w_down: torch.Tensor,
