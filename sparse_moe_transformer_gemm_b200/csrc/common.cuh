@@ -40,13 +40,10 @@ __device__ __forceinline__ void e4m3x16_to_float(const uint4& v, float f[16]) {
 }
 
 // Sixteen E2M1 codes in two 32-bit words (two per byte, the even element in
-// the low nibble, words and bytes in increasing element order), times the
-// power-of-two block scale s -> sixteen floats, exactly: the hardware
-// e2m1x2 -> f16x2 conversion takes the low nibble to the low half, every E2M1
-// value is an f16 value, and a product with a power of two stays exact in
-// fp32 down to its subnormals.
-__device__ __forceinline__ void e2m1x16_to_float(uint32_t w0, uint32_t w1, float s,
-                                                 float f[16]) {
+// the low nibble, words and bytes in increasing element order) -> sixteen
+// floats, exactly: the hardware e2m1x2 -> f16x2 conversion takes the low
+// nibble to the low half, and every E2M1 value is an f16 value.
+__device__ __forceinline__ void e2m1x16_to_float(uint32_t w0, uint32_t w1, float f[16]) {
     const uint32_t w[2] = {w0, w1};
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -55,8 +52,8 @@ __device__ __forceinline__ void e2m1x16_to_float(uint32_t w0, uint32_t w1, float
             __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(
                 (__nv_fp4x2_storage_t)((w[i] >> (8 * j)) & 0xFFu), __NV_E2M1);
             const float2 p = __half22float2(*reinterpret_cast<__half2*>(&h));
-            f[8 * i + 2 * j] = p.x * s;
-            f[8 * i + 2 * j + 1] = p.y * s;
+            f[8 * i + 2 * j] = p.x;
+            f[8 * i + 2 * j + 1] = p.y;
         }
     }
 }
