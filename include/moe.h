@@ -278,6 +278,13 @@ MOE_API int moe_forward3(const moe_config* cfg, const void* x, const void* w_gat
                  const void* s_gate_up, const void* w_down, const void* s_down, void* out,
                  void* ws, size_t ws_bytes, void* stream);
 
+/* Failure-detection self-test: one thread waits, with the library's bounded
+ * wait and a limit of limit_ns (1 ns .. 10 s), on an mbarrier that nothing
+ * completes, then records MOE_ERR_TIMEOUT in the status word of ws (read it
+ * with moe_read_status). Faults, traps and hangs nothing; the context stays
+ * usable. Not part of the layer (the pages have no counterpart). */
+MOE_API int moe_selftest_bounded_wait(void* ws, unsigned long long limit_ns, void* stream);
+
 /* Bytes of the fixed device array behind moe_route_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES (2u << 20)
 

@@ -42,7 +42,7 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permut
             "moe_permute_index", "moe_expert_gate_up", "moe_expert_gate_up_gather",
             "moe_expert_down", "moe_experts", "moe_combine", "moe_forward", "moe_read_status",
             "moe_status_string", "moe_route_noalloc", "moe_pack_weights", "moe_route2",
-            "moe_forward2", "moe_route3", "moe_forward3")
+            "moe_forward2", "moe_route3", "moe_forward3", "moe_selftest_bounded_wait")
 
 MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 # batches of at most this many token-slots (T*k) gather their token rows inside
@@ -116,6 +116,7 @@ def lib() -> ctypes.CDLL:
         "moe_forward2": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
         "moe_route3": (I, [C, P, P, P, P, P, P, P, S, P]),
         "moe_forward3": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "moe_selftest_bounded_wait": (I, [P, ctypes.c_ulonglong, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -287,6 +288,12 @@ def moe_pack_weights(cfg, which, w, w_packed, stream=None) -> None:
     """Rearrange one bf16 expert weight into the packed 128 x 64 block layout."""
     _check("moe_pack_weights", lib().moe_pack_weights(ctypes.byref(cfg), int(which), _p(w),
                                                       _p(w_packed), _s(stream)))
+
+
+def moe_selftest_bounded_wait(ws, limit_ns: int, stream=None) -> None:
+    """Run the bounded-wait self-test; its MOE_ERR_TIMEOUT lands in ws's status word."""
+    _check("moe_selftest_bounded_wait",
+           lib().moe_selftest_bounded_wait(_p(ws), int(limit_ns), _s(stream)))
 
 
 def moe_read_status(ws, stream=None) -> int:
