@@ -1,16 +1,38 @@
-// common.cuh -- small device helpers shared by the library's kernels.
+// common.cuh -- small device helpers shared by the library's kernels (the
+// bit-level ones also compile as host code, for host-side checks).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace moe {
 
+// Bit casts between float and uint32_t, for host and device code.
+__host__ __device__ __forceinline__ float f32_from_bits(uint32_t u) {
+#ifdef __CUDA_ARCH__
+    return __uint_as_float(u);
+#else
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+#endif
+}
+__host__ __device__ __forceinline__ uint32_t f32_bits(float f) {
+#ifdef __CUDA_ARCH__
+    return __float_as_uint(f);
+#else
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return u;
+#endif
+}
+
 // bf16 pair (packed in a 32-bit word, low half first) -> two floats. Exact.
-__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
-    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+__host__ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
+    return make_float2(f32_from_bits(v << 16), f32_from_bits(v & 0xFFFF0000u));
 }
 
 // Eight bf16 in a 16-byte vector -> eight floats.
@@ -65,12 +87,14 @@ __device__ __forceinline__ float e8m0_to_float(uint32_t b) {
 }
 
 // Round a float to bf16 (nearest-even) and return the 16-bit pattern.
-__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+__host__ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
     __nv_bfloat16 b = __float2bfloat16_rn(f);
-    return *reinterpret_cast<uint16_t*>(&b);
+    uint16_t u;
+    memcpy(&u, &b, sizeof u);
+    return u;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+__host__ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return (uint32_t)float_to_bf16_bits(lo) | ((uint32_t)float_to_bf16_bits(hi) << 16);
 }
 
@@ -111,12 +135,12 @@ __device__ __forceinline__ float score_value(float z, int score_fn) {
 // index). The score function (score_value) is increasing, so these are the k
 // largest scores. Lane j < k writes the j-th selection: idx_row[j] and
 // w_row[j] = scale * score_j / sum of the k scores (summed in j order).
-__device__ __forceinline__ uint32_t order_key(float f) {
-    const uint32_t b = __float_as_uint(f + 0.0f);  // -0 -> +0
+__host__ __device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t b = f32_bits(f + 0.0f);  // -0 -> +0
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
-__device__ __forceinline__ float key_value(uint32_t key) {
-    return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+__host__ __device__ __forceinline__ float key_value(uint32_t key) {
+    return f32_from_bits((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
 }
 
 //

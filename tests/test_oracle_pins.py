@@ -286,6 +286,22 @@ def test_per_expert_parameter_count_matches_the_page(golden):
     assert round((gu + dn) / 1e6, 2) * 1e6 == g["params_per_expert"]
 
 
+def test_second_variant_shapes_match_the_page(golden):
+    """The V4-Flash MoE column (the second routing and precision variant): the
+    generator's tensors at its shape give the printed ~25.2M parameters per
+    expert, and top-6 x 2048 covers the same intermediate width as Hy3's
+    top-8 x 1536."""
+    g = golden["v4_flash_moe"]
+    shp = tensor_shapes(LayerShape(T=64, d=g["d"], E=g["n_routed_experts"], k=g["top_k"],
+                                   F=g["d_ff_expert"], scale=g["routed_scaling_factor"],
+                                   score_fn="sqrtsoftplus", fp4=True))
+    per_expert = math.prod(shp["w_gate_up"][1:]) + math.prod(shp["w_down"][1:])
+    assert per_expert == 3 * 4096 * 2048 == 25_165_824
+    assert round(per_expert / 1e6, 1) * 1e6 == g["params_per_expert_printed"]
+    assert g["top_k"] * g["d_ff_expert"] == g["total_intermediate_per_token"] == 8 * 1536
+    assert shp["w_gate"] == (256, 4096)
+
+
 def test_per_expert_flops_match_the_page(golden):
     f = work.expert_flops_per_token(4096, 1536)
     assert f == 37_748_736
