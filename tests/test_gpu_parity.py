@@ -472,3 +472,38 @@ def test_fp4_decode_hy3_shape():
     res = parity.check_forward(layer, out, toks, route)
     print("fp4 decode, near ties:", len(near), res)
     _free(layer, out)
+
+
+# The largest supported shapes: 256 experts with k = 32 (the CUDA-core router's
+# 32 rounds, the one-CTA grouping over 256 experts, the 32-row combine), and
+# d = d_ff = 8192 (128 KB of staged rows on the streaming path, 128 K blocks
+# on the pair GEMMs).
+MAX = {
+    "e256_k32": LayerShape(T=40, d=256, E=256, k=32, F=128),
+    "d8192": LayerShape(T=16, d=8192, E=8, k=2, F=8192),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MAX))
+@pytest.mark.parametrize("path", [None, "stream", "gemm"])
+def test_largest_supported_shapes_every_token(name, path):
+    sh = MAX[name]
+    layer = make_layer(sh, seed=81, device="cuda")
+    route = parity.gpu_route(layer, path)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias)
+    parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer, path)
+    res = parity.check_forward(layer, out, None, route)
+    print(name, path, res)
+    _free(layer, out)
+
+
+@pytest.mark.parametrize("T", [16, 200])
+def test_router_at_d8192_on_both_kernels(T):
+    shape = LayerShape(T=T, d=8192, E=256, k=8, F=128, zipf_bias=True)
+    layer = make_layer(shape, seed=83, device="cuda", with_experts=False)
+    route = parity.gpu_route(layer)
+    ref = oracle.route(oracle.bf16_bits(layer["x"]), oracle.bf16_bits(layer["w_gate"]), shape.k,
+                       shape.scale, layer["gate_bias"].cpu().numpy())
+    parity.check_route(*route, ref)
