@@ -1,6 +1,7 @@
 """Benchmark of the routed-MoE FFN layer (Hy3 shapes) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|prefill|skewed|fp8]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--config decode|prefill|skewed|fp8|fp4_decode]
                     [--impl ours|reference] [--path auto|stream|gemm]
 
 One step = one pass of the whole layer (route, group, gate_up, down, combine)
@@ -10,11 +11,11 @@ own batch (tokens are independent: no collective on the data path) and the
 value is the tokens of all ranks over the slowest rank's time.
 
 The step is timed through the public entry points one stage at a time
-(moe_route, moe_permute_index or moe_permute, moe_expert_gate_up_gather or
+(moe_route3, moe_permute_index or moe_permute, moe_expert_gate_up_gather or
 moe_expert_gate_up, moe_expert_down, moe_combine -- the same sequence
-moe_forward runs), with CUDA events on the launching stream; ``e2e`` times
-moe_forward with the input copied in from and the output copied back to pinned
-host memory every step. bf16 expert weights for the tensor-core kernels are
+moe_forward3 runs), with CUDA events on the launching stream; ``e2e`` times
+moe_forward3 with the input copied in from and the output copied back to
+pinned host memory every step. bf16 expert weights for the tensor-core kernels are
 packed once at load (moe_pack_weights), outside every timed region.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (each
@@ -46,6 +47,9 @@ WORKLOADS = {
     "skewed": "Hy3 MoE layer, skewed routing: T=16384, logit bias 0.5*ln(Zipf(1.1) rank weight)",
     "fp8": "Hy3 MoE layer FP8 weights: T=8192, experts e4m3 + fp32 per-output-row scales",
     "tiny": "Tiny MoE layer: T=64, d=256, E=16, top-4, d_ff=128",
+    "fp4_decode": "Second routing/precision variant at the Hy3 decode shape: T=64, d=4096, "
+                  "E=192, top-6 sqrt-softplus scores (scale 1.5), d_ff=1536, experts E2M1 + "
+                  "E8M0 block-32 scales",
 }
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of the dominant kernel, from
@@ -266,7 +270,8 @@ def main():
     T, d, E, k, F = shape.T, shape.d, shape.E, shape.k, shape.F
     # bf16 weights on the tensor-core pair kernels are packed once, at load time
     # (moe_pack_weights), outside every timed region
-    packed = not shape.fp8 and args.path != "stream" and d % 256 == 0 and F % 256 == 0
+    packed = (not shape.fp8 and not shape.fp4 and args.path != "stream" and d % 256 == 0 and
+              F % 256 == 0)
     cfg = moe.config_of(shape, None if args.path == "auto" else args.path, packed=packed)
     # grouped slots per token (the shared expert, when present, is slot k of
     # every token and expert E)
@@ -280,6 +285,8 @@ def main():
         wgu, wd = moe.pack_layer_weights(cfg, wgu, wd)
         torch.cuda.synchronize(dev)
     x, wg, gb, sb = layer["x"], layer["w_gate"], layer["gate_bias"], layer["score_bias"]
+    # router options: the score bias (complete Hy3 block) and the score function
+    ropt = moe.route_options(sb, None, 1e-6, shape.score_fn)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
     counts = torch.empty(Eg, dtype=torch.int32, device=dev)
@@ -296,14 +303,15 @@ def main():
     # small batches: one grouping launch, and gate_up gathers its token rows inside
     # the GEMM on the bf16 SM-pair path (a row-gather kernel first on the others);
     # large batches: rank/scan/scatter with the permuted copy, then gate_up
-    fused_gather = (not shape.fp8 and args.path != "stream" and d % 256 == 0 and F % 256 == 0)
+    fused_gather = (not shape.fp8 and not shape.fp4 and args.path != "stream" and
+                    d % 256 == 0 and F % 256 == 0)
     n_launch = {"route": 1, "permute": 1 if gather else 3,
                 "gate_up": 2 if gather and not fused_gather else 1, "down": 1, "combine": 1}
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        moe.moe_route2(cfg, x, wg, gb, sb, idx, w, ws, stream)
+        moe.moe_route3(cfg, x, wg, gb, ropt, idx, w, ws, stream)
         if ev is not None:
             ev[1].record(stream)
         if gather:
@@ -356,20 +364,20 @@ def main():
     touched = int((counts > 0).sum().item())
     rows = int(offsets[-1].item())
     peaks, peak_src = load_peaks()
-    fp8 = shape.fp8
+    fp8, fp4 = shape.fp8, shape.fp4
     # the shared expert counts as one more touched expert with T more rows
-    lw = work.layer_work(T, d, E, ks, F, touched, fp8)
-    gw = work.gate_up_work(rows, touched, d, F, fp8)
-    dw = work.down_work(rows, touched, d, F, fp8)
+    lw = work.layer_work(T, d, E, ks, F, touched, fp8, fp4)
+    gw = work.gate_up_work(rows, touched, d, F, fp8, fp4)
+    dw = work.down_work(rows, touched, d, F, fp8, fp4)
     dominant = max(("gate_up", "down"), key=lambda s: stage_ms[s])
     dom_work = gw if dominant == "gate_up" else dw
     dom_s = stage_ms[dominant] / 1e3
-    use_stream = args.path == "stream"
+    use_stream = args.path == "stream" or fp4  # FP4 experts: the streaming kernels
     kernel_name = f"{dominant}_{'stream' if use_stream else 'gemm'}"
     # The metric's roofline: HBM for the decode workload (weights streamed once),
     # dense bf16 tensor peak for the larger batches. The tensor peak is the
     # sustained one: the kernel is timed inside a seconds-long loop.
-    if args.config in ("decode", "tiny"):
+    if args.config in ("decode", "tiny", "fp4_decode"):
         achieved = dom_work["bytes"] / dom_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
@@ -415,7 +423,8 @@ def main():
             stream.wait_event(h2d)
             if d2h[b] is not None:
                 stream.wait_event(d2h[b])  # step i-2's output has been read back
-            moe.moe_forward2(cfg, x_dev[b], wg, gb, sb, wgu, sgu, wd, sd, out_dev[b], ws, stream)
+            moe.moe_forward3(cfg, x_dev[b], wg, gb, ropt, wgu, sgu, wd, sd, out_dev[b], ws,
+                             stream)
             fwd[b] = torch.cuda.Event()
             fwd[b].record(stream)
             with torch.cuda.stream(d2h_stream):
@@ -456,6 +465,7 @@ def main():
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 weights, bf16 activations, fp32 accumulate" if fp8 else
+                     "e2m1 weights, bf16 activations, fp32 accumulate" if fp4 else
                      "bf16 (fp32 accumulate, fp32 combine)",
             "data": "synthetic (seeded; random-init weights of the Hy3 MoE layer shapes)",
             "config": {"workload": (WORKLOADS[args.config] if shape == CONFIGS[args.config] else
@@ -466,10 +476,12 @@ def main():
                        "T": T, "d": d, "E": E, "k": k,
                        "d_ff": F, "path": args.path, "parallelism": f"replicas x{world}",
                        "weights": ("e4m3 + fp32 row scales" if fp8 else
+                                   "e2m1 + e8m0 block-32 scales" if fp4 else
                                    "bf16, packed in 128x64 blocks once at load (moe_pack_weights)"
                                    if packed else "bf16, row-major"),
                        "l2": "no flush: each step streams the touched experts' weights "
-                             f"({touched} experts, {touched * work.expert_bytes(d, F, fp8) / 1e9:.2f} GB) "
+                             f"({touched} experts, "
+                             f"{touched * work.expert_bytes(d, F, fp8, fp4) / 1e9:.2f} GB) "
                              "through the 126 MB L2"},
             "roofline": roof,
             "layer_roofline": {
@@ -481,7 +493,7 @@ def main():
             "clocks": clocks.summary(),
             "e2e": {"value": replica_value(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
-                    "ms_per_step": e2e_ms, "api": "moe_forward2",
+                    "ms_per_step": e2e_ms, "api": "moe_forward3",
                     "copies": "one stream per direction, double-buffered, overlapping the compute",
                     "output_equals_staged": e2e_same},
             "gpu_launches": sum(n_launch.values()) * args.steps,

@@ -24,7 +24,20 @@
  * - FP8 weights (MOE_FLAG_FP8_WEIGHTS): w_gate_up / w_down hold e4m3 codes
  *   (one byte each) in the same layouts, and s_gate_up [E, 2*d_ff] /
  *   s_down [E, d] hold fp32 per-output-row scales; the weight value is
- *   code * scale. Without the flag both scale pointers must be NULL.
+ *   code * scale. Without the FP8 or FP4 flag both scale pointers must be
+ *   NULL (the scale pointers are void* because their element type follows
+ *   the weight format).
+ * - FP4 weights (MOE_FLAG_FP4_WEIGHTS; the V4-Flash column of "Tencent
+ *   Hy3-295B 架构深度拆解" §2.2, OCP MX E2M1 with block-32 scales):
+ *   w_gate_up [E, 2*d_ff, d/2] / w_down [E, d, d_ff/2] hold E2M1 codes two to
+ *   a byte, the even column in the low nibble (bit 3 the sign, bits 2-1 the
+ *   exponent, bit 0 the mantissa: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), and
+ *   s_gate_up [E, 2*d_ff, d/32] / s_down [E, d, d_ff/32] hold one E8M0 byte b
+ *   per 32 consecutive columns of a row, the block's scale 2^(b - 127)
+ *   (b = 255 is not a scale: unspecified output). The weight value is
+ *   code value * block scale. The experts run on the weight-streaming kernels
+ *   (MOE_FLAG_GEMM_PATH, MOE_FLAG_FP8_WEIGHTS, MOE_FLAG_PACKED_WEIGHTS or
+ *   MOE_FLAG_SHARED_EXPERT with it: MOE_ERR_INVALID_ARG).
  * - Packed bf16 weights (MOE_FLAG_PACKED_WEIGHTS): w_gate_up and w_down hold
  *   the same values rearranged by moe_pack_weights into 16 KB blocks of 128
  *   rows x 64 columns (block (e, rb, kb) = rows [128 rb, 128 rb + 128) and
@@ -93,6 +106,7 @@ extern "C" {
 #define MOE_FLAG_GEMM_PATH 0x4u   /* experts on the tensor-core grouped GEMMs */
 #define MOE_FLAG_PACKED_WEIGHTS 0x8u /* bf16 expert weights in moe_pack_weights' layout */
 #define MOE_FLAG_SHARED_EXPERT 0x10u /* expert E of the weights is a shared expert (below) */
+#define MOE_FLAG_FP4_WEIGHTS 0x20u /* expert weights are E2M1 codes + E8M0 block-32 scales */
 
 /* Which expert weight moe_pack_weights rearranges. */
 #define MOE_WEIGHTS_GATE_UP 0 /* w_gate_up [E, 2*d_ff, d] */
@@ -136,6 +150,36 @@ MOE_API int moe_route2(const moe_config* cfg, const void* x, const void* w_gate,
                const float* gate_bias, const float* score_bias, int32_t* topk_idx, float* topk_w,
                void* ws, size_t ws_bytes, void* stream);
 
+/* Router score functions (moe_route_options.score_fn). Both are increasing in
+ * the logit, so the choice is the k largest logits either way. */
+#define MOE_SCORE_SIGMOID 0       /* s = 1 / (1 + e^-z) (Hy3) */
+#define MOE_SCORE_SQRT_SOFTPLUS 1 /* s = sqrt(log(1 + e^z)) (the V4-Flash router,
+                                     "Tencent Hy3-295B 架构深度拆解" §2.2) */
+
+/* Optional router inputs, for moe_route3 / moe_forward3 (every pointer
+ * nullable: NULL turns the piece off).
+ *   score_bias   [E] fp32 e_score_correction_bias, as in moe_route2;
+ *   norm_weight  [d] fp32 route_norm weight ("Tencent Hy3-Flash QA" Q4.9):
+ *                the router scores xn = x / sqrt(mean(x^2) + norm_eps) * g
+ *                (the experts still take x); norm_eps > 0 (1e-6 is the
+ *                RMSNorm epsilon the pages give);
+ *   score_fn     MOE_SCORE_SIGMOID or MOE_SCORE_SQRT_SOFTPLUS: the score s
+ *                that is ranked (plus score_bias, if given) and renormalised,
+ *                w_j = scale * s_j / sum_{i in top-k} s_i; any other value is
+ *                MOE_ERR_INVALID_ARG. */
+typedef struct moe_route_options {
+    const float* score_bias;
+    const float* norm_weight;
+    float norm_eps;
+    int32_t score_fn;
+} moe_route_options;
+
+/* moe_route with the options above (opt NULL: moe_route). With a norm weight
+ * the routing runs on the CUDA-core router at every batch size. */
+MOE_API int moe_route3(const moe_config* cfg, const void* x, const void* w_gate,
+               const float* gate_bias, const moe_route_options* opt, int32_t* topk_idx,
+               float* topk_w, void* ws, size_t ws_bytes, void* stream);
+
 /* Group token-slots by expert (the grouping defined above): writes counts [E],
  * offsets [E+1], row_of [T*k] (int32) and x_perm [T*k, d] bf16 with
  * x_perm[row_of[t*k+j]] = x[t]. Pages: the per-expert loop with index_add_ of
@@ -161,7 +205,7 @@ MOE_API int moe_permute_index(const moe_config* cfg, const int32_t* topk_idx, in
  * h is [T*k, d_ff] bf16. Pages: "DeepSeek V4-Flash 架构 QA" Q4.5 (SwiGLU);
  * "Tencent Hy3-295B 架构深度拆解" §2.3 (fused gate_up_proj 2*1536 x 4096). */
 MOE_API int moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
-                       const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
+                       const void* w_gate_up, const void* s_gate_up, void* h, void* ws,
                        size_t ws_bytes, void* stream);
 
 /* moe_expert_gate_up with the grouped rows read from x by index: the row r
@@ -172,20 +216,20 @@ MOE_API int moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const 
  * first copy them into the workspace. */
 MOE_API int moe_expert_gate_up_gather(const moe_config* cfg, const void* x,
                               const int32_t* token_of_row, const int32_t* offsets,
-                              const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
+                              const void* w_gate_up, const void* s_gate_up, void* h, void* ws,
                               size_t ws_bytes, void* stream);
 
 /* down step: y[r, i] = bf16( <h[r], w_down[e, i]> ), fp32 accumulate; y is
  * [T*k, d] bf16. Pages: "Tencent Hy3-295B 架构深度拆解" §2.3 (down_proj
  * 4096 x 1536). */
 MOE_API int moe_expert_down(const moe_config* cfg, const void* h, const int32_t* offsets,
-                    const void* w_down, const float* s_down, void* y, void* ws, size_t ws_bytes,
+                    const void* w_down, const void* s_down, void* y, void* ws, size_t ws_bytes,
                     void* stream);
 
 /* Both expert steps (h lives in ws): y [T*k, d] bf16 from x_perm. */
 MOE_API int moe_experts(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
-                const void* w_gate_up, const float* s_gate_up, const void* w_down,
-                const float* s_down, void* y, void* ws, size_t ws_bytes, void* stream);
+                const void* w_gate_up, const void* s_gate_up, const void* w_down,
+                const void* s_down, void* y, void* ws, size_t ws_bytes, void* stream);
 
 /* fp32 combine and unpermute: out[t, :] = bf16_rne( sum_{j<k} topk_w[t, j] *
  * float(y[row_of[t*k + j], :]) ), summed in fp32 in j order, one final cast.
@@ -205,8 +249,8 @@ MOE_API int moe_combine(const moe_config* cfg, const void* y, const int32_t* row
  * gate_up as MOE_GATHER_MAX_SLOTS says). out [T, d] bf16. The intermediates
  * live in ws. Resets the workspace status word first. */
 MOE_API int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
-                const void* w_gate_up, const float* s_gate_up, const void* w_down,
-                const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream);
+                const void* w_gate_up, const void* s_gate_up, const void* w_down,
+                const void* s_down, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Rearrange one bf16 expert weight (which = MOE_WEIGHTS_GATE_UP or
  * MOE_WEIGHTS_DOWN, row-major as above) into the packed layout described
@@ -225,8 +269,21 @@ MOE_API int moe_pack_weights(const moe_config* cfg, int which, const void* w, vo
  * complete Hy3 MoE block. */
 MOE_API int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate,
                  const float* gate_bias, const float* score_bias, const void* w_gate_up,
-                 const float* s_gate_up, const void* w_down, const float* s_down, void* out,
+                 const void* s_gate_up, const void* w_down, const void* s_down, void* out,
                  void* ws, size_t ws_bytes, void* stream);
+
+/* moe_forward with the router options of moe_route3 (opt NULL: moe_forward). */
+MOE_API int moe_forward3(const moe_config* cfg, const void* x, const void* w_gate,
+                 const float* gate_bias, const moe_route_options* opt, const void* w_gate_up,
+                 const void* s_gate_up, const void* w_down, const void* s_down, void* out,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* Failure-detection self-test: one thread waits, with the library's bounded
+ * wait and a limit of limit_ns (1 ns .. 10 s), on an mbarrier that nothing
+ * completes, then records MOE_ERR_TIMEOUT in the status word of ws (read it
+ * with moe_read_status). Faults, traps and hangs nothing; the context stays
+ * usable. Not part of the layer (the pages have no counterpart). */
+MOE_API int moe_selftest_bounded_wait(void* ws, unsigned long long limit_ns, void* stream);
 
 /* Bytes of the fixed device array behind moe_route_noalloc. */
 #define MOE_NOALLOC_SCRATCH_BYTES (2u << 20)

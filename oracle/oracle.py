@@ -299,6 +299,8 @@ class OracleLayer:
             self.wd = np.ascontiguousarray(layer["q_down"].cpu().numpy())
             self.s_gu = np.ascontiguousarray(layer["s_gate_up"].cpu().numpy(), dtype=np.float32)
             self.s_d = np.ascontiguousarray(layer["s_down"].cpu().numpy(), dtype=np.float32)
+        elif self.fp4:  # the FP4 codes above are the experts' weights
+            self.wgu = self.wd = self.s_gu = self.s_d = None
         else:
             self.wgu = bf16_bits(layer["w_gate_up"])
             self.wd = bf16_bits(layer["w_down"])

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
 #include <string.h>
@@ -60,6 +61,31 @@ __device__ __forceinline__ void e4m3x16_to_float(const uint4& v, float f[16]) {
     }
 }
 
+// Sixteen E2M1 codes in two 32-bit words (two per byte, the even element in
+// the low nibble, words and bytes in increasing element order) -> sixteen
+// floats, exactly: the hardware e2m1x2 -> f16x2 conversion takes the low
+// nibble to the low half, and every E2M1 value is an f16 value.
+__device__ __forceinline__ void e2m1x16_to_float(uint32_t w0, uint32_t w1, float f[16]) {
+    const uint32_t w[2] = {w0, w1};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(
+                (__nv_fp4x2_storage_t)((w[i] >> (8 * j)) & 0xFFu), __NV_E2M1);
+            const float2 p = __half22float2(*reinterpret_cast<__half2*>(&h));
+            f[8 * i + 2 * j] = p.x;
+            f[8 * i + 2 * j + 1] = p.y;
+        }
+    }
+}
+
+// E8M0 scale byte b -> 2^(b - 127) (b = 0 gives the subnormal 2^-127; b = 255,
+// not a scale, gives infinity).
+__device__ __forceinline__ float e8m0_to_float(uint32_t b) {
+    return b ? __uint_as_float(b << 23) : __uint_as_float(0x00400000u);
+}
+
 // Round a float to bf16 (nearest-even) and return the 16-bit pattern.
 __host__ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
     __nv_bfloat16 b = __float2bfloat16_rn(f);
@@ -89,14 +115,26 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __device__ __forceinline__ float sigmoidf_acc(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// Router score functions (both increasing in the logit): 0 the sigmoid (Hy3),
+// 1 sqrt(softplus(z)) = sqrt(log(1 + e^z)) (the V4-Flash column of
+// "Tencent Hy3-295B 架构深度拆解" §2.2), evaluated as
+// sqrt(max(z, 0) + log1p(e^-|z|)), which neither overflows nor loses the
+// small softplus of a very negative logit.
+__device__ __forceinline__ float sqrt_softplusf(float z) {
+    return sqrtf(fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))));
+}
+__device__ __forceinline__ float score_value(float z, int score_fn) {
+    return score_fn ? sqrt_softplusf(z) : sigmoidf_acc(z);
+}
+
 // Warp-collective top-k of one token's router scores. sc[q] holds the biased
 // logit of expert lane + 32 q (-INFINITY where that expert does not exist, so
 // E <= 256). k <= 32 rounds; each takes the warp maximum with one redux.sync
 // on an order-preserving unsigned key of the value and, among the lanes that
 // hold it, the lowest expert index with a second one (ties to the lower
-// index). The sigmoid is increasing, so these are the k largest scores. Lane
-// j < k writes the j-th selection: idx_row[j] and
-// w_row[j] = scale * sigmoid_j / sum of the k sigmoids (summed in j order).
+// index). The score function (score_value) is increasing, so these are the k
+// largest scores. Lane j < k writes the j-th selection: idx_row[j] and
+// w_row[j] = scale * score_j / sum of the k scores (summed in j order).
 __host__ __device__ __forceinline__ uint32_t order_key(float f) {
     const uint32_t b = f32_bits(f + 0.0f);  // -0 -> +0
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
@@ -106,13 +144,14 @@ __host__ __device__ __forceinline__ float key_value(uint32_t key) {
 }
 
 //
-// With prob (the lane's 8 sigmoid scores; sc then holds the choice values
+// With prob (the lane's 8 scores; sc then holds the choice values
 // score + e_score_correction_bias), the weights renormalise prob of the chosen
-// experts instead of the sigmoid of the ranked values.
+// experts instead of the scores of the ranked values.
 __device__ __forceinline__ void warp_select_topk(float (&sc)[8], int k, float scale,
                                                  int* __restrict__ idx_row,
                                                  float* __restrict__ w_row,
-                                                 const float* prob = nullptr) {
+                                                 const float* prob = nullptr,
+                                                 int score_fn = 0) {
     const int lane = threadIdx.x & 31;
     uint32_t key[8];
 #pragma unroll
@@ -135,7 +174,7 @@ __device__ __forceinline__ void warp_select_topk(float (&sc)[8], int k, float sc
                 if ((int)(be >> 5) == q) pv = prob[q];
             pv = __shfl_sync(0xffffffffu, pv, (int)(be & 31u));
         }
-        if (lane == r) { my_e = (int)be; my_s = prob ? pv : sigmoidf_acc(key_value(m)); }
+        if (lane == r) { my_e = (int)be; my_s = prob ? pv : score_value(key_value(m), score_fn); }
         if ((int)(be & 31u) == lane) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)

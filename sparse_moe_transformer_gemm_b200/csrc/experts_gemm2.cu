@@ -481,9 +481,11 @@ struct Fp8Ctrl {
     int tile_start[MAX_E + 1];
 };
 
+constexpr int FP8_EPI_BYTES = EPI_N * BM * 2;  // one [32 tokens][128 rows] bf16 staging tile
+
 template <bool GATE_UP>
 constexpr int fp8_smem_bytes() {
-    return Fp8Shape<GATE_UP>::RING_BYTES + 1024 + (int)sizeof(Fp8Ctrl);
+    return Fp8Shape<GATE_UP>::RING_BYTES + FP8_EPI_BYTES + 1024 + (int)sizeof(Fp8Ctrl);
 }
 static_assert(fp8_smem_bytes<true>() <= 232448 && fp8_smem_bytes<false>() <= 232448,
               "fits in 227 KB");
@@ -552,7 +554,8 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     uint8_t* op_ring = smem;  // 1024-aligned operand stages first
     uint8_t* b_ring = op_ring + S::OP_STAGES * S::OP_STAGE;
     uint8_t* raw_ring = b_ring + S::B_STAGES * BH_BYTES;
-    Fp8Ctrl& c = *reinterpret_cast<Fp8Ctrl*>(smem + S::RING_BYTES);
+    uint16_t* epi = reinterpret_cast<uint16_t*>(smem + S::RING_BYTES);
+    Fp8Ctrl& c = *reinterpret_cast<Fp8Ctrl*>(smem + S::RING_BYTES + FP8_EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)(tc::cluster_ctarank() & 1u);
     const bool leader = rank == 0;
@@ -787,7 +790,11 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     } else if (warp >= 2 && warp <= 5) {
         // ---------------- epilogue (scales applied to the finished dot products)
         const int quad = warp & 3;
+        // Per 32-token chunk the four warps write bf16 into the shared [32 tokens]
+        // [128 rows] tile and, after a named barrier, store it as 256-byte row
+        // segments with 16-byte vectors (as the bf16 kernel's epilogue does).
         const int row_in_tile = quad * 32 + lane;
+        const int et = threadIdx.x - 64;  // 0..127
         uint16_t* o16 = reinterpret_cast<uint16_t*>(out);
         const bool arriver = (warp == 2 && lane == 0);
         int it = 0;
@@ -795,14 +802,18 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             const TileInfo ti = decode_tile(c, E, m_tiles, t);
             const int acc = it % S::ACC_STAGES;
             const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
-            const bool ok = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
+            const bool waited = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
+            if (tc::bar_any(1, 128, !waited)) {  // the four warps leave together
+                raise_timeout(c, status);
+                break;
+            }
             tc::fence_after_sync();
             const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
-            const int col = ti.m * 2 * BM + rank * BM + row_in_tile;
-            const long srow = (long)ti.e * a_rows_per_expert + col;
+            const int col0 = ti.m * 2 * BM + rank * BM;
+            const long srow = (long)ti.e * a_rows_per_expert + col0 + row_in_tile;
             const float sa = __ldg(scales + srow);
             const float sb = GATE_UP ? __ldg(scales + srow + a_rows_per_expert / 2) : 0.f;
-            for (int c0 = 0; ok && c0 < ti.n; c0 += 32) {
+            for (int c0 = 0; c0 < ti.n; c0 += EPI_N) {
                 uint32_t g[32];
                 tc::tmem_ld32(tbase + c0, g);
                 if constexpr (GATE_UP) {
@@ -811,30 +822,31 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int n = c0 + j;
-                        if (n < ti.len) {
-                            const float gv = __uint_as_float(g[j]) * sa;
-                            const float uv = __uint_as_float(u[j]) * sb;
-                            const float hv = silu_mul(gv, uv);
-                            o16[(size_t)(ti.row0 + n) * out_ld + col] = float_to_bf16_bits(hv);
-                        }
+                        const float gv = __uint_as_float(g[j]) * sa;
+                        const float uv = __uint_as_float(u[j]) * sb;
+                        epi[j * BM + row_in_tile] = float_to_bf16_bits(silu_mul(gv, uv));
                     }
                 } else {
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = c0 + j;
-                        if (n < ti.len)
-                            o16[(size_t)(ti.row0 + n) * out_ld + col] =
-                                float_to_bf16_bits(__uint_as_float(g[j]) * sa);
-                    }
+                    for (int j = 0; j < 32; ++j)
+                        epi[j * BM + row_in_tile] = float_to_bf16_bits(__uint_as_float(g[j]) * sa);
                 }
+                tc::bar_sync(1, 128);  // the tile is written
+#pragma unroll
+                for (int q = 0; q < EPI_N * BM / 8 / 128; ++q) {
+                    const int id = et + 128 * q;
+                    const int n = id / (BM / 8), ch = id % (BM / 8);
+                    if (c0 + n < ti.len)
+                        *reinterpret_cast<uint4*>(o16 + (size_t)(ti.row0 + c0 + n) * out_ld + col0 +
+                                                  ch * 8) =
+                            *reinterpret_cast<const uint4*>(epi + n * BM + ch * 8);
+                }
+                tc::bar_sync(1, 128);  // the tile is read
             }
+            // every warp's TMEM reads are complete before the accumulator is handed back
             tc::fence_before_sync();
-            if (tc::bar_any(1, 128, !ok)) {
-                raise_timeout(c, status);
-                break;
-            }
+            tc::bar_sync(1, 128);
             if (arriver)
                 tc::mbar_arrive_cluster(tc::map_to_cta(tc::smem_u32(&c.acc_empty[acc]), 0));
         }

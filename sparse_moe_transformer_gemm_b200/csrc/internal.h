@@ -24,6 +24,7 @@ struct WsLayout {
     size_t counters;  // int32 [ceil(T / kRouterTokens)] router arrival counters
     size_t control_end;
     size_t logits;    // fp32 [router_ksplit, T, E] partial router logits
+    size_t sumsq;     // fp32 [router_ksplit, T] route_norm partial sums of squares
     size_t hist;      // int32 [n_chunks, E]
     size_t rank;      // int32 [T*k]
     size_t idx;       // int32 [T*k]
@@ -83,6 +84,7 @@ inline WsLayout ws_layout(const moe_config& c) {
     L.counters = o; o = align256(o + sizeof(int32_t) * n_router_groups(c));
     L.control_end = o;
     L.logits = o;   o = align256(o + sizeof(float) * router_ksplit(c) * (size_t)c.T * c.E);
+    L.sumsq = o;    o = align256(o + sizeof(float) * router_ksplit(c) * (size_t)c.T);
     L.hist = o;     o = align256(o + sizeof(int32_t) * (size_t)n_permute_chunks(g) * g.E);
     L.rank = o;     o = align256(o + sizeof(int32_t) * R);
     L.idx = o;      o = align256(o + sizeof(int32_t) * R);
@@ -101,13 +103,14 @@ inline WsLayout ws_layout(const moe_config& c) {
 
 // ---- launchers (each returns cudaError_t of the launch) ----
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
-                          const float* gate_bias, const float* score_bias, int32_t* idx, float* w,
-                          float* logits, int32_t* counters, int ksplit, cudaStream_t s);
+                          const float* gate_bias, const float* score_bias, const float* norm_w,
+                          float norm_eps, int score_fn, int32_t* idx, float* w, float* logits,
+                          float* sumsq, int32_t* counters, int ksplit, cudaStream_t s);
 
 bool router_tc_supported(const moe_config& c);
 cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_gate,
-                             const float* gate_bias, const float* score_bias, int32_t* idx,
-                             float* w, int* status, cudaStream_t s);
+                             const float* gate_bias, const float* score_bias, int score_fn,
+                             int32_t* idx, float* w, int* status, cudaStream_t s);
 
 cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
                            int32_t* offsets, int32_t* row_of, void* x_perm, int32_t* hist,
@@ -120,10 +123,10 @@ cudaError_t launch_gather_rows(const moe_config& c, const void* x, const int32_t
                                const int32_t* offsets, void* x_perm, cudaStream_t s);
 
 cudaError_t launch_gate_up_stream(const moe_config& c, const void* x_perm, const int32_t* offsets,
-                                  const void* w_gate_up, const float* s_gate_up, void* h,
+                                  const void* w_gate_up, const void* s_gate_up, void* h,
                                   cudaStream_t s);
 cudaError_t launch_down_stream(const moe_config& c, const void* h, const int32_t* offsets,
-                               const void* w_down, const float* s_down, void* y, cudaStream_t s);
+                               const void* w_down, const void* s_down, void* y, cudaStream_t s);
 
 cudaError_t launch_gate_up_gemm(const moe_config& c, const void* x_perm, const int32_t* offsets,
                                 const void* w_gate_up, void* h, int* status, cudaStream_t s);

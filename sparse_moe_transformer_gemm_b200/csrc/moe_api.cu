@@ -9,7 +9,8 @@ using namespace moe;
 namespace {
 
 constexpr uint32_t kKnownFlags = MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH | MOE_FLAG_GEMM_PATH |
-                                 MOE_FLAG_PACKED_WEIGHTS | MOE_FLAG_SHARED_EXPERT;
+                                 MOE_FLAG_PACKED_WEIGHTS | MOE_FLAG_SHARED_EXPERT |
+                                 MOE_FLAG_FP4_WEIGHTS;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -20,6 +21,11 @@ int check_cfg(const moe_config* c) {
         return MOE_ERR_INVALID_ARG;
     if ((c->flags & MOE_FLAG_PACKED_WEIGHTS) &&
         (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH)))
+        return MOE_ERR_INVALID_ARG;
+    // FP4 experts: the weight-streaming kernels only, routed experts only
+    if ((c->flags & MOE_FLAG_FP4_WEIGHTS) &&
+        (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_PACKED_WEIGHTS | MOE_FLAG_GEMM_PATH |
+                     MOE_FLAG_SHARED_EXPERT)))
         return MOE_ERR_INVALID_ARG;
     if (!isfinite(c->scale)) return MOE_ERR_INVALID_ARG;
     if (c->T < 1 || c->E < 1 || c->E > 256 - shared_slots(*c) || c->k < 1 || c->k > c->E ||
@@ -37,10 +43,11 @@ int check_cfg(const moe_config* c) {
 
 bool packed(const moe_config* c) { return (c->flags & MOE_FLAG_PACKED_WEIGHTS) != 0; }
 
-// Expert weights: bf16 without the FP8 flag (no scales), e4m3 + scales with it.
-int check_expert_weights(const moe_config* c, const void* w, const float* s) {
+// Expert weights: bf16 without a quantised format (no scales); e4m3 codes +
+// fp32 row scales, or E2M1 codes + E8M0 block scales, with one.
+int check_expert_weights(const moe_config* c, const void* w, const void* s) {
     if (!w || !aligned16(w)) return MOE_ERR_INVALID_ARG;
-    if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
+    if (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_FP4_WEIGHTS)) {
         if (!s) return MOE_ERR_INVALID_ARG;
     } else if (s) {
         return MOE_ERR_INVALID_ARG;
@@ -71,9 +78,10 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA
 // the register-staged streaming kernels at every batch size measured on B200
 // (decode T=64: 1.07 ms vs 1.45 ms per layer), so they are the default. FP8
 // weights have a tensor-core path on SM pairs only (d, d_ff multiples of 256);
-// other FP8 shapes use the streaming kernels.
+// other FP8 shapes use the streaming kernels. FP4 weights have no tensor-core
+// path yet: always the streaming kernels.
 bool use_stream_path(const moe_config* c) {
-    if (c->flags & MOE_FLAG_STREAM_PATH) return true;
+    if (c->flags & (MOE_FLAG_STREAM_PATH | MOE_FLAG_FP4_WEIGHTS)) return true;
     if (c->flags & MOE_FLAG_GEMM_PATH) return false;
     return (c->flags & MOE_FLAG_FP8_WEIGHTS) != 0 && !pair_gemm_supported(*c);
 }
@@ -84,18 +92,34 @@ bool use_stream_path(const moe_config* c) {
 // of CTAs.
 constexpr int kRouterTcMinTokens = 129;
 
+// route_norm needs the per-token sum of squares next to the logits: the
+// CUDA-core router computes both exactly in fp32 (the tensor-core router's bf16
+// operands cannot carry x * g unrounded), so it serves every batch size then.
 cudaError_t route(const moe_config* c, const void* x, const void* w_gate, const float* gate_bias,
-                  const float* score_bias, int32_t* idx, float* w, void* ws, cudaStream_t s) {
+                  const moe_route_options* opt, int32_t* idx, float* w, void* ws,
+                  cudaStream_t s) {
+    const moe_route_options none = {nullptr, nullptr, 0.f, MOE_SCORE_SIGMOID};
+    const moe_route_options& o = opt ? *opt : none;
     const WsLayout L = ws_layout(*c);
-    if (router_tc_supported(*c) && c->T >= kRouterTcMinTokens)
-        return launch_router_tc(*c, x, w_gate, gate_bias, score_bias, idx, w,
+    if (!o.norm_weight && router_tc_supported(*c) && c->T >= kRouterTcMinTokens)
+        return launch_router_tc(*c, x, w_gate, gate_bias, o.score_bias, o.score_fn, idx, w,
                                 at<int>(ws, L.status), s);
-    return launch_router(*c, x, w_gate, gate_bias, score_bias, idx, w, at<float>(ws, L.logits),
+    return launch_router(*c, x, w_gate, gate_bias, o.score_bias, o.norm_weight, o.norm_eps,
+                         o.score_fn, idx, w, at<float>(ws, L.logits), at<float>(ws, L.sumsq),
                          at<int32_t>(ws, L.counters), router_ksplit(*c), s);
 }
 
+int check_route_options(const moe_route_options* opt) {
+    if (!opt) return MOE_OK;
+    if (opt->norm_weight && !(opt->norm_eps > 0.f && isfinite(opt->norm_eps)))
+        return MOE_ERR_INVALID_ARG;
+    if (opt->score_fn != MOE_SCORE_SIGMOID && opt->score_fn != MOE_SCORE_SQRT_SOFTPLUS)
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
 int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offsets,
-                    const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
+                    const void* w_gate_up, const void* s_gate_up, void* h, void* ws,
                     cudaStream_t s) {
     const moe_config g = grouped_config(*c);  // the shared expert is expert E
     if (use_stream_path(c))
@@ -103,8 +127,9 @@ int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offs
     int* status = at<int>(ws, ws_layout(*c).status);
     if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
         if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
-        return cuda_status(launch_gate_up_gemm_pair_fp8(g, x_perm, offsets, w_gate_up, s_gate_up,
-                                                        h, status, s));
+        return cuda_status(launch_gate_up_gemm_pair_fp8(g, x_perm, offsets, w_gate_up,
+                                                        static_cast<const float*>(s_gate_up), h,
+                                                        status, s));
     }
     if (pair_gemm_supported(*c))
         return cuda_status(
@@ -116,7 +141,7 @@ int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offs
 // rows of x itself (TMA tile::gather4); every other path first gathers them
 // into the workspace's x_perm region with a copy kernel.
 int experts_gate_up_gather(const moe_config* c, const void* x, const int32_t* token_of_row,
-                           const int32_t* offsets, const void* w_gate_up, const float* s_gate_up,
+                           const int32_t* offsets, const void* w_gate_up, const void* s_gate_up,
                            void* h, void* ws, cudaStream_t s) {
     const WsLayout L = ws_layout(*c);
     if (!use_stream_path(c) && !(c->flags & MOE_FLAG_FP8_WEIGHTS) && pair_gemm_supported(*c))
@@ -129,7 +154,7 @@ int experts_gate_up_gather(const moe_config* c, const void* x, const int32_t* to
 }
 
 int experts_down(const moe_config* c, const void* h, const int32_t* offsets, const void* w_down,
-                 const float* s_down, void* y, void* ws, cudaStream_t s) {
+                 const void* s_down, void* y, void* ws, cudaStream_t s) {
     const moe_config g = grouped_config(*c);
     if (use_stream_path(c))
         return cuda_status(launch_down_stream(g, h, offsets, w_down, s_down, y, s));
@@ -137,7 +162,8 @@ int experts_down(const moe_config* c, const void* h, const int32_t* offsets, con
     if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
         if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
         return cuda_status(
-            launch_down_gemm_pair_fp8(g, h, offsets, w_down, s_down, y, status, s));
+            launch_down_gemm_pair_fp8(g, h, offsets, w_down, static_cast<const float*>(s_down),
+                                      y, status, s));
     }
     if (pair_gemm_supported(*c))
         return cuda_status(launch_down_gemm_pair(g, h, offsets, w_down, packed(c), y, status, s));
@@ -165,15 +191,23 @@ int moe_workspace_init(const moe_config* cfg, void* ws, size_t ws_bytes, void* s
                                        static_cast<cudaStream_t>(stream)));
 }
 
-int moe_route2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
-               const float* score_bias, int32_t* topk_idx, float* topk_w, void* ws,
+int moe_route3(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+               const moe_route_options* opt, int32_t* topk_idx, float* topk_w, void* ws,
                size_t ws_bytes, void* stream) {
     MOE_TRY(check_cfg(cfg));
     if (!x || !w_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_route_options(opt));
     MOE_TRY(check_ws(cfg, ws, ws_bytes));
-    return cuda_status(route(cfg, x, w_gate, gate_bias, score_bias, topk_idx, topk_w, ws,
+    return cuda_status(route(cfg, x, w_gate, gate_bias, opt, topk_idx, topk_w, ws,
                              static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+               const float* score_bias, int32_t* topk_idx, float* topk_w, void* ws,
+               size_t ws_bytes, void* stream) {
+    const moe_route_options opt = {score_bias, nullptr, 0.f, MOE_SCORE_SIGMOID};
+    return moe_route3(cfg, x, w_gate, gate_bias, &opt, topk_idx, topk_w, ws, ws_bytes, stream);
 }
 
 int moe_route(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
@@ -208,7 +242,7 @@ int moe_permute_index(const moe_config* cfg, const int32_t* topk_idx, int32_t* c
 
 int moe_expert_gate_up_gather(const moe_config* cfg, const void* x, const int32_t* token_of_row,
                               const int32_t* offsets, const void* w_gate_up,
-                              const float* s_gate_up, void* h, void* ws, size_t ws_bytes,
+                              const void* s_gate_up, void* h, void* ws, size_t ws_bytes,
                               void* stream) {
     MOE_TRY(check_cfg(cfg));
     if (!x || !token_of_row || !offsets || !h || !aligned16(x) || !aligned16(h))
@@ -220,7 +254,7 @@ int moe_expert_gate_up_gather(const moe_config* cfg, const void* x, const int32_
 }
 
 int moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
-                       const void* w_gate_up, const float* s_gate_up, void* h, void* ws,
+                       const void* w_gate_up, const void* s_gate_up, void* h, void* ws,
                        size_t ws_bytes, void* stream) {
     MOE_TRY(check_cfg(cfg));
     if (!x_perm || !offsets || !h || !aligned16(x_perm) || !aligned16(h))
@@ -232,7 +266,7 @@ int moe_expert_gate_up(const moe_config* cfg, const void* x_perm, const int32_t*
 }
 
 int moe_expert_down(const moe_config* cfg, const void* h, const int32_t* offsets,
-                    const void* w_down, const float* s_down, void* y, void* ws, size_t ws_bytes,
+                    const void* w_down, const void* s_down, void* y, void* ws, size_t ws_bytes,
                     void* stream) {
     MOE_TRY(check_cfg(cfg));
     if (!h || !offsets || !y || !aligned16(h) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
@@ -242,8 +276,8 @@ int moe_expert_down(const moe_config* cfg, const void* h, const int32_t* offsets
 }
 
 int moe_experts(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
-                const void* w_gate_up, const float* s_gate_up, const void* w_down,
-                const float* s_down, void* y, void* ws, size_t ws_bytes, void* stream) {
+                const void* w_gate_up, const void* s_gate_up, const void* w_down,
+                const void* s_down, void* y, void* ws, size_t ws_bytes, void* stream) {
     MOE_TRY(check_cfg(cfg));
     if (!x_perm || !offsets || !y || !aligned16(x_perm) || !aligned16(y))
         return MOE_ERR_INVALID_ARG;
@@ -267,11 +301,12 @@ int moe_combine(const moe_config* cfg, const void* y, const int32_t* row_of, con
                                       static_cast<cudaStream_t>(stream)));
 }
 
-int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
-                 const float* score_bias, const void* w_gate_up, const float* s_gate_up,
-                 const void* w_down, const float* s_down, void* out, void* ws, size_t ws_bytes,
+int moe_forward3(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+                 const moe_route_options* opt, const void* w_gate_up, const void* s_gate_up,
+                 const void* w_down, const void* s_down, void* out, void* ws, size_t ws_bytes,
                  void* stream) {
     MOE_TRY(check_cfg(cfg));
+    MOE_TRY(check_route_options(opt));
     if (!x || !w_gate || !out || !aligned16(x) || !aligned16(w_gate) || !aligned16(out))
         return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_expert_weights(cfg, w_gate_up, s_gate_up));
@@ -289,7 +324,7 @@ int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const
     void* h = at<void>(ws, L.h);
     void* y = at<void>(ws, L.y);
     MOE_TRY(cuda_status(cudaMemsetAsync(ws, 0, L.control_end, s)));
-    MOE_TRY(cuda_status(route(cfg, x, w_gate, gate_bias, score_bias, idx, w, ws, s)));
+    MOE_TRY(cuda_status(route(cfg, x, w_gate, gate_bias, opt, idx, w, ws, s)));
     if (gather_batch(cfg)) {
         int32_t* tok = at<int32_t>(ws, L.tok);
         MOE_TRY(cuda_status(
@@ -305,10 +340,19 @@ int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const
     return cuda_status(launch_combine(*cfg, y, row_of, w, out, s));
 }
 
+int moe_forward2(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
+                 const float* score_bias, const void* w_gate_up, const void* s_gate_up,
+                 const void* w_down, const void* s_down, void* out, void* ws, size_t ws_bytes,
+                 void* stream) {
+    const moe_route_options opt = {score_bias, nullptr, 0.f, MOE_SCORE_SIGMOID};
+    return moe_forward3(cfg, x, w_gate, gate_bias, &opt, w_gate_up, s_gate_up, w_down, s_down,
+                        out, ws, ws_bytes, stream);
+}
+
 int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const float* gate_bias,
-                const void* w_gate_up, const float* s_gate_up, const void* w_down,
-                const float* s_down, void* out, void* ws, size_t ws_bytes, void* stream) {
-    return moe_forward2(cfg, x, w_gate, gate_bias, nullptr, w_gate_up, s_gate_up, w_down, s_down,
+                const void* w_gate_up, const void* s_gate_up, const void* w_down,
+                const void* s_down, void* out, void* ws, size_t ws_bytes, void* stream) {
+    return moe_forward3(cfg, x, w_gate, gate_bias, nullptr, w_gate_up, s_gate_up, w_down, s_down,
                         out, ws, ws_bytes, stream);
 }
 

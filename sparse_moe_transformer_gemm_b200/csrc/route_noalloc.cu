@@ -72,8 +72,8 @@ extern "C" int moe_route_noalloc(const moe_config* cfg, const void* x, const voi
     int32_t* counters = static_cast<int32_t*>(base);
     float* logits = reinterpret_cast<float*>(static_cast<char*>(base) + counter_bytes);
     if (cudaMemsetAsync(counters, 0, counter_bytes, s) != cudaSuccess) return MOE_ERR_CUDA;
-    return moe::launch_router(*cfg, x, w_gate, gate_bias, nullptr, topk_idx, topk_w, logits,
-                              counters, 1, s) ==
+    return moe::launch_router(*cfg, x, w_gate, gate_bias, nullptr, nullptr, 0.f, 0, topk_idx,
+                              topk_w, logits, nullptr, counters, 1, s) ==
                    cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;

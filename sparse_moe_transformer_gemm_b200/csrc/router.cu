@@ -20,6 +20,8 @@
 // this selects the k largest scores -- and the sigmoid of the k selected. With
 // an e_score_correction_bias ("Tencent Hy3-295B 架构深度拆解" §4.1 step 2) the
 // choice ranks sigmoid + bias and the weights renormalise the sigmoid scores.
+// With score_fn 1 every "sigmoid" above reads sqrt(softplus(logit)) (the
+// V4-Flash router of the same page, §2.2), also increasing in the logit.
 #include "common.cuh"
 #include "internal.h"
 
@@ -43,10 +45,10 @@ __device__ __forceinline__ void load_w(uint4 (&u)[EPW], const __nv_bfloat16* __r
 
 __global__ void __launch_bounds__(RWARPS * 32, kRouterCtasPerSm)
 router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wg,
-              const float* __restrict__ bias, const float* __restrict__ sbias, int T, int d,
-              int E, int k, float scale,
-              float* __restrict__ logits, int* __restrict__ counters, int* __restrict__ idx_out,
-              float* __restrict__ w_out) {
+              const float* __restrict__ bias, const float* __restrict__ sbias,
+              const float* __restrict__ norm_w, float norm_eps, int score_fn, int T, int d,
+              int E, int k, float scale, float* __restrict__ logits, float* __restrict__ sumsq,
+              int* __restrict__ counters, int* __restrict__ idx_out, float* __restrict__ w_out) {
     __shared__ __align__(16) float xs[RT][KC];
     __shared__ int s_last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -61,6 +63,7 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
     for (int a = 0; a < EPW; ++a)
 #pragma unroll
         for (int b = 0; b < RT; ++b) acc[a][b] = 0.f;
+    float ss_tok = 0.f;  // route_norm: sum of squares of token t0 + warp over this slice
 
     for (int kc = k0; kc < k0 + dk; kc += KC) {
         const int kw = min(KC, k0 + dk - kc);  // multiple of 128
@@ -80,6 +83,20 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
             *reinterpret_cast<float4*>(&xs[tt][c8 + 4]) = make_float4(f[4], f[5], f[6], f[7]);
         }
         __syncthreads();
+        if (norm_w) {
+            // route_norm: warp w sums the squares of token w's chunk (fixed order),
+            // then the chunk is multiplied by the norm weight; 1/rms is applied to
+            // the finished logit (logit = (1/rms) sum_c x_c g_c W_ec)
+            float ss = 0.f;
+            for (int c = lane; c < kw; c += 32) ss = fmaf(xs[warp][c], xs[warp][c], ss);
+            ss_tok += warp_sum(ss);
+            __syncthreads();
+            for (int v = threadIdx.x; v < RT * kw; v += blockDim.x) {
+                const int tt = v / kw, c = v - tt * kw;
+                xs[tt][c] *= norm_w[kc + c];
+            }
+            __syncthreads();
+        }
         // the weight vectors of the next column step are in flight while the
         // current ones are used
         uint4 cur[EPW];
@@ -123,6 +140,9 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
             }
     }
 
+    if (norm_w && blockIdx.x == 0 && lane == 0 && t0 + warp < T)
+        sumsq[(size_t)blockIdx.z * T + t0 + warp] = ss_tok;
+
     // Arrival: the last expert-block CTA of this token group does the selection.
     __threadfence();
     __syncthreads();
@@ -152,6 +172,13 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
                 }
             }
         }
+        if (norm_w) {
+            float ms = 0.f;
+            for (int p = 0; p < ks; ++p) ms += __ldcg(sumsq + (size_t)p * T + t);
+            const float inv = 1.0f / sqrtf(ms / (float)d + norm_eps);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) sc[q] *= inv;
+        }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const int e = lane + 32 * q;
@@ -168,12 +195,14 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const int e = lane + 32 * q;
-                prob[q] = (e < E) ? sigmoidf_acc(sc[q]) : 0.f;
+                prob[q] = (e < E) ? score_value(sc[q], score_fn) : 0.f;
                 sc[q] = (e < E) ? prob[q] + sbias[e] : -INFINITY;
             }
-            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k, prob);
+            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k, prob,
+                             score_fn);
         } else {
-            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k);
+            warp_select_topk(sc, k, scale, idx_out + (size_t)t * k, w_out + (size_t)t * k,
+                             nullptr, score_fn);
         }
     }
     if (threadIdx.x == 0) counters[blockIdx.y] = 0;
@@ -182,12 +211,14 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
 }  // namespace
 
 cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate,
-                          const float* gate_bias, const float* score_bias, int32_t* idx, float* w,
-                          float* logits, int32_t* counters, int ksplit, cudaStream_t s) {
+                          const float* gate_bias, const float* score_bias, const float* norm_w,
+                          float norm_eps, int score_fn, int32_t* idx, float* w, float* logits,
+                          float* sumsq, int32_t* counters, int ksplit, cudaStream_t s) {
     dim3 grid((c.E + RE - 1) / RE, n_router_groups(c), ksplit);
     router_kernel<<<grid, RWARPS * 32, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_gate), gate_bias,
-        score_bias, c.T, c.d, c.E, c.k, c.scale, logits, counters, idx, w);
+        score_bias, norm_w, norm_eps, score_fn, c.T, c.d, c.E, c.k, c.scale, logits, sumsq, counters, idx,
+        w);
     return cudaGetLastError();
 }
 

@@ -15,7 +15,9 @@
 // flight per thread), in split order (the result does not depend on timing),
 // and selects for those rows, one thread per row, ties to the lower expert
 // index. The sigmoid is increasing, so the k largest (biased) logits are the k
-// largest scores; it is evaluated for the k selected only.
+// largest scores; it is evaluated for the k selected only. With score_fn 1
+// the score is sqrt(softplus(logit)) (the V4-Flash router, same page §2.2),
+// also increasing.
 //
 // CTA: 192 threads -- warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 2-5 epilogue / reduction / selection. Waits are bounded
@@ -74,7 +76,7 @@ static_assert(BM * logit_stride(256) * 4 + 32 <= STAGES * STAGE_BYTES, "logit ro
 template <int K, bool SB>
 __device__ __forceinline__ void thread_select_topk(const float* row, const float* sbias,
                                                    const float* cbias, int E, float scale,
-                                                   int* __restrict__ idx_out,
+                                                   int score_fn, int* __restrict__ idx_out,
                                                    float* __restrict__ w_out) {
     // SB: rank sigmoid(logit) + cbias (the e_score_correction_bias) and keep
     // the sigmoid scores p of the list for the weights
@@ -95,7 +97,7 @@ __device__ __forceinline__ void thread_select_topk(const float* row, const float
             const int e = e0 + u;
             float z = z8[u], pz = 0.f;
             if (SB && e < E) {
-                pz = sigmoidf_acc(z);
+                pz = score_value(z, score_fn);
                 z = pz + cbias[e];
             }
             if (e < E && z > v[K - 1]) {
@@ -116,13 +118,29 @@ __device__ __forceinline__ void thread_select_topk(const float* row, const float
     float sum = 0.f;
 #pragma unroll
     for (int j = 0; j < K; ++j) {
-        v[j] = SB ? p[j] : sigmoidf_acc(v[j]);
+        v[j] = SB ? p[j] : score_value(v[j], score_fn);
         sum += v[j];
     }
 #pragma unroll
     for (int j = 0; j < K; ++j) {
         idx_out[j] = id[j];
         w_out[j] = scale * v[j] / sum;
+    }
+}
+
+template <bool SB>
+__device__ __forceinline__ void select_k(int k, const float* row, const float* sbias,
+                                         const float* cbias, int E, float scale, int score_fn,
+                                         int* __restrict__ idx_out, float* __restrict__ w_out) {
+    switch (k) {
+        case 1: thread_select_topk<1, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
+        case 2: thread_select_topk<2, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
+        case 3: thread_select_topk<3, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
+        case 4: thread_select_topk<4, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
+        case 5: thread_select_topk<5, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
+        case 6: thread_select_topk<6, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
+        case 7: thread_select_topk<7, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
+        default: thread_select_topk<8, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
     }
 }
 
@@ -133,8 +151,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const float* __restrict__ bias, const float* __restrict__ sbias, int T,
                  int d, int E, int k, int n_pad,
-                 float scale, int* __restrict__ idx_out, float* __restrict__ w_out,
-                 int* __restrict__ status) {
+                 float scale, int score_fn, int* __restrict__ idx_out,
+                 float* __restrict__ w_out, int* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -311,29 +329,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const float* rw = red + (split * ROWS + rr) * es;
             int* io = idx_out + t * k;
             float* wo = w_out + t * k;
-            if (sbias) {
-                switch (k) {
-                    case 1: thread_select_topk<1, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 2: thread_select_topk<2, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 3: thread_select_topk<3, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 4: thread_select_topk<4, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 5: thread_select_topk<5, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 6: thread_select_topk<6, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 7: thread_select_topk<7, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    default: thread_select_topk<8, true>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                }
-            } else {
-                switch (k) {
-                    case 1: thread_select_topk<1, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 2: thread_select_topk<2, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 3: thread_select_topk<3, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 4: thread_select_topk<4, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 5: thread_select_topk<5, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 6: thread_select_topk<6, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    case 7: thread_select_topk<7, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                    default: thread_select_topk<8, false>(rw, c.bias, c.sbias, E, scale, io, wo); break;
-                }
-            }
+            if (sbias)
+                select_k<true>(k, rw, c.bias, c.sbias, E, scale, score_fn, io, wo);
+            else
+                select_k<false>(k, rw, c.bias, c.sbias, E, scale, score_fn, io, wo);
         }
     }
 
@@ -389,8 +388,8 @@ namespace {
 
 template <int S>
 cudaError_t launch_s(dim3 grid, const CUtensorMap& mx, const CUtensorMap& mw, const moe_config& c,
-                     int n_pad, const float* gate_bias, const float* score_bias, int32_t* idx,
-                     float* w, int* status, cudaStream_t s) {
+                     int n_pad, const float* gate_bias, const float* score_bias, int score_fn,
+                     int32_t* idx, float* w, int* status, cudaStream_t s) {
     cudaError_t err = cudaFuncSetAttribute(router_tc_kernel<S>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (err != cudaSuccess) return err;
@@ -407,14 +406,14 @@ cudaError_t launch_s(dim3 grid, const CUtensorMap& mx, const CUtensorMap& mw, co
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, router_tc_kernel<S>, mx, mw, gate_bias, score_bias, c.T, c.d,
-                              c.E, c.k, n_pad, c.scale, idx, w, status);
+                              c.E, c.k, n_pad, c.scale, score_fn, idx, w, status);
 }
 
 }  // namespace
 
 cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_gate,
-                             const float* gate_bias, const float* score_bias, int32_t* idx,
-                             float* w, int* status, cudaStream_t s) {
+                             const float* gate_bias, const float* score_bias, int score_fn,
+                             int32_t* idx, float* w, int* status, cudaStream_t s) {
     const int tiles = (c.T + BM - 1) / BM;
     const int S = router_splits(c.T, c.d);
     const int n_pad = (c.E + 15) & ~15;
@@ -424,10 +423,22 @@ cudaError_t launch_router_tc(const moe_config& c, const void* x, const void* w_g
     const dim3 grid(tiles, S);
     cudaError_t err;
     switch (S) {
-        case 1: err = launch_s<1>(grid, mx, mw, c, n_pad, gate_bias, score_bias, idx, w, status, s); break;
-        case 2: err = launch_s<2>(grid, mx, mw, c, n_pad, gate_bias, score_bias, idx, w, status, s); break;
-        case 4: err = launch_s<4>(grid, mx, mw, c, n_pad, gate_bias, score_bias, idx, w, status, s); break;
-        default: err = launch_s<8>(grid, mx, mw, c, n_pad, gate_bias, score_bias, idx, w, status, s); break;
+        case 1:
+            err = launch_s<1>(grid, mx, mw, c, n_pad, gate_bias, score_bias, score_fn, idx, w,
+                               status, s);
+            break;
+        case 2:
+            err = launch_s<2>(grid, mx, mw, c, n_pad, gate_bias, score_bias, score_fn, idx, w,
+                               status, s);
+            break;
+        case 4:
+            err = launch_s<4>(grid, mx, mw, c, n_pad, gate_bias, score_bias, score_fn, idx, w,
+                               status, s);
+            break;
+        default:
+            err = launch_s<8>(grid, mx, mw, c, n_pad, gate_bias, score_bias, score_fn, idx, w,
+                               status, s);
+            break;
     }
     if (err != cudaSuccess) return err;
     return cudaGetLastError();

@@ -56,18 +56,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase of parity `parity` has completed. Returns false if the
-// wait gave up (kWaitNs elapsed) or another role raised the abort flag.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const volatile int* abort_flag) {
+// wait gave up (limit_ns elapsed) or another role raised the abort flag.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity,
+                                              const volatile int* abort_flag, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0u) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitNs) return false;
+            if (globaltimer_ns() - t0 > limit_ns) return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          const volatile int* abort_flag) {
+    return mbar_wait_for(bar, parity, abort_flag, kWaitNs);
 }
 
 // ------------------------------------------------------------------ TMA

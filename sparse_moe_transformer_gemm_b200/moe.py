@@ -31,14 +31,18 @@ MOE_FLAG_STREAM_PATH = 0x2
 MOE_FLAG_GEMM_PATH = 0x4
 MOE_FLAG_PACKED_WEIGHTS = 0x8
 MOE_FLAG_SHARED_EXPERT = 0x10
+MOE_FLAG_FP4_WEIGHTS = 0x20
 MOE_WEIGHTS_GATE_UP = 0
 MOE_WEIGHTS_DOWN = 1
+MOE_SCORE_SIGMOID = 0
+MOE_SCORE_SQRT_SOFTPLUS = 1
+SCORE_FNS = {"sigmoid": MOE_SCORE_SIGMOID, "sqrtsoftplus": MOE_SCORE_SQRT_SOFTPLUS}
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
             "moe_permute_index", "moe_expert_gate_up", "moe_expert_gate_up_gather",
             "moe_expert_down", "moe_experts", "moe_combine", "moe_forward", "moe_read_status",
             "moe_status_string", "moe_route_noalloc", "moe_pack_weights", "moe_route2",
-            "moe_forward2")
+            "moe_forward2", "moe_route3", "moe_forward3", "moe_selftest_bounded_wait")
 
 MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
 # batches of at most this many token-slots (T*k) gather their token rows inside
@@ -54,6 +58,22 @@ class MoeConfig(ctypes.Structure):
     def __repr__(self):
         return (f"MoeConfig(T={self.T}, d={self.d}, E={self.E}, k={self.k}, d_ff={self.d_ff}, "
                 f"scale={self.scale}, flags={self.flags:#x})")
+
+
+class MoeRouteOptions(ctypes.Structure):
+    """moe_route_options: score_bias [E], norm_weight [d] (device pointers), norm_eps,
+    score_fn (MOE_SCORE_*)."""
+    _fields_ = [("score_bias", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p),
+                ("norm_eps", ctypes.c_float), ("score_fn", ctypes.c_int32)]
+
+
+def route_options(score_bias=None, norm_weight=None, norm_eps: float = 1e-6,
+                  score_fn: str = "sigmoid"):
+    """Router options; score_fn is "sigmoid" or "sqrtsoftplus" (or a MOE_SCORE_* value)."""
+    fn = SCORE_FNS[score_fn] if isinstance(score_fn, str) else int(score_fn)
+    return MoeRouteOptions(None if score_bias is None else score_bias.data_ptr(),
+                           None if norm_weight is None else norm_weight.data_ptr(),
+                           float(norm_eps), fn)
 
 
 class MoeError(RuntimeError):
@@ -94,6 +114,9 @@ def lib() -> ctypes.CDLL:
         "moe_pack_weights": (I, [C, I, P, P, P]),
         "moe_route2": (I, [C, P, P, P, P, P, P, P, S, P]),
         "moe_forward2": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "moe_route3": (I, [C, P, P, P, P, P, P, P, S, P]),
+        "moe_forward3": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "moe_selftest_bounded_wait": (I, [P, ctypes.c_ulonglong, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -104,11 +127,15 @@ def lib() -> ctypes.CDLL:
 
 
 def config(T: int, d: int, E: int, k: int, d_ff: int, scale: float = 2.826, fp8: bool = False,
-           path: Optional[str] = None, packed: bool = False, shared: bool = False) -> MoeConfig:
+           path: Optional[str] = None, packed: bool = False, shared: bool = False,
+           fp4: bool = False) -> MoeConfig:
     """Build a moe_config. path: None (automatic), "stream" or "gemm"; packed: the
     bf16 expert weights are in moe_pack_weights' layout; shared: expert E of the
-    weight arrays is a shared expert."""
+    weight arrays is a shared expert; fp4: E2M1 expert weights with E8M0 block
+    scales."""
     flags = MOE_FLAG_FP8_WEIGHTS if fp8 else 0
+    if fp4:
+        flags |= MOE_FLAG_FP4_WEIGHTS
     if packed:
         flags |= MOE_FLAG_PACKED_WEIGHTS
     if shared:
@@ -233,6 +260,22 @@ def moe_forward2(cfg, x, w_gate, gate_bias, score_bias, w_gate_up, s_gate_up, w_
                               _p(s_down), _p(out), _p(ws), ws.numel(), _s(stream)))
 
 
+def moe_route3(cfg, x, w_gate, gate_bias, opt, topk_idx, topk_w, ws, stream=None) -> None:
+    _check("moe_route3", lib().moe_route3(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
+                                          None if opt is None else ctypes.byref(opt),
+                                          _p(topk_idx), _p(topk_w), _p(ws), ws.numel(),
+                                          _s(stream)))
+
+
+def moe_forward3(cfg, x, w_gate, gate_bias, opt, w_gate_up, s_gate_up, w_down, s_down, out, ws,
+                 stream=None) -> None:
+    _check("moe_forward3",
+           lib().moe_forward3(ctypes.byref(cfg), _p(x), _p(w_gate), _p(gate_bias),
+                              None if opt is None else ctypes.byref(opt), _p(w_gate_up),
+                              _p(s_gate_up), _p(w_down), _p(s_down), _p(out), _p(ws), ws.numel(),
+                              _s(stream)))
+
+
 def moe_route_noalloc(cfg, x, w_gate, gate_bias, topk_idx, topk_w, stream=None) -> None:
     """moe_route without a workspace, for callers that cannot allocate device
     memory; the scratch is a fixed 2 MiB device array inside the library."""
@@ -247,14 +290,22 @@ def moe_pack_weights(cfg, which, w, w_packed, stream=None) -> None:
                                                       _p(w_packed), _s(stream)))
 
 
+def moe_selftest_bounded_wait(ws, limit_ns: int, stream=None) -> None:
+    """Run the bounded-wait self-test; its MOE_ERR_TIMEOUT lands in ws's status word."""
+    _check("moe_selftest_bounded_wait",
+           lib().moe_selftest_bounded_wait(_p(ws), int(limit_ns), _s(stream)))
+
+
 def moe_read_status(ws, stream=None) -> int:
     return int(lib().moe_read_status(_p(ws), _s(stream)))
 
 
 def layer_args(layer: dict):
-    """(w_gate_up, s_gate_up, w_down, s_down) of a synthetic layer dict, FP8 or bf16;
-    with a shared expert, its weights follow the routed ones as expert E."""
+    """(w_gate_up, s_gate_up, w_down, s_down) of a synthetic layer dict, FP4, FP8 or
+    bf16; with a shared expert, its weights follow the routed ones as expert E."""
     cfg = layer["cfg"]
+    if getattr(cfg, "fp4", False):
+        return (layer["q4_gate_up"], layer["s4_gate_up"], layer["q4_down"], layer["s4_down"])
     if cfg.fp8:
         args = [layer["q_gate_up"], layer["s_gate_up"], layer["q_down"], layer["s_down"]]
         sh = ("q_shared_gate_up", "s_shared_gate_up", "q_shared_down", "s_shared_down")
@@ -269,7 +320,7 @@ def layer_args(layer: dict):
 def config_of(shape, path: Optional[str] = None, packed: bool = False) -> MoeConfig:
     """moe_config for a synthetic LayerShape."""
     return config(shape.T, shape.d, shape.E, shape.k, shape.F, shape.scale, shape.fp8, path,
-                  packed, getattr(shape, "shared", False))
+                  packed, getattr(shape, "shared", False), getattr(shape, "fp4", False))
 
 
 def pack_layer_weights(cfg: MoeConfig, w_gate_up: torch.Tensor, w_down: torch.Tensor,

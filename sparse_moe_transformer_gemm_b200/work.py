@@ -4,7 +4,8 @@
 kernels are tiled:
 
 * bytes  = weights of the experts that at least one token selects (plus their
-  fp32 row scales for FP8 weights) + router weight + x read + out write;
+  fp32 row scales for FP8 weights, their E8M0 block scales for FP4 weights) +
+  router weight + x read + out write;
 * flops  = 2*T*d*E (router) + 6*T*k*d*F (gate, up and down projections of the
   k selected experts; 6*d*F per token per expert is the per-expert count of
   "Tencent Hy3-Flash QA", Q2.4).
@@ -13,32 +14,42 @@ kernels are tiled:
 from __future__ import annotations
 
 
-def expert_bytes(d: int, F: int, fp8: bool = False) -> int:
-    """Weight bytes of one expert: 3*d*F elements (FP8: plus 2F + d fp32 row scales)."""
+def weight_bytes(rows: int, cols: int, fp8: bool = False, fp4: bool = False) -> int:
+    """Bytes of one [rows, cols] expert weight with its scales: bf16 2 bytes per
+    element; FP8 1 byte + an fp32 scale per row; FP4 half a byte + an E8M0 byte
+    per 32 elements of a row."""
+    if fp4:
+        return rows * cols // 2 + rows * (cols // 32)
     if fp8:
-        return 3 * d * F + (2 * F + d) * 4
-    return 3 * d * F * 2
+        return rows * cols + rows * 4
+    return rows * cols * 2
+
+
+def expert_bytes(d: int, F: int, fp8: bool = False, fp4: bool = False) -> int:
+    """Weight bytes of one expert: gate_up [2F, d] and down [d, F] with their scales."""
+    return weight_bytes(2 * F, d, fp8, fp4) + weight_bytes(d, F, fp8, fp4)
 
 
 def expert_flops_per_token(d: int, F: int) -> int:
     return 6 * d * F
 
 
-def layer_work(T: int, d: int, E: int, k: int, F: int, touched: int, fp8: bool = False) -> dict:
-    byts = touched * expert_bytes(d, F, fp8) + E * d * 2 + 2 * T * d * 2
+def layer_work(T: int, d: int, E: int, k: int, F: int, touched: int, fp8: bool = False,
+               fp4: bool = False) -> dict:
+    byts = touched * expert_bytes(d, F, fp8, fp4) + E * d * 2 + 2 * T * d * 2
     flops = 2 * T * d * E + T * k * expert_flops_per_token(d, F)
     return {"bytes": byts, "flops": flops}
 
 
-def gate_up_work(n_rows: int, touched: int, d: int, F: int, fp8: bool = False) -> dict:
+def gate_up_work(n_rows: int, touched: int, d: int, F: int, fp8: bool = False,
+                 fp4: bool = False) -> dict:
     """The gate_up step alone: touched experts' [2F, d] weights, x rows in, h out."""
-    wb = 1 if fp8 else 2
-    byts = touched * (2 * F * d * wb + (2 * F * 4 if fp8 else 0)) + n_rows * d * 2 + n_rows * F * 2
+    byts = touched * weight_bytes(2 * F, d, fp8, fp4) + n_rows * d * 2 + n_rows * F * 2
     return {"bytes": byts, "flops": 4 * n_rows * d * F}
 
 
-def down_work(n_rows: int, touched: int, d: int, F: int, fp8: bool = False) -> dict:
+def down_work(n_rows: int, touched: int, d: int, F: int, fp8: bool = False,
+              fp4: bool = False) -> dict:
     """The down step alone: touched experts' [d, F] weights, h in, y out."""
-    wb = 1 if fp8 else 2
-    byts = touched * (d * F * wb + (d * 4 if fp8 else 0)) + n_rows * F * 2 + n_rows * d * 2
+    byts = touched * weight_bytes(d, F, fp8, fp4) + n_rows * F * 2 + n_rows * d * 2
     return {"bytes": byts, "flops": 2 * n_rows * d * F}

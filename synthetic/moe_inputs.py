@@ -11,6 +11,8 @@ decode        64  4096  192   8  1536  as tiny: logit std 0.02*sqrt(4096) = 1.28
 prefill     4096  4096  192   8  1536  as decode, ~170.7 rows per expert
 skewed     16384  4096  192   8  1536  + per-expert logit bias 0.5*ln(Zipf(1.1) rank weight)
 fp8         8192  4096  192   8  1536  expert weights e4m3 + fp32 scale per output row
+fp4_decode    64  4096  192   6  1536  sqrt-softplus scores, scale 1.5; experts E2M1 +
+                                       E8M0 scale per 32 row elements (from the bf16 draw)
 =========  =====  ====  ===  ==  ====  ===============================================
 
 The Hy3 sizes (d=4096, 192 routed experts, top-8, expert d_ff=1536, router
@@ -80,6 +82,10 @@ CONFIGS = {
     "prefill": LayerShape(T=4096, d=4096, E=192, k=8, F=1536),
     "skewed": LayerShape(T=16384, d=4096, E=192, k=8, F=1536, zipf_bias=True),
     "fp8": LayerShape(T=8192, d=4096, E=192, k=8, F=1536, fp8=True),
+    # the second routing and precision variant at the decode shape: top-6
+    # sqrt-softplus scores with scale 1.5, FP4 E2M1 experts (block-32 E8M0 scales)
+    "fp4_decode": LayerShape(T=64, d=4096, E=192, k=6, F=1536, scale=1.5, fp4=True,
+                             score_fn="sqrtsoftplus"),
 }
 
 
@@ -209,8 +215,16 @@ def make_layer(cfg, seed: int = 0, device="cpu", T: Optional[int] = None,
         out["score_bias"] = torch.randn((E,), generator=gen, dtype=torch.float32,
                                         device=dev) * cfg.score_bias_std
     if cfg.fp4:
-        q4_gu, s4_gu = encode_e2m1_blocks(w_gate_up)
-        q4_d, s4_d = encode_e2m1_blocks(w_down)
+        # one expert at a time (blocks are independent): bounded temporaries at
+        # the full Hy3 sizes
+        d, F = cfg.d, cfg.F
+        q4_gu = torch.empty((E, 2 * F, d // 2), dtype=torch.uint8, device=dev)
+        s4_gu = torch.empty((E, 2 * F, d // 32), dtype=torch.uint8, device=dev)
+        q4_d = torch.empty((E, d, F // 2), dtype=torch.uint8, device=dev)
+        s4_d = torch.empty((E, d, F // 32), dtype=torch.uint8, device=dev)
+        for e in range(E):
+            q4_gu[e], s4_gu[e] = encode_e2m1_blocks(w_gate_up[e])
+            q4_d[e], s4_d[e] = encode_e2m1_blocks(w_down[e])
         out.update(q4_gate_up=q4_gu, s4_gate_up=s4_gu, q4_down=q4_d, s4_down=s4_d)
     out["route_norm_weight"] = None
     if cfg.route_norm:

@@ -24,14 +24,22 @@ MAX_ABS = 5e-2
 W_RTOL = 2e-5
 
 
+def route_options(layer):
+    """The layer's router options (score bias, route_norm, score function)."""
+    cfg = layer["cfg"]
+    return moe.route_options(layer.get("score_bias"), layer.get("route_norm_weight"),
+                             getattr(cfg, "route_norm_eps", 1e-6),
+                             getattr(cfg, "score_fn", "sigmoid"))
+
+
 def gpu_route(layer, path=None):
     cfg = moe.config_of(layer["cfg"], path)
     T, k = layer["cfg"].T, layer["cfg"].k
     ws = moe.workspace(cfg)
     idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
     w = torch.empty((T, k), dtype=torch.float32, device="cuda")
-    moe.moe_route2(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"),
-                   layer.get("score_bias"), idx, w, ws)
+    opt = route_options(layer)
+    moe.moe_route3(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"), opt, idx, w, ws)
     torch.cuda.synchronize()
     assert moe.moe_read_status(ws) == moe.MOE_OK
     return idx.cpu().numpy(), w.cpu().numpy()
@@ -44,8 +52,9 @@ def gpu_forward(layer, path=None, ws=None, out=None):
         ws = moe.workspace(cfg)
     if out is None:
         out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
-    moe.moe_forward2(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"),
-                     layer.get("score_bias"), *moe.layer_args(layer), out, ws)
+    opt = route_options(layer)
+    moe.moe_forward3(cfg, layer["x"], layer["w_gate"], layer.get("gate_bias"), opt,
+                     *moe.layer_args(layer), out, ws)
     torch.cuda.synchronize()
     assert moe.moe_read_status(ws) == moe.MOE_OK
     return out
@@ -83,12 +92,16 @@ def check_near_tie_selection(gpu_idx, scores, t, k):
 
 def oracle_out_with_selection(O, t, experts):
     """Oracle output of token t when it is routed to ``experts`` (weights from the
-    oracle's fp64 sigmoid scores, renormalised over that set; the shared expert,
-    if any, added last with weight 1)."""
-    scores = oracle.route(O.x[t:t + 1], O.wg, O.k, O.scale, O.gate_bias, want_scores=True)["scores"]
+    oracle's fp64 scores, renormalised over that set; the shared expert, if any,
+    added last with weight 1)."""
+    scores = oracle.route(O.x[t:t + 1], O.wg, O.k, O.scale, O.gate_bias, want_scores=True,
+                          norm_w=O.norm_w, norm_eps=O.norm_eps, score_fn=O.score_fn)["scores"]
     experts = np.asarray(experts, np.int32)
     xrows = np.repeat(O.x[t:t + 1], len(experts), axis=0)
-    y = oracle.expert_rows(xrows, experts, O.wgu, O.wd, O.s_gu, O.s_d)
+    if O.fp4:
+        y = oracle.expert_rows_fp4(xrows, experts, O.wgu4, O.sgu8, O.wd4, O.sd8)
+    else:
+        y = oracle.expert_rows(xrows, experts, O.wgu, O.wd, O.s_gu, O.s_d)
     s = scores[0, experts]
     w = O.scale * s / s.sum()
     if O.sh_wgu is not None:

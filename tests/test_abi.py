@@ -35,10 +35,11 @@ def test_header_constants_match_the_binding():
     m = re.search(r"#define MOE_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
     assert m and int(m.group(1)) << int(m.group(2)) == moe.MOE_NOALLOC_SCRATCH_BYTES
     for name in ("MOE_FLAG_FP8_WEIGHTS", "MOE_FLAG_STREAM_PATH", "MOE_FLAG_GEMM_PATH",
-                 "MOE_FLAG_PACKED_WEIGHTS", "MOE_FLAG_SHARED_EXPERT"):
+                 "MOE_FLAG_PACKED_WEIGHTS", "MOE_FLAG_SHARED_EXPERT", "MOE_FLAG_FP4_WEIGHTS"):
         m = re.search(r"#define %s (0x[0-9a-f]+)u" % name, text)
         assert m and int(m.group(1), 16) == getattr(moe, name), name
-    for name in ("MOE_WEIGHTS_GATE_UP", "MOE_WEIGHTS_DOWN"):
+    for name in ("MOE_WEIGHTS_GATE_UP", "MOE_WEIGHTS_DOWN", "MOE_SCORE_SIGMOID",
+                 "MOE_SCORE_SQRT_SOFTPLUS"):
         m = re.search(r"#define %s (\d+)" % name, text)
         assert m and int(m.group(1)) == getattr(moe, name), name
 
@@ -60,6 +61,48 @@ def test_shared_expert_flag_rules(lib):
     assert moe.moe_workspace_size(moe.config(**{**HY3, "E": 255}, shared=True)) > 0
     assert moe.moe_workspace_size(moe.config(**{**HY3, "E": 256}, shared=True)) == 0
     assert moe.moe_workspace_size(moe.config(**{**HY3, "E": 256})) > 0
+
+
+def test_fp4_weights_flag_rules(lib):
+    assert moe.moe_workspace_size(moe.config(**HY3, fp4=True)) > 0
+    assert moe.moe_workspace_size(moe.config(**HY3, fp4=True, path="stream")) > 0
+    for bad in (dict(fp8=True), dict(packed=True), dict(path="gemm"), dict(shared=True)):
+        assert moe.moe_workspace_size(moe.config(**HY3, fp4=True, **bad)) == 0, bad
+    # FP4 weights need their block scales
+    cfg = moe.config(**HY3, fp4=True)
+    P = ctypes.c_void_p
+    rc = _call("moe_expert_down", ctypes.byref(cfg), P(FAKE), P(FAKE), P(FAKE), None, P(FAKE),
+               P(FAKE), moe.moe_workspace_size(cfg), None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+
+
+def test_route_options_struct_matches_the_header():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    body = re.search(r"typedef struct moe_route_options \{(.*?)\} moe_route_options;", text,
+                     re.S).group(1)
+    fields = re.findall(r"(\w+);", body)
+    assert fields == [f for f, _ in moe.MoeRouteOptions._fields_]
+    assert ctypes.sizeof(moe.MoeRouteOptions) == 24
+
+
+def test_route_options_are_checked_before_any_launch(lib):
+    cfg = moe.config(**HY3)
+    ws_n = moe.moe_workspace_size(cfg)
+    P = ctypes.c_void_p
+    bad = moe.MoeRouteOptions(None, FAKE, 0.0)      # a norm weight needs eps > 0
+    rc = _call("moe_route3", ctypes.byref(cfg), P(FAKE), P(FAKE), None, ctypes.byref(bad),
+               P(FAKE), P(FAKE), P(FAKE), ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    bad = moe.MoeRouteOptions(None, FAKE, float("nan"))
+    rc = _call("moe_forward3", ctypes.byref(cfg), P(FAKE), P(FAKE), None, ctypes.byref(bad),
+               P(FAKE), None, P(FAKE), None, P(FAKE), P(FAKE), ws_n, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    for fn in (-1, 2):  # no such score function
+        bad = moe.MoeRouteOptions(None, None, 0.0, fn)
+        rc = _call("moe_route3", ctypes.byref(cfg), P(FAKE), P(FAKE), None, ctypes.byref(bad),
+                   P(FAKE), P(FAKE), P(FAKE), ws_n, None)
+        assert rc == moe.MOE_ERR_INVALID_ARG
+    assert moe.route_options(score_fn="sqrtsoftplus").score_fn == moe.MOE_SCORE_SQRT_SOFTPLUS
 
 
 def test_pack_weights_rejects_bad_arguments(lib):
@@ -185,6 +228,8 @@ def test_unsupported_shape_is_reported_by_every_entry_point(lib):
         "moe_pack_weights": (moe.MOE_WEIGHTS_GATE_UP, f, P(FAKE + (1 << 34)), None),
         "moe_route2": (f, f, None, None, f, f, f, 1 << 30, None),
         "moe_forward2": (f, f, None, None, f, None, f, None, f, f, 1 << 30, None),
+        "moe_route3": (f, f, None, None, f, f, f, 1 << 30, None),
+        "moe_forward3": (f, f, None, None, f, None, f, None, f, f, 1 << 30, None),
     }
     for fn, args in cases.items():
         assert _call(fn, ctypes.byref(cfg), *args) == moe.MOE_ERR_UNSUPPORTED_SHAPE, fn

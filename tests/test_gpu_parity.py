@@ -326,6 +326,30 @@ def test_complete_block_with_packed_weights_is_bitwise_the_same():
     assert torch.equal(out, want)
 
 
+# route_norm (RMSNorm of the router's input; the experts take x)
+NORM = {
+    "norm_decode": dataclasses.replace(CONFIGS["decode"], route_norm=True),
+    "norm_tc_sized": LayerShape(T=300, d=512, E=32, k=8, F=256, route_norm=True),
+    "norm_block": LayerShape(T=200, d=512, E=16, k=4, F=512, shared=True, score_bias_std=0.05,
+                             route_norm=True),
+}
+
+
+@pytest.mark.parametrize("name", sorted(NORM))
+def test_route_norm_every_token(name):
+    sh = NORM[name]
+    layer = make_layer(sh, seed=51, device="cuda")
+    route = parity.gpu_route(layer)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias, score_bias=O.score_bias,
+                       norm_w=O.norm_w, norm_eps=O.norm_eps)
+    parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer)
+    res = parity.check_forward(layer, out, None, route)
+    print(name, res)
+    _free(layer, out)
+
+
 def test_fp32_combine_keeps_small_terms():
     """Hy3 commentary §2.3 example: one branch output 8.2 and seven of 0.03 (all
     already bf16). An fp32 sum gives 8.375 after the cast; a bf16 running sum
@@ -385,3 +409,101 @@ def test_repeated_calls_are_bitwise_deterministic():
     a = parity.gpu_forward(layer).clone()
     b = parity.gpu_forward(layer)
     assert torch.equal(a, b)
+
+
+# The second routing and precision variant (the V4-Flash column of
+# "Tencent Hy3-295B 架构深度拆解" §2.2): sqrt(softplus) scores (scale 1.5) and FP4
+# E2M1 experts with E8M0 block-32 scales (the weight-streaming kernels).
+F4 = {
+    # the CUDA-core router (T <= 128) and the tensor-core one (T >= 129)
+    "sqrtsp_small": LayerShape(T=100, d=256, E=32, k=6, F=128, scale=1.5,
+                               score_fn="sqrtsoftplus"),
+    "sqrtsp_tc": LayerShape(T=300, d=512, E=32, k=6, F=256, scale=1.5, score_fn="sqrtsoftplus"),
+    "sqrtsp_bias": LayerShape(T=200, d=512, E=16, k=4, F=256, scale=1.5, score_fn="sqrtsoftplus",
+                              score_bias_std=0.05),
+    "fp4_tiny": LayerShape(T=64, d=256, E=16, k=4, F=128, scale=1.5, fp4=True,
+                           score_fn="sqrtsoftplus"),
+    # ~56 rows per expert: several passes of the streaming kernels' 8-row staging
+    "fp4_ragged": LayerShape(T=300, d=512, E=32, k=6, F=384, scale=1.5, fp4=True,
+                             score_fn="sqrtsoftplus", score_bias_std=0.05),
+    "fp4_sigmoid": LayerShape(T=40, d=384, E=8, k=2, F=256, fp4=True),
+}
+
+
+@pytest.mark.parametrize("name", sorted(F4))
+def test_second_variant_every_token(name):
+    sh = F4[name]
+    layer = make_layer(sh, seed=61, device="cuda")
+    route = parity.gpu_route(layer)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias, score_bias=O.score_bias,
+                       score_fn=O.score_fn)
+    parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer)
+    res = parity.check_forward(layer, out, None, route)
+    print(name, res)
+    _free(layer, out)
+
+
+@pytest.mark.parametrize("T", [7, 300])
+def test_sqrt_softplus_router_on_hy3_shape(T):
+    """sqrt-softplus top-6 at d=4096, E=192 on both router kernels."""
+    shape = dataclasses.replace(CONFIGS["decode"], T=T, k=6, scale=1.5, score_fn="sqrtsoftplus")
+    layer = make_layer(shape, seed=T + 1, device="cuda", with_experts=False)
+    route = parity.gpu_route(layer)
+    ref = oracle.route(oracle.bf16_bits(layer["x"]), oracle.bf16_bits(layer["w_gate"]), shape.k,
+                       shape.scale, score_fn="sqrtsoftplus")
+    parity.check_route(*route, ref)
+
+
+def test_fp4_decode_hy3_shape():
+    """FP4 experts at the Hy3 decode shape (T=64, d=4096, E=192, d_ff=1536), top-6
+    sqrt-softplus routing: every token routed, a sample of outputs."""
+    shape = dataclasses.replace(CONFIGS["decode"], k=6, scale=1.5, fp4=True,
+                                score_fn="sqrtsoftplus")
+    layer = make_layer(shape, seed=5, device="cuda")
+    route = parity.gpu_route(layer)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, score_fn="sqrtsoftplus")
+    near = parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer)
+    toks = np.unique(np.concatenate([parity.sample_tokens(shape.T, n=32),
+                                     near[:8].astype(np.int32)]))
+    res = parity.check_forward(layer, out, toks, route)
+    print("fp4 decode, near ties:", len(near), res)
+    _free(layer, out)
+
+
+# The largest supported shapes: 256 experts with k = 32 (the CUDA-core router's
+# 32 rounds, the one-CTA grouping over 256 experts, the 32-row combine), and
+# d = d_ff = 8192 (128 KB of staged rows on the streaming path, 128 K blocks
+# on the pair GEMMs).
+MAX = {
+    "e256_k32": LayerShape(T=40, d=256, E=256, k=32, F=128),
+    "d8192": LayerShape(T=16, d=8192, E=8, k=2, F=8192),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MAX))
+@pytest.mark.parametrize("path", [None, "stream", "gemm"])
+def test_largest_supported_shapes_every_token(name, path):
+    sh = MAX[name]
+    layer = make_layer(sh, seed=81, device="cuda")
+    route = parity.gpu_route(layer, path)
+    O = oracle.OracleLayer(layer)
+    ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias)
+    parity.check_route(*route, ref)
+    out = parity.gpu_forward(layer, path)
+    res = parity.check_forward(layer, out, None, route)
+    print(name, path, res)
+    _free(layer, out)
+
+
+@pytest.mark.parametrize("T", [16, 200])
+def test_router_at_d8192_on_both_kernels(T):
+    shape = LayerShape(T=T, d=8192, E=256, k=8, F=128, zipf_bias=True)
+    layer = make_layer(shape, seed=83, device="cuda", with_experts=False)
+    route = parity.gpu_route(layer)
+    ref = oracle.route(oracle.bf16_bits(layer["x"]), oracle.bf16_bits(layer["w_gate"]), shape.k,
+                       shape.scale, layer["gate_bias"].cpu().numpy())
+    parity.check_route(*route, ref)

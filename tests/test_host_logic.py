@@ -10,6 +10,7 @@ import torch
 from sparse_moe_transformer_gemm_b200 import build as moe_build
 from sparse_moe_transformer_gemm_b200 import moe, work
 from synthetic import CONFIGS, LayerShape, make_layer
+from synthetic.moe_inputs import encode_e2m1_blocks
 
 BASE = LayerShape(T=12, d=128, E=6, k=2, F=128)
 
@@ -63,6 +64,19 @@ def test_config_flags():
         moe.config(64, 4096, 192, 8, 1536, path="fast")
     assert moe.config_of(dataclasses.replace(CONFIGS["decode"], shared=True)).flags == \
         moe.MOE_FLAG_SHARED_EXPERT
+    assert moe.config_of(CONFIGS["fp4_decode"]).flags == moe.MOE_FLAG_FP4_WEIGHTS
+
+
+def test_fp4_layer_args_are_the_codes_and_block_scales():
+    sh = dataclasses.replace(BASE, fp4=True)
+    L = make_layer(sh, seed=2)
+    q_gu, s_gu, q_dn, s_dn = moe.layer_args(L)
+    assert q_gu.dtype == s_gu.dtype == torch.uint8
+    assert q_gu.shape == (sh.E, 2 * sh.F, sh.d // 2) and s_gu.shape == (sh.E, 2 * sh.F, sh.d // 32)
+    assert q_dn.shape == (sh.E, sh.d, sh.F // 2) and s_dn.shape == (sh.E, sh.d, sh.F // 32)
+    # one expert at a time is the same encoding as the whole tensor at once
+    q_all, s_all = encode_e2m1_blocks(L["w_gate_up"])
+    assert torch.equal(q_all, q_gu) and torch.equal(s_all, s_gu)
 
 
 @pytest.fixture(scope="module")
@@ -84,6 +98,10 @@ def test_work_accounting_matches_the_page_figures():
     # 3 d F parameters per expert, 6 d F FLOPs per token per expert (Hy3 pages)
     assert work.expert_bytes(4096, 1536) == 3 * 4096 * 1536 * 2
     assert work.expert_bytes(4096, 1536, fp8=True) == 3 * 4096 * 1536 + (2 * 1536 + 4096) * 4
+    # FP4: half a byte per weight and one E8M0 byte per 32 weights of a row
+    assert work.expert_bytes(4096, 1536, fp4=True) == 3 * 4096 * 1536 // 2 + 3 * 4096 * 1536 // 32
+    gw = work.gate_up_work(384, 150, 4096, 1536, fp4=True)
+    assert gw["bytes"] == 150 * (3072 * 4096 // 2 + 3072 * 128) + 384 * (4096 + 1536) * 2
     lw = work.layer_work(64, 4096, 192, 8, 1536, touched=175)
     assert lw["flops"] == 2 * 64 * 4096 * 192 + 6 * 64 * 8 * 4096 * 1536
     assert lw["bytes"] >= 175 * work.expert_bytes(4096, 1536)
