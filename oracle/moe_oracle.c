@@ -15,7 +15,11 @@
  *   1. logit_e = sum_c x[t,c] * Wg[e,c]  (+ gate_bias[e] when given)
  *   2. s_e     = 1 / (1 + exp(-logit_e))
  *   3. the k experts of largest s_e; equal scores go to the lower expert index
- *      (a full sort of (-s_e, e), then the first k)
+ *      (a full sort of (-s_e, e), then the first k). Both score functions
+ *      below are strictly increasing, so the order of the exact scores is the
+ *      order of the logits: the sort ranks the logits, which fp64 holds apart
+ *      where the rounded scores are not (every logit above ~37 has the fp64
+ *      sigmoid 1.0), and equal scores are exactly equal logits.
  *   4. w_j     = scale * s_j / sum_{i in top-k} s_i
  *   5. for each selected expert e:
  *        g_f = sum_c x_c Wgu[e, f, c],  u_f = sum_c x_c Wgu[e, F+f, c]
@@ -189,7 +193,9 @@ static double weight_at_fp4(const uint8_t* w, const uint8_t* scales, long e, lon
 /* ---------------------------------------------------------------- routing */
 
 typedef struct {
-    double key; /* what the choice ranks: s, plus the score bias when given */
+    double key; /* what the choice ranks: the logit (the order of the exact
+                   scores), or s plus the score bias when that is given */
+    double v;   /* the ranked value in score units: s, or s + score bias */
     double s;   /* sigmoid score */
     int e;
 } scored_expert;
@@ -207,8 +213,9 @@ static int by_score_then_index(const void* pa, const void* pb)
 }
 
 /* Route one token: steps 1-4 above. Writes k indices (descending key), their
- * k weights, optionally all E logits and scores, and the gap between the k-th
- * and (k+1)-th largest key (+inf when k == E). score_bias may be NULL. */
+ * k weights, optionally all E logits and scores, and the gap between the
+ * ranked values (in score units) of the k-th and (k+1)-th expert of the order
+ * (+inf when k == E). score_bias may be NULL. */
 static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
                         const uint16_t* wg, const float* gate_bias, const float* score_bias,
                         const float* norm_w, double norm_eps, int score_fn, int32_t* idx,
@@ -236,7 +243,8 @@ static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
         if (gate_bias)
             logit += (double)gate_bias[e];
         order[e].s = score_of(logit, score_fn);
-        order[e].key = score_bias ? order[e].s + (double)score_bias[e] : order[e].s;
+        order[e].v = score_bias ? order[e].s + (double)score_bias[e] : order[e].s;
+        order[e].key = score_bias ? order[e].v : logit;
         order[e].e = e;
         if (logits_out)
             logits_out[e] = logit;
@@ -250,7 +258,7 @@ static void route_token(int d, int E, int k, double scale, const uint16_t* xrow,
         idx[j] = order[j].e;
         w[j] = scale * order[j].s / sel_sum;
     }
-    *gap = (k < E) ? order[k - 1].key - order[k].key : INFINITY;
+    *gap = (k < E) ? order[k - 1].v - order[k].v : INFINITY;
     free(xr);
     free(order);
 }

@@ -29,7 +29,9 @@ MUTATIONS = {
     "bias_dropped": ("logit += (double)gate_bias[e];", "logit += 0.0 * gate_bias[e];"),
     "fp8_scale_dropped": ("* (double)scales[e * rows + r];", "* 1.0;"),
     "e4m3_subnormal_exponent": ("v = ldexp((double)mant / 8.0, -6);", "v = ldexp((double)mant / 8.0, -7);"),
-    "gap_wrong_neighbour": ("order[k - 1].key - order[k].key", "order[0].key - order[k].key"),
+    "gap_wrong_neighbour": ("order[k - 1].v - order[k].v", "order[0].v - order[k].v"),
+    "rank_by_rounded_score": ("order[e].key = score_bias ? order[e].v : logit;",
+                              "order[e].key = order[e].v;"),
     "score_bias_dropped": ("order[e].s + (double)score_bias[e]", "order[e].s"),
     "score_bias_in_the_weights": ("sel_sum += order[j].s;", "sel_sum += order[j].key;"),
     "shared_expert_dropped": ("a += y_shared[i];", "a += 0.0 * y_shared[i];"),

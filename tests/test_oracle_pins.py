@@ -158,6 +158,28 @@ def test_equal_scores_take_lowest_indices_and_split_the_scale(golden):
     assert np.all(r["gap"] == 0.0)
 
 
+def test_saturated_scores_rank_by_the_exact_order():
+    """Logits 45 on expert 9 and 40 on expert 3 (a zero token and a logit bias):
+    both sigmoids round to 1.0 in fp64, yet the exact scores put 9 before 3; the
+    other experts (logit 0, score 0.5) follow by index. The weights use the
+    rounded scores: 2.826 * (1, 1, 0.5 x 6) / 5."""
+    assert 1.0 / (1.0 + math.exp(-40.0)) == 1.0
+    x = np.zeros((1, 8), np.uint16)
+    wg = np.zeros((12, 8), np.uint16)
+    b = np.zeros(12, np.float32)
+    b[9], b[3] = 45.0, 40.0
+    r = oracle.route(x, wg, 1, 2.826, gate_bias=b)
+    assert r["idx"][0, 0] == 9 and r["w"][0, 0] == 2.826
+    r = oracle.route(x, wg, 8, 2.826, gate_bias=b)
+    assert r["idx"][0].tolist() == [9, 3, 0, 1, 2, 4, 5, 6]
+    want = 2.826 * np.array([1.0, 1.0] + [0.5] * 6) / 5.0
+    assert np.allclose(r["w"][0], want, rtol=1e-15, atol=0)
+    assert r["gap"][0] == 0.0   # scores 0.5 and 0.5 at the 8th and 9th places
+    # the square root of the softplus does not saturate: the same order
+    r = oracle.route(x, wg, 2, 1.5, gate_bias=b, score_fn="sqrtsoftplus")
+    assert r["idx"][0].tolist() == [9, 3]
+
+
 def test_scaled_weight_example(golden):
     """A normalised weight of 0.12 becomes 0.12 * 2.826 = 0.33912 (page prints 0.338)."""
     ex = golden["scaled_example"]
