@@ -153,3 +153,44 @@ def sample_tokens(T: int, n: int = 48, seed: int = 0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     mid = rng.choice(np.arange(8, T - 8), size=n, replace=False)
     return np.unique(np.concatenate([np.arange(8), mid, np.arange(T - 8, T)])).astype(np.int32)
+
+
+def gemm_tiles(counts, nmax: int = 256):
+    """The token tiles of the grouped GEMMs: expert e's n_e grouped rows split
+    into ceil(n_e / nmax) parts of near-equal length (the first n_e mod parts
+    one row longer). Yields (e, first row, length) with rows counted from the
+    expert's first grouped row."""
+    for e, n in enumerate(np.asarray(counts).tolist()):
+        if n == 0:
+            continue
+        nt = (n + nmax - 1) // nmax
+        base, rem = divmod(n, nt)
+        for j in range(nt):
+            yield e, j * base + min(j, rem), base + (1 if j < rem else 0)
+
+
+def tile_cover_tokens(idx: np.ndarray, E: int, edge: int = 32, nmax: int = 256) -> np.ndarray:
+    """Tokens that put a grouped row into the first and into the last ``edge``
+    rows of every (expert, token tile) of the grouped GEMMs, chosen greedily
+    (each token brings k rows). The grouping is the oracle's (row_of), so the
+    rows are those the GPU's GEMMs compute for the same routing."""
+    T, k = idx.shape
+    g = oracle.permute(idx, E)
+    offsets, row_of = g["offsets"], g["row_of"]
+    token_of_row = np.empty(T * k, dtype=np.int64)
+    token_of_row[row_of] = np.arange(T * k) // k
+    targets = {}   # target id -> set of candidate tokens
+    for e, start, n in gemm_tiles(g["counts"], nmax):
+        r0 = offsets[e] + start
+        for lo, hi in ((r0, r0 + min(edge, n)), (r0 + n - min(edge, n), r0 + n)):
+            targets[len(targets)] = set(token_of_row[lo:hi].tolist())
+    covers = {}
+    for tid, toks in targets.items():
+        for t in toks:
+            covers.setdefault(t, set()).add(tid)
+    left, chosen = set(targets), []
+    while left:
+        t = max(covers, key=lambda c: (len(covers[c] & left), -c))
+        chosen.append(t)
+        left -= covers[t]
+    return np.array(sorted(chosen), dtype=np.int32)
