@@ -278,6 +278,23 @@ MOE_API int moe_forward3(const moe_config* cfg, const void* x, const void* w_gat
                  const void* s_gate_up, const void* w_down, const void* s_down, void* out,
                  void* ws, size_t ws_bytes, void* stream);
 
+/* Expert parallelism ("DeepSeek V4-Flash 架构 QA" Q4.7, the expert-parallel
+ * strategy, and Q4.10, the MoE's all-to-all traffic): P ranks each own
+ * E_local = E/P consecutive experts. A rank receives the grouped token rows
+ * of its experts from n_src ranks, source by source, each source's rows
+ * grouped by local expert: counts [n_src, E_local] int32 (device) holds the
+ * rows of local expert e from source p at counts[p * E_local + e]. Writes
+ * expert_of_row [n_rows] int32 (device): the local expert of each received
+ * row in that arrival order, the routing (k = 1) with which moe_permute
+ * regroups the rows by expert for the local grouped GEMMs. Rows at or past
+ * the sum of counts get -1. n_src * E_local <= MOE_EP_MAX_SEGMENTS and
+ * E_local <= 256, else MOE_ERR_UNSUPPORTED_SHAPE; NULL pointers or
+ * n_rows < 1: MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE. Asynchronous on
+ * stream; allocates nothing. */
+#define MOE_EP_MAX_SEGMENTS 8192
+MOE_API int moe_ep_row_experts(const int32_t* counts, int32_t n_src, int32_t E_local,
+                               int32_t* expert_of_row, int32_t n_rows, void* stream);
+
 /* Failure-detection self-test: one thread waits, with the library's bounded
  * wait and a limit of limit_ns (1 ns .. 10 s), on an mbarrier that nothing
  * completes, then records MOE_ERR_TIMEOUT in the status word of ws (read it
@@ -290,16 +307,22 @@ MOE_API int moe_selftest_bounded_wait(void* ws, unsigned long long limit_ns, voi
 
 /* moe_route for callers that cannot allocate device memory (no workspace
  * argument). The pages have no counterpart: this is a deployment convenience.
- * Same routing as moe_route, bitwise. Its scratch -- fp32 logits [T, E] and
- * one counter per 8 tokens -- lives in a device array of
- * MOE_NOALLOC_SCRATCH_BYTES compiled into the library, held on every GPU that
- * loads it until the process exits. Returns MOE_ERR_UNSUPPORTED_SHAPE when
- * 4*T*E plus the counters (4*ceil(T/8) bytes, rounded up to 256) exceed that
- * size (T <= 2728 at E = 192), besides the shape checks of moe_route. The
- * first call on a device (that device current) looks up the array's address;
- * make it before any stream capture. All calls share the array: calls that
- * overlap on the GPU race and must be serialised by the caller. It calls no
- * allocator. */
+ * It runs the CUDA-core router with moe_route's K split S (1 <= S <= 16; S = 1
+ * for every T > 128 at E = 192): where moe_route runs that router too (T <=
+ * 128, or k > 8) the indices and weights are bitwise moe_route's. For
+ * T >= 129 with k <= 8, moe_route runs the tensor-core router, whose logits
+ * sum in another order: the same experts on every token whose k-th/(k+1)-th
+ * score gap is at least ~1e-5, the weights within ~2e-5 relative. Its scratch
+ * -- fp32 partial logits [S, T, E] and one counter per 8 tokens -- lives in a
+ * device array of MOE_NOALLOC_SCRATCH_BYTES compiled into the library, held
+ * on every GPU that loads it until the process exits. Returns
+ * MOE_ERR_UNSUPPORTED_SHAPE when 4*S*T*E plus the counters (4*ceil(T/8)
+ * bytes, rounded up to 256) exceed that size (T <= 2728 at E = 192), besides
+ * the shape checks of moe_route. The first call on a device (that device
+ * current) looks up the array's address; make it before any stream capture
+ * (later calls outside capture look it up again, so a device reset leaves no
+ * stale address). All calls share the array: calls that overlap on the GPU
+ * race and must be serialised by the caller. It calls no allocator. */
 MOE_API int moe_route_noalloc(const moe_config* cfg, const void* x, const void* w_gate,
                               const float* gate_bias, int32_t* topk_idx, float* topk_w,
                               void* stream);

@@ -14,9 +14,22 @@
 //
 // Set-up: the first call on each device, with that device current, looks up
 // the array's device address (cudaGetSymbolAddress) and remembers it; make
-// that first call before any stream capture. Host code cannot pass the array's
-// name to a kernel directly -- on the host it denotes a host-side stand-in,
-// not the device memory.
+// that first call before any stream capture. Later calls on a stream that is
+// not being captured look the address up again (cheap once the module is
+// loaded), so a device reset and a new context do not leave a stale address;
+// a call under capture uses the remembered one. Host code cannot pass the
+// array's name to a kernel directly -- on the host it denotes a host-side
+// stand-in, not the device memory.
+//
+// Kernel: the CUDA-core router with the K split that moe_route gives it, so
+// wherever moe_route runs that router (T <= 128, or shapes the tensor-core
+// router does not take) the two calls give bitwise the same indices and
+// weights. For T >= 129 on shapes the tensor-core router takes, moe_route
+// runs that one instead; its fp32 logits sum in another order, so the choice
+// agrees on every token whose k-th/(k+1)-th score gap is at least ~1e-5 and
+// the weights to ~2e-5 relative. The tensor-core router is not used here: it
+// reports a bounded wait that gave up through a status word, and this entry
+// point has no workspace to carry one back to the caller.
 //
 // Sharing: every call uses the same array, which keeps the last call's
 // contents. The counters are cleared at the start of every call; the logits
@@ -36,12 +49,15 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices];
 
-// Device address of g_route_scratch on the current device, looked up once.
-int scratch_address(void** out) {
+// Device address of g_route_scratch on the current device: looked up on every
+// call outside stream capture, remembered for calls under capture.
+int scratch_address(cudaStream_t s, void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone || g_scratch_addr[dev] == nullptr) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
             return MOE_ERR_CUDA;
@@ -62,19 +78,21 @@ extern "C" int moe_route_noalloc(const moe_config* cfg, const void* x, const voi
     if (moe_workspace_size(cfg) == 0) return MOE_ERR_UNSUPPORTED_SHAPE;  // shape and flag checks
     if (!x || !w_gate || !topk_idx || !topk_w || !aligned16(x) || !aligned16(w_gate))
         return MOE_ERR_INVALID_ARG;
+    // moe_route's K split of the CUDA-core router: the same partial sums in the
+    // same order (at most 16 slices; for T > 128 at E = 192 it is 1)
+    const int ksplit = moe::router_ksplit(*cfg);
     const size_t counter_bytes = moe::align256(sizeof(int32_t) * moe::n_router_groups(*cfg));
-    const size_t logit_bytes = sizeof(float) * (size_t)cfg->T * cfg->E;
+    const size_t logit_bytes = sizeof(float) * (size_t)ksplit * cfg->T * cfg->E;
     if (counter_bytes + logit_bytes > kScratchBytes) return MOE_ERR_UNSUPPORTED_SHAPE;
-    void* base = nullptr;
-    const int rc = scratch_address(&base);
-    if (rc != MOE_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void* base = nullptr;
+    const int rc = scratch_address(s, &base);
+    if (rc != MOE_OK) return rc;
     int32_t* counters = static_cast<int32_t*>(base);
     float* logits = reinterpret_cast<float*>(static_cast<char*>(base) + counter_bytes);
     if (cudaMemsetAsync(counters, 0, counter_bytes, s) != cudaSuccess) return MOE_ERR_CUDA;
     return moe::launch_router(*cfg, x, w_gate, gate_bias, nullptr, nullptr, 0.f, 0, topk_idx,
-                              topk_w, logits, nullptr, counters, 1, s) ==
-                   cudaSuccess
+                              topk_w, logits, nullptr, counters, ksplit, s) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }
