@@ -18,6 +18,12 @@ moe_forward3 with the input copied in from and the output copied back to
 pinned host memory every step. bf16 expert weights for the tensor-core kernels are
 packed once at load (moe_pack_weights), outside every timed region.
 
+The metric has two halves, % of the HBM roofline at decode and % of the dense
+bf16 tensor peak at prefill: the default line (``--config decode``) carries the
+prefill workload, measured in the same run the same way, as its ``prefill``
+object (``--no-prefill`` leaves it out). Tensor fractions divide by the burst
+bf16 peak (steps last milliseconds); the sustained peak is given beside it.
+
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (each
 step a bounded sample of the same workload), rank 0 only.
 """
@@ -53,14 +59,14 @@ WORKLOADS = {
 }
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of the dominant kernel, from
-# the captures summarised in profiles/, as bytes per unit of work so that a
-# smaller captured case scales to the benchmarked launch (traffic grows with
-# the touched experts at decode, with the routed rows at prefill). An entry is
-# removed when its kernel changes.
+# one capture of a smaller case of the same workload, as bytes per unit of work
+# so that it scales to the benchmarked launch (traffic grows with the touched
+# experts at decode, with the routed rows at prefill). An entry is removed when
+# its kernel changes.
 NCU_TRAFFIC = {
-    # profiles/grouped_gemm_pair_decode_E96_T32.md: 2.2437 GB for 89 touched experts
+    # bf16 pair gate_up, decode case E=96, T=32: 2.2437 GB for 89 touched experts
     ("decode", "gate_up_gemm"): {"per": "touched_expert", "bytes": 2.2437e9 / 89},
-    # profiles/grouped_gemm_pair_prefill_E96_T2048.md: 2.5880 GB for 16384 routed rows
+    # bf16 pair gate_up, prefill case E=96, T=2048: 2.5880 GB for 16384 routed rows
     ("prefill", "gate_up_gemm"): {"per": "row", "bytes": 2.5880e9 / 16384},
 }
 
@@ -217,54 +223,16 @@ def cpu_baseline(layer, shape, seconds: float):
             "sample": f"first {n} of the {shape.T} tokens of the same batch ({dt:.1f} s)"}
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=None)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="decode", choices=sorted(WORKLOADS))
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="auto", choices=["auto", "stream", "gemm"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--experts", type=int, default=None,
-                    help="override E (a smaller case of the same workload, e.g. for ncu)")
-    ap.add_argument("--tokens", type=int, default=None, help="override T")
-    ap.add_argument("--block", action="store_true",
-                    help="the complete Hy3 block: + a shared expert and an "
-                         "e_score_correction_bias (N(0, 0.05^2))")
-    args = ap.parse_args()
-    world, rank, local = dist_setup()
-    if args.steps is None:
-        args.steps = 10 if args.impl == "reference" else {"decode": 2000, "tiny": 2000}.get(
-            args.config, 200)
-    args.warmup = max(args.warmup, 3)
-
-    if args.impl == "reference":
-        run_reference(args, world, rank)
-        return
-
-    from sparse_moe_transformer_gemm_b200 import moe
-
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-        pg = dist
-
+def measure(args, name, dev, local, rank, world, pg, moe, block=False, cpu_seconds=None):
+    """Time one workload: the staged step (device time, CUDA events on the
+    launching stream) and the end-to-end moe_forward3 with host copies. Returns
+    the fields of one bench line (without the cpu baseline unless asked)."""
     import dataclasses
 
-    shape = CONFIGS[args.config]
+    shape = CONFIGS[name]
     if args.experts or args.tokens:
         shape = dataclasses.replace(shape, E=args.experts or shape.E, T=args.tokens or shape.T)
-    if args.block:
+    if block:
         shape = dataclasses.replace(shape, shared=True, score_bias_std=0.05)
     layer = make_layer(shape, seed=rank, device=dev)
     T, d, E, k, F = shape.T, shape.d, shape.E, shape.k, shape.F
@@ -367,33 +335,37 @@ def main():
     fp8, fp4 = shape.fp8, shape.fp4
     # the shared expert counts as one more touched expert with T more rows
     lw = work.layer_work(T, d, E, ks, F, touched, fp8, fp4)
-    gw = work.gate_up_work(rows, touched, d, F, fp8, fp4)
+    gw = work.gate_up_work(T, rows, touched, d, F, fp8, fp4)
     dw = work.down_work(rows, touched, d, F, fp8, fp4)
     dominant = max(("gate_up", "down"), key=lambda s: stage_ms[s])
     dom_work = gw if dominant == "gate_up" else dw
     dom_s = stage_ms[dominant] / 1e3
     use_stream = args.path == "stream" or fp4  # FP4 experts: the streaming kernels
     kernel_name = f"{dominant}_{'stream' if use_stream else 'gemm'}"
-    # The metric's roofline: HBM for the decode workload (weights streamed once),
-    # dense bf16 tensor peak for the larger batches. The tensor peak is the
-    # sustained one: the kernel is timed inside a seconds-long loop.
-    if args.config in ("decode", "tiny", "fp4_decode"):
+    # The metric's roofline: HBM for the decode workloads (weights streamed once),
+    # dense bf16 tensor peak for the larger batches. A step lasts milliseconds,
+    # so the tensor peak is the burst figure; the sustained one (a seconds-long
+    # loop under the power cap) is given beside it.
+    if name in ("decode", "tiny", "fp4_decode"):
         achieved = dom_work["bytes"] / dom_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
     else:
         achieved = dom_work["flops"] / dom_s / 1e12
-        pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        pk = peaks["bf16_tflops"]
+        sus = peaks.get("bf16_tflops_sustained")
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
-                "frac": achieved / pk, "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
-    roof["traffic"] = ncu_traffic(args.config, kernel_name, touched, rows,
-                                  shape == CONFIGS[args.config])
-    roof["traffic_source"] = "ncu capture of a smaller case, scaled (see profiles/)" \
+                "frac": achieved / pk,
+                "frac_of_sustained_peak": achieved / sus if sus else None}
+    roof["traffic"] = ncu_traffic(name, kernel_name, touched, rows, shape == CONFIGS[name])
+    roof["traffic_source"] = "ncu capture of a smaller case of the same kernel, scaled" \
         if roof["traffic"] is not None else None
     roof["kernel"] = kernel_name
-    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+    roof["peak_source"] = (f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'}"
+                           f"{', burst' if roof['bound'] == 'tensor' else ''})")
     roof["algorithmic_bytes_per_launch"] = dom_work["bytes"]
     roof["algorithmic_flops_per_launch"] = dom_work["flops"]
+    roof["implementation_bytes_per_launch"] = dom_work["implementation_bytes"]
 
     # End to end through moe_forward: every step copies its input from pinned host
     # memory and its output back to pinned host memory. The copies run on two
@@ -456,50 +428,119 @@ def main():
     e2e_same = bool(torch.equal(out_host[(e2e_steps - 1) % 2], out.cpu()))
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(layer, shape, args.cpu_seconds)
+    if cpu_seconds is not None and rank == 0 and world == 1:
+        cpu = cpu_baseline(layer, shape, cpu_seconds)
+
+    full = shape == CONFIGS[name]
+    res = {
+        "value": replica_value(T, world, ms), "ms_per_step": ms,
+        "dtype": "e4m3 weights, bf16 activations, fp32 accumulate" if fp8 else
+                 "e2m1 weights, bf16 activations, fp32 accumulate" if fp4 else
+                 "bf16 (fp32 accumulate, fp32 combine)",
+        "config": {"workload": (WORKLOADS[name] if full else
+                                f"{name} with the complete Hy3 block (+ a shared expert "
+                                "and an e_score_correction_bias)" if block and
+                                (T, E) == (CONFIGS[name].T, CONFIGS[name].E) else
+                                f"smaller case of {name}: T={T}, E={E}"),
+                   "T": T, "d": d, "E": E, "k": k,
+                   "d_ff": F, "path": args.path, "parallelism": f"replicas x{world}",
+                   "weights": ("e4m3 + fp32 row scales" if fp8 else
+                               "e2m1 + e8m0 block-32 scales" if fp4 else
+                               "bf16, packed in 128x64 blocks once at load (moe_pack_weights)"
+                               if packed else "bf16, row-major"),
+                   "l2": "no flush: each step streams the touched experts' weights "
+                         f"({touched} experts, "
+                         f"{touched * work.expert_bytes(d, F, fp8, fp4) / 1e9:.2f} GB) "
+                         "through the 126 MB L2"},
+        "roofline": roof,
+        "layer_roofline": {
+            "hbm_frac": lw["bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "tensor_frac": lw["flops"] / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "algorithmic_bytes": lw["bytes"], "algorithmic_flops": lw["flops"],
+            "touched_experts": touched},
+        "stage_ms": stage_ms,
+        "clocks": clocks.summary(),
+        "e2e": {"value": replica_value(T, world, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
+                "ms_per_step": e2e_ms, "api": "moe_forward3",
+                "copies": "one stream per direction, double-buffered, overlapping the compute",
+                "output_equals_staged": e2e_same},
+        "gpu_launches": sum(n_launch.values()) * args.steps,
+        "status": [moe.moe_status_string(status), moe.moe_status_string(status2)],
+        "cpu_baseline": cpu,
+    }
+    del layer, wgu, wd, ws, xp, h, y
+    torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "stream", "gemm"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="with --config decode, skip the prefill object of the line")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (a smaller case of the same workload, e.g. for ncu)")
+    ap.add_argument("--tokens", type=int, default=None, help="override T")
+    ap.add_argument("--block", action="store_true",
+                    help="the complete Hy3 block: + a shared expert and an "
+                         "e_score_correction_bias (N(0, 0.05^2))")
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    if args.steps is None:
+        args.steps = 10 if args.impl == "reference" else {"decode": 2000, "tiny": 2000}.get(
+            args.config, 200)
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    from sparse_moe_transformer_gemm_b200 import moe
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    head = measure(args, args.config, dev, local, rank, world, pg, moe, block=args.block,
+                   cpu_seconds=None if args.no_cpu_baseline else args.cpu_seconds)
+    # The metric has two halves: % of the HBM roofline at decode and % of the
+    # dense bf16 tensor peak at prefill. The decode line (the headline) carries
+    # the prefill workload measured in the same run, every rank taking part.
+    pre = None
+    if args.config == "decode" and not args.no_prefill and not (args.experts or args.tokens):
+        pre = measure(args, "prefill", dev, local, rank, world, pg, moe, block=args.block)
+        pre = {"metric": "MoE-layer tokens/s", "unit": "tokens/s", "steps": args.steps,
+               "warmup": args.warmup, **pre}
+        del pre["cpu_baseline"]
 
     if rank == 0:
         line = {
-            "metric": "MoE-layer tokens/s", "value": replica_value(T, world, ms), "unit": "tokens/s",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3 weights, bf16 activations, fp32 accumulate" if fp8 else
-                     "e2m1 weights, bf16 activations, fp32 accumulate" if fp4 else
-                     "bf16 (fp32 accumulate, fp32 combine)",
+            "metric": "MoE-layer tokens/s", "value": head["value"], "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": head["dtype"],
             "data": "synthetic (seeded; random-init weights of the Hy3 MoE layer shapes)",
-            "config": {"workload": (WORKLOADS[args.config] if shape == CONFIGS[args.config] else
-                                    f"{args.config} with the complete Hy3 block (+ a shared expert "
-                                    "and an e_score_correction_bias)" if args.block and
-                                    (T, E) == (CONFIGS[args.config].T, CONFIGS[args.config].E) else
-                                    f"smaller case of {args.config}: T={T}, E={E}"),
-                       "T": T, "d": d, "E": E, "k": k,
-                       "d_ff": F, "path": args.path, "parallelism": f"replicas x{world}",
-                       "weights": ("e4m3 + fp32 row scales" if fp8 else
-                                   "e2m1 + e8m0 block-32 scales" if fp4 else
-                                   "bf16, packed in 128x64 blocks once at load (moe_pack_weights)"
-                                   if packed else "bf16, row-major"),
-                       "l2": "no flush: each step streams the touched experts' weights "
-                             f"({touched} experts, "
-                             f"{touched * work.expert_bytes(d, F, fp8, fp4) / 1e9:.2f} GB) "
-                             "through the 126 MB L2"},
-            "roofline": roof,
-            "layer_roofline": {
-                "hbm_frac": lw["bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-                "tensor_frac": lw["flops"] / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
-                "algorithmic_bytes": lw["bytes"], "algorithmic_flops": lw["flops"],
-                "touched_experts": touched},
-            "stage_ms": stage_ms,
-            "clocks": clocks.summary(),
-            "e2e": {"value": replica_value(T, world, e2e_ms), "unit": "tokens/s",
-                    "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
-                    "ms_per_step": e2e_ms, "api": "moe_forward3",
-                    "copies": "one stream per direction, double-buffered, overlapping the compute",
-                    "output_equals_staged": e2e_same},
-            "gpu_launches": sum(n_launch.values()) * args.steps,
-            "status": [moe.moe_status_string(status), moe.moe_status_string(status2)],
-            "cpu_baseline": cpu,
         }
+        line.update({k: v for k, v in head.items() if k not in line})
+        if pre is not None:
+            line["prefill"] = pre
         print(json.dumps(line), flush=True)
     if pg:
         pg.barrier()

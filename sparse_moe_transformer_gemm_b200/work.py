@@ -9,6 +9,12 @@ kernels are tiled:
 * flops  = 2*T*d*E (router) + 6*T*k*d*F (gate, up and down projections of the
   k selected experts; 6*d*F per token per expert is the per-expert count of
   "Tencent Hy3-Flash QA", Q2.4).
+
+The expert steps alone: gate_up must read the touched experts' [2F, d]
+weights and the batch's tokens (T rows of x, once); down must read the
+touched experts' [d, F] weights. The intermediates between the steps (the
+permuted token rows, h [R, F], y [R, d]) and any re-read of a token row are
+implementation traffic, reported apart as ``implementation_bytes``.
 """
 
 from __future__ import annotations
@@ -41,15 +47,20 @@ def layer_work(T: int, d: int, E: int, k: int, F: int, touched: int, fp8: bool =
     return {"bytes": byts, "flops": flops}
 
 
-def gate_up_work(n_rows: int, touched: int, d: int, F: int, fp8: bool = False,
+def gate_up_work(T: int, n_rows: int, touched: int, d: int, F: int, fp8: bool = False,
                  fp4: bool = False) -> dict:
-    """The gate_up step alone: touched experts' [2F, d] weights, x rows in, h out."""
-    byts = touched * weight_bytes(2 * F, d, fp8, fp4) + n_rows * d * 2 + n_rows * F * 2
-    return {"bytes": byts, "flops": 4 * n_rows * d * F}
+    """The gate_up step alone: the touched experts' [2F, d] weights and the T
+    token rows of x (algorithmic); the n_rows grouped token rows beyond those T
+    and the h [n_rows, F] write (implementation)."""
+    return {"bytes": touched * weight_bytes(2 * F, d, fp8, fp4) + T * d * 2,
+            "flops": 4 * n_rows * d * F,
+            "implementation_bytes": (n_rows - T) * d * 2 + n_rows * F * 2}
 
 
 def down_work(n_rows: int, touched: int, d: int, F: int, fp8: bool = False,
               fp4: bool = False) -> dict:
-    """The down step alone: touched experts' [d, F] weights, h in, y out."""
-    byts = touched * weight_bytes(d, F, fp8, fp4) + n_rows * F * 2 + n_rows * d * 2
-    return {"bytes": byts, "flops": 2 * n_rows * d * F}
+    """The down step alone: the touched experts' [d, F] weights (algorithmic);
+    the h read and the y [n_rows, d] write (implementation)."""
+    return {"bytes": touched * weight_bytes(d, F, fp8, fp4),
+            "flops": 2 * n_rows * d * F,
+            "implementation_bytes": n_rows * F * 2 + n_rows * d * 2}

@@ -100,8 +100,17 @@ def test_work_accounting_matches_the_page_figures():
     assert work.expert_bytes(4096, 1536, fp8=True) == 3 * 4096 * 1536 + (2 * 1536 + 4096) * 4
     # FP4: half a byte per weight and one E8M0 byte per 32 weights of a row
     assert work.expert_bytes(4096, 1536, fp4=True) == 3 * 4096 * 1536 // 2 + 3 * 4096 * 1536 // 32
-    gw = work.gate_up_work(384, 150, 4096, 1536, fp4=True)
-    assert gw["bytes"] == 150 * (3072 * 4096 // 2 + 3072 * 128) + 384 * (4096 + 1536) * 2
+    gw = work.gate_up_work(64, 384, 150, 4096, 1536, fp4=True)
+    assert gw["bytes"] == 150 * (3072 * 4096 // 2 + 3072 * 128) + 64 * 4096 * 2
+    # the grouped rows beyond the T tokens and the h write are implementation traffic
+    assert gw["implementation_bytes"] == (384 - 64) * 4096 * 2 + 384 * 1536 * 2
+    dw = work.down_work(384, 150, 4096, 1536)
+    assert dw["bytes"] == 150 * 4096 * 1536 * 2
+    assert dw["implementation_bytes"] == 384 * (1536 + 4096) * 2
+    # the two steps' algorithmic bytes add up to the layer's, less the router and out
+    lw = work.layer_work(64, 4096, 192, 6, 1536, touched=150, fp4=True)
+    assert gw["bytes"] + work.down_work(384, 150, 4096, 1536, fp4=True)["bytes"] == \
+        lw["bytes"] - 192 * 4096 * 2 - 64 * 4096 * 2
     lw = work.layer_work(64, 4096, 192, 8, 1536, touched=175)
     assert lw["flops"] == 2 * 64 * 4096 * 192 + 6 * 64 * 8 * 4096 * 1536
     assert lw["bytes"] >= 175 * work.expert_bytes(4096, 1536)
