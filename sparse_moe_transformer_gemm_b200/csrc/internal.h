@@ -156,6 +156,9 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
                                       const void* w_down, const float* s_down, void* y,
                                       int* status, cudaStream_t s);
 
+cudaError_t launch_ep_row_experts(const int32_t* counts, int n_src, int e_local,
+                                  int32_t* expert_of_row, int n_rows, cudaStream_t s);
+
 cudaError_t launch_combine(const moe_config& c, const void* y, const int32_t* row_of,
                            const float* topk_w, void* out, cudaStream_t s);
 

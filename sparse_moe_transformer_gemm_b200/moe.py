@@ -42,9 +42,11 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permut
             "moe_permute_index", "moe_expert_gate_up", "moe_expert_gate_up_gather",
             "moe_expert_down", "moe_experts", "moe_combine", "moe_forward", "moe_read_status",
             "moe_status_string", "moe_route_noalloc", "moe_pack_weights", "moe_route2",
-            "moe_forward2", "moe_route3", "moe_forward3", "moe_selftest_bounded_wait")
+            "moe_forward2", "moe_route3", "moe_forward3", "moe_selftest_bounded_wait",
+            "moe_ep_row_experts")
 
 MOE_NOALLOC_SCRATCH_BYTES = 2 << 20
+MOE_EP_MAX_SEGMENTS = 8192
 # batches of at most this many token-slots (T*k) gather their token rows inside
 # the gate_up GEMM; larger ones write the permuted copy (moe_forward's rule)
 MOE_GATHER_MAX_SLOTS = 4096
@@ -117,6 +119,7 @@ def lib() -> ctypes.CDLL:
         "moe_route3": (I, [C, P, P, P, P, P, P, P, S, P]),
         "moe_forward3": (I, [C, P, P, P, P, P, P, P, P, P, P, S, P]),
         "moe_selftest_bounded_wait": (I, [P, ctypes.c_ulonglong, P]),
+        "moe_ep_row_experts": (I, [P, ctypes.c_int32, ctypes.c_int32, P, ctypes.c_int32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -294,6 +297,14 @@ def moe_selftest_bounded_wait(ws, limit_ns: int, stream=None) -> None:
     """Run the bounded-wait self-test; its MOE_ERR_TIMEOUT lands in ws's status word."""
     _check("moe_selftest_bounded_wait",
            lib().moe_selftest_bounded_wait(_p(ws), int(limit_ns), _s(stream)))
+
+
+def moe_ep_row_experts(counts, n_src: int, e_local: int, expert_of_row, stream=None) -> None:
+    """Local expert of every received row (expert parallelism): counts [n_src, e_local]
+    int32, expert_of_row [n_rows] int32, both on the device."""
+    _check("moe_ep_row_experts",
+           lib().moe_ep_row_experts(_p(counts), int(n_src), int(e_local), _p(expert_of_row),
+                                    int(expert_of_row.numel()), _s(stream)))
 
 
 def moe_read_status(ws, stream=None) -> int:

@@ -32,6 +32,8 @@ def test_header_constants_match_the_binding():
     text = open(os.path.join(ROOT, "include", "moe.h")).read()
     m = re.search(r"#define MOE_GATHER_MAX_SLOTS (\d+)", text)
     assert m and int(m.group(1)) == moe.MOE_GATHER_MAX_SLOTS
+    m = re.search(r"#define MOE_EP_MAX_SEGMENTS (\d+)", text)
+    assert m and int(m.group(1)) == moe.MOE_EP_MAX_SEGMENTS
     m = re.search(r"#define MOE_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
     assert m and int(m.group(1)) << int(m.group(2)) == moe.MOE_NOALLOC_SCRATCH_BYTES
     for name in ("MOE_FLAG_FP8_WEIGHTS", "MOE_FLAG_STREAM_PATH", "MOE_FLAG_GEMM_PATH",
@@ -233,3 +235,14 @@ def test_unsupported_shape_is_reported_by_every_entry_point(lib):
     }
     for fn, args in cases.items():
         assert _call(fn, ctypes.byref(cfg), *args) == moe.MOE_ERR_UNSUPPORTED_SHAPE, fn
+
+
+def test_ep_row_experts_rejects_bad_arguments_before_any_launch(lib):
+    P = ctypes.c_void_p
+    call = lambda c, n_src, el, out, n: _call("moe_ep_row_experts", c, n_src, el, out, n, None)  # noqa: E731
+    assert call(None, 2, 24, P(FAKE), 10) == moe.MOE_ERR_INVALID_ARG
+    assert call(P(FAKE), 2, 24, None, 10) == moe.MOE_ERR_INVALID_ARG
+    assert call(P(FAKE), 0, 24, P(FAKE), 10) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert call(P(FAKE), 2, 257, P(FAKE), 10) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert call(P(FAKE), 2, 24, P(FAKE), 0) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert call(P(FAKE), 33, 256, P(FAKE), 10) == moe.MOE_ERR_UNSUPPORTED_SHAPE  # 8448 segments
