@@ -80,6 +80,14 @@ __device__ __forceinline__ void e2m1x16_to_float(uint32_t w0, uint32_t w1, float
     }
 }
 
+// Two e4m3 codes placed as u = code1 << 24 | code0 << 8 (other bytes zero) ->
+// a bf16x2 whose halves are the codes' values times 2^-120: the seven
+// exponent+mantissa bits move to bf16 bits 4..10, the sign stays at bit 15
+// (the FP8 GEMM's widening multiplies by 2^120 afterwards).
+__host__ __device__ __forceinline__ uint32_t e4m3_pair_scaled_bits(uint32_t u) {
+    return ((u & 0x7F007F00u) >> 4) | (u & 0x80008000u);
+}
+
 // E8M0 scale byte b -> 2^(b - 127) (b = 0 gives the subnormal 2^-127; b = 255,
 // not a scale, gives infinity).
 __device__ __forceinline__ float e8m0_to_float(uint32_t b) {

@@ -490,41 +490,55 @@ constexpr int fp8_smem_bytes() {
 static_assert(fp8_smem_bytes<true>() <= 232448 && fp8_smem_bytes<false>() <= 232448,
               "fits in 227 KB");
 
-// Two e4m3 codes -> bf16x2, exactly: hardware e4m3x2 -> f16x2, each f16 ->
-// f32 (exact), then the high halves of the two f32 (a value with at most 4
-// significant bits has zero low halves, so keeping the high half is exact;
-// signed zeros carry over).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t q) {
-    uint32_t out;
-    asm("{\n\t.reg .b32 h2, f0, f1;\n\t.reg .b16 h0, h1;\n\t"
-        "cvt.rn.f16x2.e4m3x2 h2, %1;\n\t"
-        "mov.b32 {h0, h1}, h2;\n\t"
-        "cvt.f32.f16 f0, h0;\n\t"
-        "cvt.f32.f16 f1, h1;\n\t"
-        "prmt.b32 %0, f0, f1, 0x7632;\n\t}"
-        : "=r"(out)
-        : "h"(q));
-    return out;
+// Four e4m3 codes (one 32-bit word, code i in byte i) -> four bf16 in two
+// bf16x2 words (codes 0, 1 in lo; 2, 3 in hi; the even code in the low half),
+// exactly, on the integer and FMA pipes instead of the conversion pipe (whose
+// ~16 results per clock per SM bounded the converters): a byte permute puts
+// each code in the high byte of a 16-bit half, its seven exponent+mantissa
+// bits move down to bf16 bits 4..10 and its sign stays at bit 15. That bf16
+// reads as the code's value times 2^-120 (exponent field e = the code's, its
+// three mantissa bits on top of bf16's seven; a subnormal code, e = 0, is a
+// bf16 subnormal of the same scaled value), and one bf16x2 multiply by 2^120
+// (bf16 0x7B80: a power of two, exact, subnormal inputs included) restores
+// it. Signed zeros carry over. NaN codes (S.1111.111) give a finite value:
+// NaN weights are unspecified.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    constexpr uint32_t kTwoPow120 = 0x7B807B80u;  // bf16x2 (2^120, 2^120)
+    lo = mul_bf16x2(e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x1404)), kTwoPow120);
+    hi = mul_bf16x2(e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x3424)), kTwoPow120);
 }
 
 // Convert one raw e4m3 tile (128 rows x 64 bytes, row-major) into a bf16
 // operand tile (128 rows x 128 bytes, 128-byte swizzle) with CONV_THREADS threads;
 // thread `ct` handles 16-byte source chunks q = ct + CONV_THREADS i (row q/4,
-// elements 16(q%4)..16(q%4)+15).
+// elements 16(q%4)..16(q%4)+15). All of a thread's chunks are loaded before
+// any is widened, so that their shared-memory latencies overlap (the inline
+// loads and stores keep program order).
 template <int CONV_THREADS>
 __device__ __forceinline__ void widen_tile(uint32_t raw, uint32_t op, int ct) {
-    for (int q = ct; q < 512; q += CONV_THREADS) {
+    constexpr int PER = (512 + CONV_THREADS - 1) / CONV_THREADS;
+    uint32_t w[PER][4];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int q = ct + i * CONV_THREADS;
+        if (q < 512)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[i][0]), "=r"(w[i][1]), "=r"(w[i][2]), "=r"(w[i][3])
+                         : "r"(raw + q * 16));
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int q = ct + i * CONV_THREADS;
+        if (q >= 512) break;
         const int row = q >> 2, c = q & 3;
-        uint32_t w[4];
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                     : "r"(raw + q * 16));
         uint32_t b[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            b[2 * j] = e4m3x2_to_bf16x2((uint16_t)(w[j] & 0xFFFFu));
-            b[2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(w[j] >> 16));
-        }
+        for (int j = 0; j < 4; ++j) e4m3x4_to_bf16x4(w[i][j], b[2 * j], b[2 * j + 1]);
         const uint32_t rbase = op + row * 128;
         const int sw = row & 7;
         asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rbase + (((2 * c) ^ sw) << 4)),

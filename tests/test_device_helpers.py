@@ -13,6 +13,7 @@ import pytest
 import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+_E4M3 = {}  # the helper program's widening of all 256 codes (filled by the fixture)
 
 
 @pytest.fixture(scope="module")
@@ -32,10 +33,11 @@ def results(tmp_path_factory):
     bits = rng.integers(0, 2 ** 32, size=200_000, dtype=np.uint64).astype(np.uint32)
     f = np.concatenate([special, bits.view(np.float32), rng.normal(size=20_000).astype(np.float32)])
     f = f[~np.isnan(f)]
-    src, dst = str(d / "in.bin"), str(d / "out.bin")
+    src, dst, e8 = str(d / "in.bin"), str(d / "out.bin"), str(d / "e4m3.bin")
     f.view(np.uint32).tofile(src)
-    subprocess.run([exe, src, dst], check=True)
+    subprocess.run([exe, src, dst, e8], check=True)
     rec = np.fromfile(dst, dtype=np.uint32).reshape(-1, 5)
+    _E4M3["scaled"] = np.fromfile(e8, dtype=np.uint32)
     return f, rec
 
 
@@ -75,3 +77,21 @@ def test_bf16_pair_packing_round_trips(results):
     assert np.array_equal(lo.view(np.uint32), bf << 16)
     neg = np.isfinite(f)
     assert np.array_equal(hi[neg], -lo[neg])
+
+
+def test_scaled_e4m3_widening_is_exact_for_every_code(results):
+    """The FP8 GEMM widens e4m3 codes to bf16 with integer bit moves that give
+    value * 2^-120 (then one bf16 multiply by 2^120 on the GPU). Every non-NaN
+    code, normal, subnormal and both zeros, against the oracle's e4m3 decoding."""
+    r = _E4M3["scaled"]
+    codes = np.arange(256)
+    lo = (r & 0xFFFF).astype(np.uint16)
+    hi = (r >> 16).astype(np.uint16)
+    for half, code in ((lo, codes), (hi, 255 - codes)):
+        got = oracle.double_from_bf16(half) * 2.0 ** 120
+        want = oracle.double_from_e4m3(code.astype(np.uint8))
+        ok = ~np.isnan(want)
+        assert ok.sum() == 254
+        assert np.array_equal(got[ok], want[ok])
+        # signed zeros carry over
+        assert np.array_equal(np.signbit(got[ok]), np.signbit(want[ok]))
