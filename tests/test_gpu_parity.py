@@ -530,7 +530,8 @@ def test_fp8_weights_widen_exactly_for_every_code(path):
     y[r, i] = bf16(1.0 * value(W[e_r, i, f_r])) is each code's value itself
     (every e4m3 value is a bf16 value). The codes cover all 254 non-NaN e4m3
     patterns -- subnormals and both zeros included -- and each output is
-    compared bit for bit with the oracle's e4m3 decoding."""
+    compared with the oracle's e4m3 decoding: equal values (a -0 weight
+    gives +0, the sum of its -0 product and the other columns' +0 products)."""
     E, d, F, rows_e = 2, 256, 256, 128
     R = E * rows_e
     i = np.arange(d)[None, :, None]
@@ -551,6 +552,9 @@ def test_fp8_weights_widen_exactly_for_every_code(path):
     assert moe.moe_read_status(ws) == moe.MOE_OK
     e_of_row = np.arange(R) // rows_e
     want_codes = codes[e_of_row[:, None], np.arange(d)[None, :], f_of_row[:, None]]
-    want = oracle.bf16_from_double(oracle.double_from_e4m3(want_codes))
+    want = oracle.double_from_e4m3(want_codes)
     assert len(np.unique(want_codes)) == 254
-    assert np.array_equal(oracle.bf16_bits(y), want)
+    got = oracle.double_from_bf16(oracle.bf16_bits(y))
+    bad = np.nonzero(got != want)
+    assert bad[0].size == 0, (f"{bad[0].size} outputs differ, first code "
+                              f"{want_codes[bad][0]:#04x}: {got[bad][0]} vs {want[bad][0]}")

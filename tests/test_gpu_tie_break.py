@@ -43,7 +43,7 @@ def _router_weights():
     """W_gate of the Hy3 decode draw (seed 0) with rows 101..103 set equal to row 100."""
     wg = make_layer(CONFIGS["decode"], seed=0, device="cuda", with_experts=False)["w_gate"]
     wg = wg.clone()
-    wg[TIED[1:]] = wg[TIED[0]]
+    wg[TIED[1:]] = wg[TIED[0]].clone()
     return wg
 
 
