@@ -108,14 +108,21 @@ __device__ __forceinline__ TileInfo decode_tile(const CtrlT& c, int E, int m_til
     const int e = lo;
     const int local = t - c.tile_start[e];
     const int n_e = c.off[e + 1] - c.off[e];
+    // nt = ceil(n_e / NMAX) token tiles; all but the last hold 32q rows, so only
+    // the last one pads its MMA N to a multiple of 32 (near-equal tiles would pad
+    // every one: 341 rows as 171 + 170 run N = 192 + 192, as 192 + 149 run
+    // 192 + 160). q = ceil(ceil(n_e / 32) / nt), or NMAX / 32 if that left the
+    // last tile empty; every tile then holds 1..NMAX rows.
     const int nt = (n_e + NMAX - 1) / NMAX;
+    const int units = (n_e + 2 * NBOX - 1) / (2 * NBOX);
+    int q = (units + nt - 1) / nt;
+    if (2 * NBOX * q * (nt - 1) >= n_e) q = NMAX / (2 * NBOX);
     const int j = local / m_tiles;
-    const int base = n_e / nt, rem = n_e - base * nt;
     TileInfo ti;
     ti.e = e;
     ti.m = local - j * m_tiles;
-    ti.row0 = c.off[e] + j * base + min(j, rem);
-    ti.len = base + (j < rem ? 1 : 0);
+    ti.row0 = c.off[e] + j * 2 * NBOX * q;
+    ti.len = j < nt - 1 ? 2 * NBOX * q : n_e - 2 * NBOX * q * (nt - 1);
     ti.n = (ti.len + 2 * NBOX - 1) & ~(2 * NBOX - 1);
     return ti;
 }
@@ -469,11 +476,12 @@ struct Fp8Ctrl {
     uint64_t raw_empty[6];  // each CTA: every converter warp is done with the raw stage
     uint64_t b_full[4];     // even CTA: token bytes of both CTAs landed
     uint64_t b_empty[4];    // both CTAs: the pair MMAs finished reading the token stage
-    uint64_t op_full[6];    // even CTA: every converter warp of both CTAs filled the op stage
+    uint64_t op_full[6];    // even CTA: both CTAs' groups filled the op stage (see below)
     uint64_t op_empty[6];   // both CTAs: the pair MMAs finished reading the op stage
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
+    alignas(16) uint32_t sig[6][4];  // even CTA: landing slots of the odd CTA's ready signals
     uint32_t tmem_base;
     int abort;
     int total;
@@ -610,14 +618,14 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         if (lane == 0) {
             for (int s = 0; s < S::RAW_STAGES; ++s) {
                 tc::mbar_init(&c.raw_full[s], 1);
-                tc::mbar_init(&c.raw_empty[s], S::GROUP_WARPS);
+                tc::mbar_init(&c.raw_empty[s], 1);
             }
             for (int s = 0; s < S::B_STAGES; ++s) {
                 tc::mbar_init(&c.b_full[s], 1);
                 tc::mbar_init(&c.b_empty[s], 1);
             }
             for (int s = 0; s < S::OP_STAGES; ++s) {
-                tc::mbar_init(&c.op_full[s], 2 * S::GROUP_WARPS);
+                tc::mbar_init(&c.op_full[s], 1);
                 tc::mbar_init(&c.op_empty[s], 1);
             }
             for (int a = 0; a < S::ACC_STAGES; ++a) {
@@ -714,9 +722,16 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         }
     } else if (warp >= 6 && warp < 6 + CONV_WARPS) {
         // ---------------- converters: raw e4m3 -> bf16 operand (A) in the op stage.
-        // Each warp arrives on the even CTA's op_full on its own (after its
-        // writes are fenced to the async proxy); a warp whose bounded wait
-        // gave up stops, and the MMA's bounded wait on op_full then gives up.
+        // A group's threads fence their writes to the async proxy and meet at a
+        // named barrier; then one thread releases the raw stage and signals the
+        // even CTA's op_full: in the even CTA a local arrive that expects 16
+        // bytes, in the odd CTA a 16-byte bulk copy into the even CTA's shared
+        // memory that completes on that barrier (an async-proxy operation issued
+        // after the fenced writes). A remote mbarrier arrive with cluster-scope
+        // release, the other way to signal across the pair, stalled its warp
+        // ~1.5k cycles per K block on B200 -- longer than the widening itself.
+        // The group agrees on its bounded waits (bar.red.or) and leaves
+        // together; the MMA's bounded wait on op_full then gives up.
         const int group = (warp - 6) / S::GROUP_WARPS;
         const int ct = threadIdx.x - 192 - group * S::CONV_THREADS;  // 0..CONV_THREADS-1
         const uint32_t raw0 = tc::smem_u32(raw_ring), op0 = tc::smem_u32(op_ring);
@@ -729,8 +744,9 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
             const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
             const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
-            if (!tc::mbar_wait(&c.raw_full[rs], rph, abort_flag) ||
-                !tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag)) {
+            const bool ok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag) &&
+                            tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
+            if (tc::bar_any(2 + group, S::CONV_THREADS, !ok)) {  // the group leaves together
                 raise_timeout(c, status);
                 break;
             }
@@ -739,10 +755,15 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             widen_tile<S::CONV_THREADS>(raw, op, ct);
             if (GATE_UP) widen_tile<S::CONV_THREADS>(raw + RAW_BYTES, op + A_BYTES, ct);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) {
+            tc::bar_sync(2 + group, S::CONV_THREADS);
+            if (ct == 0) {
                 tc::mbar_arrive(&c.raw_empty[rs]);
-                tc::mbar_arrive_cluster(tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
+                if (leader)
+                    tc::mbar_arrive_expect_tx(&c.op_full[os], 16);
+                else
+                    tc::bulk_copy_to_cluster(tc::map_to_cta(tc::smem_u32(&c.sig[os][0]), 0),
+                                             scales, 16,
+                                             tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
             }
         }
     } else if (warp == 1) {

@@ -180,6 +180,18 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                  : "memory");
 }
 
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
+// global memory into the shared memory of a CTA of the cluster, completing on an
+// mbarrier of that CTA (dst_cluster and bar_cluster from map_to_cta). Not
+// multicast.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, const void* gsrc,
+                                                     uint32_t bytes, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst_cluster), "l"(gsrc), "r"(bytes), "r"(bar_cluster)
+        : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {

@@ -155,18 +155,21 @@ def sample_tokens(T: int, n: int = 48, seed: int = 0) -> np.ndarray:
     return np.unique(np.concatenate([np.arange(8), mid, np.arange(T - 8, T)])).astype(np.int32)
 
 
-def gemm_tiles(counts, nmax: int = 256):
-    """The token tiles of the grouped GEMMs: expert e's n_e grouped rows split
-    into ceil(n_e / nmax) parts of near-equal length (the first n_e mod parts
-    one row longer). Yields (e, first row, length) with rows counted from the
-    expert's first grouped row."""
+def gemm_tiles(counts, nmax: int = 256, unit: int = 32):
+    """The token tiles of the SM-pair grouped GEMMs: expert e's n_e grouped rows
+    split into nt = ceil(n_e / nmax) tiles, all but the last of unit*q rows
+    (q = ceil(ceil(n_e / unit) / nt), or nmax / unit if that left the last tile
+    empty). Yields (e, first row, length) with rows counted from the expert's
+    first grouped row."""
     for e, n in enumerate(np.asarray(counts).tolist()):
         if n == 0:
             continue
         nt = (n + nmax - 1) // nmax
-        base, rem = divmod(n, nt)
+        q = (-(-n // unit) + nt - 1) // nt
+        if unit * q * (nt - 1) >= n:
+            q = nmax // unit
         for j in range(nt):
-            yield e, j * base + min(j, rem), base + (1 if j < rem else 0)
+            yield e, j * unit * q, unit * q if j < nt - 1 else n - unit * q * (nt - 1)
 
 
 def tile_cover_tokens(idx: np.ndarray, E: int, edge: int = 32, nmax: int = 256) -> np.ndarray:
