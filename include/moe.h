@@ -35,9 +35,12 @@
  *   s_gate_up [E, 2*d_ff, d/32] / s_down [E, d, d_ff/32] hold one E8M0 byte b
  *   per 32 consecutive columns of a row, the block's scale 2^(b - 127)
  *   (b = 255 is not a scale: unspecified output). The weight value is
- *   code value * block scale. The experts run on the weight-streaming kernels
- *   (MOE_FLAG_GEMM_PATH, MOE_FLAG_FP8_WEIGHTS, MOE_FLAG_PACKED_WEIGHTS or
- *   MOE_FLAG_SHARED_EXPERT with it: MOE_ERR_INVALID_ARG).
+ *   code value * block scale. With neither path flag the experts run on the
+ *   weight-streaming kernels at up to 4 mean rows per expert (T*k <= 4*E, the
+ *   decode regime) and on the tensor-core SM-pair kernels above that (d, d_ff
+ *   multiples of 256; the streaming kernels otherwise). MOE_FLAG_FP8_WEIGHTS,
+ *   MOE_FLAG_PACKED_WEIGHTS or MOE_FLAG_SHARED_EXPERT with it:
+ *   MOE_ERR_INVALID_ARG.
  * - Packed bf16 weights (MOE_FLAG_PACKED_WEIGHTS): w_gate_up and w_down hold
  *   the same values rearranged by moe_pack_weights into 16 KB blocks of 128
  *   rows x 64 columns (block (e, rb, kb) = rows [128 rb, 128 rb + 128) and

@@ -88,6 +88,19 @@ __host__ __device__ __forceinline__ uint32_t e4m3_pair_scaled_bits(uint32_t u) {
     return ((u & 0x7F007F00u) >> 4) | (u & 0x80008000u);
 }
 
+// One byte of two E2M1 codes (the even code in the low nibble) -> a bf16x2
+// whose halves (the even code low) are the codes' values times 2^-126: the
+// byte is copied into both 16-bit halves (times 0x1001: the low nibble at bits
+// 0..3, the high one at 16..19), the three exponent+mantissa bits move to
+// bf16 bits 6..8 and the sign to bit 15 (adding sign * 4032 turns the sign's
+// copy at bit 9 into bit 15). An E2M1 value 2^(e-1) (1 + m/2) then reads as
+// 2^(e-127) (1 + m/2), and the subnormal 0.5 as the bf16 subnormal 2^-127
+// (the FP4 GEMM's widening multiplies by the block scale times 2^126).
+__host__ __device__ __forceinline__ uint32_t e2m1_pair_scaled_bits(uint32_t byte) {
+    const uint32_t t = (byte * 0x1001u) & 0x000F000Fu;
+    return (t << 6) + (t & 0x00080008u) * 4032u;
+}
+
 // E8M0 scale byte b -> 2^(b - 127) (b = 0 gives the subnormal 2^-127; b = 255,
 // not a scale, gives infinity).
 __device__ __forceinline__ float e8m0_to_float(uint32_t b) {

@@ -117,10 +117,13 @@ __device__ __forceinline__ TileInfo decode_tile(const CtrlT& c, int E, int m_til
     const int units = (n_e + 2 * NBOX - 1) / (2 * NBOX);
     int q = (units + nt - 1) / nt;
     if (2 * NBOX * q * (nt - 1) >= n_e) q = NMAX / (2 * NBOX);
-    const int j = local / m_tiles;
+    // token tiles fastest: the tiles that read the same weight rows (same m,
+    // next j) get neighbouring indices, so concurrent SM pairs stream those
+    // weights from HBM once and from L2 for the others
+    const int j = local % nt;
     TileInfo ti;
     ti.e = e;
-    ti.m = local - j * m_tiles;
+    ti.m = local / nt;
     ti.row0 = c.off[e] + j * 2 * NBOX * q;
     ti.len = j < nt - 1 ? 2 * NBOX * q : n_e - 2 * NBOX * q * (nt - 1);
     ti.n = (ti.len + 2 * NBOX - 1) & ~(2 * NBOX - 1);
@@ -440,10 +443,18 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 constexpr int THREADS_FP8 = 512;        // warps 6-14 converters, warp 15 token producer
 constexpr int RAW_BYTES = BM * BK;      // one 128 x 64 e4m3 tile
 
-template <bool GATE_UP>
+// FP4: E2M1 codes and E8M0 block scales folded into the widening (no row scale
+// in the epilogue). A raw tile is still 128 rows x 64 bytes, which holds 128
+// codes a row: two K blocks (KPR) per raw stage, so FP4 keeps FP8's TMA box and
+// ring depths while its weight stream has the same bytes in flight. (Raw
+// rings of 8 / 12 stages of one-K-block FP4 tiles stalled or faulted on B200,
+// cause not identified; that form is not used.)
+template <bool GATE_UP, bool FP4 = false>
 struct Fp8Shape {
     static constexpr int A_TILES = GATE_UP ? 2 : 1;
-    static constexpr int RAW_STAGE = A_TILES * RAW_BYTES;          // 16 KB / 8 KB
+    static constexpr int KPR = FP4 ? 2 : 1;                        // K blocks per raw stage
+    static constexpr int RAW_TILE = RAW_BYTES;                     // 128 rows x 64 bytes
+    static constexpr int RAW_STAGE = A_TILES * RAW_TILE;           // 16 KB / 8 KB
     static constexpr int OP_STAGE = A_TILES * A_BYTES;             // 32 KB / 16 KB
     static constexpr int RAW_STAGES = GATE_UP ? 4 : 6;  // multiples of GROUPS
     static constexpr int B_STAGES = GATE_UP ? 3 : 4;
@@ -460,15 +471,17 @@ struct Fp8Shape {
 
 constexpr int CONV_WARPS = 9;                          // warps 6..14 (some idle for gate_up)
 constexpr int TOKEN_WARP = 6 + CONV_WARPS;
-template <bool G>
+template <bool G, bool FP4>
 constexpr bool groups_ok() {
-    using S = Fp8Shape<G>;
-    return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES >= S::GROUPS &&
+    using S = Fp8Shape<G, FP4>;
+    return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES >= S::KPR * S::GROUPS - 1 &&
            S::GROUPS * S::GROUP_WARPS <= CONV_WARPS;
 }
 // Each group owns whole raw stages, and a group's previous operand wait proves
 // that the stage's last reader finished (parity waits cannot see a stale phase).
-static_assert(groups_ok<true>() && groups_ok<false>(), "converter grouping");
+static_assert(groups_ok<true, false>() && groups_ok<false, false>() && groups_ok<true, true>() &&
+                  groups_ok<false, true>(),
+              "converter grouping");
 static_assert(THREADS_FP8 == 32 * (TOKEN_WARP + 1), "warp roles cover the block");
 
 struct Fp8Ctrl {
@@ -491,11 +504,12 @@ struct Fp8Ctrl {
 
 constexpr int FP8_EPI_BYTES = EPI_N * BM * 2;  // one [32 tokens][128 rows] bf16 staging tile
 
-template <bool GATE_UP>
+template <bool GATE_UP, bool FP4>
 constexpr int fp8_smem_bytes() {
-    return Fp8Shape<GATE_UP>::RING_BYTES + FP8_EPI_BYTES + 1024 + (int)sizeof(Fp8Ctrl);
+    return Fp8Shape<GATE_UP, FP4>::RING_BYTES + FP8_EPI_BYTES + 1024 + (int)sizeof(Fp8Ctrl);
 }
-static_assert(fp8_smem_bytes<true>() <= 232448 && fp8_smem_bytes<false>() <= 232448,
+static_assert(fp8_smem_bytes<true, false>() <= 232448 && fp8_smem_bytes<false, false>() <= 232448 &&
+                  fp8_smem_bytes<true, true>() <= 232448 && fp8_smem_bytes<false, true>() <= 232448,
               "fits in 227 KB");
 
 // Four e4m3 codes (one 32-bit word, code i in byte i) -> four bf16 in two
@@ -559,17 +573,81 @@ __device__ __forceinline__ void widen_tile(uint32_t raw, uint32_t op, int ct) {
     }
 }
 
-// tmA: e4m3 weights [E * a_rows_per_expert, K] bytes, box 64 x 128 (no swizzle).
-// tmB: token rows [R, K] bf16, box 64 x 16. scales: [E * a_rows_per_expert] fp32.
-template <bool GATE_UP>
+// Convert one K block of a raw E2M1 tile (128 rows x 64 bytes, row-major, two K
+// blocks a row: K block `sub` in bytes 32 sub..32 sub + 31; code 2i of a row in
+// the low nibble of its byte i) into a bf16 operand tile (128 rows x 128
+// bytes, 128-byte swizzle). Thread `ct` handles 16-byte chunks q = ct +
+// CONV_THREADS i: row q/2, codes 32(q%2)..32(q%2)+31 of the K block, exactly
+// one E8M0 scale block, whose byte b is sc[i]. Each byte of codes becomes a bf16 pair worth
+// value * 2^-126 (e2m1_pair_scaled_bits); one bf16x2 multiply by 2^(b-1) -- a
+// normal bf16 for b <= 128 -- gives value * 2^(b-127) exactly; for b > 128 it
+// is two multiplies, by 2^126 and by 2^(b-127). Products of magnitude >=
+// 2^128 (b >= 253) overflow, as the value itself does in bf16.
+template <int CONV_THREADS>
+constexpr int fp4_per() {
+    return (256 + CONV_THREADS - 1) / CONV_THREADS;
+}
+template <int CONV_THREADS>
+__device__ __forceinline__ void widen_tile_fp4(uint32_t raw, uint32_t op, int ct, int sub,
+                                               const uint32_t (&sc)[fp4_per<CONV_THREADS>()]) {
+    constexpr int PER = fp4_per<CONV_THREADS>();
+    uint32_t w[PER][4];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int q = ct + i * CONV_THREADS;
+        if (q < 256)  // raw rows hold two K blocks (64 bytes): this one at 32 * sub
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[i][0]), "=r"(w[i][1]), "=r"(w[i][2]), "=r"(w[i][3])
+                         : "r"(raw + (q >> 1) * 64 + sub * 32 + (q & 1) * 16));
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int q = ct + i * CONV_THREADS;
+        if (q >= 256) break;
+        const int row = q >> 1, half = q & 1;
+        const uint32_t b = sc[i];
+        const bool one = b <= 128u;
+        const uint32_t f1 = one ? ((b + 126u) << 7) : 0x7E80u;  // 2^(b-1) or 2^126
+        const uint32_t f1x2 = f1 | (f1 << 16);
+        const uint32_t f2x2 = (b << 7) | (b << 23);                // 2^(b-127), used if b > 128
+        uint32_t o[16];
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t v = e2m1_pair_scaled_bits(__byte_perm(w[i][j4], 0u, 0x4440u | j));
+                v = mul_bf16x2(v, f1x2);
+                if (!one) v = mul_bf16x2(v, f2x2);
+                o[4 * j4 + j] = v;
+            }
+        }
+        const uint32_t rbase = op + row * 128;
+        const int sw = row & 7;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             rbase + (((4 * half + k) ^ sw) << 4)),
+                         "r"(o[4 * k]), "r"(o[4 * k + 1]), "r"(o[4 * k + 2]), "r"(o[4 * k + 3])
+                         : "memory");
+    }
+}
+
+// tmA: e4m3 weights [E * a_rows_per_expert, K] bytes, box 64 x 128 (no swizzle);
+// FP4: E2M1 codes [E * a_rows_per_expert, K / 2] bytes, box 64 x 128 (two K blocks).
+// tmB: token rows [R, K] bf16, box 64 x 16. scales_v: FP8 fp32 row scales
+// [E * a_rows_per_expert]; FP4 E8M0 block scales [E * a_rows_per_expert, K / 32]
+// bytes.
+template <bool GATE_UP, bool FP4>
 __global__ void __launch_bounds__(THREADS_FP8, 1)
 grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ TokenMaps tmB,
-                             const int* __restrict__ offsets, const float* __restrict__ scales,
+                             const int* __restrict__ offsets, const void* __restrict__ scales_v,
                              int E, int K, int a_rows_per_expert, int m_tiles,
                              __nv_bfloat16* __restrict__ out, int out_ld,
                              int* __restrict__ status) {
-    using S = Fp8Shape<GATE_UP>;
+    using S = Fp8Shape<GATE_UP, FP4>;
+    const float* __restrict__ scales = static_cast<const float*>(scales_v);
+    const uint8_t* __restrict__ scales8 = static_cast<const uint8_t*>(scales_v);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -658,7 +736,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int t = pair; t < total && ok; t += n_pairs) {
                 const TileInfo ti = decode_tile(c, E, m_tiles, t);
                 const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kr = 0; kr < KB / S::KPR; ++kr) {  // raw blocks of KPR K blocks
                     if (!tc::mbar_wait(&c.raw_empty[stage], phase ^ 1u, abort_flag)) {
                         raise_timeout(c, status);
                         ok = false;
@@ -666,9 +744,10 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     uint8_t* st = raw_ring + stage * S::RAW_STAGE;
                     tc::mbar_arrive_expect_tx(&c.raw_full[stage], S::RAW_STAGE);
-                    tc::tma_load_2d_hint(st, &tmA, &c.raw_full[stage], kb * BK, a_row, pol_w);
+                    const int kx = kr * BK;  // byte column: 64 e4m3 codes or 128 E2M1 codes
+                    tc::tma_load_2d_hint(st, &tmA, &c.raw_full[stage], kx, a_row, pol_w);
                     if (GATE_UP)
-                        tc::tma_load_2d_hint(st + RAW_BYTES, &tmA, &c.raw_full[stage], kb * BK,
+                        tc::tma_load_2d_hint(st + S::RAW_TILE, &tmA, &c.raw_full[stage], kx,
                                              a_row + a_rows_per_expert / 2, pol_w);
                     issued[stage] = true;
                     parity[stage] = phase;
@@ -735,35 +814,99 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         const int group = (warp - 6) / S::GROUP_WARPS;
         const int ct = threadIdx.x - 192 - group * S::CONV_THREADS;  // 0..CONV_THREADS-1
         const uint32_t raw0 = tc::smem_u32(raw_ring), op0 = tc::smem_u32(op_ring);
-        // this CTA's K blocks in order: j = tile_iteration * KB + kb; a group
-        // converts j = group, group + GROUPS, ... (warps past the groups idle)
+        // this CTA's K blocks in order: j = tile_iteration * KB + kb
         int n_my_tiles = 0;
         for (int t = pair; t < total; t += n_pairs) ++n_my_tiles;
-        const long n_blocks = (long)n_my_tiles * KB;
-        for (long jb = (group < S::GROUPS ? group : n_blocks); jb < n_blocks; jb += S::GROUPS) {
-            const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
-            const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
-            const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
-            const bool ok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag) &&
-                            tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
-            if (tc::bar_any(2 + group, S::CONV_THREADS, !ok)) {  // the group leaves together
-                raise_timeout(c, status);
-                break;
+        // signal one op stage (see above); ct == 0 of the group, after its barrier
+        auto signal_op = [&](int os) {
+            if (leader)
+                tc::mbar_arrive_expect_tx(&c.op_full[os], 16);
+            else
+                tc::bulk_copy_to_cluster(tc::map_to_cta(tc::smem_u32(&c.sig[os][0]), 0), scales_v,
+                                         16, tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
+        };
+        if constexpr (FP4) {
+            // A group takes raw blocks jr = group, group + GROUPS, ... and turns each
+            // into the op blocks 2 jr and 2 jr + 1. The op wait for block b stays
+            // unambiguous: the group's previous op wait (block b - 1, or
+            // b - 2 GROUPS + 1) saw the MMA finish block b - 2 GROUPS + 1 - OP_STAGES
+            // >= b - 2 OP_STAGES (OP_STAGES >= 2 GROUPS - 1), so stage b % OP_STAGES
+            // has completed b / OP_STAGES - 1 or b / OP_STAGES phases, never fewer.
+            constexpr int PER4 = fp4_per<S::CONV_THREADS>();
+            const long n_raw = (long)n_my_tiles * (KB / 2);
+            for (long jr = (group < S::GROUPS ? group : n_raw); jr < n_raw; jr += S::GROUPS) {
+                const int rs = (int)(jr % S::RAW_STAGES);
+                const uint32_t rph = (uint32_t)(jr / S::RAW_STAGES) & 1u;
+                const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
+                if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
+                    raise_timeout(c, status);
+                    break;
+                }
+                const uint32_t raw = raw0 + rs * S::RAW_STAGE;
+                bool failed = false;
+                for (int sub = 0; sub < 2; ++sub) {
+                    const long jb = 2 * jr + sub;
+                    const int os = (int)(jb % S::OP_STAGES);
+                    const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
+                    // this thread's block scales, loaded before the op wait
+                    uint32_t sc[S::A_TILES][PER4];
+                    const long it = jb / KB;
+                    const int kb = (int)(jb - it * KB);
+                    const TileInfo ti = decode_tile(c, E, m_tiles, pair + (int)it * n_pairs);
+                    const long a_row = (long)ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
+                    const long blocks = K / 32;
+#pragma unroll
+                    for (int a = 0; a < S::A_TILES; ++a)
+#pragma unroll
+                        for (int i = 0; i < PER4; ++i) {
+                            const int q = ct + i * S::CONV_THREADS;
+                            const long row = a_row + a * (a_rows_per_expert / 2) + (q >> 1);
+                            sc[a][i] = q < 256 ? __ldg(scales8 + row * blocks + 2 * kb + (q & 1)) : 0u;
+                        }
+                    const bool ook = tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
+                    if (tc::bar_any(2 + group, S::CONV_THREADS, !ook)) {
+                        raise_timeout(c, status);
+                        failed = true;
+                        break;
+                    }
+                    const uint32_t op = op0 + os * S::OP_STAGE;
+                    widen_tile_fp4<S::CONV_THREADS>(raw, op, ct, sub, sc[0]);
+                    if (GATE_UP)
+                        widen_tile_fp4<S::CONV_THREADS>(raw + S::RAW_TILE, op + A_BYTES, ct, sub,
+                                                        sc[S::A_TILES - 1]);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    tc::bar_sync(2 + group, S::CONV_THREADS);
+                    if (ct == 0) {
+                        if (sub == 1) tc::mbar_arrive(&c.raw_empty[rs]);  // both K blocks read
+                        signal_op(os);
+                    }
+                }
+                if (failed) break;
             }
-            const uint32_t raw = raw0 + rs * S::RAW_STAGE;
-            const uint32_t op = op0 + os * S::OP_STAGE;
-            widen_tile<S::CONV_THREADS>(raw, op, ct);
-            if (GATE_UP) widen_tile<S::CONV_THREADS>(raw + RAW_BYTES, op + A_BYTES, ct);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            tc::bar_sync(2 + group, S::CONV_THREADS);
-            if (ct == 0) {
-                tc::mbar_arrive(&c.raw_empty[rs]);
-                if (leader)
-                    tc::mbar_arrive_expect_tx(&c.op_full[os], 16);
-                else
-                    tc::bulk_copy_to_cluster(tc::map_to_cta(tc::smem_u32(&c.sig[os][0]), 0),
-                                             scales, 16,
-                                             tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
+        } else {
+            // a group converts the K blocks j = group, group + GROUPS, ... (warps
+            // past the groups idle)
+            const long n_blocks = (long)n_my_tiles * KB;
+            for (long jb = (group < S::GROUPS ? group : n_blocks); jb < n_blocks; jb += S::GROUPS) {
+                const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
+                const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
+                const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
+                const bool ok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag) &&
+                                tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
+                if (tc::bar_any(2 + group, S::CONV_THREADS, !ok)) {  // the group leaves together
+                    raise_timeout(c, status);
+                    break;
+                }
+                const uint32_t raw = raw0 + rs * S::RAW_STAGE;
+                const uint32_t op = op0 + os * S::OP_STAGE;
+                widen_tile<S::CONV_THREADS>(raw, op, ct);
+                if (GATE_UP) widen_tile<S::CONV_THREADS>(raw + S::RAW_TILE, op + A_BYTES, ct);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tc::bar_sync(2 + group, S::CONV_THREADS);
+                if (ct == 0) {
+                    tc::mbar_arrive(&c.raw_empty[rs]);
+                    signal_op(os);
+                }
             }
         }
     } else if (warp == 1) {
@@ -846,8 +989,10 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
             const int col0 = ti.m * 2 * BM + rank * BM;
             const long srow = (long)ti.e * a_rows_per_expert + col0 + row_in_tile;
-            const float sa = __ldg(scales + srow);
-            const float sb = GATE_UP ? __ldg(scales + srow + a_rows_per_expert / 2) : 0.f;
+            // FP8: the row scales multiply the finished dot products; FP4 folded
+            // its block scales into the widening
+            const float sa = FP4 ? 1.f : __ldg(scales + srow);
+            const float sb = FP4 ? 1.f : GATE_UP ? __ldg(scales + srow + a_rows_per_expert / 2) : 0.f;
             for (int c0 = 0; c0 < ti.n; c0 += EPI_N) {
                 uint32_t g[32];
                 tc::tmem_ld32(tbase + c0, g);
@@ -922,14 +1067,15 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-major [rows, cols] e4m3 codes (bytes), box of box_rows x 64 bytes, no swizzle.
+// Row-major [rows, cols] bytes (e4m3 codes, or E2M1 code pairs), box of
+// box_rows x box_cols bytes, no swizzle.
 bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                 uint32_t box_rows) {
+                 uint32_t box_rows, uint32_t box_cols = BK) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols};
-    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -986,12 +1132,12 @@ cudaError_t launch(const CUtensorMap& a, const TokenMaps& b, const int32_t* offs
     return cudaGetLastError();
 }
 
-template <bool GATE_UP>
+template <bool GATE_UP, bool FP4 = false>
 cudaError_t launch_fp8(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets,
-                       const float* scales, int E, int K, int a_rows_per_expert, int m_tiles,
+                       const void* scales, int E, int K, int a_rows_per_expert, int m_tiles,
                        void* out, int out_ld, int* status, cudaStream_t s) {
-    const int smem = fp8_smem_bytes<GATE_UP>();
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_fp8_kernel<GATE_UP>,
+    const int smem = fp8_smem_bytes<GATE_UP, FP4>();
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_fp8_kernel<GATE_UP, FP4>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -1006,7 +1152,7 @@ cudaError_t launch_fp8(const CUtensorMap& a, const TokenMaps& b, const int32_t* 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_fp8_kernel<GATE_UP>, a, b, offsets, scales, E,
+    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_fp8_kernel<GATE_UP, FP4>, a, b, offsets, scales, E,
                              K, a_rows_per_expert, m_tiles, static_cast<__nv_bfloat16*>(out),
                              out_ld, status);
     if (err != cudaSuccess) return err;
@@ -1042,6 +1188,33 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
         return cudaErrorInvalidValue;
     return launch_fp8<false>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d,
                              status, s);
+}
+
+cudaError_t launch_gate_up_gemm_pair_fp4(const moe_config& c, const void* x_perm,
+                                         const int32_t* offsets, const void* w_gate_up,
+                                         const void* s_gate_up, void* h, int* status,
+                                         cudaStream_t s) {
+    CUtensorMap a;
+    TokenMaps b;
+    const uint64_t R = (uint64_t)c.T * c.k;
+    if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d / 2, BM) ||
+        !make_token_maps(&b, x_perm, R, c.d))
+        return cudaErrorInvalidValue;
+    return launch_fp8<true, true>(a, b, offsets, s_gate_up, c.E, c.d, 2 * c.d_ff,
+                                  c.d_ff / (2 * BM), h, c.d_ff, status, s);
+}
+
+cudaError_t launch_down_gemm_pair_fp4(const moe_config& c, const void* h, const int32_t* offsets,
+                                      const void* w_down, const void* s_down, void* y,
+                                      int* status, cudaStream_t s) {
+    CUtensorMap a;
+    TokenMaps b;
+    const uint64_t R = (uint64_t)c.T * c.k;
+    if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff / 2, BM) ||
+        !make_token_maps(&b, h, R, c.d_ff))
+        return cudaErrorInvalidValue;
+    return launch_fp8<false, true>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y,
+                                   c.d, status, s);
 }
 
 cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,

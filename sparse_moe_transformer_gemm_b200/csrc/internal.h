@@ -159,6 +159,15 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
 cudaError_t launch_ep_row_experts(const int32_t* counts, int n_src, int e_local,
                                   int32_t* expert_of_row, int n_rows, cudaStream_t s);
 
+// FP4 (E2M1 codes + E8M0 block-32 scales) on the same SM-pair kernels.
+cudaError_t launch_gate_up_gemm_pair_fp4(const moe_config& c, const void* x_perm,
+                                         const int32_t* offsets, const void* w_gate_up,
+                                         const void* s_gate_up, void* h, int* status,
+                                         cudaStream_t s);
+cudaError_t launch_down_gemm_pair_fp4(const moe_config& c, const void* h, const int32_t* offsets,
+                                      const void* w_down, const void* s_down, void* y,
+                                      int* status, cudaStream_t s);
+
 cudaError_t launch_combine(const moe_config& c, const void* y, const int32_t* row_of,
                            const float* topk_w, void* out, cudaStream_t s);
 

@@ -22,10 +22,9 @@ int check_cfg(const moe_config* c) {
     if ((c->flags & MOE_FLAG_PACKED_WEIGHTS) &&
         (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_STREAM_PATH)))
         return MOE_ERR_INVALID_ARG;
-    // FP4 experts: the weight-streaming kernels only, routed experts only
+    // FP4 experts: routed experts only, in their own code layout
     if ((c->flags & MOE_FLAG_FP4_WEIGHTS) &&
-        (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_PACKED_WEIGHTS | MOE_FLAG_GEMM_PATH |
-                     MOE_FLAG_SHARED_EXPERT)))
+        (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_PACKED_WEIGHTS | MOE_FLAG_SHARED_EXPERT)))
         return MOE_ERR_INVALID_ARG;
     if (!isfinite(c->scale)) return MOE_ERR_INVALID_ARG;
     if (c->T < 1 || c->E < 1 || c->E > 256 - shared_slots(*c) || c->k < 1 || c->k > c->E ||
@@ -74,16 +73,26 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA
         if (rc_ != MOE_OK) return rc_;  \
     } while (0)
 
-// Automatic choice: the TMA-fed tensor-core tiles stream the weights faster than
-// the register-staged streaming kernels at every batch size measured on B200
-// (decode T=64: 1.07 ms vs 1.45 ms per layer), so they are the default. FP8
-// weights have a tensor-core path on SM pairs only (d, d_ff multiples of 256);
-// other FP8 shapes use the streaming kernels. FP4 weights have no tensor-core
-// path yet: always the streaming kernels.
+// Automatic choice: the TMA-fed tensor-core tiles stream bf16 weights faster
+// than the register-staged streaming kernels at every batch size measured on
+// B200 (decode T=64: 1.07 ms vs 1.45 ms per layer), so they are the default.
+// FP8 and FP4 weights have a tensor-core path on SM pairs only (d, d_ff
+// multiples of 256); other shapes with those weights use the streaming kernels.
+// The tensor-core FP4 path widens every weight tile to bf16 once per token
+// tile, which at a few tokens per expert costs more than the streaming
+// kernels' direct FMAs: FP4 streams up to kFp4StreamRowsPerExpert mean rows per
+// expert (measured at the Hy3 shape, top-6: 2 rows 1.27 vs 1.59 ms per layer
+// streaming vs tensor cores; 16 rows 8.1 vs 1.85 ms).
+constexpr int kFp4StreamRowsPerExpert = 4;
+bool quantised(const moe_config* c) {
+    return (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_FP4_WEIGHTS)) != 0;
+}
 bool use_stream_path(const moe_config* c) {
-    if (c->flags & (MOE_FLAG_STREAM_PATH | MOE_FLAG_FP4_WEIGHTS)) return true;
+    if (c->flags & MOE_FLAG_STREAM_PATH) return true;
     if (c->flags & MOE_FLAG_GEMM_PATH) return false;
-    return (c->flags & MOE_FLAG_FP8_WEIGHTS) != 0 && !pair_gemm_supported(*c);
+    if (quantised(c) && !pair_gemm_supported(*c)) return true;
+    return (c->flags & MOE_FLAG_FP4_WEIGHTS) &&
+           (long long)c->T * c->k <= (long long)kFp4StreamRowsPerExpert * c->E;
 }
 
 // Router: the tensor-core kernel where it applies (k <= 8) and the batch fills
@@ -125,6 +134,11 @@ int experts_gate_up(const moe_config* c, const void* x_perm, const int32_t* offs
     if (use_stream_path(c))
         return cuda_status(launch_gate_up_stream(g, x_perm, offsets, w_gate_up, s_gate_up, h, s));
     int* status = at<int>(ws, ws_layout(*c).status);
+    if (c->flags & MOE_FLAG_FP4_WEIGHTS) {
+        if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
+        return cuda_status(
+            launch_gate_up_gemm_pair_fp4(g, x_perm, offsets, w_gate_up, s_gate_up, h, status, s));
+    }
     if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
         if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
         return cuda_status(launch_gate_up_gemm_pair_fp8(g, x_perm, offsets, w_gate_up,
@@ -144,7 +158,7 @@ int experts_gate_up_gather(const moe_config* c, const void* x, const int32_t* to
                            const int32_t* offsets, const void* w_gate_up, const void* s_gate_up,
                            void* h, void* ws, cudaStream_t s) {
     const WsLayout L = ws_layout(*c);
-    if (!use_stream_path(c) && !(c->flags & MOE_FLAG_FP8_WEIGHTS) && pair_gemm_supported(*c))
+    if (!use_stream_path(c) && !quantised(c) && pair_gemm_supported(*c))
         return cuda_status(launch_gate_up_gemm_pair_gather(grouped_config(*c), x, token_of_row,
                                                            offsets, w_gate_up, packed(c), h,
                                                            at<int>(ws, L.status), s));
@@ -159,6 +173,11 @@ int experts_down(const moe_config* c, const void* h, const int32_t* offsets, con
     if (use_stream_path(c))
         return cuda_status(launch_down_stream(g, h, offsets, w_down, s_down, y, s));
     int* status = at<int>(ws, ws_layout(*c).status);
+    if (c->flags & MOE_FLAG_FP4_WEIGHTS) {
+        if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
+        return cuda_status(
+            launch_down_gemm_pair_fp4(g, h, offsets, w_down, s_down, y, status, s));
+    }
     if (c->flags & MOE_FLAG_FP8_WEIGHTS) {
         if (!pair_gemm_supported(*c)) return MOE_ERR_UNSUPPORTED_SHAPE;
         return cuda_status(
@@ -359,7 +378,7 @@ int moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const 
 int moe_pack_weights(const moe_config* cfg, int which, const void* w, void* w_packed,
                      void* stream) {
     MOE_TRY(check_cfg(cfg));
-    if (cfg->flags & MOE_FLAG_FP8_WEIGHTS) return MOE_ERR_INVALID_ARG;
+    if (cfg->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_FP4_WEIGHTS)) return MOE_ERR_INVALID_ARG;
     if (which != MOE_WEIGHTS_GATE_UP && which != MOE_WEIGHTS_DOWN) return MOE_ERR_INVALID_ARG;
     if (!w || !w_packed || !aligned16(w) || !aligned16(w_packed)) return MOE_ERR_INVALID_ARG;
     if (!pair_gemm_supported(*cfg)) return MOE_ERR_UNSUPPORTED_SHAPE;

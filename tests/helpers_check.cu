@@ -1,7 +1,7 @@
 // Host-side check of the library's bit-level helpers, compiled and run by
 // tests/test_device_helpers.py: the order-preserving keys of the routers' warp
 // top-k (order_key / key_value), the bf16 conversions and the scaled e4m3
-// widening of the FP8 GEMM. Reads float32 bit patterns from a file, writes the
+// widening of the FP8 and FP4 GEMMs. Reads float32 bit patterns from a file, writes the
 // helpers' results to another (and the widening of all 256 codes to a third).
 // No device code runs.
 #include <stdio.h>
@@ -17,6 +17,11 @@ int main(int argc, char** argv) {
         if (!e8) return 1;
         for (uint32_t i = 0; i < 256; ++i) {
             const uint32_t r = moe::e4m3_pair_scaled_bits((255u - i) << 24 | i << 8);
+            fwrite(&r, sizeof r, 1, e8);
+        }
+        // the FP4 GEMM's scaled E2M1 widening: byte i (two codes)
+        for (uint32_t i = 0; i < 256; ++i) {
+            const uint32_t r = moe::e2m1_pair_scaled_bits(i);
             fwrite(&r, sizeof r, 1, e8);
         }
         if (fclose(e8) != 0) return 1;

@@ -68,7 +68,9 @@ def test_shared_expert_flag_rules(lib):
 def test_fp4_weights_flag_rules(lib):
     assert moe.moe_workspace_size(moe.config(**HY3, fp4=True)) > 0
     assert moe.moe_workspace_size(moe.config(**HY3, fp4=True, path="stream")) > 0
-    for bad in (dict(fp8=True), dict(packed=True), dict(path="gemm"), dict(shared=True)):
+    # the tensor-core pair kernels take FP4 too (d, d_ff multiples of 256)
+    assert moe.moe_workspace_size(moe.config(**HY3, fp4=True, path="gemm")) > 0
+    for bad in (dict(fp8=True), dict(packed=True), dict(shared=True)):
         assert moe.moe_workspace_size(moe.config(**HY3, fp4=True, **bad)) == 0, bad
     # FP4 weights need their block scales
     cfg = moe.config(**HY3, fp4=True)

@@ -83,7 +83,7 @@ def test_scaled_e4m3_widening_is_exact_for_every_code(results):
     """The FP8 GEMM widens e4m3 codes to bf16 with integer bit moves that give
     value * 2^-120 (then one bf16 multiply by 2^120 on the GPU). Every non-NaN
     code, normal, subnormal and both zeros, against the oracle's e4m3 decoding."""
-    r = _E4M3["scaled"]
+    r = _E4M3["scaled"][:256]
     codes = np.arange(256)
     lo = (r & 0xFFFF).astype(np.uint16)
     hi = (r >> 16).astype(np.uint16)
@@ -95,3 +95,16 @@ def test_scaled_e4m3_widening_is_exact_for_every_code(results):
         assert np.array_equal(got[ok], want[ok])
         # signed zeros carry over
         assert np.array_equal(np.signbit(got[ok]), np.signbit(want[ok]))
+
+
+def test_scaled_e2m1_widening_is_exact_for_every_byte(results):
+    """The FP4 GEMM widens a byte of two E2M1 codes to a bf16 pair with integer
+    moves that give value * 2^-126 (the GPU then multiplies by the block scale
+    times 2^126). Every byte, both codes, against the oracle's E2M1 decoding."""
+    r = _E4M3["scaled"][256:]
+    b = np.arange(256, dtype=np.uint8)
+    for half, nib in (((r & 0xFFFF), b & 0xF), ((r >> 16), b >> 4)):
+        got = oracle.double_from_bf16(half.astype(np.uint16)) * 2.0 ** 126
+        want = oracle.double_from_e2m1(nib.astype(np.uint8))
+        assert np.array_equal(got, want)
+        assert np.array_equal(np.signbit(got), np.signbit(want))

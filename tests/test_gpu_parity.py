@@ -440,21 +440,30 @@ F4 = {
     "fp4_ragged": LayerShape(T=300, d=512, E=32, k=6, F=384, scale=1.5, fp4=True,
                              score_fn="sqrtsoftplus", score_bias_std=0.05),
     "fp4_sigmoid": LayerShape(T=40, d=384, E=8, k=2, F=256, fp4=True),
+    # d and d_ff multiples of 256: FP4 on the tensor-core SM-pair kernels
+    "fp4_pair": LayerShape(T=333, d=768, E=24, k=6, F=512, scale=1.5, fp4=True,
+                           score_fn="sqrtsoftplus", score_bias_std=0.05),
+    "fp4_pair_tiny": LayerShape(T=3, d=512, E=8, k=2, F=256, fp4=True),
 }
 
 
 @pytest.mark.parametrize("name", sorted(F4))
-def test_second_variant_every_token(name):
+@pytest.mark.parametrize("path", [None, "stream", "gemm"])
+def test_second_variant_every_token(name, path):
     sh = F4[name]
+    if path == "gemm" and (sh.d % 256 or sh.F % 256):
+        pytest.skip("the tensor-core pair kernels need d and d_ff multiples of 256")
+    if path is not None and not sh.fp4:
+        pytest.skip("the expert path matters for the FP4 experts only")
     layer = make_layer(sh, seed=61, device="cuda")
-    route = parity.gpu_route(layer)
+    route = parity.gpu_route(layer, path)
     O = oracle.OracleLayer(layer)
     ref = oracle.route(O.x, O.wg, O.k, O.scale, O.gate_bias, score_bias=O.score_bias,
                        score_fn=O.score_fn)
     parity.check_route(*route, ref)
-    out = parity.gpu_forward(layer)
+    out = parity.gpu_forward(layer, path)
     res = parity.check_forward(layer, out, None, route)
-    print(name, res)
+    print(name, path, res)
     _free(layer, out)
 
 
@@ -469,21 +478,21 @@ def test_sqrt_softplus_router_on_hy3_shape(T):
     parity.check_route(*route, ref)
 
 
-def test_fp4_decode_hy3_shape():
+@pytest.mark.parametrize("path", [None, "stream", "gemm"])
+def test_fp4_decode_hy3_shape(path):
     """FP4 experts at the Hy3 decode shape (T=64, d=4096, E=192, d_ff=1536), top-6
-    sqrt-softplus routing: every token routed, a sample of outputs."""
+    sqrt-softplus routing, on the streaming kernels (the default at this batch)
+    and on the tensor-core pair kernels: every token's routing and output."""
     shape = dataclasses.replace(CONFIGS["decode"], k=6, scale=1.5, fp4=True,
                                 score_fn="sqrtsoftplus")
     layer = make_layer(shape, seed=5, device="cuda")
-    route = parity.gpu_route(layer)
+    route = parity.gpu_route(layer, path)
     O = oracle.OracleLayer(layer)
     ref = oracle.route(O.x, O.wg, O.k, O.scale, score_fn="sqrtsoftplus")
     near = parity.check_route(*route, ref)
-    out = parity.gpu_forward(layer)
-    toks = np.unique(np.concatenate([parity.sample_tokens(shape.T, n=32),
-                                     near[:8].astype(np.int32)]))
-    res = parity.check_forward(layer, out, toks, route)
-    print("fp4 decode, near ties:", len(near), res)
+    out = parity.gpu_forward(layer, path)
+    res = parity.check_forward(layer, out, None, route)
+    print("fp4 decode", path, "near ties:", len(near), res)
     _free(layer, out)
 
 
@@ -558,3 +567,42 @@ def test_fp8_weights_widen_exactly_for_every_code(path):
     bad = np.nonzero(got != want)
     assert bad[0].size == 0, (f"{bad[0].size} outputs differ, first code "
                               f"{want_codes[bad][0]:#04x}: {got[bad][0]} vs {want[bad][0]}")
+
+
+@pytest.mark.parametrize("path", ["gemm", "stream"])
+def test_fp4_weights_widen_exactly_for_every_code_and_scale(path):
+    """moe_expert_down with FP4 weights and one-hot rows of h: y[r, i] is the
+    weight W[e_r, i, f_r] = E2M1 code value * 2^(b - 127) itself, exact in bf16.
+    Rows cover all 16 codes (both signs, the subnormal 0.5 and both zeros) under
+    block scales b from 0 to 252 -- on both sides of b = 128, where the tensor-core
+    widening switches from one multiply by 2^(b-1) to two -- compared with the
+    oracle's E2M1 and E8M0 decoding."""
+    E, d, F, rows_e = 2, 256, 256, 128
+    R = E * rows_e
+    g = torch.Generator().manual_seed(17)
+    codes = torch.randint(0, 256, (E, d, F // 2), generator=g, dtype=torch.uint8)
+    bvals = torch.tensor([0, 1, 60, 110, 120, 126, 127, 128, 129, 130, 160, 200, 250, 252],
+                         dtype=torch.uint8)
+    scales = bvals[torch.randint(0, len(bvals), (E, d, F // 32), generator=g)]
+    f_of_row = (np.arange(R) * 7 + 3) % F
+    h = torch.zeros((R, F), dtype=torch.bfloat16)
+    h[torch.arange(R), torch.from_numpy(f_of_row)] = 1.0
+    cfg = moe.config(T=R, d=d, E=E, k=1, d_ff=F, fp4=True, path=path)
+    ws = moe.workspace(cfg)
+    offsets = torch.tensor([0, rows_e, R], dtype=torch.int32, device="cuda")
+    y = torch.empty((R, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_down(cfg, h.cuda(), offsets, codes.cuda(), scales.cuda(), y, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_status(ws) == moe.MOE_OK
+    e_of_row = np.arange(R) // rows_e
+    cn, sn = codes.numpy(), scales.numpy()
+    ii = np.arange(d)[None, :]
+    byte = cn[e_of_row[:, None], ii, (f_of_row // 2)[:, None]]
+    nib = np.where((f_of_row % 2)[:, None] == 1, byte >> 4, byte & 0xF).astype(np.uint8)
+    b = sn[e_of_row[:, None], ii, (f_of_row // 32)[:, None]]
+    want = oracle.double_from_e2m1(nib) * oracle.double_from_e8m0(b)
+    assert len(np.unique(nib)) == 16 and len(np.unique(b)) == len(bvals)
+    got = oracle.double_from_bf16(oracle.bf16_bits(y))
+    bad = np.nonzero(got != want)
+    assert bad[0].size == 0, (f"{bad[0].size} outputs differ, first code {nib[bad][0]} scale "
+                              f"{b[bad][0]}: {got[bad][0]} vs {want[bad][0]}")
