@@ -98,7 +98,7 @@ struct TileInfo {
     int e, m, row0, len, n;  // n: MMA N of the pair, a multiple of 2*NBOX
 };
 
-template <typename CtrlT>
+template <int NM = NMAX, typename CtrlT>
 __device__ __forceinline__ TileInfo decode_tile(const CtrlT& c, int E, int m_tiles, int t) {
     int lo = 0, hi = E - 1;
     while (lo < hi) {
@@ -108,15 +108,15 @@ __device__ __forceinline__ TileInfo decode_tile(const CtrlT& c, int E, int m_til
     const int e = lo;
     const int local = t - c.tile_start[e];
     const int n_e = c.off[e + 1] - c.off[e];
-    // nt = ceil(n_e / NMAX) token tiles; all but the last hold 32q rows, so only
+    // nt = ceil(n_e / NM) token tiles; all but the last hold 32q rows, so only
     // the last one pads its MMA N to a multiple of 32 (near-equal tiles would pad
     // every one: 341 rows as 171 + 170 run N = 192 + 192, as 192 + 149 run
-    // 192 + 160). q = ceil(ceil(n_e / 32) / nt), or NMAX / 32 if that left the
-    // last tile empty; every tile then holds 1..NMAX rows.
-    const int nt = (n_e + NMAX - 1) / NMAX;
+    // 192 + 160). q = ceil(ceil(n_e / 32) / nt), or NM / 32 if that left the
+    // last tile empty; every tile then holds 1..NM rows.
+    const int nt = (n_e + NM - 1) / NM;
     const int units = (n_e + 2 * NBOX - 1) / (2 * NBOX);
     int q = (units + nt - 1) / nt;
-    if (2 * NBOX * q * (nt - 1) >= n_e) q = NMAX / (2 * NBOX);
+    if (2 * NBOX * q * (nt - 1) >= n_e) q = NM / (2 * NBOX);
     // token tiles fastest: the tiles that read the same weight rows (same m,
     // next j) get neighbouring indices, so concurrent SM pairs stream those
     // weights from HBM once and from L2 for the others
@@ -425,15 +425,15 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 // ======================================================================
 // FP8 (e4m3) weights. The MMA stays kind::f16 (bf16 x bf16, fp32 accumulate)
 // on weights widened on chip. Per K block, warp 0 TMA-loads this CTA's raw
-// e4m3 weight tile(s) (128 rows x 64 bytes, unswizzled) into a "raw" ring on
-// the CTA's own barrier; warp 15 loads its half of the token rows (bf16,
+// e4m3 weight tile(s) (128 rows x 64 bytes, 64-byte swizzle) into a "raw" ring
+// on the CTA's own barrier; warp 15 loads its half of the token rows (bf16,
 // 128-byte swizzle) into a token ring completing on the even CTA's barrier.
-// Converter warps, in groups that take K blocks round-robin (so the conversion
-// latencies of consecutive blocks overlap; 2 x 4 warps for gate_up, 3 x 3 for
-// down), widen the weights exactly to bf16 straight into the
-// 128-byte-swizzled operand layout of an "op" stage, release the raw stage and
-// arrive on the even CTA's operand barrier; the pair MMA reads A from the op
-// stage and B from the token stage and releases both. The raw stages live only
+// Converter warps, in two groups of four that take K blocks round-robin (so
+// the conversion latencies of consecutive blocks overlap), widen the weights
+// exactly to bf16 straight into an "op" stage of tensor memory (below),
+// release the raw stage and arrive on the even CTA's operand barrier; the pair
+// MMA reads A from the op stage and B from the token stage and releases both.
+// The raw stages live only
 // from load to conversion, so their ring keeps the weight stream deep. The
 // per-output-row fp32 scale multiplies the finished dot product in the
 // epilogue (before SiLU for gate_up, before the bf16 store for down):
@@ -443,30 +443,46 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 constexpr int THREADS_FP8 = 512;        // warps 6-14 converters, warp 15 token producer
 constexpr int RAW_BYTES = BM * BK;      // one 128 x 64 e4m3 tile
 
+// FP8 (ATM): the converters write the widened A operand straight into tensor
+// memory (tcgen05.st, one thread per A row) and the pair MMA reads A from there,
+// so the operand tiles never pass through shared memory. TMEM then holds the
+// accumulators and the A stages, which caps an FP8 token tile at NM = 192 rows
+// (gate_up: g and u, 2 x 192 columns; down: 2 x 192). The remaining 128
+// columns hold the A stages, one K block each: 2 of 64 columns (gate + up)
+// for gate_up, 4 of 32 for down. (Half-K-block stages, twice as many, measured
+// 8% slower on B200 for gate_up and 10% for down: twice the barrier and signal
+// work for half the conversion each.)
 // FP4: E2M1 codes and E8M0 block scales folded into the widening (no row scale
-// in the epilogue). A raw tile is still 128 rows x 64 bytes, which holds 128
-// codes a row: two K blocks (KPR) per raw stage, so FP4 keeps FP8's TMA box and
-// ring depths while its weight stream has the same bytes in flight. (Raw
-// rings of 8 / 12 stages of one-K-block FP4 tiles stalled or faulted on B200,
-// cause not identified; that form is not used.)
+// in the epilogue), A in shared memory. A raw tile is 128 rows x 64 bytes,
+// which holds 128 codes a row: two K blocks (KPR) per raw stage.
+constexpr int MAX_RAW_STAGES = 16, MAX_B_STAGES = 4, MAX_OP_STAGES = 6;  // Fp8Ctrl's arrays
 template <bool GATE_UP, bool FP4 = false>
 struct Fp8Shape {
+    static constexpr bool ATM = !FP4;                              // A operand in TMEM
     static constexpr int A_TILES = GATE_UP ? 2 : 1;
     static constexpr int KPR = FP4 ? 2 : 1;                        // K blocks per raw stage
+    static constexpr int NM = ATM ? 192 : NMAX;                    // token rows per pair tile
+    static constexpr int BH = (NM / 2) * BK * 2;                   // a CTA's token half (bytes)
     static constexpr int RAW_TILE = RAW_BYTES;                     // 128 rows x 64 bytes
     static constexpr int RAW_STAGE = A_TILES * RAW_TILE;           // 16 KB / 8 KB
-    static constexpr int OP_STAGE = A_TILES * A_BYTES;             // 32 KB / 16 KB
-    static constexpr int RAW_STAGES = GATE_UP ? 4 : 6;  // multiples of GROUPS
-    static constexpr int B_STAGES = GATE_UP ? 3 : 4;
-    static constexpr int OP_STAGES = GATE_UP ? 3 : 6;   // >= GROUPS (see the converters)
+    static constexpr int OP_STAGE = ATM ? 0 : A_TILES * A_BYTES;   // shared-memory op stage
+    static constexpr int RAW_STAGES = ATM ? (GATE_UP ? 8 : 12) : (GATE_UP ? 4 : 6);
+    static constexpr int B_STAGES = ATM ? 4 : (GATE_UP ? 3 : 4);
+    static constexpr int OP_STAGES = ATM ? (GATE_UP ? 2 : 4) : (GATE_UP ? 3 : 6);
     // converter warps: GROUPS groups of GROUP_WARPS take K blocks round-robin
-    static constexpr int GROUPS = GATE_UP ? 2 : 3;
-    static constexpr int GROUP_WARPS = GATE_UP ? 4 : 3;
+    // (ATM: four warps a group, one per TMEM lane quarter)
+    static constexpr int GROUPS = ATM ? 2 : (GATE_UP ? 2 : 3);
+    static constexpr int GROUP_WARPS = ATM ? 4 : (GATE_UP ? 4 : 3);
     static constexpr int CONV_THREADS = GROUP_WARPS * 32;
     static constexpr int RING_BYTES =
-        RAW_STAGES * RAW_STAGE + B_STAGES * BH_BYTES + OP_STAGES * OP_STAGE;  // 208 KB
+        RAW_STAGES * RAW_STAGE + B_STAGES * BH + OP_STAGES * OP_STAGE;
     static constexpr int ACC_STAGES = GATE_UP ? 1 : 2;
-    static constexpr int ACC_COLS = GATE_UP ? 512 : 256;
+    // TMEM columns: the accumulators, then (ATM) the A stages
+    static constexpr int U_OFF = ATM ? NM : 256;                   // gate_up's up accumulator
+    static constexpr int ACC_COLS = GATE_UP ? 2 * U_OFF : (ATM ? NM : 256);
+    static constexpr int A_COL = ACC_STAGES * ACC_COLS;
+    static constexpr int A_TILE_COLS = BK / 2;                     // one tile's K block: two bf16 a column
+    static constexpr int A_STAGE_COLS = A_TILES * A_TILE_COLS;
 };
 
 constexpr int CONV_WARPS = 9;                          // warps 6..14 (some idle for gate_up)
@@ -475,26 +491,32 @@ template <bool G, bool FP4>
 constexpr bool groups_ok() {
     using S = Fp8Shape<G, FP4>;
     return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES >= S::KPR * S::GROUPS - 1 &&
-           S::GROUPS * S::GROUP_WARPS <= CONV_WARPS;
+           S::OP_STAGES >= S::GROUPS && S::GROUPS * S::GROUP_WARPS <= CONV_WARPS &&
+           S::RAW_STAGES <= MAX_RAW_STAGES && S::B_STAGES <= MAX_B_STAGES &&
+           S::OP_STAGES <= MAX_OP_STAGES && (!S::ATM || S::GROUP_WARPS == 4) &&
+           (!S::ATM || S::A_COL + S::OP_STAGES * S::A_STAGE_COLS <= 512) &&
+           S::ACC_STAGES * S::ACC_COLS <= 512 && S::BH % 1024 == 0;
 }
 // Each group owns whole raw stages, and a group's previous operand wait proves
-// that the stage's last reader finished (parity waits cannot see a stale phase).
+// that the stage's last reader finished (parity waits cannot see a stale phase);
+// every stage index stays inside Fp8Ctrl's barrier arrays.
 static_assert(groups_ok<true, false>() && groups_ok<false, false>() && groups_ok<true, true>() &&
                   groups_ok<false, true>(),
               "converter grouping");
 static_assert(THREADS_FP8 == 32 * (TOKEN_WARP + 1), "warp roles cover the block");
 
 struct Fp8Ctrl {
-    uint64_t raw_full[6];   // each CTA: its raw weight tile(s) landed
-    uint64_t raw_empty[6];  // each CTA: every converter warp is done with the raw stage
-    uint64_t b_full[4];     // even CTA: token bytes of both CTAs landed
-    uint64_t b_empty[4];    // both CTAs: the pair MMAs finished reading the token stage
-    uint64_t op_full[6];    // even CTA: both CTAs' groups filled the op stage (see below)
-    uint64_t op_empty[6];   // both CTAs: the pair MMAs finished reading the op stage
+    uint64_t raw_full[MAX_RAW_STAGES];   // each CTA: its raw weight tile(s) landed
+    uint64_t raw_empty[MAX_RAW_STAGES];  // each CTA: the converters are done with the raw stage
+    uint64_t b_full[MAX_B_STAGES];       // even CTA: token bytes of both CTAs landed
+    uint64_t b_empty[MAX_B_STAGES];      // both CTAs: the pair MMAs finished with the token stage
+    uint64_t op_full[MAX_OP_STAGES];     // even CTA: both CTAs' groups filled the op stage
+    uint64_t op_empty[MAX_OP_STAGES];    // both CTAs: the pair MMAs finished with the op stage
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
-    alignas(16) uint32_t sig[6][4];  // even CTA: landing slots of the odd CTA's ready signals
+    alignas(16) uint32_t sig[MAX_OP_STAGES][4];  // even CTA: landing slots of the odd CTA's signals
+    alignas(16) uint32_t sig_src[4];             // odd CTA: the signals' (unread) source bytes
     uint32_t tmem_base;
     int abort;
     int total;
@@ -529,48 +551,20 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
+// The same multiply kept in program order with respect to the waits around it
+// (volatile), so that a conversion stays ahead of the wait that follows it.
+__device__ __forceinline__ uint32_t mul_bf16x2_here(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm volatile("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+template <bool HERE = false>
 __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
     constexpr uint32_t kTwoPow120 = 0x7B807B80u;  // bf16x2 (2^120, 2^120)
-    lo = mul_bf16x2(e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x1404)), kTwoPow120);
-    hi = mul_bf16x2(e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x3424)), kTwoPow120);
-}
-
-// Convert one raw e4m3 tile (128 rows x 64 bytes, row-major) into a bf16
-// operand tile (128 rows x 128 bytes, 128-byte swizzle) with CONV_THREADS threads;
-// thread `ct` handles 16-byte source chunks q = ct + CONV_THREADS i (row q/4,
-// elements 16(q%4)..16(q%4)+15). All of a thread's chunks are loaded before
-// any is widened, so that their shared-memory latencies overlap (the inline
-// loads and stores keep program order).
-template <int CONV_THREADS>
-__device__ __forceinline__ void widen_tile(uint32_t raw, uint32_t op, int ct) {
-    constexpr int PER = (512 + CONV_THREADS - 1) / CONV_THREADS;
-    uint32_t w[PER][4];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int q = ct + i * CONV_THREADS;
-        if (q < 512)
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w[i][0]), "=r"(w[i][1]), "=r"(w[i][2]), "=r"(w[i][3])
-                         : "r"(raw + q * 16));
-    }
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int q = ct + i * CONV_THREADS;
-        if (q >= 512) break;
-        const int row = q >> 2, c = q & 3;
-        uint32_t b[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) e4m3x4_to_bf16x4(w[i][j], b[2 * j], b[2 * j + 1]);
-        const uint32_t rbase = op + row * 128;
-        const int sw = row & 7;
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(rbase + (((2 * c) ^ sw) << 4)),
-                     "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3])
-                     : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         rbase + (((2 * c + 1) ^ sw) << 4)),
-                     "r"(b[4]), "r"(b[5]), "r"(b[6]), "r"(b[7])
-                     : "memory");
-    }
+    const uint32_t a = e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x1404));
+    const uint32_t b = e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x3424));
+    lo = HERE ? mul_bf16x2_here(a, kTwoPow120) : mul_bf16x2(a, kTwoPow120);
+    hi = HERE ? mul_bf16x2_here(b, kTwoPow120) : mul_bf16x2(b, kTwoPow120);
 }
 
 // Convert one K block of a raw E2M1 tile (128 rows x 64 bytes, row-major, two K
@@ -632,8 +626,9 @@ __device__ __forceinline__ void widen_tile_fp4(uint32_t raw, uint32_t op, int ct
     }
 }
 
-// tmA: e4m3 weights [E * a_rows_per_expert, K] bytes, box 64 x 128 (no swizzle);
-// FP4: E2M1 codes [E * a_rows_per_expert, K / 2] bytes, box 64 x 128 (two K blocks).
+// tmA: e4m3 weights [E * a_rows_per_expert, K] bytes, box 64 x 128, 64-byte
+// swizzle; FP4: E2M1 codes [E * a_rows_per_expert, K / 2] bytes, box 64 x 128
+// (two K blocks), no swizzle.
 // tmB: token rows [R, K] bf16, box 64 x 16. scales_v: FP8 fp32 row scales
 // [E * a_rows_per_expert]; FP4 E8M0 block scales [E * a_rows_per_expert, K / 32]
 // bytes.
@@ -653,7 +648,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* op_ring = smem;  // 1024-aligned operand stages first
     uint8_t* b_ring = op_ring + S::OP_STAGES * S::OP_STAGE;
-    uint8_t* raw_ring = b_ring + S::B_STAGES * BH_BYTES;
+    uint8_t* raw_ring = b_ring + S::B_STAGES * S::BH;
     uint16_t* epi = reinterpret_cast<uint16_t*>(smem + S::RING_BYTES);
     Fp8Ctrl& c = *reinterpret_cast<Fp8Ctrl*>(smem + S::RING_BYTES + FP8_EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -674,7 +669,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             __syncwarp();
             if (e < E) {
                 const int n_e = offsets[e + 1] - o;
-                cnt = ((n_e + NMAX - 1) / NMAX) * m_tiles;
+                cnt = ((n_e + S::NM - 1) / S::NM) * m_tiles;
             }
             int incl = cnt;
 #pragma unroll
@@ -734,7 +729,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             bool issued[S::RAW_STAGES] = {};
             bool ok = true;
             for (int t = pair; t < total && ok; t += n_pairs) {
-                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, t);
                 const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
                 for (int kr = 0; kr < KB / S::KPR; ++kr) {  // raw blocks of KPR K blocks
                     if (!tc::mbar_wait(&c.raw_empty[stage], phase ^ 1u, abort_flag)) {
@@ -772,7 +767,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             bool issued[S::B_STAGES] = {};
             bool ok = true;
             for (int t = pair; t < total && ok; t += n_pairs) {
-                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, t);
                 const int nb = ti.n / (2 * NBOX);
                 const int b_row = ti.row0 + rank * (ti.n / 2);
                 const uint32_t pair_bytes = 2u * (uint32_t)(nb * BOX_BYTES);
@@ -784,7 +779,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.b_full[stage]), 0);
                     if (leader) tc::mbar_arrive_expect_tx(&c.b_full[stage], pair_bytes);
-                    uint8_t* st = b_ring + stage * BH_BYTES;
+                    uint8_t* st = b_ring + stage * S::BH;
                     load_token_rows(st, tmB, full_leader, kb * BK, b_row, ti.n / 2, pol_x);
                     issued[stage] = true;
                     parity[stage] = phase;
@@ -800,17 +795,19 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     atomicExch(status, MOE_ERR_TIMEOUT);
         }
     } else if (warp >= 6 && warp < 6 + CONV_WARPS) {
-        // ---------------- converters: raw e4m3 -> bf16 operand (A) in the op stage.
-        // A group's threads fence their writes to the async proxy and meet at a
-        // named barrier; then one thread releases the raw stage and signals the
-        // even CTA's op_full: in the even CTA a local arrive that expects 16
-        // bytes, in the odd CTA a 16-byte bulk copy into the even CTA's shared
-        // memory that completes on that barrier (an async-proxy operation issued
-        // after the fenced writes). A remote mbarrier arrive with cluster-scope
-        // release, the other way to signal across the pair, stalled its warp
-        // ~1.5k cycles per K block on B200 -- longer than the widening itself.
-        // The group agrees on its bounded waits (bar.red.or) and leaves
-        // together; the MMA's bounded wait on op_full then gives up.
+        // ---------------- converters: raw codes -> bf16 operand (A) in the op stage
+        // (FP8: TMEM columns; FP4: a shared-memory tile). A group's threads
+        // complete their writes (FP8: tcgen05.wait::st and the tcgen05 fence;
+        // FP4: a fence to the async proxy) and meet at a named barrier; then one
+        // thread releases the raw stage and signals the even CTA's op_full: in
+        // the even CTA a local arrive that expects 16 bytes, in the odd CTA a
+        // 16-byte shared-to-shared bulk copy into the even CTA that completes on
+        // that barrier (an async-proxy operation issued after the completed
+        // writes). A remote mbarrier arrive with cluster-scope release, the
+        // other way to signal across the pair, stalled its warp ~1.5k cycles per
+        // K block on B200 -- longer than the widening itself. The group agrees
+        // on its bounded waits (bar.red.or) and leaves together; the MMA's
+        // bounded wait on op_full then gives up.
         const int group = (warp - 6) / S::GROUP_WARPS;
         const int ct = threadIdx.x - 192 - group * S::CONV_THREADS;  // 0..CONV_THREADS-1
         const uint32_t raw0 = tc::smem_u32(raw_ring), op0 = tc::smem_u32(op_ring);
@@ -822,8 +819,9 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             if (leader)
                 tc::mbar_arrive_expect_tx(&c.op_full[os], 16);
             else
-                tc::bulk_copy_to_cluster(tc::map_to_cta(tc::smem_u32(&c.sig[os][0]), 0), scales_v,
-                                         16, tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
+                tc::bulk_copy_smem_to_cluster(tc::map_to_cta(tc::smem_u32(&c.sig[os][0]), 0),
+                                              tc::smem_u32(&c.sig_src[0]), 16,
+                                              tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
         };
         if constexpr (FP4) {
             // A group takes raw blocks jr = group, group + GROUPS, ... and turns each
@@ -852,7 +850,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     uint32_t sc[S::A_TILES][PER4];
                     const long it = jb / KB;
                     const int kb = (int)(jb - it * KB);
-                    const TileInfo ti = decode_tile(c, E, m_tiles, pair + (int)it * n_pairs);
+                    const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, pair + (int)it * n_pairs);
                     const long a_row = (long)ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
                     const long blocks = K / 32;
 #pragma unroll
@@ -883,25 +881,57 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 if (failed) break;
             }
-        } else {
-            // a group converts the K blocks j = group, group + GROUPS, ... (warps
-            // past the groups idle)
+        } else if constexpr (S::ATM) {
+            // Each thread widens one A row of this CTA -- row r = 32 (warp % 4) +
+            // lane, the TMEM lane its warp may write -- for every A tile of the K
+            // block: the 64 codes of its raw row (64-byte rows, 64-byte swizzle:
+            // 16-byte chunk c of row r sits at chunk c ^ ((r / 2) % 4), so that
+            // the eight rows of a quarter-warp hit distinct banks) into 32 TMEM
+            // columns (two bf16 a column, the even K index in the low half). A
+            // group converts the K blocks j = group, group + GROUPS, ... (warps
+            // past the groups idle). The widening runs before the wait for the op
+            // stage; the writes complete (tcgen05.wait::st) before the group's
+            // barrier and the signal.
+            const int r = 32 * (warp & 3) + lane;
+            const uint32_t rsw = (uint32_t)((r >> 1) & 3);
+            const uint32_t a_lane = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + S::A_COL;
             const long n_blocks = (long)n_my_tiles * KB;
             for (long jb = (group < S::GROUPS ? group : n_blocks); jb < n_blocks; jb += S::GROUPS) {
                 const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
                 const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
                 const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
-                const bool ok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag) &&
-                                tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
-                if (tc::bar_any(2 + group, S::CONV_THREADS, !ok)) {  // the group leaves together
+                const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
+                if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
                     raise_timeout(c, status);
                     break;
                 }
-                const uint32_t raw = raw0 + rs * S::RAW_STAGE;
-                const uint32_t op = op0 + os * S::OP_STAGE;
-                widen_tile<S::CONV_THREADS>(raw, op, ct);
-                if (GATE_UP) widen_tile<S::CONV_THREADS>(raw + S::RAW_TILE, op + A_BYTES, ct);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                const uint32_t raw = raw0 + rs * S::RAW_STAGE + r * 64;
+                uint32_t w[S::A_TILES][16];
+#pragma unroll
+                for (int a = 0; a < S::A_TILES; ++a)
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(w[a][4 * ch]), "=r"(w[a][4 * ch + 1]),
+                                       "=r"(w[a][4 * ch + 2]), "=r"(w[a][4 * ch + 3])
+                                     : "r"(raw + a * S::RAW_TILE + ((ch ^ rsw) << 4)));
+                uint32_t o[S::A_TILES][32];
+#pragma unroll
+                for (int a = 0; a < S::A_TILES; ++a)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        e4m3x4_to_bf16x4<true>(w[a][j], o[a][2 * j], o[a][2 * j + 1]);
+                const bool ook = tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
+                if (tc::bar_any(2 + group, S::CONV_THREADS, !ook)) {
+                    raise_timeout(c, status);
+                    break;
+                }
+                tc::fence_after_sync();  // the MMAs that read this op stage are complete
+#pragma unroll
+                for (int a = 0; a < S::A_TILES; ++a)
+                    tc::tmem_st32(a_lane + os * S::A_STAGE_COLS + a * S::A_TILE_COLS, o[a]);
+                tc::tmem_st_wait();
+                tc::fence_before_sync();
                 tc::bar_sync(2 + group, S::CONV_THREADS);
                 if (ct == 0) {
                     tc::mbar_arrive(&c.raw_empty[rs]);
@@ -911,13 +941,13 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
-            // ---------------- MMA issuer (even CTA): A from the op stage, B from the raw stage
+            // ---------------- MMA issuer (even CTA): A from the op stage (FP8: in TMEM), B from the token stage
             int bs = 0, os = 0;
             uint32_t oph = 0, bph = 0;
             bool ok = true;
             int it = 0;
             for (int t = pair; t < total && ok; t += n_pairs, ++it) {
-                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, t);
                 const int acc = it % S::ACC_STAGES;
                 const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
                 if (!tc::mbar_wait(&c.acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -936,17 +966,26 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     tc::fence_after_sync();
                     const uint32_t a_addr = tc::smem_u32(op_ring + os * S::OP_STAGE);
-                    const uint32_t b_addr = tc::smem_u32(b_ring + bs * BH_BYTES);
+                    const uint32_t a_tm = tmem_base + S::A_COL + os * S::A_STAGE_COLS;
+                    const uint32_t b_addr = tc::smem_u32(b_ring + bs * S::BH);
 #pragma unroll
                     for (int k = 0; k < BK / UK; ++k) {
                         const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                        tc::mma_bf16_pair(d_tmem, tc::desc_sw128(a_addr + k * UK * 2), bdesc,
-                                          idesc, accum);
-                        if (GATE_UP)
-                            tc::mma_bf16_pair(d_tmem + 256,
-                                              tc::desc_sw128(a_addr + A_BYTES + k * UK * 2), bdesc,
+                        if constexpr (S::ATM) {  // K = 16 of A is 8 TMEM columns
+                            tc::mma_bf16_pair_ta(d_tmem, a_tm + k * (UK / 2), bdesc, idesc, accum);
+                            if (GATE_UP)
+                                tc::mma_bf16_pair_ta(d_tmem + S::U_OFF,
+                                                     a_tm + S::A_TILE_COLS + k * (UK / 2), bdesc,
+                                                     idesc, accum);
+                        } else {
+                            tc::mma_bf16_pair(d_tmem, tc::desc_sw128(a_addr + k * UK * 2), bdesc,
                                               idesc, accum);
+                            if (GATE_UP)
+                                tc::mma_bf16_pair(d_tmem + S::U_OFF,
+                                                  tc::desc_sw128(a_addr + A_BYTES + k * UK * 2),
+                                                  bdesc, idesc, accum);
+                        }
                     }
                     tc::mma_commit_pair(&c.op_empty[os], 0x3);
                     tc::mma_commit_pair(&c.b_empty[bs], 0x3);
@@ -977,7 +1016,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         const bool arriver = (warp == 2 && lane == 0);
         int it = 0;
         for (int t = pair; t < total; t += n_pairs, ++it) {
-            const TileInfo ti = decode_tile(c, E, m_tiles, t);
+            const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, t);
             const int acc = it % S::ACC_STAGES;
             const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
             const bool waited = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
@@ -998,7 +1037,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 tc::tmem_ld32(tbase + c0, g);
                 if constexpr (GATE_UP) {
                     uint32_t u[32];
-                    tc::tmem_ld32(tbase + 256 + c0, u);
+                    tc::tmem_ld32(tbase + S::U_OFF + c0, u);
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
@@ -1068,9 +1107,9 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 // Row-major [rows, cols] bytes (e4m3 codes, or E2M1 code pairs), box of
-// box_rows x box_cols bytes, no swizzle.
+// box_rows x box_cols bytes, no swizzle or (box_cols = 64) the 64-byte swizzle.
 bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                 uint32_t box_rows, uint32_t box_cols = BK) {
+                 uint32_t box_rows, uint32_t box_cols = BK, bool swizzle64 = false) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
@@ -1078,7 +1117,8 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1170,7 +1210,7 @@ cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm
     CUtensorMap a;
     TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
-    if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM) ||
+    if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM, BK, true) ||
         !make_token_maps(&b, x_perm, R, c.d))
         return cudaErrorInvalidValue;
     return launch_fp8<true>(a, b, offsets, s_gate_up, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h,
@@ -1183,7 +1223,7 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
     CUtensorMap a;
     TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
-    if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM) ||
+    if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM, BK, true) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
     return launch_fp8<false>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d,

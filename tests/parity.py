@@ -155,7 +155,11 @@ def sample_tokens(T: int, n: int = 48, seed: int = 0) -> np.ndarray:
     return np.unique(np.concatenate([np.arange(8), mid, np.arange(T - 8, T)])).astype(np.int32)
 
 
-def gemm_tiles(counts, nmax: int = 256, unit: int = 32):
+NMAX = 256       # token rows per tile of the bf16 and FP4 SM-pair GEMMs
+FP8_NMAX = 192   # FP8: the widened weights share tensor memory with the accumulators
+
+
+def gemm_tiles(counts, nmax: int = NMAX, unit: int = 32):
     """The token tiles of the SM-pair grouped GEMMs: expert e's n_e grouped rows
     split into nt = ceil(n_e / nmax) tiles, all but the last of unit*q rows
     (q = ceil(ceil(n_e / unit) / nt), or nmax / unit if that left the last tile
@@ -172,7 +176,7 @@ def gemm_tiles(counts, nmax: int = 256, unit: int = 32):
             yield e, j * unit * q, unit * q if j < nt - 1 else n - unit * q * (nt - 1)
 
 
-def tile_cover_tokens(idx: np.ndarray, E: int, edge: int = 32, nmax: int = 256) -> np.ndarray:
+def tile_cover_tokens(idx: np.ndarray, E: int, edge: int = 32, nmax: int = NMAX) -> np.ndarray:
     """Tokens that put a grouped row into the first and into the last ``edge``
     rows of every (expert, token tile) of the grouped GEMMs, chosen greedily
     (each token brings k rows). The grouping is the oracle's (row_of), so the

@@ -100,14 +100,33 @@ def test_hy3_shapes(name):
     # at the head and at the tail of every (expert, token tile) of the grouped
     # GEMMs under the GPU's routing
     toks = parity.sample_tokens(shape.T, n=48 if shape.T > 64 else 64)
-    cover = parity.tile_cover_tokens(route[0], shape.E)
+    nmax = parity.FP8_NMAX if shape.fp8 else parity.NMAX
+    cover = parity.tile_cover_tokens(route[0], shape.E, nmax=nmax)
     toks = np.unique(np.concatenate([toks, near[:8].astype(np.int32), cover]))
     res = parity.check_forward(layer, out, toks, route)
-    n_tiles = len(list(parity.gemm_tiles(np.bincount(route[0].ravel(), minlength=shape.E))))
+    n_tiles = len(list(parity.gemm_tiles(np.bincount(route[0].ravel(), minlength=shape.E), nmax)))
     print(name, "near-tie tokens:", len(near), near[:16].tolist(),
           f"checked tokens {len(toks)} (rows {len(toks) * shape.k}), tiles covered {n_tiles}",
           res)
     _free(layer, out)
+
+
+@pytest.mark.parametrize("T", [193, 700])
+def test_fp8_all_tokens_to_the_same_experts(T):
+    """FP8 weights on the pair GEMMs with every token on experts 0..3: T rows
+    each, in token tiles of at most 192 rows (193 as 128 + 65, 700 as
+    3 x 192 + 124); every token against the oracle."""
+    shape = LayerShape(T=T, d=512, E=16, k=4, F=256, fp8=True)
+    layer = make_layer(shape, seed=5, device="cuda")
+    b = torch.zeros(shape.E, dtype=torch.float32, device="cuda")
+    b[:4] = 40.0
+    layer["gate_bias"] = b
+    route = parity.gpu_route(layer)
+    assert np.all(np.sort(route[0], axis=1) == np.arange(4))
+    tiles = parity.gemm_tiles(np.bincount(route[0].ravel()), parity.FP8_NMAX)
+    assert [n for e, _, n in tiles if e == 0] == ([128, 65] if T == 193 else [192, 192, 192, 124])
+    out = parity.gpu_forward(layer, "gemm")
+    parity.check_forward(layer, out, None, route)
 
 
 @pytest.mark.parametrize("T", [1, 7, 64, 128, 129, 300])
