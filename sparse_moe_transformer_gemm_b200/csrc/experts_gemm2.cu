@@ -626,6 +626,16 @@ __device__ __forceinline__ void widen_tile_fp4(uint32_t raw, uint32_t op, int ct
     }
 }
 
+// One thread's widened A row for every A tile of an op stage (tiles in
+// adjacent column ranges) into its TMEM lane: one tcgen05.st.
+template <int A_TILES>
+__device__ __forceinline__ void tc_store_row(uint32_t taddr, const uint32_t (&o)[A_TILES * 32]) {
+    if constexpr (A_TILES == 2)
+        tc::tmem_st64(taddr, o);
+    else
+        tc::tmem_st32(taddr, o);
+}
+
 // tmA: e4m3 weights [E * a_rows_per_expert, K] bytes, box 64 x 128, 64-byte
 // swizzle; FP4: E2M1 codes [E * a_rows_per_expert, K / 2] bytes, box 64 x 128
 // (two K blocks), no swizzle.
@@ -915,21 +925,20 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                                      : "=r"(w[a][4 * ch]), "=r"(w[a][4 * ch + 1]),
                                        "=r"(w[a][4 * ch + 2]), "=r"(w[a][4 * ch + 3])
                                      : "r"(raw + a * S::RAW_TILE + ((ch ^ rsw) << 4)));
-                uint32_t o[S::A_TILES][32];
+                uint32_t o[S::A_TILES * 32];  // tile a in o[32 a ..], its TMEM columns in order
 #pragma unroll
                 for (int a = 0; a < S::A_TILES; ++a)
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        e4m3x4_to_bf16x4<true>(w[a][j], o[a][2 * j], o[a][2 * j + 1]);
+                        e4m3x4_to_bf16x4<true>(w[a][j], o[32 * a + 2 * j], o[32 * a + 2 * j + 1]);
                 const bool ook = tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
                 if (tc::bar_any(2 + group, S::CONV_THREADS, !ook)) {
                     raise_timeout(c, status);
                     break;
                 }
                 tc::fence_after_sync();  // the MMAs that read this op stage are complete
-#pragma unroll
-                for (int a = 0; a < S::A_TILES; ++a)
-                    tc::tmem_st32(a_lane + os * S::A_STAGE_COLS + a * S::A_TILE_COLS, o[a]);
+                // the stage's A tiles are adjacent columns: one store (x64 for gate_up)
+                tc_store_row<S::A_TILES>(a_lane + os * S::A_STAGE_COLS, o);
                 tc::tmem_st_wait();
                 tc::fence_before_sync();
                 tc::bar_sync(2 + group, S::CONV_THREADS);
