@@ -340,10 +340,11 @@ def measure(args, name, dev, local, rank, world, pg, moe, block=False, cpu_secon
     dominant = max(("gate_up", "down"), key=lambda s: stage_ms[s])
     dom_work = gw if dominant == "gate_up" else dw
     dom_s = stage_ms[dominant] / 1e3
-    # quantised weights on shapes the SM-pair kernels do not take run on the
-    # streaming kernels (moe_api's automatic choice)
+    # quantised weights on shapes the SM-pair kernels do not take, and FP4 at up
+    # to one mean row per expert, run on the streaming kernels (the library's
+    # automatic choice, include/moe.h)
     use_stream = (args.path == "stream" or ((fp8 or fp4) and (d % 256 or F % 256)) or
-                  (fp4 and args.path == "auto" and T * k <= 4 * E))
+                  (fp4 and args.path == "auto" and T * k <= E))
     kernel_name = f"{dominant}_{'stream' if use_stream else 'gemm'}"
     # The metric's roofline: HBM for the decode workloads (weights streamed once),
     # dense bf16 tensor peak for the larger batches. A step lasts milliseconds,

@@ -36,9 +36,9 @@
  *   per 32 consecutive columns of a row, the block's scale 2^(b - 127)
  *   (b = 255 is not a scale: unspecified output). The weight value is
  *   code value * block scale. With neither path flag the experts run on the
- *   weight-streaming kernels at up to 4 mean rows per expert (T*k <= 4*E, the
- *   decode regime) and on the tensor-core SM-pair kernels above that (d, d_ff
- *   multiples of 256; the streaming kernels otherwise). MOE_FLAG_FP8_WEIGHTS,
+ *   weight-streaming kernels at up to one mean row per expert (T*k <= E) and
+ *   on the tensor-core SM-pair kernels above that (d, d_ff multiples of 256;
+ *   the streaming kernels otherwise). MOE_FLAG_FP8_WEIGHTS,
  *   MOE_FLAG_PACKED_WEIGHTS or MOE_FLAG_SHARED_EXPERT with it:
  *   MOE_ERR_INVALID_ARG.
  * - Packed bf16 weights (MOE_FLAG_PACKED_WEIGHTS): w_gate_up and w_down hold

@@ -423,89 +423,90 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 }
 
 // ======================================================================
-// FP8 (e4m3) weights. The MMA stays kind::f16 (bf16 x bf16, fp32 accumulate)
-// on weights widened on chip. Per K block, warp 0 TMA-loads this CTA's raw
-// e4m3 weight tile(s) (128 rows x 64 bytes, 64-byte swizzle) into a "raw" ring
-// on the CTA's own barrier; warp 15 loads its half of the token rows (bf16,
-// 128-byte swizzle) into a token ring completing on the even CTA's barrier.
-// Converter warps, in two groups of four that take K blocks round-robin (so
-// the conversion latencies of consecutive blocks overlap), widen the weights
-// exactly to bf16 straight into an "op" stage of tensor memory (below),
-// release the raw stage and arrive on the even CTA's operand barrier; the pair
-// MMA reads A from the op stage and B from the token stage and releases both.
-// The raw stages live only
-// from load to conversion, so their ring keeps the weight stream deep. The
-// per-output-row fp32 scale multiplies the finished dot product in the
-// epilogue (before SiLU for gate_up, before the bf16 store for down):
-// sum_c x_c q_c s_row = s_row sum_c x_c q_c. Every e4m3 value is a bf16
-// value, so the widening loses nothing.
+// Quantised expert weights: FP8 (e4m3 codes, fp32 per-output-row scale) and
+// FP4 (E2M1 codes, an E8M0 scale per 32 codes of a row). The MMA stays
+// kind::f16 (bf16 x bf16, fp32 accumulate) on weights widened exactly to bf16
+// on chip. Per K block, warp 0 TMA-loads this CTA's raw weight tile(s) (128
+// rows x 64 codes: 64 bytes of e4m3, 64-byte swizzle; 32 bytes of E2M1,
+// 32-byte swizzle) into a "raw" ring on the CTA's own barrier; warp 15 loads
+// its half of the token rows (bf16, 128-byte swizzle) into a token ring
+// completing on the even CTA's barrier. Converter warps, in two groups of
+// four that take K blocks round-robin (so the latencies of consecutive blocks
+// overlap), widen the weights into an "op" stage of tensor memory, release
+// the raw stage and arrive on the even CTA's operand barrier; the pair MMA
+// reads A from TMEM (tcgen05.mma [d], [a_tmem], b_desc) and B from the token
+// stage and releases both. The raw stages live only from load to conversion,
+// so their ring keeps the weight stream deep.
+//
+// FP8: the per-output-row fp32 scale multiplies the finished dot product in
+// the epilogue (before SiLU for gate_up, before the bf16 store for down):
+// sum_c x_c q_c s_row = s_row sum_c x_c q_c. Every e4m3 value is a bf16 value,
+// so the widening loses nothing. FP4: the block scale is folded into the
+// widening (every E2M1 value times a power of two is a bf16 value, below the
+// bf16 overflow), so the epilogue applies no scale.
+//
+// A goes straight into TMEM (tcgen05.st, one thread per A row): writing it
+// as a shared-memory tile instead ran the tensor pipe at ~51% against ~57%,
+// the tile's writes and the MMA's reads competing with the raw reads. TMEM
+// then holds the accumulators and the op stages, which caps a token tile at
+// NM = 192 rows: gate_up g and u (2 x 192 columns) + 2 op stages of 64
+// (gate + up); down two accumulator stages (2 x 192) + 4 op stages of 32.
+// (Half-K-block op stages, twice as many, measured 8% slower on B200 for
+// gate_up and 10% for down: twice the barrier and signal work for half the
+// conversion each.)
 
-constexpr int THREADS_FP8 = 512;        // warps 6-14 converters, warp 15 token producer
-constexpr int RAW_BYTES = BM * BK;      // one 128 x 64 e4m3 tile
-
-// FP8 (ATM): the converters write the widened A operand straight into tensor
-// memory (tcgen05.st, one thread per A row) and the pair MMA reads A from there,
-// so the operand tiles never pass through shared memory. TMEM then holds the
-// accumulators and the A stages, which caps an FP8 token tile at NM = 192 rows
-// (gate_up: g and u, 2 x 192 columns; down: 2 x 192). The remaining 128
-// columns hold the A stages, one K block each: 2 of 64 columns (gate + up)
-// for gate_up, 4 of 32 for down. (Half-K-block stages, twice as many, measured
-// 8% slower on B200 for gate_up and 10% for down: twice the barrier and signal
-// work for half the conversion each.)
-// FP4: E2M1 codes and E8M0 block scales folded into the widening (no row scale
-// in the epilogue), A in shared memory. A raw tile is 128 rows x 64 bytes,
-// which holds 128 codes a row: two K blocks (KPR) per raw stage.
-constexpr int MAX_RAW_STAGES = 16, MAX_B_STAGES = 4, MAX_OP_STAGES = 6;  // Fp8Ctrl's arrays
-template <bool GATE_UP, bool FP4 = false>
-struct Fp8Shape {
-    static constexpr bool ATM = !FP4;                              // A operand in TMEM
+constexpr int THREADS_Q = 512;        // warps 6-14 converters, warp 15 token producer
+constexpr int MAX_RAW_STAGES = 16, MAX_B_STAGES = 4, MAX_OP_STAGES = 4;  // QCtrl's arrays
+template <bool GATE_UP, bool FP4>
+struct QShape {
     static constexpr int A_TILES = GATE_UP ? 2 : 1;
-    static constexpr int KPR = FP4 ? 2 : 1;                        // K blocks per raw stage
-    static constexpr int NM = ATM ? 192 : NMAX;                    // token rows per pair tile
+    static constexpr int RAW_ROW = FP4 ? 32 : 64;                  // bytes of 64 codes
+    static constexpr int RAW_TILE = BM * RAW_ROW;                  // 128 rows
+    static constexpr int RAW_STAGE = A_TILES * RAW_TILE;
+    static constexpr int NM = 192;                                 // token rows per pair tile
     static constexpr int BH = (NM / 2) * BK * 2;                   // a CTA's token half (bytes)
-    static constexpr int RAW_TILE = RAW_BYTES;                     // 128 rows x 64 bytes
-    static constexpr int RAW_STAGE = A_TILES * RAW_TILE;           // 16 KB / 8 KB
-    static constexpr int OP_STAGE = ATM ? 0 : A_TILES * A_BYTES;   // shared-memory op stage
-    static constexpr int RAW_STAGES = ATM ? (GATE_UP ? 8 : 12) : (GATE_UP ? 4 : 6);
-    static constexpr int B_STAGES = ATM ? 4 : (GATE_UP ? 3 : 4);
-    static constexpr int OP_STAGES = ATM ? (GATE_UP ? 2 : 4) : (GATE_UP ? 3 : 6);
-    // converter warps: GROUPS groups of GROUP_WARPS take K blocks round-robin
-    // (ATM: four warps a group, one per TMEM lane quarter)
-    static constexpr int GROUPS = ATM ? 2 : (GATE_UP ? 2 : 3);
-    static constexpr int GROUP_WARPS = ATM ? 4 : (GATE_UP ? 4 : 3);
+    static constexpr int RAW_STAGES = FP4 ? 16 : (GATE_UP ? 8 : 12);
+    static constexpr int B_STAGES = 4;
+    static constexpr int OP_STAGES = GATE_UP ? 2 : 4;
+    // converter warps: GROUPS groups of four (one per TMEM lane quarter) take
+    // K blocks round-robin
+    static constexpr int GROUPS = 2;
+    static constexpr int GROUP_WARPS = 4;
     static constexpr int CONV_THREADS = GROUP_WARPS * 32;
-    static constexpr int RING_BYTES =
-        RAW_STAGES * RAW_STAGE + B_STAGES * BH + OP_STAGES * OP_STAGE;
+    // FP4 scale chunks (8 bytes of a row: 4 K blocks), per converter group
+    static constexpr int SC_STAGES = 4;
+    static constexpr int SC_BYTES = FP4 ? GROUPS * SC_STAGES * A_TILES * BM * 8 : 0;
+    static constexpr int RING_BYTES = RAW_STAGES * RAW_STAGE + B_STAGES * BH + SC_BYTES;
     static constexpr int ACC_STAGES = GATE_UP ? 1 : 2;
-    // TMEM columns: the accumulators, then (ATM) the A stages
-    static constexpr int U_OFF = ATM ? NM : 256;                   // gate_up's up accumulator
-    static constexpr int ACC_COLS = GATE_UP ? 2 * U_OFF : (ATM ? NM : 256);
+    // TMEM columns: the accumulators, then the op stages
+    static constexpr int U_OFF = NM;                               // gate_up's up accumulator
+    static constexpr int ACC_COLS = GATE_UP ? 2 * NM : NM;
     static constexpr int A_COL = ACC_STAGES * ACC_COLS;
     static constexpr int A_TILE_COLS = BK / 2;                     // one tile's K block: two bf16 a column
     static constexpr int A_STAGE_COLS = A_TILES * A_TILE_COLS;
 };
 
-constexpr int CONV_WARPS = 9;                          // warps 6..14 (some idle for gate_up)
+constexpr int CONV_WARPS = 9;                          // warps 6..14 (warp 14 idles)
 constexpr int TOKEN_WARP = 6 + CONV_WARPS;
 template <bool G, bool FP4>
-constexpr bool groups_ok() {
-    using S = Fp8Shape<G, FP4>;
-    return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES >= S::KPR * S::GROUPS - 1 &&
-           S::OP_STAGES >= S::GROUPS && S::GROUPS * S::GROUP_WARPS <= CONV_WARPS &&
+constexpr bool shape_ok() {
+    using S = QShape<G, FP4>;
+    return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES % S::GROUPS == 0 &&
+           S::GROUPS * S::GROUP_WARPS <= CONV_WARPS && S::GROUP_WARPS == 4 &&
            S::RAW_STAGES <= MAX_RAW_STAGES && S::B_STAGES <= MAX_B_STAGES &&
-           S::OP_STAGES <= MAX_OP_STAGES && (!S::ATM || S::GROUP_WARPS == 4) &&
-           (!S::ATM || S::A_COL + S::OP_STAGES * S::A_STAGE_COLS <= 512) &&
-           S::ACC_STAGES * S::ACC_COLS <= 512 && S::BH % 1024 == 0;
+           S::OP_STAGES <= MAX_OP_STAGES && S::A_COL + S::OP_STAGES * S::A_STAGE_COLS <= 512 &&
+           S::BH % 1024 == 0 && S::RAW_TILE % 1024 == 0;
 }
-// Each group owns whole raw stages, and a group's previous operand wait proves
-// that the stage's last reader finished (parity waits cannot see a stale phase);
-// every stage index stays inside Fp8Ctrl's barrier arrays.
-static_assert(groups_ok<true, false>() && groups_ok<false, false>() && groups_ok<true, true>() &&
-                  groups_ok<false, true>(),
-              "converter grouping");
-static_assert(THREADS_FP8 == 32 * (TOKEN_WARP + 1), "warp roles cover the block");
+// Each group owns whole raw stages and op stages (both ring lengths are
+// multiples of GROUPS), and a group's previous wait on a stage proves that its
+// last reader finished (parity waits cannot see a stale phase); every stage
+// index stays inside QCtrl's barrier arrays.
+static_assert(shape_ok<true, false>() && shape_ok<false, false>() && shape_ok<true, true>() &&
+                  shape_ok<false, true>(),
+              "quantised pair GEMM shape");
+static_assert(THREADS_Q == 32 * (TOKEN_WARP + 1), "warp roles cover the block");
 
-struct Fp8Ctrl {
+struct QCtrl {
     uint64_t raw_full[MAX_RAW_STAGES];   // each CTA: its raw weight tile(s) landed
     uint64_t raw_empty[MAX_RAW_STAGES];  // each CTA: the converters are done with the raw stage
     uint64_t b_full[MAX_B_STAGES];       // even CTA: token bytes of both CTAs landed
@@ -524,15 +525,23 @@ struct Fp8Ctrl {
     int tile_start[MAX_E + 1];
 };
 
-constexpr int FP8_EPI_BYTES = EPI_N * BM * 2;  // one [32 tokens][128 rows] bf16 staging tile
+constexpr int Q_EPI_BYTES = EPI_N * BM * 2;  // one [32 tokens][128 rows] bf16 staging tile
 
 template <bool GATE_UP, bool FP4>
-constexpr int fp8_smem_bytes() {
-    return Fp8Shape<GATE_UP, FP4>::RING_BYTES + FP8_EPI_BYTES + 1024 + (int)sizeof(Fp8Ctrl);
+constexpr int q_smem_bytes() {
+    return QShape<GATE_UP, FP4>::RING_BYTES + Q_EPI_BYTES + 1024 + (int)sizeof(QCtrl);
 }
-static_assert(fp8_smem_bytes<true, false>() <= 232448 && fp8_smem_bytes<false, false>() <= 232448 &&
-                  fp8_smem_bytes<true, true>() <= 232448 && fp8_smem_bytes<false, true>() <= 232448,
+static_assert(q_smem_bytes<true, false>() <= 232448 && q_smem_bytes<false, false>() <= 232448 &&
+                  q_smem_bytes<true, true>() <= 232448 && q_smem_bytes<false, true>() <= 232448,
               "fits in 227 KB");
+
+// A bf16x2 multiply kept in program order with respect to the waits around it
+// (volatile), so that a conversion stays ahead of the wait that follows it.
+__device__ __forceinline__ uint32_t mul_bf16x2_here(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm volatile("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 
 // Four e4m3 codes (one 32-bit word, code i in byte i) -> four bf16 in two
 // bf16x2 words (codes 0, 1 in lo; 2, 3 in hi; the even code in the low half),
@@ -546,84 +555,33 @@ static_assert(fp8_smem_bytes<true, false>() <= 232448 && fp8_smem_bytes<false, f
 // (bf16 0x7B80: a power of two, exact, subnormal inputs included) restores
 // it. Signed zeros carry over. NaN codes (S.1111.111) give a finite value:
 // NaN weights are unspecified.
-__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-// The same multiply kept in program order with respect to the waits around it
-// (volatile), so that a conversion stays ahead of the wait that follows it.
-__device__ __forceinline__ uint32_t mul_bf16x2_here(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm volatile("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-template <bool HERE = false>
 __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
     constexpr uint32_t kTwoPow120 = 0x7B807B80u;  // bf16x2 (2^120, 2^120)
-    const uint32_t a = e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x1404));
-    const uint32_t b = e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x3424));
-    lo = HERE ? mul_bf16x2_here(a, kTwoPow120) : mul_bf16x2(a, kTwoPow120);
-    hi = HERE ? mul_bf16x2_here(b, kTwoPow120) : mul_bf16x2(b, kTwoPow120);
+    lo = mul_bf16x2_here(e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x1404)), kTwoPow120);
+    hi = mul_bf16x2_here(e4m3_pair_scaled_bits(__byte_perm(w, 0u, 0x3424)), kTwoPow120);
 }
 
-// Convert one K block of a raw E2M1 tile (128 rows x 64 bytes, row-major, two K
-// blocks a row: K block `sub` in bytes 32 sub..32 sub + 31; code 2i of a row in
-// the low nibble of its byte i) into a bf16 operand tile (128 rows x 128
-// bytes, 128-byte swizzle). Thread `ct` handles 16-byte chunks q = ct +
-// CONV_THREADS i: row q/2, codes 32(q%2)..32(q%2)+31 of the K block, exactly
-// one E8M0 scale block, whose byte b is sc[i]. Each byte of codes becomes a bf16 pair worth
-// value * 2^-126 (e2m1_pair_scaled_bits); one bf16x2 multiply by 2^(b-1) -- a
-// normal bf16 for b <= 128 -- gives value * 2^(b-127) exactly; for b > 128 it
-// is two multiplies, by 2^126 and by 2^(b-127). Products of magnitude >=
-// 2^128 (b >= 253) overflow, as the value itself does in bf16.
-template <int CONV_THREADS>
-constexpr int fp4_per() {
-    return (256 + CONV_THREADS - 1) / CONV_THREADS;
-}
-template <int CONV_THREADS>
-__device__ __forceinline__ void widen_tile_fp4(uint32_t raw, uint32_t op, int ct, int sub,
-                                               const uint32_t (&sc)[fp4_per<CONV_THREADS>()]) {
-    constexpr int PER = fp4_per<CONV_THREADS>();
-    uint32_t w[PER][4];
+// 32 E2M1 codes (16 bytes: code 2i in the low nibble of byte i) of one scale
+// block, whose E8M0 byte is b -> 16 bf16x2 words (byte i -> word i, the even
+// code in the low half), exactly: each byte becomes a bf16 pair worth value *
+// 2^-126 (e2m1_pair_scaled_bits); one bf16x2 multiply by 2^(b-1) -- a normal
+// bf16 for b <= 128 -- gives value * 2^(b-127); for b > 128 it is two
+// multiplies, by 2^126 and by 2^(b-127). Products of magnitude >= 2^128
+// (b >= 253) overflow, as the value itself does in bf16.
+__device__ __forceinline__ void e2m1x32_to_bf16(const uint32_t* w, uint32_t b, uint32_t* o) {
+    const bool one = b <= 128u;
+    const uint32_t f1 = one ? ((b + 126u) << 7) : 0x7E80u;  // 2^(b-1) or 2^126
+    const uint32_t f1x2 = f1 | (f1 << 16);
+    const uint32_t f2x2 = (b << 7) | (b << 23);              // 2^(b-127), used if b > 128
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int q = ct + i * CONV_THREADS;
-        if (q < 256)  // raw rows hold two K blocks (64 bytes): this one at 32 * sub
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w[i][0]), "=r"(w[i][1]), "=r"(w[i][2]), "=r"(w[i][3])
-                         : "r"(raw + (q >> 1) * 64 + sub * 32 + (q & 1) * 16));
-    }
+    for (int j4 = 0; j4 < 4; ++j4)
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int q = ct + i * CONV_THREADS;
-        if (q >= 256) break;
-        const int row = q >> 1, half = q & 1;
-        const uint32_t b = sc[i];
-        const bool one = b <= 128u;
-        const uint32_t f1 = one ? ((b + 126u) << 7) : 0x7E80u;  // 2^(b-1) or 2^126
-        const uint32_t f1x2 = f1 | (f1 << 16);
-        const uint32_t f2x2 = (b << 7) | (b << 23);                // 2^(b-127), used if b > 128
-        uint32_t o[16];
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint32_t v = e2m1_pair_scaled_bits(__byte_perm(w[i][j4], 0u, 0x4440u | j));
-                v = mul_bf16x2(v, f1x2);
-                if (!one) v = mul_bf16x2(v, f2x2);
-                o[4 * j4 + j] = v;
-            }
+        for (int j = 0; j < 4; ++j) {
+            uint32_t v = e2m1_pair_scaled_bits(__byte_perm(w[j4], 0u, 0x4440u | j));
+            v = mul_bf16x2_here(v, f1x2);
+            if (!one) v = mul_bf16x2_here(v, f2x2);
+            o[4 * j4 + j] = v;
         }
-        const uint32_t rbase = op + row * 128;
-        const int sw = row & 7;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             rbase + (((4 * half + k) ^ sw) << 4)),
-                         "r"(o[4 * k]), "r"(o[4 * k + 1]), "r"(o[4 * k + 2]), "r"(o[4 * k + 3])
-                         : "memory");
-    }
 }
 
 // One thread's widened A row for every A tile of an op stage (tiles in
@@ -636,31 +594,30 @@ __device__ __forceinline__ void tc_store_row(uint32_t taddr, const uint32_t (&o)
         tc::tmem_st32(taddr, o);
 }
 
-// tmA: e4m3 weights [E * a_rows_per_expert, K] bytes, box 64 x 128, 64-byte
-// swizzle; FP4: E2M1 codes [E * a_rows_per_expert, K / 2] bytes, box 64 x 128
-// (two K blocks), no swizzle.
-// tmB: token rows [R, K] bf16, box 64 x 16. scales_v: FP8 fp32 row scales
-// [E * a_rows_per_expert]; FP4 E8M0 block scales [E * a_rows_per_expert, K / 32]
-// bytes.
+// tmA: FP8 e4m3 weights [E * a_rows_per_expert, K] bytes, box 64 x 128,
+// 64-byte swizzle; FP4 E2M1 codes [E * a_rows_per_expert, K / 2] bytes, box 32
+// x 128, 32-byte swizzle. tmB: token rows [R, K] bf16, boxes of 16..128 rows x
+// 64. scales_v: FP8 fp32 row scales [E * a_rows_per_expert]; FP4 E8M0 block
+// scales [E * a_rows_per_expert, K / 32] bytes.
 template <bool GATE_UP, bool FP4>
-__global__ void __launch_bounds__(THREADS_FP8, 1)
+__global__ void __launch_bounds__(THREADS_Q, 1)
 grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ TokenMaps tmB,
                              const int* __restrict__ offsets, const void* __restrict__ scales_v,
                              int E, int K, int a_rows_per_expert, int m_tiles,
                              __nv_bfloat16* __restrict__ out, int out_ld,
                              int* __restrict__ status) {
-    using S = Fp8Shape<GATE_UP, FP4>;
+    using S = QShape<GATE_UP, FP4>;
     const float* __restrict__ scales = static_cast<const float*>(scales_v);
     const uint8_t* __restrict__ scales8 = static_cast<const uint8_t*>(scales_v);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* op_ring = smem;  // 1024-aligned operand stages first
-    uint8_t* b_ring = op_ring + S::OP_STAGES * S::OP_STAGE;
+    uint8_t* b_ring = smem;  // 1024-aligned stages
     uint8_t* raw_ring = b_ring + S::B_STAGES * S::BH;
+    uint8_t* sc_ring = raw_ring + S::RAW_STAGES * S::RAW_STAGE;  // FP4 only
     uint16_t* epi = reinterpret_cast<uint16_t*>(smem + S::RING_BYTES);
-    Fp8Ctrl& c = *reinterpret_cast<Fp8Ctrl*>(smem + S::RING_BYTES + FP8_EPI_BYTES);
+    QCtrl& c = *reinterpret_cast<QCtrl*>(smem + S::RING_BYTES + Q_EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)(tc::cluster_ctarank() & 1u);
     const bool leader = rank == 0;
@@ -731,7 +688,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- raw e4m3 weight producer (this CTA's rows, own barrier)
+            // ---------------- raw weight producer (this CTA's rows, own barrier)
             const uint64_t pol_w = tc::policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
@@ -741,7 +698,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int t = pair; t < total && ok; t += n_pairs) {
                 const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, t);
                 const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
-                for (int kr = 0; kr < KB / S::KPR; ++kr) {  // raw blocks of KPR K blocks
+                for (int kb = 0; kb < KB; ++kb) {
                     if (!tc::mbar_wait(&c.raw_empty[stage], phase ^ 1u, abort_flag)) {
                         raise_timeout(c, status);
                         ok = false;
@@ -749,7 +706,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                     uint8_t* st = raw_ring + stage * S::RAW_STAGE;
                     tc::mbar_arrive_expect_tx(&c.raw_full[stage], S::RAW_STAGE);
-                    const int kx = kr * BK;  // byte column: 64 e4m3 codes or 128 E2M1 codes
+                    const int kx = kb * S::RAW_ROW;  // byte column of the K block's 64 codes
                     tc::tma_load_2d_hint(st, &tmA, &c.raw_full[stage], kx, a_row, pol_w);
                     if (GATE_UP)
                         tc::tma_load_2d_hint(st + S::RAW_TILE, &tmA, &c.raw_full[stage], kx,
@@ -805,152 +762,149 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     atomicExch(status, MOE_ERR_TIMEOUT);
         }
     } else if (warp >= 6 && warp < 6 + CONV_WARPS) {
-        // ---------------- converters: raw codes -> bf16 operand (A) in the op stage
-        // (FP8: TMEM columns; FP4: a shared-memory tile). A group's threads
-        // complete their writes (FP8: tcgen05.wait::st and the tcgen05 fence;
-        // FP4: a fence to the async proxy) and meet at a named barrier; then one
-        // thread releases the raw stage and signals the even CTA's op_full: in
-        // the even CTA a local arrive that expects 16 bytes, in the odd CTA a
-        // 16-byte shared-to-shared bulk copy into the even CTA that completes on
-        // that barrier (an async-proxy operation issued after the completed
-        // writes). A remote mbarrier arrive with cluster-scope release, the
-        // other way to signal across the pair, stalled its warp ~1.5k cycles per
-        // K block on B200 -- longer than the widening itself. The group agrees
-        // on its bounded waits (bar.red.or) and leaves together; the MMA's
-        // bounded wait on op_full then gives up.
+        // ---------------- converters: raw codes -> bf16 A rows in a TMEM op stage.
+        // Each thread widens one A row of this CTA -- row r = 32 (warp % 4) +
+        // lane, the TMEM lane its warp may write -- for every A tile of the K
+        // block: the 64 codes of its raw row (the swizzle puts the eight rows of
+        // a quarter-warp's 16-byte loads on distinct banks: chunk c of row r
+        // sits at chunk c ^ ((r / 2) % 4) for e4m3, c ^ ((r / 4) % 2) for E2M1)
+        // into 32 TMEM columns (two bf16 a column, the even K index in the low
+        // half). A group converts the K blocks j = group, group + GROUPS, ...
+        // (warp 14 idles). The widening runs before the wait for the op stage.
+        //
+        // The group's threads complete their stores (tcgen05.wait::st, then the
+        // tcgen05 fence) and meet at a named barrier; then one thread releases
+        // the raw stage and signals the even CTA's op_full: in the even CTA a
+        // local arrive that expects 16 bytes, in the odd CTA a 16-byte
+        // shared-to-shared bulk copy into the even CTA that completes on that
+        // barrier. A remote mbarrier arrive with cluster-scope release, the
+        // other way to signal across the pair, stalled its warp ~1.5k cycles
+        // per K block on B200 -- longer than the widening itself. The group
+        // agrees on its bounded waits (bar.red.or) and leaves together; the
+        // MMA's bounded wait on op_full then gives up.
         const int group = (warp - 6) / S::GROUP_WARPS;
         const int ct = threadIdx.x - 192 - group * S::CONV_THREADS;  // 0..CONV_THREADS-1
-        const uint32_t raw0 = tc::smem_u32(raw_ring), op0 = tc::smem_u32(op_ring);
+        const int r = 32 * (warp & 3) + lane;
+        const uint32_t rsw = FP4 ? (uint32_t)((r >> 2) & 1) : (uint32_t)((r >> 1) & 3);
+        const uint32_t raw0 = tc::smem_u32(raw_ring) + r * S::RAW_ROW;
+        const uint32_t a_lane = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + S::A_COL;
         // this CTA's K blocks in order: j = tile_iteration * KB + kb
         int n_my_tiles = 0;
         for (int t = pair; t < total; t += n_pairs) ++n_my_tiles;
-        // signal one op stage (see above); ct == 0 of the group, after its barrier
-        auto signal_op = [&](int os) {
-            if (leader)
-                tc::mbar_arrive_expect_tx(&c.op_full[os], 16);
-            else
-                tc::bulk_copy_smem_to_cluster(tc::map_to_cta(tc::smem_u32(&c.sig[os][0]), 0),
-                                              tc::smem_u32(&c.sig_src[0]), 16,
-                                              tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
-        };
-        if constexpr (FP4) {
-            // A group takes raw blocks jr = group, group + GROUPS, ... and turns each
-            // into the op blocks 2 jr and 2 jr + 1. The op wait for block b stays
-            // unambiguous: the group's previous op wait (block b - 1, or
-            // b - 2 GROUPS + 1) saw the MMA finish block b - 2 GROUPS + 1 - OP_STAGES
-            // >= b - 2 OP_STAGES (OP_STAGES >= 2 GROUPS - 1), so stage b % OP_STAGES
-            // has completed b / OP_STAGES - 1 or b / OP_STAGES phases, never fewer.
-            constexpr int PER4 = fp4_per<S::CONV_THREADS>();
-            const long n_raw = (long)n_my_tiles * (KB / 2);
-            for (long jr = (group < S::GROUPS ? group : n_raw); jr < n_raw; jr += S::GROUPS) {
-                const int rs = (int)(jr % S::RAW_STAGES);
-                const uint32_t rph = (uint32_t)(jr / S::RAW_STAGES) & 1u;
-                const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
-                if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
-                    raise_timeout(c, status);
-                    break;
-                }
-                const uint32_t raw = raw0 + rs * S::RAW_STAGE;
-                bool failed = false;
-                for (int sub = 0; sub < 2; ++sub) {
-                    const long jb = 2 * jr + sub;
-                    const int os = (int)(jb % S::OP_STAGES);
-                    const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
-                    // this thread's block scales, loaded before the op wait
-                    uint32_t sc[S::A_TILES][PER4];
-                    const long it = jb / KB;
-                    const int kb = (int)(jb - it * KB);
+        const long n_blocks = (long)n_my_tiles * KB;
+        // FP4: the scale bytes of this thread's rows come as 8-byte chunks, one
+        // per 4 K blocks (the 32-code blocks 8 q .. 8 q + 7 of the row): chunk
+        // G = j / 4 of the CTA's block sequence, which the group uses for two of
+        // its blocks. Each thread copies its own chunks into a ring of SC_STAGES
+        // shared-memory slots with cp.async, SC_STAGES - 1 chunks ahead (loads
+        // into registers one or two blocks ahead left the converters waiting
+        // on them), and reads chunk G when the group reaches it.
+        const long n_chunks = n_blocks / 4;  // K blocks per tile: a multiple of 4
+        const long sblocks = K / 32;
+        const uint32_t sc_slot0 =
+            tc::smem_u32(sc_ring) + (uint32_t)(group * S::SC_STAGES * S::A_TILES * BM * 8 + r * 8);
+        long fetch_it = -1, fetch_row = 0;  // the tile of the last fetch and its row
+        auto fetch_chunk = [&](long G) {  // one copy group per chunk, empty past the end
+            if (G < n_chunks) {
+                const long it = G / (KB / 4);
+                const int q = (int)(G - it * (KB / 4));
+                if (it != fetch_it) {  // a new tile: one lookup per tile, not per chunk
                     const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, pair + (int)it * n_pairs);
-                    const long a_row = (long)ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
-                    const long blocks = K / 32;
+                    fetch_row = (long)ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM + r;
+                    fetch_it = it;
+                }
+                const long row = fetch_row;
+                const uint32_t dst = sc_slot0 + (uint32_t)((G % S::SC_STAGES) * S::A_TILES * BM * 8);
+#pragma unroll
+                for (int a = 0; a < S::A_TILES; ++a)
+                    tc::cp_async8(dst + a * BM * 8,
+                                  scales8 + (row + a * (a_rows_per_expert / 2)) * sblocks + 8 * q);
+            }
+            tc::cp_async_commit();
+        };
+        uint2 sc_cur[S::A_TILES] = {};
+        long cur_chunk = -1;
+        const long j0 = group < S::GROUPS ? group : n_blocks;
+        if (FP4 && j0 < n_blocks)
+            for (int g = 0; g < S::SC_STAGES - 1; ++g) fetch_chunk((j0 >> 2) + g);
+        for (long jb = j0; jb < n_blocks; jb += S::GROUPS) {
+            const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
+            const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
+            const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
+            uint32_t sc[S::A_TILES] = {};  // FP4: this block's two scale bytes per A tile
+            if constexpr (FP4) {
+                if ((jb >> 2) != cur_chunk) {
+                    cur_chunk = jb >> 2;
+                    // the slot of chunk G + SC_STAGES - 1 held chunk G - 1, read already
+                    fetch_chunk(cur_chunk + S::SC_STAGES - 1);
+                    tc::cp_async_wait_pending<S::SC_STAGES - 1>();  // chunk G has landed
+                    const uint32_t src =
+                        sc_slot0 + (uint32_t)((cur_chunk % S::SC_STAGES) * S::A_TILES * BM * 8);
 #pragma unroll
                     for (int a = 0; a < S::A_TILES; ++a)
-#pragma unroll
-                        for (int i = 0; i < PER4; ++i) {
-                            const int q = ct + i * S::CONV_THREADS;
-                            const long row = a_row + a * (a_rows_per_expert / 2) + (q >> 1);
-                            sc[a][i] = q < 256 ? __ldg(scales8 + row * blocks + 2 * kb + (q & 1)) : 0u;
-                        }
-                    const bool ook = tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
-                    if (tc::bar_any(2 + group, S::CONV_THREADS, !ook)) {
-                        raise_timeout(c, status);
-                        failed = true;
-                        break;
-                    }
-                    const uint32_t op = op0 + os * S::OP_STAGE;
-                    widen_tile_fp4<S::CONV_THREADS>(raw, op, ct, sub, sc[0]);
-                    if (GATE_UP)
-                        widen_tile_fp4<S::CONV_THREADS>(raw + S::RAW_TILE, op + A_BYTES, ct, sub,
-                                                        sc[S::A_TILES - 1]);
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    tc::bar_sync(2 + group, S::CONV_THREADS);
-                    if (ct == 0) {
-                        if (sub == 1) tc::mbar_arrive(&c.raw_empty[rs]);  // both K blocks read
-                        signal_op(os);
-                    }
+                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                     : "=r"(sc_cur[a].x), "=r"(sc_cur[a].y)
+                                     : "r"(src + a * BM * 8));
                 }
-                if (failed) break;
+                const int kq = (int)(jb & 3);  // the block's place in its chunk
+#pragma unroll
+                for (int a = 0; a < S::A_TILES; ++a)
+                    sc[a] = ((kq < 2 ? sc_cur[a].x : sc_cur[a].y) >> (16 * (kq & 1))) & 0xFFFFu;
             }
-        } else if constexpr (S::ATM) {
-            // Each thread widens one A row of this CTA -- row r = 32 (warp % 4) +
-            // lane, the TMEM lane its warp may write -- for every A tile of the K
-            // block: the 64 codes of its raw row (64-byte rows, 64-byte swizzle:
-            // 16-byte chunk c of row r sits at chunk c ^ ((r / 2) % 4), so that
-            // the eight rows of a quarter-warp hit distinct banks) into 32 TMEM
-            // columns (two bf16 a column, the even K index in the low half). A
-            // group converts the K blocks j = group, group + GROUPS, ... (warps
-            // past the groups idle). The widening runs before the wait for the op
-            // stage; the writes complete (tcgen05.wait::st) before the group's
-            // barrier and the signal.
-            const int r = 32 * (warp & 3) + lane;
-            const uint32_t rsw = (uint32_t)((r >> 1) & 3);
-            const uint32_t a_lane = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + S::A_COL;
-            const long n_blocks = (long)n_my_tiles * KB;
-            for (long jb = (group < S::GROUPS ? group : n_blocks); jb < n_blocks; jb += S::GROUPS) {
-                const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
-                const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
-                const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
-                const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
-                if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
-                    raise_timeout(c, status);
-                    break;
-                }
-                const uint32_t raw = raw0 + rs * S::RAW_STAGE + r * 64;
-                uint32_t w[S::A_TILES][16];
+            const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
+            if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
+                raise_timeout(c, status);
+                break;
+            }
+            const uint32_t raw = raw0 + rs * S::RAW_STAGE;
+            constexpr int CHUNKS = S::RAW_ROW / 16;
+            uint32_t w[S::A_TILES][4 * CHUNKS];
 #pragma unroll
-                for (int a = 0; a < S::A_TILES; ++a)
+            for (int a = 0; a < S::A_TILES; ++a)
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch)
-                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(w[a][4 * ch]), "=r"(w[a][4 * ch + 1]),
-                                       "=r"(w[a][4 * ch + 2]), "=r"(w[a][4 * ch + 3])
-                                     : "r"(raw + a * S::RAW_TILE + ((ch ^ rsw) << 4)));
-                uint32_t o[S::A_TILES * 32];  // tile a in o[32 a ..], its TMEM columns in order
+                for (int ch = 0; ch < CHUNKS; ++ch)
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[a][4 * ch]), "=r"(w[a][4 * ch + 1]),
+                                   "=r"(w[a][4 * ch + 2]), "=r"(w[a][4 * ch + 3])
+                                 : "r"(raw + a * S::RAW_TILE + ((ch ^ rsw) << 4)));
+            uint32_t o[S::A_TILES * 32];  // tile a in o[32 a ..], its TMEM columns in order
 #pragma unroll
-                for (int a = 0; a < S::A_TILES; ++a)
+            for (int a = 0; a < S::A_TILES; ++a) {
+                if constexpr (FP4) {
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch)
+                        e2m1x32_to_bf16(&w[a][4 * ch], (sc[a] >> (8 * ch)) & 0xFFu,
+                                        &o[32 * a + 16 * ch]);
+                } else {
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        e4m3x4_to_bf16x4<true>(w[a][j], o[32 * a + 2 * j], o[32 * a + 2 * j + 1]);
-                const bool ook = tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
-                if (tc::bar_any(2 + group, S::CONV_THREADS, !ook)) {
-                    raise_timeout(c, status);
-                    break;
-                }
-                tc::fence_after_sync();  // the MMAs that read this op stage are complete
-                // the stage's A tiles are adjacent columns: one store (x64 for gate_up)
-                tc_store_row<S::A_TILES>(a_lane + os * S::A_STAGE_COLS, o);
-                tc::tmem_st_wait();
-                tc::fence_before_sync();
-                tc::bar_sync(2 + group, S::CONV_THREADS);
-                if (ct == 0) {
-                    tc::mbar_arrive(&c.raw_empty[rs]);
-                    signal_op(os);
+                        e4m3x4_to_bf16x4(w[a][j], o[32 * a + 2 * j], o[32 * a + 2 * j + 1]);
                 }
             }
+            const bool ook = tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
+            if (tc::bar_any(2 + group, S::CONV_THREADS, !ook)) {
+                raise_timeout(c, status);
+                break;
+            }
+            tc::fence_after_sync();  // the MMAs that read this op stage are complete
+            tc_store_row<S::A_TILES>(a_lane + os * S::A_STAGE_COLS, o);
+            tc::tmem_st_wait();
+            tc::fence_before_sync();
+            tc::bar_sync(2 + group, S::CONV_THREADS);
+            if (ct == 0) {
+                tc::mbar_arrive(&c.raw_empty[rs]);
+                if (leader)
+                    tc::mbar_arrive_expect_tx(&c.op_full[os], 16);
+                else
+                    tc::bulk_copy_smem_to_cluster(tc::map_to_cta(tc::smem_u32(&c.sig[os][0]), 0),
+                                                  tc::smem_u32(&c.sig_src[0]), 16,
+                                                  tc::map_to_cta(tc::smem_u32(&c.op_full[os]), 0));
+            }
         }
+        if constexpr (FP4) tc::cp_async_wait_pending<0>();  // no copy outlives the loop
     } else if (warp == 1) {
         if (lane == 0 && leader) {
-            // ---------------- MMA issuer (even CTA): A from the op stage (FP8: in TMEM), B from the token stage
+            // ---------------- MMA issuer (even CTA): A from the TMEM op stage, B from the token stage
             int bs = 0, os = 0;
             uint32_t oph = 0, bph = 0;
             bool ok = true;
@@ -974,27 +928,17 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                         break;
                     }
                     tc::fence_after_sync();
-                    const uint32_t a_addr = tc::smem_u32(op_ring + os * S::OP_STAGE);
                     const uint32_t a_tm = tmem_base + S::A_COL + os * S::A_STAGE_COLS;
                     const uint32_t b_addr = tc::smem_u32(b_ring + bs * S::BH);
 #pragma unroll
-                    for (int k = 0; k < BK / UK; ++k) {
+                    for (int k = 0; k < BK / UK; ++k) {  // K = 16 of A is 8 TMEM columns
                         const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                        if constexpr (S::ATM) {  // K = 16 of A is 8 TMEM columns
-                            tc::mma_bf16_pair_ta(d_tmem, a_tm + k * (UK / 2), bdesc, idesc, accum);
-                            if (GATE_UP)
-                                tc::mma_bf16_pair_ta(d_tmem + S::U_OFF,
-                                                     a_tm + S::A_TILE_COLS + k * (UK / 2), bdesc,
-                                                     idesc, accum);
-                        } else {
-                            tc::mma_bf16_pair(d_tmem, tc::desc_sw128(a_addr + k * UK * 2), bdesc,
-                                              idesc, accum);
-                            if (GATE_UP)
-                                tc::mma_bf16_pair(d_tmem + S::U_OFF,
-                                                  tc::desc_sw128(a_addr + A_BYTES + k * UK * 2),
-                                                  bdesc, idesc, accum);
-                        }
+                        tc::mma_bf16_pair_ta(d_tmem, a_tm + k * (UK / 2), bdesc, idesc, accum);
+                        if (GATE_UP)
+                            tc::mma_bf16_pair_ta(d_tmem + S::U_OFF,
+                                                 a_tm + S::A_TILE_COLS + k * (UK / 2), bdesc,
+                                                 idesc, accum);
                     }
                     tc::mma_commit_pair(&c.op_empty[os], 0x3);
                     tc::mma_commit_pair(&c.b_empty[bs], 0x3);
@@ -1116,9 +1060,9 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 // Row-major [rows, cols] bytes (e4m3 codes, or E2M1 code pairs), box of
-// box_rows x box_cols bytes, no swizzle or (box_cols = 64) the 64-byte swizzle.
+// box_rows x box_cols bytes with the given swizzle (box_cols at most its span).
 bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                 uint32_t box_rows, uint32_t box_cols = BK, bool swizzle64 = false) {
+                 uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle swizzle) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
@@ -1126,9 +1070,7 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE,
-              swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1185,13 +1127,13 @@ template <bool GATE_UP, bool FP4 = false>
 cudaError_t launch_fp8(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets,
                        const void* scales, int E, int K, int a_rows_per_expert, int m_tiles,
                        void* out, int out_ld, int* status, cudaStream_t s) {
-    const int smem = fp8_smem_bytes<GATE_UP, FP4>();
+    const int smem = q_smem_bytes<GATE_UP, FP4>();
     cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_fp8_kernel<GATE_UP, FP4>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * sm_pairs(), 1, 1);
-    cfg.blockDim = dim3(THREADS_FP8, 1, 1);
+    cfg.blockDim = dim3(THREADS_Q, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -1219,7 +1161,7 @@ cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm
     CUtensorMap a;
     TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
-    if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM, BK, true) ||
+    if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, BM, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_token_maps(&b, x_perm, R, c.d))
         return cudaErrorInvalidValue;
     return launch_fp8<true>(a, b, offsets, s_gate_up, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), h,
@@ -1232,7 +1174,7 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
     CUtensorMap a;
     TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
-    if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM, BK, true) ||
+    if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
     return launch_fp8<false>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d,
@@ -1246,7 +1188,7 @@ cudaError_t launch_gate_up_gemm_pair_fp4(const moe_config& c, const void* x_perm
     CUtensorMap a;
     TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
-    if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d / 2, BM) ||
+    if (!make_map_u8(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d / 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_32B) ||
         !make_token_maps(&b, x_perm, R, c.d))
         return cudaErrorInvalidValue;
     return launch_fp8<true, true>(a, b, offsets, s_gate_up, c.E, c.d, 2 * c.d_ff,
@@ -1259,7 +1201,7 @@ cudaError_t launch_down_gemm_pair_fp4(const moe_config& c, const void* h, const 
     CUtensorMap a;
     TokenMaps b;
     const uint64_t R = (uint64_t)c.T * c.k;
-    if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff / 2, BM) ||
+    if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff / 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_32B) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
     return launch_fp8<false, true>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y,

@@ -79,11 +79,12 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA
 // FP8 and FP4 weights have a tensor-core path on SM pairs only (d, d_ff
 // multiples of 256); other shapes with those weights use the streaming kernels.
 // The tensor-core FP4 path widens every weight tile to bf16 once per token
-// tile, which at a few tokens per expert costs more than the streaming
-// kernels' direct FMAs: FP4 streams up to kFp4StreamRowsPerExpert mean rows per
-// expert (measured at the Hy3 shape, top-6: 2 rows 1.27 vs 1.59 ms per layer
-// streaming vs tensor cores; 16 rows 8.1 vs 1.85 ms).
-constexpr int kFp4StreamRowsPerExpert = 4;
+// tile and issues its MMAs whatever the tile's token count, which below about
+// one token per expert costs more than the streaming kernels' direct FMAs:
+// FP4 streams up to kFp4StreamRowsPerExpert mean rows per expert (measured at
+// the Hy3 shape, top-6, per layer streaming vs tensor cores: T=8 0.28 vs
+// 0.38 ms; T=64 1.27 vs 1.22 ms; T=2048 31.2 vs 1.51 ms).
+constexpr int kFp4StreamRowsPerExpert = 1;
 bool quantised(const moe_config* c) {
     return (c->flags & (MOE_FLAG_FP8_WEIGHTS | MOE_FLAG_FP4_WEIGHTS)) != 0;
 }

@@ -203,6 +203,21 @@ __device__ __forceinline__ void bulk_copy_smem_to_cluster(uint32_t dst_cluster, 
         : "memory");
 }
 
+// Asynchronous 8-byte copy global -> this CTA's shared memory (both addresses
+// 8-byte aligned), in the issuing thread's current copy group; commit closes
+// the group, and wait_pending<N> waits until at most N of the thread's groups
+// are still in flight (its earlier copies are then visible to it).
+__device__ __forceinline__ void cp_async8(uint32_t dst_smem, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait_pending() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {

@@ -156,7 +156,7 @@ def sample_tokens(T: int, n: int = 48, seed: int = 0) -> np.ndarray:
 
 
 NMAX = 256       # token rows per tile of the bf16 and FP4 SM-pair GEMMs
-FP8_NMAX = 192   # FP8: the widened weights share tensor memory with the accumulators
+FP8_NMAX = 192   # FP8 and FP4: the widened weights share tensor memory with the accumulators
 
 
 def gemm_tiles(counts, nmax: int = NMAX, unit: int = 32):
