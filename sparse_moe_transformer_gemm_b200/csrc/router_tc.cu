@@ -13,7 +13,8 @@
 // memory; after a cluster barrier, CTA j sums rows [j*128/S, (j+1)*128/S) over
 // the S CTAs through distributed shared memory (16-byte loads, several in
 // flight per thread), in split order (the result does not depend on timing),
-// and selects for those rows, one thread per row, ties to the lower expert
+// and selects for those rows, S lanes per row (each scans a contiguous range
+// of experts; shuffle merges combine the lists), ties to the lower expert
 // index. The sigmoid is increasing, so the k largest (biased) logits are the k
 // largest scores; it is evaluated for the k selected only. With score_fn 1
 // the score is sqrt(softplus(logit)) (the V4-Flash router, same page §2.2),
@@ -63,28 +64,24 @@ __host__ __device__ constexpr int logit_stride(int E) { return ((E + 31) / 32) *
 // (the selection reads up to 7 floats past a row's E logits; the ring has room)
 static_assert(BM * logit_stride(256) * 4 + 32 <= STAGES * STAGE_BYTES, "logit rows fit in the ring");
 
-// Top-k of one token by one thread, from its E logits (a shared-memory row,
-// 16-byte aligned, read as float4: with a row stride of 4 mod 32 floats the
-// 16-byte reads of a warp's rows take the minimum number of wavefronts): a
-// sorted list of the k largest (biased) logits where only a strictly greater
-// value enters, so equal values keep the lower expert index (experts are
-// visited in increasing order); then the sigmoid of the k selected,
-// renormalised (summed in list order) and scaled. A warp per token (k rounds
-// of a warp-wide argmax, one token at a time per warp) measured ~3 us per
-// token here, far slower than this scan; the bias is staged in shared memory
-// (per-element global loads of it made the scan ~3x slower).
+// Top-k of one token over the experts [e_lo, e_hi) by one thread, from its
+// logits (a shared-memory row, 16-byte aligned, read as float4: with a row
+// stride of 4 mod 32 floats the 16-byte reads of a warp's rows take the
+// minimum number of wavefronts): a sorted list (8 entries, the first K in use,
+// the rest -inf) of the K largest (biased) logits where only a strictly
+// greater value enters, so equal values keep the lower expert index (experts
+// are visited in increasing order). e_lo is a multiple of 8; e_hi is E or a
+// multiple of 8. The bias is staged in shared memory (per-element global
+// loads of it made the scan ~3x slower).
 template <int K, bool SB>
-__device__ __forceinline__ void thread_select_topk(const float* row, const float* sbias,
-                                                   const float* cbias, int E, float scale,
-                                                   int score_fn, int* __restrict__ idx_out,
-                                                   float* __restrict__ w_out) {
+__device__ __forceinline__ void scan_topk(const float* row, const float* sbias, const float* cbias,
+                                          int e_lo, int e_hi, int E, int score_fn, float (&v)[8],
+                                          float (&p)[8], int (&id)[8]) {
     // SB: rank sigmoid(logit) + cbias (the e_score_correction_bias) and keep
     // the sigmoid scores p of the list for the weights
-    float v[K], p[K];
-    int id[K];
 #pragma unroll
-    for (int j = 0; j < K; ++j) { v[j] = -INFINITY; p[j] = 0.f; id[j] = 0; }
-    for (int e0 = 0; e0 < E; e0 += 8) {
+    for (int j = 0; j < 8; ++j) { v[j] = -INFINITY; p[j] = 0.f; id[j] = 0x7fffffff; }
+    for (int e0 = e_lo; e0 < e_hi; e0 += 8) {
         // 8 logits and their biases in flight, then visited in increasing order
         const float4 a0 = *reinterpret_cast<const float4*>(row + e0);
         const float4 a1 = *reinterpret_cast<const float4*>(row + e0 + 4);
@@ -115,6 +112,68 @@ __device__ __forceinline__ void thread_select_topk(const float* row, const float
             }
         }
     }
+}
+
+// Entry a ranks before entry b: a larger value, or an equal value and a lower
+// expert index.
+__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+// Merge this lane's sorted 8-entry list with the one of lane ^ m (same order,
+// disjoint experts) into the 8 best of both, sorted, in both lanes: the
+// element-wise better of the list and the partner's reversed list is a
+// bitonic sequence holding the 8 best, and three half-cleaner stages sort it.
+__device__ __forceinline__ void merge_topk(float (&v)[8], float (&p)[8], int (&id)[8], int m) {
+    float ov[8], op[8];
+    int oi[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        ov[j] = __shfl_xor_sync(0xffffffffu, v[j], m);
+        op[j] = __shfl_xor_sync(0xffffffffu, p[j], m);
+        oi[j] = __shfl_xor_sync(0xffffffffu, id[j], m);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (ranks_before(ov[7 - j], oi[7 - j], v[j], id[j])) {
+            v[j] = ov[7 - j];
+            p[j] = op[7 - j];
+            id[j] = oi[7 - j];
+        }
+#pragma unroll
+    for (int s = 4; s > 0; s >>= 1)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if ((j & s) == 0 && ranks_before(v[j + s], id[j + s], v[j], id[j])) {
+                const float tv = v[j]; v[j] = v[j + s]; v[j + s] = tv;
+                const float tp = p[j]; p[j] = p[j + s]; p[j + s] = tp;
+                const int ti = id[j]; id[j] = id[j + s]; id[j + s] = ti;
+            }
+}
+
+// The selection of one token by P adjacent lanes (P a power of two <= 8; P
+// = 1: one thread): lane `part` scans its range of experts (contiguous,
+// increasing with part), and log2 P shuffle merges give every lane the
+// token's sorted list -- the same list, in the same order, as one thread's
+// scan of all experts. Part 0 then evaluates the score of the K selected,
+// renormalises (summed in list order) and scales. Every lane of the warp
+// takes part (the merges shuffle across the whole warp); `write` gates the
+// output. (A warp per token, k rounds of a warp-wide argmax, measured ~3 us
+// per token here.)
+template <int K, bool SB, int P>
+__device__ __forceinline__ void select_topk(const float* row, const float* sbias,
+                                            const float* cbias, int E, float scale, int score_fn,
+                                            int part, bool write, int* __restrict__ idx_out,
+                                            float* __restrict__ w_out) {
+    const int chunk = ((E + P - 1) / P + 7) & ~7;
+    const int e_lo = part * chunk;
+    const int e_hi = min(E, e_lo + chunk);
+    float v[8], p[8];
+    int id[8];
+    scan_topk<K, SB>(row, sbias, cbias, e_lo, e_hi, E, score_fn, v, p, id);
+#pragma unroll
+    for (int m = 1; m < P; m <<= 1) merge_topk(v, p, id, m);
+    if (!write || part != 0) return;
     float sum = 0.f;
 #pragma unroll
     for (int j = 0; j < K; ++j) {
@@ -128,19 +187,20 @@ __device__ __forceinline__ void thread_select_topk(const float* row, const float
     }
 }
 
-template <bool SB>
+template <bool SB, int P>
 __device__ __forceinline__ void select_k(int k, const float* row, const float* sbias,
                                          const float* cbias, int E, float scale, int score_fn,
-                                         int* __restrict__ idx_out, float* __restrict__ w_out) {
+                                         int part, bool write, int* __restrict__ idx_out,
+                                         float* __restrict__ w_out) {
     switch (k) {
-        case 1: thread_select_topk<1, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
-        case 2: thread_select_topk<2, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
-        case 3: thread_select_topk<3, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
-        case 4: thread_select_topk<4, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
-        case 5: thread_select_topk<5, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
-        case 6: thread_select_topk<6, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
-        case 7: thread_select_topk<7, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
-        default: thread_select_topk<8, SB>(row, sbias, cbias, E, scale, score_fn, idx_out, w_out); break;
+        case 1: select_topk<1, SB, P>(row, sbias, cbias, E, scale, score_fn, part, write, idx_out, w_out); break;
+        case 2: select_topk<2, SB, P>(row, sbias, cbias, E, scale, score_fn, part, write, idx_out, w_out); break;
+        case 3: select_topk<3, SB, P>(row, sbias, cbias, E, scale, score_fn, part, write, idx_out, w_out); break;
+        case 4: select_topk<4, SB, P>(row, sbias, cbias, E, scale, score_fn, part, write, idx_out, w_out); break;
+        case 5: select_topk<5, SB, P>(row, sbias, cbias, E, scale, score_fn, part, write, idx_out, w_out); break;
+        case 6: select_topk<6, SB, P>(row, sbias, cbias, E, scale, score_fn, part, write, idx_out, w_out); break;
+        case 7: select_topk<7, SB, P>(row, sbias, cbias, E, scale, score_fn, part, write, idx_out, w_out); break;
+        default: select_topk<8, SB, P>(row, sbias, cbias, E, scale, score_fn, part, write, idx_out, w_out); break;
     }
 }
 
@@ -322,18 +382,18 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         __syncthreads();
     }
     if (warp >= 2) {
-        // one thread per token row of this CTA's slice
-        const int rr = threadIdx.x - 64;
+        // S lanes per token row of this CTA's slice (ROWS * S = 128 threads)
+        const int tid = threadIdx.x - 64;
+        const int rr = tid / S, part = tid % S;
         const long t = (long)tile * BM + split * ROWS + rr;
-        if (rr < ROWS && t < T) {
-            const float* rw = red + (split * ROWS + rr) * es;
-            int* io = idx_out + t * k;
-            float* wo = w_out + t * k;
-            if (sbias)
-                select_k<true>(k, rw, c.bias, c.sbias, E, scale, score_fn, io, wo);
-            else
-                select_k<false>(k, rw, c.bias, c.sbias, E, scale, score_fn, io, wo);
-        }
+        const float* rw = red + (split * ROWS + rr) * es;
+        const bool write = t < T;
+        int* io = idx_out + (write ? t : 0) * k;
+        float* wo = w_out + (write ? t : 0) * k;
+        if (sbias)
+            select_k<true, S>(k, rw, c.bias, c.sbias, E, scale, score_fn, part, write, io, wo);
+        else
+            select_k<false, S>(k, rw, c.bias, c.sbias, E, scale, score_fn, part, write, io, wo);
     }
 
     tc::fence_before_sync();
