@@ -450,10 +450,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 // the tile's writes and the MMA's reads competing with the raw reads. TMEM
 // then holds the accumulators and the op stages, which caps a token tile at
 // NM = 192 rows: gate_up g and u (2 x 192 columns) + 2 op stages of 64
-// (gate + up); down two accumulator stages (2 x 192) + 4 op stages of 32.
-// (Half-K-block op stages, twice as many, measured 8% slower on B200 for
-// gate_up and 10% for down: twice the barrier and signal work for half the
-// conversion each.)
+// (gate + up, one K block); down two accumulator stages (2 x 192) + 2 op
+// stages of 64 (two K blocks). (Smaller op stages, twice as many, measured
+// 8-10% slower on B200: more barrier and signal work for less conversion
+// each.)
 
 constexpr int THREADS_Q = 512;        // warps 6-14 converters, warp 15 token producer
 constexpr int MAX_RAW_STAGES = 16, MAX_B_STAGES = 4, MAX_OP_STAGES = 4;  // QCtrl's arrays
@@ -467,7 +467,8 @@ struct QShape {
     static constexpr int BH = (NM / 2) * BK * 2;                   // a CTA's token half (bytes)
     static constexpr int RAW_STAGES = FP4 ? 16 : (GATE_UP ? 8 : 12);
     static constexpr int B_STAGES = 4;
-    static constexpr int OP_STAGES = GATE_UP ? 2 : 4;
+    static constexpr int KPO = GATE_UP ? 1 : 2;                    // K blocks per op stage
+    static constexpr int OP_STAGES = 2;
     // converter warps: GROUPS groups of four (one per TMEM lane quarter) take
     // K blocks round-robin
     static constexpr int GROUPS = 2;
@@ -483,7 +484,7 @@ struct QShape {
     static constexpr int ACC_COLS = GATE_UP ? 2 * NM : NM;
     static constexpr int A_COL = ACC_STAGES * ACC_COLS;
     static constexpr int A_TILE_COLS = BK / 2;                     // one tile's K block: two bf16 a column
-    static constexpr int A_STAGE_COLS = A_TILES * A_TILE_COLS;
+    static constexpr int A_STAGE_COLS = A_TILES * KPO * A_TILE_COLS;  // 64
 };
 
 constexpr int CONV_WARPS = 9;                          // warps 6..14 (warp 14 idles)
@@ -491,7 +492,7 @@ constexpr int TOKEN_WARP = 6 + CONV_WARPS;
 template <bool G, bool FP4>
 constexpr bool shape_ok() {
     using S = QShape<G, FP4>;
-    return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES % S::GROUPS == 0 &&
+    return S::RAW_STAGES % (S::KPO * S::GROUPS) == 0 && S::OP_STAGES % S::GROUPS == 0 &&
            S::GROUPS * S::GROUP_WARPS <= CONV_WARPS && S::GROUP_WARPS == 4 &&
            S::RAW_STAGES <= MAX_RAW_STAGES && S::B_STAGES <= MAX_B_STAGES &&
            S::OP_STAGES <= MAX_OP_STAGES && S::A_COL + S::OP_STAGES * S::A_STAGE_COLS <= 512 &&
@@ -824,62 +825,74 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         };
         uint2 sc_cur[S::A_TILES] = {};
         long cur_chunk = -1;
-        const long j0 = group < S::GROUPS ? group : n_blocks;
-        if (FP4 && j0 < n_blocks)
-            for (int g = 0; g < S::SC_STAGES - 1; ++g) fetch_chunk((j0 >> 2) + g);
-        for (long jb = j0; jb < n_blocks; jb += S::GROUPS) {
-            const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
-            const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
-            const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
-            uint32_t sc[S::A_TILES] = {};  // FP4: this block's two scale bytes per A tile
-            if constexpr (FP4) {
-                if ((jb >> 2) != cur_chunk) {
-                    cur_chunk = jb >> 2;
-                    // the slot of chunk G + SC_STAGES - 1 held chunk G - 1, read already
-                    fetch_chunk(cur_chunk + S::SC_STAGES - 1);
-                    tc::cp_async_wait_pending<S::SC_STAGES - 1>();  // chunk G has landed
-                    const uint32_t src =
-                        sc_slot0 + (uint32_t)((cur_chunk % S::SC_STAGES) * S::A_TILES * BM * 8);
+        // a group fills the op stages ob = group, group + GROUPS, ..., each from
+        // the raw stages of its KPO K blocks j = KPO ob + kk
+        const long n_ops = n_blocks / S::KPO;
+        const long ob0 = group < S::GROUPS ? group : n_ops;
+        if (FP4 && ob0 < n_ops)
+            for (int g = 0; g < S::SC_STAGES - 1; ++g) fetch_chunk(((ob0 * S::KPO) >> 2) + g);
+        for (long ob = ob0; ob < n_ops; ob += S::GROUPS) {
+            const int os = (int)(ob % S::OP_STAGES);
+            const uint32_t oph = (uint32_t)(ob / S::OP_STAGES) & 1u;
+            uint32_t o[S::A_TILES * S::KPO * 32];  // (tile a, block kk) at o[32 (a KPO + kk) ..]
+            bool failed = false;  // the same in every thread of the group
+#pragma unroll
+            for (int kk = 0; kk < S::KPO; ++kk) {
+                const long jb = ob * S::KPO + kk;
+                const int rs = (int)(jb % S::RAW_STAGES);
+                const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
+                uint32_t sc[S::A_TILES] = {};  // FP4: this block's two scale bytes per A tile
+                if constexpr (FP4) {
+                    if ((jb >> 2) != cur_chunk) {
+                        cur_chunk = jb >> 2;
+                        // the slot of chunk G + SC_STAGES - 1 held chunk G - 1, read already
+                        fetch_chunk(cur_chunk + S::SC_STAGES - 1);
+                        tc::cp_async_wait_pending<S::SC_STAGES - 1>();  // chunk G has landed
+                        const uint32_t src =
+                            sc_slot0 + (uint32_t)((cur_chunk % S::SC_STAGES) * S::A_TILES * BM * 8);
+#pragma unroll
+                        for (int a = 0; a < S::A_TILES; ++a)
+                            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                         : "=r"(sc_cur[a].x), "=r"(sc_cur[a].y)
+                                         : "r"(src + a * BM * 8));
+                    }
+                    const int kq = (int)(jb & 3);  // the block's place in its chunk
 #pragma unroll
                     for (int a = 0; a < S::A_TILES; ++a)
-                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
-                                     : "=r"(sc_cur[a].x), "=r"(sc_cur[a].y)
-                                     : "r"(src + a * BM * 8));
+                        sc[a] = ((kq < 2 ? sc_cur[a].x : sc_cur[a].y) >> (16 * (kq & 1))) & 0xFFFFu;
                 }
-                const int kq = (int)(jb & 3);  // the block's place in its chunk
+                const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
+                if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
+                    failed = true;
+                    break;
+                }
+                const uint32_t raw = raw0 + rs * S::RAW_STAGE;
+                constexpr int CHUNKS = S::RAW_ROW / 16;
+                uint32_t w[S::A_TILES][4 * CHUNKS];
 #pragma unroll
                 for (int a = 0; a < S::A_TILES; ++a)
-                    sc[a] = ((kq < 2 ? sc_cur[a].x : sc_cur[a].y) >> (16 * (kq & 1))) & 0xFFFFu;
+#pragma unroll
+                    for (int ch = 0; ch < CHUNKS; ++ch)
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(w[a][4 * ch]), "=r"(w[a][4 * ch + 1]),
+                                       "=r"(w[a][4 * ch + 2]), "=r"(w[a][4 * ch + 3])
+                                     : "r"(raw + a * S::RAW_TILE + ((ch ^ rsw) << 4)));
+#pragma unroll
+                for (int a = 0; a < S::A_TILES; ++a) {
+                    uint32_t* oa = &o[32 * (a * S::KPO + kk)];
+                    if constexpr (FP4) {
+#pragma unroll
+                        for (int ch = 0; ch < 2; ++ch)
+                            e2m1x32_to_bf16(&w[a][4 * ch], (sc[a] >> (8 * ch)) & 0xFFu, oa + 16 * ch);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) e4m3x4_to_bf16x4(w[a][j], oa[2 * j], oa[2 * j + 1]);
+                    }
+                }
             }
-            const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
-            if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
+            if (failed) {
                 raise_timeout(c, status);
                 break;
-            }
-            const uint32_t raw = raw0 + rs * S::RAW_STAGE;
-            constexpr int CHUNKS = S::RAW_ROW / 16;
-            uint32_t w[S::A_TILES][4 * CHUNKS];
-#pragma unroll
-            for (int a = 0; a < S::A_TILES; ++a)
-#pragma unroll
-                for (int ch = 0; ch < CHUNKS; ++ch)
-                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(w[a][4 * ch]), "=r"(w[a][4 * ch + 1]),
-                                   "=r"(w[a][4 * ch + 2]), "=r"(w[a][4 * ch + 3])
-                                 : "r"(raw + a * S::RAW_TILE + ((ch ^ rsw) << 4)));
-            uint32_t o[S::A_TILES * 32];  // tile a in o[32 a ..], its TMEM columns in order
-#pragma unroll
-            for (int a = 0; a < S::A_TILES; ++a) {
-                if constexpr (FP4) {
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch)
-                        e2m1x32_to_bf16(&w[a][4 * ch], (sc[a] >> (8 * ch)) & 0xFFu,
-                                        &o[32 * a + 16 * ch]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        e4m3x4_to_bf16x4(w[a][j], o[32 * a + 2 * j], o[32 * a + 2 * j + 1]);
-                }
             }
             const bool ook = tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
             if (tc::bar_any(2 + group, S::CONV_THREADS, !ook)) {
@@ -887,12 +900,14 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 break;
             }
             tc::fence_after_sync();  // the MMAs that read this op stage are complete
-            tc_store_row<S::A_TILES>(a_lane + os * S::A_STAGE_COLS, o);
+            tc_store_row<S::A_TILES * S::KPO>(a_lane + os * S::A_STAGE_COLS, o);
             tc::tmem_st_wait();
             tc::fence_before_sync();
             tc::bar_sync(2 + group, S::CONV_THREADS);
             if (ct == 0) {
-                tc::mbar_arrive(&c.raw_empty[rs]);
+#pragma unroll
+                for (int kk = 0; kk < S::KPO; ++kk)
+                    tc::mbar_arrive(&c.raw_empty[(int)((ob * S::KPO + kk) % S::RAW_STAGES)]);
                 if (leader)
                     tc::mbar_arrive_expect_tx(&c.op_full[os], 16);
                 else
@@ -920,35 +935,45 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 tc::fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
                 const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, ti.n);
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!tc::mbar_wait(&c.op_full[os], oph, abort_flag) ||
-                        !tc::mbar_wait(&c.b_full[bs], bph, abort_flag)) {
+                for (int ob = 0; ob < KB / S::KPO && ok; ++ob) {
+                    if (!tc::mbar_wait(&c.op_full[os], oph, abort_flag)) {
                         raise_timeout(c, status);
                         ok = false;
                         break;
                     }
-                    tc::fence_after_sync();
                     const uint32_t a_tm = tmem_base + S::A_COL + os * S::A_STAGE_COLS;
-                    const uint32_t b_addr = tc::smem_u32(b_ring + bs * S::BH);
 #pragma unroll
-                    for (int k = 0; k < BK / UK; ++k) {  // K = 16 of A is 8 TMEM columns
-                        const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
-                        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                        tc::mma_bf16_pair_ta(d_tmem, a_tm + k * (UK / 2), bdesc, idesc, accum);
-                        if (GATE_UP)
-                            tc::mma_bf16_pair_ta(d_tmem + S::U_OFF,
-                                                 a_tm + S::A_TILE_COLS + k * (UK / 2), bdesc,
-                                                 idesc, accum);
+                    for (int kk = 0; kk < S::KPO; ++kk) {
+                        if (!tc::mbar_wait(&c.b_full[bs], bph, abort_flag)) {
+                            raise_timeout(c, status);
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+                        const int kb = ob * S::KPO + kk;
+                        const uint32_t b_addr = tc::smem_u32(b_ring + bs * S::BH);
+#pragma unroll
+                        for (int k = 0; k < BK / UK; ++k) {  // K = 16 of A is 8 TMEM columns
+                            const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
+                            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                            tc::mma_bf16_pair_ta(d_tmem, a_tm + kk * S::A_TILE_COLS + k * (UK / 2),
+                                                 bdesc, idesc, accum);
+                            if (GATE_UP)  // KPO = 1: the up tile follows the gate tile
+                                tc::mma_bf16_pair_ta(d_tmem + S::U_OFF,
+                                                     a_tm + S::A_TILE_COLS + k * (UK / 2), bdesc,
+                                                     idesc, accum);
+                        }
+                        if (kk == S::KPO - 1) tc::mma_commit_pair(&c.op_empty[os], 0x3);
+                        tc::mma_commit_pair(&c.b_empty[bs], 0x3);
+                        if (++bs == S::B_STAGES) {
+                            bs = 0;
+                            bph ^= 1u;
+                        }
                     }
-                    tc::mma_commit_pair(&c.op_empty[os], 0x3);
-                    tc::mma_commit_pair(&c.b_empty[bs], 0x3);
+                    if (!ok) break;
                     if (++os == S::OP_STAGES) {
                         os = 0;
                         oph ^= 1u;
-                    }
-                    if (++bs == S::B_STAGES) {
-                        bs = 0;
-                        bph ^= 1u;
                     }
                 }
                 if (ok) tc::mma_commit_pair(&c.acc_full[acc], 0x3);
