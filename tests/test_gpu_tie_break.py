@@ -11,8 +11,11 @@ must equal the oracle's element by element, and the weights agree to a few
 fp32 ulps (the oracle renormalises in fp64).
 
 Both router kernels run: T = 64 takes the K-split CUDA-core router, T = 256
-the tensor-core router (tcgen05 logits, one thread per token's selection), at
-the Hy3 router shape d = 4096, E = 192, k = 8.
+the tensor-core router (tcgen05 logits; a 128-token tile split over 8 CTAs,
+8 lanes per token's selection, each scanning 24 experts, their lists merged),
+at the Hy3 router shape d = 4096, E = 192, k = 8. The cross-lane case puts
+the tied experts in different lanes' ranges (and, at T = 2048, the 4-way
+split's 48-expert ranges), so the merges must keep the lower index.
 """
 
 import numpy as np
@@ -30,6 +33,8 @@ D, E, K, SCALE = 4096, 192, 8, 2.826
 W_RTOL_TIE = 2e-6   # fp32 sigmoid, sum and division against fp64: a few ulps
 SIX = [5, 40, 77, 130, 160, 191]        # experts lifted by distinct logit biases
 TIED = [100, 101, 102, 103]             # experts with identical router rows
+LIFT4 = [5, 40, 77, 131]                # four experts lifted by distinct biases
+CROSS = [20, 30, 50, 70, 120, 170]      # identical rows in different selection lanes
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -44,6 +49,14 @@ def _router_weights():
     wg = make_layer(CONFIGS["decode"], seed=0, device="cuda", with_experts=False)["w_gate"]
     wg = wg.clone()
     wg[TIED[1:]] = wg[TIED[0]].clone()
+    return wg
+
+
+def _router_weights_cross():
+    """The same draw with the rows of CROSS set equal to row CROSS[0]."""
+    wg = make_layer(CONFIGS["decode"], seed=0, device="cuda", with_experts=False)["w_gate"]
+    wg = wg.clone()
+    wg[CROSS[1:]] = wg[CROSS[0]].clone()
     return wg
 
 
@@ -83,6 +96,14 @@ def _case(name, T):
     elif name == "constant_score_bias":
         x = _tokens(T, "zero")
         sb = torch.full((E,), 0.05, dtype=torch.float32, device="cuda")
+    elif name == "cross_lane_ties":
+        # four experts lifted by 3.0 .. 2.4 and the six identical rows by 1.0:
+        # the four tied experts with the lowest indices take places 5..8
+        x = _tokens(T, "mixed")
+        wg = _router_weights_cross()
+        gb = torch.zeros(E, dtype=torch.float32, device="cuda")
+        gb[LIFT4] = torch.tensor([3.0, 2.8, 2.6, 2.4], device="cuda")
+        gb[CROSS] = 1.0
     elif name == "duplicated_rows_score_bias":
         x, wg, gb, _ = _case("duplicated_rows", T)
         # small per-expert score biases (0 .. 0.004), equal on the tied four
@@ -102,14 +123,16 @@ def _expected_structure(name, idx):
         assert np.all(idx == np.array(SIX + TIED[:2])), name
     elif name == "saturated":
         assert np.all(idx == np.array([9, 3, 0, 1, 2, 4, 5, 6])), name
+    elif name == "cross_lane_ties":
+        assert np.all(idx == np.array(LIFT4 + CROSS[:4])), name
 
 
 CASES = ["all_zero", "constant_gate_bias", "duplicated_rows", "saturated",
-         "constant_score_bias", "duplicated_rows_score_bias"]
+         "constant_score_bias", "duplicated_rows_score_bias", "cross_lane_ties"]
 
 
-@pytest.mark.parametrize("T", [64, 256])
-@pytest.mark.parametrize("name", CASES)
+@pytest.mark.parametrize("name,T", [(n, T) for n in CASES for T in (64, 256)] +
+                         [("cross_lane_ties", 2048)])
 def test_exact_ties_take_the_lower_index_in_score_order(name, T):
     x, wg, gb, sb = _case(name, T)
     cfg = moe.config(T, D, E, K, 1536, SCALE)
