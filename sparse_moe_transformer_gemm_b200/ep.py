@@ -27,12 +27,15 @@ expert's weights, and the combine sums the same k rows in the same slot
 order, so a rank's result is bitwise what moe_forward gives for its tokens
 with all E experts on one GPU.
 
-Two drivers run the same three phases: ``ep_forward`` exchanges through
+Three drivers run the same phases: ``ep_forward`` exchanges through
 torch.distributed (all_to_all_single; NCCL on GPUs, any backend that has it
-on CPU tensors), and ``ep_forward_lockstep`` runs all P ranks in one process
-and exchanges by slicing (no kernel of one rank waits on another's, so the
-ranks can share one device). The compute is an ``ops`` object: ``CudaOps``
-calls the library's C ABI; the phases never compute on the host.
+on CPU tensors); ``ep_forward_pipelined`` does the same on C chunks of the
+rank's tokens with the row exchanges in flight while the experts of an
+earlier chunk run (Q4.10's point that the all-to-all time should hide
+behind the expert compute); ``ep_forward_lockstep`` runs all P ranks in one
+process and exchanges by slicing (no kernel of one rank waits on another's,
+so the ranks can share one device). The compute is an ``ops`` object:
+``CudaOps`` calls the library's C ABI; the phases never compute on the host.
 """
 
 from __future__ import annotations
@@ -84,8 +87,15 @@ class Dispatched:
 
 
 def dispatch(ops, part: Partition, x: torch.Tensor) -> Dispatched:
-    """Phase 1: route and group the rank's tokens; the send blocks per destination."""
+    """Phase 1: route and group the rank's tokens; the send blocks per destination.
+    No tokens: empty blocks (no call into ops)."""
     T = x.shape[0]
+    if T == 0:
+        k = ops.k
+        return Dispatched(torch.empty((0, k), dtype=torch.int32, device=x.device),
+                          torch.empty((0, k), dtype=torch.float32, device=x.device),
+                          torch.empty(0, dtype=torch.int32, device=x.device), x[:0],
+                          torch.zeros((part.P, part.E_local), dtype=torch.int64), 0)
     idx, w = ops.route(x)
     counts, row_of, x_perm = ops.group(idx, x)
     counts_pe = counts.to("cpu", torch.int64).view(part.P, part.E_local)
@@ -105,6 +115,8 @@ def run_experts(ops, part: Partition, rows: torch.Tensor,
 
 def combine(ops, state: Dispatched, y_back: torch.Tensor) -> torch.Tensor:
     """Phase 5: the fp32 weighted combine of the returned rows."""
+    if state.T == 0:
+        return y_back[:0]
     return ops.combine(y_back, state.row_of, state.w, state.T)
 
 
@@ -144,6 +156,72 @@ def ep_forward(ops, part: Partition, x: torch.Tensor, group=None) -> torch.Tenso
     y = run_experts(ops, part, rows, recv_counts_pe)
     y_back = _a2a_rows(dist, group, y, recv_splits, st.send_splits)
     return combine(ops, st, y_back)
+
+
+def _a2a_rows_async(dist, group, send: torch.Tensor, send_splits, recv_splits):
+    """_a2a_rows started asynchronously: (output, work handle)."""
+    out = torch.empty((sum(recv_splits),) + tuple(send.shape[1:]), dtype=send.dtype,
+                      device=send.device)
+    s = send.contiguous()
+    if send.dtype == torch.bfloat16:
+        s, o = s.view(torch.int32), out.view(torch.int32)
+    else:
+        o = out
+    work = dist.all_to_all_single(o, s, recv_splits, send_splits, group=group, async_op=True)
+    return out, (work, s)  # the send buffer stays referenced until the wait
+
+
+def chunk_bounds(T: int, chunks: int) -> List[int]:
+    """Token offsets of C near-equal contiguous chunks (empty ones when T < C)."""
+    if chunks < 1:
+        raise ValueError("chunks must be >= 1")
+    q, r = divmod(T, chunks)
+    b = [0]
+    for c in range(chunks):
+        b.append(b[-1] + q + (1 if c < r else 0))
+    return b
+
+
+def ep_forward_pipelined(ops, part: Partition, x: torch.Tensor, chunks: int = 2,
+                         group=None) -> torch.Tensor:
+    """ep_forward on `chunks` contiguous chunks of the rank's tokens, pipelined:
+    every chunk is dispatched and its rows sent first (the row exchanges in
+    flight together); then each chunk's experts run as soon as its rows have
+    arrived, and its outputs start back while the next chunk's experts run;
+    the combines come last. Every rank takes the same collective steps in the
+    same order (chunks number the same on every rank; empty chunks exchange
+    empty blocks). A token's output depends only on its own rows, so the
+    result equals ep_forward on each chunk by itself."""
+    import torch.distributed as dist
+
+    if dist.get_world_size(group) != part.P:
+        raise ValueError("the process group does not have P ranks")
+    b = chunk_bounds(x.shape[0], chunks)
+    sts, rows, recv = [], [], []
+    for c in range(chunks):
+        st = dispatch(ops, part, x[b[c]:b[c + 1]])
+        dev = st.x_perm.device
+        send_c = st.counts_pe.to(device=dev, dtype=torch.int64).contiguous()
+        recv_c = torch.empty_like(send_c)
+        dist.all_to_all_single(recv_c, send_c, group=group)  # row p goes to rank p
+        recv_counts_pe = recv_c.to("cpu")
+        sts.append(st)
+        recv.append(recv_counts_pe)
+        rows.append(_a2a_rows_async(dist, group, st.x_perm, st.send_splits,
+                                    recv_counts_pe.sum(dim=1).tolist()))
+    backs = []
+    for c in range(chunks):
+        r, (work, _) = rows[c]
+        work.wait()
+        y = run_experts(ops, part, r, recv[c])
+        backs.append(_a2a_rows_async(dist, group, y, recv[c].sum(dim=1).tolist(),
+                                     sts[c].send_splits))
+    outs = []
+    for c in range(chunks):
+        y_back, (work, _) = backs[c]
+        work.wait()
+        outs.append(combine(ops, sts[c], y_back))
+    return torch.cat(outs) if outs else x.new_empty((0, x.shape[1]))
 
 
 def ep_forward_lockstep(ops_per_rank, part: Partition, xs) -> List[torch.Tensor]:
@@ -196,6 +274,7 @@ class CudaOps:
         self.ropt = route_options
         self.stream = stream
         self.dev = w_gate.device
+        self.k = cfg.k
 
     def _cfg(self, T: int, E: int, k: int):
         return moe.MoeConfig(T, self.cfg.d, E, k, self.cfg.d_ff, self.cfg.scale, self.cfg.flags)
@@ -268,4 +347,5 @@ def ep_layer_ops(cfg, part: Partition, rank: int, w_gate, gate_bias, w_gate_up, 
 
 
 __all__ = ["Partition", "Dispatched", "dispatch", "run_experts", "combine", "ep_forward",
-           "ep_forward_lockstep", "CudaOps", "local_expert_weights", "ep_layer_ops"]
+           "ep_forward_pipelined", "chunk_bounds", "ep_forward_lockstep", "CudaOps",
+           "local_expert_weights", "ep_layer_ops"]

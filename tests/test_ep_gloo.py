@@ -7,7 +7,8 @@ compute (tests/ep_oracle_ops.py).
   output of one rank holding all experts, for P = 2 and 4, including a rank
   that receives no rows;
 * two gloo processes (the torch.distributed driver, all_to_all_single) give
-  the same bits as the lockstep driver;
+  the same bits as the lockstep driver, and so does the pipelined driver on
+  1, 3 or 30 chunks of each rank's tokens (30 > tokens: empty chunks);
 * the single-rank result matches the oracle's own forward within the layer's
   output tolerance (the EP path stores the expert outputs as bf16, as the GPU
   path does; the oracle keeps them in fp64).
@@ -86,14 +87,17 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, bias_rank0, out):
+def _worker(rank, world, port, bias_rank0, out, chunks=0):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         L = _layer(bias_rank0)
         part = ep.Partition(SHAPE.E, world)
         x = _shards(L["x"], world)[rank]
-        y = ep.ep_forward(_ops(L, part, rank), part, x)
+        if chunks:
+            y = ep.ep_forward_pipelined(_ops(L, part, rank), part, x, chunks=chunks)
+        else:
+            y = ep.ep_forward(_ops(L, part, rank), part, x)
         out[rank] = oracle.bf16_bits(y)
     finally:
         dist.destroy_process_group()
@@ -108,6 +112,30 @@ def test_two_gloo_ranks_equal_the_lockstep_driver(bias_rank0):
         mp.spawn(_worker, args=(world, port, bias_rank0, out), nprocs=world, join=True)
         res = dict(out)
     L = _layer(bias_rank0)
+    part = ep.Partition(SHAPE.E, world)
+    want = ep.ep_forward_lockstep([_ops(L, part, r) for r in range(world)], part,
+                                  _shards(L["x"], world))
+    for r in range(world):
+        assert np.array_equal(res[r], oracle.bf16_bits(want[r])), r
+
+
+def test_chunk_bounds_cover_the_tokens_in_order():
+    assert ep.chunk_bounds(10, 3) == [0, 4, 7, 10]
+    assert ep.chunk_bounds(2, 3) == [0, 1, 2, 2]
+    assert ep.chunk_bounds(0, 2) == [0, 0, 0]
+    with pytest.raises(ValueError):
+        ep.chunk_bounds(5, 0)
+
+
+@pytest.mark.parametrize("chunks", [1, 3, 30])
+def test_two_gloo_ranks_pipelined_equal_the_lockstep_driver(chunks):
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, port, True, out, chunks), nprocs=world, join=True)
+        res = dict(out)
+    L = _layer(True)
     part = ep.Partition(SHAPE.E, world)
     want = ep.ep_forward_lockstep([_ops(L, part, r) for r in range(world)], part,
                                   _shards(L["x"], world))

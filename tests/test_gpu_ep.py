@@ -7,6 +7,8 @@ is checked against the oracle by the parity tests.
 """
 
 import dataclasses
+import os
+import socket
 
 import numpy as np
 import pytest
@@ -95,3 +97,36 @@ def test_row_experts_kernel_expands_the_counts(n_src, e_local):
     got = ids.cpu().numpy()
     assert np.array_equal(got[:n], want)
     assert np.all(got[n:] == -1)
+
+
+def test_pipelined_driver_on_one_nccl_rank_equals_moe_forward_per_chunk():
+    """ep_forward_pipelined through a one-rank NCCL group: 192 tokens in three
+    chunks of 64 (the Hy3 decode shape per chunk), each chunk's output bitwise
+    moe_forward's on those tokens."""
+    import torch.distributed as dist
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1)
+    try:
+        shape = dataclasses.replace(CONFIGS["decode"], T=192)
+        L = make_layer(shape, seed=11, device="cuda")
+        cfg = moe.config_of(shape)
+        part = ep.Partition(shape.E, 1)
+        wgu, sgu, wd, sd = moe.layer_args(L)
+        ops = ep.ep_layer_ops(cfg, part, 0, L["w_gate"], L["gate_bias"], wgu, sgu, wd, sd)
+        y = ep.ep_forward_pipelined(ops, part, L["x"], chunks=3)
+        torch.cuda.synchronize()
+        for c in range(3):
+            xc = L["x"][64 * c:64 * (c + 1)].contiguous()
+            cc = moe.config_of(dataclasses.replace(shape, T=64))
+            ws = moe.workspace(cc)
+            want = torch.empty((64, shape.d), dtype=torch.bfloat16, device="cuda")
+            moe.moe_forward(cc, xc, L["w_gate"], L["gate_bias"], wgu, sgu, wd, sd, want, ws)
+            torch.cuda.synchronize()
+            assert moe.moe_read_status(ws) == moe.MOE_OK
+            assert torch.equal(y[64 * c:64 * (c + 1)], want), f"chunk {c}"
+    finally:
+        dist.destroy_process_group()
