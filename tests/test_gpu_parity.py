@@ -111,12 +111,13 @@ def test_hy3_shapes(name):
     _free(layer, out)
 
 
+@pytest.mark.parametrize("fmt", ["fp8", "fp4"])
 @pytest.mark.parametrize("T", [193, 700])
-def test_fp8_all_tokens_to_the_same_experts(T):
-    """FP8 weights on the pair GEMMs with every token on experts 0..3: T rows
-    each, in token tiles of at most 192 rows (193 as 128 + 65, 700 as
+def test_quantised_all_tokens_to_the_same_experts(T, fmt):
+    """FP8 / FP4 weights on the pair GEMMs with every token on experts 0..3: T
+    rows each, in token tiles of at most 192 rows (193 as 128 + 65, 700 as
     3 x 192 + 124); every token against the oracle."""
-    shape = LayerShape(T=T, d=512, E=16, k=4, F=256, fp8=True)
+    shape = LayerShape(T=T, d=512, E=16, k=4, F=256, fp8=fmt == "fp8", fp4=fmt == "fp4")
     layer = make_layer(shape, seed=5, device="cuda")
     b = torch.zeros(shape.E, dtype=torch.float32, device="cuda")
     b[:4] = 40.0
