@@ -449,25 +449,28 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 // as a shared-memory tile instead ran the tensor pipe at ~51% against ~57%,
 // the tile's writes and the MMA's reads competing with the raw reads. TMEM
 // then holds the accumulators and the op stages, which caps a token tile at
-// NM = 192 rows: gate_up g and u (2 x 192 columns) + 2 op stages of 64
-// (gate + up, one K block); down two accumulator stages (2 x 192) + 2 op
-// stages of 64 (two K blocks). (Smaller op stages, twice as many, measured
-// 8-10% slower on B200: more barrier and signal work for less conversion
-// each.)
+// NM = 192 rows. A pair tile takes two A tiles of 256 weight rows (128 per
+// CTA) against the same token rows -- gate_up: the gate rows m*256.. and the
+// up rows F + m*256..; down: the rows m*512.. and m*512 + 256.. -- so one
+// token stage feeds two MMAs per K step: two accumulators (2 x 192 columns)
+// + 2 op stages of 64 (both tiles' K block). (down with one A tile and a
+// double-buffered accumulator, each token stage feeding one MMA, ran 2-4%
+// slower for FP8 and 13% for FP4; smaller op stages, twice as many, 8-10%
+// slower: more barrier and signal work for less conversion each.) Where d is
+// an odd multiple of 256, down's last pair tile has its first A tile only.
 
 constexpr int THREADS_Q = 512;        // warps 6-14 converters, warp 15 token producer
 constexpr int MAX_RAW_STAGES = 16, MAX_B_STAGES = 4, MAX_OP_STAGES = 4;  // QCtrl's arrays
 template <bool GATE_UP, bool FP4>
 struct QShape {
-    static constexpr int A_TILES = GATE_UP ? 2 : 1;
+    static constexpr int A_TILES = 2;                              // A tiles per pair tile
     static constexpr int RAW_ROW = FP4 ? 32 : 64;                  // bytes of 64 codes
     static constexpr int RAW_TILE = BM * RAW_ROW;                  // 128 rows
     static constexpr int RAW_STAGE = A_TILES * RAW_TILE;
     static constexpr int NM = 192;                                 // token rows per pair tile
     static constexpr int BH = (NM / 2) * BK * 2;                   // a CTA's token half (bytes)
-    static constexpr int RAW_STAGES = FP4 ? 16 : (GATE_UP ? 8 : 12);
+    static constexpr int RAW_STAGES = FP4 ? 16 : 8;
     static constexpr int B_STAGES = 4;
-    static constexpr int KPO = GATE_UP ? 1 : 2;                    // K blocks per op stage
     static constexpr int OP_STAGES = 2;
     // converter warps: GROUPS groups of four (one per TMEM lane quarter) take
     // K blocks round-robin
@@ -478,13 +481,14 @@ struct QShape {
     static constexpr int SC_STAGES = 4;
     static constexpr int SC_BYTES = FP4 ? GROUPS * SC_STAGES * A_TILES * BM * 8 : 0;
     static constexpr int RING_BYTES = RAW_STAGES * RAW_STAGE + B_STAGES * BH + SC_BYTES;
-    static constexpr int ACC_STAGES = GATE_UP ? 1 : 2;
-    // TMEM columns: the accumulators, then the op stages
-    static constexpr int U_OFF = NM;                               // gate_up's up accumulator
-    static constexpr int ACC_COLS = GATE_UP ? 2 * NM : NM;
+    static constexpr int ACC_STAGES = 1;
+    // TMEM columns: the two accumulators, then the op stages
+    static constexpr int U_OFF = NM;                               // the second A tile's accumulator
+    static constexpr int ACC_COLS = 2 * NM;
     static constexpr int A_COL = ACC_STAGES * ACC_COLS;
     static constexpr int A_TILE_COLS = BK / 2;                     // one tile's K block: two bf16 a column
-    static constexpr int A_STAGE_COLS = A_TILES * KPO * A_TILE_COLS;  // 64
+    static constexpr int A_STAGE_COLS = A_TILES * A_TILE_COLS;     // 64
+    static constexpr int M_ROWS = GATE_UP ? 2 * BM : 4 * BM;       // weight rows per m (per expert)
 };
 
 constexpr int CONV_WARPS = 9;                          // warps 6..14 (warp 14 idles)
@@ -492,7 +496,7 @@ constexpr int TOKEN_WARP = 6 + CONV_WARPS;
 template <bool G, bool FP4>
 constexpr bool shape_ok() {
     using S = QShape<G, FP4>;
-    return S::RAW_STAGES % (S::KPO * S::GROUPS) == 0 && S::OP_STAGES % S::GROUPS == 0 &&
+    return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES % S::GROUPS == 0 &&
            S::GROUPS * S::GROUP_WARPS <= CONV_WARPS && S::GROUP_WARPS == 4 &&
            S::RAW_STAGES <= MAX_RAW_STAGES && S::B_STAGES <= MAX_B_STAGES &&
            S::OP_STAGES <= MAX_OP_STAGES && S::A_COL + S::OP_STAGES * S::A_STAGE_COLS <= 512 &&
@@ -686,6 +690,17 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     const uint32_t tmem_base = c.tmem_base;
     const int total = c.total;
     const volatile int* abort_flag = &c.abort;
+    // A pair tile's weight rows: this CTA's rows of the first A tile, the offset
+    // of the second's (gate_up: the up rows; down: 256 rows on), and whether
+    // the second exists (not in down's last tile where d is an odd multiple of
+    // 256).
+    const int b_off = GATE_UP ? a_rows_per_expert / 2 : 2 * BM;
+    auto first_row = [&](const TileInfo& ti) {
+        return ti.e * a_rows_per_expert + ti.m * S::M_ROWS + rank * BM;
+    };
+    auto has_second = [&](const TileInfo& ti) {
+        return GATE_UP || ti.m * S::M_ROWS + 2 * BM < a_rows_per_expert;
+    };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -698,7 +713,8 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             bool ok = true;
             for (int t = pair; t < total && ok; t += n_pairs) {
                 const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, t);
-                const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
+                const int a_row = first_row(ti);
+                const bool two = has_second(ti);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!tc::mbar_wait(&c.raw_empty[stage], phase ^ 1u, abort_flag)) {
                         raise_timeout(c, status);
@@ -706,12 +722,12 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                         break;
                     }
                     uint8_t* st = raw_ring + stage * S::RAW_STAGE;
-                    tc::mbar_arrive_expect_tx(&c.raw_full[stage], S::RAW_STAGE);
+                    tc::mbar_arrive_expect_tx(&c.raw_full[stage], two ? S::RAW_STAGE : S::RAW_TILE);
                     const int kx = kb * S::RAW_ROW;  // byte column of the K block's 64 codes
                     tc::tma_load_2d_hint(st, &tmA, &c.raw_full[stage], kx, a_row, pol_w);
-                    if (GATE_UP)
+                    if (two)  // (without it the stage's second tile holds stale codes, unused)
                         tc::tma_load_2d_hint(st + S::RAW_TILE, &tmA, &c.raw_full[stage], kx,
-                                             a_row + a_rows_per_expert / 2, pol_w);
+                                             a_row + b_off, pol_w);
                     issued[stage] = true;
                     parity[stage] = phase;
                     if (++stage == S::RAW_STAGES) {
@@ -804,95 +820,85 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
         const long sblocks = K / 32;
         const uint32_t sc_slot0 =
             tc::smem_u32(sc_ring) + (uint32_t)(group * S::SC_STAGES * S::A_TILES * BM * 8 + r * 8);
-        long fetch_it = -1, fetch_row = 0;  // the tile of the last fetch and its row
+        long fetch_it = -1, fetch_row = 0;  // the tile of the last fetch, its row
+        bool fetch_two = true;               // and whether it has a second A tile
         auto fetch_chunk = [&](long G) {  // one copy group per chunk, empty past the end
             if (G < n_chunks) {
                 const long it = G / (KB / 4);
                 const int q = (int)(G - it * (KB / 4));
                 if (it != fetch_it) {  // a new tile: one lookup per tile, not per chunk
                     const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, pair + (int)it * n_pairs);
-                    fetch_row = (long)ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM + r;
+                    fetch_row = (long)first_row(ti) + r;
+                    fetch_two = has_second(ti);
                     fetch_it = it;
                 }
                 const long row = fetch_row;
                 const uint32_t dst = sc_slot0 + (uint32_t)((G % S::SC_STAGES) * S::A_TILES * BM * 8);
 #pragma unroll
                 for (int a = 0; a < S::A_TILES; ++a)
-                    tc::cp_async8(dst + a * BM * 8,
-                                  scales8 + (row + a * (a_rows_per_expert / 2)) * sblocks + 8 * q);
+                    if (a == 0 || fetch_two)  // no scales past the expert's rows
+                        tc::cp_async8(dst + a * BM * 8, scales8 + (row + a * b_off) * sblocks + 8 * q);
             }
             tc::cp_async_commit();
         };
         uint2 sc_cur[S::A_TILES] = {};
         long cur_chunk = -1;
-        // a group fills the op stages ob = group, group + GROUPS, ..., each from
-        // the raw stages of its KPO K blocks j = KPO ob + kk
-        const long n_ops = n_blocks / S::KPO;
-        const long ob0 = group < S::GROUPS ? group : n_ops;
-        if (FP4 && ob0 < n_ops)
-            for (int g = 0; g < S::SC_STAGES - 1; ++g) fetch_chunk(((ob0 * S::KPO) >> 2) + g);
-        for (long ob = ob0; ob < n_ops; ob += S::GROUPS) {
-            const int os = (int)(ob % S::OP_STAGES);
-            const uint32_t oph = (uint32_t)(ob / S::OP_STAGES) & 1u;
-            uint32_t o[S::A_TILES * S::KPO * 32];  // (tile a, block kk) at o[32 (a KPO + kk) ..]
-            bool failed = false;  // the same in every thread of the group
-#pragma unroll
-            for (int kk = 0; kk < S::KPO; ++kk) {
-                const long jb = ob * S::KPO + kk;
-                const int rs = (int)(jb % S::RAW_STAGES);
-                const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
-                uint32_t sc[S::A_TILES] = {};  // FP4: this block's two scale bytes per A tile
-                if constexpr (FP4) {
-                    if ((jb >> 2) != cur_chunk) {
-                        cur_chunk = jb >> 2;
-                        // the slot of chunk G + SC_STAGES - 1 held chunk G - 1, read already
-                        fetch_chunk(cur_chunk + S::SC_STAGES - 1);
-                        tc::cp_async_wait_pending<S::SC_STAGES - 1>();  // chunk G has landed
-                        const uint32_t src =
-                            sc_slot0 + (uint32_t)((cur_chunk % S::SC_STAGES) * S::A_TILES * BM * 8);
-#pragma unroll
-                        for (int a = 0; a < S::A_TILES; ++a)
-                            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
-                                         : "=r"(sc_cur[a].x), "=r"(sc_cur[a].y)
-                                         : "r"(src + a * BM * 8));
-                    }
-                    const int kq = (int)(jb & 3);  // the block's place in its chunk
+        const long j0 = group < S::GROUPS ? group : n_blocks;
+        if (FP4 && j0 < n_blocks)
+            for (int g = 0; g < S::SC_STAGES - 1; ++g) fetch_chunk((j0 >> 2) + g);
+        for (long jb = j0; jb < n_blocks; jb += S::GROUPS) {
+            const int rs = (int)(jb % S::RAW_STAGES), os = (int)(jb % S::OP_STAGES);
+            const uint32_t rph = (uint32_t)(jb / S::RAW_STAGES) & 1u;
+            const uint32_t oph = (uint32_t)(jb / S::OP_STAGES) & 1u;
+            uint32_t sc[S::A_TILES] = {};  // FP4: this block's two scale bytes per A tile
+            if constexpr (FP4) {
+                if ((jb >> 2) != cur_chunk) {
+                    cur_chunk = jb >> 2;
+                    // the slot of chunk G + SC_STAGES - 1 held chunk G - 1, read already
+                    fetch_chunk(cur_chunk + S::SC_STAGES - 1);
+                    tc::cp_async_wait_pending<S::SC_STAGES - 1>();  // chunk G has landed
+                    const uint32_t src =
+                        sc_slot0 + (uint32_t)((cur_chunk % S::SC_STAGES) * S::A_TILES * BM * 8);
 #pragma unroll
                     for (int a = 0; a < S::A_TILES; ++a)
-                        sc[a] = ((kq < 2 ? sc_cur[a].x : sc_cur[a].y) >> (16 * (kq & 1))) & 0xFFFFu;
+                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                     : "=r"(sc_cur[a].x), "=r"(sc_cur[a].y)
+                                     : "r"(src + a * BM * 8));
                 }
-                const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
-                if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
-                    failed = true;
-                    break;
-                }
-                const uint32_t raw = raw0 + rs * S::RAW_STAGE;
-                constexpr int CHUNKS = S::RAW_ROW / 16;
-                uint32_t w[S::A_TILES][4 * CHUNKS];
+                const int kq = (int)(jb & 3);  // the block's place in its chunk
 #pragma unroll
                 for (int a = 0; a < S::A_TILES; ++a)
-#pragma unroll
-                    for (int ch = 0; ch < CHUNKS; ++ch)
-                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(w[a][4 * ch]), "=r"(w[a][4 * ch + 1]),
-                                       "=r"(w[a][4 * ch + 2]), "=r"(w[a][4 * ch + 3])
-                                     : "r"(raw + a * S::RAW_TILE + ((ch ^ rsw) << 4)));
-#pragma unroll
-                for (int a = 0; a < S::A_TILES; ++a) {
-                    uint32_t* oa = &o[32 * (a * S::KPO + kk)];
-                    if constexpr (FP4) {
-#pragma unroll
-                        for (int ch = 0; ch < 2; ++ch)
-                            e2m1x32_to_bf16(&w[a][4 * ch], (sc[a] >> (8 * ch)) & 0xFFu, oa + 16 * ch);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) e4m3x4_to_bf16x4(w[a][j], oa[2 * j], oa[2 * j + 1]);
-                    }
-                }
+                    sc[a] = ((kq < 2 ? sc_cur[a].x : sc_cur[a].y) >> (16 * (kq & 1))) & 0xFFFFu;
             }
-            if (failed) {
+            const bool rok = tc::mbar_wait(&c.raw_full[rs], rph, abort_flag);
+            if (tc::bar_any(2 + group, S::CONV_THREADS, !rok)) {  // the group leaves together
                 raise_timeout(c, status);
                 break;
+            }
+            const uint32_t raw = raw0 + rs * S::RAW_STAGE;
+            constexpr int CHUNKS = S::RAW_ROW / 16;
+            uint32_t w[S::A_TILES][4 * CHUNKS];
+#pragma unroll
+            for (int a = 0; a < S::A_TILES; ++a)
+#pragma unroll
+                for (int ch = 0; ch < CHUNKS; ++ch)
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[a][4 * ch]), "=r"(w[a][4 * ch + 1]),
+                                   "=r"(w[a][4 * ch + 2]), "=r"(w[a][4 * ch + 3])
+                                 : "r"(raw + a * S::RAW_TILE + ((ch ^ rsw) << 4)));
+            uint32_t o[S::A_TILES * 32];  // tile a in o[32 a ..], its TMEM columns in order
+#pragma unroll
+            for (int a = 0; a < S::A_TILES; ++a) {
+                if constexpr (FP4) {
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch)
+                        e2m1x32_to_bf16(&w[a][4 * ch], (sc[a] >> (8 * ch)) & 0xFFu,
+                                        &o[32 * a + 16 * ch]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        e4m3x4_to_bf16x4(w[a][j], o[32 * a + 2 * j], o[32 * a + 2 * j + 1]);
+                }
             }
             const bool ook = tc::mbar_wait(&c.op_empty[os], oph ^ 1u, abort_flag);
             if (tc::bar_any(2 + group, S::CONV_THREADS, !ook)) {
@@ -900,14 +906,12 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 break;
             }
             tc::fence_after_sync();  // the MMAs that read this op stage are complete
-            tc_store_row<S::A_TILES * S::KPO>(a_lane + os * S::A_STAGE_COLS, o);
+            tc_store_row<S::A_TILES>(a_lane + os * S::A_STAGE_COLS, o);
             tc::tmem_st_wait();
             tc::fence_before_sync();
             tc::bar_sync(2 + group, S::CONV_THREADS);
             if (ct == 0) {
-#pragma unroll
-                for (int kk = 0; kk < S::KPO; ++kk)
-                    tc::mbar_arrive(&c.raw_empty[(int)((ob * S::KPO + kk) % S::RAW_STAGES)]);
+                tc::mbar_arrive(&c.raw_empty[rs]);
                 if (leader)
                     tc::mbar_arrive_expect_tx(&c.op_full[os], 16);
                 else
@@ -935,45 +939,36 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 tc::fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
                 const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, ti.n);
-                for (int ob = 0; ob < KB / S::KPO && ok; ++ob) {
-                    if (!tc::mbar_wait(&c.op_full[os], oph, abort_flag)) {
+                const bool two = has_second(ti);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&c.op_full[os], oph, abort_flag) ||
+                        !tc::mbar_wait(&c.b_full[bs], bph, abort_flag)) {
                         raise_timeout(c, status);
                         ok = false;
                         break;
                     }
+                    tc::fence_after_sync();
                     const uint32_t a_tm = tmem_base + S::A_COL + os * S::A_STAGE_COLS;
+                    const uint32_t b_addr = tc::smem_u32(b_ring + bs * S::BH);
 #pragma unroll
-                    for (int kk = 0; kk < S::KPO; ++kk) {
-                        if (!tc::mbar_wait(&c.b_full[bs], bph, abort_flag)) {
-                            raise_timeout(c, status);
-                            ok = false;
-                            break;
-                        }
-                        tc::fence_after_sync();
-                        const int kb = ob * S::KPO + kk;
-                        const uint32_t b_addr = tc::smem_u32(b_ring + bs * S::BH);
-#pragma unroll
-                        for (int k = 0; k < BK / UK; ++k) {  // K = 16 of A is 8 TMEM columns
-                            const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
-                            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                            tc::mma_bf16_pair_ta(d_tmem, a_tm + kk * S::A_TILE_COLS + k * (UK / 2),
-                                                 bdesc, idesc, accum);
-                            if (GATE_UP)  // KPO = 1: the up tile follows the gate tile
-                                tc::mma_bf16_pair_ta(d_tmem + S::U_OFF,
-                                                     a_tm + S::A_TILE_COLS + k * (UK / 2), bdesc,
-                                                     idesc, accum);
-                        }
-                        if (kk == S::KPO - 1) tc::mma_commit_pair(&c.op_empty[os], 0x3);
-                        tc::mma_commit_pair(&c.b_empty[bs], 0x3);
-                        if (++bs == S::B_STAGES) {
-                            bs = 0;
-                            bph ^= 1u;
-                        }
+                    for (int k = 0; k < BK / UK; ++k) {  // K = 16 of A is 8 TMEM columns
+                        const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
+                        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                        tc::mma_bf16_pair_ta(d_tmem, a_tm + k * (UK / 2), bdesc, idesc, accum);
+                        if (two)  // the second A tile's columns follow the first's
+                            tc::mma_bf16_pair_ta(d_tmem + S::U_OFF,
+                                                 a_tm + S::A_TILE_COLS + k * (UK / 2), bdesc,
+                                                 idesc, accum);
                     }
-                    if (!ok) break;
+                    tc::mma_commit_pair(&c.op_empty[os], 0x3);
+                    tc::mma_commit_pair(&c.b_empty[bs], 0x3);
                     if (++os == S::OP_STAGES) {
                         os = 0;
                         oph ^= 1u;
+                    }
+                    if (++bs == S::B_STAGES) {
+                        bs = 0;
+                        bph ^= 1u;
                     }
                 }
                 if (ok) tc::mma_commit_pair(&c.acc_full[acc], 0x3);
@@ -1004,42 +999,49 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             tc::fence_after_sync();
             const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
-            const int col0 = ti.m * 2 * BM + rank * BM;
+            const int col0 = ti.m * S::M_ROWS + rank * BM;
+            const bool two = has_second(ti);
             const long srow = (long)ti.e * a_rows_per_expert + col0 + row_in_tile;
             // FP8: the row scales multiply the finished dot products; FP4 folded
             // its block scales into the widening
             const float sa = FP4 ? 1.f : __ldg(scales + srow);
-            const float sb = FP4 ? 1.f : GATE_UP ? __ldg(scales + srow + a_rows_per_expert / 2) : 0.f;
+            const float sb = (FP4 || !two) ? 1.f : __ldg(scales + srow + b_off);
+            // gate_up: h = SiLU(g) u from the two accumulators; down: the two
+            // accumulators are two 256-column ranges of y (part 1: 256 columns on)
             for (int c0 = 0; c0 < ti.n; c0 += EPI_N) {
-                uint32_t g[32];
-                tc::tmem_ld32(tbase + c0, g);
-                if constexpr (GATE_UP) {
-                    uint32_t u[32];
-                    tc::tmem_ld32(tbase + S::U_OFF + c0, u);
-                    tc::tmem_ld_wait();
+                for (int part = 0; part < (GATE_UP ? 1 : (two ? 2 : 1)); ++part) {
+                    uint32_t g[32];
+                    tc::tmem_ld32(tbase + part * S::U_OFF + c0, g);
+                    if constexpr (GATE_UP) {
+                        uint32_t u[32];
+                        tc::tmem_ld32(tbase + S::U_OFF + c0, u);
+                        tc::tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float gv = __uint_as_float(g[j]) * sa;
-                        const float uv = __uint_as_float(u[j]) * sb;
-                        epi[j * BM + row_in_tile] = float_to_bf16_bits(silu_mul(gv, uv));
+                        for (int j = 0; j < 32; ++j) {
+                            const float gv = __uint_as_float(g[j]) * sa;
+                            const float uv = __uint_as_float(u[j]) * sb;
+                            epi[j * BM + row_in_tile] = float_to_bf16_bits(silu_mul(gv, uv));
+                        }
+                    } else {
+                        tc::tmem_ld_wait();
+                        const float sp = part ? sb : sa;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            epi[j * BM + row_in_tile] = float_to_bf16_bits(__uint_as_float(g[j]) * sp);
                     }
-                } else {
-                    tc::tmem_ld_wait();
+                    tc::bar_sync(1, 128);  // the tile is written
+                    const int cp = col0 + part * b_off;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        epi[j * BM + row_in_tile] = float_to_bf16_bits(__uint_as_float(g[j]) * sa);
+                    for (int q = 0; q < EPI_N * BM / 8 / 128; ++q) {
+                        const int id = et + 128 * q;
+                        const int n = id / (BM / 8), ch = id % (BM / 8);
+                        if (c0 + n < ti.len)
+                            *reinterpret_cast<uint4*>(o16 + (size_t)(ti.row0 + c0 + n) * out_ld + cp +
+                                                      ch * 8) =
+                                *reinterpret_cast<const uint4*>(epi + n * BM + ch * 8);
+                    }
+                    tc::bar_sync(1, 128);  // the tile is read
                 }
-                tc::bar_sync(1, 128);  // the tile is written
-#pragma unroll
-                for (int q = 0; q < EPI_N * BM / 8 / 128; ++q) {
-                    const int id = et + 128 * q;
-                    const int n = id / (BM / 8), ch = id % (BM / 8);
-                    if (c0 + n < ti.len)
-                        *reinterpret_cast<uint4*>(o16 + (size_t)(ti.row0 + c0 + n) * out_ld + col0 +
-                                                  ch * 8) =
-                            *reinterpret_cast<const uint4*>(epi + n * BM + ch * 8);
-                }
-                tc::bar_sync(1, 128);  // the tile is read
             }
             // every warp's TMEM reads are complete before the accumulator is handed back
             tc::fence_before_sync();
@@ -1202,8 +1204,8 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
     if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
-    return launch_fp8<false>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y, c.d,
-                             status, s);
+    return launch_fp8<false>(a, b, offsets, s_down, c.E, c.d_ff, c.d, (c.d + 4 * BM - 1) / (4 * BM),
+                             y, c.d, status, s);
 }
 
 cudaError_t launch_gate_up_gemm_pair_fp4(const moe_config& c, const void* x_perm,
@@ -1229,8 +1231,8 @@ cudaError_t launch_down_gemm_pair_fp4(const moe_config& c, const void* h, const 
     if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff / 2, BM, 32, CU_TENSOR_MAP_SWIZZLE_32B) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
-    return launch_fp8<false, true>(a, b, offsets, s_down, c.E, c.d_ff, c.d, c.d / (2 * BM), y,
-                                   c.d, status, s);
+    return launch_fp8<false, true>(a, b, offsets, s_down, c.E, c.d_ff, c.d,
+                                   (c.d + 4 * BM - 1) / (4 * BM), y, c.d, status, s);
 }
 
 cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
