@@ -66,13 +66,21 @@ __device__ __forceinline__ void load_token_rows(uint8_t* dst, const TokenMaps& t
     }
 }
 
+// A pair tile takes two A tiles of 256 weight rows (128 per CTA) against the
+// same token rows -- gate_up: the gate rows m*256.. and the up rows
+// F + m*256..; down: the rows m*512.. and m*512 + 256.. -- into two TMEM
+// accumulators, so each token stage feeds two MMAs per K step. (down with one
+// A tile, a double-buffered accumulator and 6 stages ran 10% slower at the
+// Hy3 prefill shape and 1.5% slower at decode.) Where d is an odd multiple of
+// 256, down's last tile has its first A tile only.
 template <bool GATE_UP>
 struct Shape {
-    static constexpr int A_TILES = GATE_UP ? 2 : 1;
-    static constexpr int STAGE_BYTES = A_TILES * A_BYTES + BH_BYTES;  // 48 KB / 32 KB
-    static constexpr int STAGES = GATE_UP ? 4 : 6;
-    static constexpr int ACC_STAGES = GATE_UP ? 1 : 2;
-    static constexpr int ACC_COLS = GATE_UP ? 512 : 256;
+    static constexpr int A_TILES = 2;
+    static constexpr int STAGE_BYTES = A_TILES * A_BYTES + BH_BYTES;  // 48 KB
+    static constexpr int STAGES = 4;
+    static constexpr int ACC_STAGES = 1;
+    static constexpr int ACC_COLS = 512;                  // two accumulators of 256 columns
+    static constexpr int M_ROWS = GATE_UP ? 2 * BM : 4 * BM;  // weight rows per m (per expert)
 };
 
 struct Ctrl {
@@ -216,6 +224,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     const uint32_t tmem_base = c.tmem_base;
     const int total = c.total;
     const volatile int* abort_flag = &c.abort;
+    // the second A tile's row offset, and whether a tile has it (see Shape)
+    const int b_off = GATE_UP ? a_rows_per_expert / 2 : 2 * BM;
+    auto has_second = [&](const TileInfo& ti) {
+        return GATE_UP || ti.m * S::M_ROWS + 2 * BM < a_rows_per_expert;
+    };
 
     if (warp == 0) {
         // ---------------- producer: this CTA's weight rows and token half. Lane 0
@@ -233,9 +246,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int t = pair; t < total && ok; t += n_pairs) {
             const TileInfo ti = decode_tile(c, E, m_tiles, t);
             const int half = ti.n / 2;
-            const int a_row = ti.e * a_rows_per_expert + ti.m * 2 * BM + rank * BM;
+            const int a_row = ti.e * a_rows_per_expert + ti.m * S::M_ROWS + rank * BM;
             const int b_row = ti.row0 + rank * half;
-            const uint32_t pair_bytes = 2u * (S::A_TILES * A_BYTES + half * BK * 2);
+            const bool two = has_second(ti);
+            const uint32_t pair_bytes = 2u * ((two ? 2 : 1) * A_BYTES + half * BK * 2);
             int tok[4] = {0, 0, 0, 0};
             if (GATHER) {
                 // rows past the tile's end repeat its first row (in range, ignored)
@@ -261,15 +275,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         // 128 x 64 blocks stored contiguously: block (row / 128, kb)
                         tc::tma_load_2d_pair(s, &tmA, full_leader, 0, ((a_row / BM) * KB + kb) * BM,
                                              pol_w);
-                        if (GATE_UP)
-                            tc::tma_load_2d_pair(
-                                s + A_BYTES, &tmA, full_leader, 0,
-                                (((a_row + a_rows_per_expert / 2) / BM) * KB + kb) * BM, pol_w);
+                        if (two)
+                            tc::tma_load_2d_pair(s + A_BYTES, &tmA, full_leader, 0,
+                                                 (((a_row + b_off) / BM) * KB + kb) * BM, pol_w);
                     } else {
                         tc::tma_load_2d_pair(s, &tmA, full_leader, kb * BK, a_row, pol_w);
-                        if (GATE_UP)
+                        if (two)
                             tc::tma_load_2d_pair(s + A_BYTES, &tmA, full_leader, kb * BK,
-                                                 a_row + a_rows_per_expert / 2, pol_w);
+                                                 a_row + b_off, pol_w);
                     }
                     if (!GATHER)
                         load_token_rows(sb, tmB, full_leader, kb * BK, b_row, half, pol_x);
@@ -314,6 +327,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                 tc::fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
                 const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, ti.n);
+                const bool two = has_second(ti);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!tc::mbar_wait(&c.full[stage], phase, abort_flag)) {
                         raise_timeout(c, status);
@@ -329,7 +343,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
                         tc::mma_bf16_pair(d_tmem, tc::desc_sw128(a_addr + k * UK * 2), bdesc,
                                           idesc, accum);
-                        if (GATE_UP)
+                        if (two)
                             tc::mma_bf16_pair(d_tmem + 256,
                                               tc::desc_sw128(a_addr + A_BYTES + k * UK * 2), bdesc,
                                               idesc, accum);
@@ -372,10 +386,15 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             tc::fence_after_sync();
             const uint32_t tbase = tmem_base + acc * S::ACC_COLS + ((uint32_t)(quad * 32) << 16);
-            const int col0 = ti.m * 2 * BM + rank * BM;
-            for (int c0 = grp * EPI_N; c0 < ti.n; c0 += EPI_GROUPS * EPI_N) {
+            const int col0 = ti.m * S::M_ROWS + rank * BM;
+            const int parts = GATE_UP ? 1 : (has_second(ti) ? 2 : 1);
+            // gate_up: h = SiLU(g) u from the two accumulators; down: the two
+            // accumulators are two 256-column ranges of y (part 1: 256 columns on)
+            for (int cc = grp; cc < parts * ((ti.n + EPI_N - 1) / EPI_N); cc += EPI_GROUPS) {
+                const int nch = (ti.n + EPI_N - 1) / EPI_N;
+                const int part = cc / nch, c0 = (cc - part * nch) * EPI_N;
                 uint32_t g[32];
-                tc::tmem_ld32(tbase + c0, g);
+                tc::tmem_ld32(tbase + part * 256 + c0, g);
                 if constexpr (GATE_UP) {
                     uint32_t u[32];
                     tc::tmem_ld32(tbase + 256 + c0, u);
@@ -398,7 +417,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                     const int n = id / (BM / 8), ch = id % (BM / 8);
                     if (c0 + n < ti.len)
                         *reinterpret_cast<uint4*>(o16 + (size_t)(ti.row0 + c0 + n) * out_ld + col0 +
-                                                  ch * 8) =
+                                                  part * b_off + ch * 8) =
                             *reinterpret_cast<const uint4*>(tile + n * BM + ch * 8);
                 }
                 tc::bar_sync(bar_grp, 128);  // the group's tile is read
@@ -1270,8 +1289,8 @@ cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int3
     if (!make_weight_map(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, packed) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
-    return launch<false>(a, b, offsets, c.E, c.d_ff, c.d, c.d / (2 * BM), packed, y, c.d, status,
-                         s);
+    return launch<false>(a, b, offsets, c.E, c.d_ff, c.d, (c.d + 4 * BM - 1) / (4 * BM), packed, y,
+                         c.d, status, s);
 }
 
 namespace {
