@@ -38,7 +38,6 @@ constexpr int NMAX = 256;     // token rows per pair tile
 constexpr int NBOX = 16;      // token rows per TMA box
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int BOX_BYTES = NBOX * BK * 2;
-constexpr int BH_BYTES = (NMAX / 2) * BK * 2;  // this CTA's half of the token rows
 constexpr int EPI_GROUPS = 2;                      // epilogue warp groups (4 warps each)
 constexpr int THREADS = 64 + 128 * EPI_GROUPS;     // producer, MMA, epilogue warps
 constexpr int MAX_E = 256;
@@ -73,15 +72,25 @@ __device__ __forceinline__ void load_token_rows(uint8_t* dst, const TokenMaps& t
 // A tile, a double-buffered accumulator and 6 stages ran 10% slower at the
 // Hy3 prefill shape and 1.5% slower at decode.) Where d is an odd multiple of
 // 256, down's last tile has its first A tile only.
-template <bool GATE_UP>
+//
+// NM, the most token rows of a pair tile: 256, or 64 where no expert can have
+// more rows (T <= 64: a token takes an expert once). With NM = 64 a stage
+// holds 4 KB of token rows instead of 16, so the ring is 5 stages deep (the
+// weight stream is HBM-bound and a shallower ring measured slower), and the
+// two accumulators of 64 columns are double-buffered (the epilogue of a tile
+// overlaps the next tile's MMAs).
+template <bool GATE_UP, int NM = NMAX>
 struct Shape {
     static constexpr int A_TILES = 2;
-    static constexpr int STAGE_BYTES = A_TILES * A_BYTES + BH_BYTES;  // 48 KB
-    static constexpr int STAGES = 4;
-    static constexpr int ACC_STAGES = 1;
-    static constexpr int ACC_COLS = 512;                  // two accumulators of 256 columns
+    static constexpr int BH = (NM / 2) * BK * 2;          // this CTA's half of the token rows
+    static constexpr int STAGE_BYTES = A_TILES * A_BYTES + BH;  // 48 KB / 36 KB
+    static constexpr int STAGES = NM == NMAX ? 4 : 5;
+    static constexpr int U_OFF = NM;                      // the second accumulator's columns
+    static constexpr int ACC_COLS = 2 * NM;               // two accumulators
+    static constexpr int ACC_STAGES = 512 / ACC_COLS >= 2 ? 2 : 1;
     static constexpr int M_ROWS = GATE_UP ? 2 * BM : 4 * BM;  // weight rows per m (per expert)
 };
+constexpr int NM_SMALL = 64;
 
 struct Ctrl {
     uint64_t full[6];       // even CTA: TMA bytes of both CTAs landed
@@ -96,11 +105,16 @@ struct Ctrl {
     int tile_start[MAX_E + 1];
 };
 
-template <bool GATE_UP>
+template <bool GATE_UP, int NM>
 constexpr int smem_bytes() {
-    return Shape<GATE_UP>::STAGES * Shape<GATE_UP>::STAGE_BYTES + EPI_BYTES + 1024 +
+    return Shape<GATE_UP, NM>::STAGES * Shape<GATE_UP, NM>::STAGE_BYTES + EPI_BYTES + 1024 +
            (int)sizeof(Ctrl);
 }
+static_assert(smem_bytes<true, NMAX>() <= 232448 && smem_bytes<false, NMAX>() <= 232448 &&
+                  smem_bytes<true, NM_SMALL>() <= 232448 && smem_bytes<false, NM_SMALL>() <= 232448,
+              "fits in 227 KB");
+static_assert(Shape<true, NM_SMALL>::STAGES <= 6 && Shape<true, NMAX>::STAGES <= 6,
+              "Ctrl's stage barriers");
 
 struct TileInfo {
     int e, m, row0, len, n;  // n: MMA N of the pair, a multiple of 2*NBOX
@@ -151,14 +165,14 @@ __device__ __forceinline__ void raise_timeout(CtrlT& c, int* status) {
 // GATHER: tmB maps the unpermuted token rows x [T, K] with a one-row box and
 // the token rows of each tile are gathered by index (token_of_row) with
 // tile::gather4 instead of being read from a permuted copy.
-template <bool GATE_UP, bool GATHER>
+template <bool GATE_UP, bool GATHER, int NM>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ TokenMaps tmB, const int* __restrict__ offsets,
                          const int* __restrict__ token_of_row, int E, int K,
                          int a_rows_per_expert, int m_tiles, int packed_a,
                          __nv_bfloat16* __restrict__ out, int out_ld, int* __restrict__ status) {
-    using S = Shape<GATE_UP>;
+    using S = Shape<GATE_UP, NM>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -183,7 +197,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             __syncwarp();
             if (e < E) {
                 const int n_e = offsets[e + 1] - o;
-                cnt = ((n_e + NMAX - 1) / NMAX) * m_tiles;
+                cnt = ((n_e + NM - 1) / NM) * m_tiles;
             }
             int incl = cnt;
 #pragma unroll
@@ -244,7 +258,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         bool ok = true;
         if (!GATHER && lane != 0) ok = false;  // the copy path issues from lane 0 alone
         for (int t = pair; t < total && ok; t += n_pairs) {
-            const TileInfo ti = decode_tile(c, E, m_tiles, t);
+            const TileInfo ti = decode_tile<NM>(c, E, m_tiles, t);
             const int half = ti.n / 2;
             const int a_row = ti.e * a_rows_per_expert + ti.m * S::M_ROWS + rank * BM;
             const int b_row = ti.row0 + rank * half;
@@ -317,7 +331,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             bool ok = true;
             int it = 0;
             for (int t = pair; t < total && ok; t += n_pairs, ++it) {
-                const TileInfo ti = decode_tile(c, E, m_tiles, t);
+                const TileInfo ti = decode_tile<NM>(c, E, m_tiles, t);
                 const int acc = it % S::ACC_STAGES;
                 const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
                 if (!tc::mbar_wait(&c.acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -344,7 +358,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         tc::mma_bf16_pair(d_tmem, tc::desc_sw128(a_addr + k * UK * 2), bdesc,
                                           idesc, accum);
                         if (two)
-                            tc::mma_bf16_pair(d_tmem + 256,
+                            tc::mma_bf16_pair(d_tmem + S::U_OFF,
                                               tc::desc_sw128(a_addr + A_BYTES + k * UK * 2), bdesc,
                                               idesc, accum);
                     }
@@ -376,7 +390,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         const bool arriver = (warp == 2 && lane == 0);
         int it = 0;
         for (int t = pair; t < total; t += n_pairs, ++it) {
-            const TileInfo ti = decode_tile(c, E, m_tiles, t);
+            const TileInfo ti = decode_tile<NM>(c, E, m_tiles, t);
             const int acc = it % S::ACC_STAGES;
             const uint32_t acc_phase = (uint32_t)(it / S::ACC_STAGES) & 1u;
             const bool waited = tc::mbar_wait(&c.acc_full[acc], acc_phase, abort_flag);
@@ -394,10 +408,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                 const int nch = (ti.n + EPI_N - 1) / EPI_N;
                 const int part = cc / nch, c0 = (cc - part * nch) * EPI_N;
                 uint32_t g[32];
-                tc::tmem_ld32(tbase + part * 256 + c0, g);
+                tc::tmem_ld32(tbase + part * S::U_OFF + c0, g);
                 if constexpr (GATE_UP) {
                     uint32_t u[32];
-                    tc::tmem_ld32(tbase + 256 + c0, u);
+                    tc::tmem_ld32(tbase + S::U_OFF + c0, u);
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
@@ -1141,13 +1155,12 @@ int sm_pairs() {
     return (n > 1 ? n : 148) / 2;
 }
 
-template <bool GATE_UP, bool GATHER = false>
-cudaError_t launch(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets, int E,
-                   int K, int a_rows_per_expert, int m_tiles, bool packed_a, void* out,
-                   int out_ld, int* status, cudaStream_t s,
-                   const int32_t* token_of_row = nullptr) {
-    const int smem = smem_bytes<GATE_UP>();
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATE_UP, GATHER>,
+template <bool GATE_UP, bool GATHER, int NM>
+cudaError_t launch_nm(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets, int E,
+                      int K, int a_rows_per_expert, int m_tiles, bool packed_a, void* out,
+                      int out_ld, int* status, cudaStream_t s, const int32_t* token_of_row) {
+    const int smem = smem_bytes<GATE_UP, NM>();
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATE_UP, GATHER, NM>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -1162,11 +1175,27 @@ cudaError_t launch(const CUtensorMap& a, const TokenMaps& b, const int32_t* offs
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATE_UP, GATHER>, a, b, offsets,
+    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATE_UP, GATHER, NM>, a, b, offsets,
                              token_of_row, E, K, a_rows_per_expert, m_tiles, (int)packed_a,
                              static_cast<__nv_bfloat16*>(out), out_ld, status);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
+}
+
+// T <= 64: no expert has more than T rows (a token takes an expert once), so
+// the tiles hold at most NM_SMALL token rows (more rows would only take more
+// tiles, any NM is correct for any grouping).
+template <bool GATE_UP, bool GATHER = false>
+cudaError_t launch(int T, const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets, int E,
+                   int K, int a_rows_per_expert, int m_tiles, bool packed_a, void* out,
+                   int out_ld, int* status, cudaStream_t s,
+                   const int32_t* token_of_row = nullptr) {
+    if (T <= NM_SMALL)
+        return launch_nm<GATE_UP, GATHER, NM_SMALL>(a, b, offsets, E, K, a_rows_per_expert,
+                                                     m_tiles, packed_a, out, out_ld, status, s,
+                                                     token_of_row);
+    return launch_nm<GATE_UP, GATHER, NMAX>(a, b, offsets, E, K, a_rows_per_expert, m_tiles,
+                                            packed_a, out, out_ld, status, s, token_of_row);
 }
 
 template <bool GATE_UP, bool FP4 = false>
@@ -1263,7 +1292,7 @@ cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
     if (!make_weight_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, packed) ||
         !make_token_maps(&b, x_perm, R, c.d))
         return cudaErrorInvalidValue;
-    return launch<true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), packed, h, c.d_ff,
+    return launch<true>(c.T, a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), packed, h, c.d_ff,
                         status, s);
 }
 
@@ -1276,7 +1305,7 @@ cudaError_t launch_gate_up_gemm_pair_gather(const moe_config& c, const void* x,
     if (!make_weight_map(&a, w_gate_up, (uint64_t)c.E * 2 * c.d_ff, c.d, packed) ||
         !make_map(&b.m[0], x, (uint64_t)c.T, c.d, 1))
         return cudaErrorInvalidValue;
-    return launch<true, true>(a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), packed, h,
+    return launch<true, true>(c.T, a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), packed, h,
                               c.d_ff, status, s, token_of_row);
 }
 
@@ -1289,7 +1318,7 @@ cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int3
     if (!make_weight_map(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, packed) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
-    return launch<false>(a, b, offsets, c.E, c.d_ff, c.d, (c.d + 4 * BM - 1) / (4 * BM), packed, y,
+    return launch<false>(c.T, a, b, offsets, c.E, c.d_ff, c.d, (c.d + 4 * BM - 1) / (4 * BM), packed, y,
                          c.d, status, s);
 }
 
