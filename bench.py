@@ -319,10 +319,17 @@ def measure(args, name, dev, local, rank, world, pg, moe, block=False, cpu_secon
         pg.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
+        # the timed steps run as a user runs them: the layer's launches back to
+        # back (an event between two kernels would stop the next one from
+        # launching while the previous one finishes)
         t_begin.record(stream)
         for i in range(args.steps):
-            step(evs[i])
+            step()
         t_end.record(stream)
+        stream.synchronize()
+        # the stage breakdown: the same steps again, an event between stages
+        for i in range(args.steps):
+            step(evs[i])
         stream.synchronize()
     torch.cuda.synchronize(dev)
     if pg:
@@ -468,6 +475,8 @@ def measure(args, name, dev, local, rank, world, pg, moe, block=False, cpu_secon
             "algorithmic_bytes": lw["bytes"], "algorithmic_flops": lw["flops"],
             "touched_experts": touched},
         "stage_ms": stage_ms,
+        "stage_timing": "a second pass of the same steps with an event between stages "
+                        "(value and ms_per_step come from the pass without them)",
         "clocks": clocks.summary(),
         "e2e": {"value": replica_value(T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,

@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(CT)
 combine_kernel(const __nv_bfloat16* __restrict__ y, const int* __restrict__ row_of,
                const float* __restrict__ w, int k_routed, int k, int d,
                __nv_bfloat16* __restrict__ out) {
+    pdl_launch_and_wait();
     // k slots per token; slots at and past k_routed (the shared expert) weigh 1
     __shared__ int rows[33];
     __shared__ float wts[33];
@@ -71,10 +72,11 @@ combine_kernel(const __nv_bfloat16* __restrict__ y, const int* __restrict__ row_
 cudaError_t launch_combine(const moe_config& c, const void* y, const int32_t* row_of,
                            const float* topk_w, void* out, cudaStream_t s) {
     const dim3 grid(c.T, (c.d / 8 + CT - 1) / CT);
-    combine_kernel<<<grid, CT, 0, s>>>(static_cast<const __nv_bfloat16*>(y), row_of, topk_w, c.k,
+    const cudaError_t err = launch_pdl(combine_kernel, grid, dim3(CT), 0, s,
+                                       static_cast<const __nv_bfloat16*>(y), row_of, topk_w, c.k,
                                        c.k + shared_slots(c), c.d,
                                        static_cast<__nv_bfloat16*>(out));
-    return cudaGetLastError();
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

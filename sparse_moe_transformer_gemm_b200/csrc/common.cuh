@@ -213,6 +213,17 @@ __device__ __forceinline__ void warp_select_topk(float (&sc)[8], int k, float sc
 // SwiGLU's SiLU(g) * u with the fast exponential and division intrinsics: their
 // relative error (~1e-6) sits far below the bf16 rounding of the result
 // (2^-9), and for g below about -87 the quotient is 0, SiLU's limit.
+// Programmatic dependent launch: let the next kernel on the stream begin
+// launching (its thread blocks take SMs as this grid's leave, and wait in
+// their own pdl_launch_and_wait), then wait until the previous kernel on the
+// stream has completed and its writes are visible. Every kernel of the layer
+// calls this before it touches global memory; for a launch without the
+// programmatic-serialization attribute both steps do nothing.
+__device__ __forceinline__ void pdl_launch_and_wait() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }

@@ -17,6 +17,7 @@
 // order), then each thread takes rows of the CTA's chunk and finds its segment
 // by binary search over the prefix sums. Rows at or past the counts' total
 // get -1.
+#include "common.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -28,6 +29,7 @@ constexpr int EP_ROWS_PER_CTA = 4096;
 __global__ void __launch_bounds__(EP_THREADS)
 ep_row_experts_kernel(const int32_t* __restrict__ counts, int n_seg, int e_local,
                       int32_t* __restrict__ expert_of_row, int n_rows) {
+    pdl_launch_and_wait();
     extern __shared__ int start[];  // [n_seg + 1] exclusive prefix sums
     __shared__ int warp_tot[EP_THREADS / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -85,9 +87,10 @@ cudaError_t launch_ep_row_experts(const int32_t* counts, int n_src, int e_local,
                                   int32_t* expert_of_row, int n_rows, cudaStream_t s) {
     const int n_seg = n_src * e_local;
     const int grid = (n_rows + EP_ROWS_PER_CTA - 1) / EP_ROWS_PER_CTA;
-    ep_row_experts_kernel<<<grid, EP_THREADS, sizeof(int) * (n_seg + 1), s>>>(
-        counts, n_seg, e_local, expert_of_row, n_rows);
-    return cudaGetLastError();
+    const cudaError_t err = launch_pdl(ep_row_experts_kernel, grid, dim3(EP_THREADS),
+                                       sizeof(int) * (n_seg + 1), s, counts, n_seg, e_local,
+                                       expert_of_row, n_rows);
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

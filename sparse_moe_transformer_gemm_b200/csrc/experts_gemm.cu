@@ -139,6 +139,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const int* __restrict__ offsets, int E, int K, int a_rows_per_expert,
                     int m_tiles, __nv_bfloat16* __restrict__ out, int out_ld,
                     int* __restrict__ status) {
+    pdl_launch_and_wait();
     using S = Shape<GATE_UP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -433,10 +434,10 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const int32_t* of
     cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<GATE_UP>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    grouped_gemm_kernel<GATE_UP><<<sm_count(), THREADS, smem, s>>>(
-        a, b, offsets, E, K, a_rows_per_expert, m_tiles, static_cast<__nv_bfloat16*>(out), out_ld,
-        status);
-    return cudaGetLastError();
+    err = launch_pdl(grouped_gemm_kernel<GATE_UP>, dim3(sm_count()), dim3(THREADS), smem, s, a, b,
+                     offsets, E, K, a_rows_per_expert, m_tiles, static_cast<__nv_bfloat16*>(out),
+                     out_ld, status);
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace

@@ -172,6 +172,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const int* __restrict__ token_of_row, int E, int K,
                          int a_rows_per_expert, int m_tiles, int packed_a,
                          __nv_bfloat16* __restrict__ out, int out_ld, int* __restrict__ status) {
+    pdl_launch_and_wait();
     using S = Shape<GATE_UP, NM>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -645,6 +646,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                              int E, int K, int a_rows_per_expert, int m_tiles,
                              __nv_bfloat16* __restrict__ out, int out_ld,
                              int* __restrict__ status) {
+    pdl_launch_and_wait();
     using S = QShape<GATE_UP, FP4>;
     const float* __restrict__ scales = static_cast<const float*>(scales_v);
     const uint8_t* __restrict__ scales8 = static_cast<const uint8_t*>(scales_v);
@@ -1168,13 +1170,15 @@ cudaError_t launch_nm(const CUtensorMap& a, const TokenMaps& b, const int32_t* o
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATE_UP, GATHER, NM>, a, b, offsets,
                              token_of_row, E, K, a_rows_per_expert, m_tiles, (int)packed_a,
                              static_cast<__nv_bfloat16*>(out), out_ld, status);
@@ -1211,13 +1215,15 @@ cudaError_t launch_fp8(const CUtensorMap& a, const TokenMaps& b, const int32_t* 
     cfg.blockDim = dim3(THREADS_Q, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_fp8_kernel<GATE_UP, FP4>, a, b, offsets, scales, E,
                              K, a_rows_per_expert, m_tiles, static_cast<__nv_bfloat16*>(out),
                              out_ld, status);

@@ -223,6 +223,7 @@ __global__ void __launch_bounds__(SWARPS * 32)
 gate_up_stream_kernel(const __nv_bfloat16* __restrict__ xperm, const int* __restrict__ offsets,
                       const uint8_t* __restrict__ wgu, const void* __restrict__ s_gu,
                       __nv_bfloat16* __restrict__ h, int d, int F) {
+    pdl_launch_and_wait();
     extern __shared__ __align__(16) uint8_t smem[];
     __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
     const int e = blockIdx.y;
@@ -257,6 +258,7 @@ __global__ void __launch_bounds__(SWARPS * 32)
 down_stream_kernel(const __nv_bfloat16* __restrict__ h, const int* __restrict__ offsets,
                    const uint8_t* __restrict__ wd, const void* __restrict__ s_d,
                    __nv_bfloat16* __restrict__ y, int d, int F) {
+    pdl_launch_and_wait();
     extern __shared__ __align__(16) uint8_t smem[];
     __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(smem);
     const int e = blockIdx.y;
@@ -304,10 +306,11 @@ cudaError_t gate_up(const moe_config& c, const void* x_perm, const int32_t* offs
     const dim3 grid((c.d_ff + ROWS_PER_CTA - 1) / ROWS_PER_CTA, c.E);
     cudaError_t err = set_smem(gate_up_stream_kernel<FMT>, smem);
     if (err != cudaSuccess) return err;
-    gate_up_stream_kernel<FMT><<<grid, SWARPS * 32, smem, s>>>(
+    err = launch_pdl(
+        gate_up_stream_kernel<FMT>, grid, dim3(SWARPS * 32), smem, s,
         static_cast<const __nv_bfloat16*>(x_perm), offsets, static_cast<const uint8_t*>(w_gate_up),
         s_gate_up, static_cast<__nv_bfloat16*>(h), c.d, c.d_ff);
-    return cudaGetLastError();
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 template <int FMT>
@@ -317,10 +320,11 @@ cudaError_t down(const moe_config& c, const void* h, const int32_t* offsets, con
     const dim3 grid((c.d + ROWS_PER_CTA - 1) / ROWS_PER_CTA, c.E);
     cudaError_t err = set_smem(down_stream_kernel<FMT>, smem);
     if (err != cudaSuccess) return err;
-    down_stream_kernel<FMT><<<grid, SWARPS * 32, smem, s>>>(
+    err = launch_pdl(
+        down_stream_kernel<FMT>, grid, dim3(SWARPS * 32), smem, s,
         static_cast<const __nv_bfloat16*>(h), offsets, static_cast<const uint8_t*>(w_down), s_down,
         static_cast<__nv_bfloat16*>(y), c.d, c.d_ff);
-    return cudaGetLastError();
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -16,6 +18,26 @@ constexpr int kPermuteChunk = 2048;     // token-slots per ranking chunk
 constexpr int kStreamMaxTokens = 8;     // rows per pass of the streaming expert kernels
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Launch a kernel of the layer with programmatic stream serialization: it may
+// begin launching while the previous kernel on the stream finishes (each
+// kernel waits for its predecessor in pdl_launch_and_wait before it touches
+// global memory), which hides the launch gap between consecutive kernels.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Byte offsets of every workspace region. The control words (status word and
 // router counters) come first so that one memset clears them.

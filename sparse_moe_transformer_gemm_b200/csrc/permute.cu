@@ -78,6 +78,7 @@ constexpr int SUB = CH / RW;
 
 __global__ void __launch_bounds__(RW * 32)
 permute_rank_kernel(Slots sl, long R, int E, int* __restrict__ hist, int* __restrict__ rank) {
+    pdl_launch_and_wait();
     __shared__ int cnt[RW][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < RW * 256; i += blockDim.x) cnt[i >> 8][i & 255] = 0;
@@ -119,6 +120,7 @@ permute_rank_kernel(Slots sl, long R, int E, int* __restrict__ hist, int* __rest
 __global__ void __launch_bounds__(256)
 permute_scan_kernel(int* __restrict__ hist, int C, int E, int* __restrict__ counts,
                     int* __restrict__ offsets) {
+    pdl_launch_and_wait();
     __shared__ int tile[32][256];
     __shared__ int tot[256];
     const int e = threadIdx.x;
@@ -176,6 +178,7 @@ permute_scatter_kernel(Slots sl, const int* __restrict__ hist, const int* __rest
                        const int* __restrict__ offsets, const __nv_bfloat16* __restrict__ x,
                        long R, int E, int d, int* __restrict__ row_of,
                        __nv_bfloat16* __restrict__ xperm) {
+    pdl_launch_and_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long s = (long)blockIdx.x * 8 + warp;
     if (s >= R) return;
@@ -200,6 +203,7 @@ __global__ void __launch_bounds__(256)
 permute_index_kernel(Slots sl, const int* __restrict__ hist, const int* __restrict__ rank,
                      const int* __restrict__ offsets, long R, int E, int* __restrict__ row_of,
                      int* __restrict__ token_of_row) {
+    pdl_launch_and_wait();
     const long s = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= R) return;
     const int e = slot_expert(sl, s);
@@ -225,6 +229,7 @@ __global__ void __launch_bounds__(SW * 32)
 permute_small_kernel(Slots sl, long R, int E, int* __restrict__ counts,
                      int* __restrict__ offsets, int* __restrict__ row_of,
                      int* __restrict__ token_of_row) {
+    pdl_launch_and_wait();
     __shared__ int cnt[SW][256];
     __shared__ int base[256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,6 +312,7 @@ __global__ void __launch_bounds__(256)
 gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ token_of_row,
                    const int* __restrict__ offsets, long R, int E, int d,
                    __nv_bfloat16* __restrict__ xperm) {
+    pdl_launch_and_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long row = (long)blockIdx.x * 8 + warp;
     if (row >= R || row >= offsets[E]) return;
@@ -324,26 +330,30 @@ cudaError_t launch_permute_index(const moe_config& c, const int32_t* idx, int32_
     const Slots sl = slots_of(c, idx);
     const long R = (long)g.T * g.k;
     if (R <= kSmallSlots) {
-        permute_small_kernel<<<1, SW * 32, 0, s>>>(sl, R, g.E, counts, offsets, row_of,
-                                                   token_of_row);
-        return cudaGetLastError();
+        const cudaError_t err = launch_pdl(permute_small_kernel, dim3(1), dim3(SW * 32), 0, s, sl,
+                                           R, g.E, counts, offsets, row_of, token_of_row);
+        return err != cudaSuccess ? err : cudaGetLastError();
     }
     const int C = n_permute_chunks(g);
-    permute_rank_kernel<<<C, RW * 32, 0, s>>>(sl, R, g.E, hist, rank);
-    permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, g.E, counts, offsets);
-    permute_index_kernel<<<(unsigned)((R + 255) / 256), 256, 0, s>>>(sl, hist, rank, offsets, R,
-                                                                     g.E, row_of, token_of_row);
-    return cudaGetLastError();
+    cudaError_t err = launch_pdl(permute_rank_kernel, dim3(C), dim3(RW * 32), 0, s, sl, R, g.E,
+                                 hist, rank);
+    if (err == cudaSuccess)
+        err = launch_pdl(permute_scan_kernel, dim3(1), dim3(256), 0, s, hist, C, g.E, counts,
+                         offsets);
+    if (err == cudaSuccess)
+        err = launch_pdl(permute_index_kernel, dim3((unsigned)((R + 255) / 256)), dim3(256), 0, s,
+                         sl, hist, rank, offsets, R, g.E, row_of, token_of_row);
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const moe_config& c, const void* x, const int32_t* token_of_row,
                                const int32_t* offsets, void* x_perm, cudaStream_t s) {
     const moe_config g = grouped_config(c);
     const long R = (long)g.T * g.k;
-    gather_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), token_of_row, offsets, R, g.E, c.d,
-        static_cast<__nv_bfloat16*>(x_perm));
-    return cudaGetLastError();
+    const cudaError_t err = launch_pdl(gather_rows_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256),
+                                       0, s, static_cast<const __nv_bfloat16*>(x), token_of_row,
+                                       offsets, R, g.E, c.d, static_cast<__nv_bfloat16*>(x_perm));
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* x, int32_t* counts,
@@ -353,12 +363,16 @@ cudaError_t launch_permute(const moe_config& c, const int32_t* idx, const void* 
     const Slots sl = slots_of(c, idx);
     const long R = (long)g.T * g.k;
     const int C = n_permute_chunks(g);
-    permute_rank_kernel<<<C, RW * 32, 0, s>>>(sl, R, g.E, hist, rank);
-    permute_scan_kernel<<<1, 256, 0, s>>>(hist, C, g.E, counts, offsets);
-    permute_scatter_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(
-        sl, hist, rank, offsets, static_cast<const __nv_bfloat16*>(x), R, g.E, c.d, row_of,
-        static_cast<__nv_bfloat16*>(x_perm));
-    return cudaGetLastError();
+    cudaError_t err = launch_pdl(permute_rank_kernel, dim3(C), dim3(RW * 32), 0, s, sl, R, g.E,
+                                 hist, rank);
+    if (err == cudaSuccess)
+        err = launch_pdl(permute_scan_kernel, dim3(1), dim3(256), 0, s, hist, C, g.E, counts,
+                         offsets);
+    if (err == cudaSuccess)
+        err = launch_pdl(permute_scatter_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, s,
+                         sl, hist, rank, offsets, static_cast<const __nv_bfloat16*>(x), R, g.E,
+                         c.d, row_of, static_cast<__nv_bfloat16*>(x_perm));
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

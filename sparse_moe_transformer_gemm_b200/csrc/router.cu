@@ -49,6 +49,7 @@ router_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restri
               const float* __restrict__ norm_w, float norm_eps, int score_fn, int T, int d,
               int E, int k, float scale, float* __restrict__ logits, float* __restrict__ sumsq,
               int* __restrict__ counters, int* __restrict__ idx_out, float* __restrict__ w_out) {
+    pdl_launch_and_wait();
     __shared__ __align__(16) float xs[RT][KC];
     __shared__ int s_last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -215,11 +216,11 @@ cudaError_t launch_router(const moe_config& c, const void* x, const void* w_gate
                           float norm_eps, int score_fn, int32_t* idx, float* w, float* logits,
                           float* sumsq, int32_t* counters, int ksplit, cudaStream_t s) {
     dim3 grid((c.E + RE - 1) / RE, n_router_groups(c), ksplit);
-    router_kernel<<<grid, RWARPS * 32, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_gate), gate_bias,
-        score_bias, norm_w, norm_eps, score_fn, c.T, c.d, c.E, c.k, c.scale, logits, sumsq, counters, idx,
-        w);
-    return cudaGetLastError();
+    const cudaError_t err = launch_pdl(
+        router_kernel, grid, dim3(RWARPS * 32), 0, s, static_cast<const __nv_bfloat16*>(x),
+        static_cast<const __nv_bfloat16*>(w_gate), gate_bias, score_bias, norm_w, norm_eps, score_fn,
+        c.T, c.d, c.E, c.k, c.scale, logits, sumsq, counters, idx, w);
+    return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -213,6 +213,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                  int d, int E, int k, int n_pad,
                  float scale, int score_fn, int* __restrict__ idx_out,
                  float* __restrict__ w_out, int* __restrict__ status) {
+    pdl_launch_and_wait();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -458,13 +459,15 @@ cudaError_t launch_s(dim3 grid, const CUtensorMap& mx, const CUtensorMap& mw, co
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = S;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, router_tc_kernel<S>, mx, mw, gate_bias, score_bias, c.T, c.d,
                               c.E, c.k, n_pad, c.scale, score_fn, idx, w, status);
 }
