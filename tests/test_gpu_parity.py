@@ -34,6 +34,9 @@ SMALL = {
     # d and d_ff multiples of 256: the pair-of-SMs GEMMs (several tiles, ragged tokens)
     "pair_small": LayerShape(T=200, d=512, E=16, k=4, F=512),
     "pair_ragged": LayerShape(T=333, d=768, E=24, k=6, F=256, zipf_bias=True),
+    # ~375 rows per expert: two token tiles each (256 + a ragged tail), rows
+    # gathered by index with cp.async in the gate_up GEMM
+    "pair_multi": LayerShape(T=1500, d=512, E=8, k=2, F=256),
     # fewer grouped rows (6) than the smallest token box (16 rows)
     "pair_tiny": LayerShape(T=3, d=512, E=8, k=2, F=256),
     # the CUDA-core router (k > 8, or E not a multiple of 4)
@@ -213,7 +216,8 @@ def test_permute_index_is_bit_exact(T, E):
 
 
 @pytest.mark.parametrize("name,path", [
-    ("pair_small", None), ("pair_ragged", None), ("pair_ragged", "gemm"), ("ragged", None),
+    ("pair_small", None), ("pair_ragged", None), ("pair_multi", None), ("pair_ragged", "gemm"),
+    ("ragged", None),
     ("tiny", "stream"), ("pair_fp8", None), ("single_token", None)])
 def test_gate_up_gather_equals_permuted_copy_bitwise(name, path):
     """moe_expert_gate_up_gather (rows of x read by index inside the GEMM on the
