@@ -37,7 +37,6 @@ constexpr int UK = 16;
 constexpr int NMAX = 256;     // token rows per pair tile
 constexpr int NBOX = 16;      // token rows per TMA box
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int BOX_BYTES = NBOX * BK * 2;
 constexpr int EPI_GROUPS = 2;                      // epilogue warp groups (4 warps each)
 constexpr int THREADS = 64 + 128 * EPI_GROUPS;     // producer, MMA, epilogue warps
 constexpr int MAX_E = 256;
@@ -492,20 +491,30 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 // slower for FP8 and 13% for FP4; smaller op stages, twice as many, 8-10%
 // slower: more barrier and signal work for less conversion each.) Where d is
 // an odd multiple of 256, down's last pair tile has its first A tile only.
+//
+// Once the experts average 128+ grouped rows, down runs the transposed split
+// (TT): one A tile of 256 rows against two token sub-tiles of up to SUB = 192
+// rows each (a pair tile of up to 384 token rows; each CTA's token stage holds
+// its half of both sub-tiles in two regions), two accumulators of 192 columns
+// and 4 op stages of 32. Each K block of weights is then widened once for up
+// to 384 tokens instead of 192: at the Hy3 FP8 shape (T=8192, ~341 rows per
+// expert) down ran 12% faster (the layer 1.5% under the power cap).
 
 constexpr int THREADS_Q = 512;        // warps 6-14 converters, warp 15 token producer
 constexpr int MAX_RAW_STAGES = 16, MAX_B_STAGES = 4, MAX_OP_STAGES = 4;  // QCtrl's arrays
-template <bool GATE_UP, bool FP4>
+template <bool GATE_UP, bool FP4, bool TT = false>
 struct QShape {
-    static constexpr int A_TILES = 2;                              // A tiles per pair tile
+    static constexpr int A_TILES = TT ? 1 : 2;                     // A tiles per pair tile
     static constexpr int RAW_ROW = FP4 ? 32 : 64;                  // bytes of 64 codes
     static constexpr int RAW_TILE = BM * RAW_ROW;                  // 128 rows
     static constexpr int RAW_STAGE = A_TILES * RAW_TILE;
-    static constexpr int NM = 192;                                 // token rows per pair tile
-    static constexpr int BH = (NM / 2) * BK * 2;                   // a CTA's token half (bytes)
-    static constexpr int RAW_STAGES = FP4 ? 16 : 8;
+    static constexpr int SUB = 192;                                // token rows per accumulator
+    static constexpr int NM = TT ? 2 * SUB : SUB;                  // token rows per pair tile
+    static constexpr int REGION = (SUB / 2) * BK * 2;              // a CTA's half of SUB rows
+    static constexpr int BH = (TT ? 2 : 1) * REGION;               // a CTA's token stage (bytes)
+    static constexpr int RAW_STAGES = FP4 ? 16 : (TT ? 12 : 8);
     static constexpr int B_STAGES = 4;
-    static constexpr int OP_STAGES = 2;
+    static constexpr int OP_STAGES = TT ? 4 : 2;
     // converter warps: GROUPS groups of four (one per TMEM lane quarter) take
     // K blocks round-robin
     static constexpr int GROUPS = 2;
@@ -517,31 +526,33 @@ struct QShape {
     static constexpr int RING_BYTES = RAW_STAGES * RAW_STAGE + B_STAGES * BH + SC_BYTES;
     static constexpr int ACC_STAGES = 1;
     // TMEM columns: the two accumulators, then the op stages
-    static constexpr int U_OFF = NM;                               // the second A tile's accumulator
-    static constexpr int ACC_COLS = 2 * NM;
+    static constexpr int U_OFF = SUB;                              // the second accumulator
+    static constexpr int ACC_COLS = 2 * SUB;
     static constexpr int A_COL = ACC_STAGES * ACC_COLS;
     static constexpr int A_TILE_COLS = BK / 2;                     // one tile's K block: two bf16 a column
     static constexpr int A_STAGE_COLS = A_TILES * A_TILE_COLS;     // 64
-    static constexpr int M_ROWS = GATE_UP ? 2 * BM : 4 * BM;       // weight rows per m (per expert)
+    // weight rows (gate_up: gate rows; the up rows follow F on) per m (per expert)
+    static constexpr int M_ROWS = GATE_UP ? 2 * BM : (TT ? 2 * BM : 4 * BM);
+    static constexpr int EPI_BYTES = EPI_N * BM * 2;  // [32 tokens][128 rows] bf16 staging
 };
 
 constexpr int CONV_WARPS = 9;                          // warps 6..14 (warp 14 idles)
 constexpr int TOKEN_WARP = 6 + CONV_WARPS;
-template <bool G, bool FP4>
+template <bool G, bool FP4, bool TT = false>
 constexpr bool shape_ok() {
-    using S = QShape<G, FP4>;
+    using S = QShape<G, FP4, TT>;
     return S::RAW_STAGES % S::GROUPS == 0 && S::OP_STAGES % S::GROUPS == 0 &&
            S::GROUPS * S::GROUP_WARPS <= CONV_WARPS && S::GROUP_WARPS == 4 &&
            S::RAW_STAGES <= MAX_RAW_STAGES && S::B_STAGES <= MAX_B_STAGES &&
            S::OP_STAGES <= MAX_OP_STAGES && S::A_COL + S::OP_STAGES * S::A_STAGE_COLS <= 512 &&
-           S::BH % 1024 == 0 && S::RAW_TILE % 1024 == 0;
+           S::BH % 1024 == 0 && S::REGION % 1024 == 0 && S::RAW_TILE % 1024 == 0;
 }
 // Each group owns whole raw stages and op stages (both ring lengths are
 // multiples of GROUPS), and a group's previous wait on a stage proves that its
 // last reader finished (parity waits cannot see a stale phase); every stage
 // index stays inside QCtrl's barrier arrays.
 static_assert(shape_ok<true, false>() && shape_ok<false, false>() && shape_ok<true, true>() &&
-                  shape_ok<false, true>(),
+                  shape_ok<false, true>() && shape_ok<false, false, true>(),
               "quantised pair GEMM shape");
 static_assert(THREADS_Q == 32 * (TOKEN_WARP + 1), "warp roles cover the block");
 
@@ -564,14 +575,14 @@ struct QCtrl {
     int tile_start[MAX_E + 1];
 };
 
-constexpr int Q_EPI_BYTES = EPI_N * BM * 2;  // one [32 tokens][128 rows] bf16 staging tile
-
-template <bool GATE_UP, bool FP4>
+template <bool GATE_UP, bool FP4, bool TT = false>
 constexpr int q_smem_bytes() {
-    return QShape<GATE_UP, FP4>::RING_BYTES + Q_EPI_BYTES + 1024 + (int)sizeof(QCtrl);
+    return QShape<GATE_UP, FP4, TT>::RING_BYTES + QShape<GATE_UP, FP4, TT>::EPI_BYTES + 1024 +
+           (int)sizeof(QCtrl);
 }
 static_assert(q_smem_bytes<true, false>() <= 232448 && q_smem_bytes<false, false>() <= 232448 &&
-                  q_smem_bytes<true, true>() <= 232448 && q_smem_bytes<false, true>() <= 232448,
+                  q_smem_bytes<true, true>() <= 232448 && q_smem_bytes<false, true>() <= 232448 &&
+                  q_smem_bytes<false, false, true>() <= 232448,
               "fits in 227 KB");
 
 // A bf16x2 multiply kept in program order with respect to the waits around it
@@ -638,7 +649,7 @@ __device__ __forceinline__ void tc_store_row(uint32_t taddr, const uint32_t (&o)
 // x 128, 32-byte swizzle. tmB: token rows [R, K] bf16, boxes of 16..128 rows x
 // 64. scales_v: FP8 fp32 row scales [E * a_rows_per_expert]; FP4 E8M0 block
 // scales [E * a_rows_per_expert, K / 32] bytes.
-template <bool GATE_UP, bool FP4>
+template <bool GATE_UP, bool FP4, bool TT>
 __global__ void __launch_bounds__(THREADS_Q, 1)
 grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ TokenMaps tmB,
@@ -647,7 +658,8 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                              __nv_bfloat16* __restrict__ out, int out_ld,
                              int* __restrict__ status) {
     pdl_launch_and_wait();
-    using S = QShape<GATE_UP, FP4>;
+    using S = QShape<GATE_UP, FP4, TT>;
+    static_assert(!(TT && (FP4 || GATE_UP)), "two token sub-tiles: FP8 down only");
     const float* __restrict__ scales = static_cast<const float*>(scales_v);
     const uint8_t* __restrict__ scales8 = static_cast<const uint8_t*>(scales_v);
     extern __shared__ uint8_t smem_raw[];
@@ -657,7 +669,7 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     uint8_t* raw_ring = b_ring + S::B_STAGES * S::BH;
     uint8_t* sc_ring = raw_ring + S::RAW_STAGES * S::RAW_STAGE;  // FP4 only
     uint16_t* epi = reinterpret_cast<uint16_t*>(smem + S::RING_BYTES);
-    QCtrl& c = *reinterpret_cast<QCtrl*>(smem + S::RING_BYTES + Q_EPI_BYTES);
+    QCtrl& c = *reinterpret_cast<QCtrl*>(smem + S::RING_BYTES + S::EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)(tc::cluster_ctarank() & 1u);
     const bool leader = rank == 0;
@@ -729,13 +741,17 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
     // of the second's (gate_up: the up rows; down: 256 rows on), and whether
     // the second exists (not in down's last tile where d is an odd multiple of
     // 256).
+    // With TT (down) a pair tile has one A tile of 256 rows against up to 2 SUB
+    // token rows, SUB per accumulator.
     const int b_off = GATE_UP ? a_rows_per_expert / 2 : 2 * BM;
     auto first_row = [&](const TileInfo& ti) {
         return ti.e * a_rows_per_expert + ti.m * S::M_ROWS + rank * BM;
     };
     auto has_second = [&](const TileInfo& ti) {
-        return GATE_UP || ti.m * S::M_ROWS + 2 * BM < a_rows_per_expert;
+        return !TT && (GATE_UP || ti.m * S::M_ROWS + 2 * BM < a_rows_per_expert);
     };
+    // the tile's token rows per accumulator: n0 (at most SUB), then n1
+    auto sub_n0 = [&](const TileInfo& ti) { return TT ? min(ti.n, S::SUB) : ti.n; };
 
     if (warp == 0) {
         if (lane == 0) {
@@ -787,9 +803,10 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             bool ok = true;
             for (int t = pair; t < total && ok; t += n_pairs) {
                 const TileInfo ti = decode_tile<S::NM>(c, E, m_tiles, t);
-                const int nb = ti.n / (2 * NBOX);
-                const int b_row = ti.row0 + rank * (ti.n / 2);
-                const uint32_t pair_bytes = 2u * (uint32_t)(nb * BOX_BYTES);
+                // each CTA holds half of each accumulator's rows: n0 / 2 in the
+                // stage's first region, n1 / 2 in the second (TT)
+                const int n0 = sub_n0(ti), n1 = ti.n - n0;
+                const uint32_t pair_bytes = (uint32_t)ti.n * (BK * 2);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!tc::mbar_wait(&c.b_empty[stage], phase ^ 1u, abort_flag)) {
                         raise_timeout(c, status);
@@ -799,7 +816,11 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t full_leader = tc::map_to_cta(tc::smem_u32(&c.b_full[stage]), 0);
                     if (leader) tc::mbar_arrive_expect_tx(&c.b_full[stage], pair_bytes);
                     uint8_t* st = b_ring + stage * S::BH;
-                    load_token_rows(st, tmB, full_leader, kb * BK, b_row, ti.n / 2, pol_x);
+                    load_token_rows(st, tmB, full_leader, kb * BK, ti.row0 + rank * (n0 / 2), n0 / 2,
+                                    pol_x);
+                    if (TT && n1 > 0)
+                        load_token_rows(st + S::REGION, tmB, full_leader, kb * BK,
+                                        ti.row0 + n0 + rank * (n1 / 2), n1 / 2, pol_x);
                     issued[stage] = true;
                     parity[stage] = phase;
                     if (++stage == S::B_STAGES) {
@@ -973,7 +994,9 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 tc::fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * S::ACC_COLS;
-                const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, ti.n);
+                const int n0 = sub_n0(ti), n1 = ti.n - n0;
+                const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, n0);
+                const uint32_t idesc1 = tc::idesc_bf16_f32(2 * BM, n1 > 0 ? n1 : n0);
                 const bool two = has_second(ti);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!tc::mbar_wait(&c.op_full[os], oph, abort_flag) ||
@@ -990,6 +1013,10 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                         const uint64_t bdesc = tc::desc_sw128(b_addr + k * UK * 2);
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
                         tc::mma_bf16_pair_ta(d_tmem, a_tm + k * (UK / 2), bdesc, idesc, accum);
+                        if (TT && n1 > 0)  // the same A against the second region's rows
+                            tc::mma_bf16_pair_ta(d_tmem + S::U_OFF, a_tm + k * (UK / 2),
+                                                 tc::desc_sw128(b_addr + S::REGION + k * UK * 2),
+                                                 idesc1, accum);
                         if (two)  // the second A tile's columns follow the first's
                             tc::mma_bf16_pair_ta(d_tmem + S::U_OFF,
                                                  a_tm + S::A_TILE_COLS + k * (UK / 2), bdesc,
@@ -1039,8 +1066,37 @@ grouped_gemm_pair_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
             const long srow = (long)ti.e * a_rows_per_expert + col0 + row_in_tile;
             // FP8: the row scales multiply the finished dot products; FP4 folded
             // its block scales into the widening
-            const float sa = FP4 ? 1.f : __ldg(scales + srow);
-            const float sb = (FP4 || !two) ? 1.f : __ldg(scales + srow + b_off);
+            const float sa = FP4 || TT ? 1.f : __ldg(scales + srow);
+            const float sb = (FP4 || TT || !two) ? 1.f : __ldg(scales + srow + b_off);
+            if constexpr (TT) {
+                // part p: the tile's token rows p SUB.. (accumulator p), 128
+                // columns of y each
+                const int n0 = sub_n0(ti);
+                const int f0 = ti.m * S::M_ROWS + rank * BM;
+                const float sr = __ldg(scales + (long)ti.e * a_rows_per_expert + f0 + row_in_tile);
+                for (int part = 0; part < (ti.n > n0 ? 2 : 1); ++part) {
+                    const int np = part ? ti.n - n0 : n0, rb = part * S::SUB;
+                    for (int c0 = 0; c0 < np; c0 += EPI_N) {
+                        uint32_t g[32];
+                        tc::tmem_ld32(tbase + part * S::U_OFF + c0, g);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            epi[j * BM + row_in_tile] = float_to_bf16_bits(__uint_as_float(g[j]) * sr);
+                        tc::bar_sync(1, 128);  // the tile is written
+#pragma unroll
+                        for (int q = 0; q < EPI_N * BM / 8 / 128; ++q) {
+                            const int id = et + 128 * q;
+                            const int n = id / (BM / 8), ch = id % (BM / 8);
+                            if (rb + c0 + n < ti.len)
+                                *reinterpret_cast<uint4*>(o16 + (size_t)(ti.row0 + rb + c0 + n) * out_ld +
+                                                          f0 + ch * 8) =
+                                    *reinterpret_cast<const uint4*>(epi + n * BM + ch * 8);
+                        }
+                        tc::bar_sync(1, 128);  // the tile is read
+                    }
+                }
+            } else
             // gate_up: h = SiLU(g) u from the two accumulators; down: the two
             // accumulators are two 256-column ranges of y (part 1: 256 columns on)
             for (int c0 = 0; c0 < ti.n; c0 += EPI_N) {
@@ -1202,12 +1258,12 @@ cudaError_t launch(int T, const CUtensorMap& a, const TokenMaps& b, const int32_
                                             packed_a, out, out_ld, status, s, token_of_row);
 }
 
-template <bool GATE_UP, bool FP4 = false>
+template <bool GATE_UP, bool FP4 = false, bool TT = false>
 cudaError_t launch_fp8(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets,
                        const void* scales, int E, int K, int a_rows_per_expert, int m_tiles,
                        void* out, int out_ld, int* status, cudaStream_t s) {
-    const int smem = q_smem_bytes<GATE_UP, FP4>();
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_fp8_kernel<GATE_UP, FP4>,
+    const int smem = q_smem_bytes<GATE_UP, FP4, TT>();
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_fp8_kernel<GATE_UP, FP4, TT>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -1224,7 +1280,7 @@ cudaError_t launch_fp8(const CUtensorMap& a, const TokenMaps& b, const int32_t* 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_fp8_kernel<GATE_UP, FP4>, a, b, offsets, scales, E,
+    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_fp8_kernel<GATE_UP, FP4, TT>, a, b, offsets, scales, E,
                              K, a_rows_per_expert, m_tiles, static_cast<__nv_bfloat16*>(out),
                              out_ld, status);
     if (err != cudaSuccess) return err;
@@ -1234,6 +1290,16 @@ cudaError_t launch_fp8(const CUtensorMap& a, const TokenMaps& b, const int32_t* 
 }  // namespace
 
 bool pair_gemm_supported(const moe_config& c) { return c.d % 256 == 0 && c.d_ff % 256 == 0; }
+
+namespace {
+// The FP8 down GEMM's pair tiles: one A tile of 256 rows against two token
+// sub-tiles of up to 192 rows (each K block of weights widened once for up to
+// 384 tokens) once the experts average at least 128 grouped rows; two A tiles
+// against one token tile of up to 192 rows below that. (The same split for
+// gate_up, its gate and up rows paired in each TMEM lane quarter, measured
+// 2-3% slower: its epilogue then pairs g and u across lanes.)
+bool fp8_two_subtiles(const moe_config& g) { return (long)g.T * g.k >= 128L * g.E; }
+}  // namespace
 
 cudaError_t launch_gate_up_gemm_pair_fp8(const moe_config& c, const void* x_perm,
                                          const int32_t* offsets, const void* w_gate_up,
@@ -1258,6 +1324,9 @@ cudaError_t launch_down_gemm_pair_fp8(const moe_config& c, const void* h, const 
     if (!make_map_u8(&a, w_down, (uint64_t)c.E * c.d, c.d_ff, BM, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
+    if (fp8_two_subtiles(c))
+        return launch_fp8<false, false, true>(a, b, offsets, s_down, c.E, c.d_ff, c.d,
+                                              (c.d + 2 * BM - 1) / (2 * BM), y, c.d, status, s);
     return launch_fp8<false>(a, b, offsets, s_down, c.E, c.d_ff, c.d, (c.d + 4 * BM - 1) / (4 * BM),
                              y, c.d, status, s);
 }

@@ -176,9 +176,29 @@ def gemm_tiles(counts, nmax: int = NMAX, unit: int = 32):
             yield e, j * unit * q, unit * q if j < nt - 1 else n - unit * q * (nt - 1)
 
 
-def tile_cover_tokens(idx: np.ndarray, E: int, edge: int = 32, nmax: int = NMAX) -> np.ndarray:
+FP8_SUB = 192    # FP8 down with two token sub-tiles: rows per accumulator
+
+
+def fp8_down_tiles(counts, T: int, k: int, E: int):
+    """The token tiles of the FP8 SM-pair down GEMM, as (e, first row, length):
+    once the experts average at least 128 grouped rows (T*k >= 128 E) a pair
+    tile holds up to 2*FP8_SUB rows (gemm_tiles with that maximum) and its two
+    accumulators take rows [0, FP8_SUB) and [FP8_SUB, length); below that the
+    tiles hold up to FP8_NMAX rows, as gate_up's always do."""
+    if T * k < 128 * E:
+        yield from gemm_tiles(counts, FP8_NMAX)
+        return
+    for e, start, n in gemm_tiles(counts, 2 * FP8_SUB):
+        yield e, start, min(n, FP8_SUB)
+        if n > FP8_SUB:
+            yield e, start + FP8_SUB, n - FP8_SUB
+
+
+def tile_cover_tokens(idx: np.ndarray, E: int, edge: int = 32, nmax: int = NMAX,
+                      tiles=None) -> np.ndarray:
     """Tokens that put a grouped row into the first and into the last ``edge``
-    rows of every (expert, token tile) of the grouped GEMMs, chosen greedily
+    rows of every (expert, token tile) of the grouped GEMMs (``tiles``, else
+    gemm_tiles with ``nmax``), chosen greedily
     (each token brings k rows). The grouping is the oracle's (row_of), so the
     rows are those the GPU's GEMMs compute for the same routing."""
     T, k = idx.shape
@@ -187,7 +207,7 @@ def tile_cover_tokens(idx: np.ndarray, E: int, edge: int = 32, nmax: int = NMAX)
     token_of_row = np.empty(T * k, dtype=np.int64)
     token_of_row[row_of] = np.arange(T * k) // k
     targets = {}   # target id -> set of candidate tokens
-    for e, start, n in gemm_tiles(g["counts"], nmax):
+    for e, start, n in (gemm_tiles(g["counts"], nmax) if tiles is None else tiles):
         r0 = offsets[e] + start
         for lo, hi in ((r0, r0 + min(edge, n)), (r0 + n - min(edge, n), r0 + n)):
             targets[len(targets)] = set(token_of_row[lo:hi].tolist())

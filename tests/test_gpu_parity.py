@@ -103,11 +103,15 @@ def test_hy3_shapes(name):
     # at the head and at the tail of every (expert, token tile) of the grouped
     # GEMMs under the GPU's routing
     toks = parity.sample_tokens(shape.T, n=48 if shape.T > 64 else 64)
-    nmax = parity.FP8_NMAX if shape.fp8 else parity.NMAX
-    cover = parity.tile_cover_tokens(route[0], shape.E, nmax=nmax)
+    counts = np.bincount(route[0].ravel(), minlength=shape.E)
+    # FP8: gate_up's tiles and down's (two sub-tiles per pair tile at this shape)
+    tiles = (list(parity.gemm_tiles(counts, parity.FP8_NMAX)) +
+             list(parity.fp8_down_tiles(counts, shape.T, shape.k, shape.E)) if shape.fp8 else
+             list(parity.gemm_tiles(counts, parity.NMAX)))
+    cover = parity.tile_cover_tokens(route[0], shape.E, tiles=tiles)
     toks = np.unique(np.concatenate([toks, near[:8].astype(np.int32), cover]))
     res = parity.check_forward(layer, out, toks, route)
-    n_tiles = len(list(parity.gemm_tiles(np.bincount(route[0].ravel(), minlength=shape.E), nmax)))
+    n_tiles = len(tiles)
     print(name, "near-tie tokens:", len(near), near[:16].tolist(),
           f"checked tokens {len(toks)} (rows {len(toks) * shape.k}), tiles covered {n_tiles}",
           res)
@@ -119,7 +123,9 @@ def test_hy3_shapes(name):
 def test_quantised_all_tokens_to_the_same_experts(T, fmt):
     """FP8 / FP4 weights on the pair GEMMs with every token on experts 0..3: T
     rows each, in token tiles of at most 192 rows (193 as 128 + 65, 700 as
-    3 x 192 + 124); every token against the oracle."""
+    3 x 192 + 124); FP8 down at T=700 (T*k >= 128 E) in two pair tiles of 352
+    and 348 rows, each split 192 + the rest between its accumulators; every
+    token against the oracle."""
     shape = LayerShape(T=T, d=512, E=16, k=4, F=256, fp8=fmt == "fp8", fp4=fmt == "fp4")
     layer = make_layer(shape, seed=5, device="cuda")
     b = torch.zeros(shape.E, dtype=torch.float32, device="cuda")
@@ -127,8 +133,13 @@ def test_quantised_all_tokens_to_the_same_experts(T, fmt):
     layer["gate_bias"] = b
     route = parity.gpu_route(layer)
     assert np.all(np.sort(route[0], axis=1) == np.arange(4))
-    tiles = parity.gemm_tiles(np.bincount(route[0].ravel()), parity.FP8_NMAX)
+    counts = np.bincount(route[0].ravel())
+    tiles = parity.gemm_tiles(counts, parity.FP8_NMAX)
     assert [n for e, _, n in tiles if e == 0] == ([128, 65] if T == 193 else [192, 192, 192, 124])
+    if fmt == "fp8":
+        down = parity.fp8_down_tiles(counts, T, shape.k, shape.E)
+        assert [n for e, _, n in down if e == 0] == ([128, 65] if T == 193 else
+                                                    [192, 160, 192, 156])
     out = parity.gpu_forward(layer, "gemm")
     parity.check_forward(layer, out, None, route)
 
