@@ -30,6 +30,9 @@ SMALL = {
     "tiny_fp8": dataclasses.replace(CONFIGS["tiny"], fp8=True),
     # FP8 weights on the pair-of-SMs tensor-core path (d, d_ff multiples of 256)
     "pair_fp8": LayerShape(T=333, d=768, E=24, k=6, F=512, fp8=True),
+    # FP8 down with two token sub-tiles per pair tile (T*k >= 128 E): Zipf-hot
+    # experts take more than one pair tile, the rest one or two sub-tiles
+    "pair_fp8_subtiles": LayerShape(T=700, d=768, E=8, k=2, F=256, fp8=True, zipf_bias=True),
     "ragged_skewed": LayerShape(T=300, d=512, E=32, k=8, F=384, zipf_bias=True),
     # d and d_ff multiples of 256: the pair-of-SMs GEMMs (several tiles, ragged tokens)
     "pair_small": LayerShape(T=200, d=512, E=16, k=4, F=512),
