@@ -170,8 +170,22 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ TokenMaps tmB, const int* __restrict__ offsets,
                          const int* __restrict__ token_of_row, int E, int K,
                          int a_rows_per_expert, int m_tiles, int packed_a,
-                         __nv_bfloat16* __restrict__ out, int out_ld, int* __restrict__ status) {
-    pdl_launch_and_wait();
+                         __nv_bfloat16* __restrict__ out, int out_ld, int* __restrict__ status,
+                         const uint8_t* __restrict__ pf, long long pf_bytes) {
+    pdl_launch();
+    // The weights are read-only in the layer, so their first pf_bytes (the
+    // first experts' tiles) may be pulled into L2 before the wait for the
+    // previous kernel: thread blocks that are resident while the router and
+    // the grouping still run start the weight stream under them. One slice per
+    // CTA, in 64 KB requests.
+    if (pf_bytes > 0 && threadIdx.x == 0) {
+        const long long per = ((pf_bytes + gridDim.x - 1) / gridDim.x + 15) & ~15ll;
+        const long long b0 = (long long)blockIdx.x * per;
+        const long long b1 = b0 + per < pf_bytes ? b0 + per : pf_bytes;
+        for (long long o = b0; o < b1; o += 65536)
+            tc::prefetch_l2_bulk(pf + o, (uint32_t)(b1 - o < 65536 ? b1 - o : 65536));
+    }
+    pdl_wait();
     using S = Shape<GATE_UP, NM>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -1213,10 +1227,16 @@ int sm_pairs() {
     return (n > 1 ? n : 148) / 2;
 }
 
+// Bytes of the first experts' weights each bf16 pair GEMM pulls into L2 before
+// it waits for the previous kernel (0: none).
+constexpr long long kGateUpPrefetch = 96ll << 20;
+constexpr long long kDownPrefetch = 32ll << 20;
+
 template <bool GATE_UP, bool GATHER, int NM>
 cudaError_t launch_nm(const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets, int E,
                       int K, int a_rows_per_expert, int m_tiles, bool packed_a, void* out,
-                      int out_ld, int* status, cudaStream_t s, const int32_t* token_of_row) {
+                      int out_ld, int* status, cudaStream_t s, const int32_t* token_of_row,
+                      const void* pf, long long pf_bytes) {
     const int smem = smem_bytes<GATE_UP, NM>();
     cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATE_UP, GATHER, NM>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1237,7 +1257,8 @@ cudaError_t launch_nm(const CUtensorMap& a, const TokenMaps& b, const int32_t* o
     cfg.numAttrs = 2;
     err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATE_UP, GATHER, NM>, a, b, offsets,
                              token_of_row, E, K, a_rows_per_expert, m_tiles, (int)packed_a,
-                             static_cast<__nv_bfloat16*>(out), out_ld, status);
+                             static_cast<__nv_bfloat16*>(out), out_ld, status,
+                             static_cast<const uint8_t*>(pf), pf_bytes);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
@@ -1249,13 +1270,18 @@ template <bool GATE_UP, bool GATHER = false>
 cudaError_t launch(int T, const CUtensorMap& a, const TokenMaps& b, const int32_t* offsets, int E,
                    int K, int a_rows_per_expert, int m_tiles, bool packed_a, void* out,
                    int out_ld, int* status, cudaStream_t s,
-                   const int32_t* token_of_row = nullptr) {
+                   const int32_t* token_of_row = nullptr, const void* w = nullptr,
+                   long long w_bytes = 0) {
+    // the first experts' weights go to L2 ahead of the first tiles (see the kernel)
+    const long long cap = GATE_UP ? kGateUpPrefetch : kDownPrefetch;
+    const long long pf_bytes = w ? (w_bytes < cap ? w_bytes : cap) : 0;
     if (T <= NM_SMALL)
         return launch_nm<GATE_UP, GATHER, NM_SMALL>(a, b, offsets, E, K, a_rows_per_expert,
                                                      m_tiles, packed_a, out, out_ld, status, s,
-                                                     token_of_row);
+                                                     token_of_row, w, pf_bytes);
     return launch_nm<GATE_UP, GATHER, NMAX>(a, b, offsets, E, K, a_rows_per_expert, m_tiles,
-                                            packed_a, out, out_ld, status, s, token_of_row);
+                                            packed_a, out, out_ld, status, s, token_of_row, w,
+                                            pf_bytes);
 }
 
 template <bool GATE_UP, bool FP4 = false, bool TT = false>
@@ -1368,7 +1394,7 @@ cudaError_t launch_gate_up_gemm_pair(const moe_config& c, const void* x_perm,
         !make_token_maps(&b, x_perm, R, c.d))
         return cudaErrorInvalidValue;
     return launch<true>(c.T, a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), packed, h, c.d_ff,
-                        status, s);
+                        status, s, nullptr, w_gate_up, (long long)c.E * 2 * c.d_ff * c.d * 2);
 }
 
 cudaError_t launch_gate_up_gemm_pair_gather(const moe_config& c, const void* x,
@@ -1381,7 +1407,8 @@ cudaError_t launch_gate_up_gemm_pair_gather(const moe_config& c, const void* x,
         !make_map(&b.m[0], x, (uint64_t)c.T, c.d, 1))
         return cudaErrorInvalidValue;
     return launch<true, true>(c.T, a, b, offsets, c.E, c.d, 2 * c.d_ff, c.d_ff / (2 * BM), packed, h,
-                              c.d_ff, status, s, token_of_row);
+                              c.d_ff, status, s, token_of_row, w_gate_up,
+                              (long long)c.E * 2 * c.d_ff * c.d * 2);
 }
 
 cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int32_t* offsets,
@@ -1394,7 +1421,7 @@ cudaError_t launch_down_gemm_pair(const moe_config& c, const void* h, const int3
         !make_token_maps(&b, h, R, c.d_ff))
         return cudaErrorInvalidValue;
     return launch<false>(c.T, a, b, offsets, c.E, c.d_ff, c.d, (c.d + 4 * BM - 1) / (4 * BM), packed, y,
-                         c.d, status, s);
+                         c.d, status, s, nullptr, w_down, (long long)c.E * c.d * c.d_ff * 2);
 }
 
 namespace {
