@@ -64,10 +64,10 @@ WORKLOADS = {
 # experts at decode, with the routed rows at prefill). An entry is removed when
 # its kernel changes.
 NCU_TRAFFIC = {
-    # bf16 pair gate_up, decode case E=96, T=32: 2.2437 GB for 89 touched experts
-    ("decode", "gate_up_gemm"): {"per": "touched_expert", "bytes": 2.2437e9 / 89},
-    # bf16 pair gate_up, prefill case E=96, T=2048: 2.5878 GB for 16384 routed rows
-    ("prefill", "gate_up_gemm"): {"per": "row", "bytes": 2.5878e9 / 16384},
+    # bf16 pair gate_up, decode case E=96, T=32: 2.2438 GB for 89 touched experts
+    ("decode", "gate_up_gemm"): {"per": "touched_expert", "bytes": 2.2438e9 / 89},
+    # bf16 pair gate_up, prefill case E=96, T=2048: 2.5879 GB for 16384 routed rows
+    ("prefill", "gate_up_gemm"): {"per": "row", "bytes": 2.5879e9 / 16384},
     # FP8 pair gate_up, case E=48, T=2048 (341 rows per expert, as at T=8192):
     # 0.9362 GB for 16384 routed rows
     ("fp8", "gate_up_gemm"): {"per": "row", "bytes": 0.9362e9 / 16384},
