@@ -114,3 +114,40 @@ def test_work_accounting_matches_the_page_figures():
     lw = work.layer_work(64, 4096, 192, 8, 1536, touched=175)
     assert lw["flops"] == 2 * 64 * 4096 * 192 + 6 * 64 * 8 * 4096 * 1536
     assert lw["bytes"] >= 175 * work.expert_bytes(4096, 1536)
+
+
+def test_gemm_tile_models_partition_each_experts_rows():
+    """The token-tile models the GPU tests use to pick tokens that cover every
+    tile: per expert the tiles are contiguous, start at row 0, end at n_e, and
+    respect their maximum; all but an expert's last tile hold a multiple of 32
+    rows (gemm_tiles); FP8 down's sub-tiles hold at most 192 rows and, below
+    128 rows per expert on average, are gate_up's 192-row tiles."""
+    import numpy as np
+    import parity
+
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        E = int(rng.integers(1, 40))
+        counts = rng.integers(0, 1200, size=E)
+        counts[rng.random(E) < 0.2] = 0
+        for nmax in (64, 192, 256, 384):
+            tiles = list(parity.gemm_tiles(counts, nmax))
+            for e in range(E):
+                mine = [(s, n) for ee, s, n in tiles if ee == e]
+                assert sum(n for _, n in mine) == counts[e]
+                pos = 0
+                for j, (s, n) in enumerate(mine):
+                    assert s == pos and 0 < n <= nmax
+                    if j < len(mine) - 1:
+                        assert n % 32 == 0
+                    pos += n
+        k = 8
+        for T in (int(counts.sum()) // k, 16 * E):  # both sides of T*k = 128 E
+            down = list(parity.fp8_down_tiles(counts, T, k, E))
+            if T * k < 128 * E:
+                assert down == list(parity.gemm_tiles(counts, parity.FP8_NMAX))
+            for e in range(E):
+                mine = [(s, n) for ee, s, n in down if ee == e]
+                assert sum(n for _, n in mine) == counts[e]
+                assert all(0 < n <= parity.FP8_SUB for _, n in mine)
+                assert [s for s, _ in mine] == sorted(s for s, _ in mine)
